@@ -1,0 +1,196 @@
+"""Seeded synthetic inputs shared by the tests, the smoke check and the
+benchmark.
+
+This module only draws random numbers and builds index structures (block
+tables, selected-row lists); it holds none of the attention arithmetic, so the
+CUDA path and the CPU oracle can both be fed from it without sharing code.
+
+Recipe: every bf16 tensor is drawn as float32 ``torch.randn`` on a CPU
+``torch.Generator`` seeded per tensor and rounded to bf16 (round to nearest
+even).  Seeds for workload ``c``: Q = 1000 + c, K = 2000 + c, V = 3000 + c,
+structure (lengths, block ids, selected rows) = 4000 + c.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+
+import numpy as np
+import torch
+
+
+def randn_bf16(shape, seed: int) -> torch.Tensor:
+    g = torch.Generator().manual_seed(int(seed))
+    return torch.randn(*shape, generator=g, dtype=torch.float32).to(torch.bfloat16)
+
+
+def bits(t: torch.Tensor) -> np.ndarray:
+    """bf16 tensor (CPU or CUDA) -> numpy uint16 bit patterns, same shape."""
+    t = t.detach()
+    if t.dtype != torch.bfloat16:
+        raise TypeError("expected bf16")
+    return t.cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+# ----------------------------------------------------------------- prefill --
+
+@dataclass
+class PrefillCase:
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    Sq: int
+    Sk: int
+    dk: int
+    dv: int
+    causal: bool
+    seed: int = 0
+    scale: float = field(default=0.0)
+
+    def __post_init__(self):
+        if not self.scale:
+            self.scale = 1.0 / math.sqrt(self.dk)
+
+    @property
+    def flops(self) -> float:
+        """4 * B * Hq * Sq * Sk * d (dk = dv here), halved for causal."""
+        f = 2.0 * self.B * self.Hq * self.Sq * self.Sk * (self.dk + self.dv)
+        return f / 2 if self.causal else f
+
+
+def prefill_inputs(c: PrefillCase):
+    q = randn_bf16((c.B, c.Hq, c.Sq, c.dk), 1000 + c.seed)
+    k = randn_bf16((c.B, c.Hkv, c.Sk, c.dk), 2000 + c.seed)
+    v = randn_bf16((c.B, c.Hkv, c.Sk, c.dv), 3000 + c.seed)
+    return q, k, v
+
+
+TINY_FULL = PrefillCase("tiny_full_b1_h2_s256_d64", 1, 2, 2, 256, 256, 64, 64, False, seed=1)
+CAUSAL_MHA = PrefillCase("causal_mha_b2_h16_s2048_d128", 2, 16, 16, 2048, 2048, 128, 128, True, seed=2)
+GQA_FULL = PrefillCase("gqa_full_b1_hq32_hkv8_s4096_d256", 1, 32, 8, 4096, 4096, 256, 256, False, seed=3)
+
+
+# ------------------------------------------------------------ paged decode --
+
+@dataclass
+class PagedCase:
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    dk: int
+    dv: int
+    block_size: int
+    min_len: int
+    max_len: int
+    seed: int = 0
+    scale: float = field(default=0.0)
+    lens: tuple | None = None  # explicit per-sequence lengths (tests)
+
+    def __post_init__(self):
+        if not self.scale:
+            self.scale = 1.0 / math.sqrt(self.dk)
+
+
+def paged_inputs(c: PagedCase):
+    """Returns q [B,Hq,dk], k_cache/v_cache [nb,Hkv,bs,d] bf16, block_table
+    int32 [B, max_blocks] (-1 past the end), seq_lens int32 [B]."""
+    g = torch.Generator().manual_seed(4000 + c.seed)
+    if c.lens is not None:
+        lens = torch.tensor(c.lens, dtype=torch.int64)
+    else:
+        lens = torch.randint(c.min_len, c.max_len + 1, (c.B,), generator=g)
+    bs = c.block_size
+    nblk = (lens + bs - 1) // bs
+    max_blocks = max(1, int(nblk.max()) if c.B else 1)
+    pool = int(nblk.sum())
+    perm = torch.randperm(max(pool, 1), generator=g)[:pool]
+    table = torch.full((c.B, max_blocks), -1, dtype=torch.int32)
+    off = 0
+    for b in range(c.B):
+        n = int(nblk[b])
+        table[b, :n] = perm[off:off + n].to(torch.int32)
+        off += n
+    nb = max(pool, 1)
+    q = randn_bf16((c.B, c.Hq, c.dk), 1000 + c.seed)
+    kc = randn_bf16((nb, c.Hkv, bs, c.dk), 2000 + c.seed)
+    vc = randn_bf16((nb, c.Hkv, bs, c.dv), 3000 + c.seed)
+    return q, kc, vc, table, lens.to(torch.int32)
+
+
+def paged_bytes(c: PagedCase, seq_lens, max_blocks: int) -> int:
+    """Algorithmic HBM bytes of one paged decode: every visible K/V element
+    once, the used block-table entries, lengths, Q, fp32 O and LSE."""
+    sl = [int(x) for x in seq_lens]
+    kv = sum(sl) * c.Hkv * (c.dk + c.dv) * 2
+    tbl = sum((n + c.block_size - 1) // c.block_size for n in sl) * 4
+    return kv + tbl + c.B * 4 + c.B * c.Hq * c.dk * 2 + c.B * c.Hq * c.dv * 4 + c.B * c.Hq * 4
+
+
+PAGED_GQA = PagedCase("paged_gqa_b64_hq32_hkv8_d128_bs64", 64, 32, 8, 128, 128, 64, 1024, 8192, seed=4)
+
+
+# ----------------------------------------------------------- latent decode --
+
+@dataclass
+class LatentCase:
+    name: str
+    T: int
+    Hq: int
+    n_rows: int
+    topk: int
+    dk: int = 576
+    dv: int = 512
+    v_offset: int = 64
+    seed: int = 0
+    scale: float = field(default=0.0)
+    select_from_all: bool = False  # tests: pick rows anywhere so the mask bites
+    q_pos0: int | None = 1000      # forced position of token 0 (None: random)
+
+    def __post_init__(self):
+        if not self.scale:
+            self.scale = 1.0 / math.sqrt(self.dk)
+
+
+def latent_inputs(c: LatentCase):
+    """Returns q [T,Hq,dk], rows [n_rows,dk] bf16, idx int32 [T,topk]
+    (-1 = empty slot), q_pos int32 [T].  Key position = row index."""
+    g = torch.Generator().manual_seed(4000 + c.seed)
+    qpos = torch.randint(0, c.n_rows, (c.T,), generator=g)
+    if c.T and c.q_pos0 is not None:
+        qpos[0] = min(c.q_pos0, c.n_rows - 1)
+    idx = torch.full((c.T, c.topk), -1, dtype=torch.int32)
+    for t in range(c.T):
+        hi = c.n_rows if c.select_from_all else int(qpos[t]) + 1
+        if hi >= c.topk:
+            sel = torch.randperm(hi, generator=g)[:c.topk]
+            idx[t] = sel.to(torch.int32)
+        else:
+            idx[t, :hi] = torch.arange(hi, dtype=torch.int32)
+    row_len = max(c.dk, c.v_offset + c.dv)
+    q = randn_bf16((c.T, c.Hq, c.dk), 1000 + c.seed)
+    rows = randn_bf16((c.n_rows, row_len), 2000 + c.seed)
+    return q, rows, idx, qpos.to(torch.int32)
+
+
+def latent_visible(idx: torch.Tensor, q_pos: torch.Tensor) -> int:
+    """Number of (token, slot) pairs that are visible: idx >= 0 and
+    row (= key position) <= q_pos."""
+    v = (idx >= 0) & (idx <= q_pos.view(-1, 1))
+    return int(v.sum())
+
+
+def latent_bytes(c: LatentCase, n_visible: int) -> int:
+    """Algorithmic HBM bytes: each visible selected row once (dk-wide, which
+    covers V), the index list, Q, fp32 O and LSE."""
+    row_len = max(c.dk, c.v_offset + c.dv)
+    return (n_visible * row_len * 2 + c.T * c.topk * 4 + c.T * 4 + c.T * c.Hq * c.dk * 2
+            + c.T * c.Hq * c.dv * 4 + c.T * c.Hq * 4)
+
+
+def latent_flops(c: LatentCase, n_visible: int) -> float:
+    return 2.0 * c.Hq * (c.dk + c.dv) * n_visible
+
+
+LATENT_SPARSE = LatentCase("latent_sparse_t32_hq128_dk576_dv512_top2048", 32, 128, 65536, 2048, seed=5)
