@@ -1,0 +1,373 @@
+// decode_gather.cu -- latent (MLA-style) sparse decode over selected cache
+// rows, on the sm_100a tensor cores.
+//
+// Problem ("MLA Decode Attention Kernel API Reference", AWS Neuron NKI:
+// parameters kv_cache / kv_row_cur / prior_rows / prior_key_pos / positions):
+// every one of the 128 query heads of decode token t attends over the rows
+// idx[t][0..topk) of a latent cache whose rows are [k_pe (64) | kv_latent
+// (512)]; key = the whole 576-wide row, value = the 512-wide latent part,
+// one KV head shared by all query heads, a key visible iff its position
+// <= the token's position.  As on that page, rows are gathered straight
+// from the cache in its native row-major layout (no pre-gathered copy).
+//
+// Design (one CTA = one token x one key split x one half of dv):
+//   - the 128 heads are the MMA's M = 128 rows: S = Q K^T (K = 576) and
+//     O += P V run as tcgen05.mma with fp32 accumulators in TMEM;
+//   - O for 128 heads x 512 dims in fp32 would fill all 512 TMEM columns,
+//     leaving none for S, so the two halves of dv go to two CTAs launched
+//     side by side (each recomputes S = Q K^T; the second CTA's row reads
+//     mostly hit L2);
+//   - warps 0-3 gather 32 selected rows per tile with 16-byte cp.async into
+//     128-byte-swizzled shared memory; the same tile is the K-major B
+//     operand of QK^T and (its latent columns) the MN-major B operand of PV,
+//     so every row is read once per CTA;
+//   - Q (128 x 576, 144 KB) is loaded once by TMA;
+//   - warp 8 issues the MMAs; warps 4-7 run the online softmax (one head per
+//     thread; the visibility mask comes with the tile) and the epilogue,
+//     writing a split partial that the log-sum-exp combine merges.
+#include <cuda_runtime.h>
+#include <limits.h>
+#include <math.h>
+
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace fa {
+
+static __device__ int g_gather_err;
+
+constexpr int LG_DK = 576;
+constexpr int LG_DV = 512;
+constexpr int LG_HALF = 256;
+constexpr int LG_H = 128;
+constexpr int LG_BN = 32;                       // keys per tile
+constexpr int LG_NST = 2;                       // tile ring depth
+constexpr int LG_NCH = LG_DK / 64;              // 9 chunks of 128 bytes per row
+constexpr int LG_QCH = LG_H * 128;              // bytes of one Q chunk (16 KB)
+constexpr int LG_KCH = LG_BN * 128;             // bytes of one K chunk (4 KB)
+constexpr int LG_Q_BYTES = LG_NCH * LG_QCH;     // 144 KB
+constexpr int LG_K_BYTES = LG_NCH * LG_KCH;     // 36 KB
+constexpr int LG_OFF_K = LG_Q_BYTES;
+constexpr int LG_OFF_AUX = LG_OFF_K + LG_NST * LG_K_BYTES;
+constexpr int LG_SMEM = LG_OFF_AUX + 512 + 1024;
+constexpr int LG_PIECES = LG_BN * (LG_DK / 8);  // 16-byte pieces per tile (2304)
+constexpr int LG_T_O = 2 * LG_BN;               // TMEM column of O (S0 at 0, S1 at 32)
+static_assert(LG_SMEM <= 232448, "shared memory budget");
+static_assert(LG_PIECES % 128 == 0, "pieces per producer thread");
+
+enum { G_QFULL = 0, G_SFULL = 1, G_PREADY = 3, G_PVDONE = 5, G_DRAIN = 6, G_FULL = 7, G_EMPTY = 9, G_NBAR = 11 };
+
+struct GatherArgs {
+    const __nv_bfloat16 *rows;
+    int64_t n_rows, row_stride;
+    const int32_t *idx, *key_pos, *q_pos;
+    int topk, kps, num_splits;
+    float scale_log2;
+    float *part_o, *part_lse;
+};
+
+constexpr float kGatherRescaleThreshold = 8.0f;
+
+__global__ void __launch_bounds__(288, 1)
+latent_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const GatherArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t sQ = sbase, sK = sbase + LG_OFF_K;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + LG_OFF_AUX);
+    const uint32_t bar0 = smem_u32(bars);
+    auto bar = [&](int i) -> uint32_t { return bar0 + 8u * (uint32_t)i; };
+    int32_t *rowid = reinterpret_cast<int32_t *>(smem + LG_OFF_AUX + 8 * 16);  // [NST][32]
+    uint32_t *maskw = reinterpret_cast<uint32_t *>(rowid + LG_NST * LG_BN);    // [NST]
+    uint32_t *tmem_holder = maskw + LG_NST;
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int half = blockIdx.x, split = blockIdx.y, t = blockIdx.z;
+    const int k_begin = split * a.kps;
+    const int k_end = min(a.topk, k_begin + a.kps);
+    const int n_tiles = k_end > k_begin ? (k_end - k_begin + LG_BN - 1) / LG_BN : 0;
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar(G_QFULL), 1);
+        mbar_init(bar(G_SFULL), 1);
+        mbar_init(bar(G_SFULL + 1), 1);
+        mbar_init(bar(G_PREADY), 128);
+        mbar_init(bar(G_PREADY + 1), 128);
+        mbar_init(bar(G_PVDONE), 1);
+        mbar_init(bar(G_DRAIN), 1);
+        for (int s = 0; s < LG_NST; ++s) {
+            mbar_init(bar(G_FULL + s), 128);
+            mbar_init(bar(G_EMPTY + s), 1);
+        }
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 8) {
+        tmem_alloc(smem_u32(tmem_holder), 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+
+    if (warp < 4) {
+        // ------------------------------------------------- row gatherers --
+        const int tid = threadIdx.x;
+        if (n_tiles > 0) {
+            if (tid == 0) {
+                prefetch_tmap(&tmQ);
+                mbar_arrive_expect_tx(bar(G_QFULL), LG_Q_BYTES);
+#pragma unroll 1
+                for (int c = 0; c < LG_NCH; ++c) tma_load_2d(sQ + c * LG_QCH, &tmQ, bar(G_QFULL), c * 64, t * LG_H);
+            }
+            const int qpos = a.q_pos ? a.q_pos[t] : INT_MAX;
+            const int32_t *idx_t = a.idx + (int64_t)t * a.topk;
+            const int32_t *kp_t = a.key_pos ? a.key_pos + (int64_t)t * a.topk : nullptr;
+            volatile int *go = reinterpret_cast<volatile int *>(tmem_holder + 2);
+            bool ok = true;
+            for (int i = 0; i < n_tiles; ++i) {
+                const int s = i % LG_NST;
+                // One thread waits for the stage to be free and publishes the
+                // outcome, so all 128 gatherers take the same branch below.
+                if (tid == 0)
+                    *go = mbar_wait(bar(G_EMPTY + s), ((uint32_t)(i / LG_NST) & 1u) ^ 1u, abort_flag, &g_gather_err);
+                if (warp == 0) {
+                    __syncwarp();  // lane 0 has finished its wait
+                    const int key = k_begin + i * LG_BN + lane;
+                    int r = -1;
+                    bool vis = false;
+                    if (key < k_end) {
+                        r = idx_t[key];
+                        if (r < -1 || (int64_t)r >= a.n_rows) {
+                            atomicCAS(&g_gather_err, 0, 3 /* FA_DEVERR_BAD_ROW */);
+                            r = -1;
+                        }
+                        if (r >= 0) vis = (kp_t ? kp_t[key] : r) <= qpos;
+                    }
+                    rowid[s * LG_BN + lane] = r >= 0 ? r : 0;  // row 0 stands in for an empty slot
+                    const uint32_t m = __ballot_sync(0xffffffffu, vis);
+                    if (lane == 0) maskw[s] = m;
+                }
+                asm volatile("bar.sync 1, 128;" ::: "memory");
+                const bool proceed = *go != 0;
+                asm volatile("bar.sync 1, 128;" ::: "memory");
+                if (!proceed) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t dst0 = sK + s * LG_K_BYTES;
+#pragma unroll
+                for (int j = 0; j < LG_PIECES / 128; ++j) {
+                    const int piece = tid + 128 * j;
+                    const int row = piece / (LG_DK / 8);
+                    const int pc = piece % (LG_DK / 8);  // 16-byte piece within the row
+                    const int c = pc >> 3, sub = pc & 7;
+                    const __nv_bfloat16 *src = a.rows + (int64_t)rowid[s * LG_BN + row] * a.row_stride + pc * 8;
+                    cp_async16(dst0 + c * LG_KCH + row * 128 + ((sub ^ (row & 7)) << 4), src);
+                }
+                cp_async_commit();
+                if (i >= 1) {
+                    cp_async_wait<1>();
+                    fence_proxy_async_smem();
+                    mbar_arrive(bar(G_FULL + (i - 1) % LG_NST));
+                }
+            }
+            cp_async_wait<0>();
+            if (ok) {
+                fence_proxy_async_smem();
+                mbar_arrive(bar(G_FULL + (n_tiles - 1) % LG_NST));
+            }
+            if (tid == 0 && *abort_flag) mbar_wait_drain(bar(G_QFULL), 0);
+        }
+    } else if (warp == 8) {
+        // --------------------------------------------------- MMA issuer --
+        if (lane == 0 && n_tiles > 0) {
+            constexpr uint32_t idesc_qk = idesc_bf16_f32(128, LG_BN, false, false);
+            constexpr uint32_t idesc_pv = idesc_bf16_f32(128, LG_HALF, false, true);
+            const uint32_t tO = tmem + LG_T_O;
+            const uint32_t v_chunk0 = (uint32_t)(1 + 4 * half) * LG_KCH;  // first latent chunk of this half
+            auto issue_qk = [&](int i) -> bool {
+                const int s = i % LG_NST;
+                if (!mbar_wait(bar(G_FULL + s), (uint32_t)(i / LG_NST) & 1u, abort_flag, &g_gather_err)) return false;
+                tc_fence_after();
+                const uint32_t tS = tmem + (uint32_t)((i & 1) * LG_BN);
+#pragma unroll
+                for (int kk = 0; kk < LG_DK / 16; ++kk) {
+                    const int c = kk >> 2, sub = kk & 3;
+                    const uint64_t ad = sdesc_sw128(sQ + c * LG_QCH + sub * 32, 16, 1024);
+                    const uint64_t bd = sdesc_sw128(sK + s * LG_K_BYTES + c * LG_KCH + sub * 32, 16, 1024);
+                    mma_ss(tS, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(bar(G_SFULL + (i & 1)));
+                return true;
+            };
+            bool ok = mbar_wait(bar(G_QFULL), 0, abort_flag, &g_gather_err) && issue_qk(0);
+            for (int i = 0; ok && i < n_tiles; ++i) {
+                if (i + 1 < n_tiles && !issue_qk(i + 1)) break;
+                if (!mbar_wait(bar(G_PREADY + (i & 1)), (uint32_t)(i >> 1) & 1u, abort_flag, &g_gather_err)) break;
+                tc_fence_after();
+                const int s = i % LG_NST;
+                const uint32_t tP = tmem + (uint32_t)((i & 1) * LG_BN);
+#pragma unroll
+                for (int kk = 0; kk < LG_BN / 16; ++kk) {
+                    const uint64_t bd = sdesc_sw128(sK + s * LG_K_BYTES + v_chunk0 + kk * 2048, LG_KCH, 1024);
+                    mma_ts(tO, tP + kk * 8, bd, idesc_pv, (i > 0 || kk > 0) ? 1u : 0u);
+                }
+                mma_commit(bar(G_EMPTY + s));
+                mma_commit(bar(G_PVDONE));
+            }
+            mma_commit(bar(G_DRAIN));
+            mbar_wait_drain(bar(G_DRAIN), 0);
+        }
+        __syncwarp();
+    } else {
+        // ---------------------------------- softmax / correction / epilogue --
+        const int qd = warp & 3;
+        const int head = qd * 32 + lane;
+        const uint32_t tl = tmem + ((uint32_t)(qd * 32) << 16);
+        const float c = a.scale_log2;
+        float m_run = -INFINITY, l_run = 0.f;
+        bool ok = true;
+        for (int i = 0; i < n_tiles; ++i) {
+            const int buf = i & 1, s = i % LG_NST;
+            if (!mbar_wait(bar(G_SFULL + buf), (uint32_t)(i >> 1) & 1u, abort_flag, &g_gather_err) ||
+                !mbar_wait(bar(G_FULL + s), (uint32_t)(i / LG_NST) & 1u, abort_flag, &g_gather_err)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            uint32_t r[32];
+            tmem_ld32(tl + (uint32_t)(buf * LG_BN), r);
+            tmem_wait_ld();
+            reg_fence(r);
+            const uint32_t mask = maskw[s];
+            float x[32];
+#pragma unroll
+            for (int k = 0; k < 32; ++k) x[k] = ((mask >> k) & 1u) ? __uint_as_float(r[k]) : -INFINITY;
+            float mx0 = x[0], mx1 = x[1];
+#pragma unroll
+            for (int k = 2; k < 32; k += 2) {
+                mx0 = fmaxf(mx0, x[k]);
+                mx1 = fmaxf(mx1, x[k + 1]);
+            }
+            const float m_tile = fmaxf(mx0, mx1) * c;
+            const float m_new = fmaxf(m_run, m_tile);
+            const bool need = m_new > m_run + kGatherRescaleThreshold;
+            float alpha = 1.f;
+            if (need) {
+                alpha = ex2(m_run - m_new);
+                l_run *= alpha;
+                m_run = m_new;
+            }
+            if (i > 0 && __any_sync(0xffffffffu, need)) {
+                if (!mbar_wait(bar(G_PVDONE), (uint32_t)(i - 1) & 1u, abort_flag, &g_gather_err)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+#pragma unroll 1
+                for (int ch = 0; ch < LG_HALF / 32; ++ch) {
+                    uint32_t o[32];
+                    tmem_ld32(tl + (uint32_t)(LG_T_O + ch * 32), o);
+                    tmem_wait_ld();
+                    reg_fence(o);
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+                    tmem_st32(tl + (uint32_t)(LG_T_O + ch * 32), o);
+                }
+            }
+            const float msub = (m_run == -INFINITY) ? 0.f : m_run;
+            uint32_t pk[16];
+            float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                const float p0 = ex2(fmaf(x[2 * k], c, -msub));
+                const float p1 = ex2(fmaf(x[2 * k + 1], c, -msub));
+                s0 += p0;
+                s1 += p1;
+                pk[k] = pack_bf16x2(p0, p1);
+            }
+            l_run += s0 + s1;
+            tmem_st16(tl + (uint32_t)(buf * LG_BN), pk);
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar(G_PREADY + buf));
+        }
+        bool have_o = ok && n_tiles > 0;
+        if (have_o) {
+            if (mbar_wait(bar(G_PVDONE), (uint32_t)(n_tiles - 1) & 1u, abort_flag, &g_gather_err))
+                tc_fence_after();
+            else
+                have_o = false;
+        }
+        const bool good = have_o && l_run > 0.f;
+        const float inv_l = good ? 1.f / l_run : 0.f;
+        const int64_t prow = ((int64_t)t * LG_H + head) * a.num_splits + split;
+        float4 *dst = reinterpret_cast<float4 *>(a.part_o + prow * LG_DV + half * LG_HALF);
+#pragma unroll 1
+        for (int ch = 0; ch < LG_HALF / 32; ++ch) {
+            uint32_t o[32];
+            if (have_o) {
+                tmem_ld32(tl + (uint32_t)(LG_T_O + ch * 32), o);
+                tmem_wait_ld();
+                reg_fence(o);
+            } else {
+#pragma unroll
+                for (int k = 0; k < 32; ++k) o[k] = 0u;
+            }
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                dst[ch * 8 + k] = make_float4(__uint_as_float(o[4 * k]) * inv_l, __uint_as_float(o[4 * k + 1]) * inv_l,
+                                              __uint_as_float(o[4 * k + 2]) * inv_l,
+                                              __uint_as_float(o[4 * k + 3]) * inv_l);
+        }
+        if (half == 0) a.part_lse[prow] = good ? m_run + __log2f(l_run) : -INFINITY;
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 8) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+cudaError_t launch_decode_gather(const GatherLaunch &L, cudaStream_t stream) {
+    cudaError_t e = cudaFuncSetAttribute(latent_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, LG_SMEM);
+    if (e != cudaSuccess) return e;
+    GatherArgs a;
+    a.rows = static_cast<const __nv_bfloat16 *>(L.rows);
+    a.n_rows = L.n_rows;
+    a.row_stride = L.row_stride;
+    a.idx = L.idx;
+    a.key_pos = L.key_pos;
+    a.q_pos = L.q_pos;
+    a.topk = L.topk;
+    a.kps = L.keys_per_split;
+    a.num_splits = L.num_splits;
+    a.scale_log2 = L.scale * 1.4426950408889634f;
+    a.part_o = L.part_o;
+    a.part_lse = L.part_lse;
+    dim3 grid(2u, (unsigned)L.num_splits, (unsigned)L.T);
+    latent_decode_kernel<<<grid, 288, LG_SMEM, stream>>>(L.tmQ, a);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    return launch_combine(L.part_o, L.part_lse, L.T * L.Hq, L.num_splits, L.Hq, nullptr, 0, L.o, L.lse, L.o_bf16,
+                          LG_DV, stream);
+}
+
+cudaError_t gather_device_error(int clear, int *code) {
+    int v = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(&v, g_gather_err, sizeof(int));
+    if (e != cudaSuccess) return e;
+    *code = v;
+    if (clear && v) {
+        v = 0;
+        e = cudaMemcpyToSymbol(g_gather_err, &v, sizeof(int));
+    }
+    return e;
+}
+
+}  // namespace fa

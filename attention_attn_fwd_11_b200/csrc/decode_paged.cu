@@ -1,0 +1,400 @@
+// decode_paged.cu -- split-KV decode over a paged KV cache (sm_100a), and
+// the log-sum-exp combine shared by both decode paths.
+//
+// Decode is bandwidth-bound (about 4 FLOP per byte of K/V at head dim 128),
+// so it runs on the CUDA cores and is organised around moving bytes:
+//   - grid = (split, KV head, sequence); one CTA streams up to
+//     blocks_per_split 64-token blocks of ONE KV head and serves all
+//     Hq / Hkv query heads of that group from the same bytes;
+//   - one producer warp resolves block ids through the block table and moves
+//     each block's K and V tile (16 KB each, contiguous in the cache) with a
+//     single bulk-async copy apiece into a 3-stage shared-memory ring;
+//   - four consumer warps = eight groups of 16 lanes; a group owns 8 keys of
+//     every block and each lane 8 of the 128 head dims, so a key row is read
+//     from shared memory as one 256-byte conflict-free sweep, and the dot
+//     product is finished with a 4-step butterfly inside the 16 lanes;
+//   - each group runs its own online softmax (base 2, scale*log2(e) folded
+//     into Q) and the eight groups are merged at the end; the CTA writes one
+//     partial (O / l, log2-sum-exp) per query head and split, and the combine
+//     kernel merges the splits.
+// Sources: key j of sequence b lives in block block_table[b][j / 64], slot
+// j % 64, cache laid out [blocks, kv heads, 64, d] ("MLA Decode Attention
+// Kernel API Reference", kv_cache; the paged layout); decode is a separate
+// bandwidth-bound kernel (llama.cpp "ggml-metal: FA tensor path", the vec
+// decode rule); the split merge is the log-sum-exp ("D5") merge of the
+// nvfp4-megamoe-kernel notes.
+#include <cuda_runtime.h>
+#include <math.h>
+
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace fa {
+
+static __device__ int g_decode_err;
+
+constexpr int PD_D = 128;
+constexpr int PD_BS = 64;
+constexpr int PD_NST = 3;
+constexpr int PD_TILE = PD_BS * PD_D * 2;        // bytes of one block of K (or V) for one head
+constexpr int PD_STAGE = 2 * PD_TILE;            // K + V
+constexpr int PD_OFF_BAR = PD_NST * PD_STAGE;
+constexpr int PD_SMEM = PD_OFF_BAR + 128 + 128;  // ring + barriers + alignment slack
+
+struct PagedArgs {
+    const __nv_bfloat16 *q;
+    const __nv_bfloat16 *k_cache, *v_cache;
+    const int32_t *block_table, *seq_lens;
+    int max_blocks, Hq, Hkv, num_blocks, bps, num_splits;
+    float scale_log2;
+    float *part_o, *part_lse;
+};
+
+FA_DEV void bf16x8_to_f32(const uint4 &u, float (&f)[8]) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        f[2 * i] = __uint_as_float(w[i] << 16);
+        f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+}
+
+template <int G>
+__global__ void __launch_bounds__(160) paged_decode_kernel(const PagedArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+    const int split = blockIdx.x, hkv = blockIdx.y, b = blockIdx.z;
+
+    int seq_len = a.seq_lens[b];
+    if (seq_len < 0) seq_len = 0;
+    int nb = (seq_len + PD_BS - 1) / PD_BS;
+    if (nb > a.max_blocks) {
+        if (threadIdx.x == 0 && split == 0 && hkv == 0) atomicCAS(&g_decode_err, 0, 2 /* FA_DEVERR_BAD_BLOCK */);
+        nb = a.max_blocks;
+        seq_len = nb * PD_BS;
+    }
+    const int blk0 = split * a.bps;
+    if (blk0 >= nb) return;  // this split holds no key of this sequence (uniform exit)
+    const int nblk = min(a.bps, nb - blk0);
+
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t bar0 = sbase + PD_OFF_BAR;
+    auto full = [&](int s) { return bar0 + 8u * s; };
+    auto empty = [&](int s) { return bar0 + 8u * (PD_NST + s); };
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + PD_OFF_BAR + 8 * 2 * PD_NST);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < PD_NST; ++s) {
+            mbar_init(full(s), 1);
+            mbar_init(empty(s), 4);
+        }
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
+
+    if (warp == 4) {
+        // ---------------------------------------------------- producer --
+        const int32_t *tbl = a.block_table + (int64_t)b * a.max_blocks + blk0;
+        int32_t ids = 0;
+        for (int i = 0; i < nblk; ++i) {
+            if ((i & 31) == 0) {
+                ids = (i + lane < nblk) ? tbl[i + lane] : 0;
+                if (ids < 0 || ids >= a.num_blocks) {
+                    if (i + lane < nblk) atomicCAS(&g_decode_err, 0, 2 /* FA_DEVERR_BAD_BLOCK */);
+                    ids = 0;  // read block 0 instead of faulting
+                }
+            }
+            const int blk = __shfl_sync(0xffffffffu, ids, i & 31);
+            const int s = i % PD_NST;
+            const uint32_t ph = (uint32_t)(i / PD_NST) & 1u;
+            bool ok = true;
+            if (lane == 0) ok = mbar_wait(empty(s), ph ^ 1u, abort_flag, &g_decode_err);
+            if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
+            if (lane == 0) {
+                const int64_t off = ((int64_t)blk * a.Hkv + hkv) * (PD_BS * PD_D);
+                mbar_arrive_expect_tx(full(s), PD_STAGE);
+                bulk_load(sbase + s * PD_STAGE, a.k_cache + off, PD_TILE, full(s));
+                bulk_load(sbase + s * PD_STAGE + PD_TILE, a.v_cache + off, PD_TILE, full(s));
+            }
+        }
+        if (lane == 0 && *abort_flag) {
+            for (int i = max(0, nblk - PD_NST); i < nblk; ++i)
+                mbar_wait_drain(full(i % PD_NST), (uint32_t)(i / PD_NST) & 1u);
+        }
+        return;
+    }
+
+    // --------------------------------------------------------- consumers --
+    const int gi = warp * 2 + (lane >> 4);  // key group: keys [8 gi, 8 gi + 8) of each block
+    const int l16 = lane & 15;              // head dims [8 l16, 8 l16 + 8)
+    float qf[G][8];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+        const uint4 u = *reinterpret_cast<const uint4 *>(a.q + ((int64_t)b * a.Hq + hkv * G + g) * PD_D + l16 * 8);
+        bf16x8_to_f32(u, qf[g]);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) qf[g][e] *= a.scale_log2;
+    }
+    float m[G], l[G], o[G][8];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+        m[g] = -INFINITY;
+        l[g] = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) o[g][e] = 0.f;
+    }
+
+    bool ok = true;
+    for (int i = 0; i < nblk; ++i) {
+        const int s = i % PD_NST;
+        if (!mbar_wait(full(s), (uint32_t)(i / PD_NST) & 1u, abort_flag, &g_decode_err)) {
+            ok = false;
+            break;
+        }
+        const uint8_t *Ks = smem + s * PD_STAGE;
+        const uint8_t *Vs = Ks + PD_TILE;
+        const int j0 = (blk0 + i) * PD_BS + gi * 8;
+        float sc[8][G];
+#pragma unroll
+        for (int tt = 0; tt < 8; ++tt) {
+            float kf[8];
+            bf16x8_to_f32(*reinterpret_cast<const uint4 *>(Ks + (gi * 8 + tt) * 256 + l16 * 16), kf);
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                float part = 0.f;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) part = fmaf(qf[g][e], kf[e], part);
+                sc[tt][g] = part;
+            }
+        }
+#pragma unroll
+        for (int off = 8; off >= 1; off >>= 1)
+#pragma unroll
+            for (int tt = 0; tt < 8; ++tt)
+#pragma unroll
+                for (int g = 0; g < G; ++g) sc[tt][g] += __shfl_xor_sync(0xffffffffu, sc[tt][g], off);
+        const int nvalid = seq_len - j0;  // keys tt < nvalid are real
+#pragma unroll
+        for (int tt = 0; tt < 8; ++tt)
+            if (tt >= nvalid)
+#pragma unroll
+                for (int g = 0; g < G; ++g) sc[tt][g] = -INFINITY;
+        float p[8][G];
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            float mt = sc[0][g];
+#pragma unroll
+            for (int tt = 1; tt < 8; ++tt) mt = fmaxf(mt, sc[tt][g]);
+            const float mn = fmaxf(m[g], mt);
+            const float msub = (mn == -INFINITY) ? 0.f : mn;
+            const float alpha = ex2(m[g] - msub);
+            float ps = 0.f;
+#pragma unroll
+            for (int tt = 0; tt < 8; ++tt) {
+                p[tt][g] = ex2(sc[tt][g] - msub);
+                ps += p[tt][g];
+            }
+            l[g] = l[g] * alpha + ps;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) o[g][e] *= alpha;
+            m[g] = mn;
+        }
+#pragma unroll
+        for (int tt = 0; tt < 8; ++tt) {
+            float vf[8];
+            bf16x8_to_f32(*reinterpret_cast<const uint4 *>(Vs + (gi * 8 + tt) * 256 + l16 * 16), vf);
+#pragma unroll
+            for (int g = 0; g < G; ++g)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) o[g][e] = fmaf(p[tt][g], vf[e], o[g][e]);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty(s));
+    }
+
+    // ---- merge the eight key groups (the ring is free: every copy landed) ----
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    float *mo = reinterpret_cast<float *>(smem);    // [8][G][128]
+    float *mm = mo + 8 * G * PD_D;                  // [8][G]
+    float *ml = mm + 8 * G;                         // [8][G]
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) mo[(gi * G + g) * PD_D + l16 * 8 + e] = o[g][e];
+        if (l16 == 0) {
+            mm[gi * G + g] = m[g];
+            ml[gi * G + g] = l[g];
+        }
+    }
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    const int d = threadIdx.x;  // 0..127
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+        float M = -INFINITY;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) M = fmaxf(M, mm[k * G + g]);
+        const float msub = (M == -INFINITY) ? 0.f : M;
+        float L = 0.f, O = 0.f;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const float w = ex2(mm[k * G + g] - msub);
+            L = fmaf(w, ml[k * G + g], L);
+            O = fmaf(w, mo[(k * G + g) * PD_D + d], O);
+        }
+        const int64_t row = ((int64_t)b * a.Hq + hkv * G + g) * a.num_splits + split;
+        const bool good = ok && L > 0.f;
+        a.part_o[row * PD_D + d] = good ? O / L : 0.f;
+        if (d == 0) a.part_lse[row] = good ? msub + __log2f(L) : -INFINITY;
+    }
+}
+
+// ----------------------------------------------------------------------------
+// Log-sum-exp combine: one warp per (sequence or token, query head) merges
+// its splits' partials (O_s normalised by its own sum, lse_s in log2 units):
+//   M = max_s lse_s,  w_s = 2^(lse_s - M),  O = sum_s w_s O_s / sum_s w_s,
+//   LSE = (M + log2 sum_s w_s) * ln 2;  no valid split -> O = 0, LSE = -inf.
+struct CombineArgs {
+    const float *part_o, *part_lse;
+    int rows, num_splits, Hq;
+    // Number of splits that exist for a row: paged mode derives it from the
+    // sequence length, gather mode uses every split.
+    const int32_t *seq_lens;
+    int bps;
+    void *o;
+    float *lse;
+    int o_bf16;
+};
+
+template <int D>
+__global__ void __launch_bounds__(128) lse_combine_kernel(const CombineArgs a) {
+    const int row = blockIdx.x * 4 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= a.rows) return;
+    int ns = a.num_splits;
+    if (a.seq_lens) {
+        int sl = a.seq_lens[row / a.Hq];
+        if (sl < 0) sl = 0;
+        const int nb = (sl + PD_BS - 1) / PD_BS;
+        ns = min(ns, (nb + a.bps - 1) / a.bps);
+    }
+    const float *pl = a.part_lse + (int64_t)row * a.num_splits;
+    float M = -INFINITY;
+    for (int s = lane; s < ns; s += 32) M = fmaxf(M, pl[s]);
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    constexpr int PER = D / 32;
+    float acc[PER];
+#pragma unroll
+    for (int i = 0; i < PER; ++i) acc[i] = 0.f;
+    float L = 0.f;
+    if (M != -INFINITY) {
+        for (int s = 0; s < ns; ++s) {
+            const float w = ex2(pl[s] - M);
+            if (w == 0.f) continue;
+            L += w;
+            const float4 *src = reinterpret_cast<const float4 *>(a.part_o + ((int64_t)row * a.num_splits + s) * D);
+#pragma unroll
+            for (int i = 0; i < PER / 4; ++i) {
+                const float4 v = src[lane + 32 * i];
+                acc[4 * i] = fmaf(w, v.x, acc[4 * i]);
+                acc[4 * i + 1] = fmaf(w, v.y, acc[4 * i + 1]);
+                acc[4 * i + 2] = fmaf(w, v.z, acc[4 * i + 2]);
+                acc[4 * i + 3] = fmaf(w, v.w, acc[4 * i + 3]);
+            }
+        }
+    }
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+#pragma unroll
+    for (int i = 0; i < PER / 4; ++i) {
+        const int64_t e = (int64_t)row * D + 4 * (lane + 32 * i);
+        if (a.o_bf16) {
+            uint2 w;
+            w.x = pack_bf16x2(acc[4 * i] * inv, acc[4 * i + 1] * inv);
+            w.y = pack_bf16x2(acc[4 * i + 2] * inv, acc[4 * i + 3] * inv);
+            *reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(a.o) + e) = w;
+        } else {
+            *reinterpret_cast<float4 *>(static_cast<float *>(a.o) + e) =
+                make_float4(acc[4 * i] * inv, acc[4 * i + 1] * inv, acc[4 * i + 2] * inv, acc[4 * i + 3] * inv);
+        }
+    }
+    if (lane == 0 && a.lse) a.lse[row] = L > 0.f ? (M + __log2f(L)) * 0.69314718055994530942f : -INFINITY;
+}
+
+cudaError_t launch_combine(const float *part_o, const float *part_lse, int rows, int num_splits, int Hq,
+                           const int32_t *seq_lens, int bps, void *o, float *lse, int o_bf16, int D,
+                           cudaStream_t stream) {
+    CombineArgs c;
+    c.part_o = part_o;
+    c.part_lse = part_lse;
+    c.rows = rows;
+    c.num_splits = num_splits;
+    c.Hq = Hq;
+    c.seq_lens = seq_lens;
+    c.bps = bps;
+    c.o = o;
+    c.lse = lse;
+    c.o_bf16 = o_bf16;
+    const unsigned grid = (unsigned)((rows + 3) / 4);
+    if (D == 128)
+        lse_combine_kernel<128><<<grid, 128, 0, stream>>>(c);
+    else if (D == 512)
+        lse_combine_kernel<512><<<grid, 128, 0, stream>>>(c);
+    else
+        return cudaErrorInvalidValue;
+    return cudaGetLastError();
+}
+
+template <int G>
+static cudaError_t launch_g(const PagedArgs &a, int B, cudaStream_t stream) {
+    auto kern = paged_decode_kernel<G>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, PD_SMEM);
+    if (e != cudaSuccess) return e;
+    dim3 grid((unsigned)a.num_splits, (unsigned)a.Hkv, (unsigned)B);
+    kern<<<grid, 160, PD_SMEM, stream>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_decode_paged(const PagedLaunch &L, cudaStream_t stream) {
+    PagedArgs a;
+    a.q = static_cast<const __nv_bfloat16 *>(L.q);
+    a.k_cache = static_cast<const __nv_bfloat16 *>(L.k_cache);
+    a.v_cache = static_cast<const __nv_bfloat16 *>(L.v_cache);
+    a.block_table = L.block_table;
+    a.seq_lens = L.seq_lens;
+    a.max_blocks = L.max_blocks_per_seq;
+    a.Hq = L.Hq;
+    a.Hkv = L.Hkv;
+    a.num_blocks = L.num_blocks;
+    a.bps = L.blocks_per_split;
+    a.num_splits = L.num_splits;
+    a.scale_log2 = L.scale * 1.4426950408889634f;
+    a.part_o = L.part_o;
+    a.part_lse = L.part_lse;
+    cudaError_t e;
+    switch (L.Hq / L.Hkv) {
+        case 1: e = launch_g<1>(a, L.B, stream); break;
+        case 2: e = launch_g<2>(a, L.B, stream); break;
+        case 4: e = launch_g<4>(a, L.B, stream); break;
+        case 8: e = launch_g<8>(a, L.B, stream); break;
+        default: return cudaErrorInvalidValue;
+    }
+    if (e != cudaSuccess) return e;
+    return launch_combine(L.part_o, L.part_lse, L.B * L.Hq, L.num_splits, L.Hq, L.seq_lens, L.blocks_per_split, L.o,
+                          L.lse, L.o_bf16, PD_D, stream);
+}
+
+cudaError_t decode_device_error(int clear, int *code) {
+    int v = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(&v, g_decode_err, sizeof(int));
+    if (e != cudaSuccess) return e;
+    *code = v;
+    if (clear && v) {
+        v = 0;
+        e = cudaMemcpyToSymbol(g_decode_err, &v, sizeof(int));
+    }
+    return e;
+}
+
+}  // namespace fa

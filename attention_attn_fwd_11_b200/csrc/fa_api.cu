@@ -1,0 +1,360 @@
+// fa_api.cu -- the exported C ABI (include/fa.h): argument validation, TMA
+// tensor-map encoding, workspace sizing, and kernel launch on the caller's
+// stream.  No allocation, no synchronisation, no CPU fallback.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "../../include/fa.h"
+#include "internal.h"
+
+namespace {
+
+thread_local char g_msg[512] = "";
+
+fa_status fail(fa_status st, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_msg, sizeof g_msg, fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+fa_status cuda_fail(cudaError_t e, const char *what) {
+    return fail(FA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// cuTensorMapEncodeTiled from the driver, looked up once at run time (no
+// link-time dependency on libcuda).
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+bool get_encoder() {
+    std::call_once(g_encode_once, [] {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    });
+    return g_encode != nullptr;
+}
+
+// 4-D bf16 tensor (d, S, H, B) with 128-byte swizzle and a box of
+// (64, box_rows, 1, 1).  Strides in elements.  Dimensions of extent 1 get a
+// packed stride (their stride is never used).
+fa_status encode_4d(CUtensorMap *m, const void *base, int d, int S, int H, int B, int64_t s_s, int64_t s_h,
+                    int64_t s_b, int box_rows, const char *name) {
+    cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)(S > 0 ? S : 1), (cuuint64_t)H, (cuuint64_t)B};
+    int64_t st[3] = {s_s, s_h, s_b};
+    int64_t packed = d;
+    for (int i = 0; i < 3; ++i) {
+        if (dims[i + 1] == 1) st[i] = packed;
+        packed = st[i] * (int64_t)dims[i + 1];
+    }
+    cuuint64_t strides[3];
+    for (int i = 0; i < 3; ++i) {
+        const int64_t bytes = st[i] * 2;
+        if (bytes <= 0 || bytes % 16 != 0 || bytes >= (int64_t(1) << 40))
+            return fail(FA_ERR_INVALID_ARG, "%s: stride %d (%lld elements) must be a positive multiple of 8", name,
+                        i, (long long)st[i]);
+        strides[i] = (cuuint64_t)bytes;
+    }
+    cuuint32_t box[4] = {64u, (cuuint32_t)box_rows, 1u, 1u};
+    cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box,
+                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(FA_ERR_CUDA, "%s: cuTensorMapEncodeTiled failed (%d)", name, (int)r);
+    return FA_OK;
+}
+
+// 2-D bf16 tensor [rows, cols] (row pitch in elements), 128-byte swizzle,
+// box (64, box_rows).
+fa_status encode_2d(CUtensorMap *m, const void *base, int64_t cols, int64_t rows, int64_t pitch, int box_rows,
+                    const char *name) {
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)(pitch * 2)};
+    if ((pitch * 2) % 16 != 0) return fail(FA_ERR_INVALID_ARG, "%s: row pitch must be a multiple of 8", name);
+    cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1u, 1u};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
+                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(FA_ERR_CUDA, "%s: cuTensorMapEncodeTiled failed (%d)", name, (int)r);
+    return FA_OK;
+}
+
+bool finite_pos(float x) { return isfinite(x) && x > 0.f; }
+
+// ---------------------------------------------------------------- paged --
+
+int paged_splits(const fa_decode_paged_params *p) {
+    if (p->num_splits > 0) return p->num_splits < p->max_blocks_per_seq ? p->num_splits : p->max_blocks_per_seq;
+    // Automatic: enough (sequence, KV head, split) units to fill every SM
+    // several times over, with splits of at least 8 blocks.
+    const long long units = (long long)p->B * p->Hkv;
+    const long long want = 148LL * 2 * 6;
+    long long s = (want + units - 1) / units;
+    long long max_by_len = (p->max_blocks_per_seq + 7) / 8;
+    if (s > max_by_len) s = max_by_len;
+    if (s < 1) s = 1;
+    return (int)s;
+}
+
+fa_status check_paged(const fa_decode_paged_params *p) {
+    if (!p) return fail(FA_ERR_INVALID_ARG, "fa_decode_paged: params is NULL");
+    if (p->B < 0 || p->Hq <= 0 || p->Hkv <= 0 || p->num_blocks <= 0 || p->max_blocks_per_seq <= 0)
+        return fail(FA_ERR_INVALID_ARG, "fa_decode_paged: B >= 0, Hq, Hkv, num_blocks, max_blocks_per_seq > 0");
+    if (p->Hq % p->Hkv != 0) return fail(FA_ERR_INVALID_ARG, "fa_decode_paged: Hq %% Hkv != 0");
+    if (p->dk != 128 || p->dv != 128 || p->block_size != 64)
+        return fail(FA_ERR_UNSUPPORTED, "fa_decode_paged: supported dk = dv = 128, block_size = 64 (got %d/%d/%d)",
+                    p->dk, p->dv, p->block_size);
+    const int g = p->Hq / p->Hkv;
+    if (g != 1 && g != 2 && g != 4 && g != 8)
+        return fail(FA_ERR_UNSUPPORTED, "fa_decode_paged: Hq / Hkv must be 1, 2, 4 or 8 (got %d)", g);
+    if (!finite_pos(p->scale)) return fail(FA_ERR_INVALID_ARG, "fa_decode_paged: scale must be finite and > 0");
+    if (p->o_dtype != FA_F32 && p->o_dtype != FA_BF16) return fail(FA_ERR_INVALID_ARG, "fa_decode_paged: o_dtype");
+    return FA_OK;
+}
+
+// Shapes (above) plus the tensor pointers, for the compute call.
+fa_status check_paged_ptrs(const fa_decode_paged_params *p) {
+    fa_status st = check_paged(p);
+    if (st != FA_OK || p->B == 0) return st;
+    if (!p->q || !p->k_cache || !p->v_cache || !p->block_table || !p->seq_lens || !p->o)
+        return fail(FA_ERR_INVALID_ARG, "fa_decode_paged: NULL tensor pointer");
+    if (!aligned16(p->q) || !aligned16(p->k_cache) || !aligned16(p->v_cache) || !aligned16(p->o))
+        return fail(FA_ERR_INVALID_ARG, "fa_decode_paged: q, caches and o must be 16-byte aligned");
+    if (((uintptr_t)p->lse & 3u) || ((uintptr_t)p->block_table & 3u) || ((uintptr_t)p->seq_lens & 3u))
+        return fail(FA_ERR_INVALID_ARG, "fa_decode_paged: lse, block_table, seq_lens must be 4-byte aligned");
+    return FA_OK;
+}
+
+size_t paged_ws_bytes(const fa_decode_paged_params *p, int splits) {
+    const size_t rows = (size_t)p->B * p->Hq * (size_t)splits;
+    size_t o = rows * 128 * sizeof(float);
+    o = (o + 255) & ~size_t(255);
+    return o + ((rows * sizeof(float) + 255) & ~size_t(255));
+}
+
+// --------------------------------------------------------------- gather --
+
+int gather_splits(const fa_decode_gather_params *p) {
+    const int max_s = (p->topk + 63) / 64 > 0 ? (p->topk + 63) / 64 : 1;
+    if (p->num_splits > 0) return p->num_splits < max_s ? p->num_splits : max_s;
+    // Automatic: about two waves of (token, split) units, at least 256 keys each.
+    const long long want = 148LL * 2;
+    long long s = (want + (p->T > 0 ? p->T : 1) - 1) / (p->T > 0 ? p->T : 1);
+    long long max_by_len = (p->topk + 255) / 256;
+    if (s > max_by_len) s = max_by_len;
+    if (s < 1) s = 1;
+    return (int)s;
+}
+
+fa_status check_gather(const fa_decode_gather_params *p) {
+    if (!p) return fail(FA_ERR_INVALID_ARG, "fa_decode_gather: params is NULL");
+    if (p->T < 0 || p->Hq <= 0 || p->topk < 0 || p->n_rows <= 0)
+        return fail(FA_ERR_INVALID_ARG, "fa_decode_gather: T >= 0, Hq > 0, topk >= 0, n_rows > 0");
+    if (p->dk != 576 || p->dv != 512 || p->v_offset != 64 || p->Hq != 128)
+        return fail(FA_ERR_UNSUPPORTED, "fa_decode_gather: supported dk = 576, dv = 512, v_offset = 64, Hq = 128");
+    if (p->row_stride < 576 || p->row_stride % 8 != 0)
+        return fail(FA_ERR_INVALID_ARG, "fa_decode_gather: row_stride must be >= 576 and a multiple of 8");
+    if (p->n_rows > 0x7fffffffLL) return fail(FA_ERR_INVALID_ARG, "fa_decode_gather: n_rows must fit in int32");
+    if (!finite_pos(p->scale)) return fail(FA_ERR_INVALID_ARG, "fa_decode_gather: scale must be finite and > 0");
+    if (p->o_dtype != FA_F32 && p->o_dtype != FA_BF16) return fail(FA_ERR_INVALID_ARG, "fa_decode_gather: o_dtype");
+    return FA_OK;
+}
+
+fa_status check_gather_ptrs(const fa_decode_gather_params *p) {
+    fa_status st = check_gather(p);
+    if (st != FA_OK || p->T == 0) return st;
+    if (!p->q || !p->kv_rows || !p->o || (p->topk > 0 && !p->idx))
+        return fail(FA_ERR_INVALID_ARG, "fa_decode_gather: NULL tensor pointer");
+    if (!aligned16(p->q) || !aligned16(p->kv_rows) || !aligned16(p->o))
+        return fail(FA_ERR_INVALID_ARG, "fa_decode_gather: q, kv_rows and o must be 16-byte aligned");
+    if (((uintptr_t)p->lse & 3u) || ((uintptr_t)p->idx & 3u) || ((uintptr_t)p->key_pos & 3u) ||
+        ((uintptr_t)p->q_pos & 3u))
+        return fail(FA_ERR_INVALID_ARG, "fa_decode_gather: lse, idx, key_pos, q_pos must be 4-byte aligned");
+    return FA_OK;
+}
+
+size_t gather_ws_bytes(const fa_decode_gather_params *p, int splits) {
+    const size_t rows = (size_t)p->T * p->Hq * (size_t)splits;
+    size_t o = rows * 512 * sizeof(float);
+    o = (o + 255) & ~size_t(255);
+    return o + ((rows * sizeof(float) + 255) & ~size_t(255));
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_version(void) { return 100; }
+
+const char *fa_last_error(void) { return g_msg; }
+
+fa_status fa_fwd(const fa_fwd_params *p, void *stream) {
+    if (!p) return fail(FA_ERR_INVALID_ARG, "fa_fwd: params is NULL");
+    if (p->B < 0 || p->Hq <= 0 || p->Hkv <= 0 || p->Sq < 0 || p->Sk < 0)
+        return fail(FA_ERR_INVALID_ARG, "fa_fwd: need B >= 0, Hq > 0, Hkv > 0, Sq >= 0, Sk >= 0");
+    if (p->Hq % p->Hkv != 0) return fail(FA_ERR_INVALID_ARG, "fa_fwd: Hq (%d) %% Hkv (%d) != 0", p->Hq, p->Hkv);
+    if (p->dk != p->dv || (p->dk != 64 && p->dk != 128 && p->dk != 256))
+        return fail(FA_ERR_UNSUPPORTED, "fa_fwd: supported dk = dv in {64, 128, 256} (got %d/%d)", p->dk, p->dv);
+    if (!finite_pos(p->scale)) return fail(FA_ERR_INVALID_ARG, "fa_fwd: scale must be finite and > 0");
+    if (p->o_dtype != FA_F32 && p->o_dtype != FA_BF16) return fail(FA_ERR_INVALID_ARG, "fa_fwd: o_dtype");
+    if ((long long)p->B * p->Hq > 0x7fffffffLL || p->Sq > (1 << 30) || p->Sk > (1 << 30))
+        return fail(FA_ERR_INVALID_ARG, "fa_fwd: sizes out of range");
+    if (p->B == 0 || p->Sq == 0) return FA_OK;
+    // k and v are never read when Sk == 0 (they may then be NULL).
+    if (!p->q || !p->o || (p->Sk > 0 && (!p->k || !p->v)))
+        return fail(FA_ERR_INVALID_ARG, "fa_fwd: NULL tensor pointer");
+    if (!aligned16(p->q) || !aligned16(p->o) || (p->Sk > 0 && (!aligned16(p->k) || !aligned16(p->v))))
+        return fail(FA_ERR_INVALID_ARG, "fa_fwd: q, k, v, o must be 16-byte aligned");
+    if ((uintptr_t)p->lse & 3u) return fail(FA_ERR_INVALID_ARG, "fa_fwd: lse must be 4-byte aligned");
+    const int ovec = p->o_dtype == FA_F32 ? 4 : 8;
+    if (p->o_ss % ovec || p->o_sh % ovec || p->o_sb % ovec || p->o_ss < p->dv)
+        return fail(FA_ERR_INVALID_ARG, "fa_fwd: o strides must be multiples of %d elements and o_ss >= dv", ovec);
+    if (!get_encoder()) return fail(FA_ERR_CUDA, "fa_fwd: cuTensorMapEncodeTiled is not available");
+
+    fa::PrefillLaunch L;
+    memset(&L, 0, sizeof L);
+    const int box_k = p->dk == 256 ? 64 : 128;
+    fa_status st;
+    st = encode_4d(&L.tmQ, p->q, p->dk, p->Sq, p->Hq, p->B, p->q_ss, p->q_sh, p->q_sb, 128, "fa_fwd q");
+    if (st != FA_OK) return st;
+    // With Sk == 0 no K/V tile is ever loaded; any valid map will do.
+    const void *kb = p->Sk > 0 ? p->k : p->q;
+    const void *vb = p->Sk > 0 ? p->v : p->q;
+    st = encode_4d(&L.tmK, kb, p->dk, p->Sk, p->Hkv, p->B, p->k_ss, p->k_sh, p->k_sb, box_k, "fa_fwd k");
+    if (st != FA_OK) return st;
+    st = encode_4d(&L.tmV, vb, p->dv, p->Sk, p->Hkv, p->B, p->v_ss, p->v_sh, p->v_sb, box_k, "fa_fwd v");
+    if (st != FA_OK) return st;
+    L.B = p->B;
+    L.Hq = p->Hq;
+    L.Hkv = p->Hkv;
+    L.Sq = p->Sq;
+    L.Sk = p->Sk;
+    L.dk = p->dk;
+    L.dv = p->dv;
+    L.scale = p->scale;
+    L.causal = p->causal ? 1 : 0;
+    L.o = p->o;
+    L.o_sb = p->o_sb;
+    L.o_sh = p->o_sh;
+    L.o_ss = p->o_ss;
+    L.o_bf16 = p->o_dtype == FA_BF16;
+    L.lse = p->lse;
+    cudaError_t e = fa::launch_prefill(L, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "fa_fwd: launch");
+    return FA_OK;
+}
+
+fa_status fa_decode_paged_workspace_size(const fa_decode_paged_params *p, size_t *bytes) {
+    fa_status st = check_paged(p);
+    if (st != FA_OK) return st;
+    if (!bytes) return fail(FA_ERR_INVALID_ARG, "fa_decode_paged_workspace_size: bytes is NULL");
+    *bytes = paged_ws_bytes(p, paged_splits(p));
+    return FA_OK;
+}
+
+fa_status fa_decode_paged(const fa_decode_paged_params *p, void *stream) {
+    fa_status st = check_paged_ptrs(p);
+    if (st != FA_OK) return st;
+    if (p->B == 0) return FA_OK;
+    const int splits = paged_splits(p);
+    const size_t need = paged_ws_bytes(p, splits);
+    if (!p->workspace || p->workspace_bytes < need || ((uintptr_t)p->workspace & 255u))
+        return fail(FA_ERR_WORKSPACE, "fa_decode_paged: workspace needs %zu bytes, 256-byte aligned", need);
+    fa::PagedLaunch L;
+    L.q = p->q;
+    L.k_cache = p->k_cache;
+    L.v_cache = p->v_cache;
+    L.block_table = p->block_table;
+    L.seq_lens = p->seq_lens;
+    L.max_blocks_per_seq = p->max_blocks_per_seq;
+    L.B = p->B;
+    L.Hq = p->Hq;
+    L.Hkv = p->Hkv;
+    L.num_blocks = p->num_blocks;
+    L.scale = p->scale;
+    L.num_splits = splits;
+    L.blocks_per_split = (p->max_blocks_per_seq + splits - 1) / splits;
+    L.o = p->o;
+    L.lse = p->lse;
+    L.o_bf16 = p->o_dtype == FA_BF16;
+    const size_t rows = (size_t)p->B * p->Hq * splits;
+    L.part_o = static_cast<float *>(p->workspace);
+    L.part_lse = reinterpret_cast<float *>(static_cast<char *>(p->workspace) +
+                                           ((rows * 128 * sizeof(float) + 255) & ~size_t(255)));
+    cudaError_t e = fa::launch_decode_paged(L, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "fa_decode_paged: launch");
+    return FA_OK;
+}
+
+fa_status fa_decode_gather_workspace_size(const fa_decode_gather_params *p, size_t *bytes) {
+    fa_status st = check_gather(p);
+    if (st != FA_OK) return st;
+    if (!bytes) return fail(FA_ERR_INVALID_ARG, "fa_decode_gather_workspace_size: bytes is NULL");
+    *bytes = gather_ws_bytes(p, gather_splits(p));
+    return FA_OK;
+}
+
+fa_status fa_decode_gather(const fa_decode_gather_params *p, void *stream) {
+    fa_status st = check_gather_ptrs(p);
+    if (st != FA_OK) return st;
+    if (p->T == 0) return FA_OK;
+    const int splits = gather_splits(p);
+    const size_t need = gather_ws_bytes(p, splits);
+    if (!p->workspace || p->workspace_bytes < need || ((uintptr_t)p->workspace & 255u))
+        return fail(FA_ERR_WORKSPACE, "fa_decode_gather: workspace needs %zu bytes, 256-byte aligned", need);
+    if (!get_encoder()) return fail(FA_ERR_CUDA, "fa_decode_gather: cuTensorMapEncodeTiled is not available");
+    fa::GatherLaunch L;
+    st = encode_2d(&L.tmQ, p->q, p->dk, (int64_t)p->T * p->Hq, p->dk, 128, "fa_decode_gather q");
+    if (st != FA_OK) return st;
+    L.q = p->q;
+    L.rows = p->kv_rows;
+    L.n_rows = p->n_rows;
+    L.row_stride = p->row_stride;
+    L.idx = p->idx;
+    L.key_pos = p->key_pos;
+    L.q_pos = p->q_pos;
+    L.topk = p->topk;
+    L.T = p->T;
+    L.Hq = p->Hq;
+    L.scale = p->scale;
+    L.num_splits = splits;
+    L.keys_per_split = ((p->topk + splits - 1) / splits + 63) / 64 * 64;
+    L.o = p->o;
+    L.lse = p->lse;
+    L.o_bf16 = p->o_dtype == FA_BF16;
+    const size_t rows = (size_t)p->T * p->Hq * splits;
+    L.part_o = static_cast<float *>(p->workspace);
+    L.part_lse = reinterpret_cast<float *>(static_cast<char *>(p->workspace) +
+                                           ((rows * 512 * sizeof(float) + 255) & ~size_t(255)));
+    cudaError_t e = fa::launch_decode_gather(L, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "fa_decode_gather: launch");
+    return FA_OK;
+}
+
+fa_status fa_device_error(int clear, int *code) {
+    if (!code) return fail(FA_ERR_INVALID_ARG, "fa_device_error: code is NULL");
+    int c1 = 0, c2 = 0, c3 = 0;
+    cudaError_t e = fa::prefill_device_error(clear, &c1);
+    if (e == cudaSuccess) e = fa::decode_device_error(clear, &c2);
+    if (e == cudaSuccess) e = fa::gather_device_error(clear, &c3);
+    if (e != cudaSuccess) return cuda_fail(e, "fa_device_error");
+    *code = c1 ? c1 : (c2 ? c2 : c3);
+    return FA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,67 @@
+// internal.h -- host-side interface between the C-ABI layer (fa_api.cu) and
+// the kernel translation units.  Not part of the public ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace fa {
+
+// ---- prefill -------------------------------------------------------------
+struct PrefillLaunch {
+    CUtensorMap tmQ, tmK, tmV;
+    int B, Hq, Hkv, Sq, Sk, dk, dv;
+    float scale;
+    int causal;
+    void *o;
+    int64_t o_sb, o_sh, o_ss;
+    int o_bf16;
+    float *lse;
+};
+// Returns cudaSuccess or the launch error.
+cudaError_t launch_prefill(const PrefillLaunch &L, cudaStream_t stream);
+// Reads (and optionally clears) the prefill kernels' device error word.
+cudaError_t prefill_device_error(int clear, int *code);
+
+// ---- paged decode --------------------------------------------------------
+struct PagedLaunch {
+    const void *q, *k_cache, *v_cache;
+    const int32_t *block_table, *seq_lens;
+    int max_blocks_per_seq, B, Hq, Hkv, num_blocks;
+    float scale;
+    int blocks_per_split, num_splits;
+    void *o;
+    float *lse;
+    int o_bf16;
+    float *part_o;    // [B*Hq, num_splits, 128]
+    float *part_lse;  // [B*Hq, num_splits]   (log2 units)
+};
+cudaError_t launch_decode_paged(const PagedLaunch &L, cudaStream_t stream);
+// Log-sum-exp merge of split partials (D = 128 or 512).  seq_lens != NULL:
+// paged mode (row r belongs to sequence r / Hq, which has
+// ceil(ceil(len / 64) / bps) splits); NULL: every split exists.
+cudaError_t launch_combine(const float *part_o, const float *part_lse, int rows, int num_splits, int Hq,
+                           const int32_t *seq_lens, int bps, void *o, float *lse, int o_bf16, int D,
+                           cudaStream_t stream);
+cudaError_t decode_device_error(int clear, int *code);
+
+// ---- latent gather decode ------------------------------------------------
+struct GatherLaunch {
+    CUtensorMap tmQ;  // q viewed as [T * Hq, dk], box 64 x 128, 128-byte swizzle
+    const void *q, *rows;
+    int64_t n_rows, row_stride;
+    const int32_t *idx, *key_pos, *q_pos;
+    int topk, T, Hq;
+    float scale;
+    int keys_per_split, num_splits;
+    void *o;
+    float *lse;
+    int o_bf16;
+    float *part_o;    // [T*Hq, num_splits, 512]
+    float *part_lse;  // [T*Hq, num_splits]  (log2 units)
+};
+cudaError_t launch_decode_gather(const GatherLaunch &L, cudaStream_t stream);
+cudaError_t gather_device_error(int clear, int *code);
+
+}  // namespace fa

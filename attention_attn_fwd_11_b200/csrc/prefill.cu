@@ -1,0 +1,410 @@
+// prefill.cu -- fused attention forward (prefill) for sm_100a.
+//
+// One CTA computes one 128-row query tile of one (batch, query head):
+//
+//   warp 0      TMA producer: Q tile once, then a ring of K and V tiles
+//               (128-byte swizzled shared memory, zero fill past Sk).
+//   warp 1      MMA issuer (one thread): S = Q K^T with tcgen05.mma into
+//               TMEM (two S buffers, so QK^T of tile t+1 overlaps the
+//               softmax of tile t), then O += P V with P read from TMEM.
+//   warps 2-5   softmax / correction / epilogue, one thread per query row:
+//               S row from TMEM -> scale + mask -> online softmax in base 2
+//               (scale*log2(e) folded into one FMA) -> P as bf16 written back
+//               into the S buffer it came from -> lazy O rescale -> final
+//               O / l and LSE.
+//
+// The pages this follows (prior art, not the blueprint):
+//  - "nvfp4-megamoe-kernel CURRENT_ISSUE.md" (UMMA FMHA notes): raw QK^T from
+//    the MMA with the 1/sqrt(HD) scale applied afterwards; K-steps of 16
+//    accumulated into one TMEM tile; tcgen05.fence::after_thread_sync between
+//    MMA completion and tcgen05.ld; 32x32b TMEM loads, one row per lane and
+//    four warps covering the 128 lanes; P written to TMEM and consumed by a
+//    TMEM-operand ("TS") MMA.
+//  - llama.cpp "ggml-metal: FA tensor path", kernel_flash_attn_ext_tensor_impl:
+//    online softmax whose running max may be any value >= the true max (it
+//    cancels in O / l), skipping the O rescale when the max did not move,
+//    issuing QK^T of the next chunk before PV of the current one, and the
+//    "sum == 0 -> 0" output rule.
+// Differences from those designs: the running max is kept per row and only
+// moved when it grows by more than 2^8 (so the O rescale is rare and
+// per-row); operands are staged by TMA with 128-byte swizzle instead of
+// per-K-tile hand-written layouts; PV runs as one N = dv MMA per 16 keys.
+#include <cuda_runtime.h>
+#include <math.h>
+
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace fa {
+
+static __device__ int g_prefill_err;
+
+struct PrefillArgs {
+    int Hq, group, Sq, Sk;
+    float scale_log2;
+    int causal;
+    char *o;
+    int64_t o_sb, o_sh, o_ss;
+    int o_bf16;
+    float *lse;
+};
+
+template <int D, int BN, int NST>
+struct PrefillCfg {
+    static constexpr int BM = 128;
+    static constexpr int NCH = D / 64;            // 128-byte chunks of the head dim
+    static constexpr int Q_CHUNK = BM * 128;      // bytes of one chunk of Q
+    static constexpr int KV_CHUNK = BN * 128;     // bytes of one chunk of K or V
+    static constexpr int Q_BYTES = BM * D * 2;
+    static constexpr int KV_BYTES = BN * D * 2;
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_K = Q_BYTES;
+    static constexpr int OFF_V = OFF_K + NST * KV_BYTES;
+    static constexpr int OFF_BAR = OFF_V + NST * KV_BYTES;
+    static constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;  // barriers + alignment slack
+    static constexpr int TMEM_COLS = 512;
+    static constexpr int T_O = 2 * BN;            // TMEM column of O (S0 at 0, S1 at BN)
+    static_assert(D % 64 == 0 && D <= 256, "head dim");
+    static_assert(BN % 64 == 0 && BN <= 128, "key tile");
+    static_assert(2 * BN + D <= TMEM_COLS, "TMEM budget");
+    static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+// Barrier slots (uint64 each).
+enum { B_QFULL = 0, B_DRAIN = 1, B_SFULL = 2, B_PREADY = 4, B_PVDONE = 6, B_RING = 7 };
+
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale when the max grows by > 2^8
+
+template <int D, int BN, int NST>
+__global__ void __launch_bounds__(192, 1)
+prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+               const __grid_constant__ CUtensorMap tmV, const PrefillArgs a) {
+    using C = PrefillCfg<D, BN, NST>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t sQ = sbase + C::OFF_Q, sK = sbase + C::OFF_K, sV = sbase + C::OFF_V;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
+    const uint32_t bar0 = smem_u32(bars);
+    auto bar = [&](int i) -> uint32_t { return bar0 + 8u * (uint32_t)i; };
+    auto k_full = [&](int s) { return bar(B_RING + s); };
+    auto k_empty = [&](int s) { return bar(B_RING + NST + s); };
+    auto v_full = [&](int s) { return bar(B_RING + 2 * NST + s); };
+    auto v_empty = [&](int s) { return bar(B_RING + 3 * NST + s); };
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + 32);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int b = blockIdx.x / a.Hq;
+    const int hq = blockIdx.x % a.Hq;
+    const int hkv = hq / a.group;
+    const int qt = a.causal ? (int)(gridDim.y - 1 - blockIdx.y) : (int)blockIdx.y;
+    const int q0 = qt * C::BM;
+
+    // KV tiles this query tile needs (causal: up to the last row's diagonal).
+    int n_tiles;
+    {
+        const int last_row = min(C::BM - 1, a.Sq - 1 - q0);
+        int kmax = a.Sk - 1;
+        if (a.causal) kmax = min(kmax, q0 + last_row + a.Sk - a.Sq);
+        n_tiles = kmax < 0 ? 0 : kmax / BN + 1;
+    }
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar(B_QFULL), 1);
+        mbar_init(bar(B_DRAIN), 1);
+        mbar_init(bar(B_SFULL), 1);
+        mbar_init(bar(B_SFULL + 1), 1);
+        mbar_init(bar(B_PREADY), 128);
+        mbar_init(bar(B_PREADY + 1), 128);
+        mbar_init(bar(B_PVDONE), 1);
+        for (int s = 0; s < NST; ++s) {
+            mbar_init(k_full(s), 1);
+            mbar_init(k_empty(s), 1);
+            mbar_init(v_full(s), 1);
+            mbar_init(v_empty(s), 1);
+        }
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_holder), C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer --
+        if (lane == 0 && n_tiles > 0) {
+            prefetch_tmap(&tmQ);
+            prefetch_tmap(&tmK);
+            prefetch_tmap(&tmV);
+            mbar_arrive_expect_tx(bar(B_QFULL), C::Q_BYTES);
+#pragma unroll
+            for (int c = 0; c < C::NCH; ++c)
+                tma_load_4d(sQ + c * C::Q_CHUNK, &tmQ, bar(B_QFULL), c * 64, q0, hq, b);
+            int issued_k = 0, issued_v = 0;
+            for (int t = 0; t < n_tiles; ++t) {
+                const int s = t % NST;
+                const uint32_t ph = (uint32_t)(t / NST) & 1u;
+                if (!mbar_wait(k_empty(s), ph ^ 1u, abort_flag, &g_prefill_err)) break;
+                mbar_arrive_expect_tx(k_full(s), C::KV_BYTES);
+#pragma unroll
+                for (int c = 0; c < C::NCH; ++c)
+                    tma_load_4d(sK + s * C::KV_BYTES + c * C::KV_CHUNK, &tmK, k_full(s), c * 64, t * BN, hkv, b);
+                issued_k = t + 1;
+                if (!mbar_wait(v_empty(s), ph ^ 1u, abort_flag, &g_prefill_err)) break;
+                mbar_arrive_expect_tx(v_full(s), C::KV_BYTES);
+#pragma unroll
+                for (int c = 0; c < C::NCH; ++c)
+                    tma_load_4d(sV + s * C::KV_BYTES + c * C::KV_CHUNK, &tmV, v_full(s), c * 64, t * BN, hkv, b);
+                issued_v = t + 1;
+            }
+            if (*abort_flag) {
+                // Let the copies already in flight land before the CTA exits.
+                mbar_wait_drain(bar(B_QFULL), 0);
+                for (int t = max(0, issued_k - NST); t < issued_k; ++t)
+                    mbar_wait_drain(k_full(t % NST), (uint32_t)(t / NST) & 1u);
+                for (int t = max(0, issued_v - NST); t < issued_v; ++t)
+                    mbar_wait_drain(v_full(t % NST), (uint32_t)(t / NST) & 1u);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------- MMA issuer --
+        if (lane == 0 && n_tiles > 0) {
+            constexpr uint32_t idesc_qk = idesc_bf16_f32(128, BN, false, false);
+            constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, false, true);
+            const uint32_t tO = tmem + C::T_O;
+            auto issue_qk = [&](int t) -> bool {
+                const int s = t % NST;
+                if (!mbar_wait(k_full(s), (uint32_t)(t / NST) & 1u, abort_flag, &g_prefill_err)) return false;
+                tc_fence_after();
+                const uint32_t tS = tmem + (uint32_t)((t & 1) * BN);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const int c = kk >> 2, sub = kk & 3;
+                    const uint64_t ad = sdesc_sw128(sQ + c * C::Q_CHUNK + sub * 32, 16, 1024);
+                    const uint64_t bd = sdesc_sw128(sK + s * C::KV_BYTES + c * C::KV_CHUNK + sub * 32, 16, 1024);
+                    mma_ss(tS, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(k_empty(s));
+                mma_commit(bar(B_SFULL + (t & 1)));
+                return true;
+            };
+            bool ok = mbar_wait(bar(B_QFULL), 0, abort_flag, &g_prefill_err) && issue_qk(0);
+            for (int t = 0; ok && t < n_tiles; ++t) {
+                if (t + 1 < n_tiles && !issue_qk(t + 1)) break;
+                if (!mbar_wait(bar(B_PREADY + (t & 1)), (uint32_t)(t >> 1) & 1u, abort_flag, &g_prefill_err)) break;
+                const int s = t % NST;
+                if (!mbar_wait(v_full(s), (uint32_t)(t / NST) & 1u, abort_flag, &g_prefill_err)) break;
+                tc_fence_after();
+                const uint32_t tP = tmem + (uint32_t)((t & 1) * BN);
+#pragma unroll
+                for (int kk = 0; kk < BN / 16; ++kk) {
+                    const uint64_t bd = sdesc_sw128(sV + s * C::KV_BYTES + kk * 2048, C::KV_CHUNK, 1024);
+                    mma_ts(tO, tP + kk * 8, bd, idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
+                }
+                mma_commit(v_empty(s));
+                mma_commit(bar(B_PVDONE));
+            }
+            // Nothing of ours may still run on the tensor core once TMEM is freed.
+            mma_commit(bar(B_DRAIN));
+            mbar_wait_drain(bar(B_DRAIN), 0);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------- softmax / correction / epilogue --
+        const int qd = warp & 3;                  // TMEM lane quadrant of this warp
+        const int row = qd * 32 + lane;           // row within the tile
+        const int qrow = q0 + row;                // query index
+        const uint32_t tl = tmem + ((uint32_t)(qd * 32) << 16);
+        const float c = a.scale_log2;
+        // keys j < lim_all are visible to this row
+        const int lim_all = a.causal ? min(a.Sk, qrow + a.Sk - a.Sq + 1) : a.Sk;
+        float m_run = -INFINITY, l_run = 0.f;
+        bool ok = true;
+        for (int t = 0; t < n_tiles; ++t) {
+            const int buf = t & 1;
+            if (!mbar_wait(bar(B_SFULL + buf), (uint32_t)(t >> 1) & 1u, abort_flag, &g_prefill_err)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            float x[BN];
+            {
+                uint32_t r[BN];
+#pragma unroll
+                for (int ch = 0; ch < BN / 32; ++ch)
+                    tmem_ld32(tl + (uint32_t)(buf * BN + ch * 32), *reinterpret_cast<uint32_t(*)[32]>(&r[ch * 32]));
+                tmem_wait_ld();
+                reg_fence(r);
+#pragma unroll
+                for (int i = 0; i < BN; ++i) x[i] = __uint_as_float(r[i]);
+            }
+            const int lim = lim_all - t * BN;
+            if (lim < BN) {
+#pragma unroll
+                for (int i = 0; i < BN; ++i)
+                    if (i >= lim) x[i] = -INFINITY;
+            }
+            float mx0 = x[0], mx1 = x[1], mx2 = x[2], mx3 = x[3];
+#pragma unroll
+            for (int i = 4; i < BN; i += 4) {
+                mx0 = fmaxf(mx0, x[i]);
+                mx1 = fmaxf(mx1, x[i + 1]);
+                mx2 = fmaxf(mx2, x[i + 2]);
+                mx3 = fmaxf(mx3, x[i + 3]);
+            }
+            const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * c;
+            const float m_new = fmaxf(m_run, m_tile);
+            const bool need = m_new > m_run + kRescaleThreshold;
+            float alpha = 1.f;
+            if (need) {
+                alpha = ex2(m_run - m_new);
+                l_run *= alpha;
+                m_run = m_new;
+            }
+            if (t > 0 && __any_sync(0xffffffffu, need)) {
+                // O must hold PV of tile t-1 before it is rescaled.
+                if (!mbar_wait(bar(B_PVDONE), (uint32_t)(t - 1) & 1u, abort_flag, &g_prefill_err)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                uint32_t r[32];
+#pragma unroll
+                for (int ch = 0; ch < D / 32; ++ch) {
+                    tmem_ld32(tl + (uint32_t)(C::T_O + ch * 32), r);
+                    tmem_wait_ld();
+                    reg_fence(r);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+                    tmem_st32(tl + (uint32_t)(C::T_O + ch * 32), r);
+                }
+            }
+            const float msub = (m_run == -INFINITY) ? 0.f : m_run;
+            float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+            for (int ch = 0; ch < BN / 64; ++ch) {
+                uint32_t pk[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const float p0 = ex2(fmaf(x[ch * 64 + 2 * i], c, -msub));
+                    const float p1 = ex2(fmaf(x[ch * 64 + 2 * i + 1], c, -msub));
+                    s0 += p0;
+                    s1 += p1;
+                    pk[i] = pack_bf16x2(p0, p1);
+                }
+                tmem_st32(tl + (uint32_t)(buf * BN + ch * 32), pk);
+            }
+            l_run += s0 + s1;
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar(B_PREADY + buf));
+        }
+        // ---- epilogue: O / l, LSE ----
+        bool have_o = ok && n_tiles > 0;
+        if (have_o) {
+            if (mbar_wait(bar(B_PVDONE), (uint32_t)(n_tiles - 1) & 1u, abort_flag, &g_prefill_err))
+                tc_fence_after();
+            else
+                have_o = false;
+        }
+        const bool store = qrow < a.Sq;
+        const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+        const int64_t ooff = (int64_t)b * a.o_sb + (int64_t)hq * a.o_sh + (int64_t)qrow * a.o_ss;
+#pragma unroll
+        for (int ch = 0; ch < D / 32; ++ch) {
+            uint32_t r[32];
+            if (have_o) {
+                tmem_ld32(tl + (uint32_t)(C::T_O + ch * 32), r);
+                tmem_wait_ld();
+                reg_fence(r);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) r[i] = 0u;
+            }
+            if (store) {
+                if (a.o_bf16) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(a.o + 2 * (ooff + ch * 32));
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        uint4 w;
+                        w.x = pack_bf16x2(__uint_as_float(r[8 * i + 0]) * inv_l, __uint_as_float(r[8 * i + 1]) * inv_l);
+                        w.y = pack_bf16x2(__uint_as_float(r[8 * i + 2]) * inv_l, __uint_as_float(r[8 * i + 3]) * inv_l);
+                        w.z = pack_bf16x2(__uint_as_float(r[8 * i + 4]) * inv_l, __uint_as_float(r[8 * i + 5]) * inv_l);
+                        w.w = pack_bf16x2(__uint_as_float(r[8 * i + 6]) * inv_l, __uint_as_float(r[8 * i + 7]) * inv_l);
+                        dst[i] = w;
+                    }
+                } else {
+                    float4 *dst = reinterpret_cast<float4 *>(a.o + 4 * (ooff + ch * 32));
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        dst[i] = make_float4(__uint_as_float(r[4 * i]) * inv_l, __uint_as_float(r[4 * i + 1]) * inv_l,
+                                             __uint_as_float(r[4 * i + 2]) * inv_l, __uint_as_float(r[4 * i + 3]) * inv_l);
+                }
+            }
+        }
+        if (store && a.lse)
+            a.lse[((int64_t)b * a.Hq + hq) * a.Sq + qrow] =
+                (l_run > 0.f) ? (m_run + __log2f(l_run)) * 0.69314718055994530942f : -INFINITY;
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+template <int D, int BN, int NST>
+static cudaError_t launch_cfg(const PrefillLaunch &L, cudaStream_t stream) {
+    using C = PrefillCfg<D, BN, NST>;
+    auto kern = prefill_kernel<D, BN, NST>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    PrefillArgs a;
+    a.Hq = L.Hq;
+    a.group = L.Hq / L.Hkv;
+    a.Sq = L.Sq;
+    a.Sk = L.Sk;
+    a.scale_log2 = L.scale * 1.4426950408889634f;
+    a.causal = L.causal;
+    a.o = static_cast<char *>(L.o);
+    a.o_sb = L.o_sb;
+    a.o_sh = L.o_sh;
+    a.o_ss = L.o_ss;
+    a.o_bf16 = L.o_bf16;
+    a.lse = L.lse;
+    dim3 grid((unsigned)(L.B * L.Hq), (unsigned)((L.Sq + 127) / 128));
+    kern<<<grid, 192, C::SMEM_BYTES, stream>>>(L.tmQ, L.tmK, L.tmV, a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_prefill(const PrefillLaunch &L, cudaStream_t stream) {
+    switch (L.dk) {
+        case 64: return launch_cfg<64, 128, 4>(L, stream);
+        case 128: return launch_cfg<128, 128, 2>(L, stream);
+        case 256: return launch_cfg<256, 64, 2>(L, stream);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t prefill_device_error(int clear, int *code) {
+    int v = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(&v, g_prefill_err, sizeof(int));
+    if (e != cudaSuccess) return e;
+    *code = v;
+    if (clear && v) {
+        v = 0;
+        e = cudaMemcpyToSymbol(g_prefill_err, &v, sizeof(int));
+    }
+    return e;
+}
+
+}  // namespace fa

@@ -1,0 +1,254 @@
+"""ctypes binding over libfa.so (include/fa.h).  Argument marshalling only:
+every step of the computation runs in the library's CUDA kernels.  PyTorch
+supplies device memory and the current stream.  There is no CPU fallback:
+if the library is missing or the tensors are not on a CUDA device, calls
+raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libfa.so")
+
+FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_WORKSPACE, FA_ERR_CUDA, FA_ERR_TIMEOUT = range(6)
+FA_F32, FA_BF16 = 0, 1
+STATUS_NAMES = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED", 3: "FA_ERR_WORKSPACE",
+                4: "FA_ERR_CUDA", 5: "FA_ERR_TIMEOUT"}
+
+_vp = ctypes.c_void_p
+_i32 = ctypes.c_int
+_i64 = ctypes.c_int64
+
+
+class FwdParams(ctypes.Structure):
+    _fields_ = [("q", _vp), ("k", _vp), ("v", _vp), ("o", _vp), ("lse", _vp),
+                ("B", _i32), ("Hq", _i32), ("Hkv", _i32), ("Sq", _i32), ("Sk", _i32), ("dk", _i32), ("dv", _i32),
+                ("q_sb", _i64), ("q_sh", _i64), ("q_ss", _i64),
+                ("k_sb", _i64), ("k_sh", _i64), ("k_ss", _i64),
+                ("v_sb", _i64), ("v_sh", _i64), ("v_ss", _i64),
+                ("o_sb", _i64), ("o_sh", _i64), ("o_ss", _i64),
+                ("scale", ctypes.c_float), ("causal", _i32), ("o_dtype", _i32)]
+
+
+class PagedParams(ctypes.Structure):
+    _fields_ = [("q", _vp), ("k_cache", _vp), ("v_cache", _vp), ("block_table", _vp), ("seq_lens", _vp),
+                ("max_blocks_per_seq", _i32), ("B", _i32), ("Hq", _i32), ("Hkv", _i32), ("dk", _i32),
+                ("dv", _i32), ("block_size", _i32), ("num_blocks", _i32), ("scale", ctypes.c_float),
+                ("num_splits", _i32), ("o", _vp), ("lse", _vp), ("o_dtype", _i32), ("workspace", _vp),
+                ("workspace_bytes", ctypes.c_size_t)]
+
+
+class GatherParams(ctypes.Structure):
+    _fields_ = [("q", _vp), ("kv_rows", _vp), ("n_rows", _i64), ("row_stride", _i64), ("dk", _i32), ("dv", _i32),
+                ("v_offset", _i32), ("idx", _vp), ("topk", _i32), ("key_pos", _vp), ("q_pos", _vp), ("T", _i32),
+                ("Hq", _i32), ("scale", ctypes.c_float), ("num_splits", _i32), ("o", _vp), ("lse", _vp),
+                ("o_dtype", _i32), ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t)]
+
+
+_lib = None
+
+
+def load():
+    """Load libfa.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError("libfa.so is not built (run python -m attention_attn_fwd_11_b200.build)")
+        lib = ctypes.CDLL(LIB_PATH)
+        lib.fa_fwd.argtypes = [ctypes.POINTER(FwdParams), _vp]
+        lib.fa_fwd.restype = _i32
+        lib.fa_decode_paged_workspace_size.argtypes = [ctypes.POINTER(PagedParams), ctypes.POINTER(ctypes.c_size_t)]
+        lib.fa_decode_paged_workspace_size.restype = _i32
+        lib.fa_decode_paged.argtypes = [ctypes.POINTER(PagedParams), _vp]
+        lib.fa_decode_paged.restype = _i32
+        lib.fa_decode_gather_workspace_size.argtypes = [ctypes.POINTER(GatherParams), ctypes.POINTER(ctypes.c_size_t)]
+        lib.fa_decode_gather_workspace_size.restype = _i32
+        lib.fa_decode_gather.argtypes = [ctypes.POINTER(GatherParams), _vp]
+        lib.fa_decode_gather.restype = _i32
+        lib.fa_last_error.argtypes = []
+        lib.fa_last_error.restype = ctypes.c_char_p
+        lib.fa_device_error.argtypes = [_i32, ctypes.POINTER(_i32)]
+        lib.fa_device_error.restype = _i32
+        lib.fa_version.restype = _i32
+        _lib = lib
+    return _lib
+
+
+class FAError(RuntimeError):
+    def __init__(self, status, msg):
+        super().__init__("%s: %s" % (STATUS_NAMES.get(status, status), msg))
+        self.status = status
+
+
+def _check(st):
+    if st != FA_OK:
+        raise FAError(st, load().fa_last_error().decode())
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return _vp(stream.cuda_stream)
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("libfa works on CUDA tensors only (no CPU fallback)")
+
+
+def _odt(dtype):
+    if dtype == torch.float32:
+        return FA_F32
+    if dtype == torch.bfloat16:
+        return FA_BF16
+    raise ValueError("output dtype must be float32 or bfloat16")
+
+
+# ------------------------------------------------------------------ prefill --
+
+def fwd_params(q, k, v, o, lse, scale, causal):
+    B, Hq, Sq, dk = q.shape
+    _, Hkv, Sk, dv = v.shape
+    p = FwdParams()
+    p.q, p.k, p.v, p.o, p.lse = _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse)
+    p.B, p.Hq, p.Hkv, p.Sq, p.Sk, p.dk, p.dv = B, Hq, Hkv, Sq, Sk, dk, dv
+    p.q_sb, p.q_sh, p.q_ss = q.stride(0), q.stride(1), q.stride(2)
+    p.k_sb, p.k_sh, p.k_ss = k.stride(0), k.stride(1), k.stride(2)
+    p.v_sb, p.v_sh, p.v_ss = v.stride(0), v.stride(1), v.stride(2)
+    p.o_sb, p.o_sh, p.o_ss = o.stride(0), o.stride(1), o.stride(2)
+    p.scale = scale
+    p.causal = 1 if causal else 0
+    p.o_dtype = _odt(o.dtype)
+    return p
+
+
+def fwd(q, k, v, scale=None, causal=False, out=None, return_lse=True, out_dtype=torch.float32, stream=None):
+    """O = softmax(scale * Q K^T + mask) V.  q [B,Hq,Sq,dk], k [B,Hkv,Sk,dk],
+    v [B,Hkv,Sk,dv] bf16 CUDA tensors (any strides, head dim contiguous).
+    Returns (O [B,Hq,Sq,dv], LSE [B,Hq,Sq] fp32 or None)."""
+    _need_cuda(q, k, v)
+    for t in (q, k, v):
+        if t.dtype != torch.bfloat16 or t.dim() != 4 or t.stride(3) != 1:
+            raise ValueError("q, k, v must be 4-D bf16 with a contiguous last dim")
+    B, Hq, Sq, dk = q.shape
+    dv = v.shape[3]
+    if scale is None:
+        scale = 1.0 / math.sqrt(dk)
+    if out is None:
+        out = torch.empty((B, Hq, Sq, dv), device=q.device, dtype=out_dtype)
+    lse = torch.empty((B, Hq, Sq), device=q.device, dtype=torch.float32) if return_lse else None
+    _check(load().fa_fwd(ctypes.byref(fwd_params(q, k, v, out, lse, scale, causal)), _stream(stream)))
+    return out, lse
+
+
+# ------------------------------------------------------------- paged decode --
+
+def paged_params(q, k_cache, v_cache, block_table, seq_lens, o, lse, scale, num_splits, ws):
+    B, Hq, dk = q.shape
+    nb, Hkv, bs, _ = k_cache.shape
+    p = PagedParams()
+    p.q, p.k_cache, p.v_cache = _ptr(q), _ptr(k_cache), _ptr(v_cache)
+    p.block_table, p.seq_lens = _ptr(block_table), _ptr(seq_lens)
+    p.max_blocks_per_seq = block_table.shape[1]
+    p.B, p.Hq, p.Hkv, p.dk, p.dv, p.block_size, p.num_blocks = B, Hq, Hkv, dk, v_cache.shape[3], bs, nb
+    p.scale = scale
+    p.num_splits = num_splits
+    p.o, p.lse = _ptr(o), _ptr(lse)
+    p.o_dtype = _odt(o.dtype) if o is not None else FA_F32
+    p.workspace = _ptr(ws)
+    p.workspace_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    return p
+
+
+def paged_workspace_bytes(q, k_cache, v_cache, block_table, seq_lens, num_splits=0):
+    p = paged_params(q, k_cache, v_cache, block_table, seq_lens, None, None, 1.0, num_splits, None)
+    n = ctypes.c_size_t(0)
+    _check(load().fa_decode_paged_workspace_size(ctypes.byref(p), ctypes.byref(n)))
+    return n.value
+
+
+def decode_paged(q, k_cache, v_cache, block_table, seq_lens, scale=None, num_splits=0, out=None,
+                 return_lse=True, out_dtype=torch.float32, workspace=None, stream=None):
+    """Split-KV decode over a paged cache.  q [B,Hq,dk]; caches
+    [num_blocks,Hkv,block_size,d]; block_table int32 [B,max_blocks];
+    seq_lens int32 [B].  Returns (O [B,Hq,dv], LSE [B,Hq] or None)."""
+    _need_cuda(q, k_cache, v_cache, block_table, seq_lens)
+    B, Hq, dk = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(dk)
+    if out is None:
+        out = torch.empty((B, Hq, v_cache.shape[3]), device=q.device, dtype=out_dtype)
+    lse = torch.empty((B, Hq), device=q.device, dtype=torch.float32) if return_lse else None
+    if workspace is None:
+        n = paged_workspace_bytes(q, k_cache, v_cache, block_table, seq_lens, num_splits)
+        workspace = torch.empty(max(n, 256), device=q.device, dtype=torch.uint8)
+    p = paged_params(q, k_cache, v_cache, block_table, seq_lens, out, lse, scale, num_splits, workspace)
+    _check(load().fa_decode_paged(ctypes.byref(p), _stream(stream)))
+    return out, lse
+
+
+# ------------------------------------------------------------ gather decode --
+
+def gather_params(q, rows, idx, key_pos, q_pos, o, lse, scale, num_splits, ws, dk=576, dv=512, v_offset=64):
+    T, Hq, _ = q.shape
+    p = GatherParams()
+    p.q, p.kv_rows = _ptr(q), _ptr(rows)
+    p.n_rows, p.row_stride = rows.shape[0], rows.stride(0)
+    p.dk, p.dv, p.v_offset = dk, dv, v_offset
+    p.idx, p.topk = _ptr(idx), idx.shape[1]
+    p.key_pos, p.q_pos = _ptr(key_pos), _ptr(q_pos)
+    p.T, p.Hq = T, Hq
+    p.scale = scale
+    p.num_splits = num_splits
+    p.o, p.lse = _ptr(o), _ptr(lse)
+    p.o_dtype = _odt(o.dtype) if o is not None else FA_F32
+    p.workspace = _ptr(ws)
+    p.workspace_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    return p
+
+
+def gather_workspace_bytes(q, rows, idx, num_splits=0):
+    p = gather_params(q, rows, idx, None, None, None, None, 1.0, num_splits, None)
+    n = ctypes.c_size_t(0)
+    _check(load().fa_decode_gather_workspace_size(ctypes.byref(p), ctypes.byref(n)))
+    return n.value
+
+
+def decode_gather(q, rows, idx, key_pos=None, q_pos=None, scale=None, num_splits=0, out=None, return_lse=True,
+                  out_dtype=torch.float32, workspace=None, stream=None):
+    """Latent sparse decode.  q [T,Hq,576]; rows [n_rows, >=576] bf16 (row
+    pitch = rows.stride(0)); idx int32 [T,topk] (-1 = empty); key_pos int32
+    [T,topk] or None; q_pos int32 [T] or None.
+    Returns (O [T,Hq,512], LSE [T,Hq] or None)."""
+    _need_cuda(q, rows, idx, key_pos, q_pos)
+    if rows.stride(1) != 1:
+        raise ValueError("rows must have a contiguous last dim")
+    T, Hq, dk = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(dk)
+    if out is None:
+        out = torch.empty((T, Hq, 512), device=q.device, dtype=out_dtype)
+    lse = torch.empty((T, Hq), device=q.device, dtype=torch.float32) if return_lse else None
+    if workspace is None:
+        n = gather_workspace_bytes(q, rows, idx, num_splits)
+        workspace = torch.empty(max(n, 256), device=q.device, dtype=torch.uint8)
+    p = gather_params(q, rows, idx, key_pos, q_pos, out, lse, scale, num_splits, workspace)
+    _check(load().fa_decode_gather(ctypes.byref(p), _stream(stream)))
+    return out, lse
+
+
+def device_error(clear=True) -> int:
+    """Device-side error word (FA_DEVERR_*); synchronises the device."""
+    c = _i32(0)
+    _check(load().fa_device_error(1 if clear else 0, ctypes.byref(c)))
+    return c.value

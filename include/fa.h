@@ -1,0 +1,203 @@
+/*
+ * fa.h -- C ABI of libfa.so: fused scaled-dot-product attention forward on
+ * NVIDIA B200 (sm_100a).
+ *
+ *   O = softmax(scale * Q K^T + mask) V,   LSE = log sum_j exp(scale * q.k_j)
+ *
+ * computed with an online (streaming) softmax in hand-written CUDA kernels.
+ * The operation and its arguments follow the statements of the problem on
+ * these pages:
+ *   - "ggml-metal: FA tensor path" (llama.cpp), kernel_flash_attn_ext_tensor_impl:
+ *     Q/K/V addressed by per-dimension strides with the head dimension
+ *     contiguous, scale applied to the raw Q.K product before the mask,
+ *     consecutive query heads sharing one KV head (GQA), fp32 output, and a
+ *     row whose softmax sum is zero written as zeros;
+ *   - "nvfp4-megamoe-kernel CURRENT_ISSUE.md" (UMMA FMHA notes): the MMA
+ *     yields the unscaled dot product and 1/sqrt(HD) is applied afterwards;
+ *     the split merge ("D5 merge formula");
+ *   - "MLA Decode Attention Kernel API Reference" (AWS Neuron NKI): decode
+ *     over indexer-selected rows of a latent cache whose rows are laid out
+ *     [k_pe | kv_latent], flat row indices, and a causal mask from key
+ *     positions against the query position.
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers on the current CUDA device,
+ *     owned by the caller; the library never allocates, frees or copies them,
+ *     never synchronises, and has no CPU fallback.
+ *   - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL is
+ *     the legacy default stream).  The parameter structs are read during the
+ *     call only.
+ *   - Element strides are in ELEMENTS (not bytes); the last (head) dimension
+ *     is always contiguous.
+ *   - bf16 inputs; fp32 accumulation; fp32 (default) or bf16 output.
+ *   - LSE outputs are natural-log, fp32; a row with no visible key gets O = 0
+ *     and LSE = -inf.
+ *   - Argument errors are detected on the host before any launch and return
+ *     FA_ERR_INVALID_ARG or FA_ERR_UNSUPPORTED with a message in
+ *     fa_last_error().  Launch failures return FA_ERR_CUDA.  Errors the
+ *     kernels find on the device (a block-table or row index out of range, a
+ *     pipeline wait that timed out) cannot be returned synchronously: they
+ *     are latched in a device word read by fa_device_error().
+ */
+#ifndef FA_H
+#define FA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FA_OK = 0,
+    FA_ERR_INVALID_ARG = 1,   /* a pointer, size, stride or alignment is wrong */
+    FA_ERR_UNSUPPORTED = 2,   /* valid, but a shape this build has no kernel for */
+    FA_ERR_WORKSPACE = 3,     /* workspace missing or smaller than required */
+    FA_ERR_CUDA = 4,          /* a CUDA runtime/driver call or launch failed */
+    FA_ERR_TIMEOUT = 5        /* device: a pipeline wait gave up (see fa_device_error) */
+} fa_status;
+
+typedef enum { FA_F32 = 0, FA_BF16 = 1 } fa_dtype;
+
+/* Device-side error codes latched by the kernels (fa_device_error). */
+enum {
+    FA_DEVERR_NONE = 0,
+    FA_DEVERR_TIMEOUT = 1,      /* an mbarrier wait exceeded its time limit */
+    FA_DEVERR_BAD_BLOCK = 2,    /* block_table entry outside [0, num_blocks) */
+    FA_DEVERR_BAD_ROW = 3       /* gather index outside [-1, n_rows) */
+};
+
+/*
+ * fa_fwd -- prefill / full attention.
+ *   q: [B, Hq, Sq, dk]   k: [B, Hkv, Sk, dk]   v: [B, Hkv, Sk, dv]   (bf16)
+ *   o: [B, Hq, Sq, dv]   (o_dtype)
+ *   lse: NULL, or [B, Hq, Sq] fp32 contiguous.
+ * Strides (elements) give batch / head / sequence steps; each must be a
+ * multiple of 8 (16 bytes) for q, k, v; base pointers 16-byte aligned.
+ * Query head hq reads KV head hq / (Hq / Hkv); Hq % Hkv == 0.
+ * causal != 0: key j is visible to query i iff j <= i + Sk - Sq
+ * (bottom-right aligned, so a single decode query sees every key).
+ * scale must be finite and > 0 (the caller passes 1/sqrt(dk) for standard
+ * attention).
+ * Supported: dk == dv in {64, 128, 256}; anything else is FA_ERR_UNSUPPORTED.
+ * Sq == 0 or B == 0 is a no-op; Sk == 0 writes O = 0, LSE = -inf.
+ */
+typedef struct {
+    const void *q, *k, *v;
+    void *o;
+    float *lse;
+    int B, Hq, Hkv, Sq, Sk, dk, dv;
+    int64_t q_sb, q_sh, q_ss;
+    int64_t k_sb, k_sh, k_ss;
+    int64_t v_sb, v_sh, v_ss;
+    int64_t o_sb, o_sh, o_ss;
+    float scale;
+    int causal;
+    int o_dtype; /* fa_dtype */
+} fa_fwd_params;
+
+fa_status fa_fwd(const fa_fwd_params *p, void *stream);
+
+/*
+ * fa_decode_paged -- one query token per sequence over a paged KV cache,
+ * split along the keys, partial results merged by a log-sum-exp combine.
+ *   q: [B, Hq, dk] bf16 contiguous.
+ *   k_cache: [num_blocks, Hkv, block_size, dk], v_cache: [num_blocks, Hkv,
+ *     block_size, dv], bf16 contiguous.
+ *   block_table: [B, max_blocks_per_seq] int32; key j of sequence b is slot
+ *     j % block_size of physical block block_table[b][j / block_size].
+ *     Entries past a sequence's last block are never read.
+ *   seq_lens: [B] int32, each in [0, max_blocks_per_seq * block_size].
+ *   o: [B, Hq, dv] (o_dtype) contiguous; lse: NULL or [B, Hq] fp32.
+ *   num_splits: 0 = choose automatically, else the number of key splits
+ *     per sequence (clamped to [1, max_blocks_per_seq]).
+ *   workspace: device scratch of at least fa_decode_paged_workspace_size()
+ *     bytes, 256-byte aligned; it holds the split partials and is
+ *     overwritten on every call.
+ * Supported: dk == dv == 128, block_size == 64, Hq / Hkv in {1, 2, 4, 8}.
+ * A block id outside [0, num_blocks) is latched as FA_DEVERR_BAD_BLOCK and
+ * block 0 is read in its place (the output for that sequence is then
+ * meaningless).
+ */
+typedef struct {
+    const void *q;
+    const void *k_cache, *v_cache;
+    const int32_t *block_table;
+    const int32_t *seq_lens;
+    int max_blocks_per_seq;
+    int B, Hq, Hkv, dk, dv, block_size, num_blocks;
+    float scale;
+    int num_splits;
+    void *o;
+    float *lse;
+    int o_dtype; /* fa_dtype */
+    void *workspace;
+    size_t workspace_bytes;
+} fa_decode_paged_params;
+
+/* Workspace bytes for these shapes and num_splits; reads no pointer field. */
+fa_status fa_decode_paged_workspace_size(const fa_decode_paged_params *p, size_t *bytes);
+fa_status fa_decode_paged(const fa_decode_paged_params *p, void *stream);
+
+/*
+ * fa_decode_gather -- latent (MLA-style) sparse decode: every query head of
+ * token t attends over the cache rows idx[t][0..topk) selected for it.
+ *   q: [T, Hq, dk] bf16 contiguous, laid out like a cache row (the RoPE part
+ *     first, then the latent part).
+ *   kv_rows: n_rows rows of bf16 at a pitch of row_stride elements
+ *     (row_stride % 8 == 0); key = row[0 : dk], value = row[v_offset :
+ *     v_offset + dv].
+ *   idx: [T, topk] int32 flat row indices; -1 marks an empty slot.
+ *   key_pos: NULL (a key's position is its row index) or [T, topk] int32.
+ *   q_pos: NULL (no causal mask) or [T] int32; slot j is visible to token t
+ *     iff idx[t][j] >= 0 and key_pos <= q_pos[t].
+ *   o: [T, Hq, dv] (o_dtype) contiguous; lse: NULL or [T, Hq] fp32.
+ *   num_splits: 0 = automatic, else the number of key splits per token.
+ *   workspace: at least fa_decode_gather_workspace_size() bytes, 256-byte
+ *     aligned, overwritten on every call.
+ * Supported: dk == 576, dv == 512, v_offset == 64, Hq == 128.
+ * An index >= n_rows or < -1 is latched as FA_DEVERR_BAD_ROW and the slot is
+ * treated as empty.
+ */
+typedef struct {
+    const void *q;
+    const void *kv_rows;
+    int64_t n_rows, row_stride;
+    int dk, dv, v_offset;
+    const int32_t *idx;
+    int topk;
+    const int32_t *key_pos;
+    const int32_t *q_pos;
+    int T, Hq;
+    float scale;
+    int num_splits;
+    void *o;
+    float *lse;
+    int o_dtype; /* fa_dtype */
+    void *workspace;
+    size_t workspace_bytes;
+} fa_decode_gather_params;
+
+/* Workspace bytes for these shapes and num_splits; reads no pointer field. */
+fa_status fa_decode_gather_workspace_size(const fa_decode_gather_params *p, size_t *bytes);
+fa_status fa_decode_gather(const fa_decode_gather_params *p, void *stream);
+
+/* Message for the last non-OK status returned on this host thread. */
+const char *fa_last_error(void);
+
+/*
+ * Reads the device error word (one of FA_DEVERR_*) of the current device into
+ * *code and, if clear != 0, resets it.  This call synchronises the device.
+ * Returns FA_ERR_CUDA if the read itself fails.
+ */
+fa_status fa_device_error(int clear, int *code);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_H */

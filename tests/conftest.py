@@ -8,3 +8,17 @@ if ROOT not in sys.path:
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA GPU (B200, sm_100a) and the built CUDA library")
+
+
+def pytest_collection_modifyitems(config, items):
+    # GPU tests need a CUDA device; without one they are skipped (never run on
+    # a CPU path).  On a GPU machine a missing library makes them FAIL.
+    import pytest
+    import torch
+
+    if torch.cuda.is_available():
+        return
+    skip = pytest.mark.skip(reason="no CUDA device")
+    for it in items:
+        if "gpu" in it.keywords:
+            it.add_marker(skip)

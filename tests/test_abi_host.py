@@ -1,0 +1,135 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every function include/fa.h declares, and rejects bad arguments before any
+CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from attention_attn_fwd_11_b200 import fa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = []
+    for h in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if h.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", h)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names += re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*(fa_[A-Za-z0-9_]+)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = fa.load()
+    names = declared_functions()
+    assert "fa_fwd" in names and "fa_decode_paged" in names and "fa_decode_gather" in names
+    for n in names:
+        assert hasattr(lib, n), "libfa.so does not export " + n
+
+
+def test_version():
+    assert fa.load().fa_version() >= 100
+
+
+def fwd_params(**kw):
+    p = fa.FwdParams()
+    base = dict(q=16, k=32, v=48, o=64, lse=0, B=1, Hq=2, Hkv=2, Sq=128, Sk=128, dk=128, dv=128,
+                q_sb=2 * 128 * 128, q_sh=128 * 128, q_ss=128, k_sb=2 * 128 * 128, k_sh=128 * 128, k_ss=128,
+                v_sb=2 * 128 * 128, v_sh=128 * 128, v_ss=128, o_sb=2 * 128 * 128, o_sh=128 * 128, o_ss=128,
+                scale=0.088, causal=1, o_dtype=0)
+    base.update(kw)
+    for k_, v_ in base.items():
+        setattr(p, k_, v_)
+    return p
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(dk=96, dv=96), fa.FA_ERR_UNSUPPORTED),
+    (dict(dk=128, dv=64), fa.FA_ERR_UNSUPPORTED),
+    (dict(Hq=3, Hkv=2), fa.FA_ERR_INVALID_ARG),
+    (dict(scale=0.0), fa.FA_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), fa.FA_ERR_INVALID_ARG),
+    (dict(q=0), fa.FA_ERR_INVALID_ARG),
+    (dict(k=8), fa.FA_ERR_INVALID_ARG),
+    (dict(lse=2), fa.FA_ERR_INVALID_ARG),
+    (dict(o_dtype=7), fa.FA_ERR_INVALID_ARG),
+    (dict(o_ss=130), fa.FA_ERR_INVALID_ARG),
+    (dict(Sq=-1), fa.FA_ERR_INVALID_ARG),
+])
+def test_fwd_rejects(kw, status):
+    lib = fa.load()
+    st = lib.fa_fwd(ctypes.byref(fwd_params(**kw)), None)
+    assert st == status, lib.fa_last_error()
+    assert lib.fa_last_error().decode().startswith("fa_fwd")
+
+
+def test_fwd_null_params_and_noop():
+    lib = fa.load()
+    assert lib.fa_fwd(None, None) == fa.FA_ERR_INVALID_ARG
+    assert lib.fa_fwd(ctypes.byref(fwd_params(Sq=0)), None) == fa.FA_OK  # nothing to do, no launch
+    assert lib.fa_fwd(ctypes.byref(fwd_params(B=0)), None) == fa.FA_OK
+
+
+def paged_params(**kw):
+    p = fa.PagedParams()
+    base = dict(q=16, k_cache=32, v_cache=48, block_table=64, seq_lens=80, max_blocks_per_seq=128, B=64, Hq=32,
+                Hkv=8, dk=128, dv=128, block_size=64, num_blocks=4608, scale=0.088, num_splits=0, o=96, lse=0,
+                o_dtype=0, workspace=0, workspace_bytes=0)
+    base.update(kw)
+    for k_, v_ in base.items():
+        setattr(p, k_, v_)
+    return p
+
+
+def test_paged_workspace_size_and_validation():
+    lib = fa.load()
+    n = ctypes.c_size_t(0)
+    assert lib.fa_decode_paged_workspace_size(ctypes.byref(paged_params()), ctypes.byref(n)) == fa.FA_OK
+    splits = min(128, max(1, -(-148 * 2 * 6 // (64 * 8))), (128 + 7) // 8)
+    rows = 64 * 32 * splits
+    assert n.value == ((rows * 128 * 4 + 255) // 256) * 256 + ((rows * 4 + 255) // 256) * 256
+    assert lib.fa_decode_paged_workspace_size(ctypes.byref(paged_params(num_splits=5)), ctypes.byref(n)) == 0
+    assert n.value == ((64 * 32 * 5 * 512 + 255) // 256) * 256 + ((64 * 32 * 5 * 4 + 255) // 256) * 256
+    # the workspace check happens before any launch
+    assert lib.fa_decode_paged(ctypes.byref(paged_params()), None) == fa.FA_ERR_WORKSPACE
+    assert lib.fa_decode_paged(ctypes.byref(paged_params(workspace=256, workspace_bytes=10)), None) == fa.FA_ERR_WORKSPACE
+    assert lib.fa_decode_paged(ctypes.byref(paged_params(dk=64, dv=64)), None) == fa.FA_ERR_UNSUPPORTED
+    assert lib.fa_decode_paged(ctypes.byref(paged_params(block_size=16)), None) == fa.FA_ERR_UNSUPPORTED
+    assert lib.fa_decode_paged(ctypes.byref(paged_params(Hq=24, Hkv=8)), None) == fa.FA_ERR_UNSUPPORTED
+    assert lib.fa_decode_paged(ctypes.byref(paged_params(Hq=30, Hkv=8)), None) == fa.FA_ERR_INVALID_ARG
+    assert lib.fa_decode_paged(ctypes.byref(paged_params(k_cache=40)), None) == fa.FA_ERR_INVALID_ARG
+    assert lib.fa_decode_paged(ctypes.byref(paged_params(B=0)), None) == fa.FA_OK
+
+
+def gather_params(**kw):
+    p = fa.GatherParams()
+    base = dict(q=16, kv_rows=32, n_rows=65536, row_stride=576, dk=576, dv=512, v_offset=64, idx=48, topk=2048,
+                key_pos=0, q_pos=64, T=32, Hq=128, scale=1 / 24, num_splits=0, o=80, lse=0, o_dtype=0,
+                workspace=0, workspace_bytes=0)
+    base.update(kw)
+    for k_, v_ in base.items():
+        setattr(p, k_, v_)
+    return p
+
+
+def test_gather_workspace_size_and_validation():
+    lib = fa.load()
+    n = ctypes.c_size_t(0)
+    assert lib.fa_decode_gather_workspace_size(ctypes.byref(gather_params()), ctypes.byref(n)) == fa.FA_OK
+    assert n.value > 0 and n.value % 256 == 0
+    assert lib.fa_decode_gather(ctypes.byref(gather_params()), None) == fa.FA_ERR_WORKSPACE
+    assert lib.fa_decode_gather(ctypes.byref(gather_params(dk=128)), None) == fa.FA_ERR_UNSUPPORTED
+    assert lib.fa_decode_gather(ctypes.byref(gather_params(Hq=64)), None) == fa.FA_ERR_UNSUPPORTED
+    assert lib.fa_decode_gather(ctypes.byref(gather_params(row_stride=580)), None) == fa.FA_ERR_INVALID_ARG
+    assert lib.fa_decode_gather(ctypes.byref(gather_params(idx=50)), None) == fa.FA_ERR_INVALID_ARG
+    assert lib.fa_decode_gather(ctypes.byref(gather_params(T=0)), None) == fa.FA_OK
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    q = torch.zeros(1, 1, 128, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        fa.fwd(q, q, q)
