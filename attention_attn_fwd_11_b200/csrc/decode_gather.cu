@@ -127,8 +127,27 @@ latent_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const GatherArgs a
             const int32_t *kp_t = a.key_pos ? a.key_pos + (int64_t)t * a.topk : nullptr;
             volatile int *go = reinterpret_cast<volatile int *>(tmem_holder + 2);
             bool ok = true;
+            int sig = 0;  // next tile whose arrival is still to be signalled
+            // A tile is signalled once this thread's copies for it have landed
+            // (wait_group), made visible to the tensor core's async proxy
+            // (fence.proxy.async), then counted on the tile's full barrier.
+            auto signal_through = [&](int last, bool leave_newest) {
+                while (sig <= last) {
+                    if (leave_newest)
+                        cp_async_wait<1>();
+                    else
+                        cp_async_wait<0>();
+                    fence_proxy_async_smem();
+                    mbar_arrive(bar(G_FULL + sig % LG_NST));
+                    ++sig;
+                }
+            };
             for (int i = 0; i < n_tiles; ++i) {
                 const int s = i % LG_NST;
+                // Stage s is freed by PV of tile i - NST, which the MMA issues
+                // only after QK^T of tile i - 1: signal everything issued so far
+                // before waiting for the stage.
+                if (i >= LG_NST) signal_through(i - 1, false);
                 // One thread waits for the stage to be free and publishes the
                 // outcome, so all 128 gatherers take the same branch below.
                 if (tid == 0)
@@ -168,17 +187,13 @@ latent_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const GatherArgs a
                     cp_async16(dst0 + c * LG_KCH + row * 128 + ((sub ^ (row & 7)) << 4), src);
                 }
                 cp_async_commit();
-                if (i >= 1) {
-                    cp_async_wait<1>();
-                    fence_proxy_async_smem();
-                    mbar_arrive(bar(G_FULL + (i - 1) % LG_NST));
-                }
+                // Tile i - 1 may be signalled while tile i is still in flight.
+                if (i >= 1) signal_through(i - 1, true);
             }
-            cp_async_wait<0>();
-            if (ok) {
-                fence_proxy_async_smem();
-                mbar_arrive(bar(G_FULL + (n_tiles - 1) % LG_NST));
-            }
+            if (ok)
+                signal_through(n_tiles - 1, false);
+            else
+                cp_async_wait<0>();
             if (tid == 0 && *abort_flag) mbar_wait_drain(bar(G_QFULL), 0);
         }
     } else if (warp == 8) {
@@ -285,9 +300,11 @@ latent_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const GatherArgs a
             for (int k = 0; k < 16; ++k) {
                 const float p0 = ex2(fmaf(x[2 * k], c, -msub));
                 const float p1 = ex2(fmaf(x[2 * k + 1], c, -msub));
-                s0 += p0;
-                s1 += p1;
                 pk[k] = pack_bf16x2(p0, p1);
+                // l sums the bf16-rounded weights the MMA actually uses, so O
+                // is an exactly normalised average of V rows.
+                s0 += __uint_as_float(pk[k] << 16);
+                s1 += __uint_as_float(pk[k] & 0xffff0000u);
             }
             l_run += s0 + s1;
             tmem_st16(tl + (uint32_t)(buf * LG_BN), pk);

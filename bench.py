@@ -1,0 +1,568 @@
+#!/usr/bin/env python
+"""Benchmark of the fused attention forward hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one pass of the path over one batch of synthetic input.  The
+headline workload is causal MHA prefill, B=2, H=16, S=2048, d=128 (bf16
+in, fp32 accumulate, fp32 out), reported in TFLOP/s with the causal-halved
+count 4*B*H*S*S*d/2.  The other workloads of this path (tiny full prefill,
+GQA d=256 prefill, paged GQA decode, latent sparse decode) are timed in the
+same run and reported under "workloads".
+
+Timing: inputs already resident in HBM; several copies of every input are
+rotated so that consecutive steps never find their operands in L2; steps are
+captured in a CUDA graph and the K timed steps are bracketed by CUDA events
+on the launching stream, with a barrier and a device synchronise on both
+sides; the time is the max over ranks.  nvidia-smi clocks are sampled while
+the timed region runs.  "e2e" repeats the headline through the public API
+with pinned host buffers, host<->device copies inside the timed region.
+
+Multi-GPU (torchrun): every rank runs its own replica of the workload (the
+path has no exchange step), value = all ranks' work / max time ("weak").
+
+--impl reference times the CPU fp64 oracle (the only other implementation
+of this path) on a bounded sample of the same workload, rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "attention TFLOP/s & % dense BF16 peak (prefill); decode HBM GB/s, 1×B200"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# dram__bytes_read.sum + dram__bytes_write.sum per launch from ncu, with the
+# profile summary it comes from; None until a capture of the current kernel.
+NCU_TRAFFIC = {}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-secondary", action="store_true", help="only the headline workload")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", default=None,
+                    help="time one named workload alone (for profiling), e.g. causal_mha_b2_h16_s2048_d128")
+    ap.add_argument("--eager", action="store_true", help="with --only: launch every step eagerly (no CUDA graph)")
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------ clocks --
+
+class ClockSampler:
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self, t_from=None, t_to=None):
+        """Summary of the samples taken between host times t_from and t_to."""
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        sm = []
+        mx = None
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                ts = time.mktime(time.strptime(r[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                ts += float("0." + r[0].split(".")[1]) if "." in r[0] else 0.0
+            except Exception:
+                ts = None
+            if t_from is not None and ts is not None and not (t_from - 0.05 <= ts <= t_to + 0.05):
+                continue
+            try:
+                sm.append(float(r[1]))
+                mx = float(r[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, r[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------- helpers --
+
+def rotation_copies(footprint_bytes, l2_bytes, cap=64):
+    """Copies of the inputs so that one cycle spans > 2x L2."""
+    return int(max(1, min(cap, math.ceil(2.0 * l2_bytes / max(footprint_bytes, 1)) + 1)))
+
+
+def time_graph(torch, launch, n_copies, K, W, dist=None, window=None):
+    """Capture one graph that runs `per_graph` steps (cycling over the input
+    copies), then time K steps.  Returns (ms_total, steps); if `window` is a
+    list, the host times around the timed region are appended to it."""
+    stream = torch.cuda.Stream()
+    per_graph = n_copies * max(1, min(50, K) // n_copies)
+    with torch.cuda.stream(stream):
+        for i in range(max(W, 1)):
+            launch(i % n_copies)
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(per_graph):
+            launch(i % n_copies)
+    reps, rem = divmod(K, per_graph)
+    with torch.cuda.stream(stream):
+        g.replay()  # graph warm-up
+    stream.synchronize()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_host0 = time.time()
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        for i in range(rem):
+            launch(i % n_copies)
+        e1.record(stream)
+    stream.synchronize()
+    torch.cuda.synchronize()
+    if window is not None:
+        window += [t_host0, time.time()]
+    if dist is not None:
+        dist.barrier()
+    ms = e0.elapsed_time(e1)
+    del g
+    return ms, K
+
+
+def max_over_ranks(torch, dist, x):
+    if dist is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(torch, dist, x):
+    if dist is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# --------------------------------------------------------------- workloads --
+
+def prefill_workload(torch, fa, W_, c, l2):
+    q0, k0, v0 = W_.prefill_inputs(c)
+    foot = (q0.numel() + k0.numel() + v0.numel()) * 2 + c.B * c.Hq * c.Sq * (c.dv * 4 + 4)
+    n = rotation_copies(foot, l2)
+    bufs = []
+    for i in range(n):
+        q, k, v = q0.cuda(), k0.cuda(), v0.cuda()
+        o = torch.empty(c.B, c.Hq, c.Sq, c.dv, device="cuda")
+        lse = torch.empty(c.B, c.Hq, c.Sq, device="cuda")
+        bufs.append((q, k, v, o, lse))
+    import ctypes
+    lib = fa.load()
+    params = [fa.fwd_params(q, k, v, o, lse, c.scale, c.causal) for (q, k, v, o, lse) in bufs]
+
+    def launch(i):
+        st = lib.fa_fwd(ctypes.byref(params[i]), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+        if st != 0:
+            raise RuntimeError(lib.fa_last_error().decode())
+
+    launch.keep = bufs  # the launches hold raw pointers into these tensors
+    return launch, n, foot, 1
+
+
+def paged_workload(torch, fa, W_, c, l2):
+    q0, kc0, vc0, tb0, sl0 = W_.paged_inputs(c)
+    byts = W_.paged_bytes(c, sl0, tb0.shape[1])
+    foot = (kc0.numel() + vc0.numel()) * 2
+    n = rotation_copies(foot, l2)
+    import ctypes
+    lib = fa.load()
+    bufs, params = [], []
+    for i in range(n):
+        q, kc, vc, tb, sl = q0.cuda(), kc0.cuda(), vc0.cuda(), tb0.cuda(), sl0.cuda()
+        o = torch.empty(c.B, c.Hq, c.dv, device="cuda")
+        lse = torch.empty(c.B, c.Hq, device="cuda")
+        nws = fa.paged_workspace_bytes(q, kc, vc, tb, sl, 0)
+        ws = torch.empty(nws, dtype=torch.uint8, device="cuda")
+        bufs.append((q, kc, vc, tb, sl, o, lse, ws))
+        params.append(fa.paged_params(q, kc, vc, tb, sl, o, lse, c.scale, 0, ws))
+
+    def launch(i):
+        st = lib.fa_decode_paged(ctypes.byref(params[i]), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+        if st != 0:
+            raise RuntimeError(lib.fa_last_error().decode())
+
+    launch.keep = bufs  # the launches hold raw pointers into these tensors
+    return launch, n, byts, 2
+
+
+def latent_workload(torch, fa, W_, c, l2):
+    q0, rows0, idx0, qpos0 = W_.latent_inputs(c)
+    nvis = W_.latent_visible(idx0, qpos0)
+    byts = W_.latent_bytes(c, nvis)
+    flops = W_.latent_flops(c, nvis)
+    n = rotation_copies(byts, l2)
+    import ctypes
+    lib = fa.load()
+    bufs, params = [], []
+    for i in range(n):
+        q, rows, idx, qpos = q0.cuda(), rows0.cuda(), idx0.cuda(), qpos0.cuda()
+        o = torch.empty(c.T, c.Hq, c.dv, device="cuda")
+        lse = torch.empty(c.T, c.Hq, device="cuda")
+        nws = fa.gather_workspace_bytes(q, rows, idx, 0)
+        ws = torch.empty(nws, dtype=torch.uint8, device="cuda")
+        bufs.append((q, rows, idx, qpos, o, lse, ws))
+        params.append(fa.gather_params(q, rows, idx, None, qpos, o, lse, c.scale, 0, ws))
+
+    def launch(i):
+        st = lib.fa_decode_gather(ctypes.byref(params[i]), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+        if st != 0:
+            raise RuntimeError(lib.fa_last_error().decode())
+
+    launch.keep = bufs  # the launches hold raw pointers into these tensors
+    return launch, n, (byts, flops), 2
+
+
+def roofline(bound, achieved, peak, unit, traffic):
+    return {"bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": unit,
+            "frac": round(achieved / peak, 4), "traffic": traffic}
+
+
+# ------------------------------------------------------------ CPU baseline --
+
+def cpu_baseline_prefill(c, budget_s=10.0, max_s=30.0, max_slices=None):
+    """Time the fp64 oracle on whole (batch, head) slices of the workload
+    (all query rows, causal mask as in the workload) until ~budget_s."""
+    import numpy as np
+
+    import oracle
+    from attention_attn_fwd_11_b200 import workloads as W_
+
+    q, k, v = W_.prefill_inputs(c)
+    qb, kb, vb = W_.bits(q), W_.bits(k), W_.bits(v)
+    grp = c.Hq // c.Hkv
+    slices = [(b, h) for b in range(c.B) for h in range(c.Hq)]
+    if max_slices:
+        slices = slices[:max_slices]
+    done, t0 = 0, time.perf_counter()
+    for (b, h) in slices:
+        oracle.attention(np.ascontiguousarray(qb[b:b + 1, h:h + 1]), np.ascontiguousarray(kb[b:b + 1, h // grp:h // grp + 1]),
+                         np.ascontiguousarray(vb[b:b + 1, h // grp:h // grp + 1]), c.scale, c.causal)
+        done += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or el >= max_s:
+            break
+    el = time.perf_counter() - t0
+    flops = c.flops * done / len([(b, h) for b in range(c.B) for h in range(c.Hq)])
+    return {"value": round(flops / el / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": "%d of %d (batch, head) slices, all %d query rows each, %.1f s" % (done, c.B * c.Hq, c.Sq, el)}
+
+
+# -------------------------------------------------------------------- main --
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from attention_attn_fwd_11_b200 import workloads as W_
+
+    c = W_.CAUSAL_MHA
+    import numpy as np
+
+    import oracle
+
+    q, k, v = W_.prefill_inputs(c)
+    qb, kb, vb = W_.bits(q), W_.bits(k), W_.bits(v)
+    slices = [(b, h) for b in range(c.B) for h in range(c.Hq)]
+
+    def step(i):
+        b, h = slices[i % len(slices)]
+        oracle.attention(np.ascontiguousarray(qb[b:b + 1, h:h + 1]), np.ascontiguousarray(kb[b:b + 1, h:h + 1]),
+                         np.ascontiguousarray(vb[b:b + 1, h:h + 1]), c.scale, c.causal)
+
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(args.warmup + i)
+    el = time.perf_counter() - t0
+    flops = c.flops / len(slices) * args.steps
+    val = flops / el / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": round(val, 6), "unit": "TFLOP/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(el * 1e3 / max(args.steps, 1), 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": c.name, "B": c.B, "Hq": c.Hq, "Hkv": c.Hkv, "Sq": c.Sq, "Sk": c.Sk, "d": c.dk,
+                       "causal": c.causal, "step": "one (batch, head) slice of the workload, all query rows"},
+            "cpu_baseline": {"value": round(val, 6), "unit": "TFLOP/s", "kind": "oracle",
+                             "cores": oracle.num_threads(),
+                             "sample": "one (batch, head) slice per step (1/%d of the workload)" % len(slices)},
+            "e2e": {"value": round(val, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_only(args):
+    """One workload alone, eager or graph-launched: the command the ncu
+    profiles under profiles/ were taken with."""
+    import torch
+
+    from attention_attn_fwd_11_b200 import fa
+    from attention_attn_fwd_11_b200 import workloads as W_
+
+    torch.cuda.set_device(0)
+    l2 = torch.cuda.get_device_properties(0).L2_cache_size
+    table = {c.name: c for c in (W_.TINY_FULL, W_.CAUSAL_MHA, W_.GQA_FULL, W_.PAGED_GQA, W_.LATENT_SPARSE)}
+    if args.only not in table:
+        raise SystemExit("unknown workload %r; one of %s" % (args.only, sorted(table)))
+    c = table[args.only]
+    if isinstance(c, W_.PrefillCase):
+        launch, n, work, kpl = prefill_workload(torch, fa, W_, c, l2)
+        unit, amount = "TFLOP/s", c.flops / 1e12
+    elif isinstance(c, W_.PagedCase):
+        launch, n, work, kpl = paged_workload(torch, fa, W_, c, l2)
+        unit, amount = "GB/s", work / 1e9
+    else:
+        launch, n, work, kpl = latent_workload(torch, fa, W_, c, l2)
+        unit, amount = "GB/s", work[0] / 1e9
+    if args.eager:
+        s = torch.cuda.Stream()
+        with torch.cuda.stream(s):
+            for i in range(args.warmup):
+                launch(i % n)
+            s.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(s)
+            for i in range(args.steps):
+                launch(i % n)
+            e1.record(s)
+        s.synchronize()
+        ms = e0.elapsed_time(e1)
+    else:
+        ms, _ = time_graph(torch, launch, n, args.steps, max(args.warmup, 1))
+    assert fa.device_error() == 0
+    per = ms / max(args.steps, 1)
+    print(json.dumps({"workload": c.name, "steps": args.steps, "ms_per_step": round(per, 5),
+                      "value": round(amount / (per * 1e-3), 2), "unit": unit, "l2_copies": n,
+                      "eager": bool(args.eager)}), flush=True)
+    return 0
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    if args.only:
+        return run_only(args)
+
+    import torch
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist_
+
+        torch.cuda.set_device(local)
+        dist_.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=torch.device("cuda", local))
+        dist = dist_
+    else:
+        torch.cuda.set_device(0)
+    from attention_attn_fwd_11_b200 import fa
+    from attention_attn_fwd_11_b200 import workloads as W_
+
+    fa.load()
+    peaks, peak_src = load_peaks()
+    l2 = torch.cuda.get_device_properties(torch.cuda.current_device()).L2_cache_size
+    K, Wm = args.steps, max(args.warmup, 3)
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    phys = int(vis.split(",")[local]) if vis and vis.split(",")[local].strip().isdigit() else local
+
+    # ---- headline: causal MHA prefill ----
+    c = W_.CAUSAL_MHA
+    launch, ncopy, foot, kpl = prefill_workload(torch, fa, W_, c, l2)
+    sampler = ClockSampler(phys)
+    sampler.start()
+    time.sleep(0.3)
+    win = []
+    ms, steps = time_graph(torch, launch, ncopy, K, Wm, dist, window=win)
+    clocks = sampler.stop(win[0], win[1])
+    clocks["window_s"] = round(win[1] - win[0], 3)
+    ms = max_over_ranks(torch, dist, ms)
+    total_flops = sum_over_ranks(torch, dist, c.flops * steps)
+    value = total_flops / (ms * 1e-3) / 1e12
+    per_launch_ms = ms / steps
+    achieved = c.flops / (per_launch_ms * 1e-3) / 1e12
+    assert fa.device_error() == 0, "device error during the timed region"
+
+    result = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": steps,
+        "warmup": Wm, "ms_per_step": round(per_launch_ms, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16)",
+        "config": {"workload": c.name, "B": c.B, "Hq": c.Hq, "Hkv": c.Hkv, "Sq": c.Sq, "Sk": c.Sk, "d": c.dk,
+                   "causal": c.causal, "out": "fp32 O + fp32 LSE",
+                   "l2": "%d rotating input copies (%.0f MB per step, L2 %.0f MB)" % (ncopy, foot / 1e6, l2 / 1e6),
+                   "timing": "CUDA graph replay, CUDA events on the launching stream",
+                   "parallelism": "replicas" if world > 1 else "single GPU"},
+        "roofline": roofline("tensor", achieved, peaks["bf16_tflops"], "TFLOP/s", NCU_TRAFFIC.get(c.name)),
+        "peak_source": peak_src + " (bf16_tflops burst; kernel timed alone)",
+        "gpu_launches": steps * kpl,
+        "clocks": clocks,
+    }
+
+    # ---- e2e through the public API with pinned host buffers ----
+    q0, k0, v0 = W_.prefill_inputs(c)
+    hq, hk, hv = q0.pin_memory(), k0.pin_memory(), v0.pin_memory()
+    dq, dk_, dv_ = torch.empty_like(q0, device="cuda"), torch.empty_like(k0, device="cuda"), torch.empty_like(v0, device="cuda")
+    do = torch.empty(c.B, c.Hq, c.Sq, c.dv, device="cuda")
+    ho = torch.empty(c.B, c.Hq, c.Sq, c.dv).pin_memory()
+    hl = torch.empty(c.B, c.Hq, c.Sq).pin_memory()
+    s = torch.cuda.Stream()
+    Ke = max(3, min(K, 30))
+
+    def e2e_step():
+        dq.copy_(hq, non_blocking=True)
+        dk_.copy_(hk, non_blocking=True)
+        dv_.copy_(hv, non_blocking=True)
+        o, lse = fa.fwd(dq, dk_, dv_, scale=c.scale, causal=c.causal, out=do)
+        ho.copy_(o, non_blocking=True)
+        hl.copy_(lse, non_blocking=True)
+
+    with torch.cuda.stream(s):
+        for _ in range(Wm):
+            e2e_step()
+    s.synchronize()
+    if dist is not None:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(s):
+        e0.record(s)
+        for _ in range(Ke):
+            e2e_step()
+        e1.record(s)
+    s.synchronize()
+    ems = max_over_ranks(torch, dist, e0.elapsed_time(e1))
+    e2e_val = sum_over_ranks(torch, dist, c.flops * Ke) / (ems * 1e-3) / 1e12
+    result["e2e"] = {"value": round(e2e_val, 3), "unit": "TFLOP/s",
+                     "h2d_bytes_per_step": int((q0.numel() + k0.numel() + v0.numel()) * 2),
+                     "d2h_bytes_per_step": int(c.B * c.Hq * c.Sq * (c.dv + 1) * 4), "steps": Ke}
+    result["gpu_launches"] += Ke  # the e2e steps launch the prefill kernel too
+    del hq, hk, hv, dq, dk_, dv_, do, ho, hl
+
+    # ---- the path's other workloads ----
+    if not args.no_secondary:
+        wl = {}
+        Ks = 200
+        for cc in (W_.TINY_FULL, W_.GQA_FULL):
+            launch, ncopy, foot, kpl = prefill_workload(torch, fa, W_, cc, l2)
+            ms2, st2 = time_graph(torch, launch, ncopy, Ks, Wm, dist)
+            ms2 = max_over_ranks(torch, dist, ms2)
+            per = ms2 / st2
+            ach = cc.flops / (per * 1e-3) / 1e12
+            wl[cc.name] = {"value": round(sum_over_ranks(torch, dist, cc.flops * st2) / (ms2 * 1e-3) / 1e12, 2),
+                           "unit": "TFLOP/s", "ms_per_step": round(per, 5), "steps": st2, "l2_copies": ncopy,
+                           "roofline": roofline("tensor", ach, peaks["bf16_tflops"], "TFLOP/s",
+                                                NCU_TRAFFIC.get(cc.name))}
+            result["gpu_launches"] += st2 * kpl
+            del launch
+        pc = W_.PAGED_GQA
+        launch, ncopy, byts, kpl = paged_workload(torch, fa, W_, pc, l2)
+        ms2, st2 = time_graph(torch, launch, ncopy, Ks, Wm, dist)
+        ms2 = max_over_ranks(torch, dist, ms2)
+        per = ms2 / st2
+        ach = byts / (per * 1e-3) / 1e9
+        wl[pc.name] = {"value": round(sum_over_ranks(torch, dist, byts * st2) / (ms2 * 1e-3) / 1e9, 1), "unit": "GB/s",
+                       "ms_per_step": round(per, 5), "steps": st2, "l2_copies": ncopy, "bytes_per_step": byts,
+                       "roofline": roofline("hbm", ach, peaks["hbm_gbs"], "GB/s", NCU_TRAFFIC.get(pc.name)),
+                       "kernels": "paged decode + LSE combine"}
+        result["gpu_launches"] += st2 * kpl
+        del launch
+        try:
+            lc = W_.LATENT_SPARSE
+            launch, ncopy, (byts, flops), kpl = latent_workload(torch, fa, W_, lc, l2)
+            ms2, st2 = time_graph(torch, launch, ncopy, Ks, Wm, dist)
+            ms2 = max_over_ranks(torch, dist, ms2)
+            per = ms2 / st2
+            ach = byts / (per * 1e-3) / 1e9
+            wl[lc.name] = {"value": round(sum_over_ranks(torch, dist, byts * st2) / (ms2 * 1e-3) / 1e9, 1),
+                           "unit": "GB/s", "tflops": round(flops / (per * 1e-3) / 1e12, 2),
+                           "ms_per_step": round(per, 5), "steps": st2, "l2_copies": ncopy, "bytes_per_step": byts,
+                           "roofline": roofline("hbm", ach, peaks["hbm_gbs"], "GB/s", NCU_TRAFFIC.get(lc.name)),
+                           "kernels": "latent gather decode + LSE combine"}
+            result["gpu_launches"] += st2 * kpl
+            del launch
+        except Exception as e:  # report, never hide
+            wl[W_.LATENT_SPARSE.name] = {"error": str(e)[:200]}
+        result["workloads"] = wl
+        assert fa.device_error() == 0, "device error in a secondary workload"
+
+    # ---- CPU baseline: the oracle on this host, rank 0 at N = 1 only ----
+    if world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline_prefill(c)
+
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())
