@@ -26,6 +26,8 @@
 #include <cuda_runtime.h>
 #include <math.h>
 
+#include <mutex>
+
 #include "internal.h"
 #include "sm100.cuh"
 
@@ -383,6 +385,46 @@ cudaError_t launch_decode_paged(const PagedLaunch &L, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     return launch_combine(L.part_o, L.part_lse, L.B * L.Hq, L.num_splits, L.Hq, L.seq_lens, L.blocks_per_split, L.o,
                           L.lse, L.o_bf16, PD_D, stream);
+}
+
+// ----------------------------------------------------------------------------
+// Fixed scratch for fa_decode_paged_noalloc: callers that cannot allocate
+// device memory get the split partials placed here instead of in a
+// caller-supplied workspace.  It is a file-scope device array, so every GPU
+// that loads the library holds these bytes until the process exits.  All
+// calls share it and it keeps whatever the previous call wrote; nothing in it
+// needs to start at zero (each call writes every partial its combine reads),
+// but two such calls running on the GPU at the same time race on it.
+constexpr size_t kPagedStaticScratchBytes = size_t(8) << 20;  // 8 MiB
+static __device__ __align__(256) unsigned char g_paged_scratch[kPagedStaticScratchBytes];
+
+size_t paged_static_scratch_bytes() { return kPagedStaticScratchBytes; }
+
+cudaError_t launch_decode_paged_static(PagedLaunch L, size_t lse_offset, cudaStream_t stream) {
+    // In host code g_paged_scratch names a host-side stand-in, not device
+    // memory: the device address is looked up once per device (with that
+    // device current) and cached.
+    constexpr int kMaxDevices = 64;
+    static std::mutex mu;
+    static void *dev_ptr[kMaxDevices] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    void *base = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        if (!dev_ptr[dev]) {
+            void *ptr = nullptr;
+            e = cudaGetSymbolAddress(&ptr, g_paged_scratch);
+            if (e != cudaSuccess) return e;
+            dev_ptr[dev] = ptr;
+        }
+        base = dev_ptr[dev];
+    }
+    L.part_o = static_cast<float *>(base);
+    L.part_lse = reinterpret_cast<float *>(static_cast<char *>(base) + lse_offset);
+    return launch_decode_paged(L, stream);
 }
 
 cudaError_t decode_device_error(int clear, int *code) {

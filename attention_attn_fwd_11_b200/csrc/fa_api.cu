@@ -301,6 +301,44 @@ fa_status fa_decode_paged(const fa_decode_paged_params *p, void *stream) {
     return FA_OK;
 }
 
+fa_status fa_decode_paged_noalloc(const fa_decode_paged_params *p, void *stream) {
+    fa_status st = check_paged_ptrs(p);
+    if (st != FA_OK) return st;
+    if (p->B == 0) return FA_OK;
+    const int splits = paged_splits(p);
+    const size_t need = paged_ws_bytes(p, splits);
+    const size_t have = fa::paged_static_scratch_bytes();
+    if (need > have)
+        return fail(FA_ERR_WORKSPACE,
+                    "fa_decode_paged_noalloc: these shapes need %zu bytes of scratch but the library's fixed scratch "
+                    "holds %zu; pass fewer num_splits or call fa_decode_paged with a workspace",
+                    need, have);
+    fa::PagedLaunch L;
+    L.q = p->q;
+    L.k_cache = p->k_cache;
+    L.v_cache = p->v_cache;
+    L.block_table = p->block_table;
+    L.seq_lens = p->seq_lens;
+    L.max_blocks_per_seq = p->max_blocks_per_seq;
+    L.B = p->B;
+    L.Hq = p->Hq;
+    L.Hkv = p->Hkv;
+    L.num_blocks = p->num_blocks;
+    L.scale = p->scale;
+    L.num_splits = splits;
+    L.blocks_per_split = (p->max_blocks_per_seq + splits - 1) / splits;
+    L.o = p->o;
+    L.lse = p->lse;
+    L.o_bf16 = p->o_dtype == FA_BF16;
+    L.part_o = nullptr;
+    L.part_lse = nullptr;
+    const size_t rows = (size_t)p->B * p->Hq * splits;
+    const size_t lse_offset = (rows * 128 * sizeof(float) + 255) & ~size_t(255);
+    cudaError_t e = fa::launch_decode_paged_static(L, lse_offset, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "fa_decode_paged_noalloc: launch");
+    return FA_OK;
+}
+
 fa_status fa_decode_gather_workspace_size(const fa_decode_gather_params *p, size_t *bytes) {
     fa_status st = check_gather(p);
     if (st != FA_OK) return st;

@@ -45,6 +45,11 @@ cudaError_t launch_combine(const float *part_o, const float *part_lse, int rows,
                            const int32_t *seq_lens, int bps, void *o, float *lse, int o_bf16, int D,
                            cudaStream_t stream);
 cudaError_t decode_device_error(int clear, int *code);
+// Allocation-free variant: the partials go to a fixed device array owned by
+// the library (its size is paged_static_scratch_bytes(); partial LSEs start
+// lse_offset bytes in).  L.part_o / L.part_lse are ignored.
+size_t paged_static_scratch_bytes();
+cudaError_t launch_decode_paged_static(PagedLaunch L, size_t lse_offset, cudaStream_t stream);
 
 // ---- latent gather decode ------------------------------------------------
 struct GatherLaunch {

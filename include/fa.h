@@ -141,6 +141,31 @@ fa_status fa_decode_paged_workspace_size(const fa_decode_paged_params *p, size_t
 fa_status fa_decode_paged(const fa_decode_paged_params *p, void *stream);
 
 /*
+ * fa_decode_paged_noalloc -- the same computation as fa_decode_paged, for
+ * callers that cannot allocate device memory: for example a plugin running
+ * inside a host application that owns every device allocation, or a serving
+ * loop whose memory was fully reserved up front and which may not call
+ * cudaMalloc (which can synchronise the device or fail under pressure) on
+ * its hot path.  The pages describe no such entry point; it has no
+ * counterpart there.
+ *   Arguments are those of fa_decode_paged; workspace and workspace_bytes
+ *   are ignored.  The split partials go to a fixed scratch array inside the
+ *   library (8 MiB of device memory, held on every GPU that loads the
+ *   library until the process exits).  Shapes whose partials need more
+ *   (fa_decode_paged_workspace_size() > 8 MiB) are rejected with
+ *   FA_ERR_WORKSPACE before any launch; pass a smaller num_splits or use
+ *   fa_decode_paged.
+ *   The first call on each device looks up the scratch array's device
+ *   address with that device current; make that first call before any
+ *   stream capture.  Every call shares the one array and it keeps the last
+ *   call's contents (nothing in it needs to start at zero): calls whose
+ *   work overlaps on the GPU -- concurrent streams, or several host threads
+ *   -- race on it and must be serialised by the caller.
+ *   Nothing here allocates or frees device memory.
+ */
+fa_status fa_decode_paged_noalloc(const fa_decode_paged_params *p, void *stream);
+
+/*
  * fa_decode_gather -- latent (MLA-style) sparse decode: every query head of
  * token t attends over the cache rows idx[t][0..topk) selected for it.
  *   q: [T, Hq, dk] bf16 contiguous, laid out like a cache row (the RoPE part
