@@ -243,7 +243,10 @@ latent_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const GatherArgs a
         const int head = qd * 32 + lane;
         const uint32_t tl = tmem + ((uint32_t)(qd * 32) << 16);
         const float c = a.scale_log2;
-        float m_run = -INFINITY, l_run = 0.f;
+        // l_run: sum of the fp32 weights (gives the LSE); l_mma: sum of the
+        // bf16-rounded weights the PV MMA uses (normalises O, so a one-hot
+        // softmax returns its V row exactly).
+        float m_run = -INFINITY, l_run = 0.f, l_mma = 0.f;
         bool ok = true;
         for (int i = 0; i < n_tiles; ++i) {
             const int buf = i & 1, s = i % LG_NST;
@@ -274,6 +277,7 @@ latent_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const GatherArgs a
             if (need) {
                 alpha = ex2(m_run - m_new);
                 l_run *= alpha;
+                l_mma *= alpha;
                 m_run = m_new;
             }
             if (i > 0 && __any_sync(0xffffffffu, need)) {
@@ -295,18 +299,19 @@ latent_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const GatherArgs a
             }
             const float msub = (m_run == -INFINITY) ? 0.f : m_run;
             uint32_t pk[16];
-            float s0 = 0.f, s1 = 0.f;
+            float s0 = 0.f, s1 = 0.f, r0 = 0.f, r1 = 0.f;
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
                 const float p0 = ex2(fmaf(x[2 * k], c, -msub));
                 const float p1 = ex2(fmaf(x[2 * k + 1], c, -msub));
                 pk[k] = pack_bf16x2(p0, p1);
-                // l sums the bf16-rounded weights the MMA actually uses, so O
-                // is an exactly normalised average of V rows.
-                s0 += __uint_as_float(pk[k] << 16);
-                s1 += __uint_as_float(pk[k] & 0xffff0000u);
+                s0 += p0;
+                s1 += p1;
+                r0 += __uint_as_float(pk[k] << 16);
+                r1 += __uint_as_float(pk[k] & 0xffff0000u);
             }
             l_run += s0 + s1;
+            l_mma += r0 + r1;
             tmem_st16(tl + (uint32_t)(buf * LG_BN), pk);
             tmem_wait_st();
             tc_fence_before();
@@ -320,7 +325,7 @@ latent_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const GatherArgs a
                 have_o = false;
         }
         const bool good = have_o && l_run > 0.f;
-        const float inv_l = good ? 1.f / l_run : 0.f;
+        const float inv_l = (good && l_mma > 0.f) ? 1.f / l_mma : 0.f;
         const int64_t prow = ((int64_t)t * LG_H + head) * a.num_splits + split;
         float4 *dst = reinterpret_cast<float4 *>(a.part_o + prow * LG_DV + half * LG_HALF);
 #pragma unroll 1

@@ -96,6 +96,25 @@ fa_status encode_2d(CUtensorMap *m, const void *base, int64_t cols, int64_t rows
 
 bool finite_pos(float x) { return isfinite(x) && x > 0.f; }
 
+// SM count of the current device, looked up once per device.
+cudaError_t num_sms(int *out) {
+    constexpr int kMaxDevices = 64;
+    static int cache[kMaxDevices] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < kMaxDevices && cache[dev] > 0) {
+        *out = cache[dev];
+        return cudaSuccess;
+    }
+    int n = 0;
+    e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < kMaxDevices) cache[dev] = n;
+    *out = n;
+    return cudaSuccess;
+}
+
 // ---------------------------------------------------------------- paged --
 
 int paged_splits(const fa_decode_paged_params *p) {
@@ -254,7 +273,14 @@ fa_status fa_fwd(const fa_fwd_params *p, void *stream) {
     L.o_ss = p->o_ss;
     L.o_bf16 = p->o_dtype == FA_BF16;
     L.lse = p->lse;
-    cudaError_t e = fa::launch_prefill(L, static_cast<cudaStream_t>(stream));
+    cudaError_t e;
+    if (p->dk <= 128) {
+        int sms = 0;
+        e = num_sms(&sms);
+        if (e == cudaSuccess) e = fa::launch_prefill2(L, sms, static_cast<cudaStream_t>(stream));
+    } else {
+        e = fa::launch_prefill(L, static_cast<cudaStream_t>(stream));
+    }
     if (e != cudaSuccess) return cuda_fail(e, "fa_fwd: launch");
     return FA_OK;
 }
@@ -386,12 +412,13 @@ fa_status fa_decode_gather(const fa_decode_gather_params *p, void *stream) {
 
 fa_status fa_device_error(int clear, int *code) {
     if (!code) return fail(FA_ERR_INVALID_ARG, "fa_device_error: code is NULL");
-    int c1 = 0, c2 = 0, c3 = 0;
+    int c1 = 0, c2 = 0, c3 = 0, c4 = 0;
     cudaError_t e = fa::prefill_device_error(clear, &c1);
+    if (e == cudaSuccess) e = fa::prefill2_device_error(clear, &c4);
     if (e == cudaSuccess) e = fa::decode_device_error(clear, &c2);
     if (e == cudaSuccess) e = fa::gather_device_error(clear, &c3);
     if (e != cudaSuccess) return cuda_fail(e, "fa_device_error");
-    *code = c1 ? c1 : (c2 ? c2 : c3);
+    *code = c1 ? c1 : (c4 ? c4 : (c2 ? c2 : c3));
     return FA_OK;
 }
 

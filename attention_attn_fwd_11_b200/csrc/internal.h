@@ -23,6 +23,9 @@ struct PrefillLaunch {
 cudaError_t launch_prefill(const PrefillLaunch &L, cudaStream_t stream);
 // Reads (and optionally clears) the prefill kernels' device error word.
 cudaError_t prefill_device_error(int clear, int *code);
+// Persistent two-tile prefill (head dims 64 and 128); grid = min(units, num_sms).
+cudaError_t launch_prefill2(const PrefillLaunch &L, int num_sms, cudaStream_t stream);
+cudaError_t prefill2_device_error(int clear, int *code);
 
 // ---- paged decode --------------------------------------------------------
 struct PagedLaunch {

@@ -1,0 +1,514 @@
+// prefill2.cu -- persistent two-tile prefill for head dims 64 and 128
+// (sm_100a).
+//
+// A work unit is 256 query rows = two 128-row tiles of one (batch, query
+// head); both tiles stream the SAME K/V tiles, so every K/V byte staged in
+// shared memory feeds twice the tensor-core work of the one-tile kernel.
+//
+//   warp 0       TMA producer: Q (both tiles) per unit, then the K and V ring.
+//   warp 1       MMA issuer.  Per KV tile t:  PV0(t), QK0(t+1), PV1(t),
+//                QK1(t+1).  While softmax warpgroup A works on S0(t+1), the
+//                tensor core runs PV1(t) and QK1(t+1), and vice versa: the
+//                two softmax warpgroups ping-pong around the tensor core.
+//   warps 4-7    softmax warpgroup A (tile 0), warps 8-11 warpgroup B
+//                (tile 1): one thread per query row, online softmax in base 2
+//                with lazy per-row rescale, P (bf16) written into the S
+//                buffer in TMEM, epilogue O / l and LSE.
+//   TMEM         S0 | S1 | O0 | O1   (128 + 128 + d + d columns).
+//
+// The grid is persistent (one CTA per SM).  Units are ordered longest
+// first (causal: the last query rows see the most keys) and dealt to the
+// CTAs in a serpentine order, so every SM ends up with a similar amount of
+// work.  The epilogue of one unit overlaps the first QK^T of the next; an
+// o_free / unit_start handshake keeps the next unit's first P V from
+// overwriting an O accumulator that is still being read out.
+//
+// The pages this follows are the same as for the one-tile kernel
+// (prefill.cu): the UMMA FMHA notes (raw QK^T, K-steps of 16, TMEM 32x32b
+// reads one row per lane, P in TMEM for a TMEM-operand MMA) and llama.cpp's
+// Metal tensor kernel (online softmax with any max >= the true one, skipped
+// rescales, QK^T of the next chunk issued before PV of the current one).
+#include <cuda_runtime.h>
+#include <math.h>
+
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace fa {
+
+static __device__ int g_prefill2_err;
+
+struct Prefill2Args {
+    int Hq, group, Sq, Sk, BH, n_qp, n_units;
+    float scale_log2;
+    int causal;
+    char *o;
+    int64_t o_sb, o_sh, o_ss;
+    int o_bf16;
+    float *lse;
+};
+
+template <int D>
+struct P2Cfg {
+    static constexpr int BM = 128;
+    static constexpr int BN = 128;
+    static constexpr int NST = D == 128 ? 2 : 4;
+    static constexpr int NCH = D / 64;
+    static constexpr int Q_CHUNK = BM * 128;
+    static constexpr int KV_CHUNK = BN * 128;
+    static constexpr int Q_TILE = BM * D * 2;
+    static constexpr int KV_BYTES = BN * D * 2;
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_K = 2 * Q_TILE;
+    static constexpr int OFF_V = OFF_K + NST * KV_BYTES;
+    static constexpr int OFF_BAR = OFF_V + NST * KV_BYTES;
+    static constexpr int SMEM_BYTES = OFF_BAR + 512 + 1024;
+    static constexpr int T_O = 2 * BN;  // O0 at T_O, O1 at T_O + D
+    static_assert(2 * BN + 2 * D <= 512, "TMEM budget");
+    static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+enum {
+    P2_QFULL = 0, P2_QEMPTY = 1, P2_SFULL = 2, P2_PREADY = 4, P2_ODONE = 6, P2_OFREE = 8, P2_USTART = 10,
+    P2_DRAIN = 12, P2_RING = 13
+};
+
+constexpr float kP2RescaleThreshold = 8.0f;
+
+struct UnitInfo {
+    int b, hq, q0, n[2], N;
+};
+
+FA_DEV bool p2_unit(const Prefill2Args &a, int round, UnitInfo &u) {
+    const int G = gridDim.x, c = blockIdx.x;
+    const int idx = round * G + ((round & 1) ? (G - 1 - c) : c);
+    if (idx >= a.n_units) return false;
+    const int qp = a.causal ? (a.n_qp - 1 - idx / a.BH) : (idx / a.BH);
+    const int bh = idx % a.BH;
+    u.b = bh / a.Hq;
+    u.hq = bh % a.Hq;
+    u.q0 = qp * 256;
+    u.N = 0;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const int r0 = u.q0 + 128 * i;
+        int n = 0;
+        if (r0 < a.Sq) {
+            const int last = min(r0 + 127, a.Sq - 1);
+            int kmax = a.Sk - 1;
+            if (a.causal) kmax = min(kmax, last + a.Sk - a.Sq);
+            n = kmax < 0 ? 0 : kmax / 128 + 1;
+        }
+        u.n[i] = n;
+        u.N = max(u.N, n);
+    }
+    return true;
+}
+
+template <int D>
+__global__ void __launch_bounds__(384, 1)
+prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                const __grid_constant__ CUtensorMap tmV, const Prefill2Args a) {
+    using C = P2Cfg<D>;
+    constexpr int BN = C::BN, NST = C::NST;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t sQ = sbase + C::OFF_Q, sK = sbase + C::OFF_K, sV = sbase + C::OFF_V;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
+    const uint32_t bar0 = smem_u32(bars);
+    auto bar = [&](int i) -> uint32_t { return bar0 + 8u * (uint32_t)i; };
+    auto k_full = [&](int s) { return bar(P2_RING + s); };
+    auto k_empty = [&](int s) { return bar(P2_RING + NST + s); };
+    auto v_full = [&](int s) { return bar(P2_RING + 2 * NST + s); };
+    auto v_empty = [&](int s) { return bar(P2_RING + 3 * NST + s); };
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + 40);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar(P2_QFULL), 1);
+        mbar_init(bar(P2_QEMPTY), 1);
+        mbar_init(bar(P2_DRAIN), 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(bar(P2_SFULL + i), 1);
+            mbar_init(bar(P2_PREADY + i), 128);
+            mbar_init(bar(P2_ODONE + i), 1);
+            mbar_init(bar(P2_OFREE + i), 128);
+            mbar_init(bar(P2_USTART + i), 1);
+        }
+        for (int s = 0; s < NST; ++s) {
+            mbar_init(k_full(s), 1);
+            mbar_init(k_empty(s), 1);
+            mbar_init(v_full(s), 1);
+            mbar_init(v_empty(s), 1);
+        }
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_holder), 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer --
+        if (lane == 0) {
+            prefetch_tmap(&tmQ);
+            prefetch_tmap(&tmK);
+            prefetch_tmap(&tmV);
+            int kc = 0, uc = 0, issued = 0;
+            bool ok = true;
+            UnitInfo u;
+            for (int r = 0; ok && p2_unit(a, r, u); ++r, ++uc) {
+                const int hkv = u.hq / a.group;
+                if (!mbar_wait(bar(P2_QEMPTY), ((uint32_t)uc & 1u) ^ 1u, abort_flag, &g_prefill2_err)) break;
+                mbar_arrive_expect_tx(bar(P2_QFULL), 2 * C::Q_TILE);
+#pragma unroll
+                for (int i = 0; i < 2; ++i)
+#pragma unroll
+                    for (int c = 0; c < C::NCH; ++c)
+                        tma_load_4d(sQ + i * C::Q_TILE + c * C::Q_CHUNK, &tmQ, bar(P2_QFULL), c * 64, u.q0 + 128 * i,
+                                    u.hq, u.b);
+                for (int t = 0; t < u.N; ++t, ++kc) {
+                    const int s = kc % NST;
+                    const uint32_t ph = (uint32_t)(kc / NST) & 1u;
+                    if (!mbar_wait(k_empty(s), ph ^ 1u, abort_flag, &g_prefill2_err)) { ok = false; break; }
+                    mbar_arrive_expect_tx(k_full(s), C::KV_BYTES);
+#pragma unroll
+                    for (int c = 0; c < C::NCH; ++c)
+                        tma_load_4d(sK + s * C::KV_BYTES + c * C::KV_CHUNK, &tmK, k_full(s), c * 64, t * BN, hkv, u.b);
+                    if (!mbar_wait(v_empty(s), ph ^ 1u, abort_flag, &g_prefill2_err)) { ok = false; break; }
+                    mbar_arrive_expect_tx(v_full(s), C::KV_BYTES);
+#pragma unroll
+                    for (int c = 0; c < C::NCH; ++c)
+                        tma_load_4d(sV + s * C::KV_BYTES + c * C::KV_CHUNK, &tmV, v_full(s), c * 64, t * BN, hkv, u.b);
+                    issued = kc + 1;
+                }
+            }
+            if (*abort_flag) {
+                // Let the copies still in flight land before the CTA exits.
+                mbar_wait_drain(bar(P2_QFULL), (uint32_t)(max(uc - 1, 0)) & 1u);
+                for (int k = max(0, issued - NST); k < issued; ++k) {
+                    mbar_wait_drain(k_full(k % NST), (uint32_t)(k / NST) & 1u);
+                    mbar_wait_drain(v_full(k % NST), (uint32_t)(k / NST) & 1u);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------- MMA issuer --
+        if (lane == 0) {
+            constexpr uint32_t idesc_qk = idesc_bf16_f32(128, BN, false, false);
+            constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, false, true);
+            auto qk = [&](int i, int s) {
+                const uint32_t tS = tmem + (uint32_t)(i * BN);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const int c = kk >> 2, sub = kk & 3;
+                    const uint64_t ad = sdesc_sw128(sQ + i * C::Q_TILE + c * C::Q_CHUNK + sub * 32, 16, 1024);
+                    const uint64_t bd = sdesc_sw128(sK + s * C::KV_BYTES + c * C::KV_CHUNK + sub * 32, 16, 1024);
+                    mma_ss(tS, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(bar(P2_SFULL + i));
+            };
+            auto pv = [&](int i, int s, bool first) {
+                const uint32_t tO = tmem + (uint32_t)(C::T_O + i * D);
+                const uint32_t tP = tmem + (uint32_t)(i * BN);
+#pragma unroll
+                for (int kk = 0; kk < BN / 16; ++kk) {
+                    const uint64_t bd = sdesc_sw128(sV + s * C::KV_BYTES + kk * 2048, C::KV_CHUNK, 1024);
+                    mma_ts(tO, tP + kk * 8, bd, idesc_pv, (!first || kk > 0) ? 1u : 0u);
+                }
+                mma_commit(bar(P2_ODONE + i));
+            };
+            int kc = 0, uc = 0;
+            int pcnt[2] = {0, 0};
+            bool ok = true;
+            UnitInfo u;
+            for (int r = 0; ok && p2_unit(a, r, u); ++r, ++uc) {
+                // The previous unit's O accumulators must have been read out.
+                for (int i = 0; i < 2; ++i) {
+                    if (uc > 0 &&
+                        !mbar_wait(bar(P2_OFREE + i), (uint32_t)(uc - 1) & 1u, abort_flag, &g_prefill2_err)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive(bar(P2_USTART + i));
+                }
+                if (!ok || !mbar_wait(bar(P2_QFULL), (uint32_t)uc & 1u, abort_flag, &g_prefill2_err)) break;
+                tc_fence_after();
+                if (u.N == 0) {
+                    mma_commit(bar(P2_QEMPTY));
+                    continue;
+                }
+                {
+                    const int s0 = kc % NST;
+                    if (!mbar_wait(k_full(s0), (uint32_t)(kc / NST) & 1u, abort_flag, &g_prefill2_err)) break;
+                    tc_fence_after();
+                    if (u.n[0] > 0) qk(0, s0);
+                    if (u.n[1] > 0) qk(1, s0);
+                    mma_commit(k_empty(s0));
+                    if (u.N == 1) mma_commit(bar(P2_QEMPTY));
+                }
+                for (int t = 0; t < u.N; ++t) {
+                    const int kt = kc + t;
+                    const int s = kt % NST;
+                    const bool has_next = t + 1 < u.N;
+                    const int s1 = (kt + 1) % NST;
+                    bool v_ready = false;
+                    if (t < u.n[0]) {
+                        if (!mbar_wait(bar(P2_PREADY + 0), (uint32_t)pcnt[0] & 1u, abort_flag, &g_prefill2_err) ||
+                            !mbar_wait(v_full(s), (uint32_t)(kt / NST) & 1u, abort_flag, &g_prefill2_err)) {
+                            ok = false;
+                            break;
+                        }
+                        ++pcnt[0];
+                        v_ready = true;
+                        tc_fence_after();
+                        pv(0, s, t == 0);
+                    }
+                    if (has_next) {
+                        if (!mbar_wait(k_full(s1), (uint32_t)((kt + 1) / NST) & 1u, abort_flag, &g_prefill2_err)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        if (t + 1 < u.n[0]) qk(0, s1);
+                    }
+                    if (t < u.n[1]) {
+                        if (!mbar_wait(bar(P2_PREADY + 1), (uint32_t)pcnt[1] & 1u, abort_flag, &g_prefill2_err) ||
+                            (!v_ready &&
+                             !mbar_wait(v_full(s), (uint32_t)(kt / NST) & 1u, abort_flag, &g_prefill2_err))) {
+                            ok = false;
+                            break;
+                        }
+                        ++pcnt[1];
+                        tc_fence_after();
+                        pv(1, s, t == 0);
+                    }
+                    if (has_next && t + 1 < u.n[1]) qk(1, s1);
+                    mma_commit(v_empty(s));
+                    if (has_next) {
+                        mma_commit(k_empty(s1));
+                        if (t + 2 == u.N) mma_commit(bar(P2_QEMPTY));  // the unit's last QK^T is issued
+                    }
+                }
+                kc += u.N;
+            }
+            mma_commit(bar(P2_DRAIN));
+            mbar_wait_drain(bar(P2_DRAIN), 0);
+        }
+        __syncwarp();
+    } else if (warp >= 4) {
+        // ------------------------------- softmax / correction / epilogue --
+        const int ti = (warp - 4) >> 2;              // which query tile of the unit
+        const int qd = warp & 3;                     // TMEM lane quadrant
+        const int row = qd * 32 + lane;
+        const uint32_t tl = tmem + ((uint32_t)(qd * 32) << 16);
+        const uint32_t tS = tl + (uint32_t)(ti * BN);
+        const uint32_t tO = tl + (uint32_t)(C::T_O + ti * D);
+        const float c = a.scale_log2;
+        int scnt = 0, pv_base = 0, uc = 0;
+        bool ok = true;
+        UnitInfo u;
+        for (int r = 0; ok && p2_unit(a, r, u); ++r, ++uc) {
+            if (!mbar_wait(bar(P2_USTART + ti), (uint32_t)uc & 1u, abort_flag, &g_prefill2_err)) break;
+            const int n = u.n[ti];
+            const int qrow = u.q0 + 128 * ti + row;
+            const int lim_all = a.causal ? min(a.Sk, qrow + a.Sk - a.Sq + 1) : a.Sk;
+            float m_run = -INFINITY, l_run = 0.f;
+            for (int t = 0; t < n; ++t) {
+                if (!mbar_wait(bar(P2_SFULL + ti), (uint32_t)scnt & 1u, abort_flag, &g_prefill2_err)) {
+                    ok = false;
+                    break;
+                }
+                ++scnt;
+                tc_fence_after();
+                float x[BN];
+                {
+                    uint32_t rr[BN];
+#pragma unroll
+                    for (int ch = 0; ch < BN / 32; ++ch)
+                        tmem_ld32(tS + (uint32_t)(ch * 32), *reinterpret_cast<uint32_t(*)[32]>(&rr[ch * 32]));
+                    tmem_wait_ld();
+                    reg_fence(rr);
+#pragma unroll
+                    for (int k = 0; k < BN; ++k) x[k] = __uint_as_float(rr[k]);
+                }
+                const int lim = lim_all - t * BN;
+                if (lim < BN) {
+#pragma unroll
+                    for (int k = 0; k < BN; ++k)
+                        if (k >= lim) x[k] = -INFINITY;
+                }
+                float mx0 = x[0], mx1 = x[1], mx2 = x[2], mx3 = x[3];
+#pragma unroll
+                for (int k = 4; k < BN; k += 4) {
+                    mx0 = fmaxf(mx0, x[k]);
+                    mx1 = fmaxf(mx1, x[k + 1]);
+                    mx2 = fmaxf(mx2, x[k + 2]);
+                    mx3 = fmaxf(mx3, x[k + 3]);
+                }
+                const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * c;
+                const float m_new = fmaxf(m_run, m_tile);
+                const bool need = m_new > m_run + kP2RescaleThreshold;
+                float alpha = 1.f;
+                if (need) {
+                    alpha = ex2(m_run - m_new);
+                    l_run *= alpha;
+                    m_run = m_new;
+                }
+                if (t > 0 && __any_sync(0xffffffffu, need)) {
+                    if (!mbar_wait(bar(P2_ODONE + ti), (uint32_t)(pv_base + t - 1) & 1u, abort_flag,
+                                   &g_prefill2_err)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+#pragma unroll 1
+                    for (int ch = 0; ch < D / 32; ++ch) {
+                        uint32_t o[32];
+                        tmem_ld32(tO + (uint32_t)(ch * 32), o);
+                        tmem_wait_ld();
+                        reg_fence(o);
+#pragma unroll
+                        for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+                        tmem_st32(tO + (uint32_t)(ch * 32), o);
+                    }
+                }
+                const float msub = (m_run == -INFINITY) ? 0.f : m_run;
+                float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+                for (int g = 0; g < BN / 32; ++g) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) {
+                        const float p0 = ex2(fmaf(x[g * 32 + 2 * k], c, -msub));
+                        const float p1 = ex2(fmaf(x[g * 32 + 2 * k + 1], c, -msub));
+                        s0 += p0;
+                        s1 += p1;
+                        pk[k] = pack_bf16x2(p0, p1);
+                    }
+                    tmem_st16(tS + (uint32_t)(g * 16), pk);
+                }
+                l_run += s0 + s1;
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(bar(P2_PREADY + ti));
+            }
+            // ---- epilogue ----
+            bool have_o = ok && n > 0;
+            if (have_o) {
+                if (mbar_wait(bar(P2_ODONE + ti), (uint32_t)(pv_base + n - 1) & 1u, abort_flag, &g_prefill2_err))
+                    tc_fence_after();
+                else
+                    have_o = false;
+            }
+            pv_base += n;
+            const bool store = qrow < a.Sq;
+            const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+            const int64_t ooff = (int64_t)u.b * a.o_sb + (int64_t)u.hq * a.o_sh + (int64_t)qrow * a.o_ss;
+#pragma unroll 1
+            for (int ch = 0; ch < D / 32; ++ch) {
+                uint32_t o[32];
+                if (have_o) {
+                    tmem_ld32(tO + (uint32_t)(ch * 32), o);
+                    tmem_wait_ld();
+                    reg_fence(o);
+                } else {
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) o[k] = 0u;
+                }
+                if (store) {
+                    if (a.o_bf16) {
+                        uint4 *dst = reinterpret_cast<uint4 *>(a.o + 2 * (ooff + ch * 32));
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            uint4 w;
+                            w.x = pack_bf16x2(__uint_as_float(o[8 * k + 0]) * inv_l, __uint_as_float(o[8 * k + 1]) * inv_l);
+                            w.y = pack_bf16x2(__uint_as_float(o[8 * k + 2]) * inv_l, __uint_as_float(o[8 * k + 3]) * inv_l);
+                            w.z = pack_bf16x2(__uint_as_float(o[8 * k + 4]) * inv_l, __uint_as_float(o[8 * k + 5]) * inv_l);
+                            w.w = pack_bf16x2(__uint_as_float(o[8 * k + 6]) * inv_l, __uint_as_float(o[8 * k + 7]) * inv_l);
+                            dst[k] = w;
+                        }
+                    } else {
+                        float4 *dst = reinterpret_cast<float4 *>(a.o + 4 * (ooff + ch * 32));
+#pragma unroll
+                        for (int k = 0; k < 8; ++k)
+                            dst[k] = make_float4(__uint_as_float(o[4 * k]) * inv_l, __uint_as_float(o[4 * k + 1]) * inv_l,
+                                                 __uint_as_float(o[4 * k + 2]) * inv_l,
+                                                 __uint_as_float(o[4 * k + 3]) * inv_l);
+                    }
+                }
+            }
+            if (store && a.lse)
+                a.lse[((int64_t)u.b * a.Hq + u.hq) * a.Sq + qrow] =
+                    (l_run > 0.f) ? (m_run + __log2f(l_run)) * 0.69314718055994530942f : -INFINITY;
+            // O of this tile has been read out: the next unit may overwrite it.
+            tc_fence_before();
+            mbar_arrive(bar(P2_OFREE + ti));
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+template <int D>
+static cudaError_t launch_p2(const PrefillLaunch &L, int num_sms, cudaStream_t stream) {
+    using C = P2Cfg<D>;
+    auto kern = prefill2_kernel<D>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    Prefill2Args a;
+    a.Hq = L.Hq;
+    a.group = L.Hq / L.Hkv;
+    a.Sq = L.Sq;
+    a.Sk = L.Sk;
+    a.BH = L.B * L.Hq;
+    a.n_qp = (L.Sq + 255) / 256;
+    a.n_units = a.BH * a.n_qp;
+    a.scale_log2 = L.scale * 1.4426950408889634f;
+    a.causal = L.causal;
+    a.o = static_cast<char *>(L.o);
+    a.o_sb = L.o_sb;
+    a.o_sh = L.o_sh;
+    a.o_ss = L.o_ss;
+    a.o_bf16 = L.o_bf16;
+    a.lse = L.lse;
+    const int grid = a.n_units < num_sms ? a.n_units : num_sms;
+    kern<<<grid, 384, C::SMEM_BYTES, stream>>>(L.tmQ, L.tmK, L.tmV, a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_prefill2(const PrefillLaunch &L, int num_sms, cudaStream_t stream) {
+    switch (L.dk) {
+        case 64: return launch_p2<64>(L, num_sms, stream);
+        case 128: return launch_p2<128>(L, num_sms, stream);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t prefill2_device_error(int clear, int *code) {
+    int v = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(&v, g_prefill2_err, sizeof(int));
+    if (e != cudaSuccess) return e;
+    *code = v;
+    if (clear && v) {
+        v = 0;
+        e = cudaMemcpyToSymbol(g_prefill2_err, &v, sizeof(int));
+    }
+    return e;
+}
+
+}  // namespace fa

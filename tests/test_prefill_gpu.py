@@ -156,3 +156,11 @@ def test_causal_mha_config_sampled():
 def test_gqa_config_sampled():
     """B=1, Hq=32, Hkv=8, S=4096, d=256, full -- the benchmark launch, sampled rows."""
     check_sampled(W.GQA_FULL, n_rows=12)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+def test_many_units_per_cta(d, causal):
+    """More (batch, head, 256-row) units than SMs, several rounds per CTA of
+    the persistent kernel, odd GQA ratio, ragged last unit."""
+    run_and_check(2, 80, 16, 600, 600, d, causal, seed=90 + d + causal)
