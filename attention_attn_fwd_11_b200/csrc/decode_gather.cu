@@ -10,21 +10,25 @@
 // <= the token's position.  As on that page, rows are gathered straight
 // from the cache in its native row-major layout (no pre-gathered copy).
 //
-// Design (one CTA = one token x one key split x one half of dv):
-//   - the 128 heads are the MMA's M = 128 rows: S = Q K^T (K = 576) and
-//     O += P V run as tcgen05.mma with fp32 accumulators in TMEM;
-//   - O for 128 heads x 512 dims in fp32 would fill all 512 TMEM columns,
-//     leaving none for S, so the two halves of dv go to two CTAs launched
-//     side by side (each recomputes S = Q K^T; the second CTA's row reads
-//     mostly hit L2);
+// Design: a cluster of two CTAs handles one (token, key split).
+//   - The 128 heads are the MMA's M = 128 rows.  O for 128 heads x 512 dims
+//     in fp32 would fill all 512 TMEM columns, so CTA r keeps the O half
+//     for latent dims [256 r, 256 r + 256).
+//   - The 576-wide score contraction is split between the two CTAs along
+//     the columns of a row: CTA 0 owns row columns [0, 320) (the RoPE part
+//     and latent [0, 256)), CTA 1 owns [320, 576).  Each CTA gathers ONLY
+//     its columns of every selected row -- exactly the columns its PV needs
+//     as well -- so each row is read from memory once per cluster and no
+//     score is computed twice.  Each CTA holds the matching part of Q.
+//   - Partial scores (128 heads x 32 keys, fp32) are swapped through
+//     distributed shared memory every tile; both CTAs add own + peer (the
+//     same sum in either order), so both run the identical online softmax.
 //   - warps 0-3 gather 32 selected rows per tile with 16-byte cp.async into
-//     128-byte-swizzled shared memory; the same tile is the K-major B
-//     operand of QK^T and (its latent columns) the MN-major B operand of PV,
-//     so every row is read once per CTA;
-//   - Q (128 x 576, 144 KB) is loaded once by TMA;
-//   - warp 8 issues the MMAs; warps 4-7 run the online softmax (one head per
-//     thread; the visibility mask comes with the tile) and the epilogue,
-//     writing a split partial that the log-sum-exp combine merges.
+//     128-byte-swizzled shared memory (4-tile ring); the tile is the K-major
+//     B operand of the partial QK^T and, through its latent columns, the
+//     MN-major B operand of PV; warp 8 issues the MMAs; warps 4-7 run the
+//     exchange, the softmax (one head per thread) and the epilogue, which
+//     writes a split partial for the log-sum-exp combine.
 #include <cuda_runtime.h>
 #include <limits.h>
 #include <math.h>
@@ -40,22 +44,24 @@ constexpr int LG_DK = 576;
 constexpr int LG_DV = 512;
 constexpr int LG_HALF = 256;
 constexpr int LG_H = 128;
-constexpr int LG_BN = 32;                       // keys per tile
-constexpr int LG_NST = 2;                       // tile ring depth
-constexpr int LG_NCH = LG_DK / 64;              // 9 chunks of 128 bytes per row
-constexpr int LG_QCH = LG_H * 128;              // bytes of one Q chunk (16 KB)
-constexpr int LG_KCH = LG_BN * 128;             // bytes of one K chunk (4 KB)
-constexpr int LG_Q_BYTES = LG_NCH * LG_QCH;     // 144 KB
-constexpr int LG_K_BYTES = LG_NCH * LG_KCH;     // 36 KB
-constexpr int LG_OFF_K = LG_Q_BYTES;
-constexpr int LG_OFF_AUX = LG_OFF_K + LG_NST * LG_K_BYTES;
-constexpr int LG_SMEM = LG_OFF_AUX + 512 + 1024;
-constexpr int LG_PIECES = LG_BN * (LG_DK / 8);  // 16-byte pieces per tile (2304)
-constexpr int LG_T_O = 2 * LG_BN;               // TMEM column of O (S0 at 0, S1 at 32)
+constexpr int LG_BN = 32;                        // keys per tile
+constexpr int LG_NST = 4;                        // gather ring depth
+constexpr int LG_NCH_MAX = 5;                    // 128-byte column chunks per CTA (5 or 4)
+constexpr int LG_QCH = LG_H * 128;               // bytes of one Q chunk (16 KB)
+constexpr int LG_KCH = LG_BN * 128;              // bytes of one K chunk (4 KB)
+constexpr int LG_KSTAGE = LG_NCH_MAX * LG_KCH;   // 20 KB
+constexpr int LG_XBUF = LG_H * LG_BN * 4;        // one partial-score exchange slot (16 KB)
+constexpr int LG_OFF_K = LG_NCH_MAX * LG_QCH;    // Q: 80 KB
+constexpr int LG_OFF_X = LG_OFF_K + LG_NST * LG_KSTAGE;
+constexpr int LG_OFF_AUX = LG_OFF_X + 2 * LG_XBUF;
+constexpr int LG_SMEM = LG_OFF_AUX + 1024 + 1024;
+constexpr int LG_T_O = 2 * LG_BN;                // TMEM column of O (S0 at 0, S1 at 32)
 static_assert(LG_SMEM <= 232448, "shared memory budget");
-static_assert(LG_PIECES % 128 == 0, "pieces per producer thread");
 
-enum { G_QFULL = 0, G_SFULL = 1, G_PREADY = 3, G_PVDONE = 5, G_DRAIN = 6, G_FULL = 7, G_EMPTY = 9, G_NBAR = 11 };
+enum {
+    G_QFULL = 0, G_SFULL = 1, G_PREADY = 3, G_PVDONE = 5, G_DRAIN = 6, G_XFULL = 7, G_XFREE = 9, G_FULL = 11,
+    G_EMPTY = 11 + LG_NST, G_NBAR = 11 + 2 * LG_NST
+};
 
 struct GatherArgs {
     const __nv_bfloat16 *rows;
@@ -68,34 +74,42 @@ struct GatherArgs {
 
 constexpr float kGatherRescaleThreshold = 8.0f;
 
-__global__ void __launch_bounds__(288, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(288, 1)
 latent_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const GatherArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
-    const uint32_t sQ = sbase, sK = sbase + LG_OFF_K;
+    const uint32_t sQ = sbase, sK = sbase + LG_OFF_K, sX = sbase + LG_OFF_X;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + LG_OFF_AUX);
     const uint32_t bar0 = smem_u32(bars);
     auto bar = [&](int i) -> uint32_t { return bar0 + 8u * (uint32_t)i; };
-    int32_t *rowid = reinterpret_cast<int32_t *>(smem + LG_OFF_AUX + 8 * 16);  // [NST][32]
-    uint32_t *maskw = reinterpret_cast<uint32_t *>(rowid + LG_NST * LG_BN);    // [NST]
+    int32_t *rowid = reinterpret_cast<int32_t *>(smem + LG_OFF_AUX + 8 * 32);   // [NST][32]
+    uint32_t *maskw = reinterpret_cast<uint32_t *>(rowid + LG_NST * LG_BN);     // [NST]
     uint32_t *tmem_holder = maskw + LG_NST;
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
+    volatile int *go = reinterpret_cast<volatile int *>(tmem_holder + 2);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int half = blockIdx.x, split = blockIdx.y, t = blockIdx.z;
+    const uint32_t rank = cluster_ctarank();  // 0 or 1 (blockIdx.x)
+    const uint32_t peer = rank ^ 1u;
+    const int split = blockIdx.y, t = blockIdx.z;
+    const int chunk0 = rank == 0 ? 0 : 5;     // first 128-byte column chunk of a row this CTA owns
+    const int nch = rank == 0 ? 5 : 4;        // chunks it owns
+    const int vch = rank == 0 ? 1 : 0;        // its first latent (V) chunk, in local chunk numbers
     const int k_begin = split * a.kps;
     const int k_end = min(a.topk, k_begin + a.kps);
     const int n_tiles = k_end > k_begin ? (k_end - k_begin + LG_BN - 1) / LG_BN : 0;
 
     if (threadIdx.x == 0) {
         mbar_init(bar(G_QFULL), 1);
-        mbar_init(bar(G_SFULL), 1);
-        mbar_init(bar(G_SFULL + 1), 1);
-        mbar_init(bar(G_PREADY), 128);
-        mbar_init(bar(G_PREADY + 1), 128);
         mbar_init(bar(G_PVDONE), 1);
         mbar_init(bar(G_DRAIN), 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(bar(G_SFULL + i), 1);
+            mbar_init(bar(G_PREADY + i), 128);
+            mbar_init(bar(G_XFULL + i), 128);  // the peer's 128 softmax threads
+            mbar_init(bar(G_XFREE + i), 128);
+        }
         for (int s = 0; s < LG_NST; ++s) {
             mbar_init(bar(G_FULL + s), 128);
             mbar_init(bar(G_EMPTY + s), 1);
@@ -110,6 +124,8 @@ latent_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const GatherArgs a
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    // The peer's barriers must exist before anyone arrives on them remotely.
+    cluster_sync();
     const uint32_t tmem = *tmem_holder;
 
     if (warp < 4) {
@@ -118,19 +134,25 @@ latent_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const GatherArgs a
         if (n_tiles > 0) {
             if (tid == 0) {
                 prefetch_tmap(&tmQ);
-                mbar_arrive_expect_tx(bar(G_QFULL), LG_Q_BYTES);
-#pragma unroll 1
-                for (int c = 0; c < LG_NCH; ++c) tma_load_2d(sQ + c * LG_QCH, &tmQ, bar(G_QFULL), c * 64, t * LG_H);
+                mbar_arrive_expect_tx(bar(G_QFULL), nch * LG_QCH);
+                for (int c = 0; c < nch; ++c)
+                    tma_load_2d(sQ + c * LG_QCH, &tmQ, bar(G_QFULL), (chunk0 + c) * 64, t * LG_H);
             }
             const int qpos = a.q_pos ? a.q_pos[t] : INT_MAX;
             const int32_t *idx_t = a.idx + (int64_t)t * a.topk;
             const int32_t *kp_t = a.key_pos ? a.key_pos + (int64_t)t * a.topk : nullptr;
-            volatile int *go = reinterpret_cast<volatile int *>(tmem_holder + 2);
+            const int pieces_per_row = nch * 8;
+            const int n_pieces = LG_BN * pieces_per_row;  // 1280 or 1024: a multiple of 128
             bool ok = true;
             int sig = 0;  // next tile whose arrival is still to be signalled
             // A tile is signalled once this thread's copies for it have landed
             // (wait_group), made visible to the tensor core's async proxy
             // (fence.proxy.async), then counted on the tile's full barrier.
+            // (wait_group<N> returns once at most N of this thread's most
+            // recent copy groups are still pending; one group per tile.)
+            // Signalling each tile as soon as the next one is issued measured
+            // faster than keeping more tiles unsignalled in flight: the MMA
+            // needs tile i + 1 right after tile i.
             auto signal_through = [&](int last, bool leave_newest) {
                 while (sig <= last) {
                     if (leave_newest)
@@ -145,9 +167,9 @@ latent_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const GatherArgs a
             for (int i = 0; i < n_tiles; ++i) {
                 const int s = i % LG_NST;
                 // Stage s is freed by PV of tile i - NST, which the MMA issues
-                // only after QK^T of tile i - 1: signal everything issued so far
-                // before waiting for the stage.
-                if (i >= LG_NST) signal_through(i - 1, false);
+                // only after QK^T of tile i - NST + 1; every tile up to i - 2
+                // was signalled at the end of the previous iteration, so this
+                // wait cannot deadlock.
                 // One thread waits for the stage to be free and publishes the
                 // outcome, so all 128 gatherers take the same branch below.
                 if (tid == 0)
@@ -176,18 +198,18 @@ latent_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const GatherArgs a
                     ok = false;
                     break;
                 }
-                const uint32_t dst0 = sK + s * LG_K_BYTES;
-#pragma unroll
-                for (int j = 0; j < LG_PIECES / 128; ++j) {
-                    const int piece = tid + 128 * j;
-                    const int row = piece / (LG_DK / 8);
-                    const int pc = piece % (LG_DK / 8);  // 16-byte piece within the row
+                const uint32_t dst0 = sK + s * LG_KSTAGE;
+#pragma unroll 2
+                for (int piece = tid; piece < n_pieces; piece += 128) {
+                    const int row = piece / pieces_per_row;
+                    const int pc = piece - row * pieces_per_row;  // 16-byte piece within this CTA's columns
                     const int c = pc >> 3, sub = pc & 7;
-                    const __nv_bfloat16 *src = a.rows + (int64_t)rowid[s * LG_BN + row] * a.row_stride + pc * 8;
+                    const __nv_bfloat16 *src =
+                        a.rows + (int64_t)rowid[s * LG_BN + row] * a.row_stride + chunk0 * 64 + pc * 8;
                     cp_async16(dst0 + c * LG_KCH + row * 128 + ((sub ^ (row & 7)) << 4), src);
                 }
                 cp_async_commit();
-                // Tile i - 1 may be signalled while tile i is still in flight.
+                // Tiles up to i - 2 are signalled while i - 1 and i stay in flight.
                 if (i >= 1) signal_through(i - 1, true);
             }
             if (ok)
@@ -202,17 +224,15 @@ latent_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const GatherArgs a
             constexpr uint32_t idesc_qk = idesc_bf16_f32(128, LG_BN, false, false);
             constexpr uint32_t idesc_pv = idesc_bf16_f32(128, LG_HALF, false, true);
             const uint32_t tO = tmem + LG_T_O;
-            const uint32_t v_chunk0 = (uint32_t)(1 + 4 * half) * LG_KCH;  // first latent chunk of this half
             auto issue_qk = [&](int i) -> bool {
                 const int s = i % LG_NST;
                 if (!mbar_wait(bar(G_FULL + s), (uint32_t)(i / LG_NST) & 1u, abort_flag, &g_gather_err)) return false;
                 tc_fence_after();
                 const uint32_t tS = tmem + (uint32_t)((i & 1) * LG_BN);
-#pragma unroll
-                for (int kk = 0; kk < LG_DK / 16; ++kk) {
+                for (int kk = 0; kk < nch * 4; ++kk) {
                     const int c = kk >> 2, sub = kk & 3;
                     const uint64_t ad = sdesc_sw128(sQ + c * LG_QCH + sub * 32, 16, 1024);
-                    const uint64_t bd = sdesc_sw128(sK + s * LG_K_BYTES + c * LG_KCH + sub * 32, 16, 1024);
+                    const uint64_t bd = sdesc_sw128(sK + s * LG_KSTAGE + c * LG_KCH + sub * 32, 16, 1024);
                     mma_ss(tS, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
                 }
                 mma_commit(bar(G_SFULL + (i & 1)));
@@ -227,7 +247,7 @@ latent_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const GatherArgs a
                 const uint32_t tP = tmem + (uint32_t)((i & 1) * LG_BN);
 #pragma unroll
                 for (int kk = 0; kk < LG_BN / 16; ++kk) {
-                    const uint64_t bd = sdesc_sw128(sK + s * LG_K_BYTES + v_chunk0 + kk * 2048, LG_KCH, 1024);
+                    const uint64_t bd = sdesc_sw128(sK + s * LG_KSTAGE + vch * LG_KCH + kk * 2048, LG_KCH, 1024);
                     mma_ts(tO, tP + kk * 8, bd, idesc_pv, (i > 0 || kk > 0) ? 1u : 0u);
                 }
                 mma_commit(bar(G_EMPTY + s));
@@ -238,11 +258,16 @@ latent_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const GatherArgs a
         }
         __syncwarp();
     } else {
-        // ---------------------------------- softmax / correction / epilogue --
+        // ------------------- score exchange / softmax / correction / epilogue --
         const int qd = warp & 3;
         const int head = qd * 32 + lane;
         const uint32_t tl = tmem + ((uint32_t)(qd * 32) << 16);
         const float c = a.scale_log2;
+        // Exchange slot of this head: 8 pieces of 16 bytes, swizzled by head.
+        const uint32_t my_x = sX + (uint32_t)head * 128u;
+        const uint32_t peer_x = map_to_rank(my_x, peer);
+        const uint32_t peer_xfull = map_to_rank(bar(G_XFULL), peer);
+        const uint32_t peer_xfree = map_to_rank(bar(G_XFREE), peer);
         // l_run: sum of the fp32 weights (gives the LSE); l_mma: sum of the
         // bf16-rounded weights the PV MMA uses (normalises O, so a one-hot
         // softmax returns its V row exactly).
@@ -250,7 +275,8 @@ latent_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const GatherArgs a
         bool ok = true;
         for (int i = 0; i < n_tiles; ++i) {
             const int buf = i & 1, s = i % LG_NST;
-            if (!mbar_wait(bar(G_SFULL + buf), (uint32_t)(i >> 1) & 1u, abort_flag, &g_gather_err) ||
+            const uint32_t ph = (uint32_t)(i >> 1) & 1u;
+            if (!mbar_wait(bar(G_SFULL + buf), ph, abort_flag, &g_gather_err) ||
                 !mbar_wait(bar(G_FULL + s), (uint32_t)(i / LG_NST) & 1u, abort_flag, &g_gather_err)) {
                 ok = false;
                 break;
@@ -260,10 +286,37 @@ latent_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const GatherArgs a
             tmem_ld32(tl + (uint32_t)(buf * LG_BN), r);
             tmem_wait_ld();
             reg_fence(r);
-            const uint32_t mask = maskw[s];
-            float x[32];
+            // Send this CTA's partial scores to the peer, once the peer has
+            // read what was sent through this slot two tiles ago.
+            if (!mbar_wait(bar(G_XFREE + buf), ph ^ 1u, abort_flag, &g_gather_err)) {
+                ok = false;
+                break;
+            }
 #pragma unroll
-            for (int k = 0; k < 32; ++k) x[k] = ((mask >> k) & 1u) ? __uint_as_float(r[k]) : -INFINITY;
+            for (int k = 0; k < 8; ++k)
+                st_cluster_v4(peer_x + (uint32_t)(buf * LG_XBUF) + (uint32_t)((k ^ (head & 7)) << 4), r[4 * k],
+                              r[4 * k + 1], r[4 * k + 2], r[4 * k + 3]);
+            mbar_arrive_cluster(peer_xfull + 8u * (uint32_t)buf);
+            if (!mbar_wait_cluster(bar(G_XFULL + buf), ph, abort_flag, &g_gather_err)) {
+                ok = false;
+                break;
+            }
+            const uint4 *xin = reinterpret_cast<const uint4 *>(smem + LG_OFF_X + buf * LG_XBUF + head * 128);
+            float x[32];
+            const uint32_t mask = maskw[s];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const uint4 w = xin[k ^ (head & 7)];
+                const float v0 = __uint_as_float(r[4 * k]) + __uint_as_float(w.x);
+                const float v1 = __uint_as_float(r[4 * k + 1]) + __uint_as_float(w.y);
+                const float v2 = __uint_as_float(r[4 * k + 2]) + __uint_as_float(w.z);
+                const float v3 = __uint_as_float(r[4 * k + 3]) + __uint_as_float(w.w);
+                x[4 * k] = ((mask >> (4 * k)) & 1u) ? v0 : -INFINITY;
+                x[4 * k + 1] = ((mask >> (4 * k + 1)) & 1u) ? v1 : -INFINITY;
+                x[4 * k + 2] = ((mask >> (4 * k + 2)) & 1u) ? v2 : -INFINITY;
+                x[4 * k + 3] = ((mask >> (4 * k + 3)) & 1u) ? v3 : -INFINITY;
+            }
+            mbar_arrive_cluster(peer_xfree + 8u * (uint32_t)buf);  // my slot may be refilled
             float mx0 = x[0], mx1 = x[1];
 #pragma unroll
             for (int k = 2; k < 32; k += 2) {
@@ -299,7 +352,7 @@ latent_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const GatherArgs a
             }
             const float msub = (m_run == -INFINITY) ? 0.f : m_run;
             uint32_t pk[16];
-            float s0 = 0.f, s1 = 0.f, r0 = 0.f, r1 = 0.f;
+            float s0 = 0.f, s1 = 0.f, q0 = 0.f, q1 = 0.f;
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
                 const float p0 = ex2(fmaf(x[2 * k], c, -msub));
@@ -307,11 +360,11 @@ latent_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const GatherArgs a
                 pk[k] = pack_bf16x2(p0, p1);
                 s0 += p0;
                 s1 += p1;
-                r0 += __uint_as_float(pk[k] << 16);
-                r1 += __uint_as_float(pk[k] & 0xffff0000u);
+                q0 += __uint_as_float(pk[k] << 16);
+                q1 += __uint_as_float(pk[k] & 0xffff0000u);
             }
             l_run += s0 + s1;
-            l_mma += r0 + r1;
+            l_mma += q0 + q1;
             tmem_st16(tl + (uint32_t)(buf * LG_BN), pk);
             tmem_wait_st();
             tc_fence_before();
@@ -327,7 +380,7 @@ latent_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const GatherArgs a
         const bool good = have_o && l_run > 0.f;
         const float inv_l = (good && l_mma > 0.f) ? 1.f / l_mma : 0.f;
         const int64_t prow = ((int64_t)t * LG_H + head) * a.num_splits + split;
-        float4 *dst = reinterpret_cast<float4 *>(a.part_o + prow * LG_DV + half * LG_HALF);
+        float4 *dst = reinterpret_cast<float4 *>(a.part_o + prow * LG_DV + rank * LG_HALF);
 #pragma unroll 1
         for (int ch = 0; ch < LG_HALF / 32; ++ch) {
             uint32_t o[32];
@@ -345,7 +398,7 @@ latent_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const GatherArgs a
                                               __uint_as_float(o[4 * k + 2]) * inv_l,
                                               __uint_as_float(o[4 * k + 3]) * inv_l);
         }
-        if (half == 0) a.part_lse[prow] = good ? m_run + __log2f(l_run) : -INFINITY;
+        if (rank == 0) a.part_lse[prow] = good ? m_run + __log2f(l_run) : -INFINITY;
     }
 
     tc_fence_before();
@@ -354,6 +407,8 @@ latent_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const GatherArgs a
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
+    // No CTA may leave while its peer can still write into its shared memory.
+    cluster_sync();
 }
 
 cudaError_t launch_decode_gather(const GatherLaunch &L, cudaStream_t stream) {

@@ -2,21 +2,25 @@
 // the log-sum-exp combine shared by both decode paths.
 //
 // Decode is bandwidth-bound (about 4 FLOP per byte of K/V at head dim 128),
-// so it runs on the CUDA cores and is organised around moving bytes:
+// so everything is organised around moving bytes with as few instructions
+// per byte as possible:
 //   - grid = (split, KV head, sequence); one CTA streams up to
 //     blocks_per_split 64-token blocks of ONE KV head and serves all
 //     Hq / Hkv query heads of that group from the same bytes;
-//   - one producer warp resolves block ids through the block table and moves
-//     each block's K and V tile (16 KB each, contiguous in the cache) with a
-//     single bulk-async copy apiece into a 3-stage shared-memory ring;
-//   - four consumer warps = eight groups of 16 lanes; a group owns 8 keys of
-//     every block and each lane 8 of the 128 head dims, so a key row is read
-//     from shared memory as one 256-byte conflict-free sweep, and the dot
-//     product is finished with a 4-step butterfly inside the 16 lanes;
-//   - each group runs its own online softmax (base 2, scale*log2(e) folded
-//     into Q) and the eight groups are merged at the end; the CTA writes one
-//     partial (O / l, log2-sum-exp) per query head and split, and the combine
-//     kernel merges the splits.
+//   - one producer warp resolves block ids through the block table (32 table
+//     entries per coalesced read) and moves each block's K and V tile with
+//     TMA tensor copies into a 3-stage, 128-byte-swizzled shared-memory ring;
+//   - four consumer warps each own 16 of the block's 64 keys.  The small
+//     contractions run as warp-level bf16 MMAs (m16n8k16, fp32 accumulate):
+//     the query heads are the M rows (padded to 16), so QK^T is 16 MMAs and
+//     PV 16 MMAs per warp per block, with the score fragments reused directly
+//     as the P operand; swizzled ldmatrix reads are bank-conflict free.
+//     (The 128-row tcgen05 MMA would leave 124 of 128 rows idle here and
+//     needs TMEM allocation per CTA for no throughput gain: the tensor core
+//     is nowhere near the limit in decode.)
+//   - each warp keeps its own online softmax (base 2); the four warps merge
+//     at the end, and the CTA writes one partial (O / l, log2-sum-exp) per
+//     query head and split for the combine kernel.
 // Sources: key j of sequence b lives in block block_table[b][j / 64], slot
 // j % 64, cache laid out [blocks, kv heads, 64, d] ("MLA Decode Attention
 // Kernel API Reference", kv_cache; the paged layout); decode is a separate
@@ -41,30 +45,22 @@ constexpr int PD_NST = 3;
 constexpr int PD_TILE = PD_BS * PD_D * 2;        // bytes of one block of K (or V) for one head
 constexpr int PD_STAGE = 2 * PD_TILE;            // K + V
 constexpr int PD_OFF_BAR = PD_NST * PD_STAGE;
-constexpr int PD_SMEM = PD_OFF_BAR + 128 + 128;  // ring + barriers + alignment slack
+constexpr int PD_SMEM = PD_OFF_BAR + 128 + 1024;  // ring + barriers + 1024-byte alignment slack
 
 struct PagedArgs {
     const __nv_bfloat16 *q;
-    const __nv_bfloat16 *k_cache, *v_cache;
     const int32_t *block_table, *seq_lens;
     int max_blocks, Hq, Hkv, num_blocks, bps, num_splits;
     float scale_log2;
     float *part_o, *part_lse;
 };
 
-FA_DEV void bf16x8_to_f32(const uint4 &u, float (&f)[8]) {
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        f[2 * i] = __uint_as_float(w[i] << 16);
-        f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
-    }
-}
-
 template <int G>
-__global__ void __launch_bounds__(160) paged_decode_kernel(const PagedArgs a) {
+__global__ void __launch_bounds__(160) paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
+                                                           const __grid_constant__ CUtensorMap tmV,
+                                                           const PagedArgs a) {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int split = blockIdx.x, hkv = blockIdx.y, b = blockIdx.z;
 
     int seq_len = a.seq_lens[b];
@@ -98,8 +94,13 @@ __global__ void __launch_bounds__(160) paged_decode_kernel(const PagedArgs a) {
 
     if (warp == 4) {
         // ---------------------------------------------------- producer --
+        if (lane == 0) {
+            prefetch_tmap(&tmK);
+            prefetch_tmap(&tmV);
+        }
         const int32_t *tbl = a.block_table + (int64_t)b * a.max_blocks + blk0;
         int32_t ids = 0;
+        int issued = 0;
         for (int i = 0; i < nblk; ++i) {
             if ((i & 31) == 0) {
                 ids = (i + lane < nblk) ? tbl[i + lane] : 0;
@@ -115,38 +116,48 @@ __global__ void __launch_bounds__(160) paged_decode_kernel(const PagedArgs a) {
             if (lane == 0) ok = mbar_wait(empty(s), ph ^ 1u, abort_flag, &g_decode_err);
             if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
             if (lane == 0) {
-                const int64_t off = ((int64_t)blk * a.Hkv + hkv) * (PD_BS * PD_D);
+                const int row0 = (blk * a.Hkv + hkv) * PD_BS;  // first cache row of this (block, head)
+                const uint32_t dst = sbase + s * PD_STAGE;
                 mbar_arrive_expect_tx(full(s), PD_STAGE);
-                bulk_load(sbase + s * PD_STAGE, a.k_cache + off, PD_TILE, full(s));
-                bulk_load(sbase + s * PD_STAGE + PD_TILE, a.v_cache + off, PD_TILE, full(s));
+                tma_load_2d(dst, &tmK, full(s), 0, row0);
+                tma_load_2d(dst + PD_TILE / 2, &tmK, full(s), 64, row0);
+                tma_load_2d(dst + PD_TILE, &tmV, full(s), 0, row0);
+                tma_load_2d(dst + PD_TILE + PD_TILE / 2, &tmV, full(s), 64, row0);
             }
+            issued = i + 1;
         }
         if (lane == 0 && *abort_flag) {
-            for (int i = max(0, nblk - PD_NST); i < nblk; ++i)
+            for (int i = max(0, issued - PD_NST); i < issued; ++i)
                 mbar_wait_drain(full(i % PD_NST), (uint32_t)(i / PD_NST) & 1u);
         }
         return;
     }
 
     // --------------------------------------------------------- consumers --
-    const int gi = warp * 2 + (lane >> 4);  // key group: keys [8 gi, 8 gi + 8) of each block
-    const int l16 = lane & 15;              // head dims [8 l16, 8 l16 + 8)
-    float qf[G][8];
+    // Warp w owns keys [16 w, 16 w + 16) of every block.  MMA fragment roles:
+    // gid = lane / 4 is the M row (query head, valid when gid < G), tig =
+    // lane % 4 picks the column pairs.
+    const int gid = lane >> 2, tig = lane & 3;
+    const bool head_ok = gid < G;
+    uint32_t qa[8][2];
+    {
+        const uint32_t *qp = reinterpret_cast<const uint32_t *>(
+            a.q + ((int64_t)b * a.Hq + (int64_t)hkv * G + (head_ok ? gid : 0)) * PD_D);
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-        const uint4 u = *reinterpret_cast<const uint4 *>(a.q + ((int64_t)b * a.Hq + hkv * G + g) * PD_D + l16 * 8);
-        bf16x8_to_f32(u, qf[g]);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) qf[g][e] *= a.scale_log2;
+        for (int ks = 0; ks < 8; ++ks) {
+            qa[ks][0] = head_ok ? qp[(ks * 16 + 2 * tig) >> 1] : 0u;
+            qa[ks][1] = head_ok ? qp[(ks * 16 + 8 + 2 * tig) >> 1] : 0u;
+        }
     }
-    float m[G], l[G], o[G][8];
+    const float c = a.scale_log2;
+    float m_run = -INFINITY, l_run = 0.f;
+    float o[16][4];
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-        m[g] = -INFINITY;
-        l[g] = 0.f;
+    for (int nt = 0; nt < 16; ++nt)
 #pragma unroll
-        for (int e = 0; e < 8; ++e) o[g][e] = 0.f;
-    }
+        for (int e = 0; e < 4; ++e) o[nt][e] = 0.f;
+    // ldmatrix lane roles: matrix mi = lane / 8, row lr = lane % 8
+    const int mi = lane >> 3, lr = lane & 7;
 
     bool ok = true;
     for (int i = 0; i < nblk; ++i) {
@@ -155,79 +166,84 @@ __global__ void __launch_bounds__(160) paged_decode_kernel(const PagedArgs a) {
             ok = false;
             break;
         }
-        const uint8_t *Ks = smem + s * PD_STAGE;
-        const uint8_t *Vs = Ks + PD_TILE;
-        const int j0 = (blk0 + i) * PD_BS + gi * 8;
-        float sc[8][G];
+        const uint32_t sK = sbase + s * PD_STAGE;
+        const uint32_t sV = sK + PD_TILE;
+        // ---- S = Q K^T for this warp's 16 keys (two n-tiles of 8) ----
+        float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        {
+            const int key = warp * 16 + (mi >> 1) * 8 + lr;
 #pragma unroll
-        for (int tt = 0; tt < 8; ++tt) {
-            float kf[8];
-            bf16x8_to_f32(*reinterpret_cast<const uint4 *>(Ks + (gi * 8 + tt) * 256 + l16 * 16), kf);
-#pragma unroll
-            for (int g = 0; g < G; ++g) {
-                float part = 0.f;
-#pragma unroll
-                for (int e = 0; e < 8; ++e) part = fmaf(qf[g][e], kf[e], part);
-                sc[tt][g] = part;
+            for (int ks = 0; ks < 8; ++ks) {
+                const int d0 = ks * 16 + (mi & 1) * 8;
+                const uint32_t addr = sK + (uint32_t)((d0 >> 6) * (PD_TILE / 2) + key * 128 +
+                                                      ((((d0 & 63) >> 3) ^ (key & 7)) << 4));
+                uint32_t b00, b01, b10, b11;
+                ldsm_x4(addr, b00, b01, b10, b11);
+                mma_16816(sc[0], qa[ks][0], 0u, qa[ks][1], 0u, b00, b01);
+                mma_16816(sc[1], qa[ks][0], 0u, qa[ks][1], 0u, b10, b11);
             }
         }
+        // ---- online softmax over the 4 scores this thread holds ----
+        const int key0 = (blk0 + i) * PD_BS + warp * 16 + 2 * tig;
+        float x[4];
 #pragma unroll
-        for (int off = 8; off >= 1; off >>= 1)
+        for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-            for (int tt = 0; tt < 8; ++tt)
+            for (int e = 0; e < 2; ++e)
+                x[nt * 2 + e] = (key0 + nt * 8 + e < seq_len) ? sc[nt][e] * c : -INFINITY;
+        float mt = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+        mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 1));
+        mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 2));
+        const float mn = fmaxf(m_run, mt);
+        const float msub = (mn == -INFINITY) ? 0.f : mn;
+        const float alpha = ex2(m_run - msub);
+        float p[4];
 #pragma unroll
-                for (int g = 0; g < G; ++g) sc[tt][g] += __shfl_xor_sync(0xffffffffu, sc[tt][g], off);
-        const int nvalid = seq_len - j0;  // keys tt < nvalid are real
+        for (int k = 0; k < 4; ++k) p[k] = ex2(x[k] - msub);
+        l_run = l_run * alpha + (p[0] + p[1]) + (p[2] + p[3]);
+        m_run = mn;
 #pragma unroll
-        for (int tt = 0; tt < 8; ++tt)
-            if (tt >= nvalid)
-#pragma unroll
-                for (int g = 0; g < G; ++g) sc[tt][g] = -INFINITY;
-        float p[8][G];
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-            float mt = sc[0][g];
-#pragma unroll
-            for (int tt = 1; tt < 8; ++tt) mt = fmaxf(mt, sc[tt][g]);
-            const float mn = fmaxf(m[g], mt);
-            const float msub = (mn == -INFINITY) ? 0.f : mn;
-            const float alpha = ex2(m[g] - msub);
-            float ps = 0.f;
-#pragma unroll
-            for (int tt = 0; tt < 8; ++tt) {
-                p[tt][g] = ex2(sc[tt][g] - msub);
-                ps += p[tt][g];
-            }
-            l[g] = l[g] * alpha + ps;
-#pragma unroll
-            for (int e = 0; e < 8; ++e) o[g][e] *= alpha;
-            m[g] = mn;
+        for (int nt = 0; nt < 16; ++nt) {
+            o[nt][0] *= alpha;
+            o[nt][1] *= alpha;
         }
+        // ---- O += P V: the score fragments are the A operand ----
+        const uint32_t pa0 = pack_bf16x2(p[0], p[1]);
+        const uint32_t pa2 = pack_bf16x2(p[2], p[3]);
+        {
+            const int key = warp * 16 + (mi & 1) * 8 + lr;
 #pragma unroll
-        for (int tt = 0; tt < 8; ++tt) {
-            float vf[8];
-            bf16x8_to_f32(*reinterpret_cast<const uint4 *>(Vs + (gi * 8 + tt) * 256 + l16 * 16), vf);
-#pragma unroll
-            for (int g = 0; g < G; ++g)
-#pragma unroll
-                for (int e = 0; e < 8; ++e) o[g][e] = fmaf(p[tt][g], vf[e], o[g][e]);
+            for (int pr = 0; pr < 8; ++pr) {
+                const int nt = 2 * pr + (mi >> 1);  // 8-wide slice of head dims
+                const uint32_t addr = sV + (uint32_t)(((nt * 8) >> 6) * (PD_TILE / 2) + key * 128 +
+                                                      (((nt & 7) ^ (key & 7)) << 4));
+                uint32_t v0l, v0h, v1l, v1h;
+                ldsm_x4_t(addr, v0l, v0h, v1l, v1h);
+                mma_16816(o[2 * pr], pa0, 0u, pa2, 0u, v0l, v0h);
+                mma_16816(o[2 * pr + 1], pa0, 0u, pa2, 0u, v1l, v1h);
+            }
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(empty(s));
     }
+    // the four lanes of a quad hold partial sums of the same head
+    l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
+    l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
 
-    // ---- merge the eight key groups (the ring is free: every copy landed) ----
+    // ---- merge the four warps (the ring is free: every copy has landed) ----
     asm volatile("bar.sync 1, 128;" ::: "memory");
-    float *mo = reinterpret_cast<float *>(smem);    // [8][G][128]
-    float *mm = mo + 8 * G * PD_D;                  // [8][G]
-    float *ml = mm + 8 * G;                         // [8][G]
+    float *mo = reinterpret_cast<float *>(smem);  // [4][G][128]
+    float *mm = mo + 4 * G * PD_D;                 // [4][G]
+    float *ml = mm + 4 * G;                        // [4][G]
+    if (head_ok) {
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) mo[(gi * G + g) * PD_D + l16 * 8 + e] = o[g][e];
-        if (l16 == 0) {
-            mm[gi * G + g] = m[g];
-            ml[gi * G + g] = l[g];
+        for (int nt = 0; nt < 16; ++nt) {
+            mo[(warp * G + gid) * PD_D + nt * 8 + 2 * tig] = o[nt][0];
+            mo[(warp * G + gid) * PD_D + nt * 8 + 2 * tig + 1] = o[nt][1];
+        }
+        if (tig == 0) {
+            mm[warp * G + gid] = m_run;
+            ml[warp * G + gid] = l_run;
         }
     }
     asm volatile("bar.sync 1, 128;" ::: "memory");
@@ -236,11 +252,11 @@ __global__ void __launch_bounds__(160) paged_decode_kernel(const PagedArgs a) {
     for (int g = 0; g < G; ++g) {
         float M = -INFINITY;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) M = fmaxf(M, mm[k * G + g]);
+        for (int k = 0; k < 4; ++k) M = fmaxf(M, mm[k * G + g]);
         const float msub = (M == -INFINITY) ? 0.f : M;
         float L = 0.f, O = 0.f;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
+        for (int k = 0; k < 4; ++k) {
             const float w = ex2(mm[k * G + g] - msub);
             L = fmaf(w, ml[k * G + g], L);
             O = fmaf(w, mo[(k * G + g) * PD_D + d], O);
@@ -349,20 +365,18 @@ cudaError_t launch_combine(const float *part_o, const float *part_lse, int rows,
 }
 
 template <int G>
-static cudaError_t launch_g(const PagedArgs &a, int B, cudaStream_t stream) {
+static cudaError_t launch_g(const PagedLaunch &L, const PagedArgs &a, int B, cudaStream_t stream) {
     auto kern = paged_decode_kernel<G>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, PD_SMEM);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)a.num_splits, (unsigned)a.Hkv, (unsigned)B);
-    kern<<<grid, 160, PD_SMEM, stream>>>(a);
+    kern<<<grid, 160, PD_SMEM, stream>>>(L.tmK, L.tmV, a);
     return cudaGetLastError();
 }
 
 cudaError_t launch_decode_paged(const PagedLaunch &L, cudaStream_t stream) {
     PagedArgs a;
     a.q = static_cast<const __nv_bfloat16 *>(L.q);
-    a.k_cache = static_cast<const __nv_bfloat16 *>(L.k_cache);
-    a.v_cache = static_cast<const __nv_bfloat16 *>(L.v_cache);
     a.block_table = L.block_table;
     a.seq_lens = L.seq_lens;
     a.max_blocks = L.max_blocks_per_seq;
@@ -376,10 +390,10 @@ cudaError_t launch_decode_paged(const PagedLaunch &L, cudaStream_t stream) {
     a.part_lse = L.part_lse;
     cudaError_t e;
     switch (L.Hq / L.Hkv) {
-        case 1: e = launch_g<1>(a, L.B, stream); break;
-        case 2: e = launch_g<2>(a, L.B, stream); break;
-        case 4: e = launch_g<4>(a, L.B, stream); break;
-        case 8: e = launch_g<8>(a, L.B, stream); break;
+        case 1: e = launch_g<1>(L, a, L.B, stream); break;
+        case 2: e = launch_g<2>(L, a, L.B, stream); break;
+        case 4: e = launch_g<4>(L, a, L.B, stream); break;
+        case 8: e = launch_g<8>(L, a, L.B, stream); break;
         default: return cudaErrorInvalidValue;
     }
     if (e != cudaSuccess) return e;

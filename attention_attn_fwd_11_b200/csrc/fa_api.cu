@@ -159,6 +159,18 @@ fa_status check_paged_ptrs(const fa_decode_paged_params *p) {
     return FA_OK;
 }
 
+// Both caches as 2-D [num_blocks * Hkv * 64 rows, 128] bf16 tensors for TMA
+// (128-byte swizzle, 64 x 64 boxes).
+fa_status encode_paged_caches(const fa_decode_paged_params *p, fa::PagedLaunch *L) {
+    if (!get_encoder()) return fail(FA_ERR_CUDA, "fa_decode_paged: cuTensorMapEncodeTiled is not available");
+    const int64_t rows = (int64_t)p->num_blocks * p->Hkv * p->block_size;
+    if (rows >= (int64_t(1) << 31))
+        return fail(FA_ERR_INVALID_ARG, "fa_decode_paged: num_blocks * Hkv * block_size must be < 2^31");
+    fa_status st = encode_2d(&L->tmK, p->k_cache, p->dk, rows, p->dk, 64, "fa_decode_paged k_cache");
+    if (st != FA_OK) return st;
+    return encode_2d(&L->tmV, p->v_cache, p->dv, rows, p->dv, 64, "fa_decode_paged v_cache");
+}
+
 size_t paged_ws_bytes(const fa_decode_paged_params *p, int splits) {
     const size_t rows = (size_t)p->B * p->Hq * (size_t)splits;
     size_t o = rows * 128 * sizeof(float);
@@ -171,10 +183,12 @@ size_t paged_ws_bytes(const fa_decode_paged_params *p, int splits) {
 int gather_splits(const fa_decode_gather_params *p) {
     const int max_s = (p->topk + 63) / 64 > 0 ? (p->topk + 63) / 64 : 1;
     if (p->num_splits > 0) return p->num_splits < max_s ? p->num_splits : max_s;
-    // Automatic: about two waves of (token, split) units, at least 256 keys each.
-    const long long want = 148LL * 2;
-    long long s = (want + (p->T > 0 ? p->T : 1) - 1) / (p->T > 0 ? p->T : 1);
-    long long max_by_len = (p->topk + 255) / 256;
+    // Automatic: one two-CTA cluster per (token, split) and at most one wave
+    // of clusters (74 on 148 SMs), with at least 128 keys per split.
+    const long long want = 74;
+    const long long T = p->T > 0 ? p->T : 1;
+    long long s = want / T;
+    long long max_by_len = (p->topk + 127) / 128;
     if (s > max_by_len) s = max_by_len;
     if (s < 1) s = 1;
     return (int)s;
@@ -302,6 +316,8 @@ fa_status fa_decode_paged(const fa_decode_paged_params *p, void *stream) {
     if (!p->workspace || p->workspace_bytes < need || ((uintptr_t)p->workspace & 255u))
         return fail(FA_ERR_WORKSPACE, "fa_decode_paged: workspace needs %zu bytes, 256-byte aligned", need);
     fa::PagedLaunch L;
+    st = encode_paged_caches(p, &L);
+    if (st != FA_OK) return st;
     L.q = p->q;
     L.k_cache = p->k_cache;
     L.v_cache = p->v_cache;
@@ -340,6 +356,8 @@ fa_status fa_decode_paged_noalloc(const fa_decode_paged_params *p, void *stream)
                     "holds %zu; pass fewer num_splits or call fa_decode_paged with a workspace",
                     need, have);
     fa::PagedLaunch L;
+    st = encode_paged_caches(p, &L);
+    if (st != FA_OK) return st;
     L.q = p->q;
     L.k_cache = p->k_cache;
     L.v_cache = p->v_cache;

@@ -29,6 +29,7 @@ cudaError_t prefill2_device_error(int clear, int *code);
 
 // ---- paged decode --------------------------------------------------------
 struct PagedLaunch {
+    CUtensorMap tmK, tmV;  // caches viewed as [blocks * Hkv * 64 rows, 128], box 64 x 64, 128-byte swizzle
     const void *q, *k_cache, *v_cache;
     const int32_t *block_table, *seq_lens;
     int max_blocks_per_seq, B, Hq, Hkv, num_blocks;

@@ -52,7 +52,12 @@ template <int D>
 struct P2Cfg {
     static constexpr int BM = 128;
     static constexpr int BN = 128;
-    static constexpr int NST = D == 128 ? 2 : 4;
+#ifdef FA_P2_NSTK
+    static constexpr int NSTK = FA_P2_NSTK;
+#else
+    static constexpr int NSTK = D == 128 ? 2 : 4;  // K ring depth
+#endif
+    static constexpr int NSTV = D == 128 ? 2 : 4;  // V ring depth
     static constexpr int NCH = D / 64;
     static constexpr int Q_CHUNK = BM * 128;
     static constexpr int KV_CHUNK = BN * 128;
@@ -60,8 +65,8 @@ struct P2Cfg {
     static constexpr int KV_BYTES = BN * D * 2;
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_K = 2 * Q_TILE;
-    static constexpr int OFF_V = OFF_K + NST * KV_BYTES;
-    static constexpr int OFF_BAR = OFF_V + NST * KV_BYTES;
+    static constexpr int OFF_V = OFF_K + NSTK * KV_BYTES;
+    static constexpr int OFF_BAR = OFF_V + NSTV * KV_BYTES;
     static constexpr int SMEM_BYTES = OFF_BAR + 512 + 1024;
     static constexpr int T_O = 2 * BN;  // O0 at T_O, O1 at T_O + D
     static_assert(2 * BN + 2 * D <= 512, "TMEM budget");
@@ -74,6 +79,13 @@ enum {
 };
 
 constexpr float kP2RescaleThreshold = 8.0f;
+
+// Every FA_EXP2_POLY_EVERY-th pair of softmax elements takes 2^x on the FMA
+// pipe (ex2_poly) instead of the MUFU unit, which the two softmax
+// warpgroups otherwise saturate (0 = never).
+#ifndef FA_EXP2_POLY_EVERY
+#define FA_EXP2_POLY_EVERY 0
+#endif
 
 struct UnitInfo {
     int b, hq, q0, n[2], N;
@@ -105,12 +117,26 @@ FA_DEV bool p2_unit(const Prefill2Args &a, int round, UnitInfo &u) {
     return true;
 }
 
+// 384 threads = three warpgroups: warpgroup 0 holds the producer (warp 0)
+// and the MMA issuer (warp 1), warpgroups 1 and 2 are the softmax groups.
+// setmaxnreg then moves registers from warpgroup 0 to the softmax groups
+// (FA_P2_NO_SETMAXNREG turns that off; FA_P2_THREADS=320 packs the softmax
+// warps into warps 2-9 instead).
+#ifndef FA_P2_THREADS
+#define FA_P2_THREADS 384
+#endif
+#if !defined(FA_P2_NO_SETMAXNREG) && FA_P2_THREADS == 384
+#define FA_P2_SETMAXNREG 1
+#endif
+constexpr int P2_THREADS = FA_P2_THREADS;
+constexpr int P2_SOFTMAX_WARP0 = P2_THREADS == 384 ? 4 : 2;
+
 template <int D>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(P2_THREADS, 1)
 prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const Prefill2Args a) {
     using C = P2Cfg<D>;
-    constexpr int BN = C::BN, NST = C::NST;
+    constexpr int BN = C::BN, NSTK = C::NSTK, NSTV = C::NSTV;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
@@ -119,9 +145,9 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     const uint32_t bar0 = smem_u32(bars);
     auto bar = [&](int i) -> uint32_t { return bar0 + 8u * (uint32_t)i; };
     auto k_full = [&](int s) { return bar(P2_RING + s); };
-    auto k_empty = [&](int s) { return bar(P2_RING + NST + s); };
-    auto v_full = [&](int s) { return bar(P2_RING + 2 * NST + s); };
-    auto v_empty = [&](int s) { return bar(P2_RING + 3 * NST + s); };
+    auto k_empty = [&](int s) { return bar(P2_RING + NSTK + s); };
+    auto v_full = [&](int s) { return bar(P2_RING + 2 * NSTK + s); };
+    auto v_empty = [&](int s) { return bar(P2_RING + 2 * NSTK + NSTV + s); };
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + 40);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
 
@@ -139,9 +165,11 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             mbar_init(bar(P2_OFREE + i), 128);
             mbar_init(bar(P2_USTART + i), 1);
         }
-        for (int s = 0; s < NST; ++s) {
+        for (int s = 0; s < NSTK; ++s) {
             mbar_init(k_full(s), 1);
             mbar_init(k_empty(s), 1);
+        }
+        for (int s = 0; s < NSTV; ++s) {
             mbar_init(v_full(s), 1);
             mbar_init(v_empty(s), 1);
         }
@@ -156,7 +184,21 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
+#if defined(FA_P2_SETMAXNREG) && FA_P2_THREADS == 384
+    // Registers move from the producer/MMA warpgroup (warps 0-3) to the two
+    // softmax warpgroups: 128 * 96 + 256 * 200 = 63488 <= 384 * 168, the
+    // launch allocation (checked on the host before launch).  Each setmaxnreg
+    // sits at the top of its role's branch so the compiler applies the
+    // matching budget to that role's code.
+#define P2_REGS_LOW() asm volatile("setmaxnreg.dec.sync.aligned.u32 96;\n" ::: "memory")
+#define P2_REGS_HIGH() asm volatile("setmaxnreg.inc.sync.aligned.u32 200;\n" ::: "memory")
+#else
+#define P2_REGS_LOW() ((void)0)
+#define P2_REGS_HIGH() ((void)0)
+#endif
 
+    if (warp < P2_SOFTMAX_WARP0) {
+    P2_REGS_LOW();
     if (warp == 0) {
         // ------------------------------------------------ TMA producer --
         if (lane == 0) {
@@ -177,28 +219,33 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                         tma_load_4d(sQ + i * C::Q_TILE + c * C::Q_CHUNK, &tmQ, bar(P2_QFULL), c * 64, u.q0 + 128 * i,
                                     u.hq, u.b);
                 for (int t = 0; t < u.N; ++t, ++kc) {
-                    const int s = kc % NST;
-                    const uint32_t ph = (uint32_t)(kc / NST) & 1u;
-                    if (!mbar_wait(k_empty(s), ph ^ 1u, abort_flag, &g_prefill2_err)) { ok = false; break; }
-                    mbar_arrive_expect_tx(k_full(s), C::KV_BYTES);
+                    const int sk = kc % NSTK, sv = kc % NSTV;
+                    if (!mbar_wait(k_empty(sk), ((uint32_t)(kc / NSTK) & 1u) ^ 1u, abort_flag, &g_prefill2_err)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(k_full(sk), C::KV_BYTES);
 #pragma unroll
                     for (int c = 0; c < C::NCH; ++c)
-                        tma_load_4d(sK + s * C::KV_BYTES + c * C::KV_CHUNK, &tmK, k_full(s), c * 64, t * BN, hkv, u.b);
-                    if (!mbar_wait(v_empty(s), ph ^ 1u, abort_flag, &g_prefill2_err)) { ok = false; break; }
-                    mbar_arrive_expect_tx(v_full(s), C::KV_BYTES);
+                        tma_load_4d(sK + sk * C::KV_BYTES + c * C::KV_CHUNK, &tmK, k_full(sk), c * 64, t * BN, hkv, u.b);
+                    if (!mbar_wait(v_empty(sv), ((uint32_t)(kc / NSTV) & 1u) ^ 1u, abort_flag, &g_prefill2_err)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(v_full(sv), C::KV_BYTES);
 #pragma unroll
                     for (int c = 0; c < C::NCH; ++c)
-                        tma_load_4d(sV + s * C::KV_BYTES + c * C::KV_CHUNK, &tmV, v_full(s), c * 64, t * BN, hkv, u.b);
+                        tma_load_4d(sV + sv * C::KV_BYTES + c * C::KV_CHUNK, &tmV, v_full(sv), c * 64, t * BN, hkv, u.b);
                     issued = kc + 1;
                 }
             }
             if (*abort_flag) {
                 // Let the copies still in flight land before the CTA exits.
                 mbar_wait_drain(bar(P2_QFULL), (uint32_t)(max(uc - 1, 0)) & 1u);
-                for (int k = max(0, issued - NST); k < issued; ++k) {
-                    mbar_wait_drain(k_full(k % NST), (uint32_t)(k / NST) & 1u);
-                    mbar_wait_drain(v_full(k % NST), (uint32_t)(k / NST) & 1u);
-                }
+                for (int k = max(0, issued - NSTK); k < issued; ++k)
+                    mbar_wait_drain(k_full(k % NSTK), (uint32_t)(k / NSTK) & 1u);
+                for (int k = max(0, issued - NSTV); k < issued; ++k)
+                    mbar_wait_drain(v_full(k % NSTV), (uint32_t)(k / NSTV) & 1u);
             }
         }
     } else if (warp == 1) {
@@ -248,8 +295,8 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                     continue;
                 }
                 {
-                    const int s0 = kc % NST;
-                    if (!mbar_wait(k_full(s0), (uint32_t)(kc / NST) & 1u, abort_flag, &g_prefill2_err)) break;
+                    const int s0 = kc % NSTK;
+                    if (!mbar_wait(k_full(s0), (uint32_t)(kc / NSTK) & 1u, abort_flag, &g_prefill2_err)) break;
                     tc_fence_after();
                     if (u.n[0] > 0) qk(0, s0);
                     if (u.n[1] > 0) qk(1, s0);
@@ -258,13 +305,13 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 }
                 for (int t = 0; t < u.N; ++t) {
                     const int kt = kc + t;
-                    const int s = kt % NST;
+                    const int s = kt % NSTV;  // V stage of tile t
                     const bool has_next = t + 1 < u.N;
-                    const int s1 = (kt + 1) % NST;
+                    const int s1 = (kt + 1) % NSTK;  // K stage of tile t + 1
                     bool v_ready = false;
                     if (t < u.n[0]) {
                         if (!mbar_wait(bar(P2_PREADY + 0), (uint32_t)pcnt[0] & 1u, abort_flag, &g_prefill2_err) ||
-                            !mbar_wait(v_full(s), (uint32_t)(kt / NST) & 1u, abort_flag, &g_prefill2_err)) {
+                            !mbar_wait(v_full(s), (uint32_t)(kt / NSTV) & 1u, abort_flag, &g_prefill2_err)) {
                             ok = false;
                             break;
                         }
@@ -274,7 +321,7 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                         pv(0, s, t == 0);
                     }
                     if (has_next) {
-                        if (!mbar_wait(k_full(s1), (uint32_t)((kt + 1) / NST) & 1u, abort_flag, &g_prefill2_err)) {
+                        if (!mbar_wait(k_full(s1), (uint32_t)((kt + 1) / NSTK) & 1u, abort_flag, &g_prefill2_err)) {
                             ok = false;
                             break;
                         }
@@ -284,7 +331,7 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                     if (t < u.n[1]) {
                         if (!mbar_wait(bar(P2_PREADY + 1), (uint32_t)pcnt[1] & 1u, abort_flag, &g_prefill2_err) ||
                             (!v_ready &&
-                             !mbar_wait(v_full(s), (uint32_t)(kt / NST) & 1u, abort_flag, &g_prefill2_err))) {
+                             !mbar_wait(v_full(s), (uint32_t)(kt / NSTV) & 1u, abort_flag, &g_prefill2_err))) {
                             ok = false;
                             break;
                         }
@@ -305,9 +352,11 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             mbar_wait_drain(bar(P2_DRAIN), 0);
         }
         __syncwarp();
-    } else if (warp >= 4) {
+    }
+    } else {
+        P2_REGS_HIGH();
         // ------------------------------- softmax / correction / epilogue --
-        const int ti = (warp - 4) >> 2;              // which query tile of the unit
+        const int ti = (warp - P2_SOFTMAX_WARP0) >> 2;  // which query tile of the unit
         const int qd = warp & 3;                     // TMEM lane quadrant
         const int row = qd * 32 + lane;
         const uint32_t tl = tmem + ((uint32_t)(qd * 32) << 16);
@@ -382,15 +431,25 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                         tmem_st32(tO + (uint32_t)(ch * 32), o);
                     }
                 }
-                const float msub = (m_run == -INFINITY) ? 0.f : m_run;
+                const bool empty_row = m_run == -INFINITY;  // no visible key so far: P = 0
+                const float msub = empty_row ? 0.f : m_run;
                 float s0 = 0.f, s1 = 0.f;
 #pragma unroll
                 for (int g = 0; g < BN / 32; ++g) {
                     uint32_t pk[16];
 #pragma unroll
                     for (int k = 0; k < 16; ++k) {
-                        const float p0 = ex2(fmaf(x[g * 32 + 2 * k], c, -msub));
-                        const float p1 = ex2(fmaf(x[g * 32 + 2 * k + 1], c, -msub));
+                        const float a0 = fmaf(x[g * 32 + 2 * k], c, -msub);
+                        const float a1 = fmaf(x[g * 32 + 2 * k + 1], c, -msub);
+                        float p0, p1;
+                        if (FA_EXP2_POLY_EVERY > 0 && (k % (FA_EXP2_POLY_EVERY > 0 ? FA_EXP2_POLY_EVERY : 1)) ==
+                                                          (FA_EXP2_POLY_EVERY > 0 ? FA_EXP2_POLY_EVERY - 1 : 0)) {
+                            p0 = empty_row ? 0.f : ex2_poly(a0);
+                            p1 = empty_row ? 0.f : ex2_poly(a1);
+                        } else {
+                            p0 = ex2(a0);
+                            p1 = ex2(a1);
+                        }
                         s0 += p0;
                         s1 += p1;
                         pk[k] = pack_bf16x2(p0, p1);
@@ -486,8 +545,17 @@ static cudaError_t launch_p2(const PrefillLaunch &L, int num_sms, cudaStream_t s
     a.o_ss = L.o_ss;
     a.o_bf16 = L.o_bf16;
     a.lse = L.lse;
+#if defined(FA_P2_SETMAXNREG) && FA_P2_THREADS == 384
+    {
+        // The register split inside the kernel needs the full launch allocation.
+        cudaFuncAttributes fattr;
+        e = cudaFuncGetAttributes(&fattr, kern);
+        if (e != cudaSuccess) return e;
+        if (fattr.numRegs < 168) return cudaErrorInvalidConfiguration;
+    }
+#endif
     const int grid = a.n_units < num_sms ? a.n_units : num_sms;
-    kern<<<grid, 384, C::SMEM_BYTES, stream>>>(L.tmQ, L.tmK, L.tmV, a);
+    kern<<<grid, P2_THREADS, C::SMEM_BYTES, stream>>>(L.tmQ, L.tmK, L.tmV, a);
     return cudaGetLastError();
 }
 

@@ -44,10 +44,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # dram__bytes_read.sum + dram__bytes_write.sum per launch from ncu, with the
 # profile summary it comes from; None until a capture of the current kernel.
-NCU_TRAFFIC = {
-    # profiles/paged_decode_kernel_gqa_b64_hq32_hkv8_d128.md
-    "paged_gqa_b64_hq32_hkv8_d128_bs64": 1236590416,
-}
+NCU_TRAFFIC = {}
 
 
 def parse_args():
