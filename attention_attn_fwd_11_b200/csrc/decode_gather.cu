@@ -26,8 +26,9 @@
 //   - warps 0-3 gather 32 selected rows per tile with 16-byte cp.async into
 //     128-byte-swizzled shared memory (4-tile ring); the tile is the K-major
 //     B operand of the partial QK^T and, through its latent columns, the
-//     MN-major B operand of PV; warp 8 issues the MMAs; warps 4-7 run the
-//     exchange, the softmax (one head per thread) and the epilogue, which
+//     MN-major B operand of PV; warp 8 issues the MMAs; warp 9 moves the
+//     partial scores between the pair (one bulk shared-memory copy per tile);
+//     warps 4-7 run the softmax (one head per thread) and the epilogue, which
 //     writes a split partial for the log-sum-exp combine.
 #include <cuda_runtime.h>
 #include <limits.h>
@@ -39,6 +40,17 @@
 namespace fa {
 
 static __device__ int g_gather_err;
+
+#ifdef FA_LG_TRACE
+// Debug-only trace of the first cluster: clock64 stamps in fixed slots
+// [rank][event][tile < 64].
+constexpr int kLgTraceCap = 2 * 16 * 64;
+static __device__ unsigned long long g_lg_trace[kLgTraceCap];
+#define LG_TRACE(ev, i) \
+    do { if (blockIdx.y == 0 && blockIdx.z == 0 && (i) < 64) g_lg_trace[(rank * 16 + (ev)) * 64 + (i)] = clock64(); } while (0)
+#else
+#define LG_TRACE(ev, i) ((void)0)
+#endif
 
 constexpr int LG_DK = 576;
 constexpr int LG_DV = 512;
@@ -52,15 +64,23 @@ constexpr int LG_KCH = LG_BN * 128;              // bytes of one K chunk (4 KB)
 constexpr int LG_KSTAGE = LG_NCH_MAX * LG_KCH;   // 20 KB
 constexpr int LG_XBUF = LG_H * LG_BN * 4;        // one partial-score exchange slot (16 KB)
 constexpr int LG_OFF_K = LG_NCH_MAX * LG_QCH;    // Q: 80 KB
-constexpr int LG_OFF_X = LG_OFF_K + LG_NST * LG_KSTAGE;
-constexpr int LG_OFF_AUX = LG_OFF_X + 2 * LG_XBUF;
+constexpr int LG_OFF_X = LG_OFF_K + LG_NST * LG_KSTAGE;     // xin[2]: the peer's partial scores land here
+constexpr int LG_OFF_XO = LG_OFF_X + 2 * LG_XBUF;            // xout[2]: this CTA's partial scores, sent from here
+constexpr int LG_OFF_AUX = LG_OFF_XO + 2 * LG_XBUF;
 constexpr int LG_SMEM = LG_OFF_AUX + 1024 + 1024;
-constexpr int LG_T_O = 2 * LG_BN;                // TMEM column of O (S0 at 0, S1 at 32)
+#ifndef FA_LG_NSB
+#define FA_LG_NSB 2
+#endif
+// S buffers in TMEM.  2: QK^T of tile i + 1 is issued before PV of tile i.
+// 3: QK^T runs two tiles ahead and the softmax warps hand tile i + 1's
+// partial scores to the exchange before the softmax of tile i.
+constexpr int LG_NSB = FA_LG_NSB;
+constexpr int LG_T_O = LG_NSB * LG_BN;           // TMEM column of O (S buffers at 0, 32, 64)
 static_assert(LG_SMEM <= 232448, "shared memory budget");
 
 enum {
-    G_QFULL = 0, G_SFULL = 1, G_PREADY = 3, G_PVDONE = 5, G_DRAIN = 6, G_XFULL = 7, G_XFREE = 9, G_FULL = 11,
-    G_EMPTY = 11 + LG_NST, G_NBAR = 11 + 2 * LG_NST
+    G_QFULL = 0, G_SFULL = 1, G_PREADY = 4, G_PVDONE = 7, G_DRAIN = 8, G_XFULL = 9, G_XFREE = 11, G_XOREADY = 13,
+    G_XOFREE = 15, G_XREAD = 17, G_FULL = 19, G_EMPTY = 19 + LG_NST, G_NBAR = 19 + 2 * LG_NST
 };
 
 struct GatherArgs {
@@ -74,7 +94,7 @@ struct GatherArgs {
 
 constexpr float kGatherRescaleThreshold = 8.0f;
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(288, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
 latent_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const GatherArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -83,7 +103,7 @@ latent_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const GatherArgs a
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + LG_OFF_AUX);
     const uint32_t bar0 = smem_u32(bars);
     auto bar = [&](int i) -> uint32_t { return bar0 + 8u * (uint32_t)i; };
-    int32_t *rowid = reinterpret_cast<int32_t *>(smem + LG_OFF_AUX + 8 * 32);   // [NST][32]
+    int32_t *rowid = reinterpret_cast<int32_t *>(smem + LG_OFF_AUX + 8 * 40);   // [NST][32]
     uint32_t *maskw = reinterpret_cast<uint32_t *>(rowid + LG_NST * LG_BN);     // [NST]
     uint32_t *tmem_holder = maskw + LG_NST;
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
@@ -104,11 +124,16 @@ latent_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const GatherArgs a
         mbar_init(bar(G_QFULL), 1);
         mbar_init(bar(G_PVDONE), 1);
         mbar_init(bar(G_DRAIN), 1);
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < LG_NSB; ++i) {
             mbar_init(bar(G_SFULL + i), 1);
             mbar_init(bar(G_PREADY + i), 128);
-            mbar_init(bar(G_XFULL + i), 128);  // the peer's 128 softmax threads
-            mbar_init(bar(G_XFREE + i), 128);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(bar(G_XFULL + i), 1);    // own arrive.expect_tx + the peer's bulk copy bytes
+            mbar_init(bar(G_XFREE + i), 1);    // one remote arrive from the peer's exchange thread
+            mbar_init(bar(G_XOREADY + i), 128);  // softmax threads: partial scores are in xout
+            mbar_init(bar(G_XOFREE + i), 1);   // exchange thread: xout has been copied out
+            mbar_init(bar(G_XREAD + i), 128);  // softmax threads: xin has been read
         }
         for (int s = 0; s < LG_NST; ++s) {
             mbar_init(bar(G_FULL + s), 128);
@@ -144,34 +169,11 @@ latent_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const GatherArgs a
             const int pieces_per_row = nch * 8;
             const int n_pieces = LG_BN * pieces_per_row;  // 1280 or 1024: a multiple of 128
             bool ok = true;
-            int sig = 0;  // next tile whose arrival is still to be signalled
-            // A tile is signalled once this thread's copies for it have landed
-            // (wait_group), made visible to the tensor core's async proxy
-            // (fence.proxy.async), then counted on the tile's full barrier.
-            // (wait_group<N> returns once at most N of this thread's most
-            // recent copy groups are still pending; one group per tile.)
-            // Signalling each tile as soon as the next one is issued measured
-            // faster than keeping more tiles unsignalled in flight: the MMA
-            // needs tile i + 1 right after tile i.
-            auto signal_through = [&](int last, bool leave_newest) {
-                while (sig <= last) {
-                    if (leave_newest)
-                        cp_async_wait<1>();
-                    else
-                        cp_async_wait<0>();
-                    fence_proxy_async_smem();
-                    mbar_arrive(bar(G_FULL + sig % LG_NST));
-                    ++sig;
-                }
-            };
             for (int i = 0; i < n_tiles; ++i) {
                 const int s = i % LG_NST;
-                // Stage s is freed by PV of tile i - NST, which the MMA issues
-                // only after QK^T of tile i - NST + 1; every tile up to i - 2
-                // was signalled at the end of the previous iteration, so this
-                // wait cannot deadlock.
-                // One thread waits for the stage to be free and publishes the
-                // outcome, so all 128 gatherers take the same branch below.
+                // One thread waits for the stage to be free (PV of tile i - NST
+                // has read it) and publishes the outcome, so all 128 gatherers
+                // take the same branch below.
                 if (tid == 0)
                     *go = mbar_wait(bar(G_EMPTY + s), ((uint32_t)(i / LG_NST) & 1u) ^ 1u, abort_flag, &g_gather_err);
                 if (warp == 0) {
@@ -208,14 +210,14 @@ latent_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const GatherArgs a
                         a.rows + (int64_t)rowid[s * LG_BN + row] * a.row_stride + chunk0 * 64 + pc * 8;
                     cp_async16(dst0 + c * LG_KCH + row * 128 + ((sub ^ (row & 7)) << 4), src);
                 }
-                cp_async_commit();
-                // Tiles up to i - 2 are signalled while i - 1 and i stay in flight.
-                if (i >= 1) signal_through(i - 1, true);
+                // The tile's full barrier gets this thread's arrival when its
+                // copies have landed; consumers fence into the async proxy
+                // after waiting on it.  Nothing here blocks, so up to NST
+                // tiles are in flight.
+                cp_async_arrive_noinc(bar(G_FULL + s));
+                if (tid == 0) LG_TRACE(0, i);
             }
-            if (ok)
-                signal_through(n_tiles - 1, false);
-            else
-                cp_async_wait<0>();
+            cp_async_wait<0>();
             if (tid == 0 && *abort_flag) mbar_wait_drain(bar(G_QFULL), 0);
         }
     } else if (warp == 8) {
@@ -227,24 +229,30 @@ latent_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const GatherArgs a
             auto issue_qk = [&](int i) -> bool {
                 const int s = i % LG_NST;
                 if (!mbar_wait(bar(G_FULL + s), (uint32_t)(i / LG_NST) & 1u, abort_flag, &g_gather_err)) return false;
+                fence_proxy_async_smem();  // the gathered rows were written by cp.async (generic proxy)
                 tc_fence_after();
-                const uint32_t tS = tmem + (uint32_t)((i & 1) * LG_BN);
+                const uint32_t tS = tmem + (uint32_t)((i % LG_NSB) * LG_BN);
                 for (int kk = 0; kk < nch * 4; ++kk) {
                     const int c = kk >> 2, sub = kk & 3;
                     const uint64_t ad = sdesc_sw128(sQ + c * LG_QCH + sub * 32, 16, 1024);
                     const uint64_t bd = sdesc_sw128(sK + s * LG_KSTAGE + c * LG_KCH + sub * 32, 16, 1024);
                     mma_ss(tS, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
                 }
-                mma_commit(bar(G_SFULL + (i & 1)));
+                mma_commit(bar(G_SFULL + i % LG_NSB));
+                LG_TRACE(2, i);
                 return true;
             };
-            bool ok = mbar_wait(bar(G_QFULL), 0, abort_flag, &g_gather_err) && issue_qk(0);
+            // QK^T runs NSB - 1 tiles ahead of PV: S buffer (i + NSB - 1) % NSB
+            // held P of tile i - 1, which PV(i - 1) (issued before) consumed.
+            bool ok = mbar_wait(bar(G_QFULL), 0, abort_flag, &g_gather_err);
+            for (int j = 0; ok && j < LG_NSB - 1 && j < n_tiles; ++j) ok = issue_qk(j);
             for (int i = 0; ok && i < n_tiles; ++i) {
-                if (i + 1 < n_tiles && !issue_qk(i + 1)) break;
-                if (!mbar_wait(bar(G_PREADY + (i & 1)), (uint32_t)(i >> 1) & 1u, abort_flag, &g_gather_err)) break;
+                if (i + LG_NSB - 1 < n_tiles && !issue_qk(i + LG_NSB - 1)) break;
+                if (!mbar_wait(bar(G_PREADY + i % LG_NSB), (uint32_t)(i / LG_NSB) & 1u, abort_flag, &g_gather_err))
+                    break;
                 tc_fence_after();
                 const int s = i % LG_NST;
-                const uint32_t tP = tmem + (uint32_t)((i & 1) * LG_BN);
+                const uint32_t tP = tmem + (uint32_t)((i % LG_NSB) * LG_BN);
 #pragma unroll
                 for (int kk = 0; kk < LG_BN / 16; ++kk) {
                     const uint64_t bd = sdesc_sw128(sK + s * LG_KSTAGE + vch * LG_KCH + kk * 2048, LG_KCH, 1024);
@@ -252,9 +260,40 @@ latent_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const GatherArgs a
                 }
                 mma_commit(bar(G_EMPTY + s));
                 mma_commit(bar(G_PVDONE));
+                LG_TRACE(3, i);
             }
             mma_commit(bar(G_DRAIN));
             mbar_wait_drain(bar(G_DRAIN), 0);
+        }
+        __syncwarp();
+    } else if (warp == 9) {
+        if (lane == 0 && n_tiles > 0) {
+            // ------------------------- partial-score exchange thread --
+            // Per tile: once this CTA's partial scores are in xout and the
+            // peer has released its xin slot, one bulk copy moves the 16 KB
+            // slot into the peer's xin and completes on the peer's xfull;
+            // once the local softmax has read its own xin, the peer is told
+            // it may refill that slot.
+            const uint32_t sXO = sbase + LG_OFF_XO;
+            const uint32_t peer_xin = map_to_rank(sX, peer);
+            const uint32_t peer_xfull = map_to_rank(bar(G_XFULL), peer);
+            const uint32_t peer_xfree = map_to_rank(bar(G_XFREE), peer);
+            for (int i = 0; i < n_tiles; ++i) {
+                const int buf = i & 1;
+                const uint32_t ph = (uint32_t)(i >> 1) & 1u;
+                if (!mbar_wait(bar(G_XOREADY + buf), ph, abort_flag, &g_gather_err) ||
+                    !mbar_wait_cluster(bar(G_XFREE + buf), ph ^ 1u, abort_flag, &g_gather_err))
+                    break;
+                mbar_arrive_expect_tx(bar(G_XFULL + buf), LG_XBUF);  // arm for the peer's copy
+                bulk_copy_to_peer(peer_xin + (uint32_t)(buf * LG_XBUF), sXO + (uint32_t)(buf * LG_XBUF), LG_XBUF,
+                                  peer_xfull + 8u * (uint32_t)buf);
+                bulk_commit();
+                bulk_wait_read0();
+                mbar_arrive(bar(G_XOFREE + buf));
+                if (!mbar_wait(bar(G_XREAD + buf), ph, abort_flag, &g_gather_err)) break;
+                mbar_arrive_cluster(peer_xfree + 8u * (uint32_t)buf);
+            }
+            bulk_wait0();  // every copy into the peer has landed before this CTA can finish
         }
         __syncwarp();
     } else {
@@ -263,44 +302,54 @@ latent_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const GatherArgs a
         const int head = qd * 32 + lane;
         const uint32_t tl = tmem + ((uint32_t)(qd * 32) << 16);
         const float c = a.scale_log2;
-        // Exchange slot of this head: 8 pieces of 16 bytes, swizzled by head.
-        const uint32_t my_x = sX + (uint32_t)head * 128u;
-        const uint32_t peer_x = map_to_rank(my_x, peer);
-        const uint32_t peer_xfull = map_to_rank(bar(G_XFULL), peer);
-        const uint32_t peer_xfree = map_to_rank(bar(G_XFREE), peer);
+        // Exchange: each head's 32 partial scores are 8 pieces of 16 bytes,
+        // swizzled by head, written to xout; the exchange thread (warp 8)
+        // moves the slot to the peer, whose scores arrive in xin.
         // l_run: sum of the fp32 weights (gives the LSE); l_mma: sum of the
         // bf16-rounded weights the PV MMA uses (normalises O, so a one-hot
         // softmax returns its V row exactly).
         float m_run = -INFINITY, l_run = 0.f, l_mma = 0.f;
-        bool ok = true;
-        for (int i = 0; i < n_tiles; ++i) {
-            const int buf = i & 1, s = i % LG_NST;
-            const uint32_t ph = (uint32_t)(i >> 1) & 1u;
-            if (!mbar_wait(bar(G_SFULL + buf), ph, abort_flag, &g_gather_err) ||
-                !mbar_wait(bar(G_FULL + s), (uint32_t)(i / LG_NST) & 1u, abort_flag, &g_gather_err)) {
-                ok = false;
-                break;
-            }
+        // Software pipeline: the partial scores of tile i + 1 are loaded and
+        // handed to the exchange before the softmax of tile i runs, so the
+        // pair's exchange latency overlaps the previous tile's softmax.
+        auto send = [&](int j, uint32_t (&r)[32]) -> bool {
+            const int jb = j & 1;  // exchange slot
+            const uint32_t jph = (uint32_t)(j >> 1) & 1u;
+            if (!mbar_wait(bar(G_SFULL + j % LG_NSB), (uint32_t)(j / LG_NSB) & 1u, abort_flag, &g_gather_err))
+                return false;
+            if (head == 0) LG_TRACE(4, j);
             tc_fence_after();
-            uint32_t r[32];
-            tmem_ld32(tl + (uint32_t)(buf * LG_BN), r);
+            tmem_ld32(tl + (uint32_t)((j % LG_NSB) * LG_BN), r);
             tmem_wait_ld();
             reg_fence(r);
-            // Send this CTA's partial scores to the peer, once the peer has
-            // read what was sent through this slot two tiles ago.
-            if (!mbar_wait(bar(G_XFREE + buf), ph ^ 1u, abort_flag, &g_gather_err)) {
-                ok = false;
-                break;
-            }
+            if (head == 0) LG_TRACE(8, j);
+            // xout[jb] is reusable once the exchange thread copied it out (two tiles ago)
+            if (!mbar_wait(bar(G_XOFREE + jb), jph ^ 1u, abort_flag, &g_gather_err)) return false;
 #pragma unroll
             for (int k = 0; k < 8; ++k)
-                st_cluster_v4(peer_x + (uint32_t)(buf * LG_XBUF) + (uint32_t)((k ^ (head & 7)) << 4), r[4 * k],
-                              r[4 * k + 1], r[4 * k + 2], r[4 * k + 3]);
-            mbar_arrive_cluster(peer_xfull + 8u * (uint32_t)buf);
-            if (!mbar_wait_cluster(bar(G_XFULL + buf), ph, abort_flag, &g_gather_err)) {
+                *reinterpret_cast<uint4 *>(smem + LG_OFF_XO + jb * LG_XBUF + head * 128 + ((k ^ (head & 7)) << 4)) =
+                    make_uint4(r[4 * k], r[4 * k + 1], r[4 * k + 2], r[4 * k + 3]);
+            fence_proxy_async_smem();  // generic stores -> visible to the bulk copy
+            mbar_arrive(bar(G_XOREADY + jb));
+            if (head == 0) LG_TRACE(5, j);
+            return true;
+        };
+        uint32_t r[32], rn[32];
+        constexpr bool kPipe = LG_NSB >= 3;
+        bool ok = !kPipe || n_tiles == 0 || send(0, r);
+        for (int i = 0; ok && i < n_tiles; ++i) {
+            const int buf = i & 1, s = i % LG_NST;
+            const uint32_t ph = (uint32_t)(i >> 1) & 1u;
+            if (kPipe ? (i + 1 < n_tiles && !send(i + 1, rn)) : !send(i, r)) {
                 ok = false;
                 break;
             }
+            if (!mbar_wait(bar(G_FULL + s), (uint32_t)(i / LG_NST) & 1u, abort_flag, &g_gather_err) ||
+                !mbar_wait_cluster(bar(G_XFULL + buf), ph, abort_flag, &g_gather_err)) {
+                ok = false;
+                break;
+            }
+            if (head == 0) LG_TRACE(6, i);
             const uint4 *xin = reinterpret_cast<const uint4 *>(smem + LG_OFF_X + buf * LG_XBUF + head * 128);
             float x[32];
             const uint32_t mask = maskw[s];
@@ -316,7 +365,12 @@ latent_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const GatherArgs a
                 x[4 * k + 2] = ((mask >> (4 * k + 2)) & 1u) ? v2 : -INFINITY;
                 x[4 * k + 3] = ((mask >> (4 * k + 3)) & 1u) ? v3 : -INFINITY;
             }
-            mbar_arrive_cluster(peer_xfree + 8u * (uint32_t)buf);  // my slot may be refilled
+            if (kPipe) {
+#pragma unroll
+                for (int k = 0; k < 32; ++k) r[k] = rn[k];  // the next tile's partial scores
+            }
+            mbar_arrive(bar(G_XREAD + buf));  // xin[buf] read: the exchange thread releases it to the peer
+            if (head == 0) LG_TRACE(10, i);
             float mx0 = x[0], mx1 = x[1];
 #pragma unroll
             for (int k = 2; k < 32; k += 2) {
@@ -350,6 +404,7 @@ latent_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const GatherArgs a
                     tmem_st32(tl + (uint32_t)(LG_T_O + ch * 32), o);
                 }
             }
+            if (head == 0) LG_TRACE(11, i);
             const float msub = (m_run == -INFINITY) ? 0.f : m_run;
             uint32_t pk[16];
             float s0 = 0.f, s1 = 0.f, q0 = 0.f, q1 = 0.f;
@@ -365,10 +420,11 @@ latent_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const GatherArgs a
             }
             l_run += s0 + s1;
             l_mma += q0 + q1;
-            tmem_st16(tl + (uint32_t)(buf * LG_BN), pk);
+            tmem_st16(tl + (uint32_t)((i % LG_NSB) * LG_BN), pk);
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(bar(G_PREADY + buf));
+            mbar_arrive(bar(G_PREADY + i % LG_NSB));
+            if (head == 0) LG_TRACE(7, i);
         }
         bool have_o = ok && n_tiles > 0;
         if (have_o) {
@@ -428,12 +484,22 @@ cudaError_t launch_decode_gather(const GatherLaunch &L, cudaStream_t stream) {
     a.part_o = L.part_o;
     a.part_lse = L.part_lse;
     dim3 grid(2u, (unsigned)L.num_splits, (unsigned)L.T);
-    latent_decode_kernel<<<grid, 288, LG_SMEM, stream>>>(L.tmQ, a);
+    latent_decode_kernel<<<grid, 320, LG_SMEM, stream>>>(L.tmQ, a);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     return launch_combine(L.part_o, L.part_lse, L.T * L.Hq, L.num_splits, L.Hq, nullptr, 0, L.o, L.lse, L.o_bf16,
                           LG_DV, stream);
 }
+
+#ifdef FA_LG_TRACE
+}  // namespace fa
+extern "C" int fa_debug_lg_trace_read(unsigned long long *host, int cap) {
+    int n = cap < fa::kLgTraceCap ? cap : fa::kLgTraceCap;
+    cudaMemcpyFromSymbol(host, fa::g_lg_trace, n * sizeof(unsigned long long));
+    return n;
+}
+namespace fa {
+#endif
 
 cudaError_t gather_device_error(int clear, int *code) {
     int v = 0;

@@ -38,6 +38,22 @@ namespace fa {
 
 static __device__ int g_prefill2_err;
 
+#ifdef FA_P2_TRACE
+// Debug-only event trace of CTA 0's first unit: clock64 stamps stored to
+// fixed slots [event][tile t < 64][sub < 8] (plain stores, so tracing does
+// not stall the warp), read back by fa_debug_trace_read.
+constexpr int kTraceCap = 32 * 64 * 8;
+static __device__ unsigned long long g_trace[kTraceCap];
+static __device__ unsigned int g_trace_n;
+FA_DEV void trace(int ev, int t, int sub, int uc) {
+    if (blockIdx.x != 0 || uc != 0 || t >= 64 || ev >= 32) return;
+    g_trace[(ev * 64 + t) * 8 + sub] = clock64();
+}
+#define TRACE(ev, t, sub) trace(ev, t, sub, uc)
+#else
+#define TRACE(ev, t, sub) ((void)0)
+#endif
+
 struct Prefill2Args {
     int Hq, group, Sq, Sk, BH, n_qp, n_units;
     float scale_log2;
@@ -75,10 +91,39 @@ struct P2Cfg {
 
 enum {
     P2_QFULL = 0, P2_QEMPTY = 1, P2_SFULL = 2, P2_PREADY = 4, P2_ODONE = 6, P2_OFREE = 8, P2_USTART = 10,
-    P2_DRAIN = 12, P2_RING = 13
+    P2_DRAIN = 12, P2_SFREE = 13, P2_RING = 15
 };
 
+// FA_P2_HOIST: the softmax signals as soon as S is in registers, and the
+// MMA issues the upper half of the next QK^T (keys 64..127, TMEM columns
+// that P does not use) before the current PV; only the lower half stays
+// between PV and the next softmax.
+#ifndef FA_P2_HOIST
+#define FA_P2_HOIST 0
+#endif
+
 constexpr float kP2RescaleThreshold = 8.0f;
+
+// FA_P2_SPIN: the MMA thread polls the P-ready barriers (lower wake-up
+// latency on the critical path).
+#ifndef FA_P2_SPIN
+#define FA_P2_SPIN 0
+#endif
+#if FA_P2_SPIN
+#define P2_MMA_WAIT mbar_wait_spin
+#else
+#define P2_MMA_WAIT mbar_wait
+#endif
+// FA_P2_MAXCHAINS: independent three-input-max chains in the row max (4 or 8).
+#ifndef FA_P2_MAXCHAINS
+#define FA_P2_MAXCHAINS 4
+#endif
+
+// FA_P2_PACKED: the softmax uses the packed f32x2 FMA/ADD and three-input
+// max instructions (fewer issue slots per element).
+#ifndef FA_P2_PACKED
+#define FA_P2_PACKED 1
+#endif
 
 // Every FA_EXP2_POLY_EVERY-th pair of softmax elements takes 2^x on the FMA
 // pipe (ex2_poly) instead of the MUFU unit, which the two softmax
@@ -164,6 +209,7 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             mbar_init(bar(P2_ODONE + i), 1);
             mbar_init(bar(P2_OFREE + i), 128);
             mbar_init(bar(P2_USTART + i), 1);
+            mbar_init(bar(P2_SFREE + i), 128);
         }
         for (int s = 0; s < NSTK; ++s) {
             mbar_init(k_full(s), 1);
@@ -224,6 +270,7 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                         ok = false;
                         break;
                     }
+                    TRACE(1, t, 0);
                     mbar_arrive_expect_tx(k_full(sk), C::KV_BYTES);
 #pragma unroll
                     for (int c = 0; c < C::NCH; ++c)
@@ -232,6 +279,7 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                         ok = false;
                         break;
                     }
+                    TRACE(2, t, 0);
                     mbar_arrive_expect_tx(v_full(sv), C::KV_BYTES);
 #pragma unroll
                     for (int c = 0; c < C::NCH; ++c)
@@ -264,6 +312,20 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 }
                 mma_commit(bar(P2_SFULL + i));
             };
+            // Half of QK^T: keys [64 h, 64 h + 64) of the K tile into TMEM
+            // columns [64 h, 64 h + 64) of S_i.
+            auto qk_half = [&](int i, int s, int h) {
+                constexpr uint32_t idesc_half = idesc_bf16_f32(128, BN / 2, false, false);
+                const uint32_t tS = tmem + (uint32_t)(i * BN + h * (BN / 2));
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const int c = kk >> 2, sub = kk & 3;
+                    const uint64_t ad = sdesc_sw128(sQ + i * C::Q_TILE + c * C::Q_CHUNK + sub * 32, 16, 1024);
+                    const uint64_t bd = sdesc_sw128(
+                        sK + s * C::KV_BYTES + c * C::KV_CHUNK + h * (BN / 2) * 128 + sub * 32, 16, 1024);
+                    mma_ss(tS, ad, bd, idesc_half, kk > 0 ? 1u : 0u);
+                }
+            };
             auto pv = [&](int i, int s, bool first) {
                 const uint32_t tO = tmem + (uint32_t)(C::T_O + i * D);
                 const uint32_t tP = tmem + (uint32_t)(i * BN);
@@ -276,6 +338,7 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             };
             int kc = 0, uc = 0;
             int pcnt[2] = {0, 0};
+            int fcnt[2] = {0, 0};  // S-free phases consumed (hoisting only)
             bool ok = true;
             UnitInfo u;
             for (int r = 0; ok && p2_unit(a, r, u); ++r, ++uc) {
@@ -309,37 +372,82 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                     const bool has_next = t + 1 < u.N;
                     const int s1 = (kt + 1) % NSTK;  // K stage of tile t + 1
                     bool v_ready = false;
+#if FA_P2_HOIST
+                    if (has_next) {
+                        if (!mbar_wait(k_full(s1), (uint32_t)((kt + 1) / NSTK) & 1u, abort_flag, &g_prefill2_err)) {
+                            ok = false;
+                            break;
+                        }
+                    }
+                    // Every S-free phase is consumed; while there is a next tile the
+                    // upper half of its QK^T goes ahead of this tile's PV.
+                    for (int i = 0; ok && i < 2; ++i) {
+                        if (t >= u.n[i]) continue;
+                        if (!P2_MMA_WAIT(bar(P2_SFREE + i), (uint32_t)fcnt[i] & 1u, abort_flag, &g_prefill2_err)) {
+                            ok = false;
+                            break;
+                        }
+                        ++fcnt[i];
+                        if (has_next && t + 1 < u.n[i]) {
+                            tc_fence_after();
+                            qk_half(i, s1, 1);
+                        }
+                    }
+                    if (!ok) break;
+#endif
                     if (t < u.n[0]) {
-                        if (!mbar_wait(bar(P2_PREADY + 0), (uint32_t)pcnt[0] & 1u, abort_flag, &g_prefill2_err) ||
+                        if (!P2_MMA_WAIT(bar(P2_PREADY + 0), (uint32_t)pcnt[0] & 1u, abort_flag, &g_prefill2_err) ||
                             !mbar_wait(v_full(s), (uint32_t)(kt / NSTV) & 1u, abort_flag, &g_prefill2_err)) {
                             ok = false;
                             break;
                         }
                         ++pcnt[0];
                         v_ready = true;
+                        TRACE(3, t, 0);
                         tc_fence_after();
                         pv(0, s, t == 0);
+                        TRACE(5, t, 0);
                     }
                     if (has_next) {
+#if !FA_P2_HOIST
                         if (!mbar_wait(k_full(s1), (uint32_t)((kt + 1) / NSTK) & 1u, abort_flag, &g_prefill2_err)) {
                             ok = false;
                             break;
                         }
+#endif
                         tc_fence_after();
-                        if (t + 1 < u.n[0]) qk(0, s1);
+                        if (t + 1 < u.n[0]) {
+#if FA_P2_HOIST
+                            qk_half(0, s1, 0);
+                            mma_commit(bar(P2_SFULL + 0));
+#else
+                            qk(0, s1);
+#endif
+                            TRACE(7, t + 1, 0);
+                        }
                     }
                     if (t < u.n[1]) {
-                        if (!mbar_wait(bar(P2_PREADY + 1), (uint32_t)pcnt[1] & 1u, abort_flag, &g_prefill2_err) ||
+                        if (!P2_MMA_WAIT(bar(P2_PREADY + 1), (uint32_t)pcnt[1] & 1u, abort_flag, &g_prefill2_err) ||
                             (!v_ready &&
                              !mbar_wait(v_full(s), (uint32_t)(kt / NSTV) & 1u, abort_flag, &g_prefill2_err))) {
                             ok = false;
                             break;
                         }
                         ++pcnt[1];
+                        TRACE(4, t, 0);
                         tc_fence_after();
                         pv(1, s, t == 0);
+                        TRACE(6, t, 0);
                     }
-                    if (has_next && t + 1 < u.n[1]) qk(1, s1);
+                    if (has_next && t + 1 < u.n[1]) {
+#if FA_P2_HOIST
+                        qk_half(1, s1, 0);
+                        mma_commit(bar(P2_SFULL + 1));
+#else
+                        qk(1, s1);
+#endif
+                        TRACE(8, t + 1, 0);
+                    }
                     mma_commit(v_empty(s));
                     if (has_next) {
                         mma_commit(k_empty(s1));
@@ -378,6 +486,7 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                     break;
                 }
                 ++scnt;
+                if (lane == 0) TRACE(9 + ti, t, qd);
                 tc_fence_after();
                 float x[BN];
                 {
@@ -390,12 +499,44 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 #pragma unroll
                     for (int k = 0; k < BN; ++k) x[k] = __uint_as_float(rr[k]);
                 }
+#if FA_P2_HOIST
+                tc_fence_before();
+                mbar_arrive(bar(P2_SFREE + ti));  // S is in registers: its upper half may be overwritten
+#endif
+                if (lane == 0) TRACE(11 + ti, t, qd);
                 const int lim = lim_all - t * BN;
                 if (lim < BN) {
 #pragma unroll
                     for (int k = 0; k < BN; ++k)
                         if (k >= lim) x[k] = -INFINITY;
                 }
+#if FA_P2_PACKED
+                // four independent chains of three-input maxima
+                static_assert(BN % 16 == 0, "tile width");
+#if FA_P2_MAXCHAINS == 8
+                float mc[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) mc[j] = x[j];
+#pragma unroll
+                for (int k = 8; k < BN; k += 16)  // x[8 .. BN-1], two per chain per step
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) mc[j] = fmax3(mc[j], x[k + 2 * j], x[k + 2 * j + 1]);
+                const float m_tile = fmax3(fmax3(mc[0], mc[1], mc[2]), fmax3(mc[3], mc[4], mc[5]), fmaxf(mc[6], mc[7])) * c;
+#else
+                float mx0 = x[0], mx1 = x[1], mx2 = x[2], mx3 = x[3];
+#pragma unroll
+                for (int k = 4; k + 8 <= BN; k += 8) {  // x[4 .. BN-5]
+                    mx0 = fmax3(mx0, x[k], x[k + 1]);
+                    mx1 = fmax3(mx1, x[k + 2], x[k + 3]);
+                    mx2 = fmax3(mx2, x[k + 4], x[k + 5]);
+                    mx3 = fmax3(mx3, x[k + 6], x[k + 7]);
+                }
+                mx0 = fmax3(mx0, x[BN - 4], x[BN - 3]);  // the last four
+                mx1 = fmax3(mx1, x[BN - 2], x[BN - 1]);
+                const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * c;
+#endif
+                if (lane == 0) TRACE(19 + ti, t, qd);
+#else
                 float mx0 = x[0], mx1 = x[1], mx2 = x[2], mx3 = x[3];
 #pragma unroll
                 for (int k = 4; k < BN; k += 4) {
@@ -405,6 +546,7 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                     mx3 = fmaxf(mx3, x[k + 3]);
                 }
                 const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * c;
+#endif
                 const float m_new = fmaxf(m_run, m_tile);
                 const bool need = m_new > m_run + kP2RescaleThreshold;
                 float alpha = 1.f;
@@ -433,6 +575,46 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 }
                 const bool empty_row = m_run == -INFINITY;  // no visible key so far: P = 0
                 const float msub = empty_row ? 0.f : m_run;
+#if FA_P2_PACKED
+                // p = 2^(x * c - m) on pairs: one f32x2 FMA per pair, two MUFU
+                // ex2, one bf16x2 convert; the row sum in two packed
+                // accumulators (one f32x2 add per pair).
+                {
+                    const uint64_t c2 = f2_pack(c, c);
+                    const uint64_t nm2 = f2_pack(-msub, -msub);
+                    uint64_t acc0 = f2_pack(0.f, 0.f), acc1 = acc0;
+#pragma unroll
+                    for (int g = 0; g < BN / 32; ++g) {
+                        uint32_t pk[16];
+#pragma unroll
+                        for (int k = 0; k < 16; ++k) {
+                            float a0, a1;
+                            f2_unpack(f2_fma(f2_pack(x[g * 32 + 2 * k], x[g * 32 + 2 * k + 1]), c2, nm2), a0, a1);
+                            float p0, p1;
+                            if (FA_EXP2_POLY_EVERY > 0 &&
+                                (k % (FA_EXP2_POLY_EVERY > 0 ? FA_EXP2_POLY_EVERY : 1)) ==
+                                    (FA_EXP2_POLY_EVERY > 0 ? FA_EXP2_POLY_EVERY - 1 : 0)) {
+                                ex2_poly2(a0, a1, p0, p1);
+                                if (empty_row) p0 = p1 = 0.f;
+                            } else {
+                                p0 = ex2(a0);
+                                p1 = ex2(a1);
+                            }
+                            if (k & 1)
+                                acc1 = f2_add(acc1, f2_pack(p0, p1));
+                            else
+                                acc0 = f2_add(acc0, f2_pack(p0, p1));
+                            pk[k] = pack_bf16x2(p0, p1);
+                        }
+                        tmem_st16(tS + (uint32_t)(g * 16), pk);
+                    }
+                    if (lane == 0) TRACE(21 + ti, t, qd);
+                    float u0, u1, u2, u3;
+                    f2_unpack(acc0, u0, u1);
+                    f2_unpack(acc1, u2, u3);
+                    l_run += (u0 + u1) + (u2 + u3);
+                }
+#else
                 float s0 = 0.f, s1 = 0.f;
 #pragma unroll
                 for (int g = 0; g < BN / 32; ++g) {
@@ -457,11 +639,14 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                     tmem_st16(tS + (uint32_t)(g * 16), pk);
                 }
                 l_run += s0 + s1;
+#endif
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(bar(P2_PREADY + ti));
+                if (lane == 0) TRACE(13 + ti, t, qd);
             }
             // ---- epilogue ----
+            if (row == 0) TRACE(15 + ti, 0, 0);
             bool have_o = ok && n > 0;
             if (have_o) {
                 if (mbar_wait(bar(P2_ODONE + ti), (uint32_t)(pv_base + n - 1) & 1u, abort_flag, &g_prefill2_err))
@@ -510,6 +695,7 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 a.lse[((int64_t)u.b * a.Hq + u.hq) * a.Sq + qrow] =
                     (l_run > 0.f) ? (m_run + __log2f(l_run)) * 0.69314718055994530942f : -INFINITY;
             // O of this tile has been read out: the next unit may overwrite it.
+            if (row == 0) TRACE(17 + ti, 0, 0);
             tc_fence_before();
             mbar_arrive(bar(P2_OFREE + ti));
         }
@@ -566,6 +752,16 @@ cudaError_t launch_prefill2(const PrefillLaunch &L, int num_sms, cudaStream_t st
         default: return cudaErrorInvalidValue;
     }
 }
+
+#ifdef FA_P2_TRACE
+}  // namespace fa
+extern "C" int fa_debug_trace_read(unsigned long long *host, int cap) {
+    int n = cap < fa::kTraceCap ? cap : fa::kTraceCap;
+    cudaMemcpyFromSymbol(host, fa::g_trace, n * sizeof(unsigned long long));
+    return n;
+}
+namespace fa {
+#endif
 
 cudaError_t prefill2_device_error(int clear, int *code) {
     int v = 0;

@@ -82,6 +82,28 @@ FA_DEV bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag, i
     }
 }
 
+FA_DEV bool mbar_test(uint32_t bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
+// Bounded wait that polls with test_wait (no suspend) for the first few
+// thousand iterations: lower wake-up latency for a thread on the critical
+// path, then the usual bounded try_wait loop.
+FA_DEV bool mbar_wait_spin(uint32_t bar, uint32_t parity, volatile int *abort_flag, int *err) {
+#pragma unroll 1
+    for (int i = 0; i < 4096; ++i)
+        if (mbar_test(bar, parity)) return true;
+    return mbar_wait(bar, parity, abort_flag, err);
+}
+
 // Bounded wait used only while draining after an abort: no abort flag, no
 // error latch; gives up silently after kWaitLimitNs.
 FA_DEV bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
@@ -150,6 +172,22 @@ FA_DEV bool mbar_wait_cluster(uint32_t bar, uint32_t parity, volatile int *abort
     }
 }
 
+// Bulk copy of `bytes` from this CTA's shared memory to another CTA's
+// shared memory in the cluster (dst and the mbarrier are shared::cluster
+// addresses); completion is counted in bytes on that (remote) mbarrier.
+FA_DEV void bulk_copy_to_peer(uint32_t dst_cluster, uint32_t src_cta, uint32_t bytes, uint32_t remote_bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            dst_cluster),
+        "r"(src_cta), "r"(bytes), "r"(remote_bar)
+        : "memory");
+}
+FA_DEV void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Waits until every committed bulk copy of this thread has finished READING its source.
+FA_DEV void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// Waits until every committed bulk copy of this thread has completed.
+FA_DEV void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // ------------------------------------------------------------------ TMA --
 
 FA_DEV void prefetch_tmap(const CUtensorMap *m) {
@@ -181,6 +219,11 @@ FA_DEV void cp_async16(uint32_t dst, const void *src) {
                  : "memory");
 }
 FA_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// The mbarrier receives one arrival (counted against its expected count)
+// once every cp.async this thread issued so far has completed.
+FA_DEV void cp_async_arrive_noinc(uint32_t bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
 template <int N>
 FA_DEV void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
@@ -364,6 +407,57 @@ FA_DEV float ex2_poly(float x) {
     const float f = x - (t - 12582912.f);
     const float p = fmaf(fmaf(fmaf(0.0551716685f, f, 0.2426111251f), f, 0.6932609677f), f, 0.9999280572f);
     return __int_as_float(__float_as_int(p) + __float_as_int(t) * 8388608);
+}
+
+// Packed fp32 pairs (sm_100 f32x2 instructions): one instruction applies the
+// operation to both halves of a 64-bit register pair.
+FA_DEV uint64_t f2_pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+FA_DEV void f2_unpack(uint64_t v, float &lo, float &hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+FA_DEV uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+FA_DEV uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+FA_DEV uint64_t f2_mul(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+// Three-input maximum (one instruction).
+FA_DEV float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// ex2_poly on a packed pair, with the f32x2 instructions where they exist.
+FA_DEV void ex2_poly2(float a0, float a1, float &p0, float &p1) {
+    a0 = fmaxf(a0, -126.f);
+    a1 = fmaxf(a1, -126.f);
+    const uint64_t magic = f2_pack(12582912.f, 12582912.f);
+    const uint64_t nmagic = f2_pack(-12582912.f, -12582912.f);
+    const uint64_t x = f2_pack(a0, a1);
+    const uint64_t t = f2_add(x, magic);
+    const uint64_t f = f2_add(x, f2_mul(f2_add(t, nmagic), f2_pack(-1.f, -1.f)));
+    uint64_t q = f2_fma(f2_pack(0.0551716685f, 0.0551716685f), f, f2_pack(0.2426111251f, 0.2426111251f));
+    q = f2_fma(q, f, f2_pack(0.6932609677f, 0.6932609677f));
+    q = f2_fma(q, f, f2_pack(0.9999280572f, 0.9999280572f));
+    float q0, q1, t0, t1;
+    f2_unpack(q, q0, q1);
+    f2_unpack(t, t0, t1);
+    p0 = __int_as_float(__float_as_int(q0) + __float_as_int(t0) * 8388608);
+    p1 = __int_as_float(__float_as_int(q1) + __float_as_int(t1) * 8388608);
 }
 
 FA_DEV uint32_t pack_bf16x2(float lo, float hi) {
