@@ -42,12 +42,15 @@ static __device__ int g_prefill2_err;
 // Debug-only event trace of CTA 0's first unit: clock64 stamps stored to
 // fixed slots [event][tile t < 64][sub < 8] (plain stores, so tracing does
 // not stall the warp), read back by fa_debug_trace_read.
-constexpr int kTraceCap = 32 * 64 * 8;
+#ifndef FA_P2_TRACE_CTA
+#define FA_P2_TRACE_CTA 0
+#endif
+constexpr int kTraceCap = 2 * 32 * 64 * 8;
 static __device__ unsigned long long g_trace[kTraceCap];
 static __device__ unsigned int g_trace_n;
 FA_DEV void trace(int ev, int t, int sub, int uc) {
-    if (blockIdx.x != 0 || uc != 0 || t >= 64 || ev >= 32) return;
-    g_trace[(ev * 64 + t) * 8 + sub] = clock64();
+    if (blockIdx.x != FA_P2_TRACE_CTA || uc >= 2 || t >= 64 || ev >= 32) return;
+    g_trace[((uc * 32 + ev) * 64 + t) * 8 + sub] = clock64();
 }
 #define TRACE(ev, t, sub) trace(ev, t, sub, uc)
 #else

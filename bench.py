@@ -44,7 +44,14 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # dram__bytes_read.sum + dram__bytes_write.sum per launch from ncu, with the
 # profile summary it comes from; None until a capture of the current kernel.
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    # dram__bytes_read.sum + dram__bytes_write.sum of one launch; the summary
+    # under profiles/ named for the kernel and workload gives the capture.
+    "causal_mha_b2_h16_s2048_d128": 54141184,
+    "gqa_full_b1_hq32_hkv8_s4096_d256": 210472960,
+    "paged_gqa_b64_hq32_hkv8_d128_bs64": 1237055008,
+    "latent_sparse_t32_hq128_dk576_dv512_top2048": 45249792,
+}
 
 
 def parse_args():
@@ -183,18 +190,18 @@ def time_graph(torch, launch, n_copies, K, W, dist=None, window=None):
     return ms, K
 
 
-def max_over_ranks(torch, dist, x):
+def max_over_ranks(torch, dist, x, device="cuda"):
     if dist is None:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
 
-def sum_over_ranks(torch, dist, x):
+def sum_over_ranks(torch, dist, x, device="cuda"):
     if dist is None:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.SUM)
     return float(t.item())
 
