@@ -53,7 +53,7 @@ bool get_encoder() {
 // (64, box_rows, 1, 1).  Strides in elements.  Dimensions of extent 1 get a
 // packed stride (their stride is never used).
 fa_status encode_4d(CUtensorMap *m, const void *base, int d, int S, int H, int B, int64_t s_s, int64_t s_h,
-                    int64_t s_b, int box_rows, const char *name) {
+                    int64_t s_b, int box_rows, const char *name, int elem_bytes = 2) {
     cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)(S > 0 ? S : 1), (cuuint64_t)H, (cuuint64_t)B};
     int64_t st[3] = {s_s, s_h, s_b};
     int64_t packed = d;
@@ -63,15 +63,17 @@ fa_status encode_4d(CUtensorMap *m, const void *base, int d, int S, int H, int B
     }
     cuuint64_t strides[3];
     for (int i = 0; i < 3; ++i) {
-        const int64_t bytes = st[i] * 2;
+        const int64_t bytes = st[i] * elem_bytes;
         if (bytes <= 0 || bytes % 16 != 0 || bytes >= (int64_t(1) << 40))
-            return fail(FA_ERR_INVALID_ARG, "%s: stride %d (%lld elements) must be a positive multiple of 8", name,
-                        i, (long long)st[i]);
+            return fail(FA_ERR_INVALID_ARG, "%s: stride %d (%lld elements) must be a positive multiple of %d", name,
+                        i, (long long)st[i], 16 / elem_bytes);
         strides[i] = (cuuint64_t)bytes;
     }
-    cuuint32_t box[4] = {64u, (cuuint32_t)box_rows, 1u, 1u};
+    // The box is 128 bytes wide (64 bf16 or 32 fp32 elements) and box_rows high.
+    cuuint32_t box[4] = {(cuuint32_t)(128 / elem_bytes), (cuuint32_t)box_rows, 1u, 1u};
     cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
-    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box,
+    CUresult r = g_encode(m, elem_bytes == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
+                          const_cast<void *>(base), dims, strides, box,
                           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(FA_ERR_CUDA, "%s: cuTensorMapEncodeTiled failed (%d)", name, (int)r);
@@ -272,6 +274,11 @@ fa_status fa_fwd(const fa_fwd_params *p, void *stream) {
     if (st != FA_OK) return st;
     st = encode_4d(&L.tmV, vb, p->dv, p->Sk, p->Hkv, p->B, p->v_ss, p->v_sh, p->v_sb, box_k, "fa_fwd v");
     if (st != FA_OK) return st;
+    if (p->dk <= 128) {  // the two-tile kernel writes O with TMA stores
+        st = encode_4d(&L.tmO, p->o, p->dv, p->Sq, p->Hq, p->B, p->o_ss, p->o_sh, p->o_sb, 128, "fa_fwd o",
+                       p->o_dtype == FA_F32 ? 4 : 2);
+        if (st != FA_OK) return st;
+    }
     L.B = p->B;
     L.Hq = p->Hq;
     L.Hkv = p->Hkv;

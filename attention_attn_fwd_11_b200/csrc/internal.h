@@ -11,6 +11,7 @@ namespace fa {
 // ---- prefill -------------------------------------------------------------
 struct PrefillLaunch {
     CUtensorMap tmQ, tmK, tmV;
+    CUtensorMap tmO;  // O as (dv, Sq, Hq, B), box 128 bytes x 128 rows, 128-byte swizzle (two-tile kernel)
     int B, Hq, Hkv, Sq, Sk, dk, dv;
     float scale;
     int causal;

@@ -85,7 +85,9 @@ struct P2Cfg {
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_K = 2 * Q_TILE;
     static constexpr int OFF_V = OFF_K + NSTK * KV_BYTES;
-    static constexpr int OFF_BAR = OFF_V + NSTV * KV_BYTES;
+    static constexpr int OFF_STG = OFF_V + NSTV * KV_BYTES;  // epilogue staging, 16 KB per softmax group
+    static constexpr int STG_BYTES = 128 * 128;              // 128 rows x 128 bytes
+    static constexpr int OFF_BAR = OFF_STG + 2 * STG_BYTES;
     static constexpr int SMEM_BYTES = OFF_BAR + 512 + 1024;
     static constexpr int T_O = 2 * BN;  // O0 at T_O, O1 at T_O + D
     static_assert(2 * BN + 2 * D <= 512, "TMEM budget");
@@ -182,7 +184,8 @@ constexpr int P2_SOFTMAX_WARP0 = P2_THREADS == 384 ? 4 : 2;
 template <int D>
 __global__ void __launch_bounds__(P2_THREADS, 1)
 prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                const __grid_constant__ CUtensorMap tmV, const Prefill2Args a) {
+                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                const Prefill2Args a) {
     using C = P2Cfg<D>;
     constexpr int BN = C::BN, NSTK = C::NSTK, NSTV = C::NSTV;
     extern __shared__ uint8_t smem_raw[];
@@ -345,12 +348,22 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             bool ok = true;
             UnitInfo u;
             for (int r = 0; ok && p2_unit(a, r, u); ++r, ++uc) {
-                // The previous unit's O accumulators must have been read out.
+                // O of tile i from the previous unit must have been read out
+                // before this unit's first PV into it.  A tile with work waits
+                // just before that PV (its QK^T and softmax may start at once);
+                // a tile without work consumes the signal here.  Either way the
+                // signal of every unit is consumed exactly once, and a softmax
+                // group cannot run more than one unit ahead (unit_start).
+                bool ofree_due[2] = {false, false};
                 for (int i = 0; i < 2; ++i) {
-                    if (uc > 0 &&
-                        !mbar_wait(bar(P2_OFREE + i), (uint32_t)(uc - 1) & 1u, abort_flag, &g_prefill2_err)) {
-                        ok = false;
-                        break;
+                    if (uc > 0) {
+                        if (u.n[i] > 0) {
+                            ofree_due[i] = true;
+                        } else if (!mbar_wait(bar(P2_OFREE + i), (uint32_t)(uc - 1) & 1u, abort_flag,
+                                              &g_prefill2_err)) {
+                            ok = false;
+                            break;
+                        }
                     }
                     mbar_arrive(bar(P2_USTART + i));
                 }
@@ -406,6 +419,13 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                         }
                         ++pcnt[0];
                         v_ready = true;
+                        if (ofree_due[0]) {
+                            if (!mbar_wait(bar(P2_OFREE + 0), (uint32_t)(uc - 1) & 1u, abort_flag, &g_prefill2_err)) {
+                                ok = false;
+                                break;
+                            }
+                            ofree_due[0] = false;
+                        }
                         TRACE(3, t, 0);
                         tc_fence_after();
                         pv(0, s, t == 0);
@@ -437,6 +457,13 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                             break;
                         }
                         ++pcnt[1];
+                        if (ofree_due[1]) {
+                            if (!mbar_wait(bar(P2_OFREE + 1), (uint32_t)(uc - 1) & 1u, abort_flag, &g_prefill2_err)) {
+                                ok = false;
+                                break;
+                            }
+                            ofree_due[1] = false;
+                        }
                         TRACE(4, t, 0);
                         tc_fence_after();
                         pv(1, s, t == 0);
@@ -658,51 +685,70 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                     have_o = false;
             }
             pv_base += n;
-            const bool store = qrow < a.Sq;
-            const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
-            const int64_t ooff = (int64_t)u.b * a.o_sb + (int64_t)u.hq * a.o_sh + (int64_t)qrow * a.o_ss;
-#pragma unroll 1
-            for (int ch = 0; ch < D / 32; ++ch) {
-                uint32_t o[32];
-                if (have_o) {
-                    tmem_ld32(tO + (uint32_t)(ch * 32), o);
-                    tmem_wait_ld();
-                    reg_fence(o);
-                } else {
+            // O row -> registers, then TMEM is handed back at once.
+            uint32_t ov[D];
+            if (have_o) {
 #pragma unroll
-                    for (int k = 0; k < 32; ++k) o[k] = 0u;
-                }
-                if (store) {
-                    if (a.o_bf16) {
-                        uint4 *dst = reinterpret_cast<uint4 *>(a.o + 2 * (ooff + ch * 32));
+                for (int ch = 0; ch < D / 32; ++ch)
+                    tmem_ld32(tO + (uint32_t)(ch * 32), *reinterpret_cast<uint32_t(*)[32]>(&ov[ch * 32]));
+                tmem_wait_ld();
+                reg_fence(ov);
+            } else {
 #pragma unroll
-                        for (int k = 0; k < 4; ++k) {
-                            uint4 w;
-                            w.x = pack_bf16x2(__uint_as_float(o[8 * k + 0]) * inv_l, __uint_as_float(o[8 * k + 1]) * inv_l);
-                            w.y = pack_bf16x2(__uint_as_float(o[8 * k + 2]) * inv_l, __uint_as_float(o[8 * k + 3]) * inv_l);
-                            w.z = pack_bf16x2(__uint_as_float(o[8 * k + 4]) * inv_l, __uint_as_float(o[8 * k + 5]) * inv_l);
-                            w.w = pack_bf16x2(__uint_as_float(o[8 * k + 6]) * inv_l, __uint_as_float(o[8 * k + 7]) * inv_l);
-                            dst[k] = w;
-                        }
-                    } else {
-                        float4 *dst = reinterpret_cast<float4 *>(a.o + 4 * (ooff + ch * 32));
-#pragma unroll
-                        for (int k = 0; k < 8; ++k)
-                            dst[k] = make_float4(__uint_as_float(o[4 * k]) * inv_l, __uint_as_float(o[4 * k + 1]) * inv_l,
-                                                 __uint_as_float(o[4 * k + 2]) * inv_l,
-                                                 __uint_as_float(o[4 * k + 3]) * inv_l);
-                    }
-                }
+                for (int k = 0; k < D; ++k) ov[k] = 0u;
             }
-            if (store && a.lse)
-                a.lse[((int64_t)u.b * a.Hq + u.hq) * a.Sq + qrow] =
-                    (l_run > 0.f) ? (m_run + __log2f(l_run)) * 0.69314718055994530942f : -INFINITY;
-            // O of this tile has been read out: the next unit may overwrite it.
             if (row == 0) TRACE(17 + ti, 0, 0);
             tc_fence_before();
-            mbar_arrive(bar(P2_OFREE + ti));
+            mbar_arrive(bar(P2_OFREE + ti));  // O of this tile may be overwritten by the next unit
+            const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+            if (qrow < a.Sq && a.lse)
+                a.lse[((int64_t)u.b * a.Hq + u.hq) * a.Sq + qrow] =
+                    (l_run > 0.f) ? (m_run + __log2f(l_run)) * 0.69314718055994530942f : -INFINITY;
+            // Rows are written through a 16 KB staging tile (128 rows x 128
+            // bytes, 128-byte swizzle) by TMA tensor stores; rows past Sq are
+            // clipped by the store.
+            const uint32_t stg = sbase + C::OFF_STG + ti * C::STG_BYTES;
+            const bool tile_live = u.q0 + 128 * ti < a.Sq;
+            // One 128-byte slice of every row per store: 32 fp32 or 64 bf16.
+            auto store_slice = [&](int ch, int col0, const uint32_t (&w)[32]) {
+                if (row == 0) bulk_wait_read0();  // the previous store has read the staging tile
+                named_bar_sync(1 + ti, 128);
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    *reinterpret_cast<uint4 *>(smem + C::OFF_STG + ti * C::STG_BYTES + row * 128 +
+                                               ((j ^ (row & 7)) << 4)) =
+                        make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+                fence_proxy_async_smem();
+                named_bar_sync(1 + ti, 128);
+                if (row == 0 && tile_live) {
+                    tma_store_4d(&tmO, stg, col0, u.q0 + 128 * ti, u.hq, u.b);
+                    bulk_commit();
+                }
+                (void)ch;
+            };
+            if (a.o_bf16) {
+#pragma unroll
+                for (int ch = 0; ch < D / 64; ++ch) {
+                    uint32_t w[32];
+#pragma unroll
+                    for (int k = 0; k < 32; ++k)
+                        w[k] = pack_bf16x2(__uint_as_float(ov[ch * 64 + 2 * k]) * inv_l,
+                                           __uint_as_float(ov[ch * 64 + 2 * k + 1]) * inv_l);
+                    store_slice(ch, ch * 64, w);
+                }
+            } else {
+#pragma unroll
+                for (int ch = 0; ch < D / 32; ++ch) {
+                    uint32_t w[32];
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) w[k] = __float_as_uint(__uint_as_float(ov[ch * 32 + k]) * inv_l);
+                    store_slice(ch, ch * 32, w);
+                }
+            }
         }
     }
+
+    if (warp >= P2_SOFTMAX_WARP0 && lane == 0) bulk_wait0();  // epilogue stores have landed
 
     tc_fence_before();
     __syncthreads();
@@ -744,7 +790,7 @@ static cudaError_t launch_p2(const PrefillLaunch &L, int num_sms, cudaStream_t s
     }
 #endif
     const int grid = a.n_units < num_sms ? a.n_units : num_sms;
-    kern<<<grid, P2_THREADS, C::SMEM_BYTES, stream>>>(L.tmQ, L.tmK, L.tmV, a);
+    kern<<<grid, P2_THREADS, C::SMEM_BYTES, stream>>>(L.tmQ, L.tmK, L.tmV, L.tmO, a);
     return cudaGetLastError();
 }
 
