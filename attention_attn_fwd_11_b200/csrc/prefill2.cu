@@ -96,8 +96,20 @@ struct P2Cfg {
 
 enum {
     P2_QFULL = 0, P2_QEMPTY = 1, P2_SFULL = 2, P2_PREADY = 4, P2_ODONE = 6, P2_OFREE = 8, P2_USTART = 10,
-    P2_DRAIN = 12, P2_SFREE = 13, P2_RING = 15
+    P2_DRAIN = 12, P2_SFREE = 13, P2_PLO = 15, P2_RING = 17
 };
+
+// FA_P2_SPLITP: the softmax signals when P of keys 0..63 is in TMEM, and the
+// MMA runs that half of PV while the exponentials of keys 64..127 are
+// still being computed.
+#ifndef FA_P2_SPLITP
+#define FA_P2_SPLITP 1
+#endif
+#if FA_P2_SPLITP
+#define P2_PFIRST P2_PLO
+#else
+#define P2_PFIRST P2_PREADY
+#endif
 
 // FA_P2_HOIST: the softmax signals as soon as S is in registers, and the
 // MMA issues the upper half of the next QK^T (keys 64..127, TMEM columns
@@ -109,16 +121,6 @@ enum {
 
 constexpr float kP2RescaleThreshold = 8.0f;
 
-// FA_P2_SPIN: the MMA thread polls the P-ready barriers (lower wake-up
-// latency on the critical path).
-#ifndef FA_P2_SPIN
-#define FA_P2_SPIN 0
-#endif
-#if FA_P2_SPIN
-#define P2_MMA_WAIT mbar_wait_spin
-#else
-#define P2_MMA_WAIT mbar_wait
-#endif
 // FA_P2_MAXCHAINS: independent three-input-max chains in the row max (4 or 8).
 #ifndef FA_P2_MAXCHAINS
 #define FA_P2_MAXCHAINS 4
@@ -137,8 +139,12 @@ constexpr float kP2RescaleThreshold = 8.0f;
 #define FA_EXP2_POLY_EVERY 0
 #endif
 
+// One unit: query rows [q0, q0 + 256) of head hq in batch b, as two
+// 128-row tiles with n0 and n1 key tiles (N = the larger).  Plain scalars,
+// never an indexed array, so that a unit's fields stay in registers.
 struct UnitInfo {
-    int b, hq, q0, n[2], N;
+    int b, hq, q0, n0, n1, N;
+    FA_DEV int nt(int i) const { return i ? n1 : n0; }
 };
 
 FA_DEV bool p2_unit(const Prefill2Args &a, int round, UnitInfo &u) {
@@ -150,20 +156,21 @@ FA_DEV bool p2_unit(const Prefill2Args &a, int round, UnitInfo &u) {
     u.b = bh / a.Hq;
     u.hq = bh % a.Hq;
     u.q0 = qp * 256;
-    u.N = 0;
+    int n[2];
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
         const int r0 = u.q0 + 128 * i;
-        int n = 0;
+        n[i] = 0;
         if (r0 < a.Sq) {
             const int last = min(r0 + 127, a.Sq - 1);
             int kmax = a.Sk - 1;
             if (a.causal) kmax = min(kmax, last + a.Sk - a.Sq);
-            n = kmax < 0 ? 0 : kmax / 128 + 1;
+            n[i] = kmax < 0 ? 0 : kmax / 128 + 1;
         }
-        u.n[i] = n;
-        u.N = max(u.N, n);
     }
+    u.n0 = n[0];
+    u.n1 = n[1];
+    u.N = max(n[0], n[1]);
     return true;
 }
 
@@ -216,6 +223,7 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             mbar_init(bar(P2_OFREE + i), 128);
             mbar_init(bar(P2_USTART + i), 1);
             mbar_init(bar(P2_SFREE + i), 128);
+            mbar_init(bar(P2_PLO + i), 128);
         }
         for (int s = 0; s < NSTK; ++s) {
             mbar_init(k_full(s), 1);
@@ -257,11 +265,27 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             prefetch_tmap(&tmQ);
             prefetch_tmap(&tmK);
             prefetch_tmap(&tmV);
-            int kc = 0, uc = 0, issued = 0;
+            int kc = 0, uc = 0, issued_k = 0, issued_v = 0;
             bool ok = true;
             UnitInfo u;
             for (int r = 0; ok && p2_unit(a, r, u); ++r, ++uc) {
                 const int hkv = u.hq / a.group;
+                auto load_k = [&](int t, int kt) -> bool {
+                    const int sk = kt % NSTK;
+                    if (!mbar_wait(k_empty(sk), ((uint32_t)(kt / NSTK) & 1u) ^ 1u, abort_flag, &g_prefill2_err))
+                        return false;
+                    TRACE(1, t, 0);
+                    mbar_arrive_expect_tx(k_full(sk), C::KV_BYTES);
+#pragma unroll
+                    for (int c = 0; c < C::NCH; ++c)
+                        tma_load_4d(sK + sk * C::KV_BYTES + c * C::KV_CHUNK, &tmK, k_full(sk), c * 64, t * BN, hkv, u.b);
+                    issued_k = kt + 1;
+                    return true;
+                };
+                // K of the unit's first tile goes ahead of Q: it only needs a
+                // free ring slot, while Q waits for the previous unit's last
+                // QK^T; the unit's first QK^T needs both.
+                if (u.N > 0 && !load_k(0, kc)) break;
                 if (!mbar_wait(bar(P2_QEMPTY), ((uint32_t)uc & 1u) ^ 1u, abort_flag, &g_prefill2_err)) break;
                 mbar_arrive_expect_tx(bar(P2_QFULL), 2 * C::Q_TILE);
 #pragma unroll
@@ -271,16 +295,11 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                         tma_load_4d(sQ + i * C::Q_TILE + c * C::Q_CHUNK, &tmQ, bar(P2_QFULL), c * 64, u.q0 + 128 * i,
                                     u.hq, u.b);
                 for (int t = 0; t < u.N; ++t, ++kc) {
-                    const int sk = kc % NSTK, sv = kc % NSTV;
-                    if (!mbar_wait(k_empty(sk), ((uint32_t)(kc / NSTK) & 1u) ^ 1u, abort_flag, &g_prefill2_err)) {
+                    const int sv = kc % NSTV;
+                    if (t > 0 && !load_k(t, kc)) {
                         ok = false;
                         break;
                     }
-                    TRACE(1, t, 0);
-                    mbar_arrive_expect_tx(k_full(sk), C::KV_BYTES);
-#pragma unroll
-                    for (int c = 0; c < C::NCH; ++c)
-                        tma_load_4d(sK + sk * C::KV_BYTES + c * C::KV_CHUNK, &tmK, k_full(sk), c * 64, t * BN, hkv, u.b);
                     if (!mbar_wait(v_empty(sv), ((uint32_t)(kc / NSTV) & 1u) ^ 1u, abort_flag, &g_prefill2_err)) {
                         ok = false;
                         break;
@@ -290,60 +309,89 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 #pragma unroll
                     for (int c = 0; c < C::NCH; ++c)
                         tma_load_4d(sV + sv * C::KV_BYTES + c * C::KV_CHUNK, &tmV, v_full(sv), c * 64, t * BN, hkv, u.b);
-                    issued = kc + 1;
+                    issued_v = kc + 1;
                 }
             }
             if (*abort_flag) {
                 // Let the copies still in flight land before the CTA exits.
                 mbar_wait_drain(bar(P2_QFULL), (uint32_t)(max(uc - 1, 0)) & 1u);
-                for (int k = max(0, issued - NSTK); k < issued; ++k)
+                for (int k = max(0, issued_k - NSTK); k < issued_k; ++k)
                     mbar_wait_drain(k_full(k % NSTK), (uint32_t)(k / NSTK) & 1u);
-                for (int k = max(0, issued - NSTV); k < issued; ++k)
+                for (int k = max(0, issued_v - NSTV); k < issued_v; ++k)
                     mbar_wait_drain(v_full(k % NSTV), (uint32_t)(k / NSTV) & 1u);
             }
         }
     } else if (warp == 1) {
         // ------------------------------------------------- MMA issuer --
-        if (lane == 0) {
+        // The whole warp runs the issue loop; one elected lane issues each
+        // MMA and commit.
+        {
             constexpr uint32_t idesc_qk = idesc_bf16_f32(128, BN, false, false);
             constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, false, true);
+            int kc = 0, uc = 0;
+            int pcnt[2] = {0, 0};  // P-ready phases consumed per tile
+            int tr_t = 0;          // tile index for trace stamps
+            (void)tr_t;
+            // Operand descriptors are built once per tile base; stepping an
+            // operand by b bytes adds b / 16 to the descriptor's address
+            // field, which cannot carry out of it (shared addresses < 256 KB).
+            const uint64_t qdesc = sdesc_sw128(sQ, 16, 1024);
             auto qk = [&](int i, int s) {
                 const uint32_t tS = tmem + (uint32_t)(i * BN);
+                const uint64_t ad0 = qdesc + (uint64_t)((i * C::Q_TILE) >> 4);
+                const uint64_t bd0 = sdesc_sw128(sK + s * C::KV_BYTES, 16, 1024);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const int c = kk >> 2, sub = kk & 3;
-                    const uint64_t ad = sdesc_sw128(sQ + i * C::Q_TILE + c * C::Q_CHUNK + sub * 32, 16, 1024);
-                    const uint64_t bd = sdesc_sw128(sK + s * C::KV_BYTES + c * C::KV_CHUNK + sub * 32, 16, 1024);
-                    mma_ss(tS, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
+                    const uint64_t ad = ad0 + (uint64_t)((c * C::Q_CHUNK + sub * 32) >> 4);
+                    const uint64_t bd = bd0 + (uint64_t)((c * C::KV_CHUNK + sub * 32) >> 4);
+                    mma_ss_warp(tS, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
+                    TRACE(25 + i, tr_t, kk);
                 }
-                mma_commit(bar(P2_SFULL + i));
+                mma_commit_warp(bar(P2_SFULL + i));
             };
             // Half of QK^T: keys [64 h, 64 h + 64) of the K tile into TMEM
             // columns [64 h, 64 h + 64) of S_i.
             auto qk_half = [&](int i, int s, int h) {
                 constexpr uint32_t idesc_half = idesc_bf16_f32(128, BN / 2, false, false);
                 const uint32_t tS = tmem + (uint32_t)(i * BN + h * (BN / 2));
+                const uint64_t ad0 = qdesc + (uint64_t)((i * C::Q_TILE) >> 4);
+                const uint64_t bd0 = sdesc_sw128(sK + s * C::KV_BYTES + h * (BN / 2) * 128, 16, 1024);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const int c = kk >> 2, sub = kk & 3;
-                    const uint64_t ad = sdesc_sw128(sQ + i * C::Q_TILE + c * C::Q_CHUNK + sub * 32, 16, 1024);
-                    const uint64_t bd = sdesc_sw128(
-                        sK + s * C::KV_BYTES + c * C::KV_CHUNK + h * (BN / 2) * 128 + sub * 32, 16, 1024);
-                    mma_ss(tS, ad, bd, idesc_half, kk > 0 ? 1u : 0u);
+                    const uint64_t ad = ad0 + (uint64_t)((c * C::Q_CHUNK + sub * 32) >> 4);
+                    const uint64_t bd = bd0 + (uint64_t)((c * C::KV_CHUNK + sub * 32) >> 4);
+                    mma_ss_warp(tS, ad, bd, idesc_half, kk > 0 ? 1u : 0u);
                 }
             };
-            auto pv = [&](int i, int s, bool first) {
+            // PV over the 16-key steps [k0, k1) of the tile; the last part commits.
+            auto pv = [&](int i, int s, bool first, int k0, int k1) {
                 const uint32_t tO = tmem + (uint32_t)(C::T_O + i * D);
                 const uint32_t tP = tmem + (uint32_t)(i * BN);
+                const uint64_t bd0 = sdesc_sw128(sV + s * C::KV_BYTES, C::KV_CHUNK, 1024);
 #pragma unroll
-                for (int kk = 0; kk < BN / 16; ++kk) {
-                    const uint64_t bd = sdesc_sw128(sV + s * C::KV_BYTES + kk * 2048, C::KV_CHUNK, 1024);
-                    mma_ts(tO, tP + kk * 8, bd, idesc_pv, (!first || kk > 0) ? 1u : 0u);
+                for (int kk = k0; kk < k1; ++kk) {
+                    const uint64_t bd = bd0 + (uint64_t)(kk * (2048 >> 4));
+                    mma_ts_warp(tO, tP + kk * 8, bd, idesc_pv, (!first || kk > 0) ? 1u : 0u);
+                    TRACE(23 + i, tr_t, kk);
                 }
-                mma_commit(bar(P2_ODONE + i));
+                if (k1 == BN / 16) mma_commit_warp(bar(P2_ODONE + i));
             };
-            int kc = 0, uc = 0;
-            int pcnt[2] = {0, 0};
+            // PV of tile i: whole, or (FA_P2_SPLITP) the lower half as soon as
+            // it is in TMEM and the upper half once the rest is.
+            auto pv_tile = [&](int i, int s, bool first) -> bool {
+#if FA_P2_SPLITP
+                pv(i, s, first, 0, BN / 32);
+                if (!mbar_wait_warp(bar(P2_PREADY + i), (uint32_t)pcnt[i] & 1u, abort_flag, &g_prefill2_err))
+                    return false;
+                tc_fence_after();
+                pv(i, s, first, BN / 32, BN / 16);
+#else
+                pv(i, s, first, 0, BN / 16);
+#endif
+                return true;
+            };
             int fcnt[2] = {0, 0};  // S-free phases consumed (hoisting only)
             bool ok = true;
             UnitInfo u;
@@ -357,40 +405,41 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 bool ofree_due[2] = {false, false};
                 for (int i = 0; i < 2; ++i) {
                     if (uc > 0) {
-                        if (u.n[i] > 0) {
+                        if (u.nt(i) > 0) {
                             ofree_due[i] = true;
-                        } else if (!mbar_wait(bar(P2_OFREE + i), (uint32_t)(uc - 1) & 1u, abort_flag,
+                        } else if (!mbar_wait_warp(bar(P2_OFREE + i), (uint32_t)(uc - 1) & 1u, abort_flag,
                                               &g_prefill2_err)) {
                             ok = false;
                             break;
                         }
                     }
-                    mbar_arrive(bar(P2_USTART + i));
+                    mbar_arrive_warp(bar(P2_USTART + i));  // one arrival per warp
                 }
-                if (!ok || !mbar_wait(bar(P2_QFULL), (uint32_t)uc & 1u, abort_flag, &g_prefill2_err)) break;
+                if (!ok || !mbar_wait_warp(bar(P2_QFULL), (uint32_t)uc & 1u, abort_flag, &g_prefill2_err)) break;
                 tc_fence_after();
                 if (u.N == 0) {
-                    mma_commit(bar(P2_QEMPTY));
+                    mma_commit_warp(bar(P2_QEMPTY));
                     continue;
                 }
                 {
                     const int s0 = kc % NSTK;
-                    if (!mbar_wait(k_full(s0), (uint32_t)(kc / NSTK) & 1u, abort_flag, &g_prefill2_err)) break;
+                    if (!mbar_wait_warp(k_full(s0), (uint32_t)(kc / NSTK) & 1u, abort_flag, &g_prefill2_err)) break;
                     tc_fence_after();
-                    if (u.n[0] > 0) qk(0, s0);
-                    if (u.n[1] > 0) qk(1, s0);
-                    mma_commit(k_empty(s0));
-                    if (u.N == 1) mma_commit(bar(P2_QEMPTY));
+                    if (u.n0 > 0) qk(0, s0);
+                    if (u.n1 > 0) qk(1, s0);
+                    mma_commit_warp(k_empty(s0));
+                    if (u.N == 1) mma_commit_warp(bar(P2_QEMPTY));
                 }
                 for (int t = 0; t < u.N; ++t) {
                     const int kt = kc + t;
                     const int s = kt % NSTV;  // V stage of tile t
                     const bool has_next = t + 1 < u.N;
+                    tr_t = t;
                     const int s1 = (kt + 1) % NSTK;  // K stage of tile t + 1
                     bool v_ready = false;
 #if FA_P2_HOIST
                     if (has_next) {
-                        if (!mbar_wait(k_full(s1), (uint32_t)((kt + 1) / NSTK) & 1u, abort_flag, &g_prefill2_err)) {
+                        if (!mbar_wait_warp(k_full(s1), (uint32_t)((kt + 1) / NSTK) & 1u, abort_flag, &g_prefill2_err)) {
                             ok = false;
                             break;
                         }
@@ -398,29 +447,30 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                     // Every S-free phase is consumed; while there is a next tile the
                     // upper half of its QK^T goes ahead of this tile's PV.
                     for (int i = 0; ok && i < 2; ++i) {
-                        if (t >= u.n[i]) continue;
-                        if (!P2_MMA_WAIT(bar(P2_SFREE + i), (uint32_t)fcnt[i] & 1u, abort_flag, &g_prefill2_err)) {
+                        if (t >= u.nt(i)) continue;
+                        if (!mbar_wait_warp(bar(P2_SFREE + i), (uint32_t)fcnt[i] & 1u, abort_flag, &g_prefill2_err)) {
                             ok = false;
                             break;
                         }
                         ++fcnt[i];
-                        if (has_next && t + 1 < u.n[i]) {
+                        if (has_next && t + 1 < u.nt(i)) {
                             tc_fence_after();
                             qk_half(i, s1, 1);
                         }
                     }
                     if (!ok) break;
 #endif
-                    if (t < u.n[0]) {
-                        if (!P2_MMA_WAIT(bar(P2_PREADY + 0), (uint32_t)pcnt[0] & 1u, abort_flag, &g_prefill2_err) ||
-                            !mbar_wait(v_full(s), (uint32_t)(kt / NSTV) & 1u, abort_flag, &g_prefill2_err)) {
+                    if (t < u.n0) {
+                        TRACE(27, t, 0);
+                        if (!mbar_wait_warp(bar(P2_PFIRST + 0), (uint32_t)pcnt[0] & 1u, abort_flag, &g_prefill2_err) ||
+                            (TRACE(27, t, 1), false) ||
+                            !mbar_wait_warp(v_full(s), (uint32_t)(kt / NSTV) & 1u, abort_flag, &g_prefill2_err)) {
                             ok = false;
                             break;
                         }
-                        ++pcnt[0];
                         v_ready = true;
                         if (ofree_due[0]) {
-                            if (!mbar_wait(bar(P2_OFREE + 0), (uint32_t)(uc - 1) & 1u, abort_flag, &g_prefill2_err)) {
+                            if (!mbar_wait_warp(bar(P2_OFREE + 0), (uint32_t)(uc - 1) & 1u, abort_flag, &g_prefill2_err)) {
                                 ok = false;
                                 break;
                             }
@@ -428,37 +478,42 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                         }
                         TRACE(3, t, 0);
                         tc_fence_after();
-                        pv(0, s, t == 0);
+                        if (!pv_tile(0, s, t == 0)) {
+                            ok = false;
+                            break;
+                        }
+                        ++pcnt[0];
                         TRACE(5, t, 0);
                     }
                     if (has_next) {
 #if !FA_P2_HOIST
-                        if (!mbar_wait(k_full(s1), (uint32_t)((kt + 1) / NSTK) & 1u, abort_flag, &g_prefill2_err)) {
+                        TRACE(28, t, 0);
+                        if (!mbar_wait_warp(k_full(s1), (uint32_t)((kt + 1) / NSTK) & 1u, abort_flag, &g_prefill2_err)) {
                             ok = false;
                             break;
                         }
 #endif
+                        TRACE(28, t, 1);
                         tc_fence_after();
-                        if (t + 1 < u.n[0]) {
+                        if (t + 1 < u.n0) {
 #if FA_P2_HOIST
                             qk_half(0, s1, 0);
-                            mma_commit(bar(P2_SFULL + 0));
+                            mma_commit_warp(bar(P2_SFULL + 0));
 #else
                             qk(0, s1);
 #endif
                             TRACE(7, t + 1, 0);
                         }
                     }
-                    if (t < u.n[1]) {
-                        if (!P2_MMA_WAIT(bar(P2_PREADY + 1), (uint32_t)pcnt[1] & 1u, abort_flag, &g_prefill2_err) ||
+                    if (t < u.n1) {
+                        if (!mbar_wait_warp(bar(P2_PFIRST + 1), (uint32_t)pcnt[1] & 1u, abort_flag, &g_prefill2_err) ||
                             (!v_ready &&
-                             !mbar_wait(v_full(s), (uint32_t)(kt / NSTV) & 1u, abort_flag, &g_prefill2_err))) {
+                             !mbar_wait_warp(v_full(s), (uint32_t)(kt / NSTV) & 1u, abort_flag, &g_prefill2_err))) {
                             ok = false;
                             break;
                         }
-                        ++pcnt[1];
                         if (ofree_due[1]) {
-                            if (!mbar_wait(bar(P2_OFREE + 1), (uint32_t)(uc - 1) & 1u, abort_flag, &g_prefill2_err)) {
+                            if (!mbar_wait_warp(bar(P2_OFREE + 1), (uint32_t)(uc - 1) & 1u, abort_flag, &g_prefill2_err)) {
                                 ok = false;
                                 break;
                             }
@@ -466,30 +521,34 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                         }
                         TRACE(4, t, 0);
                         tc_fence_after();
-                        pv(1, s, t == 0);
+                        if (!pv_tile(1, s, t == 0)) {
+                            ok = false;
+                            break;
+                        }
+                        ++pcnt[1];
                         TRACE(6, t, 0);
                     }
-                    if (has_next && t + 1 < u.n[1]) {
+                    if (has_next && t + 1 < u.n1) {
 #if FA_P2_HOIST
                         qk_half(1, s1, 0);
-                        mma_commit(bar(P2_SFULL + 1));
+                        mma_commit_warp(bar(P2_SFULL + 1));
 #else
                         qk(1, s1);
 #endif
                         TRACE(8, t + 1, 0);
                     }
-                    mma_commit(v_empty(s));
+                    mma_commit_warp(v_empty(s));
                     if (has_next) {
-                        mma_commit(k_empty(s1));
-                        if (t + 2 == u.N) mma_commit(bar(P2_QEMPTY));  // the unit's last QK^T is issued
+                        mma_commit_warp(k_empty(s1));
+                        if (t + 2 == u.N) mma_commit_warp(bar(P2_QEMPTY));  // the unit's last QK^T is issued
                     }
                 }
                 kc += u.N;
             }
-            mma_commit(bar(P2_DRAIN));
+            mma_commit_warp(bar(P2_DRAIN));
             mbar_wait_drain(bar(P2_DRAIN), 0);
+            __syncwarp();
         }
-        __syncwarp();
     }
     } else {
         P2_REGS_HIGH();
@@ -506,7 +565,7 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         UnitInfo u;
         for (int r = 0; ok && p2_unit(a, r, u); ++r, ++uc) {
             if (!mbar_wait(bar(P2_USTART + ti), (uint32_t)uc & 1u, abort_flag, &g_prefill2_err)) break;
-            const int n = u.n[ti];
+            const int n = u.nt(ti);
             const int qrow = u.q0 + 128 * ti + row;
             const int lim_all = a.causal ? min(a.Sk, qrow + a.Sk - a.Sq + 1) : a.Sk;
             float m_run = -INFINITY, l_run = 0.f;
@@ -637,6 +696,13 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                             pk[k] = pack_bf16x2(p0, p1);
                         }
                         tmem_st16(tS + (uint32_t)(g * 16), pk);
+#if FA_P2_SPLITP
+                        if (g == BN / 64 - 1) {  // keys 0..63 of P are stored
+                            tmem_wait_st();
+                            tc_fence_before();
+                            mbar_arrive(bar(P2_PLO + ti));
+                        }
+#endif
                     }
                     if (lane == 0) TRACE(21 + ti, t, qd);
                     float u0, u1, u2, u3;
@@ -667,6 +733,13 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                         pk[k] = pack_bf16x2(p0, p1);
                     }
                     tmem_st16(tS + (uint32_t)(g * 16), pk);
+#if FA_P2_SPLITP
+                    if (g == BN / 64 - 1) {
+                        tmem_wait_st();
+                        tc_fence_before();
+                        mbar_arrive(bar(P2_PLO + ti));
+                    }
+#endif
                 }
                 l_run += s0 + s1;
 #endif

@@ -52,8 +52,23 @@ FA_DEV void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
                  : "memory");
 }
 
+// FA_WAIT_HINT_NS > 0: a thread whose phase is not complete may stay
+// suspended up to that many nanoseconds (it resumes as soon as the phase
+// completes); 0 leaves the limit to the hardware.
+#ifndef FA_WAIT_HINT_NS
+#define FA_WAIT_HINT_NS 0
+#endif
 FA_DEV bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     uint32_t done;
+#if FA_WAIT_HINT_NS > 0
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(bar), "r"(parity), "n"(FA_WAIT_HINT_NS)
+        : "memory");
+#else
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
@@ -61,6 +76,7 @@ FA_DEV bool mbar_try_wait(uint32_t bar, uint32_t parity) {
         : "=r"(done)
         : "r"(bar), "r"(parity)
         : "memory");
+#endif
     return done != 0;
 }
 
@@ -302,6 +318,54 @@ FA_DEV void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t i
 FA_DEV void mma_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
                  : "memory");
+}
+
+// Warp-collective forms: the whole warp executes them convergently and one
+// elected lane issues the operation.  An issuer loop run by a full warp keeps
+// its control flow and operands warp-uniform; run by one lane of a diverged
+// warp, every mbarrier wait between MMAs stalled the tensor pipe for tens of
+// cycles.
+FA_DEV void mma_ss_warp(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+FA_DEV void mma_ts_warp(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+FA_DEV void mma_commit_warp(uint32_t bar) {
+    asm volatile(
+        "{\n\t.reg .pred e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(bar)
+        : "memory");
+}
+
+FA_DEV void mbar_arrive_warp(uint32_t bar) {
+    asm volatile(
+        "{\n\t.reg .pred e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];\n\t}" ::"r"(bar)
+        : "memory");
+}
+
+// Bounded wait by a whole warp; the result is made warp-uniform, so a warp
+// never diverges on it (an abort seen by one lane is seen by all).
+FA_DEV bool mbar_wait_warp(uint32_t bar, uint32_t parity, volatile int *abort_flag, int *err) {
+    const bool r = mbar_wait(bar, parity, abort_flag, err);
+    return __all_sync(0xffffffffu, r);
 }
 
 // Instruction descriptor for kind::f16 with bf16 A/B and fp32 D.
