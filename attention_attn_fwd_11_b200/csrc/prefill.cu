@@ -175,13 +175,15 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         }
     } else if (warp == 1) {
         // ------------------------------------------------- MMA issuer --
-        if (lane == 0 && n_tiles > 0) {
+        // The whole warp runs the issue loop; one elected lane issues each
+        // MMA and commit.
+        if (n_tiles > 0) {
             constexpr uint32_t idesc_qk = idesc_bf16_f32(128, BN, false, false);
             constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, false, true);
             const uint32_t tO = tmem + C::T_O;
             auto issue_qk = [&](int t) -> bool {
                 const int s = t % NST;
-                if (!mbar_wait(k_full(s), (uint32_t)(t / NST) & 1u, abort_flag, &g_prefill_err)) return false;
+                if (!mbar_wait_warp(k_full(s), (uint32_t)(t / NST) & 1u, abort_flag, &g_prefill_err)) return false;
                 tc_fence_after();
                 const uint32_t tS = tmem + (uint32_t)((t & 1) * BN);
 #pragma unroll
@@ -189,30 +191,30 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                     const int c = kk >> 2, sub = kk & 3;
                     const uint64_t ad = sdesc_sw128(sQ + c * C::Q_CHUNK + sub * 32, 16, 1024);
                     const uint64_t bd = sdesc_sw128(sK + s * C::KV_BYTES + c * C::KV_CHUNK + sub * 32, 16, 1024);
-                    mma_ss(tS, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
+                    mma_ss_warp(tS, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
                 }
-                mma_commit(k_empty(s));
-                mma_commit(bar(B_SFULL + (t & 1)));
+                mma_commit_warp(k_empty(s));
+                mma_commit_warp(bar(B_SFULL + (t & 1)));
                 return true;
             };
-            bool ok = mbar_wait(bar(B_QFULL), 0, abort_flag, &g_prefill_err) && issue_qk(0);
+            bool ok = mbar_wait_warp(bar(B_QFULL), 0, abort_flag, &g_prefill_err) && issue_qk(0);
             for (int t = 0; ok && t < n_tiles; ++t) {
                 if (t + 1 < n_tiles && !issue_qk(t + 1)) break;
-                if (!mbar_wait(bar(B_PREADY + (t & 1)), (uint32_t)(t >> 1) & 1u, abort_flag, &g_prefill_err)) break;
+                if (!mbar_wait_warp(bar(B_PREADY + (t & 1)), (uint32_t)(t >> 1) & 1u, abort_flag, &g_prefill_err)) break;
                 const int s = t % NST;
-                if (!mbar_wait(v_full(s), (uint32_t)(t / NST) & 1u, abort_flag, &g_prefill_err)) break;
+                if (!mbar_wait_warp(v_full(s), (uint32_t)(t / NST) & 1u, abort_flag, &g_prefill_err)) break;
                 tc_fence_after();
                 const uint32_t tP = tmem + (uint32_t)((t & 1) * BN);
 #pragma unroll
                 for (int kk = 0; kk < BN / 16; ++kk) {
                     const uint64_t bd = sdesc_sw128(sV + s * C::KV_BYTES + kk * 2048, C::KV_CHUNK, 1024);
-                    mma_ts(tO, tP + kk * 8, bd, idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
+                    mma_ts_warp(tO, tP + kk * 8, bd, idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
                 }
-                mma_commit(v_empty(s));
-                mma_commit(bar(B_PVDONE));
+                mma_commit_warp(v_empty(s));
+                mma_commit_warp(bar(B_PVDONE));
             }
             // Nothing of ours may still run on the tensor core once TMEM is freed.
-            mma_commit(bar(B_DRAIN));
+            mma_commit_warp(bar(B_DRAIN));
             mbar_wait_drain(bar(B_DRAIN), 0);
         }
         __syncwarp();
