@@ -96,7 +96,7 @@ struct P2Cfg {
 
 enum {
     P2_QFULL = 0, P2_QEMPTY = 1, P2_SFULL = 2, P2_PREADY = 4, P2_ODONE = 6, P2_OFREE = 8, P2_USTART = 10,
-    P2_DRAIN = 12, P2_SFREE = 13, P2_PLO = 15, P2_RING = 17
+    P2_DRAIN = 12, P2_PLO = 13, P2_RING = 15
 };
 
 // FA_P2_SPLITP: the softmax signals when P of keys 0..63 is in TMEM, and the
@@ -111,13 +111,6 @@ enum {
 #define P2_PFIRST P2_PREADY
 #endif
 
-// FA_P2_HOIST: the softmax signals as soon as S is in registers, and the
-// MMA issues the upper half of the next QK^T (keys 64..127, TMEM columns
-// that P does not use) before the current PV; only the lower half stays
-// between PV and the next softmax.
-#ifndef FA_P2_HOIST
-#define FA_P2_HOIST 0
-#endif
 
 constexpr float kP2RescaleThreshold = 8.0f;
 
@@ -222,7 +215,6 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             mbar_init(bar(P2_ODONE + i), 1);
             mbar_init(bar(P2_OFREE + i), 128);
             mbar_init(bar(P2_USTART + i), 1);
-            mbar_init(bar(P2_SFREE + i), 128);
             mbar_init(bar(P2_PLO + i), 128);
         }
         for (int s = 0; s < NSTK; ++s) {
@@ -321,6 +313,23 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                     mbar_wait_drain(v_full(k % NSTV), (uint32_t)(k / NSTV) & 1u);
             }
         }
+#ifdef FA_P2_TRACE
+    } else if (warp == 2) {
+        // Trace builds only: stamp the moment each K and V tile lands.
+        if (lane == 0) {
+            int kc = 0, uc = 0;
+            UnitInfo u;
+            for (int r = 0; p2_unit(a, r, u); ++r, ++uc)
+                for (int t = 0; t < u.N; ++t, ++kc) {
+                    for (int n = 0; n < (1 << 24) && !mbar_test(k_full(kc % NSTK), (uint32_t)(kc / NSTK) & 1u); ++n) {
+                    }
+                    TRACE(29, t, 0);
+                    for (int n = 0; n < (1 << 24) && !mbar_test(v_full(kc % NSTV), (uint32_t)(kc / NSTV) & 1u); ++n) {
+                    }
+                    TRACE(29, t, 1);
+                }
+        }
+#endif
     } else if (warp == 1) {
         // ------------------------------------------------- MMA issuer --
         // The whole warp runs the issue loop; one elected lane issues each
@@ -350,21 +359,6 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 }
                 mma_commit_warp(bar(P2_SFULL + i));
             };
-            // Half of QK^T: keys [64 h, 64 h + 64) of the K tile into TMEM
-            // columns [64 h, 64 h + 64) of S_i.
-            auto qk_half = [&](int i, int s, int h) {
-                constexpr uint32_t idesc_half = idesc_bf16_f32(128, BN / 2, false, false);
-                const uint32_t tS = tmem + (uint32_t)(i * BN + h * (BN / 2));
-                const uint64_t ad0 = qdesc + (uint64_t)((i * C::Q_TILE) >> 4);
-                const uint64_t bd0 = sdesc_sw128(sK + s * C::KV_BYTES + h * (BN / 2) * 128, 16, 1024);
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const int c = kk >> 2, sub = kk & 3;
-                    const uint64_t ad = ad0 + (uint64_t)((c * C::Q_CHUNK + sub * 32) >> 4);
-                    const uint64_t bd = bd0 + (uint64_t)((c * C::KV_CHUNK + sub * 32) >> 4);
-                    mma_ss_warp(tS, ad, bd, idesc_half, kk > 0 ? 1u : 0u);
-                }
-            };
             // PV over the 16-key steps [k0, k1) of the tile; the last part commits.
             auto pv = [&](int i, int s, bool first, int k0, int k1) {
                 const uint32_t tO = tmem + (uint32_t)(C::T_O + i * D);
@@ -392,7 +386,6 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 #endif
                 return true;
             };
-            int fcnt[2] = {0, 0};  // S-free phases consumed (hoisting only)
             bool ok = true;
             UnitInfo u;
             for (int r = 0; ok && p2_unit(a, r, u); ++r, ++uc) {
@@ -436,107 +429,41 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                     const bool has_next = t + 1 < u.N;
                     tr_t = t;
                     const int s1 = (kt + 1) % NSTK;  // K stage of tile t + 1
-                    bool v_ready = false;
-#if FA_P2_HOIST
-                    if (has_next) {
-                        if (!mbar_wait_warp(k_full(s1), (uint32_t)((kt + 1) / NSTK) & 1u, abort_flag, &g_prefill2_err)) {
-                            ok = false;
-                            break;
-                        }
+                    // This step's V and the next step's K landed long before P
+                    // is ready: waiting for them first leaves nothing but the
+                    // P-ready wait between a softmax and the MMAs after it.
+                    TRACE(28, t, 0);
+                    if (!mbar_wait_warp(v_full(s), (uint32_t)(kt / NSTV) & 1u, abort_flag, &g_prefill2_err) ||
+                        (has_next &&
+                         !mbar_wait_warp(k_full(s1), (uint32_t)((kt + 1) / NSTK) & 1u, abort_flag, &g_prefill2_err))) {
+                        ok = false;
+                        break;
                     }
-                    // Every S-free phase is consumed; while there is a next tile the
-                    // upper half of its QK^T goes ahead of this tile's PV.
-                    for (int i = 0; ok && i < 2; ++i) {
-                        if (t >= u.nt(i)) continue;
-                        if (!mbar_wait_warp(bar(P2_SFREE + i), (uint32_t)fcnt[i] & 1u, abort_flag, &g_prefill2_err)) {
-                            ok = false;
-                            break;
-                        }
-                        ++fcnt[i];
-                        if (has_next && t + 1 < u.nt(i)) {
+                    TRACE(28, t, 1);
+#pragma unroll
+                    for (int i = 0; i < 2; ++i) {
+                        if (ok && t < u.nt(i)) {
+                            if (ofree_due[i]) {
+                                ok = mbar_wait_warp(bar(P2_OFREE + i), (uint32_t)(uc - 1) & 1u, abort_flag,
+                                                    &g_prefill2_err);
+                                ofree_due[i] = false;
+                            }
+                            if (i == 0) TRACE(27, t, 0);
+                            ok = ok && mbar_wait_warp(bar(P2_PFIRST + i), (uint32_t)pcnt[i] & 1u, abort_flag,
+                                                      &g_prefill2_err);
+                            if (i == 0) TRACE(27, t, 1);
+                            TRACE(3 + i, t, 0);
                             tc_fence_after();
-                            qk_half(i, s1, 1);
+                            ok = ok && pv_tile(i, s, t == 0);
+                            ++pcnt[i];
+                            TRACE(5 + i, t, 0);
+                        }
+                        if (ok && has_next && t + 1 < u.nt(i)) {
+                            qk(i, s1);
+                            TRACE(7 + i, t + 1, 0);
                         }
                     }
                     if (!ok) break;
-#endif
-                    if (t < u.n0) {
-                        TRACE(27, t, 0);
-                        if (!mbar_wait_warp(bar(P2_PFIRST + 0), (uint32_t)pcnt[0] & 1u, abort_flag, &g_prefill2_err) ||
-                            (TRACE(27, t, 1), false) ||
-                            !mbar_wait_warp(v_full(s), (uint32_t)(kt / NSTV) & 1u, abort_flag, &g_prefill2_err)) {
-                            ok = false;
-                            break;
-                        }
-                        v_ready = true;
-                        if (ofree_due[0]) {
-                            if (!mbar_wait_warp(bar(P2_OFREE + 0), (uint32_t)(uc - 1) & 1u, abort_flag, &g_prefill2_err)) {
-                                ok = false;
-                                break;
-                            }
-                            ofree_due[0] = false;
-                        }
-                        TRACE(3, t, 0);
-                        tc_fence_after();
-                        if (!pv_tile(0, s, t == 0)) {
-                            ok = false;
-                            break;
-                        }
-                        ++pcnt[0];
-                        TRACE(5, t, 0);
-                    }
-                    if (has_next) {
-#if !FA_P2_HOIST
-                        TRACE(28, t, 0);
-                        if (!mbar_wait_warp(k_full(s1), (uint32_t)((kt + 1) / NSTK) & 1u, abort_flag, &g_prefill2_err)) {
-                            ok = false;
-                            break;
-                        }
-#endif
-                        TRACE(28, t, 1);
-                        tc_fence_after();
-                        if (t + 1 < u.n0) {
-#if FA_P2_HOIST
-                            qk_half(0, s1, 0);
-                            mma_commit_warp(bar(P2_SFULL + 0));
-#else
-                            qk(0, s1);
-#endif
-                            TRACE(7, t + 1, 0);
-                        }
-                    }
-                    if (t < u.n1) {
-                        if (!mbar_wait_warp(bar(P2_PFIRST + 1), (uint32_t)pcnt[1] & 1u, abort_flag, &g_prefill2_err) ||
-                            (!v_ready &&
-                             !mbar_wait_warp(v_full(s), (uint32_t)(kt / NSTV) & 1u, abort_flag, &g_prefill2_err))) {
-                            ok = false;
-                            break;
-                        }
-                        if (ofree_due[1]) {
-                            if (!mbar_wait_warp(bar(P2_OFREE + 1), (uint32_t)(uc - 1) & 1u, abort_flag, &g_prefill2_err)) {
-                                ok = false;
-                                break;
-                            }
-                            ofree_due[1] = false;
-                        }
-                        TRACE(4, t, 0);
-                        tc_fence_after();
-                        if (!pv_tile(1, s, t == 0)) {
-                            ok = false;
-                            break;
-                        }
-                        ++pcnt[1];
-                        TRACE(6, t, 0);
-                    }
-                    if (has_next && t + 1 < u.n1) {
-#if FA_P2_HOIST
-                        qk_half(1, s1, 0);
-                        mma_commit_warp(bar(P2_SFULL + 1));
-#else
-                        qk(1, s1);
-#endif
-                        TRACE(8, t + 1, 0);
-                    }
                     mma_commit_warp(v_empty(s));
                     if (has_next) {
                         mma_commit_warp(k_empty(s1));
@@ -588,10 +515,6 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 #pragma unroll
                     for (int k = 0; k < BN; ++k) x[k] = __uint_as_float(rr[k]);
                 }
-#if FA_P2_HOIST
-                tc_fence_before();
-                mbar_arrive(bar(P2_SFREE + ti));  // S is in registers: its upper half may be overwritten
-#endif
                 if (lane == 0) TRACE(11 + ti, t, qd);
                 const int lim = lim_all - t * BN;
                 if (lim < BN) {
@@ -669,6 +592,7 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 // ex2, one bf16x2 convert; the row sum in two packed
                 // accumulators (one f32x2 add per pair).
                 {
+                    if (lane == 0) TRACE(30, t, qd + 4 * ti);
                     const uint64_t c2 = f2_pack(c, c);
                     const uint64_t nm2 = f2_pack(-msub, -msub);
                     uint64_t acc0 = f2_pack(0.f, 0.f), acc1 = acc0;
@@ -698,6 +622,7 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                         tmem_st16(tS + (uint32_t)(g * 16), pk);
 #if FA_P2_SPLITP
                         if (g == BN / 64 - 1) {  // keys 0..63 of P are stored
+                            if (lane == 0) TRACE(31, t, qd + 4 * ti);
                             tmem_wait_st();
                             tc_fence_before();
                             mbar_arrive(bar(P2_PLO + ti));

@@ -47,8 +47,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 NCU_TRAFFIC = {
     # dram__bytes_read.sum + dram__bytes_write.sum of one launch; the summary
     # under profiles/ named for the kernel and workload gives the capture.
-    "causal_mha_b2_h16_s2048_d128": 54141184,
-    "gqa_full_b1_hq32_hkv8_s4096_d256": 210472960,
+    "causal_mha_b2_h16_s2048_d128": 53822720,
+    "gqa_full_b1_hq32_hkv8_s4096_d256": 215805440,
     "paged_gqa_b64_hq32_hkv8_d128_bs64": 1237055008,
     "latent_sparse_t32_hq128_dk576_dv512_top2048": 45249792,
 }
