@@ -186,13 +186,12 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 if (!mbar_wait_warp(k_full(s), (uint32_t)(t / NST) & 1u, abort_flag, &g_prefill_err)) return false;
                 tc_fence_after();
                 const uint32_t tS = tmem + (uint32_t)((t & 1) * BN);
+                const uint64_t ad0 = sdesc_sw128(sQ, 16, 1024);
+                const uint64_t bd0 = sdesc_sw128(sK + s * C::KV_BYTES, 16, 1024);
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const int c = kk >> 2, sub = kk & 3;
-                    const uint64_t ad = sdesc_sw128(sQ + c * C::Q_CHUNK + sub * 32, 16, 1024);
-                    const uint64_t bd = sdesc_sw128(sK + s * C::KV_BYTES + c * C::KV_CHUNK + sub * 32, 16, 1024);
-                    mma_ss_warp(tS, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
-                }
+                for (int c = 0; c < C::NCH; ++c)  // four 16-wide K steps per 64-column chunk
+                    mma_ss4_warp<2, 4, 6>(tS, ad0 + (uint64_t)((c * C::Q_CHUNK) >> 4),
+                                          bd0 + (uint64_t)((c * C::KV_CHUNK) >> 4), idesc_qk, c > 0 ? 1u : 0u);
                 mma_commit_warp(k_empty(s));
                 mma_commit_warp(bar(B_SFULL + (t & 1)));
                 return true;
@@ -205,11 +204,11 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 if (!mbar_wait_warp(v_full(s), (uint32_t)(t / NST) & 1u, abort_flag, &g_prefill_err)) break;
                 tc_fence_after();
                 const uint32_t tP = tmem + (uint32_t)((t & 1) * BN);
+                const uint64_t bd0 = sdesc_sw128(sV + s * C::KV_BYTES, C::KV_CHUNK, 1024);
 #pragma unroll
-                for (int kk = 0; kk < BN / 16; ++kk) {
-                    const uint64_t bd = sdesc_sw128(sV + s * C::KV_BYTES + kk * 2048, C::KV_CHUNK, 1024);
-                    mma_ts_warp(tO, tP + kk * 8, bd, idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
-                }
+                for (int kb = 0; kb < BN / 16; kb += 4)
+                    mma_ts4_warp<8, (2048 >> 4)>(tO, tP + (uint32_t)(kb * 8), bd0 + (uint64_t)(kb * (2048 >> 4)),
+                                                 idesc_pv, (t > 0 || kb > 0) ? 1u : 0u);
                 mma_commit_warp(v_empty(s));
                 mma_commit_warp(bar(B_PVDONE));
             }

@@ -52,7 +52,14 @@ FA_DEV void trace(int ev, int t, int sub, int uc) {
     if (blockIdx.x != FA_P2_TRACE_CTA || uc >= 2 || t >= 64 || ev >= 32) return;
     g_trace[((uc * 32 + ev) * 64 + t) * 8 + sub] = clock64();
 }
-#define TRACE(ev, t, sub) trace(ev, t, sub, uc)
+// FA_P2_TRACE_MASK selects the events a trace build records (bit ev).
+#ifndef FA_P2_TRACE_MASK
+#define FA_P2_TRACE_MASK 0xffffffffu
+#endif
+#define TRACE(ev, t, sub)                                                  \
+    do {                                                                   \
+        if ((FA_P2_TRACE_MASK >> (ev)) & 1u) trace(ev, t, sub, uc);        \
+    } while (0)
 #else
 #define TRACE(ev, t, sub) ((void)0)
 #endif
@@ -313,7 +320,7 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                     mbar_wait_drain(v_full(k % NSTV), (uint32_t)(k / NSTV) & 1u);
             }
         }
-#ifdef FA_P2_TRACE
+#if defined(FA_P2_TRACE) && ((FA_P2_TRACE_MASK >> 29) & 1u)
     } else if (warp == 2) {
         // Trace builds only: stamp the moment each K and V tile lands.
         if (lane == 0) {
@@ -350,25 +357,24 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 const uint64_t ad0 = qdesc + (uint64_t)((i * C::Q_TILE) >> 4);
                 const uint64_t bd0 = sdesc_sw128(sK + s * C::KV_BYTES, 16, 1024);
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const int c = kk >> 2, sub = kk & 3;
-                    const uint64_t ad = ad0 + (uint64_t)((c * C::Q_CHUNK + sub * 32) >> 4);
-                    const uint64_t bd = bd0 + (uint64_t)((c * C::KV_CHUNK + sub * 32) >> 4);
-                    mma_ss_warp(tS, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
-                    TRACE(25 + i, tr_t, kk);
+                for (int c = 0; c < C::NCH; ++c) {  // four 16-wide K steps per 64-column chunk
+                    mma_ss4_warp<2, 4, 6>(tS, ad0 + (uint64_t)((c * C::Q_CHUNK) >> 4),
+                                          bd0 + (uint64_t)((c * C::KV_CHUNK) >> 4), idesc_qk, c > 0 ? 1u : 0u);
+                    TRACE(25 + i, tr_t, c);
                 }
                 mma_commit_warp(bar(P2_SFULL + i));
             };
-            // PV over the 16-key steps [k0, k1) of the tile; the last part commits.
+            // PV over the 16-key steps [k0, k1) of the tile (k0, k1 multiples
+            // of 4); the part that ends the tile commits.
             auto pv = [&](int i, int s, bool first, int k0, int k1) {
                 const uint32_t tO = tmem + (uint32_t)(C::T_O + i * D);
                 const uint32_t tP = tmem + (uint32_t)(i * BN);
                 const uint64_t bd0 = sdesc_sw128(sV + s * C::KV_BYTES, C::KV_CHUNK, 1024);
 #pragma unroll
-                for (int kk = k0; kk < k1; ++kk) {
-                    const uint64_t bd = bd0 + (uint64_t)(kk * (2048 >> 4));
-                    mma_ts_warp(tO, tP + kk * 8, bd, idesc_pv, (!first || kk > 0) ? 1u : 0u);
-                    TRACE(23 + i, tr_t, kk);
+                for (int kb = k0; kb < k1; kb += 4) {
+                    mma_ts4_warp<8, (2048 >> 4)>(tO, tP + (uint32_t)(kb * 8), bd0 + (uint64_t)(kb * (2048 >> 4)),
+                                                 idesc_pv, (!first || kb > 0) ? 1u : 0u);
+                    TRACE(23 + i, tr_t, kb);
                 }
                 if (k1 == BN / 16) mma_commit_warp(bar(P2_ODONE + i));
             };

@@ -361,6 +361,48 @@ FA_DEV void mbar_arrive_warp(uint32_t bar) {
         : "memory");
 }
 
+// Four MMAs of one operand walk from one elected lane of a convergent warp,
+// with nothing between them: the descriptors of MMA i are those of MMA 0
+// plus O1/O2/O3 (16-byte units; a walk along K never carries out of the
+// 14-bit address field).  The first MMA accumulates into D iff acc0 != 0,
+// the other three always do.
+template <uint32_t O1, uint32_t O2, uint32_t O3>
+FA_DEV void mma_ss4_warp(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc, uint32_t acc0) {
+    asm volatile(
+        "{\n\t.reg .pred p, q, e;\n\t.reg .b64 a1, a2, a3, b1, b2, b3;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "setp.eq.b32 q, 0, 0;\n\t"
+        "add.s64 a1, %1, %5;\n\tadd.s64 a2, %1, %6;\n\tadd.s64 a3, %1, %7;\n\t"
+        "add.s64 b1, %2, %5;\n\tadd.s64 b2, %2, %6;\n\tadd.s64 b3, %2, %7;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a1, b1, %3, q;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a2, b2, %3, q;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a3, b3, %3, q;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(acc0), "n"(O1), "n"(O2), "n"(O3)
+        : "memory");
+}
+
+// Four TMEM-A MMAs from one elected lane: A steps by AO columns, the B
+// descriptor by BO (16-byte units) per MMA.
+template <uint32_t AO, uint32_t BO>
+FA_DEV void mma_ts4_warp(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc, uint32_t acc0) {
+    asm volatile(
+        "{\n\t.reg .pred p, q, e;\n\t.reg .b32 a1, a2, a3;\n\t.reg .b64 b1, b2, b3;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "setp.eq.b32 q, 0, 0;\n\t"
+        "add.u32 a1, %1, %5;\n\tadd.u32 a2, %1, %6;\n\tadd.u32 a3, %1, %7;\n\t"
+        "add.s64 b1, %2, %8;\n\tadd.s64 b2, %2, %9;\n\tadd.s64 b3, %2, %10;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], b1, %3, q;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a2], b2, %3, q;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a3], b3, %3, q;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(acc0), "n"(AO), "n"(2 * AO), "n"(3 * AO), "n"(BO), "n"(2 * BO),
+        "n"(3 * BO)
+        : "memory");
+}
+
 // Bounded wait by a whole warp; the result is made warp-uniform, so a warp
 // never diverges on it (an abort seen by one lane is seen by all).
 FA_DEV bool mbar_wait_warp(uint32_t bar, uint32_t parity, volatile int *abort_flag, int *err) {
