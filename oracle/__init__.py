@@ -44,6 +44,11 @@ def _load():
         lib.oracle_num_threads.restype = i32
         lib.oracle_attention.argtypes = [P, P, P] + [i32] * 7 + [i64] * 9 + [f64, i32, P, P]
         lib.oracle_attention.restype = i32
+        lib.oracle_attention_ext.argtypes = ([P, P, P] + [i32] * 7 + [i64] * 9 + [f64, i32, P, i64, i64, i64]
+                                             + [f64, f64, P, P, P])
+        lib.oracle_attention_ext.restype = i32
+        lib.oracle_alibi_slope.argtypes = [i32, i32, f64]
+        lib.oracle_alibi_slope.restype = f64
         lib.oracle_paged_gather.argtypes = [P, i32, i32, i32, i32, P, i32, P, i32, i32, P]
         lib.oracle_paged_gather.restype = i32
         lib.oracle_decode_paged.argtypes = [P, P, P, P, i32, P] + [i32] * 7 + [f64, P, P]
@@ -93,6 +98,52 @@ def attention(q, k, v, scale, causal=False):
                                   *qs, *ks, *vs, float(scale), int(bool(causal)), _ptr(o), _ptr(lse))
     if rc != 0:
         raise ValueError("oracle_attention rejected its arguments")
+    return o, lse
+
+
+def alibi_slope(h, Hq, max_bias):
+    """ALiBi slope of query head h (see oracle_alibi_slope)."""
+    return float(_load().oracle_alibi_slope(int(h), int(Hq), float(max_bias)))
+
+
+def attention_ext(q, k, v, scale, causal=False, mask=None, max_bias=0.0, softcap=0.0, sinks=None):
+    """Dense attention with the score modifiers (oracle_attention_ext).
+    mask: float16 array of shape [Bm, Hm, Sq, Sk] with Bm in {1, B} and
+    Hm in {1, Hq} (size-1 dims broadcast), or None.  sinks: [Hq] or None.
+    Returns (O [B,Hq,Sq,dv] float64, LSE [B,Hq,Sq] float64)."""
+    q, k, v = _u16(q), _u16(k), _u16(v)
+    B, Hq, Sq, dk = q.shape
+    _, Hkv, Sk, _ = k.shape
+    dv = v.shape[3]
+    for t in (q, k, v):
+        if t.size and t.strides[3] != 2:
+            raise ValueError("last dimension must be contiguous")
+    qs = [s // 2 for s in q.strides[:3]]
+    ks = [s // 2 for s in k.strides[:3]]
+    vs = [s // 2 for s in v.strides[:3]]
+    mptr, msb, msh, mss = None, 0, 0, 0
+    if mask is not None:
+        mask = np.ascontiguousarray(np.asarray(mask, dtype=np.float16))
+        Bm, Hm, Sqm, Skm = mask.shape
+        if Bm not in (1, B) or Hm not in (1, Hq) or Sqm != Sq or Skm != Sk:
+            raise ValueError("mask must be [1|B, 1|Hq, Sq, Sk]")
+        mask = mask.view(np.uint16)
+        msb = 0 if Bm == 1 else mask.strides[0] // 2
+        msh = 0 if Hm == 1 else mask.strides[1] // 2
+        mss = mask.strides[2] // 2
+        mptr = _ptr(mask)
+    sk = None
+    if sinks is not None:
+        sk = np.ascontiguousarray(np.asarray(sinks, dtype=np.float64))
+        if sk.shape != (Hq,):
+            raise ValueError("sinks must have one value per query head")
+    o = np.zeros((B, Hq, Sq, dv), np.float64)
+    lse = np.zeros((B, Hq, Sq), np.float64)
+    rc = _load().oracle_attention_ext(_ptr(q), _ptr(k), _ptr(v), B, Hq, Hkv, Sq, Sk, dk, dv, *qs, *ks, *vs,
+                                      float(scale), int(bool(causal)), mptr, msb, msh, mss, float(max_bias),
+                                      float(softcap), _ptr(sk), _ptr(o), _ptr(lse))
+    if rc != 0:
+        raise ValueError("oracle_attention_ext rejected its arguments")
     return o, lse
 
 

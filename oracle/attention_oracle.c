@@ -43,7 +43,12 @@
  *  - the max is per row (not one max shared by several rows);
  *  - LSE is in natural-log units;
  *  - a gather slot with row index < 0 is empty; key position defaults to the
- *    row index; a slot is visible iff kpos <= q_pos (no q_pos: all visible).
+ *    row index; a slot is visible iff kpos <= q_pos (no q_pos: all visible);
+ *  - score modifiers (oracle_attention_ext): the ALiBi constants m0, m1 and
+ *    n_head_log2 as stated at oracle_alibi_slope; softcap applies to the
+ *    scaled score as the page writes it (softcap * tanh(scale * dot)); a row
+ *    whose every kept score is -inf (mask) and which has no sink gives O = 0
+ *    and LSE = -inf; the LSE includes the sink term.
  *
  * Inputs are bf16 bit patterns (uint16), widened exactly to double.
  */
@@ -156,6 +161,140 @@ int oracle_attention(const uint16_t *q, const uint16_t *k, const uint16_t *v,
         }
         free(keys);
         free(vals);
+        free(orow);
+    }
+    return bad ? -1 : 0;
+}
+
+/*
+ * IEEE half-precision bit pattern -> double, exactly (sign, 5-bit exponent,
+ * 10-bit mantissa; subnormals, infinities and NaN included).
+ */
+static double f16_bits_to_double(uint16_t h)
+{
+    const int sign = (h >> 15) & 1;
+    const int e = (h >> 10) & 0x1f;
+    const int m = h & 0x3ff;
+    double v;
+    if (e == 0)
+        v = ldexp((double)m, -24);                 /* subnormal: m * 2^-14 / 2^10 */
+    else if (e == 31)
+        v = m ? NAN : INFINITY;
+    else
+        v = ldexp((double)(m + 1024), e - 25);     /* (1 + m/2^10) * 2^(e-15) */
+    return sign ? -v : v;
+}
+
+/*
+ * ALiBi slope of query head h, from "ggml-metal: FA tensor path"
+ * (kernel_flash_attn_ext_tensor_impl, the ALiBi block): heads below
+ * n_head_log2 take m0^(h+1), the rest m1^(2(h - n_head_log2) + 1).  The page
+ * receives m0, m1 and n_head_log2 from its host code without showing how
+ * they are formed; read here (and in the library) as n_head_log2 = the
+ * largest power of two <= Hq, m0 = 2^(-max_bias / n_head_log2),
+ * m1 = 2^(-max_bias / 2 / n_head_log2).  max_bias == 0 means slope 1.
+ */
+double oracle_alibi_slope(int h, int Hq, double max_bias)
+{
+    if (max_bias == 0.0) return 1.0;
+    int n2 = 1;
+    while (n2 * 2 <= Hq) n2 *= 2;
+    const double m0 = pow(2.0, -max_bias / n2);
+    const double m1 = pow(2.0, -max_bias / 2.0 / n2);
+    return h < n2 ? pow(m0, h + 1) : pow(m1, 2 * (h - n2) + 1);
+}
+
+/*
+ * Dense attention with the score modifiers of the llama.cpp tensor kernel
+ * ("ggml-metal: FA tensor path", kernel_flash_attn_ext_tensor_impl: the
+ * score loop, and the "final: sinks" block), applied in the page's order:
+ *
+ *   s_j  = scale * (q . k_j)
+ *   s_j  = softcap * tanh(s_j)                 if softcap != 0
+ *   s_j += slope_h * mask[b][h][i][j]          if mask != NULL
+ *   keys hidden by the causal rule are left out, as in oracle_attention;
+ *   a sink (if sinks != NULL) is one more logit sinks[h] in the softmax
+ *   denominator with no value row:
+ *     m = max(max_j s_j, sink),  l = sum_j exp(s_j - m) + exp(sink - m),
+ *     O = sum_j exp(s_j - m) v_j / l,  LSE = m + ln(l).
+ *   With no key left and no sink: O = 0, LSE = -inf.
+ *
+ * mask: IEEE f16 bit patterns; element (b, h, i, j) at
+ * b*m_sb + h*m_sh + i*m_ss + j (strides in elements, 0 broadcasts).
+ * sinks: one value per query head, natural-log units.
+ */
+int oracle_attention_ext(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                         int B, int Hq, int Hkv, int Sq, int Sk, int dk, int dv,
+                         int64_t q_sb, int64_t q_sh, int64_t q_ss,
+                         int64_t k_sb, int64_t k_sh, int64_t k_ss,
+                         int64_t v_sb, int64_t v_sh, int64_t v_ss,
+                         double scale, int causal,
+                         const uint16_t *mask, int64_t m_sb, int64_t m_sh, int64_t m_ss,
+                         double max_bias, double softcap, const double *sinks,
+                         double *o, double *lse)
+{
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || Sq < 0 || Sk < 0 ||
+        dk <= 0 || dv <= 0)
+        return -1;
+    const int group = Hq / Hkv;
+    const int n_bh = B * Hq;
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic)
+    for (int bh = 0; bh < n_bh; ++bh) {
+        const int b = bh / Hq, hq = bh % Hq;
+        const int hkv = hq / group;
+        const double slope = oracle_alibi_slope(hq, Hq, max_bias);
+        double *s = (double *)malloc(sizeof(double) * (size_t)(Sk > 0 ? Sk : 1));
+        int *vis = (int *)malloc(sizeof(int) * (size_t)(Sk > 0 ? Sk : 1));
+        double *orow = (double *)malloc(sizeof(double) * (size_t)dv);
+        if (!s || !vis || !orow) {
+#pragma omp atomic write
+            bad = 1;
+        } else {
+            const uint16_t *qb = q + b * q_sb + hq * q_sh;
+            for (int i = 0; i < Sq; ++i) {
+                const uint16_t *qr = qb + (int64_t)i * q_ss;
+                double m = -INFINITY;
+                int n = 0;
+                for (int j = 0; j < Sk; ++j) {
+                    vis[j] = !(causal && (int64_t)j > (int64_t)i + Sk - Sq);
+                    if (!vis[j]) continue;
+                    const uint16_t *kr = k + b * k_sb + hkv * k_sh + (int64_t)j * k_ss;
+                    double dot = 0.0;
+                    for (int d = 0; d < dk; ++d)
+                        dot += bf16_bits_to_double(qr[d]) * bf16_bits_to_double(kr[d]);
+                    double sj = scale * dot;
+                    if (softcap != 0.0) sj = softcap * tanh(sj);
+                    if (mask) sj += slope * f16_bits_to_double(mask[b * m_sb + hq * m_sh + (int64_t)i * m_ss + j]);
+                    s[j] = sj;
+                    if (sj > m) m = sj;
+                    ++n;
+                }
+                const double sink = sinks ? sinks[hq] : -INFINITY;
+                if (sink > m) m = sink;
+                for (int d = 0; d < dv; ++d) orow[d] = 0.0;
+                double l = 0.0, lse_i = -INFINITY;
+                if (m != -INFINITY) {
+                    for (int j = 0; j < Sk; ++j) {
+                        if (!vis[j]) continue;
+                        const double w = exp(s[j] - m);
+                        if (w == 0.0) continue;
+                        l += w;
+                        const uint16_t *vr = v + b * v_sb + hkv * v_sh + (int64_t)j * v_ss;
+                        for (int d = 0; d < dv; ++d) orow[d] += w * bf16_bits_to_double(vr[d]);
+                    }
+                    if (sinks) l += exp(sink - m);
+                    for (int d = 0; d < dv; ++d) orow[d] /= l;
+                    lse_i = m + log(l);
+                }
+                (void)n;
+                const int64_t r = ((int64_t)b * Hq + hq) * Sq + i;
+                if (o) memcpy(o + r * dv, orow, sizeof(double) * (size_t)dv);
+                if (lse) lse[r] = lse_i;
+            }
+        }
+        free(s);
+        free(vis);
         free(orow);
     }
     return bad ? -1 : 0;
