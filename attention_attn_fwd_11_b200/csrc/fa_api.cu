@@ -259,6 +259,13 @@ fa_status fa_fwd(const fa_fwd_params *p, void *stream) {
     const int ovec = p->o_dtype == FA_F32 ? 4 : 8;
     if (p->o_ss % ovec || p->o_sh % ovec || p->o_sb % ovec || p->o_ss < p->dv)
         return fail(FA_ERR_INVALID_ARG, "fa_fwd: o strides must be multiples of %d elements and o_ss >= dv", ovec);
+    if (!isfinite(p->max_bias) || p->max_bias < 0.f || !isfinite(p->softcap) || p->softcap < 0.f)
+        return fail(FA_ERR_INVALID_ARG, "fa_fwd: max_bias and softcap must be finite and >= 0");
+    if (p->mask && (!aligned16(p->mask) || p->m_ss % 8 || p->m_sh % 8 || p->m_sb % 8 || p->m_ss < p->Sk ||
+                    p->m_sh < 0 || p->m_sb < 0))
+        return fail(FA_ERR_INVALID_ARG,
+                    "fa_fwd: mask must be 16-byte aligned, its strides multiples of 8 elements, m_ss >= Sk");
+    if ((uintptr_t)p->sinks & 3u) return fail(FA_ERR_INVALID_ARG, "fa_fwd: sinks must be 4-byte aligned");
     if (!get_encoder()) return fail(FA_ERR_CUDA, "fa_fwd: cuTensorMapEncodeTiled is not available");
 
     fa::PrefillLaunch L;
@@ -294,6 +301,20 @@ fa_status fa_fwd(const fa_fwd_params *p, void *stream) {
     L.o_ss = p->o_ss;
     L.o_bf16 = p->o_dtype == FA_BF16;
     L.lse = p->lse;
+    L.mods.mask = static_cast<const __half *>(p->mask);
+    L.mods.m_sb = p->m_sb;
+    L.mods.m_sh = p->m_sh;
+    L.mods.m_ss = p->m_ss;
+    L.mods.softcap = p->softcap;
+    L.mods.sinks = p->sinks;
+    if (p->max_bias > 0.f) {  // ALiBi bases, as read in score_mods.cuh
+        int n2 = 1;
+        while (n2 * 2 <= p->Hq) n2 *= 2;
+        L.mods.n_head_log2 = n2;
+        L.mods.log2_m0 = -p->max_bias / (float)n2;
+        L.mods.log2_m1 = -p->max_bias / 2.f / (float)n2;
+    }
+    L.has_mods = p->mask || p->softcap > 0.f || p->sinks;
     cudaError_t e;
     if (p->dk <= 128) {
         int sms = 0;

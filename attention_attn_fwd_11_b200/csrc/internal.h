@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "score_mods.cuh"
+
 namespace fa {
 
 // ---- prefill -------------------------------------------------------------
@@ -19,6 +21,8 @@ struct PrefillLaunch {
     int64_t o_sb, o_sh, o_ss;
     int o_bf16;
     float *lse;
+    ScoreMods mods;  // all-zero: no modifiers
+    bool has_mods;   // a mask, a softcap or sinks is given
 };
 // Returns cudaSuccess or the launch error.
 cudaError_t launch_prefill(const PrefillLaunch &L, cudaStream_t stream);

@@ -33,6 +33,7 @@
 #include <math.h>
 
 #include "internal.h"
+#include "score_mods.cuh"
 #include "sm100.cuh"
 
 namespace fa {
@@ -41,7 +42,8 @@ static __device__ int g_prefill_err;
 
 struct PrefillArgs {
     int Hq, group, Sq, Sk;
-    float scale_log2;
+    float scale, scale_log2;
+    ScoreMods mods;  // used by the MODS instantiation only
     int causal;
     char *o;
     int64_t o_sb, o_sh, o_ss;
@@ -75,7 +77,7 @@ enum { B_QFULL = 0, B_DRAIN = 1, B_SFULL = 2, B_PREADY = 4, B_PVDONE = 6, B_RING
 
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale when the max grows by > 2^8
 
-template <int D, int BN, int NST>
+template <int D, int BN, int NST, bool MODS>
 __global__ void __launch_bounds__(192, 1)
 prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const PrefillArgs a) {
@@ -223,10 +225,21 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         const int row = qd * 32 + lane;           // row within the tile
         const int qrow = q0 + row;                // query index
         const uint32_t tl = tmem + ((uint32_t)(qd * 32) << 16);
-        const float c = a.scale_log2;
+        // With modifiers the scores are turned into base-2 units before the
+        // row max, so the exponent factor is 1.
+        // Only a mask or a softcap changes the scores themselves; sinks act in
+        // the epilogue alone.
+        const bool transform = MODS && (a.mods.mask != nullptr || a.mods.softcap != 0.f);
+        const float c = transform ? 1.f : a.scale_log2;
         // keys j < lim_all are visible to this row
         const int lim_all = a.causal ? min(a.Sk, qrow + a.Sk - a.Sq + 1) : a.Sk;
-        float m_run = -INFINITY, l_run = 0.f;
+        const float slope = MODS ? alibi_slope(a.mods, hq) : 1.f;
+        const __half *mrow = MODS ? mask_row(a.mods, b, hq, qrow, a.Sq) : nullptr;
+        (void)slope;
+        (void)mrow;
+        // l_run sums the fp32 weights (it gives the LSE); with modifiers l_o
+        // sums the bf16-rounded weights PV uses and normalises O.
+        float m_run = -INFINITY, l_run = 0.f, l_o = 0.f;
         bool ok = true;
         for (int t = 0; t < n_tiles; ++t) {
             const int buf = t & 1;
@@ -247,7 +260,9 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 for (int i = 0; i < BN; ++i) x[i] = __uint_as_float(r[i]);
             }
             const int lim = lim_all - t * BN;
-            if (lim < BN) {
+            if (transform) {
+                modify_scores<BN>(x, a.mods, a.scale, slope, mrow, t * BN, a.Sk, lim);
+            } else if (lim < BN) {
 #pragma unroll
                 for (int i = 0; i < BN; ++i)
                     if (i >= lim) x[i] = -INFINITY;
@@ -267,6 +282,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             if (need) {
                 alpha = ex2(m_run - m_new);
                 l_run *= alpha;
+                l_o *= alpha;
                 m_run = m_new;
             }
             if (t > 0 && __any_sync(0xffffffffu, need)) {
@@ -288,7 +304,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 }
             }
             const float msub = (m_run == -INFINITY) ? 0.f : m_run;
-            float s0 = 0.f, s1 = 0.f;
+            float s0 = 0.f, s1 = 0.f, r0 = 0.f, r1 = 0.f;
 #pragma unroll
             for (int ch = 0; ch < BN / 64; ++ch) {
                 uint32_t pk[32];
@@ -299,10 +315,15 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                     s0 += p0;
                     s1 += p1;
                     pk[i] = pack_bf16x2(p0, p1);
+                    if constexpr (MODS) {
+                        r0 += __uint_as_float(pk[i] << 16);
+                        r1 += __uint_as_float(pk[i] & 0xffff0000u);
+                    }
                 }
                 tmem_st32(tl + (uint32_t)(buf * BN + ch * 32), pk);
             }
             l_run += s0 + s1;
+            l_o += r0 + r1;
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(bar(B_PREADY + buf));
@@ -316,7 +337,12 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 have_o = false;
         }
         const bool store = qrow < a.Sq;
-        const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+        float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+        float lse2 = l_run > 0.f ? m_run + __log2f(l_run) : -INFINITY;
+        if constexpr (MODS) {
+            inv_l = l_o > 0.f ? 1.f / l_o : 0.f;
+            if (a.mods.sinks) inv_l = sink_normalise(m_run, l_run, l_o, a.mods.sinks[hq], &lse2);
+        }
         const int64_t ooff = (int64_t)b * a.o_sb + (int64_t)hq * a.o_sh + (int64_t)qrow * a.o_ss;
 #pragma unroll
         for (int ch = 0; ch < D / 32; ++ch) {
@@ -350,9 +376,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 }
             }
         }
-        if (store && a.lse)
-            a.lse[((int64_t)b * a.Hq + hq) * a.Sq + qrow] =
-                (l_run > 0.f) ? (m_run + __log2f(l_run)) * 0.69314718055994530942f : -INFINITY;
+        if (store && a.lse) a.lse[((int64_t)b * a.Hq + hq) * a.Sq + qrow] = lse2 * 0.69314718055994530942f;
     }
 
     tc_fence_before();
@@ -363,10 +387,10 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     }
 }
 
-template <int D, int BN, int NST>
+template <int D, int BN, int NST, bool MODS>
 static cudaError_t launch_cfg(const PrefillLaunch &L, cudaStream_t stream) {
     using C = PrefillCfg<D, BN, NST>;
-    auto kern = prefill_kernel<D, BN, NST>;
+    auto kern = prefill_kernel<D, BN, NST, MODS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     PrefillArgs a;
@@ -374,7 +398,9 @@ static cudaError_t launch_cfg(const PrefillLaunch &L, cudaStream_t stream) {
     a.group = L.Hq / L.Hkv;
     a.Sq = L.Sq;
     a.Sk = L.Sk;
+    a.scale = L.scale;
     a.scale_log2 = L.scale * 1.4426950408889634f;
+    a.mods = L.mods;
     a.causal = L.causal;
     a.o = static_cast<char *>(L.o);
     a.o_sb = L.o_sb;
@@ -389,9 +415,11 @@ static cudaError_t launch_cfg(const PrefillLaunch &L, cudaStream_t stream) {
 
 cudaError_t launch_prefill(const PrefillLaunch &L, cudaStream_t stream) {
     switch (L.dk) {
-        case 64: return launch_cfg<64, 128, 4>(L, stream);
-        case 128: return launch_cfg<128, 128, 2>(L, stream);
-        case 256: return launch_cfg<256, 64, 2>(L, stream);
+        case 64: return L.has_mods ? launch_cfg<64, 128, 4, true>(L, stream) : launch_cfg<64, 128, 4, false>(L, stream);
+        case 128:
+            return L.has_mods ? launch_cfg<128, 128, 2, true>(L, stream) : launch_cfg<128, 128, 2, false>(L, stream);
+        case 256:
+            return L.has_mods ? launch_cfg<256, 64, 2, true>(L, stream) : launch_cfg<256, 64, 2, false>(L, stream);
         default: return cudaErrorInvalidValue;
     }
 }

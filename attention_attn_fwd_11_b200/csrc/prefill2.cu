@@ -32,6 +32,7 @@
 #include <math.h>
 
 #include "internal.h"
+#include "score_mods.cuh"
 #include "sm100.cuh"
 
 namespace fa {
@@ -66,7 +67,8 @@ FA_DEV void trace(int ev, int t, int sub, int uc) {
 
 struct Prefill2Args {
     int Hq, group, Sq, Sk, BH, n_qp, n_units;
-    float scale_log2;
+    float scale, scale_log2;
+    ScoreMods mods;  // used by the MODS instantiation only
     int causal;
     char *o;
     int64_t o_sb, o_sh, o_ss;
@@ -188,7 +190,7 @@ FA_DEV bool p2_unit(const Prefill2Args &a, int round, UnitInfo &u) {
 constexpr int P2_THREADS = FA_P2_THREADS;
 constexpr int P2_SOFTMAX_WARP0 = P2_THREADS == 384 ? 4 : 2;
 
-template <int D>
+template <int D, bool MODS>
 __global__ void __launch_bounds__(P2_THREADS, 1)
 prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
@@ -492,7 +494,12 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         const uint32_t tl = tmem + ((uint32_t)(qd * 32) << 16);
         const uint32_t tS = tl + (uint32_t)(ti * BN);
         const uint32_t tO = tl + (uint32_t)(C::T_O + ti * D);
-        const float c = a.scale_log2;
+        // With modifiers the scores are turned into base-2 units before the
+        // row max, so the exponent factor is 1.
+        // Only a mask or a softcap changes the scores themselves; sinks act in
+        // the epilogue alone.
+        const bool transform = MODS && (a.mods.mask != nullptr || a.mods.softcap != 0.f);
+        const float c = transform ? 1.f : a.scale_log2;
         int scnt = 0, pv_base = 0, uc = 0;
         bool ok = true;
         UnitInfo u;
@@ -501,7 +508,15 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             const int n = u.nt(ti);
             const int qrow = u.q0 + 128 * ti + row;
             const int lim_all = a.causal ? min(a.Sk, qrow + a.Sk - a.Sq + 1) : a.Sk;
-            float m_run = -INFINITY, l_run = 0.f;
+            const float slope = MODS ? alibi_slope(a.mods, u.hq) : 1.f;
+            const __half *mrow = MODS ? mask_row(a.mods, u.b, u.hq, qrow, a.Sq) : nullptr;
+            (void)slope;
+            (void)mrow;
+            // l_run sums the fp32 weights (it gives the LSE).  With modifiers,
+            // l_o sums the bf16-rounded weights the PV MMA actually uses and
+            // normalises O, so that the few-key rows ALiBi and masks produce
+            // keep the accuracy of the many-key ones.
+            float m_run = -INFINITY, l_run = 0.f, l_o = 0.f;
             for (int t = 0; t < n; ++t) {
                 if (!mbar_wait(bar(P2_SFULL + ti), (uint32_t)scnt & 1u, abort_flag, &g_prefill2_err)) {
                     ok = false;
@@ -523,7 +538,9 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 }
                 if (lane == 0) TRACE(11 + ti, t, qd);
                 const int lim = lim_all - t * BN;
-                if (lim < BN) {
+                if (transform) {
+                    modify_scores<BN>(x, a.mods, a.scale, slope, mrow, t * BN, a.Sk, lim);
+                } else if (lim < BN) {
 #pragma unroll
                     for (int k = 0; k < BN; ++k)
                         if (k >= lim) x[k] = -INFINITY;
@@ -571,6 +588,7 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 if (need) {
                     alpha = ex2(m_run - m_new);
                     l_run *= alpha;
+                    l_o *= alpha;
                     m_run = m_new;
                 }
                 if (t > 0 && __any_sync(0xffffffffu, need)) {
@@ -601,7 +619,7 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                     if (lane == 0) TRACE(30, t, qd + 4 * ti);
                     const uint64_t c2 = f2_pack(c, c);
                     const uint64_t nm2 = f2_pack(-msub, -msub);
-                    uint64_t acc0 = f2_pack(0.f, 0.f), acc1 = acc0;
+                    uint64_t acc0 = f2_pack(0.f, 0.f), acc1 = acc0, accr = acc0;
 #pragma unroll
                     for (int g = 0; g < BN / 32; ++g) {
                         uint32_t pk[16];
@@ -624,6 +642,9 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                             else
                                 acc0 = f2_add(acc0, f2_pack(p0, p1));
                             pk[k] = pack_bf16x2(p0, p1);
+                            if constexpr (MODS)
+                                accr = f2_add(accr, f2_pack(__uint_as_float(pk[k] << 16),
+                                                            __uint_as_float(pk[k] & 0xffff0000u)));
                         }
                         tmem_st16(tS + (uint32_t)(g * 16), pk);
 #if FA_P2_SPLITP
@@ -640,6 +661,11 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                     f2_unpack(acc0, u0, u1);
                     f2_unpack(acc1, u2, u3);
                     l_run += (u0 + u1) + (u2 + u3);
+                    if constexpr (MODS) {
+                        float r0, r1;
+                        f2_unpack(accr, r0, r1);
+                        l_o += r0 + r1;
+                    }
                 }
 #else
                 float s0 = 0.f, s1 = 0.f;
@@ -704,10 +730,14 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             if (row == 0) TRACE(17 + ti, 0, 0);
             tc_fence_before();
             mbar_arrive(bar(P2_OFREE + ti));  // O of this tile may be overwritten by the next unit
-            const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+            float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+            float lse2 = l_run > 0.f ? m_run + __log2f(l_run) : -INFINITY;
+            if constexpr (MODS) {
+                inv_l = l_o > 0.f ? 1.f / l_o : 0.f;
+                if (a.mods.sinks) inv_l = sink_normalise(m_run, l_run, l_o, a.mods.sinks[u.hq], &lse2);
+            }
             if (qrow < a.Sq && a.lse)
-                a.lse[((int64_t)u.b * a.Hq + u.hq) * a.Sq + qrow] =
-                    (l_run > 0.f) ? (m_run + __log2f(l_run)) * 0.69314718055994530942f : -INFINITY;
+                a.lse[((int64_t)u.b * a.Hq + u.hq) * a.Sq + qrow] = lse2 * 0.69314718055994530942f;
             // Rows are written through a 16 KB staging tile (128 rows x 128
             // bytes, 128-byte swizzle) by TMA tensor stores; rows past Sq are
             // clipped by the store.
@@ -762,10 +792,10 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     }
 }
 
-template <int D>
+template <int D, bool MODS>
 static cudaError_t launch_p2(const PrefillLaunch &L, int num_sms, cudaStream_t stream) {
     using C = P2Cfg<D>;
-    auto kern = prefill2_kernel<D>;
+    auto kern = prefill2_kernel<D, MODS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     Prefill2Args a;
@@ -776,7 +806,9 @@ static cudaError_t launch_p2(const PrefillLaunch &L, int num_sms, cudaStream_t s
     a.BH = L.B * L.Hq;
     a.n_qp = (L.Sq + 255) / 256;
     a.n_units = a.BH * a.n_qp;
+    a.scale = L.scale;
     a.scale_log2 = L.scale * 1.4426950408889634f;
+    a.mods = L.mods;
     a.causal = L.causal;
     a.o = static_cast<char *>(L.o);
     a.o_sb = L.o_sb;
@@ -800,8 +832,9 @@ static cudaError_t launch_p2(const PrefillLaunch &L, int num_sms, cudaStream_t s
 
 cudaError_t launch_prefill2(const PrefillLaunch &L, int num_sms, cudaStream_t stream) {
     switch (L.dk) {
-        case 64: return launch_p2<64>(L, num_sms, stream);
-        case 128: return launch_p2<128>(L, num_sms, stream);
+        case 64: return L.has_mods ? launch_p2<64, true>(L, num_sms, stream) : launch_p2<64, false>(L, num_sms, stream);
+        case 128:
+            return L.has_mods ? launch_p2<128, true>(L, num_sms, stream) : launch_p2<128, false>(L, num_sms, stream);
         default: return cudaErrorInvalidValue;
     }
 }

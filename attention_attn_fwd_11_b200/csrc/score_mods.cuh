@@ -1,0 +1,137 @@
+// score_mods.cuh -- optional score modifiers of the prefill kernels:
+// additive f16 mask, ALiBi slopes, logit softcap and attention sinks.
+//
+// These follow the llama.cpp tensor kernel ("ggml-metal: FA tensor path",
+// kernel_flash_attn_ext_tensor_impl), in the order its score loop applies
+// them:
+//
+//   s  = scale * (q . k)
+//   s  = softcap * tanh(s)                 if softcap != 0
+//   s += slope_h * mask[b][h][i][j]        if a mask is given
+//
+// slope_h is 1 unless max_bias != 0.  Otherwise it is
+// m0^(h+1) for h < n_head_log2 and m1^(2(h - n_head_log2) + 1) above (the
+// page's ALiBi block); the host forms log2(m0) = -max_bias / n_head_log2 and
+// log2(m1) = -max_bias / 2 / n_head_log2 with n_head_log2 the largest power
+// of two <= Hq.  A sink (the page's "final: sinks" block) is one more logit
+// per head in the softmax denominator, with no value row.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "sm100.cuh"
+
+namespace fa {
+
+struct ScoreMods {
+    const __half *mask;        // NULL: no mask
+    int64_t m_sb, m_sh, m_ss;  // element strides (0 broadcasts); all multiples of 8
+    float log2_m0, log2_m1;    // ALiBi bases as base-2 logarithms
+    int n_head_log2;           // 0: ALiBi off (slope 1)
+    float softcap;             // 0: off
+    const float *sinks;        // NULL: no sinks; else [Hq], natural-log units
+};
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+FA_DEV float alibi_slope(const ScoreMods &m, int h) {
+    if (m.n_head_log2 == 0) return 1.f;
+    return h < m.n_head_log2 ? exp2f(m.log2_m0 * (float)(h + 1))
+                             : exp2f(m.log2_m1 * (float)(2 * (h - m.n_head_log2) + 1));
+}
+
+// Row of the mask for (b, h, query row i), or NULL (no mask, or a row past
+// the end of the queries).
+FA_DEV const __half *mask_row(const ScoreMods &m, int b, int h, int i, int Sq) {
+    if (!m.mask || i >= Sq) return nullptr;
+    return m.mask + (int64_t)b * m.m_sb + (int64_t)h * m.m_sh + (int64_t)i * m.m_ss;
+}
+
+// tanh(s) = 1 - 2 / (e^(2s) + 1), with e^(2s) from ex2: exact limits +-1 for
+// |s| large, absolute error of order 1e-7 elsewhere.
+FA_DEV float tanh_via_exp(float s) {
+    const float e = ex2(2.f * kLog2e * s);
+    return 1.f - 2.f * __frcp_rn(e + 1.f);
+}
+
+// Raw scores x[k] (unscaled q.k of keys key0 + k) -> base-2 scores
+// (modified score) * log2(e); keys k >= lim are hidden (-inf).  mrow: this
+// row's mask or NULL; keys at or past Sk are never read from it.
+// Raw scores x[k] (unscaled q.k of keys key0 + k) -> base-2 scores
+// (modified score) * log2(e); keys k >= lim are hidden (-inf).  mrow: this
+// row's mask or NULL; keys at or past Sk are never read from it.  The mask
+// is read 64 keys at a time: a chunk wholly inside the row issues its eight
+// 16-byte loads before the first is used.
+template <int BN>
+FA_DEV void modify_scores(float (&x)[BN], const ScoreMods &m, float scale, float slope, const __half *mrow,
+                          int key0, int Sk, int lim) {
+    static_assert(BN % 64 == 0, "tile width");
+    const float cs = scale * kLog2e;   // raw score -> base-2 units, without softcap
+    const float cm = slope * kLog2e;   // mask value -> base-2 units
+    const uint64_t cs2 = f2_pack(cs, cs), cm2 = f2_pack(cm, cm);
+#pragma unroll
+    for (int h = 0; h < BN / 64; ++h) {
+        const int kc = key0 + 64 * h;
+        const bool whole = mrow && kc + 64 <= Sk;
+        uint4 w[8];
+        if (whole) {
+#pragma unroll
+            for (int g = 0; g < 8; ++g) w[g] = __ldg(reinterpret_cast<const uint4 *>(mrow + kc + 8 * g));
+        }
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+            uint32_t mw[4] = {0u, 0u, 0u, 0u};  // four f16 pairs (zero: no mask value)
+            if (whole) {
+                mw[0] = w[g].x;
+                mw[1] = w[g].y;
+                mw[2] = w[g].z;
+                mw[3] = w[g].w;
+            } else if (mrow) {  // the row's last, partial chunk: element loads up to Sk
+                const uint16_t *mr = reinterpret_cast<const uint16_t *>(mrow);
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    if (kc + 8 * g + j < Sk) mw[j >> 1] |= (uint32_t)mr[kc + 8 * g + j] << (16 * (j & 1));
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int k = 64 * h + 8 * g + 2 * j;
+                const float2 mf = __half22float2(*reinterpret_cast<const __half2 *>(&mw[j]));
+                uint64_t y;
+                if (m.softcap != 0.f) {
+                    const float s0 = m.softcap * tanh_via_exp(x[k] * scale);
+                    const float s1 = m.softcap * tanh_via_exp(x[k + 1] * scale);
+                    y = f2_fma(f2_pack(mf.x, mf.y), cm2, f2_mul(f2_pack(s0, s1), f2_pack(kLog2e, kLog2e)));
+                } else {
+                    y = f2_fma(f2_pack(x[k], x[k + 1]), cs2, f2_mul(f2_pack(mf.x, mf.y), cm2));
+                }
+                f2_unpack(y, x[k], x[k + 1]);
+            }
+        }
+    }
+    if (lim < BN) {
+#pragma unroll
+        for (int k = 0; k < BN; ++k)
+            if (k >= lim) x[k] = -INFINITY;
+    }
+}
+
+// Epilogue with a sink: O was accumulated relative to m_run (base 2);
+// l_run is the fp32 weight sum and l_o the sum of the bf16-rounded weights O
+// was built from.  Returns the factor that normalises O and, in *lse2, the
+// base-2 log-sum-exp including the sink.
+FA_DEV float sink_normalise(float m_run, float l_run, float l_o, float sink_nat, float *lse2) {
+    const float sk = sink_nat * kLog2e;
+    const float mm = fmaxf(m_run, sk);
+    if (mm == -INFINITY) {
+        *lse2 = -INFINITY;
+        return 0.f;
+    }
+    const float a_o = l_run > 0.f ? ex2(m_run - mm) : 0.f;
+    const float e_s = ex2(sk - mm);
+    *lse2 = mm + __log2f(l_run * a_o + e_s);
+    return a_o / (l_o * a_o + e_s);
+}
+
+}  // namespace fa

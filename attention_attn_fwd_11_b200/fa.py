@@ -32,7 +32,9 @@ class FwdParams(ctypes.Structure):
                 ("k_sb", _i64), ("k_sh", _i64), ("k_ss", _i64),
                 ("v_sb", _i64), ("v_sh", _i64), ("v_ss", _i64),
                 ("o_sb", _i64), ("o_sh", _i64), ("o_ss", _i64),
-                ("scale", ctypes.c_float), ("causal", _i32), ("o_dtype", _i32)]
+                ("scale", ctypes.c_float), ("causal", _i32), ("o_dtype", _i32),
+                ("mask", _vp), ("m_sb", _i64), ("m_sh", _i64), ("m_ss", _i64),
+                ("max_bias", ctypes.c_float), ("softcap", ctypes.c_float), ("sinks", _vp)]
 
 
 class PagedParams(ctypes.Structure):
@@ -116,7 +118,7 @@ def _odt(dtype):
 
 # ------------------------------------------------------------------ prefill --
 
-def fwd_params(q, k, v, o, lse, scale, causal):
+def fwd_params(q, k, v, o, lse, scale, causal, mask=None, max_bias=0.0, softcap=0.0, sinks=None):
     B, Hq, Sq, dk = q.shape
     _, Hkv, Sk, dv = v.shape
     p = FwdParams()
@@ -129,14 +131,34 @@ def fwd_params(q, k, v, o, lse, scale, causal):
     p.scale = scale
     p.causal = 1 if causal else 0
     p.o_dtype = _odt(o.dtype)
+    if mask is not None:  # [Bm, Hm, Sq, Sk] f16; a size-1 batch or head dim broadcasts
+        p.mask = _ptr(mask)
+        p.m_sb = 0 if mask.shape[0] == 1 else mask.stride(0)
+        p.m_sh = 0 if mask.shape[1] == 1 else mask.stride(1)
+        p.m_ss = mask.stride(2)
+    p.max_bias = max_bias
+    p.softcap = softcap
+    p.sinks = _ptr(sinks)
     return p
 
 
-def fwd(q, k, v, scale=None, causal=False, out=None, return_lse=True, out_dtype=torch.float32, stream=None):
+def fwd(q, k, v, scale=None, causal=False, out=None, return_lse=True, out_dtype=torch.float32, stream=None,
+        mask=None, max_bias=0.0, softcap=0.0, sinks=None):
     """O = softmax(scale * Q K^T + mask) V.  q [B,Hq,Sq,dk], k [B,Hkv,Sk,dk],
     v [B,Hkv,Sk,dv] bf16 CUDA tensors (any strides, head dim contiguous).
+    Score modifiers (see fa_fwd in include/fa.h): mask [1|B, 1|Hq, Sq, Sk]
+    float16 CUDA tensor with a contiguous last dim, max_bias (ALiBi slopes
+    applied to the mask), softcap, sinks [Hq] float32 CUDA tensor.
     Returns (O [B,Hq,Sq,dv], LSE [B,Hq,Sq] fp32 or None)."""
     _need_cuda(q, k, v)
+    if mask is not None:
+        _need_cuda(mask)
+        if mask.dtype != torch.float16 or mask.dim() != 4 or mask.stride(3) != 1:
+            raise ValueError("mask must be a 4-D float16 tensor with a contiguous last dim")
+    if sinks is not None:
+        _need_cuda(sinks)
+        if sinks.dtype != torch.float32 or sinks.shape != (q.shape[1],) or not sinks.is_contiguous():
+            raise ValueError("sinks must be a contiguous float32 tensor of shape [Hq]")
     for t in (q, k, v):
         if t.dtype != torch.bfloat16 or t.dim() != 4 or t.stride(3) != 1:
             raise ValueError("q, k, v must be 4-D bf16 with a contiguous last dim")
@@ -147,7 +169,8 @@ def fwd(q, k, v, scale=None, causal=False, out=None, return_lse=True, out_dtype=
     if out is None:
         out = torch.empty((B, Hq, Sq, dv), device=q.device, dtype=out_dtype)
     lse = torch.empty((B, Hq, Sq), device=q.device, dtype=torch.float32) if return_lse else None
-    _check(load().fa_fwd(ctypes.byref(fwd_params(q, k, v, out, lse, scale, causal)), _stream(stream)))
+    params = fwd_params(q, k, v, out, lse, scale, causal, mask, max_bias, softcap, sinks)
+    _check(load().fa_fwd(ctypes.byref(params), _stream(stream)))
     return out, lse
 
 

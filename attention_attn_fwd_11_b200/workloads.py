@@ -8,7 +8,8 @@ CUDA path and the CPU oracle can both be fed from it without sharing code.
 Recipe: every bf16 tensor is drawn as float32 ``torch.randn`` on a CPU
 ``torch.Generator`` seeded per tensor and rounded to bf16 (round to nearest
 even).  Seeds for workload ``c``: Q = 1000 + c, K = 2000 + c, V = 3000 + c,
-structure (lengths, block ids, selected rows) = 4000 + c.
+structure (lengths, block ids, selected rows) = 4000 + c, additive masks =
+5000 + c, sink logits = 6000 + c.
 """
 from __future__ import annotations
 
@@ -69,6 +70,48 @@ def prefill_inputs(c: PrefillCase):
 TINY_FULL = PrefillCase("tiny_full_b1_h2_s256_d64", 1, 2, 2, 256, 256, 64, 64, False, seed=1)
 CAUSAL_MHA = PrefillCase("causal_mha_b2_h16_s2048_d128", 2, 16, 16, 2048, 2048, 128, 128, True, seed=2)
 GQA_FULL = PrefillCase("gqa_full_b1_hq32_hkv8_s4096_d256", 1, 32, 8, 4096, 4096, 256, 256, False, seed=3)
+
+
+# ------------------------------------------------ prefill score modifiers --
+# Inputs for the optional score modifiers (additive f16 mask, ALiBi, softcap,
+# sinks).  Random numbers and position distances only; the modifiers' own
+# arithmetic lives in the kernels and in the oracle.
+
+def random_mask(Bm: int, Hm: int, Sq: int, Sk: int, seed: int, scale: float = 2.0, hide_frac: float = 0.1):
+    """[Bm, Hm, Sq, Sk] float16: N(0, scale^2) values with a seeded fraction
+    of entries set to -inf (hidden keys)."""
+    g = torch.Generator().manual_seed(5000 + seed)
+    m = torch.randn(Bm, Hm, Sq, Sk, generator=g) * scale
+    hide = torch.rand(Bm, Hm, Sq, Sk, generator=g) < hide_frac
+    m[hide] = -math.inf
+    return m.to(torch.float16)
+
+
+def distance_mask(Sq: int, Sk: int, causal: bool = True):
+    """[1, 1, Sq, Sk] float16 position distances for ALiBi: key j of query i
+    (bottom-right aligned, query position i + Sk - Sq) holds -(pos_i - j);
+    with causal, keys after the query are -inf."""
+    i = torch.arange(Sq).view(Sq, 1) + (Sk - Sq)
+    j = torch.arange(Sk).view(1, Sk)
+    d = (j - i).to(torch.float32)
+    if causal:
+        d[j > i] = -math.inf
+    else:
+        d = -d.abs()
+    return d.view(1, 1, Sq, Sk).to(torch.float16)
+
+
+def random_sinks(Hq: int, seed: int):
+    """[Hq] float32 sink logits, N(0, 1)."""
+    g = torch.Generator().manual_seed(6000 + seed)
+    return torch.randn(Hq, generator=g)
+
+
+# C2's shape with every modifier on: ALiBi (max_bias 8) over a head-shared
+# distance mask, softcap 30, one sink per head.
+MODS_C2 = PrefillCase("causal_mha_mods_b2_h16_s2048_d128", 2, 16, 16, 2048, 2048, 128, 128, True, seed=2)
+MODS_C2_MAX_BIAS = 8.0
+MODS_C2_SOFTCAP = 30.0
 
 
 # ------------------------------------------------------------ paged decode --

@@ -210,17 +210,27 @@ def sum_over_ranks(torch, dist, x, device="cuda"):
 
 def prefill_workload(torch, fa, W_, c, l2):
     q0, k0, v0 = W_.prefill_inputs(c)
+    mods = c.name == W_.MODS_C2.name  # every score modifier on: ALiBi distance mask, softcap, sinks
+    m0 = W_.distance_mask(c.Sq, c.Sk, causal=True) if mods else None
+    s0 = W_.random_sinks(c.Hq, seed=c.seed) if mods else None
     foot = (q0.numel() + k0.numel() + v0.numel()) * 2 + c.B * c.Hq * c.Sq * (c.dv * 4 + 4)
+    if mods:
+        foot += m0.numel() * 2
     n = rotation_copies(foot, l2)
     bufs = []
     for i in range(n):
         q, k, v = q0.cuda(), k0.cuda(), v0.cuda()
         o = torch.empty(c.B, c.Hq, c.Sq, c.dv, device="cuda")
         lse = torch.empty(c.B, c.Hq, c.Sq, device="cuda")
-        bufs.append((q, k, v, o, lse))
+        extra = (m0.cuda(), s0.cuda()) if mods else (None, None)
+        bufs.append((q, k, v, o, lse) + extra)
     import ctypes
     lib = fa.load()
-    params = [fa.fwd_params(q, k, v, o, lse, c.scale, c.causal) for (q, k, v, o, lse) in bufs]
+    if mods:
+        params = [fa.fwd_params(q, k, v, o, lse, c.scale, c.causal, mask=m, max_bias=W_.MODS_C2_MAX_BIAS,
+                                softcap=W_.MODS_C2_SOFTCAP, sinks=sk) for (q, k, v, o, lse, m, sk) in bufs]
+    else:
+        params = [fa.fwd_params(q, k, v, o, lse, c.scale, c.causal) for (q, k, v, o, lse, _, _) in bufs]
 
     def launch(i):
         st = lib.fa_fwd(ctypes.byref(params[i]), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
@@ -372,7 +382,8 @@ def run_only(args):
 
     torch.cuda.set_device(0)
     l2 = torch.cuda.get_device_properties(0).L2_cache_size
-    table = {c.name: c for c in (W_.TINY_FULL, W_.CAUSAL_MHA, W_.GQA_FULL, W_.PAGED_GQA, W_.LATENT_SPARSE)}
+    table = {c.name: c for c in (W_.TINY_FULL, W_.CAUSAL_MHA, W_.GQA_FULL, W_.MODS_C2, W_.PAGED_GQA,
+                                 W_.LATENT_SPARSE)}
     if args.only not in table:
         raise SystemExit("unknown workload %r; one of %s" % (args.only, sorted(table)))
     c = table[args.only]
@@ -516,7 +527,7 @@ def main():
     if not args.no_secondary:
         wl = {}
         Ks = 200
-        for cc in (W_.TINY_FULL, W_.GQA_FULL):
+        for cc in (W_.TINY_FULL, W_.GQA_FULL, W_.MODS_C2):
             launch, ncopy, foot, kpl = prefill_workload(torch, fa, W_, cc, l2)
             ms2, st2 = time_graph(torch, launch, ncopy, Ks, Wm, dist)
             ms2 = max_over_ranks(torch, dist, ms2)

@@ -82,6 +82,28 @@ enum {
  * attention).
  * Supported: dk == dv in {64, 128, 256}; anything else is FA_ERR_UNSUPPORTED.
  * Sq == 0 or B == 0 is a no-op; Sk == 0 writes O = 0, LSE = -inf.
+ *
+ * Score modifiers (all off when zero / NULL), as the llama.cpp tensor
+ * kernel applies them ("ggml-metal: FA tensor path",
+ * kernel_flash_attn_ext_tensor_impl: the score loop, the ALiBi block and the
+ * "final: sinks" block), in this order on every visible key:
+ *   s = scale * q.k;  if softcap > 0: s = softcap * tanh(s);
+ *   if mask: s += slope_h * mask[b][h][i][j]
+ * mask: NULL, or IEEE f16 values; element (b, h, i, j) at
+ *   b*m_sb + h*m_sh + i*m_ss + j (elements; m_sb / m_sh may be 0 to
+ *   broadcast; all three multiples of 8, m_ss >= Sk, 16-byte aligned base).
+ *   -inf hides a key.  The causal rule, if set, applies as well.
+ * max_bias: ALiBi.  0 gives slope 1; > 0 gives query head h the slope m0^(h+1)
+ *   (h < n) or m1^(2(h-n)+1) (h >= n), with n the largest power of two
+ *   <= Hq, m0 = 2^(-max_bias/n), m1 = 2^(-max_bias/(2n)).  The slope scales
+ *   the mask (which then holds position distances); without a mask it has
+ *   no effect.
+ * sinks: NULL, or [Hq] fp32 logits (natural-log units): one more term
+ *   exp(sink_h) in each row's softmax denominator, with no value row.  The
+ *   returned LSE includes it; a row with no visible key then gets O = 0 and
+ *   LSE = sink_h.
+ * These run in the same kernels.  Each row loads its 2-byte mask values per
+ * key tile straight from global memory.
  */
 typedef struct {
     const void *q, *k, *v;
@@ -95,6 +117,12 @@ typedef struct {
     float scale;
     int causal;
     int o_dtype; /* fa_dtype */
+    /* score modifiers (zero / NULL: off) */
+    const void *mask; /* f16 */
+    int64_t m_sb, m_sh, m_ss;
+    float max_bias;
+    float softcap;
+    const float *sinks;
 } fa_fwd_params;
 
 fa_status fa_fwd(const fa_fwd_params *p, void *stream);

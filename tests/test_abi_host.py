@@ -58,6 +58,15 @@ def fwd_params(**kw):
     (dict(o_dtype=7), fa.FA_ERR_INVALID_ARG),
     (dict(o_ss=130), fa.FA_ERR_INVALID_ARG),
     (dict(Sq=-1), fa.FA_ERR_INVALID_ARG),
+    # score modifiers
+    (dict(softcap=-1.0), fa.FA_ERR_INVALID_ARG),
+    (dict(softcap=float("inf")), fa.FA_ERR_INVALID_ARG),
+    (dict(max_bias=-2.0), fa.FA_ERR_INVALID_ARG),
+    (dict(mask=8, m_ss=128), fa.FA_ERR_INVALID_ARG),          # mask base not 16-byte aligned
+    (dict(mask=16, m_ss=130), fa.FA_ERR_INVALID_ARG),         # row stride not a multiple of 8
+    (dict(mask=16, m_ss=120), fa.FA_ERR_INVALID_ARG),         # row stride < Sk
+    (dict(mask=16, m_ss=128, m_sh=4), fa.FA_ERR_INVALID_ARG),  # head stride not a multiple of 8
+    (dict(sinks=2), fa.FA_ERR_INVALID_ARG),                   # sinks not 4-byte aligned
 ])
 def test_fwd_rejects(kw, status):
     lib = fa.load()
