@@ -49,6 +49,7 @@ NCU_TRAFFIC = {
     # under profiles/ named for the kernel and workload gives the capture.
     "causal_mha_b2_h16_s2048_d128": 53822720,
     "gqa_full_b1_hq32_hkv8_s4096_d256": 215805440,
+    "causal_mha_mods_b2_h16_s2048_d128": 59766528,
     "paged_gqa_b64_hq32_hkv8_d128_bs64": 1237055008,
     "latent_sparse_t32_hq128_dk576_dv512_top2048": 45249792,
 }
