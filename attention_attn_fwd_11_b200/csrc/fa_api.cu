@@ -243,8 +243,13 @@ fa_status fa_fwd(const fa_fwd_params *p, void *stream) {
     if (p->B < 0 || p->Hq <= 0 || p->Hkv <= 0 || p->Sq < 0 || p->Sk < 0)
         return fail(FA_ERR_INVALID_ARG, "fa_fwd: need B >= 0, Hq > 0, Hkv > 0, Sq >= 0, Sk >= 0");
     if (p->Hq % p->Hkv != 0) return fail(FA_ERR_INVALID_ARG, "fa_fwd: Hq (%d) %% Hkv (%d) != 0", p->Hq, p->Hkv);
-    if (p->dk != p->dv || (p->dk != 64 && p->dk != 128 && p->dk != 256))
-        return fail(FA_ERR_UNSUPPORTED, "fa_fwd: supported dk = dv in {64, 128, 256} (got %d/%d)", p->dk, p->dv);
+    const bool pair_ok = (p->dk == p->dv && (p->dk == 64 || p->dk == 128 || p->dk == 256)) ||
+                         (p->dk == 192 && (p->dv == 128 || p->dv == 192)) || (p->dk == 320 && p->dv == 256);
+    if (!pair_ok)
+        return fail(FA_ERR_UNSUPPORTED,
+                    "fa_fwd: supported (dk, dv) = (64, 64), (128, 128), (256, 256), (192, 128), (320, 256); got "
+                    "(%d, %d)",
+                    p->dk, p->dv);
     if (!finite_pos(p->scale)) return fail(FA_ERR_INVALID_ARG, "fa_fwd: scale must be finite and > 0");
     if (p->o_dtype != FA_F32 && p->o_dtype != FA_BF16) return fail(FA_ERR_INVALID_ARG, "fa_fwd: o_dtype");
     if ((long long)p->B * p->Hq > 0x7fffffffLL || p->Sq > (1 << 30) || p->Sk > (1 << 30))
@@ -270,7 +275,10 @@ fa_status fa_fwd(const fa_fwd_params *p, void *stream) {
 
     fa::PrefillLaunch L;
     memset(&L, 0, sizeof L);
-    const int box_k = p->dk == 256 ? 64 : 128;
+    // The two-tile kernel takes dk = dv <= 128 (K/V tiles of 128 keys); the
+    // one-tile kernel the rest (64-key tiles, except 128 for (192, 128)).
+    const bool two_tile = p->dk == p->dv && p->dk <= 128;
+    const int box_k = two_tile || (p->dk == 192 && p->dv == 128) ? 128 : 64;
     fa_status st;
     st = encode_4d(&L.tmQ, p->q, p->dk, p->Sq, p->Hq, p->B, p->q_ss, p->q_sh, p->q_sb, 128, "fa_fwd q");
     if (st != FA_OK) return st;
@@ -281,7 +289,7 @@ fa_status fa_fwd(const fa_fwd_params *p, void *stream) {
     if (st != FA_OK) return st;
     st = encode_4d(&L.tmV, vb, p->dv, p->Sk, p->Hkv, p->B, p->v_ss, p->v_sh, p->v_sb, box_k, "fa_fwd v");
     if (st != FA_OK) return st;
-    if (p->dk <= 128) {  // the two-tile kernel writes O with TMA stores
+    if (two_tile) {  // the two-tile kernel writes O with TMA stores
         st = encode_4d(&L.tmO, p->o, p->dv, p->Sq, p->Hq, p->B, p->o_ss, p->o_sh, p->o_sb, 128, "fa_fwd o",
                        p->o_dtype == FA_F32 ? 4 : 2);
         if (st != FA_OK) return st;
@@ -316,7 +324,7 @@ fa_status fa_fwd(const fa_fwd_params *p, void *stream) {
     }
     L.has_mods = p->mask || p->softcap > 0.f || p->sinks;
     cudaError_t e;
-    if (p->dk <= 128) {
+    if (two_tile) {
         int sms = 0;
         e = num_sms(&sms);
         if (e == cudaSuccess) e = fa::launch_prefill2(L, sms, static_cast<cudaStream_t>(stream));

@@ -51,24 +51,27 @@ struct PrefillArgs {
     float *lse;
 };
 
-template <int D, int BN, int NST>
+// DK: head dim of Q and K; DV: head dim of V and O.
+template <int DK, int DV, int BN, int NST>
 struct PrefillCfg {
     static constexpr int BM = 128;
-    static constexpr int NCH = D / 64;            // 128-byte chunks of the head dim
+    static constexpr int NCHK = DK / 64;          // 128-byte chunks of a Q or K row
+    static constexpr int NCHV = DV / 64;          // 128-byte chunks of a V row
     static constexpr int Q_CHUNK = BM * 128;      // bytes of one chunk of Q
     static constexpr int KV_CHUNK = BN * 128;     // bytes of one chunk of K or V
-    static constexpr int Q_BYTES = BM * D * 2;
-    static constexpr int KV_BYTES = BN * D * 2;
+    static constexpr int Q_BYTES = BM * DK * 2;
+    static constexpr int K_BYTES = BN * DK * 2;
+    static constexpr int V_BYTES = BN * DV * 2;
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_K = Q_BYTES;
-    static constexpr int OFF_V = OFF_K + NST * KV_BYTES;
-    static constexpr int OFF_BAR = OFF_V + NST * KV_BYTES;
+    static constexpr int OFF_V = OFF_K + NST * K_BYTES;
+    static constexpr int OFF_BAR = OFF_V + NST * V_BYTES;
     static constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;  // barriers + alignment slack
     static constexpr int TMEM_COLS = 512;
     static constexpr int T_O = 2 * BN;            // TMEM column of O (S0 at 0, S1 at BN)
-    static_assert(D % 64 == 0 && D <= 256, "head dim");
+    static_assert(DK % 64 == 0 && DV % 64 == 0 && DV <= 256, "head dims");
     static_assert(BN % 64 == 0 && BN <= 128, "key tile");
-    static_assert(2 * BN + D <= TMEM_COLS, "TMEM budget");
+    static_assert(2 * BN + DV <= TMEM_COLS, "TMEM budget");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
@@ -77,11 +80,11 @@ enum { B_QFULL = 0, B_DRAIN = 1, B_SFULL = 2, B_PREADY = 4, B_PVDONE = 6, B_RING
 
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale when the max grows by > 2^8
 
-template <int D, int BN, int NST, bool MODS>
+template <int DK, int DV, int BN, int NST, bool MODS>
 __global__ void __launch_bounds__(192, 1)
 prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const PrefillArgs a) {
-    using C = PrefillCfg<D, BN, NST>;
+    using C = PrefillCfg<DK, DV, BN, NST>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
@@ -147,23 +150,23 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             prefetch_tmap(&tmV);
             mbar_arrive_expect_tx(bar(B_QFULL), C::Q_BYTES);
 #pragma unroll
-            for (int c = 0; c < C::NCH; ++c)
+            for (int c = 0; c < C::NCHK; ++c)
                 tma_load_4d(sQ + c * C::Q_CHUNK, &tmQ, bar(B_QFULL), c * 64, q0, hq, b);
             int issued_k = 0, issued_v = 0;
             for (int t = 0; t < n_tiles; ++t) {
                 const int s = t % NST;
                 const uint32_t ph = (uint32_t)(t / NST) & 1u;
                 if (!mbar_wait(k_empty(s), ph ^ 1u, abort_flag, &g_prefill_err)) break;
-                mbar_arrive_expect_tx(k_full(s), C::KV_BYTES);
+                mbar_arrive_expect_tx(k_full(s), C::K_BYTES);
 #pragma unroll
-                for (int c = 0; c < C::NCH; ++c)
-                    tma_load_4d(sK + s * C::KV_BYTES + c * C::KV_CHUNK, &tmK, k_full(s), c * 64, t * BN, hkv, b);
+                for (int c = 0; c < C::NCHK; ++c)
+                    tma_load_4d(sK + s * C::K_BYTES + c * C::KV_CHUNK, &tmK, k_full(s), c * 64, t * BN, hkv, b);
                 issued_k = t + 1;
                 if (!mbar_wait(v_empty(s), ph ^ 1u, abort_flag, &g_prefill_err)) break;
-                mbar_arrive_expect_tx(v_full(s), C::KV_BYTES);
+                mbar_arrive_expect_tx(v_full(s), C::V_BYTES);
 #pragma unroll
-                for (int c = 0; c < C::NCH; ++c)
-                    tma_load_4d(sV + s * C::KV_BYTES + c * C::KV_CHUNK, &tmV, v_full(s), c * 64, t * BN, hkv, b);
+                for (int c = 0; c < C::NCHV; ++c)
+                    tma_load_4d(sV + s * C::V_BYTES + c * C::KV_CHUNK, &tmV, v_full(s), c * 64, t * BN, hkv, b);
                 issued_v = t + 1;
             }
             if (*abort_flag) {
@@ -181,7 +184,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         // MMA and commit.
         if (n_tiles > 0) {
             constexpr uint32_t idesc_qk = idesc_bf16_f32(128, BN, false, false);
-            constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, false, true);
+            constexpr uint32_t idesc_pv = idesc_bf16_f32(128, DV, false, true);
             const uint32_t tO = tmem + C::T_O;
             auto issue_qk = [&](int t) -> bool {
                 const int s = t % NST;
@@ -189,9 +192,9 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 tc_fence_after();
                 const uint32_t tS = tmem + (uint32_t)((t & 1) * BN);
                 const uint64_t ad0 = sdesc_sw128(sQ, 16, 1024);
-                const uint64_t bd0 = sdesc_sw128(sK + s * C::KV_BYTES, 16, 1024);
+                const uint64_t bd0 = sdesc_sw128(sK + s * C::K_BYTES, 16, 1024);
 #pragma unroll
-                for (int c = 0; c < C::NCH; ++c)  // four 16-wide K steps per 64-column chunk
+                for (int c = 0; c < C::NCHK; ++c)  // four 16-wide K steps per 64-column chunk
                     mma_ss4_warp<2, 4, 6>(tS, ad0 + (uint64_t)((c * C::Q_CHUNK) >> 4),
                                           bd0 + (uint64_t)((c * C::KV_CHUNK) >> 4), idesc_qk, c > 0 ? 1u : 0u);
                 mma_commit_warp(k_empty(s));
@@ -206,7 +209,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 if (!mbar_wait_warp(v_full(s), (uint32_t)(t / NST) & 1u, abort_flag, &g_prefill_err)) break;
                 tc_fence_after();
                 const uint32_t tP = tmem + (uint32_t)((t & 1) * BN);
-                const uint64_t bd0 = sdesc_sw128(sV + s * C::KV_BYTES, C::KV_CHUNK, 1024);
+                const uint64_t bd0 = sdesc_sw128(sV + s * C::V_BYTES, C::KV_CHUNK, 1024);
 #pragma unroll
                 for (int kb = 0; kb < BN / 16; kb += 4)
                     mma_ts4_warp<8, (2048 >> 4)>(tO, tP + (uint32_t)(kb * 8), bd0 + (uint64_t)(kb * (2048 >> 4)),
@@ -294,7 +297,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 tc_fence_after();
                 uint32_t r[32];
 #pragma unroll
-                for (int ch = 0; ch < D / 32; ++ch) {
+                for (int ch = 0; ch < DV / 32; ++ch) {
                     tmem_ld32(tl + (uint32_t)(C::T_O + ch * 32), r);
                     tmem_wait_ld();
                     reg_fence(r);
@@ -345,7 +348,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         }
         const int64_t ooff = (int64_t)b * a.o_sb + (int64_t)hq * a.o_sh + (int64_t)qrow * a.o_ss;
 #pragma unroll
-        for (int ch = 0; ch < D / 32; ++ch) {
+        for (int ch = 0; ch < DV / 32; ++ch) {
             uint32_t r[32];
             if (have_o) {
                 tmem_ld32(tl + (uint32_t)(C::T_O + ch * 32), r);
@@ -387,10 +390,10 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     }
 }
 
-template <int D, int BN, int NST, bool MODS>
+template <int DK, int DV, int BN, int NST, bool MODS>
 static cudaError_t launch_cfg(const PrefillLaunch &L, cudaStream_t stream) {
-    using C = PrefillCfg<D, BN, NST>;
-    auto kern = prefill_kernel<D, BN, NST, MODS>;
+    using C = PrefillCfg<DK, DV, BN, NST>;
+    auto kern = prefill_kernel<DK, DV, BN, NST, MODS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     PrefillArgs a;
@@ -414,14 +417,14 @@ static cudaError_t launch_cfg(const PrefillLaunch &L, cudaStream_t stream) {
 }
 
 cudaError_t launch_prefill(const PrefillLaunch &L, cudaStream_t stream) {
-    switch (L.dk) {
-        case 64: return L.has_mods ? launch_cfg<64, 128, 4, true>(L, stream) : launch_cfg<64, 128, 4, false>(L, stream);
-        case 128:
-            return L.has_mods ? launch_cfg<128, 128, 2, true>(L, stream) : launch_cfg<128, 128, 2, false>(L, stream);
-        case 256:
-            return L.has_mods ? launch_cfg<256, 64, 2, true>(L, stream) : launch_cfg<256, 64, 2, false>(L, stream);
-        default: return cudaErrorInvalidValue;
-    }
+#define FA_PREFILL_CFG(DK_, DV_, BN_, NST_) \
+    (L.has_mods ? launch_cfg<DK_, DV_, BN_, NST_, true>(L, stream) : launch_cfg<DK_, DV_, BN_, NST_, false>(L, stream))
+    if (L.dk == 256 && L.dv == 256) return FA_PREFILL_CFG(256, 256, 64, 2);
+    if (L.dk == 192 && L.dv == 128) return FA_PREFILL_CFG(192, 128, 128, 2);
+    if (L.dk == 192 && L.dv == 192) return FA_PREFILL_CFG(192, 192, 64, 3);
+    if (L.dk == 320 && L.dv == 256) return FA_PREFILL_CFG(320, 256, 64, 2);
+#undef FA_PREFILL_CFG
+    return cudaErrorInvalidValue;
 }
 
 cudaError_t prefill_device_error(int clear, int *code) {

@@ -55,7 +55,8 @@ class PrefillCase:
 
     @property
     def flops(self) -> float:
-        """4 * B * Hq * Sq * Sk * d (dk = dv here), halved for causal."""
+        """2 * B * Hq * Sq * Sk * (dk + dv): the QK^T and PV contractions,
+        halved for causal."""
         f = 2.0 * self.B * self.Hq * self.Sq * self.Sk * (self.dk + self.dv)
         return f / 2 if self.causal else f
 
@@ -70,6 +71,12 @@ def prefill_inputs(c: PrefillCase):
 TINY_FULL = PrefillCase("tiny_full_b1_h2_s256_d64", 1, 2, 2, 256, 256, 64, 64, False, seed=1)
 CAUSAL_MHA = PrefillCase("causal_mha_b2_h16_s2048_d128", 2, 16, 16, 2048, 2048, 128, 128, True, seed=2)
 GQA_FULL = PrefillCase("gqa_full_b1_hq32_hkv8_s4096_d256", 1, 32, 8, 4096, 4096, 256, 256, False, seed=3)
+# More head sizes: a latent-attention prefill head (dk = 128 + 64 rotary,
+# dv = 128), the (192, 192) pair with GQA and the (320, 256) pair.
+CAUSAL_DK192 = PrefillCase("causal_mha_b2_h16_s2048_dk192_dv128", 2, 16, 16, 2048, 2048, 192, 128, True, seed=7)
+CAUSAL_DK192_DV192 = PrefillCase("causal_gqa_b2_hq16_hkv4_s2048_dk192_dv192", 2, 16, 4, 2048, 2048, 192, 192, True,
+                                 seed=9)
+CAUSAL_DK320 = PrefillCase("causal_gqa_b1_hq16_hkv4_s4096_dk320_dv256", 1, 16, 4, 4096, 4096, 320, 256, True, seed=8)
 
 
 # ------------------------------------------------ prefill score modifiers --

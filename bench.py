@@ -52,6 +52,9 @@ NCU_TRAFFIC = {
     "causal_mha_mods_b2_h16_s2048_d128": 59766528,
     "paged_gqa_b64_hq32_hkv8_d128_bs64": 1237055008,
     "latent_sparse_t32_hq128_dk576_dv512_top2048": 45249792,
+    "causal_mha_b2_h16_s2048_dk192_dv128": 73713408,
+    "causal_gqa_b2_hq16_hkv4_s2048_dk192_dv192": 40004096,
+    "causal_gqa_b1_hq16_hkv4_s4096_dk320_dv256": 77931264,
 }
 
 
@@ -383,8 +386,8 @@ def run_only(args):
 
     torch.cuda.set_device(0)
     l2 = torch.cuda.get_device_properties(0).L2_cache_size
-    table = {c.name: c for c in (W_.TINY_FULL, W_.CAUSAL_MHA, W_.GQA_FULL, W_.MODS_C2, W_.PAGED_GQA,
-                                 W_.LATENT_SPARSE)}
+    table = {c.name: c for c in (W_.TINY_FULL, W_.CAUSAL_MHA, W_.GQA_FULL, W_.MODS_C2, W_.CAUSAL_DK192,
+                                 W_.CAUSAL_DK192_DV192, W_.CAUSAL_DK320, W_.PAGED_GQA, W_.LATENT_SPARSE)}
     if args.only not in table:
         raise SystemExit("unknown workload %r; one of %s" % (args.only, sorted(table)))
     c = table[args.only]
@@ -528,7 +531,8 @@ def main():
     if not args.no_secondary:
         wl = {}
         Ks = 200
-        for cc in (W_.TINY_FULL, W_.GQA_FULL, W_.MODS_C2):
+        for cc in (W_.TINY_FULL, W_.GQA_FULL, W_.MODS_C2, W_.CAUSAL_DK192, W_.CAUSAL_DK192_DV192,
+                   W_.CAUSAL_DK320):
             launch, ncopy, foot, kpl = prefill_workload(torch, fa, W_, cc, l2)
             ms2, st2 = time_graph(torch, launch, ncopy, Ks, Wm, dist)
             ms2 = max_over_ranks(torch, dist, ms2)

@@ -80,7 +80,9 @@ enum {
  * (bottom-right aligned, so a single decode query sees every key).
  * scale must be finite and > 0 (the caller passes 1/sqrt(dk) for standard
  * attention).
- * Supported: dk == dv in {64, 128, 256}; anything else is FA_ERR_UNSUPPORTED.
+ * Supported (dk, dv): (64, 64), (128, 128), (192, 192), (256, 256),
+ * (192, 128) and (320, 256) (the pairs up to dv = 256 of the llama.cpp
+ * tensor path's head-size table); anything else is FA_ERR_UNSUPPORTED.
  * Sq == 0 or B == 0 is a no-op; Sk == 0 writes O = 0, LSE = -inf.
  *
  * Score modifiers (all off when zero / NULL), as the llama.cpp tensor
