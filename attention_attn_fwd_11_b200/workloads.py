@@ -9,7 +9,7 @@ Recipe: every bf16 tensor is drawn as float32 ``torch.randn`` on a CPU
 ``torch.Generator`` seeded per tensor and rounded to bf16 (round to nearest
 even).  Seeds for workload ``c``: Q = 1000 + c, K = 2000 + c, V = 3000 + c,
 structure (lengths, block ids, selected rows) = 4000 + c, additive masks =
-5000 + c, sink logits = 6000 + c.
+5000 + c, sink logits = 6000 + c, quantised K/V blocks = 7000 + c.
 """
 from __future__ import annotations
 
@@ -112,6 +112,36 @@ def random_sinks(Hq: int, seed: int):
     """[Hq] float32 sink logits, N(0, 1)."""
     g = torch.Generator().manual_seed(6000 + seed)
     return torch.randn(Hq, generator=g)
+
+
+# ---------------------------------------------------- quantised K/V rows --
+# ggml q8_0 / q4_0 blocks drawn directly as random codes and scales (no
+# quantiser runs here): q8_0 codes are a rounded N(0, 40^2) clipped to
+# [-127, 127], q4_0 nibbles a rounded N(8, 2.5^2) clipped to [0, 15]; the f16
+# scales are uniform in [0.02, 0.03) (q8_0) and [0.3, 0.5) (q4_0), so the
+# decoded values have roughly unit spread like the bf16 inputs.  Seed
+# 7000 + c.
+
+QUANT_BLOCK_BYTES = {"q8_0": 34, "q4_0": 18}
+
+
+def random_quant_rows(shape, row_elems: int, qtype: str, seed: int):
+    """uint8 tensor [*shape, row_elems / 32 * block bytes] of ggml blocks."""
+    g = torch.Generator().manual_seed(7000 + seed)
+    nb = row_elems // 32
+    n = int(np.prod(shape)) * nb
+    if qtype == "q8_0":
+        d = torch.empty(n).uniform_(0.02, 0.03, generator=g).to(torch.float16)
+        q = (torch.randn(n, 32, generator=g) * 40).round().clamp(-127, 127).to(torch.int8)
+        body = q.view(torch.uint8)
+    elif qtype == "q4_0":
+        d = torch.empty(n).uniform_(0.3, 0.5, generator=g).to(torch.float16)
+        nib = (torch.randn(n, 32, generator=g) * 2.5 + 8).round().clamp(0, 15).to(torch.uint8)
+        body = nib[:, :16] | (nib[:, 16:] << 4)
+    else:
+        raise ValueError(qtype)
+    blocks = torch.cat([d.view(torch.uint8).view(n, 2), body], dim=1)
+    return blocks.reshape(*shape, nb * QUANT_BLOCK_BYTES[qtype]).contiguous()
 
 
 # C2's shape with every modifier on: ALiBi (max_bias 8) over a head-shared

@@ -59,6 +59,10 @@ def _load():
         lib.oracle_decode_latent.restype = i32
         lib.oracle_lse_combine.argtypes = [i32, i32, i32, P, P, P, P]
         lib.oracle_lse_combine.restype = None
+        lib.oracle_round_bf16.argtypes = [f64]
+        lib.oracle_round_bf16.restype = ctypes.c_uint16
+        lib.oracle_dequant_rows.argtypes = [P, i32, i64, i32, i64, P]
+        lib.oracle_dequant_rows.restype = i32
         _lib = lib
     return _lib
 
@@ -236,3 +240,26 @@ def lse_combine(o_parts, lse_parts):
     lse = np.zeros((R,), np.float64)
     _load().oracle_lse_combine(n, R, dv, _ptr(o_parts), _ptr(lse_parts), _ptr(o), _ptr(lse))
     return o, lse
+
+
+QUANT_TYPES = {"q8_0": (8, 34), "q4_0": (4, 18)}  # oracle type code, bytes per 32-value block
+
+
+def round_bf16(x) -> int:
+    """bf16 bit pattern of x, rounded to nearest with ties to even."""
+    return int(_load().oracle_round_bf16(float(x)))
+
+
+def dequant_rows(src, qtype, row_elems):
+    """Quantised rows -> bf16 bit patterns.  src: uint8 [..., row_bytes]
+    (each row holds row_elems / 32 ggml blocks of type ``qtype``, 'q8_0' or
+    'q4_0', then any padding); returns uint16 [..., row_elems]."""
+    code, bb = QUANT_TYPES[qtype]
+    src = np.ascontiguousarray(src, dtype=np.uint8)
+    lead = src.shape[:-1]
+    n_rows = int(np.prod(lead)) if lead else 1
+    out = np.empty(lead + (row_elems,), np.uint16)
+    rc = _load().oracle_dequant_rows(_ptr(src), code, n_rows, row_elems, src.shape[-1], _ptr(out))
+    if rc:
+        raise ValueError("oracle_dequant_rows: bad arguments")
+    return out

@@ -494,3 +494,77 @@ void oracle_lse_combine(int n_parts, int R, int dv, const double *o_parts,
         lse[r] = L;
     }
 }
+
+/*
+ * Quantised K/V rows -> bf16: the pre-pass that the llama.cpp tensor path
+ * runs before its 16-bit kernels ("ggml-metal: FA tensor path",
+ * ggml_metal_op_flash_attn_ext_use_kv_f16: a quantised KV cache is
+ * dequantised first, then the 16-bit attention kernels run on it).  The
+ * block layouts are ggml's:
+ *   q8_0 (type 8): 34 bytes per 32 values -- a little-endian f16 scale d,
+ *                  then 32 int8 codes q; value j = d * q_j.
+ *   q4_0 (type 4): 18 bytes per 32 values -- f16 scale d, then 16 bytes;
+ *                  byte j holds value j in its low nibble and value j + 16
+ *                  in its high nibble; value = d * (nibble - 8).
+ * Reading: the pages dequantise to f16; the attention kernels here take
+ * bf16 operands, so each value d * q (exact in double) is rounded once, to
+ * nearest with ties to even, to bf16.
+ */
+
+/* double -> bf16 bit pattern, round to nearest, ties to even, from the
+ * definition: scale |x| so that one bf16 unit in the last place is 1, round
+ * to the nearest integer (rint under the default rounding mode), scale back.
+ * bf16 has 8 significant bits, exponents down to -126 for normals and a
+ * subnormal step of 2^-133; results of 2^128 or more become infinity. */
+static uint16_t double_to_bf16_rne(double x)
+{
+    if (isnan(x)) return 0x7fc0;
+    const uint16_t sign = signbit(x) ? 0x8000 : 0;
+    const double a = fabs(x);
+    if (a == 0.0) return sign;
+    if (isinf(a)) return sign | 0x7f80;
+    int E;
+    frexp(a, &E);                         /* a in [2^(E-1), 2^E) */
+    int ulp_exp = (E - 1) - 7;            /* 8 significant bits */
+    if (ulp_exp < -133) ulp_exp = -133;   /* subnormal range */
+    const double r = ldexp(rint(ldexp(a, -ulp_exp)), ulp_exp);
+    if (r >= ldexp(1.0, 128)) return sign | 0x7f80;
+    const float f = (float)r;             /* exact: r is a bf16 value */
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    return sign | (uint16_t)((u >> 16) & 0x7fff);
+}
+
+uint16_t oracle_round_bf16(double x) { return double_to_bf16_rne(x); }
+
+/*
+ * n_rows rows of row_elems values each (row_elems a multiple of 32); row r
+ * starts at src + r * src_row_bytes.  dst: [n_rows][row_elems] bf16 bits.
+ * Returns 0, or -1 on bad arguments.
+ */
+int oracle_dequant_rows(const uint8_t *src, int type, int64_t n_rows, int row_elems,
+                        int64_t src_row_bytes, uint16_t *dst)
+{
+    const int block_bytes = type == 8 ? 34 : type == 4 ? 18 : 0;
+    if (!block_bytes || row_elems <= 0 || row_elems % 32 || n_rows < 0 ||
+        src_row_bytes < (int64_t)(row_elems / 32) * block_bytes)
+        return -1;
+    for (int64_t r = 0; r < n_rows; ++r) {
+        const uint8_t *row = src + r * src_row_bytes;
+        for (int blk = 0; blk < row_elems / 32; ++blk) {
+            const uint8_t *p = row + (int64_t)blk * block_bytes;
+            const double d = f16_bits_to_double((uint16_t)(p[0] | (p[1] << 8)));
+            for (int j = 0; j < 32; ++j) {
+                int q;
+                if (type == 8) {
+                    q = (int)(int8_t)p[2 + j];
+                } else {
+                    const uint8_t byte = p[2 + (j % 16)];
+                    q = (j < 16 ? (byte & 0x0f) : (byte >> 4)) - 8;
+                }
+                dst[r * row_elems + blk * 32 + j] = double_to_bf16_rne(d * (double)q);
+            }
+        }
+    }
+    return 0;
+}
