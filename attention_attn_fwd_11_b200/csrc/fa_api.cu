@@ -464,6 +464,48 @@ fa_status fa_decode_gather(const fa_decode_gather_params *p, void *stream) {
     return FA_OK;
 }
 
+fa_status fa_kv_dequant_n(const fa_kv_dequant_params *p, int n, void *stream) {
+    if (!p) return fail(FA_ERR_INVALID_ARG, "fa_kv_dequant: params is NULL");
+    if (n < 1 || n > fa::kMaxDequantSegs)
+        return fail(FA_ERR_INVALID_ARG, "fa_kv_dequant_n: n must be in [1, %d]", fa::kMaxDequantSegs);
+    fa::KvDequantLaunch L[fa::kMaxDequantSegs];
+    bool any = false;
+    for (int i = 0; i < n; ++i) {
+        const fa_kv_dequant_params *q = p + i;
+        if (q->type != FA_KV_Q8_0 && q->type != FA_KV_Q4_0)
+            return fail(FA_ERR_UNSUPPORTED, "fa_kv_dequant: type %d (supported: FA_KV_Q8_0, FA_KV_Q4_0)", q->type);
+        if (q->type != p->type) return fail(FA_ERR_INVALID_ARG, "fa_kv_dequant_n: every entry must have one type");
+        if (q->n_rows < 0 || q->row_elems <= 0 || q->row_elems % 32 != 0)
+            return fail(FA_ERR_INVALID_ARG, "fa_kv_dequant: need n_rows >= 0 and row_elems a positive multiple of 32");
+        const int64_t block_bytes = q->type == FA_KV_Q8_0 ? 34 : 18;
+        if (q->src_row_bytes < q->row_elems / 32 * block_bytes || q->src_row_bytes % 2 != 0)
+            return fail(FA_ERR_INVALID_ARG, "fa_kv_dequant: src_row_bytes must be even and >= %lld",
+                        (long long)(q->row_elems / 32 * block_bytes));
+        if (q->dst_row_stride < q->row_elems || q->dst_row_stride % 8 != 0)
+            return fail(FA_ERR_INVALID_ARG, "fa_kv_dequant: dst_row_stride must be a multiple of 8 and >= row_elems");
+        if (q->n_rows > 0) {
+            if (!q->src || !q->dst) return fail(FA_ERR_INVALID_ARG, "fa_kv_dequant: NULL pointer");
+            if (reinterpret_cast<uintptr_t>(q->src) % 2 != 0 || reinterpret_cast<uintptr_t>(q->dst) % 16 != 0)
+                return fail(FA_ERR_INVALID_ARG, "fa_kv_dequant: src must be 2-byte and dst 16-byte aligned");
+            const int64_t pitch = q->src_row_bytes > 2 * q->dst_row_stride ? q->src_row_bytes : 2 * q->dst_row_stride;
+            if (q->n_rows > (INT64_MAX / 4) / pitch)
+                return fail(FA_ERR_INVALID_ARG, "fa_kv_dequant: rows * pitch overflows");
+            any = true;
+        }
+        L[i] = fa::KvDequantLaunch{q->src, q->type, q->n_rows, q->row_elems, q->src_row_bytes, q->dst,
+                                   q->dst_row_stride};
+    }
+    if (!any) return FA_OK;
+    int sms = 0;
+    cudaError_t e = num_sms(&sms);
+    if (e != cudaSuccess) return cuda_fail(e, "fa_kv_dequant");
+    e = fa::launch_kv_dequant(L, n, sms, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "fa_kv_dequant launch");
+    return FA_OK;
+}
+
+fa_status fa_kv_dequant(const fa_kv_dequant_params *p, void *stream) { return fa_kv_dequant_n(p, 1, stream); }
+
 fa_status fa_device_error(int clear, int *code) {
     if (!code) return fail(FA_ERR_INVALID_ARG, "fa_device_error: code is NULL");
     int c1 = 0, c2 = 0, c3 = 0, c4 = 0;

@@ -78,4 +78,17 @@ struct GatherLaunch {
 cudaError_t launch_decode_gather(const GatherLaunch &L, cudaStream_t stream);
 cudaError_t gather_device_error(int clear, int *code);
 
+// Quantised K/V rows -> bf16 (kv_dequant.cu).  type: 8 = q8_0, 4 = q4_0.
+struct KvDequantLaunch {
+    const void *src;
+    int type;
+    int64_t n_rows;
+    int row_elems;
+    int64_t src_row_bytes;
+    void *dst;
+    int64_t dst_row_stride;
+};
+constexpr int kMaxDequantSegs = 4;  // tensors one launch converts (all of one type)
+cudaError_t launch_kv_dequant(const KvDequantLaunch *L, int n, int num_sms, cudaStream_t stream);
+
 }  // namespace fa

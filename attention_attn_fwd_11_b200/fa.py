@@ -52,6 +52,14 @@ class GatherParams(ctypes.Structure):
                 ("o_dtype", _i32), ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t)]
 
 
+class KvDequantParams(ctypes.Structure):
+    _fields_ = [("src", _vp), ("type", _i32), ("n_rows", _i64), ("row_elems", _i32), ("src_row_bytes", _i64),
+                ("dst", _vp), ("dst_row_stride", _i64)]
+
+
+FA_KV_Q8_0, FA_KV_Q4_0 = 8, 4
+KV_QUANT = {"q8_0": (FA_KV_Q8_0, 34), "q4_0": (FA_KV_Q4_0, 18)}  # type code, bytes per 32-value block
+
 _lib = None
 
 
@@ -72,6 +80,10 @@ def load():
         lib.fa_decode_gather_workspace_size.restype = _i32
         lib.fa_decode_gather.argtypes = [ctypes.POINTER(GatherParams), _vp]
         lib.fa_decode_gather.restype = _i32
+        lib.fa_kv_dequant.argtypes = [ctypes.POINTER(KvDequantParams), _vp]
+        lib.fa_kv_dequant.restype = _i32
+        lib.fa_kv_dequant_n.argtypes = [ctypes.POINTER(KvDequantParams), _i32, _vp]
+        lib.fa_kv_dequant_n.restype = _i32
         lib.fa_last_error.argtypes = []
         lib.fa_last_error.restype = ctypes.c_char_p
         lib.fa_device_error.argtypes = [_i32, ctypes.POINTER(_i32)]
@@ -275,3 +287,69 @@ def device_error(clear=True) -> int:
     c = _i32(0)
     _check(load().fa_device_error(1 if clear else 0, ctypes.byref(c)))
     return c.value
+
+
+# ------------------------------------------------------ quantised K/V rows --
+
+def kv_dequant_params(src, qtype, row_elems, dst):
+    """Marshal a fa_kv_dequant call: src uint8 [..., row_bytes] (rows of
+    ggml blocks), dst bf16 [..., >= row_elems] with unit stride in the last
+    dimension and the same leading shape, both contiguous over the rows."""
+    code, _ = KV_QUANT[qtype]
+    p = KvDequantParams()
+    p.src, p.type, p.row_elems, p.dst = _ptr(src), code, row_elems, _ptr(dst)
+    p.n_rows = src.numel() // src.shape[-1] if src.dim() else 0
+    p.src_row_bytes = src.stride(-2) if src.dim() > 1 else src.shape[-1]
+    p.dst_row_stride = dst.stride(-2) if dst.dim() > 1 else dst.shape[-1]
+    return p
+
+
+def _dequant_entry(src, qtype, row_elems, out):
+    _need_cuda(src, out)
+    if src.dtype != torch.uint8:
+        raise ValueError("src must be uint8 blocks")
+    if src.stride(-1) != 1:
+        raise ValueError("src rows must be contiguous")
+    lead = src.shape[:-1]
+    if out is None:
+        out = torch.empty(lead + (row_elems,), device=src.device, dtype=torch.bfloat16)
+    if out.dtype != torch.bfloat16 or out.shape[:-1] != lead or out.shape[-1] < row_elems or out.stride(-1) != 1:
+        raise ValueError("out must be bf16 [..., >= row_elems] with the rows of src")
+    s2, o2 = src.reshape(-1, src.shape[-1]), out.reshape(-1, out.shape[-1])
+    if s2.data_ptr() != src.data_ptr() or o2.data_ptr() != out.data_ptr():
+        raise ValueError("leading dimensions must collapse to one row stride")
+    return kv_dequant_params(s2, qtype, row_elems, o2), out
+
+
+def kv_dequant(src, qtype, row_elems, out=None, stream=None):
+    """Quantised rows -> bf16 rows on the GPU (fa_kv_dequant).  src: uint8
+    CUDA tensor [..., row_bytes] whose rows each hold row_elems / 32 ggml
+    blocks of ``qtype`` ('q8_0' or 'q4_0'); the leading dimensions must
+    collapse to one row index with a single stride.  Returns (or fills) a
+    bf16 tensor [..., row_elems]."""
+    p, out = _dequant_entry(src, qtype, row_elems, out)
+    _check(load().fa_kv_dequant(ctypes.byref(p), _stream(stream)))
+    return out
+
+
+def kv_dequant_many(entries, stream=None):
+    """Several conversions in one launch (fa_kv_dequant_n).  entries: list of
+    (src, qtype, row_elems, out-or-None), 1 to 4 of them, one qtype.
+    Returns the list of outputs."""
+    made = [_dequant_entry(*e) for e in entries]
+    arr = (KvDequantParams * len(made))(*[m[0] for m in made])
+    _check(load().fa_kv_dequant_n(arr, len(made), _stream(stream)))
+    return [m[1] for m in made]
+
+
+def fwd_quant(q, k_blocks, v_blocks, qtype, dk, dv, scale=None, causal=False, out=None, return_lse=True,
+              out_dtype=torch.float32, k_buf=None, v_buf=None, stream=None, **mods):
+    """Prefill over quantised K/V, the pages' way: dequantise K and V to bf16
+    (one fa_kv_dequant_n launch for both) and run fa_fwd on them.  k_blocks /
+    v_blocks: uint8 [B, Hkv, Sk, dk / 32 * block bytes] and [..., dv / 32 *
+    block bytes]; k_buf / v_buf: optional bf16 [B, Hkv, Sk, dk / dv] buffers
+    for the dequantised rows (allocated when absent).  Other arguments as
+    fwd()."""
+    k, v = kv_dequant_many([(k_blocks, qtype, dk, k_buf), (v_blocks, qtype, dv, v_buf)], stream=stream)
+    return fwd(q, k, v, scale=scale, causal=causal, out=out, return_lse=return_lse, out_dtype=out_dtype,
+               stream=stream, **mods)

@@ -144,6 +144,11 @@ def random_quant_rows(shape, row_elems: int, qtype: str, seed: int):
     return blocks.reshape(*shape, nb * QUANT_BLOCK_BYTES[qtype]).contiguous()
 
 
+# The causal MHA shape with q8_0 K/V (the prefill reads the dequantised rows).
+QUANT_C2 = PrefillCase("causal_mha_q8_0kv_b2_h16_s2048_d128", 2, 16, 16, 2048, 2048, 128, 128, True, seed=2)
+QUANT_C2_TYPE = "q8_0"
+
+
 # C2's shape with every modifier on: ALiBi (max_bias 8) over a head-shared
 # distance mask, softcap 30, one sink per head.
 MODS_C2 = PrefillCase("causal_mha_mods_b2_h16_s2048_d128", 2, 16, 16, 2048, 2048, 128, 128, True, seed=2)

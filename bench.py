@@ -54,6 +54,7 @@ NCU_TRAFFIC = {
     "latent_sparse_t32_hq128_dk576_dv512_top2048": 45249792,
     "causal_mha_b2_h16_s2048_dk192_dv128": 73713408,
     "causal_gqa_b2_hq16_hkv4_s2048_dk192_dv192": 40004096,
+    "kv_dequant causal_mha_q8_0kv_b2_h16_s2048_d128": 17835776,
     "causal_gqa_b1_hq16_hkv4_s4096_dk320_dv256": 77931264,
 }
 
@@ -245,6 +246,45 @@ def prefill_workload(torch, fa, W_, c, l2):
     return launch, n, foot, 1
 
 
+def quant_prefill_workload(torch, fa, W_, c, qtype, l2, dequant_only=False):
+    """Prefill over quantised K/V the pages' way: one fa_kv_dequant_n launch
+    (K rows and V rows) into bf16 buffers, then fa_fwd.  With dequant_only,
+    the step is the dequant launch alone (its HBM roofline)."""
+    import ctypes
+    q0 = W_.randn_bf16((c.B, c.Hq, c.Sq, c.dk), 1000 + c.seed)
+    kb0 = W_.random_quant_rows((c.B, c.Hkv, c.Sk), c.dk, qtype, c.seed)
+    vb0 = W_.random_quant_rows((c.B, c.Hkv, c.Sk), c.dv, qtype, c.seed + 100)
+    kv_bf16 = c.B * c.Hkv * c.Sk * (c.dk + c.dv) * 2
+    dq_bytes = kb0.numel() + vb0.numel() + kv_bf16  # quantised blocks read + bf16 rows written
+    foot = q0.numel() * 2 + dq_bytes + c.B * c.Hq * c.Sq * (c.dv * 4 + 4)
+    n = rotation_copies(foot, l2)
+    lib = fa.load()
+    bufs, params = [], []
+    for i in range(n):
+        q, kb, vb = q0.cuda(), kb0.cuda(), vb0.cuda()
+        kbuf = torch.empty(c.B, c.Hkv, c.Sk, c.dk, device="cuda", dtype=torch.bfloat16)
+        vbuf = torch.empty(c.B, c.Hkv, c.Sk, c.dv, device="cuda", dtype=torch.bfloat16)
+        o = torch.empty(c.B, c.Hq, c.Sq, c.dv, device="cuda")
+        lse = torch.empty(c.B, c.Hq, c.Sq, device="cuda")
+        bufs.append((q, kb, vb, kbuf, vbuf, o, lse))
+        pkv = (fa.KvDequantParams * 2)(fa.kv_dequant_params(kb.view(-1, kb.shape[-1]), qtype, c.dk, kbuf.view(-1, c.dk)),
+                                       fa.kv_dequant_params(vb.view(-1, vb.shape[-1]), qtype, c.dv, vbuf.view(-1, c.dv)))
+        pf = fa.fwd_params(q, kbuf, vbuf, o, lse, c.scale, c.causal)
+        params.append((pkv, pf))
+
+    def launch(i):
+        st_ = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+        pkv, pf = params[i]
+        st = lib.fa_kv_dequant_n(pkv, 2, st_)
+        if st == 0 and not dequant_only:
+            st = lib.fa_fwd(ctypes.byref(pf), st_)
+        if st != 0:
+            raise RuntimeError(lib.fa_last_error().decode())
+
+    launch.keep = bufs
+    return launch, n, dq_bytes, 1 if dequant_only else 2
+
+
 def paged_workload(torch, fa, W_, c, l2):
     q0, kc0, vc0, tb0, sl0 = W_.paged_inputs(c)
     byts = W_.paged_bytes(c, sl0, tb0.shape[1])
@@ -387,11 +427,17 @@ def run_only(args):
     torch.cuda.set_device(0)
     l2 = torch.cuda.get_device_properties(0).L2_cache_size
     table = {c.name: c for c in (W_.TINY_FULL, W_.CAUSAL_MHA, W_.GQA_FULL, W_.MODS_C2, W_.CAUSAL_DK192,
-                                 W_.CAUSAL_DK192_DV192, W_.CAUSAL_DK320, W_.PAGED_GQA, W_.LATENT_SPARSE)}
+                                 W_.CAUSAL_DK192_DV192, W_.CAUSAL_DK320, W_.PAGED_GQA, W_.LATENT_SPARSE,
+                                 W_.QUANT_C2)}
+    table["kv_dequant_" + W_.QUANT_C2.name] = W_.QUANT_C2
     if args.only not in table:
         raise SystemExit("unknown workload %r; one of %s" % (args.only, sorted(table)))
     c = table[args.only]
-    if isinstance(c, W_.PrefillCase):
+    if c is W_.QUANT_C2:
+        only_dq = args.only.startswith("kv_dequant_")
+        launch, n, work, kpl = quant_prefill_workload(torch, fa, W_, c, W_.QUANT_C2_TYPE, l2, dequant_only=only_dq)
+        unit, amount = ("GB/s", work / 1e9) if only_dq else ("TFLOP/s", c.flops / 1e12)
+    elif isinstance(c, W_.PrefillCase):
         launch, n, work, kpl = prefill_workload(torch, fa, W_, c, l2)
         unit, amount = "TFLOP/s", c.flops / 1e12
     elif isinstance(c, W_.PagedCase):
@@ -544,6 +590,26 @@ def main():
                                                 NCU_TRAFFIC.get(cc.name))}
             result["gpu_launches"] += st2 * kpl
             del launch
+        # prefill over q8_0 K/V: two dequant launches + fa_fwd per step
+        qc = W_.QUANT_C2
+        launch, ncopy, dq_bytes, kpl = quant_prefill_workload(torch, fa, W_, qc, W_.QUANT_C2_TYPE, l2)
+        ms2, st2 = time_graph(torch, launch, ncopy, Ks, Wm, dist)
+        ms2 = max_over_ranks(torch, dist, ms2)
+        per = ms2 / st2
+        result["gpu_launches"] += st2 * kpl
+        del launch
+        launch, ncopy_d, _, kpl_d = quant_prefill_workload(torch, fa, W_, qc, W_.QUANT_C2_TYPE, l2, dequant_only=True)
+        msd, std_ = time_graph(torch, launch, ncopy_d, Ks, Wm, dist)
+        msd = max_over_ranks(torch, dist, msd)
+        perd = msd / std_
+        result["gpu_launches"] += std_ * kpl_d
+        del launch
+        wl[qc.name] = {"value": round(sum_over_ranks(torch, dist, qc.flops * st2) / (ms2 * 1e-3) / 1e12, 2),
+                       "unit": "TFLOP/s", "ms_per_step": round(per, 5), "steps": st2, "l2_copies": ncopy,
+                       "kernels": "kv_dequant (%s K and V rows -> bf16, one launch) + prefill" % W_.QUANT_C2_TYPE,
+                       "dequant": {"ms_per_step": round(perd, 5), "bytes_per_step": dq_bytes,
+                                   "roofline": roofline("hbm", dq_bytes / (perd * 1e-3) / 1e9, peaks["hbm_gbs"],
+                                                        "GB/s", NCU_TRAFFIC.get("kv_dequant " + qc.name))}}
         pc = W_.PAGED_GQA
         launch, ncopy, byts, kpl = paged_workload(torch, fa, W_, pc, l2)
         ms2, st2 = time_graph(torch, launch, ncopy, Ks, Wm, dist)

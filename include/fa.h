@@ -234,6 +234,53 @@ typedef struct {
     size_t workspace_bytes;
 } fa_decode_gather_params;
 
+/*
+ * fa_kv_dequant -- quantised K or V rows to bf16: the pre-pass that
+ * "ggml-metal: FA tensor path" (ggml_metal_op_flash_attn_ext_use_kv_f16)
+ * runs on a quantised KV cache before its 16-bit attention kernels.  Feed
+ * the bf16 rows it writes to fa_fwd (or, laid out as a paged cache, to
+ * fa_decode_paged).
+ *   src: n_rows rows; row r starts at byte r * src_row_bytes and holds
+ *     row_elems / 32 consecutive ggml blocks of `type`, then any padding
+ *     (never read):
+ *       FA_KV_Q8_0: 34 bytes per block -- little-endian f16 scale d, then 32
+ *         int8 codes q; value j = d * q_j;
+ *       FA_KV_Q4_0: 18 bytes per block -- f16 scale d, then 16 bytes; byte j
+ *         holds value j in its low nibble and value j + 16 in its high
+ *         nibble; value = d * (nibble - 8).
+ *   dst: bf16 rows at a pitch of dst_row_stride elements; the first
+ *     row_elems elements of each row are written, the rest left as they are.
+ *   Each value d * q is exact in fp32 and rounded once, to nearest even, to
+ *   bf16 (the pages dequantise to f16; the attention kernels here take bf16).
+ * Requirements: row_elems > 0 and a multiple of 32; src 2-byte aligned and
+ * src_row_bytes even and >= row_elems / 32 * block bytes; dst 16-byte
+ * aligned, dst_row_stride a multiple of 8 and >= row_elems; n_rows >= 0
+ * (0 launches nothing).  src and dst must not overlap.  Non-finite scales
+ * decode as IEEE arithmetic gives them (inf * 0 = NaN).
+ */
+typedef enum { FA_KV_Q8_0 = 8, FA_KV_Q4_0 = 4 } fa_kv_quant;
+
+typedef struct {
+    const void *src;
+    int type; /* fa_kv_quant */
+    int64_t n_rows;
+    int row_elems;
+    int64_t src_row_bytes;
+    void *dst;
+    int64_t dst_row_stride;
+} fa_kv_dequant_params;
+
+fa_status fa_kv_dequant(const fa_kv_dequant_params *p, void *stream);
+
+/*
+ * fa_kv_dequant_n -- n (1 to 4) independent fa_kv_dequant conversions in one
+ * launch, e.g. a layer's K rows and V rows.  p points to n entries, each
+ * checked as fa_kv_dequant checks it; all must have the same type.  Entries
+ * with n_rows == 0 are skipped.  No two entries' dst ranges may overlap, and
+ * no dst range may overlap any src range.
+ */
+fa_status fa_kv_dequant_n(const fa_kv_dequant_params *p, int n, void *stream);
+
 /* Workspace bytes for these shapes and num_splits; reads no pointer field. */
 fa_status fa_decode_gather_workspace_size(const fa_decode_gather_params *p, size_t *bytes);
 fa_status fa_decode_gather(const fa_decode_gather_params *p, void *stream);

@@ -137,6 +137,51 @@ def test_gather_workspace_size_and_validation():
     assert lib.fa_decode_gather(ctypes.byref(gather_params(T=0)), None) == fa.FA_OK
 
 
+def dequant_params(**kw):
+    p = fa.KvDequantParams()
+    base = dict(src=2, type=fa.FA_KV_Q8_0, n_rows=1024, row_elems=128, src_row_bytes=136, dst=16, dst_row_stride=128)
+    base.update(kw)
+    for k_, v_ in base.items():
+        setattr(p, k_, v_)
+    return p
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(type=5), fa.FA_ERR_UNSUPPORTED),
+    (dict(row_elems=48), fa.FA_ERR_INVALID_ARG),             # not a multiple of 32
+    (dict(row_elems=0), fa.FA_ERR_INVALID_ARG),
+    (dict(n_rows=-1), fa.FA_ERR_INVALID_ARG),
+    (dict(src_row_bytes=134), fa.FA_ERR_INVALID_ARG),        # shorter than 4 q8_0 blocks
+    (dict(src_row_bytes=137), fa.FA_ERR_INVALID_ARG),        # odd pitch
+    (dict(dst_row_stride=120), fa.FA_ERR_INVALID_ARG),       # < row_elems
+    (dict(dst_row_stride=132), fa.FA_ERR_INVALID_ARG),       # not a multiple of 8
+    (dict(src=3), fa.FA_ERR_INVALID_ARG),                    # src not 2-byte aligned
+    (dict(dst=24), fa.FA_ERR_INVALID_ARG),                   # dst not 16-byte aligned
+    (dict(src=0), fa.FA_ERR_INVALID_ARG),
+    (dict(type=fa.FA_KV_Q4_0, src_row_bytes=70), fa.FA_ERR_INVALID_ARG),   # 4 q4_0 blocks need 72
+])
+def test_kv_dequant_rejects(kw, status):
+    assert fa.load().fa_kv_dequant(ctypes.byref(dequant_params(**kw)), None) == status
+
+
+def test_kv_dequant_n_checks_every_entry():
+    lib = fa.load()
+    two = (fa.KvDequantParams * 2)(dequant_params(), dequant_params(type=fa.FA_KV_Q4_0, src_row_bytes=72))
+    assert lib.fa_kv_dequant_n(two, 2, None) == fa.FA_ERR_INVALID_ARG          # mixed types
+    two = (fa.KvDequantParams * 2)(dequant_params(), dequant_params(dst=8))
+    assert lib.fa_kv_dequant_n(two, 2, None) == fa.FA_ERR_INVALID_ARG          # second entry misaligned
+    assert lib.fa_kv_dequant_n(two, 0, None) == fa.FA_ERR_INVALID_ARG
+    assert lib.fa_kv_dequant_n(two, 5, None) == fa.FA_ERR_INVALID_ARG
+    empty = (fa.KvDequantParams * 2)(dequant_params(n_rows=0, src=0, dst=0), dequant_params(n_rows=0))
+    assert lib.fa_kv_dequant_n(empty, 2, None) == fa.FA_OK
+
+
+def test_kv_dequant_null_params_and_noop():
+    lib = fa.load()
+    assert lib.fa_kv_dequant(None, None) == fa.FA_ERR_INVALID_ARG
+    assert lib.fa_kv_dequant(ctypes.byref(dequant_params(n_rows=0, src=0, dst=0)), None) == fa.FA_OK
+
+
 def test_binding_refuses_cpu_tensors():
     import torch
     q = torch.zeros(1, 1, 128, 64, dtype=torch.bfloat16)
