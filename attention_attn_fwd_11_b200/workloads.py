@@ -216,6 +216,59 @@ def paged_bytes(c: PagedCase, seq_lens, max_blocks: int) -> int:
 PAGED_GQA = PagedCase("paged_gqa_b64_hq32_hkv8_d128_bs64", 64, 32, 8, 128, 128, 64, 1024, 8192, seed=4)
 
 
+# ----------------------------------------------------------- paged prefill --
+# Chunked prefill: Sq new query rows per sequence over a paged cache whose
+# lengths (which include the new rows) are drawn as for the paged decode,
+# from [max(min_len, Sq), max_len].  Pool, table and caches follow the paged
+# decode recipe; Q is [B, Hq, Sq, d].
+
+@dataclass
+class PagedPrefillCase:
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    Sq: int
+    d: int
+    min_len: int
+    max_len: int
+    causal: bool = True
+    block_size: int = 64
+    seed: int = 0
+    scale: float = field(default=0.0)
+    lens: tuple | None = None  # explicit per-sequence lengths (tests)
+
+    def __post_init__(self):
+        if not self.scale:
+            self.scale = 1.0 / math.sqrt(self.d)
+
+    def flops(self, seq_lens) -> float:
+        """2 * Hq * (dk + dv) per visible (query, key) pair: with causal,
+        query i of a sequence of L keys sees max(0, L - Sq + i + 1) keys."""
+        pairs = 0
+        for L in (int(x) for x in seq_lens):
+            if self.causal:
+                lo = L - self.Sq + 1  # keys seen by query 0
+                pairs += sum(max(0, lo + i) for i in range(self.Sq))
+            else:
+                pairs += self.Sq * L
+        return 2.0 * self.Hq * 2 * self.d * pairs
+
+
+def paged_prefill_inputs(c: PagedPrefillCase):
+    """Returns q [B,Hq,Sq,d], k_cache/v_cache [nb,Hkv,bs,d] bf16, block_table
+    int32 [B, max_blocks] (-1 past the end), seq_lens int32 [B]."""
+    pc = PagedCase(c.name, c.B, c.Hq, c.Hkv, c.d, c.d, c.block_size, max(c.min_len, c.Sq), c.max_len, seed=c.seed,
+                   lens=c.lens)
+    _, kc, vc, table, lens = paged_inputs(pc)
+    q = randn_bf16((c.B, c.Hq, c.Sq, c.d), 1000 + c.seed)
+    return q, kc, vc, table, lens
+
+
+PAGED_PREFILL = PagedPrefillCase("paged_prefill_gqa_b16_hq32_hkv8_sq512_d128_bs64", 16, 32, 8, 512, 128, 1024, 8192,
+                                 seed=6)
+
+
 # ----------------------------------------------------------- latent decode --
 
 @dataclass

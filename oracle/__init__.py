@@ -190,6 +190,26 @@ def decode_paged(q, k_cache, v_cache, block_table, seq_lens, scale):
     return o, lse
 
 
+def prefill_paged(q, k_cache, v_cache, block_table, seq_lens, scale, causal=True):
+    """Chunked prefill over a paged cache: per sequence b, its keys are
+    gathered from the cache (paged_gather) and the dense oracle runs on
+    them.  q [B,Hq,Sq,dk]; caches [num_blocks,Hkv,block_size,d]; seq_lens
+    counts the Sq new keys too.  Returns (O [B,Hq,Sq,dv], LSE [B,Hq,Sq])
+    float64."""
+    q = _u16(q)
+    bs = k_cache.shape[2]
+    sl = np.ascontiguousarray(seq_lens, dtype=np.int32)
+    kk = paged_gather(k_cache, block_table, sl, bs)
+    vv = paged_gather(v_cache, block_table, sl, bs)
+    B, Hq, Sq, _ = q.shape
+    o = np.zeros((B, Hq, Sq, vv.shape[3]), np.float64)
+    lse = np.zeros((B, Hq, Sq), np.float64)
+    for b in range(B):
+        n = int(sl[b])
+        o[b:b + 1], lse[b:b + 1] = attention(q[b:b + 1], kk[b:b + 1, :, :n], vv[b:b + 1, :, :n], scale, causal)
+    return o, lse
+
+
 def latent_gather(rows, idx, row_len):
     """Materialise the selected rows: returns (rows [T,topk,row_len] uint16,
     valid [T,topk] uint8)."""

@@ -1,0 +1,68 @@
+"""Pins for the oracle's chunked prefill over a paged cache
+(oracle.prefill_paged): the decode call with Sq > 1 (the paged decode's
+table walk and the prefill's bottom-right causal rule).  Each pin compares
+against an independent route: the oracle's separate paged-decode function,
+dense attention over a cache whose table is the identity, and the causal
+rule's closed form for rows that see no key."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from attention_attn_fwd_11_b200 import workloads as W
+
+
+def case(B, Hq, Hkv, Sq, d, lens, causal=True, seed=0):
+    c = W.PagedPrefillCase("t", B, Hq, Hkv, Sq, d, 0, 0, causal=causal, seed=seed, lens=tuple(lens))
+    q, kc, vc, table, sl = W.paged_prefill_inputs(c)
+    return c, W.bits(q), W.bits(kc), W.bits(vc), table.numpy(), sl.numpy()
+
+
+def test_one_new_row_equals_paged_decode():
+    # Sq = 1 is the decode: the last position sees every key.
+    c, q, kc, vc, table, sl = case(3, 4, 2, 1, 64, (70, 1, 200), seed=1)
+    o, lse = oracle.prefill_paged(q, kc, vc, table, sl, c.scale, causal=True)
+    od, ld = oracle.decode_paged(q[:, :, 0], kc, vc, table, sl, c.scale)
+    assert np.allclose(o[:, :, 0], od, rtol=0, atol=1e-13)
+    assert np.allclose(lse[:, :, 0], ld, rtol=0, atol=1e-13)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_identity_table_equals_dense(causal):
+    # A cache laid out so that sequence b's keys are blocks b*nb .. b*nb+nb-1
+    # in order: the paged result equals dense attention over those keys.
+    B, Hkv, Hq, Sq, d, L = 2, 2, 4, 37, 64, 150
+    nb = (L + 63) // 64
+    rng = np.random.default_rng(3)
+    k = W.bits(W.randn_bf16((B, Hkv, nb * 64, d), 11))
+    v = W.bits(W.randn_bf16((B, Hkv, nb * 64, d), 12))
+    q = W.bits(W.randn_bf16((B, Hq, Sq, d), 13))
+    # [B, Hkv, nb, 64, d] -> [B * nb, Hkv, 64, d]
+    kc = k.reshape(B, Hkv, nb, 64, d).transpose(0, 2, 1, 3, 4).reshape(B * nb, Hkv, 64, d).copy()
+    vc = v.reshape(B, Hkv, nb, 64, d).transpose(0, 2, 1, 3, 4).reshape(B * nb, Hkv, 64, d).copy()
+    table = np.arange(B * nb, dtype=np.int32).reshape(B, nb)
+    sl = np.array([L, L - 50], np.int32)
+    o, lse = oracle.prefill_paged(q, kc, vc, table, sl, 0.125, causal=causal)
+    for b in range(B):
+        n = int(sl[b])
+        od, ld = oracle.attention(q[b:b + 1], k[b:b + 1, :, :n], v[b:b + 1, :, :n], 0.125, causal)
+        assert np.array_equal(o[b:b + 1], od) and np.array_equal(lse[b:b + 1], ld)
+    # a permuted table over a permuted pool gives the same numbers
+    perm = rng.permutation(B * nb)
+    inv = np.argsort(perm)
+    o2, l2 = oracle.prefill_paged(q, kc[perm], vc[perm], inv[table].astype(np.int32), sl, 0.125, causal=causal)
+    assert np.array_equal(o, o2) and np.array_equal(lse, l2)
+
+
+def test_rows_before_the_first_key_are_empty():
+    # seq_len < Sq: query i sits at position seq_len - Sq + i, so the first
+    # Sq - seq_len rows see no key (O = 0, LSE = -inf) and the rest see
+    # exactly i - (Sq - seq_len) + 1 keys.
+    c, q, kc, vc, table, sl = case(1, 2, 1, 20, 64, (12,), seed=2)
+    o, lse = oracle.prefill_paged(q, kc, vc, table, sl, c.scale, causal=True)
+    assert np.all(lse[0, :, :8] == -np.inf) and np.all(o[0, :, :8] == 0)
+    assert np.all(np.isfinite(lse[0, :, 8:]))
+    # row 8 sees key 0 only: O = v_0 exactly
+    vv = oracle.paged_gather(vc, table, sl, 64)
+    v0 = torch.from_numpy(vv[0, 0, 0].view(np.int16)).view(torch.bfloat16).double().numpy()
+    assert np.array_equal(o[0, 0, 8], v0)
