@@ -247,7 +247,7 @@ fa_status fa_fwd(const fa_fwd_params *p, void *stream) {
                          (p->dk == 192 && (p->dv == 128 || p->dv == 192)) || (p->dk == 320 && p->dv == 256);
     if (!pair_ok)
         return fail(FA_ERR_UNSUPPORTED,
-                    "fa_fwd: supported (dk, dv) = (64, 64), (128, 128), (256, 256), (192, 128), (320, 256); got "
+                    "fa_fwd: supported (dk, dv) = (64, 64), (128, 128), (192, 192), (256, 256), (192, 128), (320, 256); got "
                     "(%d, %d)",
                     p->dk, p->dv);
     if (!finite_pos(p->scale)) return fail(FA_ERR_INVALID_ARG, "fa_fwd: scale must be finite and > 0");
@@ -332,6 +332,77 @@ fa_status fa_fwd(const fa_fwd_params *p, void *stream) {
         e = fa::launch_prefill(L, static_cast<cudaStream_t>(stream));
     }
     if (e != cudaSuccess) return cuda_fail(e, "fa_fwd: launch");
+    return FA_OK;
+}
+
+fa_status fa_prefill_paged(const fa_prefill_paged_params *p, void *stream) {
+    if (!p) return fail(FA_ERR_INVALID_ARG, "fa_prefill_paged: params is NULL");
+    if (p->B < 0 || p->Hq <= 0 || p->Hkv <= 0 || p->Sq < 0 || p->num_blocks <= 0 || p->max_blocks_per_seq <= 0)
+        return fail(FA_ERR_INVALID_ARG,
+                    "fa_prefill_paged: need B >= 0, Hq > 0, Hkv > 0, Sq >= 0, num_blocks > 0, max_blocks_per_seq > 0");
+    if (p->Hq % p->Hkv != 0)
+        return fail(FA_ERR_INVALID_ARG, "fa_prefill_paged: Hq (%d) %% Hkv (%d) != 0", p->Hq, p->Hkv);
+    if (p->dk != p->dv || (p->dk != 64 && p->dk != 128) || p->block_size != 64)
+        return fail(FA_ERR_UNSUPPORTED, "fa_prefill_paged: supported dk = dv in {64, 128}, block_size = 64 (got %d/%d/%d)",
+                    p->dk, p->dv, p->block_size);
+    if (!finite_pos(p->scale)) return fail(FA_ERR_INVALID_ARG, "fa_prefill_paged: scale must be finite and > 0");
+    if (p->o_dtype != FA_F32 && p->o_dtype != FA_BF16) return fail(FA_ERR_INVALID_ARG, "fa_prefill_paged: o_dtype");
+    if ((long long)p->B * p->Hq > 0x7fffffffLL || p->Sq > (1 << 30) ||
+        (long long)p->max_blocks_per_seq * p->block_size > (1 << 30) || (long long)p->B * p->max_blocks_per_seq > 0x7fffffffLL)
+        return fail(FA_ERR_INVALID_ARG, "fa_prefill_paged: sizes out of range");
+    if (p->B == 0 || p->Sq == 0) return FA_OK;
+    if (!p->q || !p->o || !p->k_cache || !p->v_cache || !p->block_table || !p->seq_lens)
+        return fail(FA_ERR_INVALID_ARG, "fa_prefill_paged: NULL tensor pointer");
+    if (!aligned16(p->q) || !aligned16(p->o) || !aligned16(p->k_cache) || !aligned16(p->v_cache))
+        return fail(FA_ERR_INVALID_ARG, "fa_prefill_paged: q, caches and o must be 16-byte aligned");
+    if (((uintptr_t)p->lse | (uintptr_t)p->block_table | (uintptr_t)p->seq_lens) & 3u)
+        return fail(FA_ERR_INVALID_ARG, "fa_prefill_paged: lse, block_table, seq_lens must be 4-byte aligned");
+    const int ovec = p->o_dtype == FA_F32 ? 4 : 8;
+    if (p->o_ss % ovec || p->o_sh % ovec || p->o_sb % ovec || p->o_ss < p->dv)
+        return fail(FA_ERR_INVALID_ARG, "fa_prefill_paged: o strides must be multiples of %d elements and o_ss >= dv",
+                    ovec);
+    if (!get_encoder()) return fail(FA_ERR_CUDA, "fa_prefill_paged: cuTensorMapEncodeTiled is not available");
+
+    fa::PrefillLaunch L;
+    memset(&L, 0, sizeof L);
+    fa_status st;
+    st = encode_4d(&L.tmQ, p->q, p->dk, p->Sq, p->Hq, p->B, p->q_ss, p->q_sh, p->q_sb, 128, "fa_prefill_paged q");
+    if (st != FA_OK) return st;
+    // The caches as (d, 64 slots, Hkv, num_blocks), 64-row boxes.
+    const int64_t bs = p->block_size;
+    st = encode_4d(&L.tmK, p->k_cache, p->dk, p->block_size, p->Hkv, p->num_blocks, p->dk, bs * p->dk,
+                   bs * p->dk * p->Hkv, 64, "fa_prefill_paged k_cache");
+    if (st != FA_OK) return st;
+    st = encode_4d(&L.tmV, p->v_cache, p->dv, p->block_size, p->Hkv, p->num_blocks, p->dv, bs * p->dv,
+                   bs * p->dv * p->Hkv, 64, "fa_prefill_paged v_cache");
+    if (st != FA_OK) return st;
+    st = encode_4d(&L.tmO, p->o, p->dv, p->Sq, p->Hq, p->B, p->o_ss, p->o_sh, p->o_sb, 128, "fa_prefill_paged o",
+                   p->o_dtype == FA_F32 ? 4 : 2);
+    if (st != FA_OK) return st;
+    L.B = p->B;
+    L.Hq = p->Hq;
+    L.Hkv = p->Hkv;
+    L.Sq = p->Sq;
+    L.Sk = 0;
+    L.dk = p->dk;
+    L.dv = p->dv;
+    L.scale = p->scale;
+    L.causal = p->causal ? 1 : 0;
+    L.o = p->o;
+    L.o_sb = p->o_sb;
+    L.o_sh = p->o_sh;
+    L.o_ss = p->o_ss;
+    L.o_bf16 = p->o_dtype == FA_BF16;
+    L.lse = p->lse;
+    L.has_mods = false;
+    L.block_table = p->block_table;
+    L.seq_lens = p->seq_lens;
+    L.max_blocks = p->max_blocks_per_seq;
+    L.num_blocks = p->num_blocks;
+    int sms = 0;
+    cudaError_t e = num_sms(&sms);
+    if (e == cudaSuccess) e = fa::launch_prefill2(L, sms, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "fa_prefill_paged: launch");
     return FA_OK;
 }
 

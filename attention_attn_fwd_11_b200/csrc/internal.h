@@ -23,6 +23,13 @@ struct PrefillLaunch {
     float *lse;
     ScoreMods mods;  // all-zero: no modifiers
     bool has_mods;   // a mask, a softcap or sinks is given
+    // Paged K/V (two-tile kernel only; block_table == NULL: dense K/V).
+    // tmK / tmV then view the caches [num_blocks, Hkv, 64, d] as
+    // (d, 64, Hkv, num_blocks) with 64-row boxes, and the keys of sequence b
+    // are min(seq_lens[b], max_blocks * 64) (Sk is unused).
+    const int32_t *block_table;
+    const int32_t *seq_lens;
+    int max_blocks, num_blocks;
 };
 // Returns cudaSuccess or the launch error.
 cudaError_t launch_prefill(const PrefillLaunch &L, cudaStream_t stream);

@@ -74,7 +74,18 @@ struct Prefill2Args {
     int64_t o_sb, o_sh, o_ss;
     int o_bf16;
     float *lse;
+    // Paged K/V: block_table [B, max_blocks] and seq_lens [B] (NULL: dense).
+    const int32_t *block_table;
+    const int32_t *seq_lens;
+    int max_blocks, num_blocks;
 };
+
+// Keys of batch entry b: Sk, or its clamped sequence length when paged.
+FA_DEV int p2_keys(const Prefill2Args &a, int b) {
+    if (!a.seq_lens) return a.Sk;
+    const int n = __ldg(a.seq_lens + b);
+    return n < 0 ? 0 : min(n, a.max_blocks * 64);
+}
 
 template <int D>
 struct P2Cfg {
@@ -142,10 +153,11 @@ constexpr float kP2RescaleThreshold = 8.0f;
 #endif
 
 // One unit: query rows [q0, q0 + 256) of head hq in batch b, as two
-// 128-row tiles with n0 and n1 key tiles (N = the larger).  Plain scalars,
-// never an indexed array, so that a unit's fields stay in registers.
+// 128-row tiles with n0 and n1 key tiles (N = the larger) over Sk keys.
+// Plain scalars, never an indexed array, so that a unit's fields stay in
+// registers.
 struct UnitInfo {
-    int b, hq, q0, n0, n1, N;
+    int b, hq, q0, n0, n1, N, Sk;
     FA_DEV int nt(int i) const { return i ? n1 : n0; }
 };
 
@@ -158,6 +170,7 @@ FA_DEV bool p2_unit(const Prefill2Args &a, int round, UnitInfo &u) {
     u.b = bh / a.Hq;
     u.hq = bh % a.Hq;
     u.q0 = qp * 256;
+    u.Sk = p2_keys(a, u.b);
     int n[2];
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
@@ -165,8 +178,8 @@ FA_DEV bool p2_unit(const Prefill2Args &a, int round, UnitInfo &u) {
         n[i] = 0;
         if (r0 < a.Sq) {
             const int last = min(r0 + 127, a.Sq - 1);
-            int kmax = a.Sk - 1;
-            if (a.causal) kmax = min(kmax, last + a.Sk - a.Sq);
+            int kmax = u.Sk - 1;
+            if (a.causal) kmax = min(kmax, last + u.Sk - a.Sq);
             n[i] = kmax < 0 ? 0 : kmax / 128 + 1;
         }
     }
@@ -271,15 +284,42 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             UnitInfo u;
             for (int r = 0; ok && p2_unit(a, r, u); ++r, ++uc) {
                 const int hkv = u.hq / a.group;
+                // Key tile t of K or V into the ring slot at dst.  Dense: one
+                // 128-row box per 64-column chunk.  Paged: the tile's two
+                // 64-key blocks, each a 64-row box per chunk, land 8 KB apart
+                // -- the layout one 128-row box gives under the 128-byte
+                // swizzle.  A block past the sequence's last re-reads the last
+                // (its keys are masked); an entry outside [0, num_blocks) is
+                // latched as FA_DEVERR_BAD_BLOCK and block 0 read instead.
+                auto load_tile = [&](uint32_t dst, const CUtensorMap *tm, uint32_t full, int t) {
+                    if (a.block_table) {
+                        const int nblk = (u.Sk + 63) / 64;
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const int j = min(2 * t + h, nblk - 1);
+                            int blk = __ldg(a.block_table + (int64_t)u.b * a.max_blocks + j);
+                            if (blk < 0 || blk >= a.num_blocks) {
+                                atomicCAS(&g_prefill2_err, 0, 2 /* FA_DEVERR_BAD_BLOCK */);
+                                blk = 0;
+                            }
+#pragma unroll
+                            for (int c = 0; c < C::NCH; ++c)
+                                tma_load_4d(dst + c * C::KV_CHUNK + h * (C::KV_CHUNK / 2), tm, full, c * 64, 0, hkv,
+                                            blk);
+                        }
+                    } else {
+#pragma unroll
+                        for (int c = 0; c < C::NCH; ++c)
+                            tma_load_4d(dst + c * C::KV_CHUNK, tm, full, c * 64, t * BN, hkv, u.b);
+                    }
+                };
                 auto load_k = [&](int t, int kt) -> bool {
                     const int sk = kt % NSTK;
                     if (!mbar_wait(k_empty(sk), ((uint32_t)(kt / NSTK) & 1u) ^ 1u, abort_flag, &g_prefill2_err))
                         return false;
                     TRACE(1, t, 0);
                     mbar_arrive_expect_tx(k_full(sk), C::KV_BYTES);
-#pragma unroll
-                    for (int c = 0; c < C::NCH; ++c)
-                        tma_load_4d(sK + sk * C::KV_BYTES + c * C::KV_CHUNK, &tmK, k_full(sk), c * 64, t * BN, hkv, u.b);
+                    load_tile(sK + sk * C::KV_BYTES, &tmK, k_full(sk), t);
                     issued_k = kt + 1;
                     return true;
                 };
@@ -307,9 +347,7 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                     }
                     TRACE(2, t, 0);
                     mbar_arrive_expect_tx(v_full(sv), C::KV_BYTES);
-#pragma unroll
-                    for (int c = 0; c < C::NCH; ++c)
-                        tma_load_4d(sV + sv * C::KV_BYTES + c * C::KV_CHUNK, &tmV, v_full(sv), c * 64, t * BN, hkv, u.b);
+                    load_tile(sV + sv * C::KV_BYTES, &tmV, v_full(sv), t);
                     issued_v = kc + 1;
                 }
             }
@@ -507,7 +545,7 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             if (!mbar_wait(bar(P2_USTART + ti), (uint32_t)uc & 1u, abort_flag, &g_prefill2_err)) break;
             const int n = u.nt(ti);
             const int qrow = u.q0 + 128 * ti + row;
-            const int lim_all = a.causal ? min(a.Sk, qrow + a.Sk - a.Sq + 1) : a.Sk;
+            const int lim_all = a.causal ? min(u.Sk, qrow + u.Sk - a.Sq + 1) : u.Sk;
             const float slope = MODS ? alibi_slope(a.mods, u.hq) : 1.f;
             const __half *mrow = MODS ? mask_row(a.mods, u.b, u.hq, qrow, a.Sq) : nullptr;
             (void)slope;
@@ -539,7 +577,7 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 if (lane == 0) TRACE(11 + ti, t, qd);
                 const int lim = lim_all - t * BN;
                 if (transform) {
-                    modify_scores<BN>(x, a.mods, a.scale, slope, mrow, t * BN, a.Sk, lim);
+                    modify_scores<BN>(x, a.mods, a.scale, slope, mrow, t * BN, u.Sk, lim);
                 } else if (lim < BN) {
 #pragma unroll
                     for (int k = 0; k < BN; ++k)
@@ -816,6 +854,10 @@ static cudaError_t launch_p2(const PrefillLaunch &L, int num_sms, cudaStream_t s
     a.o_ss = L.o_ss;
     a.o_bf16 = L.o_bf16;
     a.lse = L.lse;
+    a.block_table = L.block_table;
+    a.seq_lens = L.seq_lens;
+    a.max_blocks = L.max_blocks;
+    a.num_blocks = L.num_blocks;
 #if defined(FA_P2_SETMAXNREG) && FA_P2_THREADS == 384
     {
         // The register split inside the kernel needs the full launch allocation.

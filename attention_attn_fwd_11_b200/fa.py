@@ -45,6 +45,14 @@ class PagedParams(ctypes.Structure):
                 ("workspace_bytes", ctypes.c_size_t)]
 
 
+class PrefillPagedParams(ctypes.Structure):
+    _fields_ = [("q", _vp), ("q_sb", _i64), ("q_sh", _i64), ("q_ss", _i64), ("k_cache", _vp), ("v_cache", _vp),
+                ("block_table", _vp), ("seq_lens", _vp), ("max_blocks_per_seq", _i32), ("B", _i32), ("Hq", _i32),
+                ("Hkv", _i32), ("Sq", _i32), ("dk", _i32), ("dv", _i32), ("block_size", _i32), ("num_blocks", _i32),
+                ("scale", ctypes.c_float), ("causal", _i32), ("o", _vp), ("o_sb", _i64), ("o_sh", _i64),
+                ("o_ss", _i64), ("lse", _vp), ("o_dtype", _i32)]
+
+
 class GatherParams(ctypes.Structure):
     _fields_ = [("q", _vp), ("kv_rows", _vp), ("n_rows", _i64), ("row_stride", _i64), ("dk", _i32), ("dv", _i32),
                 ("v_offset", _i32), ("idx", _vp), ("topk", _i32), ("key_pos", _vp), ("q_pos", _vp), ("T", _i32),
@@ -72,6 +80,8 @@ def load():
         lib = ctypes.CDLL(LIB_PATH)
         lib.fa_fwd.argtypes = [ctypes.POINTER(FwdParams), _vp]
         lib.fa_fwd.restype = _i32
+        lib.fa_prefill_paged.argtypes = [ctypes.POINTER(PrefillPagedParams), _vp]
+        lib.fa_prefill_paged.restype = _i32
         lib.fa_decode_paged_workspace_size.argtypes = [ctypes.POINTER(PagedParams), ctypes.POINTER(ctypes.c_size_t)]
         lib.fa_decode_paged_workspace_size.restype = _i32
         lib.fa_decode_paged.argtypes = [ctypes.POINTER(PagedParams), _vp]
@@ -229,6 +239,51 @@ def decode_paged(q, k_cache, v_cache, block_table, seq_lens, scale=None, num_spl
         workspace = torch.empty(max(n, 256), device=q.device, dtype=torch.uint8)
     p = paged_params(q, k_cache, v_cache, block_table, seq_lens, out, lse, scale, num_splits, workspace)
     _check(load().fa_decode_paged(ctypes.byref(p), _stream(stream)))
+    return out, lse
+
+
+# ----------------------------------------------------------- paged prefill --
+
+def prefill_paged_params(q, k_cache, v_cache, block_table, seq_lens, o, lse, scale, causal):
+    B, Hq, Sq, dk = q.shape
+    nb, Hkv, bs, _ = k_cache.shape
+    p = PrefillPagedParams()
+    p.q, p.q_sb, p.q_sh, p.q_ss = _ptr(q), q.stride(0), q.stride(1), q.stride(2)
+    p.k_cache, p.v_cache = _ptr(k_cache), _ptr(v_cache)
+    p.block_table, p.seq_lens = _ptr(block_table), _ptr(seq_lens)
+    p.max_blocks_per_seq = block_table.shape[1]
+    p.B, p.Hq, p.Hkv, p.Sq, p.dk, p.dv = B, Hq, Hkv, Sq, dk, v_cache.shape[3]
+    p.block_size, p.num_blocks = bs, nb
+    p.scale, p.causal = scale, 1 if causal else 0
+    p.o, p.o_sb, p.o_sh, p.o_ss = _ptr(o), o.stride(0), o.stride(1), o.stride(2)
+    p.lse = _ptr(lse)
+    p.o_dtype = _odt(o.dtype)
+    return p
+
+
+def prefill_paged(q, k_cache, v_cache, block_table, seq_lens, scale=None, causal=True, out=None,
+                  return_lse=True, out_dtype=torch.float32, stream=None):
+    """Chunked prefill over a paged cache (fa_prefill_paged).  q [B,Hq,Sq,d]
+    bf16 (head dim contiguous); caches [num_blocks,Hkv,64,d] bf16
+    contiguous; block_table int32 [B,max_blocks]; seq_lens int32 [B] (keys
+    including the Sq new ones).  Returns (O [B,Hq,Sq,d], LSE [B,Hq,Sq] or
+    None)."""
+    _need_cuda(q, k_cache, v_cache, block_table, seq_lens, out)
+    for t in (q, k_cache, v_cache):
+        if t.dtype != torch.bfloat16 or t.stride(-1) != 1:
+            raise ValueError("q and the caches must be bf16 with a contiguous head dimension")
+    if not (k_cache.is_contiguous() and v_cache.is_contiguous()):
+        raise ValueError("the caches must be contiguous")
+    if block_table.dtype != torch.int32 or seq_lens.dtype != torch.int32 or not block_table.is_contiguous():
+        raise ValueError("block_table and seq_lens must be contiguous int32")
+    B, Hq, Sq, dk = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(dk)
+    if out is None:
+        out = torch.empty((B, Hq, Sq, v_cache.shape[3]), device=q.device, dtype=out_dtype)
+    lse = torch.empty((B, Hq, Sq), device=q.device, dtype=torch.float32) if return_lse else None
+    p = prefill_paged_params(q, k_cache, v_cache, block_table, seq_lens, out, lse, scale, causal)
+    _check(load().fa_prefill_paged(ctypes.byref(p), _stream(stream)))
     return out, lse
 
 

@@ -55,6 +55,7 @@ NCU_TRAFFIC = {
     "causal_mha_b2_h16_s2048_dk192_dv128": 73713408,
     "causal_gqa_b2_hq16_hkv4_s2048_dk192_dv192": 40004096,
     "kv_dequant causal_mha_q8_0kv_b2_h16_s2048_d128": 17835776,
+    "paged_prefill_gqa_b16_hq32_hkv8_sq512_d128_bs64": 651085568,
     "causal_gqa_b1_hq16_hkv4_s4096_dk320_dv256": 77931264,
 }
 
@@ -285,6 +286,30 @@ def quant_prefill_workload(torch, fa, W_, c, qtype, l2, dequant_only=False):
     return launch, n, dq_bytes, 1 if dequant_only else 2
 
 
+def paged_prefill_workload(torch, fa, W_, c, l2):
+    """Chunked prefill over the paged cache: one fa_prefill_paged per step."""
+    import ctypes
+    q0, kc0, vc0, table0, sl0 = W_.paged_prefill_inputs(c)
+    foot = (q0.numel() + kc0.numel() + vc0.numel()) * 2 + c.B * c.Hq * c.Sq * (c.d * 4 + 4)
+    n = rotation_copies(foot, l2)
+    lib = fa.load()
+    bufs, params = [], []
+    for i in range(n):
+        q, kc, vc, tb, sl = q0.cuda(), kc0.cuda(), vc0.cuda(), table0.cuda(), sl0.cuda()
+        o = torch.empty(c.B, c.Hq, c.Sq, c.d, device="cuda")
+        lse = torch.empty(c.B, c.Hq, c.Sq, device="cuda")
+        bufs.append((q, kc, vc, tb, sl, o, lse))
+        params.append(fa.prefill_paged_params(q, kc, vc, tb, sl, o, lse, c.scale, c.causal))
+
+    def launch(i):
+        st = lib.fa_prefill_paged(ctypes.byref(params[i]), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+        if st != 0:
+            raise RuntimeError(lib.fa_last_error().decode())
+
+    launch.keep = bufs
+    return launch, n, c.flops(sl0), 1
+
+
 def paged_workload(torch, fa, W_, c, l2):
     q0, kc0, vc0, tb0, sl0 = W_.paged_inputs(c)
     byts = W_.paged_bytes(c, sl0, tb0.shape[1])
@@ -428,7 +453,7 @@ def run_only(args):
     l2 = torch.cuda.get_device_properties(0).L2_cache_size
     table = {c.name: c for c in (W_.TINY_FULL, W_.CAUSAL_MHA, W_.GQA_FULL, W_.MODS_C2, W_.CAUSAL_DK192,
                                  W_.CAUSAL_DK192_DV192, W_.CAUSAL_DK320, W_.PAGED_GQA, W_.LATENT_SPARSE,
-                                 W_.QUANT_C2)}
+                                 W_.QUANT_C2, W_.PAGED_PREFILL)}
     table["kv_dequant_" + W_.QUANT_C2.name] = W_.QUANT_C2
     if args.only not in table:
         raise SystemExit("unknown workload %r; one of %s" % (args.only, sorted(table)))
@@ -440,6 +465,9 @@ def run_only(args):
     elif isinstance(c, W_.PrefillCase):
         launch, n, work, kpl = prefill_workload(torch, fa, W_, c, l2)
         unit, amount = "TFLOP/s", c.flops / 1e12
+    elif isinstance(c, W_.PagedPrefillCase):
+        launch, n, work, kpl = paged_prefill_workload(torch, fa, W_, c, l2)
+        unit, amount = "TFLOP/s", work / 1e12
     elif isinstance(c, W_.PagedCase):
         launch, n, work, kpl = paged_workload(torch, fa, W_, c, l2)
         unit, amount = "GB/s", work / 1e9
@@ -610,6 +638,20 @@ def main():
                        "dequant": {"ms_per_step": round(perd, 5), "bytes_per_step": dq_bytes,
                                    "roofline": roofline("hbm", dq_bytes / (perd * 1e-3) / 1e9, peaks["hbm_gbs"],
                                                         "GB/s", NCU_TRAFFIC.get("kv_dequant " + qc.name))}}
+        # chunked prefill over the paged cache
+        ppc = W_.PAGED_PREFILL
+        launch, ncopy, pflops, kpl = paged_prefill_workload(torch, fa, W_, ppc, l2)
+        ms2, st2 = time_graph(torch, launch, ncopy, Ks, Wm, dist)
+        ms2 = max_over_ranks(torch, dist, ms2)
+        per = ms2 / st2
+        ach = pflops / (per * 1e-3) / 1e12
+        wl[ppc.name] = {"value": round(sum_over_ranks(torch, dist, pflops * st2) / (ms2 * 1e-3) / 1e12, 2),
+                        "unit": "TFLOP/s", "ms_per_step": round(per, 5), "steps": st2, "l2_copies": ncopy,
+                        "flops_per_step": pflops,
+                        "roofline": roofline("tensor", ach, peaks["bf16_tflops"], "TFLOP/s",
+                                             NCU_TRAFFIC.get(ppc.name))}
+        result["gpu_launches"] += st2 * kpl
+        del launch
         pc = W_.PAGED_GQA
         launch, ncopy, byts, kpl = paged_workload(torch, fa, W_, pc, l2)
         ms2, st2 = time_graph(torch, launch, ncopy, Ks, Wm, dist)

@@ -130,6 +130,52 @@ typedef struct {
 fa_status fa_fwd(const fa_fwd_params *p, void *stream);
 
 /*
+ * fa_prefill_paged -- chunked prefill over a paged KV cache: the decode call
+ * of fa_decode_paged with Sq > 1 new query rows per sequence, computed by the
+ * prefill kernel with its key tiles gathered through the block table.
+ *   q: [B, Hq, Sq, dk] bf16, strides as in fa_fwd (multiples of 8 elements,
+ *     16-byte aligned base).
+ *   k_cache: [num_blocks, Hkv, block_size, dk], v_cache: [num_blocks, Hkv,
+ *     block_size, dv], bf16 contiguous, 16-byte aligned.
+ *   block_table: [B, max_blocks_per_seq] int32; key j of sequence b is slot
+ *     j % block_size of block block_table[b][j / block_size].
+ *   seq_lens: [B] int32, the keys of each sequence INCLUDING its Sq new
+ *     tokens (the caller writes their K/V into the cache first); values are
+ *     clamped to [0, max_blocks_per_seq * block_size].
+ *   causal != 0: query i of sequence b sits at position seq_lens[b] - Sq + i
+ *     and sees keys j <= that position (bottom-right, as in fa_fwd); a row
+ *     with no visible key (seq_lens[b] < Sq) gets O = 0, LSE = -inf.
+ *   o: [B, Hq, Sq, dv] (o_dtype) with strides o_sb, o_sh, o_ss (multiples of
+ *     4 elements for fp32, 8 for bf16; o_ss >= dv); lse: NULL or [B, Hq, Sq]
+ *     fp32 contiguous.
+ * Supported: dk == dv in {64, 128}, block_size == 64, Hq % Hkv == 0.  No
+ * score modifiers on this path.
+ * Cache slots past seq_lens[b] inside the sequence's last block are read and
+ * must hold finite values (their weight is zero, and 0 * NaN is NaN).
+ * Entries past a sequence's last block are never read.  A block id outside
+ * [0, num_blocks) is latched as FA_DEVERR_BAD_BLOCK and block 0 is read in
+ * its place (that sequence's output is then meaningless).
+ * Sq == 0 or B == 0 is a no-op.
+ */
+typedef struct {
+    const void *q;
+    int64_t q_sb, q_sh, q_ss;
+    const void *k_cache, *v_cache;
+    const int32_t *block_table;
+    const int32_t *seq_lens;
+    int max_blocks_per_seq;
+    int B, Hq, Hkv, Sq, dk, dv, block_size, num_blocks;
+    float scale;
+    int causal;
+    void *o;
+    int64_t o_sb, o_sh, o_ss;
+    float *lse;
+    int o_dtype; /* fa_dtype */
+} fa_prefill_paged_params;
+
+fa_status fa_prefill_paged(const fa_prefill_paged_params *p, void *stream);
+
+/*
  * fa_decode_paged -- one query token per sequence over a paged KV cache,
  * split along the keys, partial results merged by a log-sum-exp combine.
  *   q: [B, Hq, dk] bf16 contiguous.
@@ -146,6 +192,8 @@ fa_status fa_fwd(const fa_fwd_params *p, void *stream);
  *     bytes, 256-byte aligned; it holds the split partials and is
  *     overwritten on every call.
  * Supported: dk == dv == 128, block_size == 64, Hq / Hkv in {1, 2, 4, 8}.
+ * Cache slots past seq_lens[b] inside the sequence's last block are read and
+ * must hold finite values (their weight is zero, and 0 * NaN is NaN).
  * A block id outside [0, num_blocks) is latched as FA_DEVERR_BAD_BLOCK and
  * block 0 is read in its place (the output for that sequence is then
  * meaningless).

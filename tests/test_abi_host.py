@@ -137,6 +137,44 @@ def test_gather_workspace_size_and_validation():
     assert lib.fa_decode_gather(ctypes.byref(gather_params(T=0)), None) == fa.FA_OK
 
 
+def prefill_paged_params(**kw):
+    p = fa.PrefillPagedParams()
+    base = dict(q=16, q_sb=16 * 32 * 512 * 128, q_sh=512 * 128, q_ss=128, k_cache=32, v_cache=48, block_table=64,
+                seq_lens=80, max_blocks_per_seq=128, B=16, Hq=32, Hkv=8, Sq=512, dk=128, dv=128, block_size=64,
+                num_blocks=4096, scale=0.088, causal=1, o=96, o_sb=16 * 32 * 512 * 128, o_sh=512 * 128, o_ss=128,
+                lse=0, o_dtype=0)
+    base.update(kw)
+    for k_, v_ in base.items():
+        setattr(p, k_, v_)
+    return p
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(dk=256, dv=256), fa.FA_ERR_UNSUPPORTED),
+    (dict(dk=128, dv=64), fa.FA_ERR_UNSUPPORTED),
+    (dict(block_size=16), fa.FA_ERR_UNSUPPORTED),
+    (dict(Hq=30), fa.FA_ERR_INVALID_ARG),
+    (dict(num_blocks=0), fa.FA_ERR_INVALID_ARG),
+    (dict(max_blocks_per_seq=0), fa.FA_ERR_INVALID_ARG),
+    (dict(scale=0.0), fa.FA_ERR_INVALID_ARG),
+    (dict(o_dtype=7), fa.FA_ERR_INVALID_ARG),
+    (dict(k_cache=40), fa.FA_ERR_INVALID_ARG),             # not 16-byte aligned
+    (dict(block_table=66), fa.FA_ERR_INVALID_ARG),         # not 4-byte aligned
+    (dict(seq_lens=0), fa.FA_ERR_INVALID_ARG),
+    (dict(o_ss=120), fa.FA_ERR_INVALID_ARG),               # o_ss < dv
+    (dict(o_sh=6), fa.FA_ERR_INVALID_ARG),                 # fp32 strides must be multiples of 4
+])
+def test_prefill_paged_rejects(kw, status):
+    assert fa.load().fa_prefill_paged(ctypes.byref(prefill_paged_params(**kw)), None) == status
+
+
+def test_prefill_paged_null_and_noop():
+    lib = fa.load()
+    assert lib.fa_prefill_paged(None, None) == fa.FA_ERR_INVALID_ARG
+    assert lib.fa_prefill_paged(ctypes.byref(prefill_paged_params(B=0)), None) == fa.FA_OK
+    assert lib.fa_prefill_paged(ctypes.byref(prefill_paged_params(Sq=0)), None) == fa.FA_OK
+
+
 def dequant_params(**kw):
     p = fa.KvDequantParams()
     base = dict(src=2, type=fa.FA_KV_Q8_0, n_rows=1024, row_elems=128, src_row_bytes=136, dst=16, dst_row_stride=128)

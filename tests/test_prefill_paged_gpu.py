@@ -1,0 +1,84 @@
+"""Chunked prefill over a paged cache (fa_prefill_paged) against the oracle's
+prefill_paged (table gather + dense attention per sequence), element by
+element on the same seeded inputs."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from attention_attn_fwd_11_b200 import fa
+from attention_attn_fwd_11_b200 import workloads as W
+from parity import check
+
+pytestmark = pytest.mark.gpu
+
+
+def run(B, Hq, Hkv, Sq, d, lens, causal, seed, out_dtype=torch.float32, seq_major=False):
+    c = W.PagedPrefillCase("t", B, Hq, Hkv, Sq, d, 0, 0, causal=causal, seed=seed, lens=tuple(lens))
+    q, kc, vc, table, sl = W.paged_prefill_inputs(c)
+    qd = q.cuda()
+    if seq_major:  # Q stored [B, Sq, Hq, d], viewed as [B, Hq, Sq, d]
+        qd = q.permute(0, 2, 1, 3).contiguous().cuda().permute(0, 2, 1, 3)
+    o, lse = fa.prefill_paged(qd, kc.cuda(), vc.cuda(), table.cuda(), sl.cuda(), scale=c.scale, causal=causal,
+                              out_dtype=out_dtype)
+    torch.cuda.synchronize()
+    assert fa.device_error() == 0
+    o_ref, l_ref = oracle.prefill_paged(W.bits(q), W.bits(kc), W.bits(vc), table.numpy(), sl.numpy(), c.scale,
+                                        causal)
+    bf = out_dtype == torch.bfloat16
+    check(o, o_ref, lse, l_ref, max_abs=2e-2 if bf else 1e-2, min_cos=0.9999 if bf else 0.99999,
+          what="paged prefill d%d Sq%d lens %s causal %d" % (d, Sq, list(lens), causal))
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+def test_ragged_lengths_gqa(d, causal):
+    # Sq = 300 spans a two-tile unit plus a partial one; lengths end inside
+    # blocks, inside the second half of a 128-key tile, and on a block edge.
+    run(4, 8, 2, 300, d, (300, 517, 1088, 333), causal, seed=d)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_short_sequences_and_empty_rows(d):
+    # seq_len < Sq: the first rows see no key; seq_len = 0: every row empty;
+    # 1 key: the tile's second block lies past the end.
+    run(3, 4, 4, 40, d, (17, 0, 1), True, seed=3)
+
+
+def test_one_new_row_is_the_decode():
+    run(5, 8, 1, 1, 128, (1, 64, 65, 1000, 4096), True, seed=4)
+
+
+def test_bf16_output_and_sequence_major_q():
+    run(2, 8, 2, 200, 128, (700, 260), True, seed=5, out_dtype=torch.bfloat16, seq_major=True)
+
+
+def test_bad_block_id_is_latched():
+    c = W.PagedPrefillCase("t", 2, 4, 2, 64, 64, 0, 0, seed=6, lens=(200, 100))
+    q, kc, vc, table, sl = W.paged_prefill_inputs(c)
+    bad = table.clone()
+    bad[1, 1] = kc.shape[0] + 5  # outside [0, num_blocks)
+    fa.prefill_paged(q.cuda(), kc.cuda(), vc.cuda(), bad.cuda(), sl.cuda(), causal=True)
+    torch.cuda.synchronize()
+    assert fa.device_error(clear=True) == 2  # FA_DEVERR_BAD_BLOCK
+    assert fa.device_error() == 0
+
+
+def test_workload_sampled_rows():
+    # The benchmark's workload at full size: two sequences, the first and the
+    # last 64 new rows of every head, against the oracle.  Rows [r0, r0 + n)
+    # of a sequence of L keys are the last n rows of one of L - Sq + r0 + n.
+    c = W.PAGED_PREFILL
+    q, kc, vc, table, sl = W.paged_prefill_inputs(c)
+    o, lse = fa.prefill_paged(q.cuda(), kc.cuda(), vc.cuda(), table.cuda(), sl.cuda(), scale=c.scale, causal=True)
+    torch.cuda.synchronize()
+    assert fa.device_error() == 0
+    kb, vb = W.bits(kc), W.bits(vc)
+    n = 64
+    for b in (0, int(np.argmax(sl.numpy()))):
+        for r0 in (0, c.Sq - n):
+            Lb = int(sl[b]) - c.Sq + r0 + n
+            o_ref, l_ref = oracle.prefill_paged(W.bits(q[b:b + 1, :, r0:r0 + n]), kb, vb, table[b:b + 1].numpy(),
+                                                np.array([Lb], np.int32), c.scale, True)
+            check(o[b:b + 1, :, r0:r0 + n], o_ref, lse[b:b + 1, :, r0:r0 + n], l_ref,
+                  what="paged prefill workload b%d rows %d.." % (b, r0))
