@@ -25,6 +25,12 @@ def randn_bf16(shape, seed: int) -> torch.Tensor:
     return torch.randn(*shape, generator=g, dtype=torch.float32).to(torch.bfloat16)
 
 
+def randn_scaled_bf16(shape, seed: int, std: float) -> torch.Tensor:
+    """N(0, std^2) drawn in float32, rounded to bf16."""
+    g = torch.Generator().manual_seed(int(seed))
+    return (torch.randn(*shape, generator=g, dtype=torch.float32) * std).to(torch.bfloat16)
+
+
 def bits(t: torch.Tensor) -> np.ndarray:
     """bf16 tensor (CPU or CUDA) -> numpy uint16 bit patterns, same shape."""
     t = t.detach()
@@ -332,3 +338,40 @@ def latent_flops(c: LatentCase, n_visible: int) -> float:
 
 
 LATENT_SPARSE = LatentCase("latent_sparse_t32_hq128_dk576_dv512_top2048", 32, 128, 65536, 2048, seed=5)
+
+
+# ---------------------------------------------------------- MLA decode tail --
+# The projections after the latent decode: o_lat [T, Hq, R] -> out-absorb
+# w_abs [Hq, V, R] -> u [T, Hq*V] -> o-projection w_o [Hd, Hq*V] -> y [T, Hd].
+# o_lat ~ N(0, 1); weights ~ N(0, 1/fan_in) so that u and y stay O(1); all
+# rounded to bf16.  Seeds: o_lat 1000 + c, w_abs 2000 + c, w_o 3000 + c.
+
+@dataclass
+class MlaTailCase:
+    name: str
+    T: int
+    Hq: int
+    R: int = 512       # kv_lora_rank
+    V: int = 128       # v_head_dim
+    Hd: int = 7168     # hidden
+    seed: int = 0
+
+    @property
+    def flops(self) -> float:
+        return 2.0 * self.T * self.Hq * self.V * (self.R + self.Hd)
+
+    @property
+    def bytes(self) -> int:
+        """Weights, the latent input and the fp32 output, each once."""
+        return 2 * (self.Hq * self.V * self.R + self.Hd * self.Hq * self.V + self.T * self.Hq * self.R) + \
+            4 * self.T * self.Hd
+
+
+def mla_tail_inputs(c: MlaTailCase):
+    o_lat = randn_bf16((c.T, c.Hq, c.R), 1000 + c.seed)
+    w_abs = randn_scaled_bf16((c.Hq, c.V, c.R), 2000 + c.seed, 1.0 / math.sqrt(c.R))
+    w_o = randn_scaled_bf16((c.Hd, c.Hq * c.V), 3000 + c.seed, 1.0 / math.sqrt(c.Hq * c.V))
+    return o_lat, w_abs, w_o
+
+
+MLA_TAIL = MlaTailCase("mla_tail_t32_hq128_r512_v128_hidden7168", 32, 128, seed=10)

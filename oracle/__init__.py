@@ -59,6 +59,8 @@ def _load():
         lib.oracle_decode_latent.restype = i32
         lib.oracle_lse_combine.argtypes = [i32, i32, i32, P, P, P, P]
         lib.oracle_lse_combine.restype = None
+        lib.oracle_mla_tail.argtypes = [P, P, P, i32, i32, i32, i32, i32, P, P]
+        lib.oracle_mla_tail.restype = i32
         lib.oracle_round_bf16.argtypes = [f64]
         lib.oracle_round_bf16.restype = ctypes.c_uint16
         lib.oracle_dequant_rows.argtypes = [P, i32, i64, i32, i64, P]
@@ -283,3 +285,22 @@ def dequant_rows(src, qtype, row_elems):
     if rc:
         raise ValueError("oracle_dequant_rows: bad arguments")
     return out
+
+
+def mla_tail(o_lat, w_abs, w_o):
+    """MLA decode tail.  o_lat [T, Hq, R] (latent attention output),
+    w_abs [Hq, V, R] (out-absorb), w_o [Hd, Hq*V] (o-projection, row = output
+    feature), all bf16 bits.  Returns (u [T, Hq*V], y [T, Hd]) float64."""
+    o_lat = np.ascontiguousarray(_u16(o_lat))
+    w_abs = np.ascontiguousarray(_u16(w_abs))
+    w_o = np.ascontiguousarray(_u16(w_o))
+    T, Hq, R = o_lat.shape
+    _, V, R2 = w_abs.shape
+    Hd, K = w_o.shape
+    if w_abs.shape[0] != Hq or R2 != R or K != Hq * V:
+        raise ValueError("mla_tail: shapes do not match")
+    u = np.zeros((T, Hq * V), np.float64)
+    y = np.zeros((T, Hd), np.float64)
+    if _load().oracle_mla_tail(_ptr(o_lat), _ptr(w_abs), _ptr(w_o), T, Hq, R, V, Hd, _ptr(u), _ptr(y)):
+        raise ValueError("oracle_mla_tail rejected its arguments")
+    return u, y

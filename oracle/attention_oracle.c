@@ -568,3 +568,46 @@ int oracle_dequant_rows(const uint8_t *src, int type, int64_t n_rows, int row_el
     }
     return 0;
 }
+
+/*
+ * MLA decode tail: the projections that follow the latent attention in
+ * "MLA Decode Attention Kernel API Reference" (AWS Neuron NKI), parameters
+ * out_absorb_w and o_proj_w and the Notes on the two tails.  For every token
+ * t and head h the latent attention output o[t][h][0..R) (R = kv_lora_rank)
+ * is mapped out of the latent space by that head's out_absorb_w[h]
+ * ([V][R], V = v_head_dim):
+ *   u[t][h*V + v] = sum_c w_abs[h][v][c] * o[t][h][c]
+ * and the heads' outputs, concatenated, go through the o-projection:
+ *   y[t][j] = sum_k u[t][k] * w_o[j][k]         (k over Hq*V)
+ * Reading: the page gives o_proj_w as [n_heads * v_head_dim, hidden]; here
+ * it is stored transposed, w_o[j][k] = o_proj_w[k][j] (row = output
+ * feature), which is the same matrix.  u and y are exact sums in double (no
+ * rounding of u).  Inputs are bf16 bits; u is [T][Hq*V], y is [T][Hd].
+ * Returns 0, or -1 on bad arguments.
+ */
+int oracle_mla_tail(const uint16_t *o_lat, const uint16_t *w_abs, const uint16_t *w_o, int T, int Hq, int R, int V,
+                    int Hd, double *u, double *y)
+{
+    if (T < 0 || Hq <= 0 || R <= 0 || V <= 0 || Hd <= 0 || !o_lat || !w_abs || !w_o || !u || !y) return -1;
+    const int64_t K = (int64_t)Hq * V;
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int t = 0; t < T; ++t)
+        for (int h = 0; h < Hq; ++h)
+            for (int v = 0; v < V; ++v) {
+                double acc = 0.0;
+                const uint16_t *w = w_abs + ((int64_t)h * V + v) * R;
+                const uint16_t *o = o_lat + ((int64_t)t * Hq + h) * R;
+                for (int c = 0; c < R; ++c) acc += bf16_bits_to_double(w[c]) * bf16_bits_to_double(o[c]);
+                u[(int64_t)t * K + (int64_t)h * V + v] = acc;
+            }
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int t = 0; t < T; ++t)
+        for (int j = 0; j < Hd; ++j) {
+            double acc = 0.0;
+            const uint16_t *w = w_o + (int64_t)j * K;
+            const double *ut = u + (int64_t)t * K;
+            for (int64_t k = 0; k < K; ++k) acc += ut[k] * bf16_bits_to_double(w[k]);
+            y[(int64_t)t * Hd + j] = acc;
+        }
+    return 0;
+}
