@@ -230,6 +230,21 @@ size_t gather_ws_bytes(const fa_decode_gather_params *p, int splits) {
     return o + ((rows * sizeof(float) + 255) & ~size_t(255));
 }
 
+fa_status check_tail(const fa_mla_tail_params *p) {
+    if (!p) return fail(FA_ERR_INVALID_ARG, "fa_mla_tail: params is NULL");
+    if (p->T < 0 || p->Hq <= 0 || p->R <= 0 || p->V <= 0 || p->Hd <= 0)
+        return fail(FA_ERR_INVALID_ARG, "fa_mla_tail: need T >= 0 and Hq, R, V, Hd > 0");
+    if (p->V != 128 || p->R % 64 != 0 || p->Hd % 128 != 0 || ((int64_t)p->Hq * p->V) % 64 != 0 || p->T > 256)
+        return fail(FA_ERR_UNSUPPORTED,
+                    "fa_mla_tail: supported V = 128, R % 64 == 0, Hd % 128 == 0, T <= 256 (got V %d R %d Hd %d T %d)",
+                    p->V, p->R, p->Hd, p->T);
+    if ((int64_t)p->Hq * p->V > (1 << 30) || p->R > (1 << 20) || p->Hd > (1 << 24))
+        return fail(FA_ERR_INVALID_ARG, "fa_mla_tail: sizes out of range");
+    if (p->y_dtype != FA_F32 && p->y_dtype != FA_BF16) return fail(FA_ERR_INVALID_ARG, "fa_mla_tail: y_dtype");
+    if (p->num_splits < 0) return fail(FA_ERR_INVALID_ARG, "fa_mla_tail: num_splits must be >= 0");
+    return FA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -535,6 +550,63 @@ fa_status fa_decode_gather(const fa_decode_gather_params *p, void *stream) {
     return FA_OK;
 }
 
+fa_status fa_mla_tail_workspace_size(const fa_mla_tail_params *p, size_t *bytes) {
+    fa_status st = check_tail(p);
+    if (st != FA_OK) return st;
+    if (!bytes) return fail(FA_ERR_INVALID_ARG, "fa_mla_tail_workspace_size: bytes is NULL");
+    fa::TailLaunch L;
+    memset(&L, 0, sizeof L);
+    L.T = p->T;
+    L.Hq = p->Hq;
+    L.R = p->R;
+    L.V = p->V;
+    L.Hd = p->Hd;
+    *bytes = fa::mla_tail_ws_bytes(L);
+    return FA_OK;
+}
+
+fa_status fa_mla_tail(const fa_mla_tail_params *p, void *stream) {
+    fa_status st = check_tail(p);
+    if (st != FA_OK) return st;
+    if (p->T == 0) return FA_OK;
+    if (!p->o_lat || !p->w_abs || !p->w_o || !p->y) return fail(FA_ERR_INVALID_ARG, "fa_mla_tail: NULL pointer");
+    if (!aligned16(p->o_lat) || !aligned16(p->w_abs) || !aligned16(p->w_o) || !aligned16(p->y))
+        return fail(FA_ERR_INVALID_ARG, "fa_mla_tail: o_lat, w_abs, w_o and y must be 16-byte aligned");
+    fa::TailLaunch L;
+    memset(&L, 0, sizeof L);
+    L.T = p->T;
+    L.Hq = p->Hq;
+    L.R = p->R;
+    L.V = p->V;
+    L.Hd = p->Hd;
+    L.splits = p->num_splits;
+    const size_t need = fa::mla_tail_ws_bytes(L);
+    if (!p->workspace || p->workspace_bytes < need || ((uintptr_t)p->workspace & 255u))
+        return fail(FA_ERR_WORKSPACE, "fa_mla_tail: workspace must be 256-byte aligned and >= %zu bytes", need);
+    if (!get_encoder()) return fail(FA_ERR_CUDA, "fa_mla_tail: cuTensorMapEncodeTiled is not available");
+    const int NP = (p->T + 15) / 16 * 16;
+    const int64_t K = (int64_t)p->Hq * p->V;
+    // (inner, rows, batch, 1) views; element strides.
+    st = encode_4d(&L.tmAbsA, p->w_abs, p->R, p->V, p->Hq, 1, p->R, (int64_t)p->V * p->R,
+                   (int64_t)p->Hq * p->V * p->R, 128, "fa_mla_tail w_abs");
+    if (st != FA_OK) return st;
+    st = encode_4d(&L.tmAbsB, p->o_lat, p->R, p->T, p->Hq, 1, (int64_t)p->Hq * p->R, p->R,
+                   (int64_t)p->T * p->Hq * p->R, NP, "fa_mla_tail o_lat");
+    if (st != FA_OK) return st;
+    st = encode_4d(&L.tmOA, p->w_o, (int)K, p->Hd, 1, 1, K, K * p->Hd, K * p->Hd, 128, "fa_mla_tail w_o");
+    if (st != FA_OK) return st;
+    st = encode_4d(&L.tmOB, p->workspace, (int)K, p->T, 1, 1, K, K * p->T, K * p->T, NP, "fa_mla_tail u");
+    if (st != FA_OK) return st;
+    L.y = p->y;
+    L.y_bf16 = p->y_dtype == FA_BF16;
+    L.workspace = p->workspace;
+    int sms = 0;
+    cudaError_t e = num_sms(&sms);
+    if (e == cudaSuccess) e = fa::launch_mla_tail(L, sms, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "fa_mla_tail: launch");
+    return FA_OK;
+}
+
 fa_status fa_kv_dequant_n(const fa_kv_dequant_params *p, int n, void *stream) {
     if (!p) return fail(FA_ERR_INVALID_ARG, "fa_kv_dequant: params is NULL");
     if (n < 1 || n > fa::kMaxDequantSegs)
@@ -579,13 +651,14 @@ fa_status fa_kv_dequant(const fa_kv_dequant_params *p, void *stream) { return fa
 
 fa_status fa_device_error(int clear, int *code) {
     if (!code) return fail(FA_ERR_INVALID_ARG, "fa_device_error: code is NULL");
-    int c1 = 0, c2 = 0, c3 = 0, c4 = 0;
+    int c1 = 0, c2 = 0, c3 = 0, c4 = 0, c5 = 0;
     cudaError_t e = fa::prefill_device_error(clear, &c1);
+    if (e == cudaSuccess) e = fa::tail_device_error(clear, &c5);
     if (e == cudaSuccess) e = fa::prefill2_device_error(clear, &c4);
     if (e == cudaSuccess) e = fa::decode_device_error(clear, &c2);
     if (e == cudaSuccess) e = fa::gather_device_error(clear, &c3);
     if (e != cudaSuccess) return cuda_fail(e, "fa_device_error");
-    *code = c1 ? c1 : (c4 ? c4 : (c2 ? c2 : c3));
+    *code = c1 ? c1 : (c4 ? c4 : (c2 ? c2 : (c3 ? c3 : c5)));
     return FA_OK;
 }
 

@@ -85,6 +85,25 @@ struct GatherLaunch {
 cudaError_t launch_decode_gather(const GatherLaunch &L, cudaStream_t stream);
 cudaError_t gather_device_error(int clear, int *code);
 
+// MLA decode tail (mla_tail.cu): out-absorb then o-projection.
+struct TailLaunch {
+    CUtensorMap tmAbsA;  // w_abs as (R, V, Hq): K-major weight rows, 128-row boxes
+    CUtensorMap tmAbsB;  // o_lat as (R, T, Hq): token rows, NP-row boxes
+    CUtensorMap tmOA;    // w_o as (Hq*V, Hd): 128-row boxes
+    CUtensorMap tmOB;    // u (workspace) as (Hq*V, T): NP-row boxes
+    int T, Hq, R, V, Hd;
+    int splits;          // 0: automatic
+    void *y;
+    int y_bf16;
+    void *workspace;     // u [T][Hq*V] bf16
+};
+constexpr int kMaxTailSplits = 8;  // K splits of one tile form one (portable) cluster
+// o-projection K splits for L.splits (0: automatic) on num_sms SMs.
+int mla_tail_splits(const TailLaunch &L, int num_sms);
+size_t mla_tail_ws_bytes(const TailLaunch &L);
+cudaError_t launch_mla_tail(const TailLaunch &L, int num_sms, cudaStream_t stream);
+cudaError_t tail_device_error(int clear, int *code);
+
 // Quantised K/V rows -> bf16 (kv_dequant.cu).  type: 8 = q8_0, 4 = q4_0.
 struct KvDequantLaunch {
     const void *src;

@@ -60,6 +60,12 @@ class GatherParams(ctypes.Structure):
                 ("o_dtype", _i32), ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t)]
 
 
+class MlaTailParams(ctypes.Structure):
+    _fields_ = [("o_lat", _vp), ("w_abs", _vp), ("w_o", _vp), ("T", _i32), ("Hq", _i32), ("R", _i32), ("V", _i32),
+                ("Hd", _i32), ("y", _vp), ("y_dtype", _i32), ("num_splits", _i32), ("workspace", _vp),
+                ("workspace_bytes", ctypes.c_size_t)]
+
+
 class KvDequantParams(ctypes.Structure):
     _fields_ = [("src", _vp), ("type", _i32), ("n_rows", _i64), ("row_elems", _i32), ("src_row_bytes", _i64),
                 ("dst", _vp), ("dst_row_stride", _i64)]
@@ -90,6 +96,10 @@ def load():
         lib.fa_decode_gather_workspace_size.restype = _i32
         lib.fa_decode_gather.argtypes = [ctypes.POINTER(GatherParams), _vp]
         lib.fa_decode_gather.restype = _i32
+        lib.fa_mla_tail_workspace_size.argtypes = [ctypes.POINTER(MlaTailParams), ctypes.POINTER(ctypes.c_size_t)]
+        lib.fa_mla_tail_workspace_size.restype = _i32
+        lib.fa_mla_tail.argtypes = [ctypes.POINTER(MlaTailParams), _vp]
+        lib.fa_mla_tail.restype = _i32
         lib.fa_kv_dequant.argtypes = [ctypes.POINTER(KvDequantParams), _vp]
         lib.fa_kv_dequant.restype = _i32
         lib.fa_kv_dequant_n.argtypes = [ctypes.POINTER(KvDequantParams), _i32, _vp]
@@ -408,3 +418,46 @@ def fwd_quant(q, k_blocks, v_blocks, qtype, dk, dv, scale=None, causal=False, ou
     k, v = kv_dequant_many([(k_blocks, qtype, dk, k_buf), (v_blocks, qtype, dv, v_buf)], stream=stream)
     return fwd(q, k, v, scale=scale, causal=causal, out=out, return_lse=return_lse, out_dtype=out_dtype,
                stream=stream, **mods)
+
+
+# --------------------------------------------------------- MLA decode tail --
+
+def mla_tail_params(o_lat, w_abs, w_o, y, num_splits=0, workspace=None):
+    T, Hq, R = o_lat.shape
+    p = MlaTailParams()
+    p.o_lat, p.w_abs, p.w_o, p.y = _ptr(o_lat), _ptr(w_abs), _ptr(w_o), _ptr(y)
+    p.T, p.Hq, p.R, p.V, p.Hd = T, Hq, R, w_abs.shape[1], w_o.shape[0]
+    p.y_dtype = _odt(y.dtype)
+    p.num_splits = num_splits
+    p.workspace = _ptr(workspace)
+    p.workspace_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    return p
+
+
+def mla_tail_workspace_bytes(o_lat, w_abs, w_o, num_splits=0):
+    p = MlaTailParams()
+    p.T, p.Hq, p.R = o_lat.shape
+    p.V, p.Hd = w_abs.shape[1], w_o.shape[0]
+    p.y_dtype, p.num_splits = FA_F32, num_splits
+    n = ctypes.c_size_t(0)
+    _check(load().fa_mla_tail_workspace_size(ctypes.byref(p), ctypes.byref(n)))
+    return n.value
+
+
+def mla_tail(o_lat, w_abs, w_o, out=None, out_dtype=torch.float32, num_splits=0, workspace=None, stream=None):
+    """MLA decode tail (fa_mla_tail): y [T, Hd] = o-projection of the
+    per-head out-absorb of o_lat [T, Hq, R].  w_abs [Hq, V, R]; w_o
+    [Hd, Hq*V] (row = output feature).  All bf16, contiguous."""
+    _need_cuda(o_lat, w_abs, w_o, out, workspace)
+    for t in (o_lat, w_abs, w_o):
+        if t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError("o_lat, w_abs and w_o must be contiguous bf16")
+    T = o_lat.shape[0]
+    if out is None:
+        out = torch.empty((T, w_o.shape[0]), device=o_lat.device, dtype=out_dtype)
+    if workspace is None:
+        n = mla_tail_workspace_bytes(o_lat, w_abs, w_o, num_splits)
+        workspace = torch.empty(max(n, 256), device=o_lat.device, dtype=torch.uint8)
+    p = mla_tail_params(o_lat, w_abs, w_o, out, num_splits, workspace)
+    _check(load().fa_mla_tail(ctypes.byref(p), _stream(stream)))
+    return out

@@ -56,6 +56,7 @@ NCU_TRAFFIC = {
     "causal_gqa_b2_hq16_hkv4_s2048_dk192_dv192": 40004096,
     "kv_dequant causal_mha_q8_0kv_b2_h16_s2048_d128": 17835776,
     "paged_prefill_gqa_b16_hq32_hkv8_sq512_d128_bs64": 651085568,
+    "mla_tail_t32_hq128_r512_v128_hidden7168": 257049088,
     "causal_gqa_b1_hq16_hkv4_s4096_dk320_dv256": 77931264,
 }
 
@@ -310,6 +311,31 @@ def paged_prefill_workload(torch, fa, W_, c, l2):
     return launch, n, c.flops(sl0), 1
 
 
+def mla_tail_workload(torch, fa, W_, c, l2):
+    """The MLA decode tail: one fa_mla_tail (out-absorb GEMM, o-projection
+    GEMM, split reduce) per step."""
+    import ctypes
+    o0, wa0, wo0 = W_.mla_tail_inputs(c)
+    foot = c.bytes
+    n = rotation_copies(foot, l2)
+    lib = fa.load()
+    bufs, params = [], []
+    for i in range(n):
+        o, wa, wo = o0.cuda(), wa0.cuda(), wo0.cuda()
+        y = torch.empty(c.T, c.Hd, device="cuda")
+        ws = torch.empty(max(fa.mla_tail_workspace_bytes(o, wa, wo), 256), device="cuda", dtype=torch.uint8)
+        bufs.append((o, wa, wo, y, ws))
+        params.append(fa.mla_tail_params(o, wa, wo, y, 0, ws))
+
+    def launch(i):
+        st = lib.fa_mla_tail(ctypes.byref(params[i]), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+        if st != 0:
+            raise RuntimeError(lib.fa_last_error().decode())
+
+    launch.keep = bufs
+    return launch, n, c.bytes, 3
+
+
 def paged_workload(torch, fa, W_, c, l2):
     q0, kc0, vc0, tb0, sl0 = W_.paged_inputs(c)
     byts = W_.paged_bytes(c, sl0, tb0.shape[1])
@@ -453,7 +479,7 @@ def run_only(args):
     l2 = torch.cuda.get_device_properties(0).L2_cache_size
     table = {c.name: c for c in (W_.TINY_FULL, W_.CAUSAL_MHA, W_.GQA_FULL, W_.MODS_C2, W_.CAUSAL_DK192,
                                  W_.CAUSAL_DK192_DV192, W_.CAUSAL_DK320, W_.PAGED_GQA, W_.LATENT_SPARSE,
-                                 W_.QUANT_C2, W_.PAGED_PREFILL)}
+                                 W_.QUANT_C2, W_.PAGED_PREFILL, W_.MLA_TAIL)}
     table["kv_dequant_" + W_.QUANT_C2.name] = W_.QUANT_C2
     if args.only not in table:
         raise SystemExit("unknown workload %r; one of %s" % (args.only, sorted(table)))
@@ -465,6 +491,9 @@ def run_only(args):
     elif isinstance(c, W_.PrefillCase):
         launch, n, work, kpl = prefill_workload(torch, fa, W_, c, l2)
         unit, amount = "TFLOP/s", c.flops / 1e12
+    elif isinstance(c, W_.MlaTailCase):
+        launch, n, work, kpl = mla_tail_workload(torch, fa, W_, c, l2)
+        unit, amount = "GB/s", work / 1e9
     elif isinstance(c, W_.PagedPrefillCase):
         launch, n, work, kpl = paged_prefill_workload(torch, fa, W_, c, l2)
         unit, amount = "TFLOP/s", work / 1e12
@@ -680,6 +709,20 @@ def main():
             del launch
         except Exception as e:  # report, never hide
             wl[W_.LATENT_SPARSE.name] = {"error": str(e)[:200]}
+        # MLA decode tail (out-absorb + o-projection)
+        mc = W_.MLA_TAIL
+        launch, ncopy, byts, kpl = mla_tail_workload(torch, fa, W_, mc, l2)
+        ms2, st2 = time_graph(torch, launch, ncopy, Ks, Wm, dist)
+        ms2 = max_over_ranks(torch, dist, ms2)
+        per = ms2 / st2
+        ach = byts / (per * 1e-3) / 1e9
+        wl[mc.name] = {"value": round(sum_over_ranks(torch, dist, byts * st2) / (ms2 * 1e-3) / 1e9, 1),
+                       "unit": "GB/s", "tflops": round(mc.flops / (per * 1e-3) / 1e12, 2),
+                       "ms_per_step": round(per, 5), "steps": st2, "l2_copies": ncopy, "bytes_per_step": byts,
+                       "roofline": roofline("hbm", ach, peaks["hbm_gbs"], "GB/s", NCU_TRAFFIC.get(mc.name)),
+                       "kernels": "out-absorb GEMM + o-projection GEMM (split K) + split reduce"}
+        result["gpu_launches"] += st2 * kpl
+        del launch
         result["workloads"] = wl
         assert fa.device_error() == 0, "device error in a secondary workload"
 

@@ -283,6 +283,44 @@ typedef struct {
 } fa_decode_gather_params;
 
 /*
+ * fa_mla_tail -- the projections after the latent decode ("MLA Decode
+ * Attention Kernel API Reference", parameters out_absorb_w and o_proj_w):
+ * the per-head out-absorb, then the o-projection of the concatenated heads,
+ *   u[t][h*V + v] = sum_c w_abs[h][v][c] * o_lat[t][h][c]
+ *   y[t][j]       = sum_k w_o[j][k] * u[t][k]
+ *   o_lat: [T, Hq, R] bf16 contiguous -- the latent attention output
+ *     (fa_decode_gather with o_dtype FA_BF16; R = kv_lora_rank = its dv).
+ *   w_abs: [Hq, V, R] bf16 contiguous (out_absorb_w; V = v_head_dim).
+ *   w_o: [Hd, Hq*V] bf16 contiguous -- the page's o_proj_w [Hq*V, Hd]
+ *     stored transposed (row = output feature, the nn.Linear layout), so
+ *     both contractions run along contiguous memory.
+ *   y: [T, Hd] (y_dtype) contiguous.
+ *   u lives in the workspace as bf16, the operand type of the second
+ *   contraction; both contractions accumulate in fp32.
+ *   num_splits: 0 = automatic, else the number of K splits of the
+ *     o-projection (clamped to [1, min(8, Hq*V / 64)]).  The splits of one
+ *     128-row tile form a thread-block cluster that adds its partial sums in
+ *     split order, so results do not depend on timing.
+ *   workspace: at least fa_mla_tail_workspace_size() bytes (u), 256-byte
+ *     aligned, overwritten on every call.
+ * Supported: V == 128, R a positive multiple of 64, Hd a positive multiple
+ * of 128, Hq * V a multiple of 64, T <= 256.  T == 0 is a no-op.
+ */
+typedef struct {
+    const void *o_lat, *w_abs, *w_o;
+    int T, Hq, R, V, Hd;
+    void *y;
+    int y_dtype; /* fa_dtype */
+    int num_splits;
+    void *workspace;
+    size_t workspace_bytes;
+} fa_mla_tail_params;
+
+/* Workspace bytes for these shapes and num_splits; reads no pointer field. */
+fa_status fa_mla_tail_workspace_size(const fa_mla_tail_params *p, size_t *bytes);
+fa_status fa_mla_tail(const fa_mla_tail_params *p, void *stream);
+
+/*
  * fa_kv_dequant -- quantised K or V rows to bf16: the pre-pass that
  * "ggml-metal: FA tensor path" (ggml_metal_op_flash_attn_ext_use_kv_f16)
  * runs on a quantised KV cache before its 16-bit attention kernels.  Feed

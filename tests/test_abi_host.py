@@ -175,6 +175,33 @@ def test_prefill_paged_null_and_noop():
     assert lib.fa_prefill_paged(ctypes.byref(prefill_paged_params(Sq=0)), None) == fa.FA_OK
 
 
+def tail_params(**kw):
+    p = fa.MlaTailParams()
+    base = dict(o_lat=16, w_abs=32, w_o=48, T=32, Hq=128, R=512, V=128, Hd=7168, y=64, y_dtype=0, num_splits=0,
+                workspace=0, workspace_bytes=0)
+    base.update(kw)
+    for k_, v_ in base.items():
+        setattr(p, k_, v_)
+    return p
+
+
+def test_mla_tail_workspace_size_and_validation():
+    lib = fa.load()
+    n = ctypes.c_size_t(0)
+    # the workspace holds u (32 x 16384 bf16) whatever the split count
+    for ns in (0, 3, 200):
+        assert lib.fa_mla_tail_workspace_size(ctypes.byref(tail_params(num_splits=ns)), ctypes.byref(n)) == fa.FA_OK
+        assert n.value == 32 * 16384 * 2
+    assert lib.fa_mla_tail(ctypes.byref(tail_params()), None) == fa.FA_ERR_WORKSPACE
+    for kw in (dict(V=64), dict(R=500), dict(Hd=7000), dict(T=257)):
+        assert lib.fa_mla_tail(ctypes.byref(tail_params(**kw)), None) == fa.FA_ERR_UNSUPPORTED, kw
+    for kw in (dict(T=-1), dict(Hq=0), dict(y_dtype=5), dict(num_splits=-2), dict(w_o=40)):
+        st = lib.fa_mla_tail(ctypes.byref(tail_params(workspace=256, workspace_bytes=1 << 30, **kw)), None)
+        assert st == fa.FA_ERR_INVALID_ARG, kw
+    assert lib.fa_mla_tail(ctypes.byref(tail_params(T=0)), None) == fa.FA_OK
+    assert lib.fa_mla_tail(None, None) == fa.FA_ERR_INVALID_ARG
+
+
 def dequant_params(**kw):
     p = fa.KvDequantParams()
     base = dict(src=2, type=fa.FA_KV_Q8_0, n_rows=1024, row_elems=128, src_row_bytes=136, dst=16, dst_row_stride=128)

@@ -1,0 +1,63 @@
+"""MLA decode tail on the GPU (fa_mla_tail: out-absorb then o-projection)
+against the oracle's mla_tail on the same seeded inputs.
+
+Tolerance: u is held in bf16 between the two contractions (the operand type
+of the second), which the fp64 oracle does not do.  With the workload's
+scaling (u, y ~ N(0, 1), weights ~ N(0, 1/fan_in)) that rounding moves y by
+about 2^-9 / sqrt(3) ~ 1.1e-3 rms, so max |dy| stays well inside 1e-2 and the
+cosine above 0.99999; bf16 output adds up to half an ulp of y (2e-2)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from attention_attn_fwd_11_b200 import fa
+from attention_attn_fwd_11_b200 import workloads as W
+from parity import check
+
+pytestmark = pytest.mark.gpu
+
+
+def run(c, num_splits=0, out_dtype=torch.float32, rows=None):
+    o_lat, w_abs, w_o = W.mla_tail_inputs(c)
+    y = fa.mla_tail(o_lat.cuda(), w_abs.cuda(), w_o.cuda(), out_dtype=out_dtype, num_splits=num_splits)
+    torch.cuda.synchronize()
+    assert fa.device_error() == 0
+    w_ref = w_o if rows is None else w_o[rows]
+    _, y_ref = oracle.mla_tail(W.bits(o_lat), W.bits(w_abs), W.bits(w_ref))
+    got = y if rows is None else y[:, rows]
+    bf = out_dtype == torch.bfloat16
+    check(got, y_ref, max_abs=2e-2 if bf else 1e-2, min_cos=0.9999 if bf else 0.99999,
+          what="%s splits %d" % (c.name, num_splits))
+    return y
+
+
+@pytest.mark.parametrize("T", [1, 5, 16, 32, 40, 129])
+def test_token_counts(T):
+    # T spans N = 16 .. 144 (padded to 16) and one or several 32-column reads.
+    run(W.MlaTailCase("t", T, 4, R=128, V=128, Hd=256, seed=T))
+
+
+@pytest.mark.parametrize("splits", [1, 3, 7, 8, 64])
+def test_split_counts(splits):
+    # 8 heads x 128 = 1024 = 16 stages of K: 3 and 7 give uneven splits (7
+    # becomes 6 splits of 3 stages); 64 is clamped to one cluster of 8.
+    run(W.MlaTailCase("t", 24, 8, R=192, V=128, Hd=384, seed=40 + splits), num_splits=splits)
+
+
+def test_bf16_output_and_determinism():
+    c = W.MlaTailCase("t", 32, 16, R=256, V=128, Hd=512, seed=50)
+    y1 = run(c, out_dtype=torch.bfloat16)
+    o_lat, w_abs, w_o = W.mla_tail_inputs(c)
+    y2 = fa.mla_tail(o_lat.cuda(), w_abs.cuda(), w_o.cuda(), out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
+
+
+def test_workload_sampled_features():
+    # The benchmark's shape (T 32, Hq 128, R 512, V 128, hidden 7168): the
+    # o-projection is separable by output feature, so 384 sampled rows of
+    # w_o give those columns of y exactly.
+    c = W.MLA_TAIL
+    rows = np.sort(np.random.default_rng(0).choice(c.Hd, 384, replace=False))
+    run(c, rows=torch.from_numpy(rows))
