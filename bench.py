@@ -720,7 +720,7 @@ def main():
                        "unit": "GB/s", "tflops": round(mc.flops / (per * 1e-3) / 1e12, 2),
                        "ms_per_step": round(per, 5), "steps": st2, "l2_copies": ncopy, "bytes_per_step": byts,
                        "roofline": roofline("hbm", ach, peaks["hbm_gbs"], "GB/s", NCU_TRAFFIC.get(mc.name)),
-                       "kernels": "out-absorb GEMM + o-projection GEMM (split K) + split reduce"}
+                       "kernels": "out-absorb GEMM + o-projection GEMM (split K, cluster reduce)"}
         result["gpu_launches"] += st2 * kpl
         del launch
         result["workloads"] = wl
