@@ -49,11 +49,19 @@ FA_DEV const __half *mask_row(const ScoreMods &m, int b, int h, int i, int Sq) {
     return m.mask + (int64_t)b * m.m_sb + (int64_t)h * m.m_sh + (int64_t)i * m.m_ss;
 }
 
+// 1/x from the approximate reciprocal instruction (one MUFU operation,
+// within about an ulp; 1/inf = 0).
+FA_DEV float rcp_approx(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // tanh(s) = 1 - 2 / (e^(2s) + 1), with e^(2s) from ex2: exact limits +-1 for
-// |s| large, absolute error of order 1e-7 elsewhere.
+// |s| large, absolute error of order 1e-7 elsewhere.  Two MUFU operations.
 FA_DEV float tanh_via_exp(float s) {
     const float e = ex2(2.f * kLog2e * s);
-    return 1.f - 2.f * __frcp_rn(e + 1.f);
+    return 1.f - 2.f * rcp_approx(e + 1.f);
 }
 
 // Raw scores x[k] (unscaled q.k of keys key0 + k) -> base-2 scores
