@@ -338,6 +338,13 @@ fa_status fa_fwd(const fa_fwd_params *p, void *stream) {
         L.mods.log2_m1 = -p->max_bias / 2.f / (float)n2;
     }
     L.has_mods = p->mask || p->softcap > 0.f || p->sinks;
+    if (two_tile && p->mask && p->Sk > 0) {
+        // Head and batch dimensions of stride 0 are broadcast: size 1, coordinate 0.
+        st = encode_4d(&L.tmM, p->mask, p->Sk, p->Sq, p->m_sh ? p->Hq : 1, p->m_sb ? p->B : 1, p->m_ss,
+                       p->m_sh ? p->m_sh : p->m_ss * p->Sq, p->m_sb ? p->m_sb : p->m_ss * p->Sq, 128, "fa_fwd mask");
+        if (st != FA_OK) return st;
+        L.mask_staged = true;
+    }
     cudaError_t e;
     if (two_tile) {
         int sms = 0;

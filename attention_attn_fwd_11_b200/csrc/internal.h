@@ -23,6 +23,10 @@ struct PrefillLaunch {
     float *lse;
     ScoreMods mods;  // all-zero: no modifiers
     bool has_mods;   // a mask, a softcap or sinks is given
+    // Two-tile kernel with a mask: the mask as (Sk, Sq, Hm, Bm) f16 with
+    // 64 x 128 boxes (128-byte swizzle), staged by TMA.
+    CUtensorMap tmM;
+    bool mask_staged;
     // Paged K/V (two-tile kernel only; block_table == NULL: dense K/V).
     // tmK / tmV then view the caches [num_blocks, Hkv, 64, d] as
     // (d, 64, Hkv, num_blocks) with 64-row boxes, and the keys of sequence b

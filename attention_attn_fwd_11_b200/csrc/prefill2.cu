@@ -74,6 +74,9 @@ struct Prefill2Args {
     int64_t o_sb, o_sh, o_ss;
     int o_bf16;
     float *lse;
+    // The mask arrives through TMA into each softmax group's staging tile,
+    // 64 keys at a time (MODS with a mask, two-tile kernel).
+    int mask_staged;
     // Paged K/V: block_table [B, max_blocks] and seq_lens [B] (NULL: dense).
     const int32_t *block_table;
     const int32_t *seq_lens;
@@ -116,7 +119,10 @@ struct P2Cfg {
 
 enum {
     P2_QFULL = 0, P2_QEMPTY = 1, P2_SFULL = 2, P2_PREADY = 4, P2_ODONE = 6, P2_OFREE = 8, P2_USTART = 10,
-    P2_DRAIN = 12, P2_PLO = 13, P2_RING = 15
+    P2_DRAIN = 12, P2_PLO = 13, P2_RING = 15,
+    // staged mask (per query tile): chunk landed, chunk read, staging tile
+    // free after the unit's epilogue
+    P2_MFULL = 32, P2_MEMPTY = 34, P2_SFREE = 36
 };
 
 // FA_P2_SPLITP: the softmax signals when P of keys 0..63 is in TMEM, and the
@@ -207,6 +213,7 @@ template <int D, bool MODS>
 __global__ void __launch_bounds__(P2_THREADS, 1)
 prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                const __grid_constant__ CUtensorMap tmM,
                 const Prefill2Args a) {
     using C = P2Cfg<D>;
     constexpr int BN = C::BN, NSTK = C::NSTK, NSTV = C::NSTV;
@@ -238,6 +245,9 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             mbar_init(bar(P2_OFREE + i), 128);
             mbar_init(bar(P2_USTART + i), 1);
             mbar_init(bar(P2_PLO + i), 128);
+            mbar_init(bar(P2_MFULL + i), 1);
+            mbar_init(bar(P2_MEMPTY + i), 128);
+            mbar_init(bar(P2_SFREE + i), 1);
         }
         for (int s = 0; s < NSTK; ++s) {
             mbar_init(k_full(s), 1);
@@ -359,6 +369,37 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 for (int k = max(0, issued_v - NSTV); k < issued_v; ++k)
                     mbar_wait_drain(v_full(k % NSTV), (uint32_t)(k / NSTV) & 1u);
             }
+        }
+    } else if (MODS && warp >= 2 && a.mask_staged) {
+        // ----------------------------------------------- mask loaders --
+        // Warp 2 + i fills query tile i's staging tile with 64-key chunks of
+        // the mask (128 rows x 128 bytes, 128-byte swizzle; rows past Sq and
+        // keys past Sk read as zero), in the order its softmax group uses
+        // them.  Before a unit's first chunk it waits until the group's
+        // previous epilogue has finished with the tile.
+        if (lane == 0) {
+            const int ti = warp - 2;
+            const uint32_t stg = sbase + C::OFF_STG + ti * C::STG_BYTES;
+            prefetch_tmap(&tmM);
+            int f = 0, uc = 0;
+            bool mok = true;
+            UnitInfo u;
+            for (int r = 0; mok && p2_unit(a, r, u); ++r, ++uc) {
+                if (uc > 0 && !mbar_wait(bar(P2_SFREE + ti), (uint32_t)(uc - 1) & 1u, abort_flag, &g_prefill2_err))
+                    break;
+                const int n = u.nt(ti);
+                const int hm = a.mods.m_sh ? u.hq : 0, bm = a.mods.m_sb ? u.b : 0;
+                for (int t = 0; mok && t < n; ++t)
+                    for (int h = 0; h < BN / 64; ++h, ++f) {
+                        if (!mbar_wait(bar(P2_MEMPTY + ti), ((uint32_t)f & 1u) ^ 1u, abort_flag, &g_prefill2_err)) {
+                            mok = false;
+                            break;
+                        }
+                        mbar_arrive_expect_tx(bar(P2_MFULL + ti), C::STG_BYTES);
+                        tma_load_4d(stg, &tmM, bar(P2_MFULL + ti), t * BN + 64 * h, u.q0 + 128 * ti, hm, bm);
+                    }
+            }
+            if (*abort_flag && f > 0) mbar_wait_drain(bar(P2_MFULL + ti), (uint32_t)(f - 1) & 1u);
         }
 #if defined(FA_P2_TRACE) && ((FA_P2_TRACE_MASK >> 29) & 1u)
     } else if (warp == 2) {
@@ -538,9 +579,10 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         // the epilogue alone.
         const bool transform = MODS && (a.mods.mask != nullptr || a.mods.softcap != 0.f);
         const float c = transform ? 1.f : a.scale_log2;
-        int scnt = 0, pv_base = 0, uc = 0;
+        int scnt = 0, pv_base = 0, uc = 0, mcnt = 0;
         bool ok = true;
         UnitInfo u;
+        const uint8_t *mstg = smem + C::OFF_STG + ti * C::STG_BYTES + row * 128;  // this row of the staging tile
         for (int r = 0; ok && p2_unit(a, r, u); ++r, ++uc) {
             if (!mbar_wait(bar(P2_USTART + ti), (uint32_t)uc & 1u, abort_flag, &g_prefill2_err)) break;
             const int n = u.nt(ti);
@@ -576,7 +618,21 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 }
                 if (lane == 0) TRACE(11 + ti, t, qd);
                 const int lim = lim_all - t * BN;
-                if (transform) {
+                if (MODS && a.mask_staged) {
+                    // this row's 64 mask values of each chunk from the staging tile
+#pragma unroll
+                    for (int h = 0; h < BN / 64; ++h) {
+                        if (!mbar_wait(bar(P2_MFULL + ti), (uint32_t)mcnt & 1u, abort_flag, &g_prefill2_err)) ok = false;
+                        uint4 w[8];
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) w[j] = *reinterpret_cast<const uint4 *>(mstg + ((j ^ (row & 7)) << 4));
+                        mbar_arrive(bar(P2_MEMPTY + ti));
+                        ++mcnt;
+                        modify_chunk(&x[64 * h], w, a.mods, a.scale, slope);
+                    }
+                    if (!ok) break;
+                    hide_keys<BN>(x, lim);
+                } else if (transform) {
                     modify_scores<BN>(x, a.mods, a.scale, slope, mrow, t * BN, u.Sk, lim);
                 } else if (lim < BN) {
 #pragma unroll
@@ -817,6 +873,10 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                     store_slice(ch, ch * 32, w);
                 }
             }
+            if (MODS && a.mask_staged && row == 0) {
+                bulk_wait_read0();  // the last O store has read the staging tile
+                mbar_arrive(bar(P2_SFREE + ti));
+            }
         }
     }
 
@@ -854,6 +914,7 @@ static cudaError_t launch_p2(const PrefillLaunch &L, int num_sms, cudaStream_t s
     a.o_ss = L.o_ss;
     a.o_bf16 = L.o_bf16;
     a.lse = L.lse;
+    a.mask_staged = MODS && L.mask_staged ? 1 : 0;
     a.block_table = L.block_table;
     a.seq_lens = L.seq_lens;
     a.max_blocks = L.max_blocks;
@@ -868,7 +929,7 @@ static cudaError_t launch_p2(const PrefillLaunch &L, int num_sms, cudaStream_t s
     }
 #endif
     const int grid = a.n_units < num_sms ? a.n_units : num_sms;
-    kern<<<grid, P2_THREADS, C::SMEM_BYTES, stream>>>(L.tmQ, L.tmK, L.tmV, L.tmO, a);
+    kern<<<grid, P2_THREADS, C::SMEM_BYTES, stream>>>(L.tmQ, L.tmK, L.tmV, L.tmO, L.tmM, a);
     return cudaGetLastError();
 }
 

@@ -64,65 +64,75 @@ FA_DEV float tanh_via_exp(float s) {
     return 1.f - 2.f * rcp_approx(e + 1.f);
 }
 
-// Raw scores x[k] (unscaled q.k of keys key0 + k) -> base-2 scores
-// (modified score) * log2(e); keys k >= lim are hidden (-inf).  mrow: this
-// row's mask or NULL; keys at or past Sk are never read from it.
-// Raw scores x[k] (unscaled q.k of keys key0 + k) -> base-2 scores
-// (modified score) * log2(e); keys k >= lim are hidden (-inf).  mrow: this
-// row's mask or NULL; keys at or past Sk are never read from it.  The mask
-// is read 64 keys at a time: a chunk wholly inside the row issues its eight
-// 16-byte loads before the first is used.
-template <int BN>
-FA_DEV void modify_scores(float (&x)[BN], const ScoreMods &m, float scale, float slope, const __half *mrow,
-                          int key0, int Sk, int lim) {
-    static_assert(BN % 64 == 0, "tile width");
+// One 64-key chunk: raw scores x[0..64) (unscaled q.k) and the chunk's mask
+// values w (64 f16 in key order; all zero without a mask) -> base-2 scores
+// (modified score) * log2(e).
+FA_DEV void modify_chunk(float *x, const uint4 (&w)[8], const ScoreMods &m, float scale, float slope) {
     const float cs = scale * kLog2e;   // raw score -> base-2 units, without softcap
     const float cm = slope * kLog2e;   // mask value -> base-2 units
     const uint64_t cs2 = f2_pack(cs, cs), cm2 = f2_pack(cm, cm);
 #pragma unroll
-    for (int h = 0; h < BN / 64; ++h) {
-        const int kc = key0 + 64 * h;
-        const bool whole = mrow && kc + 64 <= Sk;
-        uint4 w[8];
-        if (whole) {
+    for (int g = 0; g < 8; ++g) {
+        const uint32_t mw[4] = {w[g].x, w[g].y, w[g].z, w[g].w};  // four f16 pairs
 #pragma unroll
-            for (int g = 0; g < 8; ++g) w[g] = __ldg(reinterpret_cast<const uint4 *>(mrow + kc + 8 * g));
-        }
-#pragma unroll
-        for (int g = 0; g < 8; ++g) {
-            uint32_t mw[4] = {0u, 0u, 0u, 0u};  // four f16 pairs (zero: no mask value)
-            if (whole) {
-                mw[0] = w[g].x;
-                mw[1] = w[g].y;
-                mw[2] = w[g].z;
-                mw[3] = w[g].w;
-            } else if (mrow) {  // the row's last, partial chunk: element loads up to Sk
-                const uint16_t *mr = reinterpret_cast<const uint16_t *>(mrow);
-#pragma unroll
-                for (int j = 0; j < 8; ++j)
-                    if (kc + 8 * g + j < Sk) mw[j >> 1] |= (uint32_t)mr[kc + 8 * g + j] << (16 * (j & 1));
+        for (int j = 0; j < 4; ++j) {
+            const int k = 8 * g + 2 * j;
+            const float2 mf = __half22float2(*reinterpret_cast<const __half2 *>(&mw[j]));
+            uint64_t y;
+            if (m.softcap != 0.f) {
+                const float s0 = m.softcap * tanh_via_exp(x[k] * scale);
+                const float s1 = m.softcap * tanh_via_exp(x[k + 1] * scale);
+                y = f2_fma(f2_pack(mf.x, mf.y), cm2, f2_mul(f2_pack(s0, s1), f2_pack(kLog2e, kLog2e)));
+            } else {
+                y = f2_fma(f2_pack(x[k], x[k + 1]), cs2, f2_mul(f2_pack(mf.x, mf.y), cm2));
             }
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int k = 64 * h + 8 * g + 2 * j;
-                const float2 mf = __half22float2(*reinterpret_cast<const __half2 *>(&mw[j]));
-                uint64_t y;
-                if (m.softcap != 0.f) {
-                    const float s0 = m.softcap * tanh_via_exp(x[k] * scale);
-                    const float s1 = m.softcap * tanh_via_exp(x[k + 1] * scale);
-                    y = f2_fma(f2_pack(mf.x, mf.y), cm2, f2_mul(f2_pack(s0, s1), f2_pack(kLog2e, kLog2e)));
-                } else {
-                    y = f2_fma(f2_pack(x[k], x[k + 1]), cs2, f2_mul(f2_pack(mf.x, mf.y), cm2));
-                }
-                f2_unpack(y, x[k], x[k + 1]);
-            }
+            f2_unpack(y, x[k], x[k + 1]);
         }
     }
+}
+
+// Keys k >= lim of the tile are hidden (-inf).
+template <int BN>
+FA_DEV void hide_keys(float (&x)[BN], int lim) {
     if (lim < BN) {
 #pragma unroll
         for (int k = 0; k < BN; ++k)
             if (k >= lim) x[k] = -INFINITY;
     }
+}
+
+// Raw scores x[k] (unscaled q.k of keys key0 + k) -> base-2 scores
+// (modified score) * log2(e); keys k >= lim are hidden (-inf).  mrow: this
+// row's mask in global memory or NULL; keys at or past Sk are never read
+// from it.  The mask is read 64 keys at a time: a chunk wholly inside the row
+// issues its eight 16-byte loads before the first is used.
+template <int BN>
+FA_DEV void modify_scores(float (&x)[BN], const ScoreMods &m, float scale, float slope, const __half *mrow,
+                          int key0, int Sk, int lim) {
+    static_assert(BN % 64 == 0, "tile width");
+#pragma unroll
+    for (int h = 0; h < BN / 64; ++h) {
+        const int kc = key0 + 64 * h;
+        uint4 w[8];
+        if (mrow && kc + 64 <= Sk) {
+#pragma unroll
+            for (int g = 0; g < 8; ++g) w[g] = __ldg(reinterpret_cast<const uint4 *>(mrow + kc + 8 * g));
+        } else {
+            uint32_t mw[32];  // f16 pairs; zero: no mask value
+#pragma unroll
+            for (int j = 0; j < 32; ++j) mw[j] = 0u;
+            if (mrow) {  // the row's last, partial chunk: element loads up to Sk
+                const uint16_t *mr = reinterpret_cast<const uint16_t *>(mrow);
+#pragma unroll
+                for (int e = 0; e < 64; ++e)
+                    if (kc + e < Sk) mw[e >> 1] |= (uint32_t)mr[kc + e] << (16 * (e & 1));
+            }
+#pragma unroll
+            for (int g = 0; g < 8; ++g) w[g] = make_uint4(mw[4 * g], mw[4 * g + 1], mw[4 * g + 2], mw[4 * g + 3]);
+        }
+        modify_chunk(&x[64 * h], w, m, scale, slope);
+    }
+    hide_keys<BN>(x, lim);
 }
 
 // Epilogue with a sink: O was accumulated relative to m_run (base 2);
