@@ -175,12 +175,13 @@ def fwd_params(q, k, v, o, lse, scale, causal, mask=None, max_bias=0.0, softcap=
 
 
 def fwd(q, k, v, scale=None, causal=False, out=None, return_lse=True, out_dtype=torch.float32, stream=None,
-        mask=None, max_bias=0.0, softcap=0.0, sinks=None):
+        mask=None, max_bias=0.0, softcap=0.0, sinks=None, lse=None):
     """O = softmax(scale * Q K^T + mask) V.  q [B,Hq,Sq,dk], k [B,Hkv,Sk,dk],
     v [B,Hkv,Sk,dv] bf16 CUDA tensors (any strides, head dim contiguous).
     Score modifiers (see fa_fwd in include/fa.h): mask [1|B, 1|Hq, Sq, Sk]
     float16 CUDA tensor with a contiguous last dim, max_bias (ALiBi slopes
-    applied to the mask), softcap, sinks [Hq] float32 CUDA tensor.
+    applied to the mask), softcap, sinks [Hq] float32 CUDA tensor.  out and
+    lse may be given preallocated (lse: contiguous float32 [B,Hq,Sq]).
     Returns (O [B,Hq,Sq,dv], LSE [B,Hq,Sq] fp32 or None)."""
     _need_cuda(q, k, v)
     if mask is not None:
@@ -200,7 +201,11 @@ def fwd(q, k, v, scale=None, causal=False, out=None, return_lse=True, out_dtype=
         scale = 1.0 / math.sqrt(dk)
     if out is None:
         out = torch.empty((B, Hq, Sq, dv), device=q.device, dtype=out_dtype)
-    lse = torch.empty((B, Hq, Sq), device=q.device, dtype=torch.float32) if return_lse else None
+    if lse is not None:
+        if lse.dtype != torch.float32 or tuple(lse.shape) != (B, Hq, Sq) or not lse.is_contiguous() or not lse.is_cuda:
+            raise ValueError("lse must be a contiguous float32 CUDA tensor [B, Hq, Sq]")
+    elif return_lse:
+        lse = torch.empty((B, Hq, Sq), device=q.device, dtype=torch.float32)
     params = fwd_params(q, k, v, out, lse, scale, causal, mask, max_bias, softcap, sinks)
     _check(load().fa_fwd(ctypes.byref(params), _stream(stream)))
     return out, lse
