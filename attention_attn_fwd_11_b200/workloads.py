@@ -128,11 +128,16 @@ def random_sinks(Hq: int, seed: int):
 # decoded values have roughly unit spread like the bf16 inputs.  Seed
 # 7000 + c.
 
-QUANT_BLOCK_BYTES = {"q8_0": 34, "q4_0": 18}
+QUANT_BLOCK_BYTES = {"q8_0": 34, "q4_0": 18, "fp8_e4m3": 32}  # bytes per 32 values
+
+# FP8 E4M3 rows hold N(0, 16^2) draws cast to float8_e4m3fn by torch, read
+# back with the per-tensor scale FP8_SCALE = 1/16 (values of unit spread).
+FP8_SCALE = 1.0 / 16.0
 
 
 def random_quant_rows(shape, row_elems: int, qtype: str, seed: int):
-    """uint8 tensor [*shape, row_elems / 32 * block bytes] of ggml blocks."""
+    """uint8 tensor [*shape, row_elems / 32 * block bytes]: ggml blocks, or
+    FP8 E4M3 bytes."""
     g = torch.Generator().manual_seed(7000 + seed)
     nb = row_elems // 32
     n = int(np.prod(shape)) * nb
@@ -140,6 +145,9 @@ def random_quant_rows(shape, row_elems: int, qtype: str, seed: int):
         d = torch.empty(n).uniform_(0.02, 0.03, generator=g).to(torch.float16)
         q = (torch.randn(n, 32, generator=g) * 40).round().clamp(-127, 127).to(torch.int8)
         body = q.view(torch.uint8)
+    elif qtype == "fp8_e4m3":
+        x = torch.randn(int(np.prod(shape)), row_elems, generator=g) / FP8_SCALE
+        return x.to(torch.float8_e4m3fn).view(torch.uint8).reshape(*shape, row_elems).contiguous()
     elif qtype == "q4_0":
         d = torch.empty(n).uniform_(0.3, 0.5, generator=g).to(torch.float16)
         nib = (torch.randn(n, 32, generator=g) * 2.5 + 8).round().clamp(0, 15).to(torch.uint8)

@@ -65,6 +65,10 @@ def _load():
         lib.oracle_round_bf16.restype = ctypes.c_uint16
         lib.oracle_dequant_rows.argtypes = [P, i32, i64, i32, i64, P]
         lib.oracle_dequant_rows.restype = i32
+        lib.oracle_dequant_rows_scaled.argtypes = [P, i32, i64, i32, i64, f64, P]
+        lib.oracle_dequant_rows_scaled.restype = i32
+        lib.oracle_e4m3_to_double.argtypes = [ctypes.c_uint8]
+        lib.oracle_e4m3_to_double.restype = f64
         _lib = lib
     return _lib
 
@@ -264,7 +268,7 @@ def lse_combine(o_parts, lse_parts):
     return o, lse
 
 
-QUANT_TYPES = {"q8_0": (8, 34), "q4_0": (4, 18)}  # oracle type code, bytes per 32-value block
+QUANT_TYPES = {"q8_0": (8, 34), "q4_0": (4, 18), "fp8_e4m3": (2, 32)}  # type code, bytes per 32 values
 
 
 def round_bf16(x) -> int:
@@ -272,16 +276,23 @@ def round_bf16(x) -> int:
     return int(_load().oracle_round_bf16(float(x)))
 
 
-def dequant_rows(src, qtype, row_elems):
+def e4m3_value(b) -> float:
+    """The value of one FP8 E4M3 byte."""
+    return float(_load().oracle_e4m3_to_double(int(b)))
+
+
+def dequant_rows(src, qtype, row_elems, scale=1.0):
     """Quantised rows -> bf16 bit patterns.  src: uint8 [..., row_bytes]
-    (each row holds row_elems / 32 ggml blocks of type ``qtype``, 'q8_0' or
-    'q4_0', then any padding); returns uint16 [..., row_elems]."""
+    (each row holds row_elems values of type ``qtype`` -- 'q8_0' or 'q4_0'
+    ggml blocks, or 'fp8_e4m3' bytes times ``scale`` -- then any padding);
+    returns uint16 [..., row_elems]."""
     code, bb = QUANT_TYPES[qtype]
     src = np.ascontiguousarray(src, dtype=np.uint8)
     lead = src.shape[:-1]
     n_rows = int(np.prod(lead)) if lead else 1
     out = np.empty(lead + (row_elems,), np.uint16)
-    rc = _load().oracle_dequant_rows(_ptr(src), code, n_rows, row_elems, src.shape[-1], _ptr(out))
+    rc = _load().oracle_dequant_rows_scaled(_ptr(src), code, n_rows, row_elems, src.shape[-1], float(scale),
+                                            _ptr(out))
     if rc:
         raise ValueError("oracle_dequant_rows: bad arguments")
     return out

@@ -538,10 +538,49 @@ static uint16_t double_to_bf16_rne(double x)
 uint16_t oracle_round_bf16(double x) { return double_to_bf16_rne(x); }
 
 /*
+ * OCP FP8 E4M3 ("e4m3fn") byte -> double, exactly: sign, 4-bit exponent with
+ * bias 7, 3-bit mantissa; exponent 0 is subnormal (m * 2^-9); S.1111.111 is
+ * NaN and there are no infinities (largest finite 448).
+ */
+static double e4m3_to_double(uint8_t b)
+{
+    const int sign = b >> 7, e = (b >> 3) & 15, m = b & 7;
+    double v;
+    if (e == 15 && m == 7)
+        v = NAN;
+    else if (e == 0)
+        v = ldexp((double)m, -9);
+    else
+        v = ldexp((double)(8 + m), e - 10);  /* (1 + m/8) * 2^(e-7) */
+    return sign ? -v : v;
+}
+
+double oracle_e4m3_to_double(uint8_t b) { return e4m3_to_double(b); }
+
+int oracle_dequant_rows(const uint8_t *src, int type, int64_t n_rows, int row_elems,
+                        int64_t src_row_bytes, uint16_t *dst);
+
+/*
  * n_rows rows of row_elems values each (row_elems a multiple of 32); row r
  * starts at src + r * src_row_bytes.  dst: [n_rows][row_elems] bf16 bits.
+ * type 8 (q8_0) and 4 (q4_0): ggml blocks as above.  type 2 (fp8 e4m3): one
+ * byte per value, value = e4m3 * scale (one scale for the whole tensor, as
+ * FP8 KV caches keep it), the exact product rounded once to bf16.
  * Returns 0, or -1 on bad arguments.
  */
+int oracle_dequant_rows_scaled(const uint8_t *src, int type, int64_t n_rows, int row_elems,
+                               int64_t src_row_bytes, double scale, uint16_t *dst)
+{
+    if (type == 2) {
+        if (row_elems <= 0 || row_elems % 32 || n_rows < 0 || src_row_bytes < row_elems) return -1;
+        for (int64_t r = 0; r < n_rows; ++r)
+            for (int j = 0; j < row_elems; ++j)
+                dst[r * row_elems + j] = double_to_bf16_rne(e4m3_to_double(src[r * src_row_bytes + j]) * scale);
+        return 0;
+    }
+    return oracle_dequant_rows(src, type, n_rows, row_elems, src_row_bytes, dst);
+}
+
 int oracle_dequant_rows(const uint8_t *src, int type, int64_t n_rows, int row_elems,
                         int64_t src_row_bytes, uint16_t *dst)
 {

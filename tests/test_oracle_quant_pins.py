@@ -111,3 +111,46 @@ def test_bad_arguments():
         oracle.dequant_rows(np.zeros((1, 34), np.uint8), "q8_0", 48)   # not a multiple of 32
     with pytest.raises(ValueError):
         oracle.dequant_rows(np.zeros((1, 30), np.uint8), "q8_0", 32)   # row too short
+
+
+# ------------------------------------------------------------ FP8 E4M3 --
+
+@pytest.mark.parametrize("b,v", [
+    (0x00, 0.0), (0x80, -0.0), (0x38, 1.0), (0xB8, -1.0), (0x40, 2.0), (0x30, 0.5),
+    (0x01, 2.0 ** -9),        # smallest subnormal
+    (0x07, 7 * 2.0 ** -9),    # largest subnormal
+    (0x08, 2.0 ** -6),        # smallest normal
+    (0x7E, 448.0),            # largest finite
+    (0x3C, 1.5),
+])
+def test_e4m3_worked_values(b, v):
+    got = oracle.e4m3_value(b)
+    assert got == v and np.signbit(got) == np.signbit(v)
+
+
+def test_e4m3_nan_and_all_bytes_match_torch():
+    import math
+    assert math.isnan(oracle.e4m3_value(0x7F)) and math.isnan(oracle.e4m3_value(0xFF))
+    allb = np.arange(256, dtype=np.uint8)
+    want = torch.from_numpy(allb).view(torch.float8_e4m3fn).double().numpy()
+    got = np.array([oracle.e4m3_value(b) for b in allb])
+    assert np.array_equal(np.isnan(got), np.isnan(want))
+    ok = ~np.isnan(want)
+    assert np.array_equal(got[ok], want[ok])
+
+
+def test_fp8_rows_scaled_round_once():
+    # value = e4m3 * scale, rounded once to bf16: compare with the exact
+    # product (float64) rounded by torch's float32 -> bf16 conversion, which is
+    # a single rounding whenever the product is exact in float32.
+    rng = np.random.default_rng(3)
+    src = rng.integers(0, 256, (9, 64 + 8), dtype=np.uint8)
+    src[src == 0x7F] = 0x7E
+    src[src == 0xFF] = 0xFE
+    scale = 0.75  # 3 * 2^-2: e4m3 (4 significant bits) * scale stays exact in float32
+    got = oracle.dequant_rows(src, "fp8_e4m3", 64, scale=scale)
+    exact = torch.from_numpy(src[:, :64].copy()).view(torch.float8_e4m3fn).double().numpy() * scale
+    assert np.array_equal(got, bf16_bits_torch(exact))
+    # a scale whose product needs rounding: 1 + 2^-8 rounds to 1 (ties to even)
+    one = np.full((1, 32), 0x38, np.uint8)
+    assert np.all(oracle.dequant_rows(one, "fp8_e4m3", 32, scale=1.0 + 2.0 ** -8) == 0x3F80)
