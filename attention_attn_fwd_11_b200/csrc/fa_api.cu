@@ -622,28 +622,33 @@ fa_status fa_kv_dequant_n(const fa_kv_dequant_params *p, int n, void *stream) {
     bool any = false;
     for (int i = 0; i < n; ++i) {
         const fa_kv_dequant_params *q = p + i;
-        if (q->type != FA_KV_Q8_0 && q->type != FA_KV_Q4_0)
-            return fail(FA_ERR_UNSUPPORTED, "fa_kv_dequant: type %d (supported: FA_KV_Q8_0, FA_KV_Q4_0)", q->type);
+        if (q->type != FA_KV_Q8_0 && q->type != FA_KV_Q4_0 && q->type != FA_KV_FP8_E4M3)
+            return fail(FA_ERR_UNSUPPORTED, "fa_kv_dequant: type %d (supported: FA_KV_Q8_0, FA_KV_Q4_0, FA_KV_FP8_E4M3)",
+                        q->type);
+        if (q->type == FA_KV_FP8_E4M3 && !isfinite(q->scale))
+            return fail(FA_ERR_INVALID_ARG, "fa_kv_dequant: the fp8 scale must be finite");
         if (q->type != p->type) return fail(FA_ERR_INVALID_ARG, "fa_kv_dequant_n: every entry must have one type");
         if (q->n_rows < 0 || q->row_elems <= 0 || q->row_elems % 32 != 0)
             return fail(FA_ERR_INVALID_ARG, "fa_kv_dequant: need n_rows >= 0 and row_elems a positive multiple of 32");
-        const int64_t block_bytes = q->type == FA_KV_Q8_0 ? 34 : 18;
-        if (q->src_row_bytes < q->row_elems / 32 * block_bytes || q->src_row_bytes % 2 != 0)
-            return fail(FA_ERR_INVALID_ARG, "fa_kv_dequant: src_row_bytes must be even and >= %lld",
-                        (long long)(q->row_elems / 32 * block_bytes));
+        const int64_t block_bytes = q->type == FA_KV_Q8_0 ? 34 : (q->type == FA_KV_Q4_0 ? 18 : 32);
+        const int64_t src_align = q->type == FA_KV_FP8_E4M3 ? 8 : 2;
+        if (q->src_row_bytes < q->row_elems / 32 * block_bytes || q->src_row_bytes % src_align != 0)
+            return fail(FA_ERR_INVALID_ARG, "fa_kv_dequant: src_row_bytes must be a multiple of %lld and >= %lld",
+                        (long long)src_align, (long long)(q->row_elems / 32 * block_bytes));
         if (q->dst_row_stride < q->row_elems || q->dst_row_stride % 8 != 0)
             return fail(FA_ERR_INVALID_ARG, "fa_kv_dequant: dst_row_stride must be a multiple of 8 and >= row_elems");
         if (q->n_rows > 0) {
             if (!q->src || !q->dst) return fail(FA_ERR_INVALID_ARG, "fa_kv_dequant: NULL pointer");
-            if (reinterpret_cast<uintptr_t>(q->src) % 2 != 0 || reinterpret_cast<uintptr_t>(q->dst) % 16 != 0)
-                return fail(FA_ERR_INVALID_ARG, "fa_kv_dequant: src must be 2-byte and dst 16-byte aligned");
+            if (reinterpret_cast<uintptr_t>(q->src) % src_align != 0 || reinterpret_cast<uintptr_t>(q->dst) % 16 != 0)
+                return fail(FA_ERR_INVALID_ARG, "fa_kv_dequant: src must be %lld-byte and dst 16-byte aligned",
+                            (long long)src_align);
             const int64_t pitch = q->src_row_bytes > 2 * q->dst_row_stride ? q->src_row_bytes : 2 * q->dst_row_stride;
             if (q->n_rows > (INT64_MAX / 4) / pitch)
                 return fail(FA_ERR_INVALID_ARG, "fa_kv_dequant: rows * pitch overflows");
             any = true;
         }
-        L[i] = fa::KvDequantLaunch{q->src, q->type, q->n_rows, q->row_elems, q->src_row_bytes, q->dst,
-                                   q->dst_row_stride};
+        L[i] = fa::KvDequantLaunch{q->src,     q->type, q->n_rows,         q->row_elems,
+                                   q->src_row_bytes, q->dst, q->dst_row_stride, q->scale};
     }
     if (!any) return FA_OK;
     int sms = 0;

@@ -108,7 +108,8 @@ size_t mla_tail_ws_bytes(const TailLaunch &L);
 cudaError_t launch_mla_tail(const TailLaunch &L, int num_sms, cudaStream_t stream);
 cudaError_t tail_device_error(int clear, int *code);
 
-// Quantised K/V rows -> bf16 (kv_dequant.cu).  type: 8 = q8_0, 4 = q4_0.
+// Quantised K/V rows -> bf16 (kv_dequant.cu).  type: 8 = q8_0, 4 = q4_0,
+// 2 = fp8 e4m3 times `scale`.
 struct KvDequantLaunch {
     const void *src;
     int type;
@@ -117,6 +118,7 @@ struct KvDequantLaunch {
     int64_t src_row_bytes;
     void *dst;
     int64_t dst_row_stride;
+    float scale;
 };
 constexpr int kMaxDequantSegs = 4;  // tensors one launch converts (all of one type)
 cudaError_t launch_kv_dequant(const KvDequantLaunch *L, int n, int num_sms, cudaStream_t stream);

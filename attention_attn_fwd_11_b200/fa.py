@@ -68,11 +68,12 @@ class MlaTailParams(ctypes.Structure):
 
 class KvDequantParams(ctypes.Structure):
     _fields_ = [("src", _vp), ("type", _i32), ("n_rows", _i64), ("row_elems", _i32), ("src_row_bytes", _i64),
-                ("dst", _vp), ("dst_row_stride", _i64)]
+                ("dst", _vp), ("dst_row_stride", _i64), ("scale", ctypes.c_float)]
 
 
-FA_KV_Q8_0, FA_KV_Q4_0 = 8, 4
-KV_QUANT = {"q8_0": (FA_KV_Q8_0, 34), "q4_0": (FA_KV_Q4_0, 18)}  # type code, bytes per 32-value block
+FA_KV_Q8_0, FA_KV_Q4_0, FA_KV_FP8_E4M3 = 8, 4, 2
+KV_QUANT = {"q8_0": (FA_KV_Q8_0, 34), "q4_0": (FA_KV_Q4_0, 18),
+            "fp8_e4m3": (FA_KV_FP8_E4M3, 32)}  # type code, bytes per 32 values
 
 _lib = None
 
@@ -361,20 +362,22 @@ def device_error(clear=True) -> int:
 
 # ------------------------------------------------------ quantised K/V rows --
 
-def kv_dequant_params(src, qtype, row_elems, dst):
+def kv_dequant_params(src, qtype, row_elems, dst, kv_scale=1.0):
     """Marshal a fa_kv_dequant call: src uint8 [..., row_bytes] (rows of
-    ggml blocks), dst bf16 [..., >= row_elems] with unit stride in the last
-    dimension and the same leading shape, both contiguous over the rows."""
+    ggml blocks or fp8 bytes), dst bf16 [..., >= row_elems] with unit stride
+    in the last dimension and the same leading shape, both contiguous over
+    the rows; kv_scale: the fp8 tensor scale."""
     code, _ = KV_QUANT[qtype]
     p = KvDequantParams()
     p.src, p.type, p.row_elems, p.dst = _ptr(src), code, row_elems, _ptr(dst)
+    p.scale = kv_scale
     p.n_rows = src.numel() // src.shape[-1] if src.dim() else 0
     p.src_row_bytes = src.stride(-2) if src.dim() > 1 else src.shape[-1]
     p.dst_row_stride = dst.stride(-2) if dst.dim() > 1 else dst.shape[-1]
     return p
 
 
-def _dequant_entry(src, qtype, row_elems, out):
+def _dequant_entry(src, qtype, row_elems, out, kv_scale=1.0):
     _need_cuda(src, out)
     if src.dtype != torch.uint8:
         raise ValueError("src must be uint8 blocks")
@@ -388,24 +391,24 @@ def _dequant_entry(src, qtype, row_elems, out):
     s2, o2 = src.reshape(-1, src.shape[-1]), out.reshape(-1, out.shape[-1])
     if s2.data_ptr() != src.data_ptr() or o2.data_ptr() != out.data_ptr():
         raise ValueError("leading dimensions must collapse to one row stride")
-    return kv_dequant_params(s2, qtype, row_elems, o2), out
+    return kv_dequant_params(s2, qtype, row_elems, o2, kv_scale), out
 
 
-def kv_dequant(src, qtype, row_elems, out=None, stream=None):
+def kv_dequant(src, qtype, row_elems, out=None, stream=None, kv_scale=1.0):
     """Quantised rows -> bf16 rows on the GPU (fa_kv_dequant).  src: uint8
-    CUDA tensor [..., row_bytes] whose rows each hold row_elems / 32 ggml
-    blocks of ``qtype`` ('q8_0' or 'q4_0'); the leading dimensions must
-    collapse to one row index with a single stride.  Returns (or fills) a
-    bf16 tensor [..., row_elems]."""
-    p, out = _dequant_entry(src, qtype, row_elems, out)
+    CUDA tensor [..., row_bytes] whose rows each hold row_elems values of
+    ``qtype`` ('q8_0' or 'q4_0' ggml blocks, or 'fp8_e4m3' bytes read as
+    e4m3 * kv_scale); the leading dimensions must collapse to one row index
+    with a single stride.  Returns (or fills) a bf16 tensor [..., row_elems]."""
+    p, out = _dequant_entry(src, qtype, row_elems, out, kv_scale)
     _check(load().fa_kv_dequant(ctypes.byref(p), _stream(stream)))
     return out
 
 
 def kv_dequant_many(entries, stream=None):
     """Several conversions in one launch (fa_kv_dequant_n).  entries: list of
-    (src, qtype, row_elems, out-or-None), 1 to 4 of them, one qtype.
-    Returns the list of outputs."""
+    (src, qtype, row_elems, out-or-None[, kv_scale]), 1 to 4 of them, one
+    qtype.  Returns the list of outputs."""
     made = [_dequant_entry(*e) for e in entries]
     arr = (KvDequantParams * len(made))(*[m[0] for m in made])
     _check(load().fa_kv_dequant_n(arr, len(made), _stream(stream)))
@@ -413,14 +416,15 @@ def kv_dequant_many(entries, stream=None):
 
 
 def fwd_quant(q, k_blocks, v_blocks, qtype, dk, dv, scale=None, causal=False, out=None, return_lse=True,
-              out_dtype=torch.float32, k_buf=None, v_buf=None, stream=None, **mods):
+              out_dtype=torch.float32, k_buf=None, v_buf=None, stream=None, k_scale=1.0, v_scale=1.0, **mods):
     """Prefill over quantised K/V, the pages' way: dequantise K and V to bf16
     (one fa_kv_dequant_n launch for both) and run fa_fwd on them.  k_blocks /
     v_blocks: uint8 [B, Hkv, Sk, dk / 32 * block bytes] and [..., dv / 32 *
     block bytes]; k_buf / v_buf: optional bf16 [B, Hkv, Sk, dk / dv] buffers
-    for the dequantised rows (allocated when absent).  Other arguments as
-    fwd()."""
-    k, v = kv_dequant_many([(k_blocks, qtype, dk, k_buf), (v_blocks, qtype, dv, v_buf)], stream=stream)
+    for the dequantised rows (allocated when absent); k_scale / v_scale: the
+    fp8 tensor scales.  Other arguments as fwd()."""
+    k, v = kv_dequant_many([(k_blocks, qtype, dk, k_buf, k_scale), (v_blocks, qtype, dv, v_buf, v_scale)],
+                           stream=stream)
     return fwd(q, k, v, scale=scale, causal=causal, out=out, return_lse=return_lse, out_dtype=out_dtype,
                stream=stream, **mods)
 

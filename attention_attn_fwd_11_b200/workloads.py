@@ -161,6 +161,8 @@ def random_quant_rows(shape, row_elems: int, qtype: str, seed: int):
 # The causal MHA shape with q8_0 K/V (the prefill reads the dequantised rows).
 QUANT_C2 = PrefillCase("causal_mha_q8_0kv_b2_h16_s2048_d128", 2, 16, 16, 2048, 2048, 128, 128, True, seed=2)
 QUANT_C2_TYPE = "q8_0"
+# ... and with FP8 E4M3 K/V (per-tensor scale FP8_SCALE).
+FP8_C2 = PrefillCase("causal_mha_fp8kv_b2_h16_s2048_d128", 2, 16, 16, 2048, 2048, 128, 128, True, seed=2)
 
 
 # C2's shape with every modifier on: ALiBi (max_bias 8) over a head-shared

@@ -57,6 +57,7 @@ NCU_TRAFFIC = {
     "causal_mha_b2_h16_s2048_dk192_dv128": 73713408,
     "causal_gqa_b2_hq16_hkv4_s2048_dk192_dv192": 40004096,
     "kv_dequant causal_mha_q8_0kv_b2_h16_s2048_d128": 17835776,
+    "kv_dequant causal_mha_fp8kv_b2_h16_s2048_d128": 16799744,
     "paged_prefill_gqa_b16_hq32_hkv8_sq512_d128_bs64": 651760896,
     "mla_tail_t32_hq128_r512_v128_hidden7168": 257049088,
     "causal_gqa_b1_hq16_hkv4_s4096_dk320_dv256": 77931264,
@@ -258,6 +259,7 @@ def quant_prefill_workload(torch, fa, W_, c, qtype, l2, dequant_only=False):
     q0 = W_.randn_bf16((c.B, c.Hq, c.Sq, c.dk), 1000 + c.seed)
     kb0 = W_.random_quant_rows((c.B, c.Hkv, c.Sk), c.dk, qtype, c.seed)
     vb0 = W_.random_quant_rows((c.B, c.Hkv, c.Sk), c.dv, qtype, c.seed + 100)
+    kv_scale = W_.FP8_SCALE if qtype == "fp8_e4m3" else 1.0
     kv_bf16 = c.B * c.Hkv * c.Sk * (c.dk + c.dv) * 2
     dq_bytes = kb0.numel() + vb0.numel() + kv_bf16  # quantised blocks read + bf16 rows written
     foot = q0.numel() * 2 + dq_bytes + c.B * c.Hq * c.Sq * (c.dv * 4 + 4)
@@ -271,8 +273,9 @@ def quant_prefill_workload(torch, fa, W_, c, qtype, l2, dequant_only=False):
         o = torch.empty(c.B, c.Hq, c.Sq, c.dv, device="cuda")
         lse = torch.empty(c.B, c.Hq, c.Sq, device="cuda")
         bufs.append((q, kb, vb, kbuf, vbuf, o, lse))
-        pkv = (fa.KvDequantParams * 2)(fa.kv_dequant_params(kb.view(-1, kb.shape[-1]), qtype, c.dk, kbuf.view(-1, c.dk)),
-                                       fa.kv_dequant_params(vb.view(-1, vb.shape[-1]), qtype, c.dv, vbuf.view(-1, c.dv)))
+        pkv = (fa.KvDequantParams * 2)(
+            fa.kv_dequant_params(kb.view(-1, kb.shape[-1]), qtype, c.dk, kbuf.view(-1, c.dk), kv_scale),
+            fa.kv_dequant_params(vb.view(-1, vb.shape[-1]), qtype, c.dv, vbuf.view(-1, c.dv), kv_scale))
         pf = fa.fwd_params(q, kbuf, vbuf, o, lse, c.scale, c.causal)
         params.append((pkv, pf))
 
@@ -483,12 +486,15 @@ def run_only(args):
                                  W_.CAUSAL_DK192_DV192, W_.CAUSAL_DK320, W_.PAGED_GQA, W_.LATENT_SPARSE,
                                  W_.QUANT_C2, W_.PAGED_PREFILL, W_.MLA_TAIL)}
     table["kv_dequant_" + W_.QUANT_C2.name] = W_.QUANT_C2
+    table[W_.FP8_C2.name] = W_.FP8_C2
+    table["kv_dequant_" + W_.FP8_C2.name] = W_.FP8_C2
     if args.only not in table:
         raise SystemExit("unknown workload %r; one of %s" % (args.only, sorted(table)))
     c = table[args.only]
-    if c is W_.QUANT_C2:
+    if c is W_.QUANT_C2 or c is W_.FP8_C2:
         only_dq = args.only.startswith("kv_dequant_")
-        launch, n, work, kpl = quant_prefill_workload(torch, fa, W_, c, W_.QUANT_C2_TYPE, l2, dequant_only=only_dq)
+        qt = W_.QUANT_C2_TYPE if c is W_.QUANT_C2 else "fp8_e4m3"
+        launch, n, work, kpl = quant_prefill_workload(torch, fa, W_, c, qt, l2, dequant_only=only_dq)
         unit, amount = ("GB/s", work / 1e9) if only_dq else ("TFLOP/s", c.flops / 1e12)
     elif isinstance(c, W_.PrefillCase):
         launch, n, work, kpl = prefill_workload(torch, fa, W_, c, l2)

@@ -333,7 +333,11 @@ fa_status fa_mla_tail(const fa_mla_tail_params *p, void *stream);
  *         int8 codes q; value j = d * q_j;
  *       FA_KV_Q4_0: 18 bytes per block -- f16 scale d, then 16 bytes; byte j
  *         holds value j in its low nibble and value j + 16 in its high
- *         nibble; value = d * (nibble - 8).
+ *         nibble; value = d * (nibble - 8);
+ *       FA_KV_FP8_E4M3: one OCP FP8 E4M3 byte per value (32 bytes per 32
+ *         values), value = e4m3 * scale with one fp32 scale for the tensor,
+ *         as FP8 KV caches keep it; the exact product is rounded once.
+ *         src must be 8-byte aligned and src_row_bytes a multiple of 8.
  *   dst: bf16 rows at a pitch of dst_row_stride elements; the first
  *     row_elems elements of each row are written, the rest left as they are.
  *   Each value d * q is exact in fp32 and rounded once, to nearest even, to
@@ -344,7 +348,7 @@ fa_status fa_mla_tail(const fa_mla_tail_params *p, void *stream);
  * (0 launches nothing).  src and dst must not overlap.  Non-finite scales
  * decode as IEEE arithmetic gives them (inf * 0 = NaN).
  */
-typedef enum { FA_KV_Q8_0 = 8, FA_KV_Q4_0 = 4 } fa_kv_quant;
+typedef enum { FA_KV_Q8_0 = 8, FA_KV_Q4_0 = 4, FA_KV_FP8_E4M3 = 2 } fa_kv_quant;
 
 typedef struct {
     const void *src;
@@ -354,6 +358,7 @@ typedef struct {
     int64_t src_row_bytes;
     void *dst;
     int64_t dst_row_stride;
+    float scale; /* FA_KV_FP8_E4M3 only: the tensor's scale (finite) */
 } fa_kv_dequant_params;
 
 fa_status fa_kv_dequant(const fa_kv_dequant_params *p, void *stream);

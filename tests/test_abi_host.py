@@ -204,7 +204,8 @@ def test_mla_tail_workspace_size_and_validation():
 
 def dequant_params(**kw):
     p = fa.KvDequantParams()
-    base = dict(src=2, type=fa.FA_KV_Q8_0, n_rows=1024, row_elems=128, src_row_bytes=136, dst=16, dst_row_stride=128)
+    base = dict(src=2, type=fa.FA_KV_Q8_0, n_rows=1024, row_elems=128, src_row_bytes=136, dst=16, dst_row_stride=128,
+                scale=1.0)
     base.update(kw)
     for k_, v_ in base.items():
         setattr(p, k_, v_)
@@ -224,6 +225,10 @@ def dequant_params(**kw):
     (dict(dst=24), fa.FA_ERR_INVALID_ARG),                   # dst not 16-byte aligned
     (dict(src=0), fa.FA_ERR_INVALID_ARG),
     (dict(type=fa.FA_KV_Q4_0, src_row_bytes=70), fa.FA_ERR_INVALID_ARG),   # 4 q4_0 blocks need 72
+    (dict(type=fa.FA_KV_FP8_E4M3, src_row_bytes=132, src=8), fa.FA_ERR_INVALID_ARG),  # fp8 pitch % 8
+    (dict(type=fa.FA_KV_FP8_E4M3, src_row_bytes=136, src=4), fa.FA_ERR_INVALID_ARG),  # fp8 src % 8
+    (dict(type=fa.FA_KV_FP8_E4M3, src_row_bytes=120, src=8), fa.FA_ERR_INVALID_ARG),  # < 128 bytes
+    (dict(type=fa.FA_KV_FP8_E4M3, src_row_bytes=128, src=8, scale=float("inf")), fa.FA_ERR_INVALID_ARG),
 ])
 def test_kv_dequant_rejects(kw, status):
     assert fa.load().fa_kv_dequant(ctypes.byref(dequant_params(**kw)), None) == status

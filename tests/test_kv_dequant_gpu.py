@@ -14,7 +14,7 @@ from parity import check
 
 pytestmark = pytest.mark.gpu
 
-BB = {"q8_0": 34, "q4_0": 18}
+BB = {"q8_0": 34, "q4_0": 18, "fp8_e4m3": 32}
 
 
 def bits_of(t):
@@ -81,3 +81,62 @@ def test_prefill_over_quantised_kv(qtype, d):
 
 def test_prefill_over_quantised_kv_pair():
     run_quant(1, 4, 1, 200, 260, 192, 128, False, "q8_0", seed=11)
+
+
+@pytest.mark.parametrize("row_elems", [32, 128, 576])
+@pytest.mark.parametrize("kv_scale", [1.0 / 16, 0.3, -2.5])
+def test_fp8_bit_exact_with_pitches(row_elems, kv_scale):
+    # every byte value but the two NaN codes, any scale: the exact product
+    # rounded once must match the oracle bit for bit
+    rng = np.random.default_rng(row_elems)
+    n_rows = 777
+    row_bytes = row_elems + 16
+    src = rng.integers(0, 256, (n_rows, row_bytes), dtype=np.uint8)
+    src[src == 0x7F] = 0x00
+    src[src == 0xFF] = 0x80
+    pitch = row_elems + 8
+    buf = torch.full((n_rows, pitch), float("nan"), dtype=torch.bfloat16, device="cuda")
+    out = fa.kv_dequant(torch.from_numpy(src).cuda(), "fp8_e4m3", row_elems, out=buf[:, :row_elems],
+                        kv_scale=kv_scale)
+    torch.cuda.synchronize()
+    want = oracle.dequant_rows(src, "fp8_e4m3", row_elems, scale=np.float32(kv_scale))
+    assert np.array_equal(bits_of(out), want)
+    assert torch.isnan(buf[:, row_elems:].float()).all()
+
+
+def test_prefill_over_fp8_kv():
+    B, Hq, Hkv, Sq, Sk, d = 2, 4, 2, 300, 333, 128
+    q = W.randn_bf16((B, Hq, Sq, d), 1000 + 31)
+    kb = W.random_quant_rows((B, Hkv, Sk), d, "fp8_e4m3", 31)
+    vb = W.random_quant_rows((B, Hkv, Sk), d, "fp8_e4m3", 32)
+    sc = 1.0 / d ** 0.5
+    o, lse = fa.fwd_quant(q.cuda(), kb.cuda(), vb.cuda(), "fp8_e4m3", d, d, scale=sc, causal=True,
+                          k_scale=W.FP8_SCALE, v_scale=W.FP8_SCALE)
+    torch.cuda.synchronize()
+    assert fa.device_error() == 0
+    kbits = oracle.dequant_rows(kb.numpy(), "fp8_e4m3", d, scale=W.FP8_SCALE)
+    vbits = oracle.dequant_rows(vb.numpy(), "fp8_e4m3", d, scale=W.FP8_SCALE)
+    o_ref, l_ref = oracle.attention(W.bits(q), kbits, vbits, sc, True)
+    check(o, o_ref, lse, l_ref, what="fp8 kv prefill")
+
+
+@pytest.mark.parametrize("target,direction,want", [
+    (1 + 2.0 ** -8, +1, 0x3F81),      # fp32 lands on the 1 / 1+2^-7 midpoint, exact value above it
+    (1 + 3 * 2.0 ** -8, -1, 0x3F81),  # lands on the 1+2^-7 / 1+2^-6 midpoint, exact value below it
+])
+def test_fp8_double_rounding_cases(target, direction, want):
+    # 1.125 (e4m3 0x39) times a scale chosen so that fp32 rounding of the
+    # product gives exactly a bf16 midpoint while the exact product lies on
+    # one side: rounding the fp32 product (ties to even) would give the other
+    # neighbour; the single rounding of the exact value gives `want`.
+    s = np.float32(target / 1.125)
+    s = np.nextafter(s, np.float32(np.inf) if direction > 0 else np.float32(-np.inf))
+    assert np.float32(1.125) * s == np.float32(target)
+    src = np.zeros((1, 32), np.uint8)
+    src[0, 0], src[0, 1] = 0x39, 0xB9
+    out = fa.kv_dequant(torch.from_numpy(src).cuda(), "fp8_e4m3", 32, kv_scale=float(s))
+    torch.cuda.synchronize()
+    got = bits_of(out)[0]
+    ref = oracle.dequant_rows(src, "fp8_e4m3", 32, scale=float(s))[0]
+    assert got[0] == want and got[1] == (want | 0x8000)
+    assert np.array_equal(got, ref)
