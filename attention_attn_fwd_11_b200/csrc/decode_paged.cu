@@ -47,15 +47,59 @@ constexpr int PD_STAGE = 2 * PD_TILE;            // K + V
 constexpr int PD_OFF_BAR = PD_NST * PD_STAGE;
 constexpr int PD_SMEM = PD_OFF_BAR + 128 + 1024;  // ring + barriers + 1024-byte alignment slack
 
+// q8_0 caches (the dequant prologue): a cache row is 4 ggml q8_0 blocks
+// (f16 scale + 32 int8 codes, 34 bytes), 136 bytes for 128 values.  A
+// (block, head) tile of K or V is 64 such rows, contiguous, moved with one
+// bulk copy.  Each consumer warp converts its own 16 keys of K and V into a
+// private bf16 buffer laid out like the bf16 ring (two 64-column halves,
+// 128-byte swizzle), then runs the bf16 path on it.
+#ifndef FA_PD_Q8_PRMT
+#define FA_PD_Q8_PRMT 1
+#endif
+constexpr int PDQ_ROW = 136;
+constexpr int PDQ_TILE = PD_BS * PDQ_ROW;          // 8704 bytes
+constexpr int PDQ_STAGE = 2 * PDQ_TILE;            // K + V, 17 KB (1024-byte multiple)
+constexpr int PDQ_NST = 4;
+constexpr int PDQ_WBUF = 2 * 16 * PD_D * 2;        // one warp's 16 keys of K and V in bf16: 8 KB
+constexpr int PDQ_OFF_WB = PDQ_NST * PDQ_STAGE;
+constexpr int PDQ_OFF_BAR = PDQ_OFF_WB + 4 * PDQ_WBUF;
+constexpr int PDQ_SMEM = PDQ_OFF_BAR + 128 + 1024;
+
+// Two int8 codes (low and high byte of w) times the block scale d -> a bf16
+// pair.  A code's byte xor 0x80 is code + 128; OR-ed into the mantissa of
+// 2^23 it gives 2^23 + code + 128 exactly, and subtracting 2^23 + 128
+// leaves the code (both steps exact).  code * d is exact in fp32 (8 + 11
+// significant bits), so the bf16 conversion is the only rounding -- the
+// same value the pre-pass (fa_kv_dequant) writes.
+FA_DEV uint32_t q8_pair_to_bf16(uint32_t w, uint64_t d2) {
+#if FA_PD_Q8_PRMT
+    // byte permutes build both fp32 patterns; the subtract and the scale run
+    // as packed fp32 pairs
+    const uint32_t x = w ^ 0x8080u;
+    const uint64_t f = f2_pack(__uint_as_float(__byte_perm(x, 0x4B000000u, 0x7440)),
+                               __uint_as_float(__byte_perm(x, 0x4B000000u, 0x7441)));
+    float a, b;
+    f2_unpack(f2_mul(f2_add(f, f2_pack(-8388736.f, -8388736.f)), d2), a, b);
+    return pack_bf16x2(a, b);
+#else
+    float d, d_;
+    f2_unpack(d2, d, d_);
+    const float f0 = __uint_as_float(0x4B000000u | ((w & 0xffu) ^ 0x80u)) - 8388736.f;
+    const float f1 = __uint_as_float(0x4B000000u | (((w >> 8) & 0xffu) ^ 0x80u)) - 8388736.f;
+    return pack_bf16x2(f0 * d, f1 * d);
+#endif
+}
+
 struct PagedArgs {
     const __nv_bfloat16 *q;
+    const uint8_t *kq, *vq;  // q8_0 caches (KVQ instantiation)
     const int32_t *block_table, *seq_lens;
     int max_blocks, Hq, Hkv, num_blocks, bps, num_splits;
     float scale_log2;
     float *part_o, *part_lse;
 };
 
-template <int G>
+template <int G, bool KVQ>
 __global__ void __launch_bounds__(160) paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                                                            const __grid_constant__ CUtensorMap tmV,
                                                            const PagedArgs a) {
@@ -75,15 +119,18 @@ __global__ void __launch_bounds__(160) paged_decode_kernel(const __grid_constant
     if (blk0 >= nb) return;  // this split holds no key of this sequence (uniform exit)
     const int nblk = min(a.bps, nb - blk0);
 
+    constexpr int NST = KVQ ? PDQ_NST : PD_NST;
+    constexpr int STAGE = KVQ ? PDQ_STAGE : PD_STAGE;
+    constexpr int OFF_BAR = KVQ ? PDQ_OFF_BAR : PD_OFF_BAR;
     const uint32_t sbase = smem_u32(smem);
-    const uint32_t bar0 = sbase + PD_OFF_BAR;
+    const uint32_t bar0 = sbase + OFF_BAR;
     auto full = [&](int s) { return bar0 + 8u * s; };
-    auto empty = [&](int s) { return bar0 + 8u * (PD_NST + s); };
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + PD_OFF_BAR + 8 * 2 * PD_NST);
+    auto empty = [&](int s) { return bar0 + 8u * (NST + s); };
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_BAR + 8 * 2 * NST);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
-        for (int s = 0; s < PD_NST; ++s) {
+        for (int s = 0; s < NST; ++s) {
             mbar_init(full(s), 1);
             mbar_init(empty(s), 4);
         }
@@ -94,7 +141,7 @@ __global__ void __launch_bounds__(160) paged_decode_kernel(const __grid_constant
 
     if (warp == 4) {
         // ---------------------------------------------------- producer --
-        if (lane == 0) {
+        if (!KVQ && lane == 0) {
             prefetch_tmap(&tmK);
             prefetch_tmap(&tmV);
         }
@@ -110,25 +157,33 @@ __global__ void __launch_bounds__(160) paged_decode_kernel(const __grid_constant
                 }
             }
             const int blk = __shfl_sync(0xffffffffu, ids, i & 31);
-            const int s = i % PD_NST;
-            const uint32_t ph = (uint32_t)(i / PD_NST) & 1u;
+            const int s = i % NST;
+            const uint32_t ph = (uint32_t)(i / NST) & 1u;
             bool ok = true;
             if (lane == 0) ok = mbar_wait(empty(s), ph ^ 1u, abort_flag, &g_decode_err);
             if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
             if (lane == 0) {
-                const int row0 = (blk * a.Hkv + hkv) * PD_BS;  // first cache row of this (block, head)
-                const uint32_t dst = sbase + s * PD_STAGE;
-                mbar_arrive_expect_tx(full(s), PD_STAGE);
-                tma_load_2d(dst, &tmK, full(s), 0, row0);
-                tma_load_2d(dst + PD_TILE / 2, &tmK, full(s), 64, row0);
-                tma_load_2d(dst + PD_TILE, &tmV, full(s), 0, row0);
-                tma_load_2d(dst + PD_TILE + PD_TILE / 2, &tmV, full(s), 64, row0);
+                if constexpr (KVQ) {
+                    const int64_t off = ((int64_t)blk * a.Hkv + hkv) * PDQ_TILE;  // this (block, head) tile
+                    const uint32_t dst = sbase + s * PDQ_STAGE;
+                    mbar_arrive_expect_tx(full(s), PDQ_STAGE);
+                    bulk_load(dst, a.kq + off, PDQ_TILE, full(s));
+                    bulk_load(dst + PDQ_TILE, a.vq + off, PDQ_TILE, full(s));
+                } else {
+                    const int row0 = (blk * a.Hkv + hkv) * PD_BS;  // first cache row of this (block, head)
+                    const uint32_t dst = sbase + s * PD_STAGE;
+                    mbar_arrive_expect_tx(full(s), PD_STAGE);
+                    tma_load_2d(dst, &tmK, full(s), 0, row0);
+                    tma_load_2d(dst + PD_TILE / 2, &tmK, full(s), 64, row0);
+                    tma_load_2d(dst + PD_TILE, &tmV, full(s), 0, row0);
+                    tma_load_2d(dst + PD_TILE + PD_TILE / 2, &tmV, full(s), 64, row0);
+                }
             }
             issued = i + 1;
         }
         if (lane == 0 && *abort_flag) {
-            for (int i = max(0, issued - PD_NST); i < issued; ++i)
-                mbar_wait_drain(full(i % PD_NST), (uint32_t)(i / PD_NST) & 1u);
+            for (int i = max(0, issued - NST); i < issued; ++i)
+                mbar_wait_drain(full(i % NST), (uint32_t)(i / NST) & 1u);
         }
         return;
     }
@@ -161,21 +216,61 @@ __global__ void __launch_bounds__(160) paged_decode_kernel(const __grid_constant
 
     bool ok = true;
     for (int i = 0; i < nblk; ++i) {
-        const int s = i % PD_NST;
-        if (!mbar_wait(full(s), (uint32_t)(i / PD_NST) & 1u, abort_flag, &g_decode_err)) {
+        const int s = i % NST;
+        if (!mbar_wait(full(s), (uint32_t)(i / NST) & 1u, abort_flag, &g_decode_err)) {
             ok = false;
             break;
         }
-        const uint32_t sK = sbase + s * PD_STAGE;
-        const uint32_t sV = sK + PD_TILE;
+        // K and V tiles of this warp's keys: the ring stage (bf16), or the
+        // warp's private buffer after the q8_0 prologue.  `kof` maps a key of
+        // the block to its row in the tile; `hstr` is the byte distance
+        // between the two 64-column halves.
+        uint32_t sK, sV, hstr;
+        int kof;
+        if constexpr (KVQ) {
+            // lane (lk, h) converts row lk's half h (two q8_0 blocks, 64 values)
+            // of K and of V into eight 16-byte chunks of the swizzled buffer
+            const int lk = lane >> 1, h = lane & 1;
+            const uint8_t *raw = smem + s * PDQ_STAGE + (warp * 16 + lk) * PDQ_ROW + 68 * h;
+            uint8_t *wb = smem + PDQ_OFF_WB + warp * PDQ_WBUF + h * (16 * 128) + lk * 128;
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {  // K, then V
+#pragma unroll
+                for (int qb = 0; qb < 2; ++qb) {
+                    const uint8_t *p = raw + t * PDQ_TILE + 34 * qb;
+                    const float d = __half2float(*reinterpret_cast<const __half *>(p));
+                    const uint64_t d2 = f2_pack(d, d);
+                    const uint16_t *cw = reinterpret_cast<const uint16_t *>(p + 2);
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj) {
+                        const int j = 4 * qb + jj;  // 16-byte chunk of the half-row
+                        const uint4 v = make_uint4(q8_pair_to_bf16(cw[4 * jj], d2), q8_pair_to_bf16(cw[4 * jj + 1], d2),
+                                                   q8_pair_to_bf16(cw[4 * jj + 2], d2),
+                                                   q8_pair_to_bf16(cw[4 * jj + 3], d2));
+                        *reinterpret_cast<uint4 *>(wb + t * (2 * 16 * 128) + ((j ^ (lk & 7)) << 4)) = v;
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(empty(s));  // the raw stage may be refilled now
+            sK = sbase + PDQ_OFF_WB + warp * PDQ_WBUF;
+            sV = sK + 2 * 16 * 128;
+            hstr = 16 * 128;
+            kof = warp * 16;
+        } else {
+            sK = sbase + s * PD_STAGE;
+            sV = sK + PD_TILE;
+            hstr = PD_TILE / 2;
+            kof = 0;
+        }
         // ---- S = Q K^T for this warp's 16 keys (two n-tiles of 8) ----
         float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
         {
-            const int key = warp * 16 + (mi >> 1) * 8 + lr;
+            const int key = warp * 16 + (mi >> 1) * 8 + lr - kof;
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
                 const int d0 = ks * 16 + (mi & 1) * 8;
-                const uint32_t addr = sK + (uint32_t)((d0 >> 6) * (PD_TILE / 2) + key * 128 +
+                const uint32_t addr = sK + (uint32_t)(d0 >> 6) * hstr + (uint32_t)(key * 128 +
                                                       ((((d0 & 63) >> 3) ^ (key & 7)) << 4));
                 uint32_t b00, b01, b10, b11;
                 ldsm_x4(addr, b00, b01, b10, b11);
@@ -211,11 +306,11 @@ __global__ void __launch_bounds__(160) paged_decode_kernel(const __grid_constant
         const uint32_t pa0 = pack_bf16x2(p[0], p[1]);
         const uint32_t pa2 = pack_bf16x2(p[2], p[3]);
         {
-            const int key = warp * 16 + (mi & 1) * 8 + lr;
+            const int key = warp * 16 + (mi & 1) * 8 + lr - kof;
 #pragma unroll
             for (int pr = 0; pr < 8; ++pr) {
                 const int nt = 2 * pr + (mi >> 1);  // 8-wide slice of head dims
-                const uint32_t addr = sV + (uint32_t)(((nt * 8) >> 6) * (PD_TILE / 2) + key * 128 +
+                const uint32_t addr = sV + (uint32_t)((nt * 8) >> 6) * hstr + (uint32_t)(key * 128 +
                                                       (((nt & 7) ^ (key & 7)) << 4));
                 uint32_t v0l, v0h, v1l, v1h;
                 ldsm_x4_t(addr, v0l, v0h, v1l, v1h);
@@ -224,7 +319,7 @@ __global__ void __launch_bounds__(160) paged_decode_kernel(const __grid_constant
             }
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(empty(s));
+        if (!KVQ && lane == 0) mbar_arrive(empty(s));
     }
     // the four lanes of a quad hold partial sums of the same head
     l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
@@ -364,19 +459,27 @@ cudaError_t launch_combine(const float *part_o, const float *part_lse, int rows,
     return cudaGetLastError();
 }
 
-template <int G>
+template <int G, bool KVQ>
 static cudaError_t launch_g(const PagedLaunch &L, const PagedArgs &a, int B, cudaStream_t stream) {
-    auto kern = paged_decode_kernel<G>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, PD_SMEM);
+    auto kern = paged_decode_kernel<G, KVQ>;
+    constexpr int smem = KVQ ? PDQ_SMEM : PD_SMEM;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)a.num_splits, (unsigned)a.Hkv, (unsigned)B);
-    kern<<<grid, 160, PD_SMEM, stream>>>(L.tmK, L.tmV, a);
+    kern<<<grid, 160, smem, stream>>>(L.tmK, L.tmV, a);
     return cudaGetLastError();
+}
+
+template <int G>
+static cudaError_t launch_gq(const PagedLaunch &L, const PagedArgs &a, int B, cudaStream_t stream) {
+    return L.kv_q8 ? launch_g<G, true>(L, a, B, stream) : launch_g<G, false>(L, a, B, stream);
 }
 
 cudaError_t launch_decode_paged(const PagedLaunch &L, cudaStream_t stream) {
     PagedArgs a;
     a.q = static_cast<const __nv_bfloat16 *>(L.q);
+    a.kq = static_cast<const uint8_t *>(L.k_cache);
+    a.vq = static_cast<const uint8_t *>(L.v_cache);
     a.block_table = L.block_table;
     a.seq_lens = L.seq_lens;
     a.max_blocks = L.max_blocks_per_seq;
@@ -390,10 +493,10 @@ cudaError_t launch_decode_paged(const PagedLaunch &L, cudaStream_t stream) {
     a.part_lse = L.part_lse;
     cudaError_t e;
     switch (L.Hq / L.Hkv) {
-        case 1: e = launch_g<1>(L, a, L.B, stream); break;
-        case 2: e = launch_g<2>(L, a, L.B, stream); break;
-        case 4: e = launch_g<4>(L, a, L.B, stream); break;
-        case 8: e = launch_g<8>(L, a, L.B, stream); break;
+        case 1: e = launch_gq<1>(L, a, L.B, stream); break;
+        case 2: e = launch_gq<2>(L, a, L.B, stream); break;
+        case 4: e = launch_gq<4>(L, a, L.B, stream); break;
+        case 8: e = launch_gq<8>(L, a, L.B, stream); break;
         default: return cudaErrorInvalidValue;
     }
     if (e != cudaSuccess) return e;

@@ -145,6 +145,9 @@ fa_status check_paged(const fa_decode_paged_params *p) {
         return fail(FA_ERR_UNSUPPORTED, "fa_decode_paged: Hq / Hkv must be 1, 2, 4 or 8 (got %d)", g);
     if (!finite_pos(p->scale)) return fail(FA_ERR_INVALID_ARG, "fa_decode_paged: scale must be finite and > 0");
     if (p->o_dtype != FA_F32 && p->o_dtype != FA_BF16) return fail(FA_ERR_INVALID_ARG, "fa_decode_paged: o_dtype");
+    if (p->kv_type != FA_KV_BF16 && p->kv_type != FA_KV_Q8_0)
+        return fail(FA_ERR_UNSUPPORTED, "fa_decode_paged: kv_type must be FA_KV_BF16 or FA_KV_Q8_0 (got %d)",
+                    p->kv_type);
     return FA_OK;
 }
 
@@ -164,6 +167,11 @@ fa_status check_paged_ptrs(const fa_decode_paged_params *p) {
 // Both caches as 2-D [num_blocks * Hkv * 64 rows, 128] bf16 tensors for TMA
 // (128-byte swizzle, 64 x 64 boxes).
 fa_status encode_paged_caches(const fa_decode_paged_params *p, fa::PagedLaunch *L) {
+    memset(L, 0, sizeof *L);
+    if (p->kv_type == FA_KV_Q8_0) {  // q8_0 tiles move with plain bulk copies: no tensor maps
+        L->kv_q8 = true;
+        return FA_OK;
+    }
     if (!get_encoder()) return fail(FA_ERR_CUDA, "fa_decode_paged: cuTensorMapEncodeTiled is not available");
     const int64_t rows = (int64_t)p->num_blocks * p->Hkv * p->block_size;
     if (rows >= (int64_t(1) << 31))

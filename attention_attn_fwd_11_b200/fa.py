@@ -42,7 +42,7 @@ class PagedParams(ctypes.Structure):
                 ("max_blocks_per_seq", _i32), ("B", _i32), ("Hq", _i32), ("Hkv", _i32), ("dk", _i32),
                 ("dv", _i32), ("block_size", _i32), ("num_blocks", _i32), ("scale", ctypes.c_float),
                 ("num_splits", _i32), ("o", _vp), ("lse", _vp), ("o_dtype", _i32), ("workspace", _vp),
-                ("workspace_bytes", ctypes.c_size_t)]
+                ("workspace_bytes", ctypes.c_size_t), ("kv_type", _i32)]
 
 
 class PrefillPagedParams(ctypes.Structure):
@@ -221,7 +221,11 @@ def paged_params(q, k_cache, v_cache, block_table, seq_lens, o, lse, scale, num_
     p.q, p.k_cache, p.v_cache = _ptr(q), _ptr(k_cache), _ptr(v_cache)
     p.block_table, p.seq_lens = _ptr(block_table), _ptr(seq_lens)
     p.max_blocks_per_seq = block_table.shape[1]
-    p.B, p.Hq, p.Hkv, p.dk, p.dv, p.block_size, p.num_blocks = B, Hq, Hkv, dk, v_cache.shape[3], bs, nb
+    dv = v_cache.shape[3]
+    if k_cache.dtype == torch.uint8:  # q8_0 rows: 34 bytes per 32 values
+        p.kv_type = FA_KV_Q8_0
+        dv = v_cache.shape[3] // 34 * 32
+    p.B, p.Hq, p.Hkv, p.dk, p.dv, p.block_size, p.num_blocks = B, Hq, Hkv, dk, dv, bs, nb
     p.scale = scale
     p.num_splits = num_splits
     p.o, p.lse = _ptr(o), _ptr(lse)
@@ -241,14 +245,16 @@ def paged_workspace_bytes(q, k_cache, v_cache, block_table, seq_lens, num_splits
 def decode_paged(q, k_cache, v_cache, block_table, seq_lens, scale=None, num_splits=0, out=None,
                  return_lse=True, out_dtype=torch.float32, workspace=None, stream=None):
     """Split-KV decode over a paged cache.  q [B,Hq,dk]; caches
-    [num_blocks,Hkv,block_size,d]; block_table int32 [B,max_blocks];
+    [num_blocks,Hkv,block_size,d] bf16, or uint8 [...,136] of q8_0 rows
+    (dequantised in the kernel); block_table int32 [B,max_blocks];
     seq_lens int32 [B].  Returns (O [B,Hq,dv], LSE [B,Hq] or None)."""
     _need_cuda(q, k_cache, v_cache, block_table, seq_lens)
     B, Hq, dk = q.shape
     if scale is None:
         scale = 1.0 / math.sqrt(dk)
+    dv = v_cache.shape[3] // 34 * 32 if v_cache.dtype == torch.uint8 else v_cache.shape[3]
     if out is None:
-        out = torch.empty((B, Hq, v_cache.shape[3]), device=q.device, dtype=out_dtype)
+        out = torch.empty((B, Hq, dv), device=q.device, dtype=out_dtype)
     lse = torch.empty((B, Hq), device=q.device, dtype=torch.float32) if return_lse else None
     if workspace is None:
         n = paged_workspace_bytes(q, k_cache, v_cache, block_table, seq_lens, num_splits)

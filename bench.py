@@ -53,6 +53,7 @@ NCU_TRAFFIC = {
     "gqa_full_b1_hq32_hkv8_s4096_d256": 215937536,
     "causal_mha_mods_b2_h16_s2048_d128": 58235904,
     "paged_gqa_b64_hq32_hkv8_d128_bs64": 1237055008,
+    "paged_gqa_q8_0kv_b64_hq32_hkv8_d128_bs64": None,  # the q8_0 kernel changed after its capture
     "latent_sparse_t32_hq128_dk576_dv512_top2048": 45249792,
     "causal_mha_b2_h16_s2048_dk192_dv128": 73713408,
     "causal_gqa_b2_hq16_hkv4_s2048_dk192_dv192": 40004096,
@@ -341,10 +342,14 @@ def mla_tail_workload(torch, fa, W_, c, l2):
     return launch, n, c.bytes, 3
 
 
-def paged_workload(torch, fa, W_, c, l2):
+def paged_workload(torch, fa, W_, c, l2, q8=False):
+    """Paged decode (decode kernel + LSE combine per step); q8: the caches
+    hold q8_0 rows, converted inside the decode kernel."""
     q0, kc0, vc0, tb0, sl0 = W_.paged_inputs(c)
-    byts = W_.paged_bytes(c, sl0, tb0.shape[1])
-    foot = (kc0.numel() + vc0.numel()) * 2
+    if q8:
+        kc0, vc0 = W_.paged_q8_caches(c, kc0.shape[0])
+    byts = W_.paged_bytes(c, sl0, tb0.shape[1], q8=q8)
+    foot = (kc0.numel() + vc0.numel()) * kc0.element_size()
     n = rotation_copies(foot, l2)
     import ctypes
     lib = fa.load()
@@ -485,6 +490,7 @@ def run_only(args):
     table = {c.name: c for c in (W_.TINY_FULL, W_.CAUSAL_MHA, W_.GQA_FULL, W_.MODS_C2, W_.CAUSAL_DK192,
                                  W_.CAUSAL_DK192_DV192, W_.CAUSAL_DK320, W_.PAGED_GQA, W_.LATENT_SPARSE,
                                  W_.QUANT_C2, W_.PAGED_PREFILL, W_.MLA_TAIL)}
+    table[W_.PAGED_Q8_NAME] = W_.PAGED_GQA
     table["kv_dequant_" + W_.QUANT_C2.name] = W_.QUANT_C2
     table[W_.FP8_C2.name] = W_.FP8_C2
     table["kv_dequant_" + W_.FP8_C2.name] = W_.FP8_C2
@@ -506,7 +512,7 @@ def run_only(args):
         launch, n, work, kpl = paged_prefill_workload(torch, fa, W_, c, l2)
         unit, amount = "TFLOP/s", work / 1e12
     elif isinstance(c, W_.PagedCase):
-        launch, n, work, kpl = paged_workload(torch, fa, W_, c, l2)
+        launch, n, work, kpl = paged_workload(torch, fa, W_, c, l2, q8=args.only == W_.PAGED_Q8_NAME)
         unit, amount = "GB/s", work / 1e9
     else:
         launch, n, work, kpl = latent_workload(torch, fa, W_, c, l2)
@@ -724,6 +730,20 @@ def main():
                        "ms_per_step": round(per, 5), "steps": st2, "l2_copies": ncopy, "bytes_per_step": byts,
                        "roofline": roofline("hbm", ach, peaks["hbm_gbs"], "GB/s", NCU_TRAFFIC.get(pc.name)),
                        "kernels": "paged decode + LSE combine"}
+        result["gpu_launches"] += st2 * kpl
+        del launch
+        # the same decode over q8_0 caches (dequant prologue in the kernel)
+        launch, ncopy, byts, kpl = paged_workload(torch, fa, W_, pc, l2, q8=True)
+        ms2, st2 = time_graph(torch, launch, ncopy, Ks, Wm, dist)
+        ms2 = max_over_ranks(torch, dist, ms2)
+        per = ms2 / st2
+        ach = byts / (per * 1e-3) / 1e9
+        wl[W_.PAGED_Q8_NAME] = {"value": round(sum_over_ranks(torch, dist, byts * st2) / (ms2 * 1e-3) / 1e9, 1),
+                                "unit": "GB/s", "ms_per_step": round(per, 5), "steps": st2, "l2_copies": ncopy,
+                                "bytes_per_step": byts,
+                                "roofline": roofline("hbm", ach, peaks["hbm_gbs"], "GB/s",
+                                                     NCU_TRAFFIC.get(W_.PAGED_Q8_NAME)),
+                                "kernels": "paged decode with the q8_0 prologue + LSE combine"}
         result["gpu_launches"] += st2 * kpl
         del launch
         try:

@@ -60,6 +60,9 @@ typedef enum {
 
 typedef enum { FA_F32 = 0, FA_BF16 = 1 } fa_dtype;
 
+/* K/V storage types: bf16, or quantised rows (see fa_kv_dequant). */
+typedef enum { FA_KV_BF16 = 0, FA_KV_Q8_0 = 8, FA_KV_Q4_0 = 4, FA_KV_FP8_E4M3 = 2 } fa_kv_quant;
+
 /* Device-side error codes latched by the kernels (fa_device_error). */
 enum {
     FA_DEVERR_NONE = 0,
@@ -180,7 +183,12 @@ fa_status fa_prefill_paged(const fa_prefill_paged_params *p, void *stream);
  * split along the keys, partial results merged by a log-sum-exp combine.
  *   q: [B, Hq, dk] bf16 contiguous.
  *   k_cache: [num_blocks, Hkv, block_size, dk], v_cache: [num_blocks, Hkv,
- *     block_size, dv], bf16 contiguous.
+ *     block_size, dv], bf16 contiguous (kv_type FA_KV_BF16); or, with
+ *     kv_type FA_KV_Q8_0, rows of dk values stored as dk / 32 ggml q8_0
+ *     blocks (136 bytes for 128 values, layout as in fa_kv_dequant),
+ *     [num_blocks, Hkv, block_size, 136] bytes.  The kernel converts each
+ *     tile in shared memory (the same single rounding to bf16 as
+ *     fa_kv_dequant), so the cache is read once, at 1.06 bytes per value.
  *   block_table: [B, max_blocks_per_seq] int32; key j of sequence b is slot
  *     j % block_size of physical block block_table[b][j / block_size].
  *     Entries past a sequence's last block are never read.
@@ -193,7 +201,8 @@ fa_status fa_prefill_paged(const fa_prefill_paged_params *p, void *stream);
  *     overwritten on every call.
  * Supported: dk == dv == 128, block_size == 64, Hq / Hkv in {1, 2, 4, 8}.
  * Cache slots past seq_lens[b] inside the sequence's last block are read and
- * must hold finite values (their weight is zero, and 0 * NaN is NaN).
+ * must hold finite values (their weight is zero, and 0 * NaN is NaN; for
+ * q8_0 their scales must be finite).
  * A block id outside [0, num_blocks) is latched as FA_DEVERR_BAD_BLOCK and
  * block 0 is read in its place (the output for that sequence is then
  * meaningless).
@@ -212,6 +221,7 @@ typedef struct {
     int o_dtype; /* fa_dtype */
     void *workspace;
     size_t workspace_bytes;
+    int kv_type; /* FA_KV_BF16 (0) or FA_KV_Q8_0 */
 } fa_decode_paged_params;
 
 /* Workspace bytes for these shapes and num_splits; reads no pointer field. */
@@ -348,8 +358,6 @@ fa_status fa_mla_tail(const fa_mla_tail_params *p, void *stream);
  * (0 launches nothing).  src and dst must not overlap.  Non-finite scales
  * decode as IEEE arithmetic gives them (inf * 0 = NaN).
  */
-typedef enum { FA_KV_Q8_0 = 8, FA_KV_Q4_0 = 4, FA_KV_FP8_E4M3 = 2 } fa_kv_quant;
-
 typedef struct {
     const void *src;
     int type; /* fa_kv_quant */

@@ -1,0 +1,65 @@
+"""Paged decode over q8_0 caches (the dequant prologue inside the decode
+kernel) against the oracle: the oracle dequantises the caches (one rounding
+to bf16, as the kernel does) and runs its paged decode on them."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from attention_attn_fwd_11_b200 import fa
+from attention_attn_fwd_11_b200 import workloads as W
+from parity import check
+
+pytestmark = pytest.mark.gpu
+
+
+def run(B, Hq, Hkv, lens, seed, num_splits=0, out_dtype=torch.float32):
+    c = W.PagedCase("t", B, Hq, Hkv, 128, 128, 64, 1, 1, seed=seed, lens=tuple(lens))
+    q, _, _, table, sl = W.paged_inputs(c)
+    nb = max(1, int(sum((n + 63) // 64 for n in lens)))
+    kq, vq = W.paged_q8_caches(c, nb)
+    o, lse = fa.decode_paged(q.cuda(), kq.cuda(), vq.cuda(), table.cuda(), sl.cuda(), scale=c.scale,
+                             num_splits=num_splits, out_dtype=out_dtype)
+    torch.cuda.synchronize()
+    assert fa.device_error() == 0
+    kb = oracle.dequant_rows(kq.numpy(), "q8_0", 128)
+    vb = oracle.dequant_rows(vq.numpy(), "q8_0", 128)
+    o_ref, l_ref = oracle.decode_paged(W.bits(q), kb, vb, table.numpy(), sl.numpy(), c.scale)
+    bf = out_dtype == torch.bfloat16
+    check(o, o_ref, lse, l_ref, max_abs=2e-2 if bf else 1e-2, min_cos=0.9999 if bf else 0.99999,
+          what="q8_0 paged decode lens %s" % (list(lens),))
+
+
+@pytest.mark.parametrize("g", [1, 2, 4, 8])
+def test_group_sizes_ragged_lengths(g):
+    # Hkv 2 KV heads with g query heads each; lengths inside, on and just past block edges
+    run(5, 2 * g, 2, (1, 63, 64, 65, 1000), seed=g)
+
+
+@pytest.mark.parametrize("splits", [1, 3, 7])
+def test_split_counts(splits):
+    run(3, 16, 4, (3000, 129, 64 * 9 + 5), seed=10 + splits, num_splits=splits)
+
+
+def test_bf16_output_and_zero_length():
+    run(4, 8, 8, (0, 200, 1, 4097), seed=20, out_dtype=torch.bfloat16)
+
+
+def test_workload_shape():
+    # the benchmark's decode (B 64, Hq 32, Hkv 8, lengths 1024..8192) over q8_0 caches
+    c = W.PAGED_GQA
+    q, _, _, table, sl = W.paged_inputs(c)
+    kq, vq = W.paged_q8_caches(c, int(table.max()) + 1)
+    o, lse = fa.decode_paged(q.cuda(), kq.cuda(), vq.cuda(), table.cuda(), sl.cuda(), scale=c.scale)
+    torch.cuda.synchronize()
+    assert fa.device_error() == 0
+    # sampled sequences: the oracle decodes rows 0, 31 and 63 on their own
+    for b in (0, 31, 63):
+        n = int(sl[b])
+        nbk = (n + 63) // 64
+        ids = table[b, :nbk].numpy()
+        kb = oracle.dequant_rows(kq[ids].numpy(), "q8_0", 128)
+        vb = oracle.dequant_rows(vq[ids].numpy(), "q8_0", 128)
+        tb1 = np.arange(nbk, dtype=np.int32)[None]
+        o_ref, l_ref = oracle.decode_paged(W.bits(q[b:b + 1]), kb, vb, tb1, np.array([n], np.int32), c.scale)
+        check(o[b:b + 1], o_ref, lse[b:b + 1], l_ref, what="q8_0 workload seq %d" % b)
