@@ -52,8 +52,8 @@ NCU_TRAFFIC = {
     "causal_mha_b2_h16_s2048_d128": 54526208,
     "gqa_full_b1_hq32_hkv8_s4096_d256": 215937536,
     "causal_mha_mods_b2_h16_s2048_d128": 58235904,
-    "paged_gqa_b64_hq32_hkv8_d128_bs64": 1237055008,
-    "paged_gqa_q8_0kv_b64_hq32_hkv8_d128_bs64": None,  # the q8_0 kernel changed after its capture
+    "paged_gqa_b64_hq32_hkv8_d128_bs64": 1236853248,
+    "paged_gqa_q8_0kv_b64_hq32_hkv8_d128_bs64": 660243200,
     "latent_sparse_t32_hq128_dk576_dv512_top2048": 45249792,
     "causal_mha_b2_h16_s2048_dk192_dv128": 73713408,
     "causal_gqa_b2_hq16_hkv4_s2048_dk192_dv192": 40004096,
