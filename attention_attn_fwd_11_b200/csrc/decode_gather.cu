@@ -117,7 +117,12 @@ latent_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const GatherArgs a
     const int nch = rank == 0 ? 5 : 4;        // chunks it owns
     const int vch = rank == 0 ? 1 : 0;        // its first latent (V) chunk, in local chunk numbers
     const int k_begin = split * a.kps;
-    const int k_end = min(a.topk, k_begin + a.kps);
+    int k_end = min(a.topk, k_begin + a.kps);
+    // Contiguous rows (idx == NULL: key j is row j) positioned at their row
+    // index: keys past the token's position are never visible, so its tiles
+    // stop there (a causal prefill in latent space skips its masked half).
+    // Both CTAs of the pair see the same t and split, so they agree.
+    if (!a.idx && !a.key_pos && a.q_pos) k_end = min(k_end, a.q_pos[t] + 1);
     const int n_tiles = k_end > k_begin ? (k_end - k_begin + LG_BN - 1) / LG_BN : 0;
 
     if (threadIdx.x == 0) {
@@ -164,7 +169,7 @@ latent_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const GatherArgs a
                     tma_load_2d(sQ + c * LG_QCH, &tmQ, bar(G_QFULL), (chunk0 + c) * 64, t * LG_H);
             }
             const int qpos = a.q_pos ? a.q_pos[t] : INT_MAX;
-            const int32_t *idx_t = a.idx + (int64_t)t * a.topk;
+            const int32_t *idx_t = a.idx ? a.idx + (int64_t)t * a.topk : nullptr;
             const int32_t *kp_t = a.key_pos ? a.key_pos + (int64_t)t * a.topk : nullptr;
             const int pieces_per_row = nch * 8;
             const int n_pieces = LG_BN * pieces_per_row;  // 1280 or 1024: a multiple of 128
@@ -182,7 +187,7 @@ latent_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const GatherArgs a
                     int r = -1;
                     bool vis = false;
                     if (key < k_end) {
-                        r = idx_t[key];
+                        r = idx_t ? idx_t[key] : key;
                         if (r < -1 || (int64_t)r >= a.n_rows) {
                             atomicCAS(&g_gather_err, 0, 3 /* FA_DEVERR_BAD_ROW */);
                             r = -1;

@@ -221,8 +221,10 @@ fa_status check_gather(const fa_decode_gather_params *p) {
 fa_status check_gather_ptrs(const fa_decode_gather_params *p) {
     fa_status st = check_gather(p);
     if (st != FA_OK || p->T == 0) return st;
-    if (!p->q || !p->kv_rows || !p->o || (p->topk > 0 && !p->idx))
+    if (!p->q || !p->kv_rows || !p->o)
         return fail(FA_ERR_INVALID_ARG, "fa_decode_gather: NULL tensor pointer");
+    if (!p->idx && p->topk > p->n_rows)
+        return fail(FA_ERR_INVALID_ARG, "fa_decode_gather: with idx NULL, topk (%d) must be <= n_rows", p->topk);
     if (!aligned16(p->q) || !aligned16(p->kv_rows) || !aligned16(p->o))
         return fail(FA_ERR_INVALID_ARG, "fa_decode_gather: q, kv_rows and o must be 16-byte aligned");
     if (((uintptr_t)p->lse & 3u) || ((uintptr_t)p->idx & 3u) || ((uintptr_t)p->key_pos & 3u) ||

@@ -311,13 +311,14 @@ def prefill_paged(q, k_cache, v_cache, block_table, seq_lens, scale=None, causal
 
 # ------------------------------------------------------------ gather decode --
 
-def gather_params(q, rows, idx, key_pos, q_pos, o, lse, scale, num_splits, ws, dk=576, dv=512, v_offset=64):
+def gather_params(q, rows, idx, key_pos, q_pos, o, lse, scale, num_splits, ws, dk=576, dv=512, v_offset=64,
+                  topk=None):
     T, Hq, _ = q.shape
     p = GatherParams()
     p.q, p.kv_rows = _ptr(q), _ptr(rows)
     p.n_rows, p.row_stride = rows.shape[0], rows.stride(0)
     p.dk, p.dv, p.v_offset = dk, dv, v_offset
-    p.idx, p.topk = _ptr(idx), idx.shape[1]
+    p.idx, p.topk = _ptr(idx), (idx.shape[1] if idx is not None else int(topk))
     p.key_pos, p.q_pos = _ptr(key_pos), _ptr(q_pos)
     p.T, p.Hq = T, Hq
     p.scale = scale
@@ -329,17 +330,18 @@ def gather_params(q, rows, idx, key_pos, q_pos, o, lse, scale, num_splits, ws, d
     return p
 
 
-def gather_workspace_bytes(q, rows, idx, num_splits=0):
-    p = gather_params(q, rows, idx, None, None, None, None, 1.0, num_splits, None)
+def gather_workspace_bytes(q, rows, idx, num_splits=0, topk=None):
+    p = gather_params(q, rows, idx, None, None, None, None, 1.0, num_splits, None, topk=topk)
     n = ctypes.c_size_t(0)
     _check(load().fa_decode_gather_workspace_size(ctypes.byref(p), ctypes.byref(n)))
     return n.value
 
 
 def decode_gather(q, rows, idx, key_pos=None, q_pos=None, scale=None, num_splits=0, out=None, return_lse=True,
-                  out_dtype=torch.float32, workspace=None, stream=None):
+                  out_dtype=torch.float32, workspace=None, stream=None, topk=None):
     """Latent sparse decode.  q [T,Hq,576]; rows [n_rows, >=576] bf16 (row
-    pitch = rows.stride(0)); idx int32 [T,topk] (-1 = empty); key_pos int32
+    pitch = rows.stride(0)); idx int32 [T,topk] (-1 = empty), or None with
+    ``topk`` given: every token reads rows 0 .. topk - 1; key_pos int32
     [T,topk] or None; q_pos int32 [T] or None.
     Returns (O [T,Hq,512], LSE [T,Hq] or None)."""
     _need_cuda(q, rows, idx, key_pos, q_pos)
@@ -352,11 +354,29 @@ def decode_gather(q, rows, idx, key_pos=None, q_pos=None, scale=None, num_splits
         out = torch.empty((T, Hq, 512), device=q.device, dtype=out_dtype)
     lse = torch.empty((T, Hq), device=q.device, dtype=torch.float32) if return_lse else None
     if workspace is None:
-        n = gather_workspace_bytes(q, rows, idx, num_splits)
+        n = gather_workspace_bytes(q, rows, idx, num_splits, topk=topk)
         workspace = torch.empty(max(n, 256), device=q.device, dtype=torch.uint8)
-    p = gather_params(q, rows, idx, key_pos, q_pos, out, lse, scale, num_splits, workspace)
+    p = gather_params(q, rows, idx, key_pos, q_pos, out, lse, scale, num_splits, workspace, topk=topk)
     _check(load().fa_decode_gather(ctypes.byref(p), _stream(stream)))
     return out, lse
+
+
+def prefill_latent(q, rows, causal=True, scale=None, num_splits=0, out=None, return_lse=True,
+                   out_dtype=torch.float32, workspace=None, stream=None):
+    """Prefill in latent space (MLA with the absorbed query): Sq new tokens,
+    each with Hq = 128 heads, against the Sk latent rows [k_pe | kv_latent]
+    of the sequence, rows 0 .. Sk - 1 of ``rows`` -- the (dk, dv) = (576,
+    512) attention of the llama.cpp tensor path's head-size table, all heads
+    sharing one latent row per key.  q [Sq, 128, 576]; with causal, new
+    token t sits at position Sk - Sq + t.  Runs fa_decode_gather with
+    contiguous rows (idx NULL).  Returns (O [Sq, 128, 512], LSE [Sq, 128])."""
+    _need_cuda(q, rows)
+    Sq, Sk = q.shape[0], rows.shape[0]
+    q_pos = None
+    if causal:
+        q_pos = torch.arange(Sk - Sq, Sk, device=q.device, dtype=torch.int32)
+    return decode_gather(q, rows, None, q_pos=q_pos, scale=scale, num_splits=num_splits, out=out,
+                         return_lse=return_lse, out_dtype=out_dtype, workspace=workspace, stream=stream, topk=Sk)
 
 
 def device_error(clear=True) -> int:

@@ -395,3 +395,36 @@ def mla_tail_inputs(c: MlaTailCase):
 
 
 MLA_TAIL = MlaTailCase("mla_tail_t32_hq128_r512_v128_hidden7168", 32, 128, seed=10)
+
+
+# ------------------------------------------------------ latent prefill --
+# MLA prefill in latent space: Sq new tokens x 128 heads against the Sk
+# latent rows of the sequence (rows [k_pe | kv_latent]), causal.  Q and rows
+# are N(0, 1) bf16 (seeds 1000 + c, 2000 + c); scale 1/sqrt(576).
+
+@dataclass
+class LatentPrefillCase:
+    name: str
+    Sq: int
+    Sk: int
+    Hq: int = 128
+    causal: bool = True
+    seed: int = 0
+
+    @property
+    def flops(self) -> float:
+        """2 * Hq * (576 + 512) per visible (token, key) pair."""
+        if self.causal:
+            pairs = sum(max(0, self.Sk - self.Sq + t + 1) for t in range(self.Sq))
+        else:
+            pairs = self.Sq * self.Sk
+        return 2.0 * self.Hq * (576 + 512) * pairs
+
+
+def latent_prefill_inputs(c: LatentPrefillCase):
+    q = randn_bf16((c.Sq, c.Hq, 576), 1000 + c.seed)
+    rows = randn_bf16((c.Sk, 576), 2000 + c.seed)
+    return q, rows
+
+
+LATENT_PREFILL = LatentPrefillCase("latent_prefill_sq512_sk4096_hq128", 512, 4096, seed=12)

@@ -342,6 +342,34 @@ def mla_tail_workload(torch, fa, W_, c, l2):
     return launch, n, c.bytes, 3
 
 
+def latent_prefill_workload(torch, fa, W_, c, l2):
+    """MLA prefill in latent space: one contiguous-row fa_decode_gather per
+    step (+ its LSE combine)."""
+    import ctypes
+    q0, r0 = W_.latent_prefill_inputs(c)
+    foot = (q0.numel() + r0.numel()) * 2 + c.Sq * c.Hq * (512 * 4 + 4)
+    n = rotation_copies(foot, l2)
+    lib = fa.load()
+    bufs, params = [], []
+    for i in range(n):
+        q, rows = q0.cuda(), r0.cuda()
+        qpos = torch.arange(c.Sk - c.Sq, c.Sk, device="cuda", dtype=torch.int32) if c.causal else None
+        o = torch.empty(c.Sq, c.Hq, 512, device="cuda")
+        lse = torch.empty(c.Sq, c.Hq, device="cuda")
+        ws = torch.empty(max(fa.gather_workspace_bytes(q, rows, None, 0, topk=c.Sk), 256), device="cuda",
+                         dtype=torch.uint8)
+        bufs.append((q, rows, qpos, o, lse, ws))
+        params.append(fa.gather_params(q, rows, None, None, qpos, o, lse, 1.0 / 24, 0, ws, topk=c.Sk))
+
+    def launch(i):
+        st = lib.fa_decode_gather(ctypes.byref(params[i]), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+        if st != 0:
+            raise RuntimeError(lib.fa_last_error().decode())
+
+    launch.keep = bufs
+    return launch, n, c.flops, 2
+
+
 def paged_workload(torch, fa, W_, c, l2, q8=False):
     """Paged decode (decode kernel + LSE combine per step); q8: the caches
     hold q8_0 rows, converted inside the decode kernel."""
@@ -491,6 +519,7 @@ def run_only(args):
                                  W_.CAUSAL_DK192_DV192, W_.CAUSAL_DK320, W_.PAGED_GQA, W_.LATENT_SPARSE,
                                  W_.QUANT_C2, W_.PAGED_PREFILL, W_.MLA_TAIL)}
     table[W_.PAGED_Q8_NAME] = W_.PAGED_GQA
+    table[W_.LATENT_PREFILL.name] = W_.LATENT_PREFILL
     table["kv_dequant_" + W_.QUANT_C2.name] = W_.QUANT_C2
     table[W_.FP8_C2.name] = W_.FP8_C2
     table["kv_dequant_" + W_.FP8_C2.name] = W_.FP8_C2
@@ -505,6 +534,9 @@ def run_only(args):
     elif isinstance(c, W_.PrefillCase):
         launch, n, work, kpl = prefill_workload(torch, fa, W_, c, l2)
         unit, amount = "TFLOP/s", c.flops / 1e12
+    elif isinstance(c, W_.LatentPrefillCase):
+        launch, n, work, kpl = latent_prefill_workload(torch, fa, W_, c, l2)
+        unit, amount = "TFLOP/s", work / 1e12
     elif isinstance(c, W_.MlaTailCase):
         launch, n, work, kpl = mla_tail_workload(torch, fa, W_, c, l2)
         unit, amount = "GB/s", work / 1e9

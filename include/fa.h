@@ -261,7 +261,11 @@ fa_status fa_decode_paged_noalloc(const fa_decode_paged_params *p, void *stream)
  *   kv_rows: n_rows rows of bf16 at a pitch of row_stride elements
  *     (row_stride % 8 == 0); key = row[0 : dk], value = row[v_offset :
  *     v_offset + dv].
- *   idx: [T, topk] int32 flat row indices; -1 marks an empty slot.
+ *   idx: [T, topk] int32 flat row indices; -1 marks an empty slot.  NULL:
+ *     every token reads the contiguous rows 0 .. topk - 1 (topk <= n_rows) --
+ *     a prefill in latent space.  With idx and key_pos NULL and q_pos given,
+ *     a token's keys past q_pos[t] are skipped outright (they are never
+ *     visible), so a causal latent prefill does only its visible half.
  *   key_pos: NULL (a key's position is its row index) or [T, topk] int32.
  *   q_pos: NULL (no causal mask) or [T] int32; slot j is visible to token t
  *     iff idx[t][j] >= 0 and key_pos <= q_pos[t].
