@@ -88,6 +88,7 @@ struct GatherArgs {
     int64_t n_rows, row_stride;
     const int32_t *idx, *key_pos, *q_pos;
     int topk, kps, num_splits;
+    int dk512;  // rows of 512 with V = K (v_offset 0): 256 + 256 columns per pair
     float scale_log2;
     float *part_o, *part_lse;
 };
@@ -113,9 +114,13 @@ latent_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const GatherArgs a
     const uint32_t rank = cluster_ctarank();  // 0 or 1 (blockIdx.x)
     const uint32_t peer = rank ^ 1u;
     const int split = blockIdx.y, t = blockIdx.z;
-    const int chunk0 = rank == 0 ? 0 : 5;     // first 128-byte column chunk of a row this CTA owns
-    const int nch = rank == 0 ? 5 : 4;        // chunks it owns
-    const int vch = rank == 0 ? 1 : 0;        // its first latent (V) chunk, in local chunk numbers
+    // Column split of a row between the pair.  576-wide rows [k_pe | latent]:
+    // CTA 0 owns [0, 320) (k_pe and latent [0, 256)), CTA 1 [320, 576).
+    // 512-wide rows with V = K: CTA r owns [256 r, 256 r + 256).  Either way
+    // each CTA's V half is latent dims [256 r, 256 r + 256).
+    const int chunk0 = a.dk512 ? 4 * (int)rank : (rank == 0 ? 0 : 5);  // first 128-byte chunk it owns
+    const int nch = a.dk512 ? 4 : (rank == 0 ? 5 : 4);                  // chunks it owns
+    const int vch = a.dk512 ? 0 : (rank == 0 ? 1 : 0);                  // its first V chunk, local numbering
     const int k_begin = split * a.kps;
     int k_end = min(a.topk, k_begin + a.kps);
     // Contiguous rows (idx == NULL: key j is row j) positioned at their row
@@ -486,6 +491,7 @@ cudaError_t launch_decode_gather(const GatherLaunch &L, cudaStream_t stream) {
     a.kps = L.keys_per_split;
     a.num_splits = L.num_splits;
     a.scale_log2 = L.scale * 1.4426950408889634f;
+    a.dk512 = L.dk == 512 ? 1 : 0;
     a.part_o = L.part_o;
     a.part_lse = L.part_lse;
     dim3 grid(2u, (unsigned)L.num_splits, (unsigned)L.T);

@@ -208,10 +208,13 @@ fa_status check_gather(const fa_decode_gather_params *p) {
     if (!p) return fail(FA_ERR_INVALID_ARG, "fa_decode_gather: params is NULL");
     if (p->T < 0 || p->Hq <= 0 || p->topk < 0 || p->n_rows <= 0)
         return fail(FA_ERR_INVALID_ARG, "fa_decode_gather: T >= 0, Hq > 0, topk >= 0, n_rows > 0");
-    if (p->dk != 576 || p->dv != 512 || p->v_offset != 64 || p->Hq != 128)
-        return fail(FA_ERR_UNSUPPORTED, "fa_decode_gather: supported dk = 576, dv = 512, v_offset = 64, Hq = 128");
-    if (p->row_stride < 576 || p->row_stride % 8 != 0)
-        return fail(FA_ERR_INVALID_ARG, "fa_decode_gather: row_stride must be >= 576 and a multiple of 8");
+    const bool lat576 = p->dk == 576 && p->dv == 512 && p->v_offset == 64;
+    const bool lat512 = p->dk == 512 && p->dv == 512 && p->v_offset == 0;
+    if (!(lat576 || lat512) || p->Hq != 128)
+        return fail(FA_ERR_UNSUPPORTED,
+                    "fa_decode_gather: supported (dk, dv, v_offset) = (576, 512, 64) or (512, 512, 0), Hq = 128");
+    if (p->row_stride < p->dk || p->row_stride % 8 != 0)
+        return fail(FA_ERR_INVALID_ARG, "fa_decode_gather: row_stride must be >= dk and a multiple of 8");
     if (p->n_rows > 0x7fffffffLL) return fail(FA_ERR_INVALID_ARG, "fa_decode_gather: n_rows must fit in int32");
     if (!finite_pos(p->scale)) return fail(FA_ERR_INVALID_ARG, "fa_decode_gather: scale must be finite and > 0");
     if (p->o_dtype != FA_F32 && p->o_dtype != FA_BF16) return fail(FA_ERR_INVALID_ARG, "fa_decode_gather: o_dtype");
@@ -552,6 +555,7 @@ fa_status fa_decode_gather(const fa_decode_gather_params *p, void *stream) {
     L.topk = p->topk;
     L.T = p->T;
     L.Hq = p->Hq;
+    L.dk = p->dk;
     L.scale = p->scale;
     L.num_splits = splits;
     L.keys_per_split = ((p->topk + splits - 1) / splits + 63) / 64 * 64;

@@ -79,6 +79,7 @@ struct GatherLaunch {
     int64_t n_rows, row_stride;
     const int32_t *idx, *key_pos, *q_pos;
     int topk, T, Hq;
+    int dk;  // 576 (rows [k_pe | latent], V at 64) or 512 (V = K)
     float scale;
     int keys_per_split, num_splits;
     void *o;

@@ -330,15 +330,16 @@ def gather_params(q, rows, idx, key_pos, q_pos, o, lse, scale, num_splits, ws, d
     return p
 
 
-def gather_workspace_bytes(q, rows, idx, num_splits=0, topk=None):
-    p = gather_params(q, rows, idx, None, None, None, None, 1.0, num_splits, None, topk=topk)
+def gather_workspace_bytes(q, rows, idx, num_splits=0, topk=None, dk=576):
+    p = gather_params(q, rows, idx, None, None, None, None, 1.0, num_splits, None, topk=topk, dk=dk,
+                      v_offset=64 if dk == 576 else 0)
     n = ctypes.c_size_t(0)
     _check(load().fa_decode_gather_workspace_size(ctypes.byref(p), ctypes.byref(n)))
     return n.value
 
 
 def decode_gather(q, rows, idx, key_pos=None, q_pos=None, scale=None, num_splits=0, out=None, return_lse=True,
-                  out_dtype=torch.float32, workspace=None, stream=None, topk=None):
+                  out_dtype=torch.float32, workspace=None, stream=None, topk=None, dk=576):
     """Latent sparse decode.  q [T,Hq,576]; rows [n_rows, >=576] bf16 (row
     pitch = rows.stride(0)); idx int32 [T,topk] (-1 = empty), or None with
     ``topk`` given: every token reads rows 0 .. topk - 1; key_pos int32
@@ -354,29 +355,33 @@ def decode_gather(q, rows, idx, key_pos=None, q_pos=None, scale=None, num_splits
         out = torch.empty((T, Hq, 512), device=q.device, dtype=out_dtype)
     lse = torch.empty((T, Hq), device=q.device, dtype=torch.float32) if return_lse else None
     if workspace is None:
-        n = gather_workspace_bytes(q, rows, idx, num_splits, topk=topk)
+        n = gather_workspace_bytes(q, rows, idx, num_splits, topk=topk, dk=dk)
         workspace = torch.empty(max(n, 256), device=q.device, dtype=torch.uint8)
-    p = gather_params(q, rows, idx, key_pos, q_pos, out, lse, scale, num_splits, workspace, topk=topk)
+    p = gather_params(q, rows, idx, key_pos, q_pos, out, lse, scale, num_splits, workspace, topk=topk,
+                      dk=dk, v_offset=64 if dk == 576 else 0)
     _check(load().fa_decode_gather(ctypes.byref(p), _stream(stream)))
     return out, lse
 
 
 def prefill_latent(q, rows, causal=True, scale=None, num_splits=0, out=None, return_lse=True,
-                   out_dtype=torch.float32, workspace=None, stream=None):
+                   out_dtype=torch.float32, workspace=None, stream=None, dk=576):
     """Prefill in latent space (MLA with the absorbed query): Sq new tokens,
     each with Hq = 128 heads, against the Sk latent rows [k_pe | kv_latent]
     of the sequence, rows 0 .. Sk - 1 of ``rows`` -- the (dk, dv) = (576,
     512) attention of the llama.cpp tensor path's head-size table, all heads
     sharing one latent row per key.  q [Sq, 128, 576]; with causal, new
-    token t sits at position Sk - Sq + t.  Runs fa_decode_gather with
-    contiguous rows (idx NULL).  Returns (O [Sq, 128, 512], LSE [Sq, 128])."""
+    token t sits at position Sk - Sq + t.  dk=512: the (512, 512) pair, rows
+    of 512 that are both key and value (q [Sq, 128, 512]).  Runs
+    fa_decode_gather with contiguous rows (idx NULL).
+    Returns (O [Sq, 128, 512], LSE [Sq, 128])."""
     _need_cuda(q, rows)
     Sq, Sk = q.shape[0], rows.shape[0]
     q_pos = None
     if causal:
         q_pos = torch.arange(Sk - Sq, Sk, device=q.device, dtype=torch.int32)
     return decode_gather(q, rows, None, q_pos=q_pos, scale=scale, num_splits=num_splits, out=out,
-                         return_lse=return_lse, out_dtype=out_dtype, workspace=workspace, stream=stream, topk=Sk)
+                         return_lse=return_lse, out_dtype=out_dtype, workspace=workspace, stream=stream, topk=Sk,
+                         dk=dk)
 
 
 def device_error(clear=True) -> int:

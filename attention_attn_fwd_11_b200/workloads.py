@@ -410,21 +410,23 @@ class LatentPrefillCase:
     Hq: int = 128
     causal: bool = True
     seed: int = 0
+    dk: int = 576  # 576: rows [k_pe | latent]; 512: rows that are both key and value
 
     @property
     def flops(self) -> float:
-        """2 * Hq * (576 + 512) per visible (token, key) pair."""
+        """2 * Hq * (dk + 512) per visible (token, key) pair."""
         if self.causal:
             pairs = sum(max(0, self.Sk - self.Sq + t + 1) for t in range(self.Sq))
         else:
             pairs = self.Sq * self.Sk
-        return 2.0 * self.Hq * (576 + 512) * pairs
+        return 2.0 * self.Hq * (self.dk + 512) * pairs
 
 
 def latent_prefill_inputs(c: LatentPrefillCase):
-    q = randn_bf16((c.Sq, c.Hq, 576), 1000 + c.seed)
-    rows = randn_bf16((c.Sk, 576), 2000 + c.seed)
+    q = randn_bf16((c.Sq, c.Hq, c.dk), 1000 + c.seed)
+    rows = randn_bf16((c.Sk, c.dk), 2000 + c.seed)
     return q, rows
 
 
 LATENT_PREFILL = LatentPrefillCase("latent_prefill_sq512_sk4096_hq128", 512, 4096, seed=12)
+LATENT_PREFILL_512 = LatentPrefillCase("latent_prefill_dk512_sq512_sk4096_hq128", 512, 4096, seed=13, dk=512)

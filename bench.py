@@ -356,10 +356,11 @@ def latent_prefill_workload(torch, fa, W_, c, l2):
         qpos = torch.arange(c.Sk - c.Sq, c.Sk, device="cuda", dtype=torch.int32) if c.causal else None
         o = torch.empty(c.Sq, c.Hq, 512, device="cuda")
         lse = torch.empty(c.Sq, c.Hq, device="cuda")
-        ws = torch.empty(max(fa.gather_workspace_bytes(q, rows, None, 0, topk=c.Sk), 256), device="cuda",
+        ws = torch.empty(max(fa.gather_workspace_bytes(q, rows, None, 0, topk=c.Sk, dk=c.dk), 256), device="cuda",
                          dtype=torch.uint8)
         bufs.append((q, rows, qpos, o, lse, ws))
-        params.append(fa.gather_params(q, rows, None, None, qpos, o, lse, 1.0 / 24, 0, ws, topk=c.Sk))
+        params.append(fa.gather_params(q, rows, None, None, qpos, o, lse, 1.0 / math.sqrt(c.dk), 0, ws, topk=c.Sk,
+                                       dk=c.dk, v_offset=64 if c.dk == 576 else 0))
 
     def launch(i):
         st = lib.fa_decode_gather(ctypes.byref(params[i]), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
@@ -520,6 +521,7 @@ def run_only(args):
                                  W_.QUANT_C2, W_.PAGED_PREFILL, W_.MLA_TAIL)}
     table[W_.PAGED_Q8_NAME] = W_.PAGED_GQA
     table[W_.LATENT_PREFILL.name] = W_.LATENT_PREFILL
+    table[W_.LATENT_PREFILL_512.name] = W_.LATENT_PREFILL_512
     table["kv_dequant_" + W_.QUANT_C2.name] = W_.QUANT_C2
     table[W_.FP8_C2.name] = W_.FP8_C2
     table["kv_dequant_" + W_.FP8_C2.name] = W_.FP8_C2

@@ -273,7 +273,9 @@ fa_status fa_decode_paged_noalloc(const fa_decode_paged_params *p, void *stream)
  *   num_splits: 0 = automatic, else the number of key splits per token.
  *   workspace: at least fa_decode_gather_workspace_size() bytes, 256-byte
  *     aligned, overwritten on every call.
- * Supported: dk == 576, dv == 512, v_offset == 64, Hq == 128.
+ * Supported: (dk, dv, v_offset) = (576, 512, 64) -- rows [k_pe | latent] --
+ * or (512, 512, 0) -- rows whose whole 512 columns are both key and value;
+ * Hq == 128.
  * An index >= n_rows or < -1 is latched as FA_DEVERR_BAD_ROW and the slot is
  * treated as empty.
  */

@@ -132,6 +132,15 @@ def test_gather_workspace_size_and_validation():
     assert lib.fa_decode_gather(ctypes.byref(gather_params()), None) == fa.FA_ERR_WORKSPACE
     assert lib.fa_decode_gather(ctypes.byref(gather_params(dk=128)), None) == fa.FA_ERR_UNSUPPORTED
     assert lib.fa_decode_gather(ctypes.byref(gather_params(Hq=64)), None) == fa.FA_ERR_UNSUPPORTED
+    # 512-wide rows that are both key and value: accepted (then the missing workspace is reported)
+    assert lib.fa_decode_gather(ctypes.byref(gather_params(dk=512, dv=512, v_offset=0, row_stride=512)),
+                                None) == fa.FA_ERR_WORKSPACE
+    assert lib.fa_decode_gather(ctypes.byref(gather_params(dk=512, dv=512, v_offset=64)), None) == fa.FA_ERR_UNSUPPORTED
+    assert lib.fa_decode_gather(ctypes.byref(gather_params(dk=512, dv=512, v_offset=0, row_stride=504)),
+                                None) == fa.FA_ERR_INVALID_ARG
+    # idx NULL (contiguous rows): topk must not exceed n_rows
+    assert lib.fa_decode_gather(ctypes.byref(gather_params(idx=0, topk=70000, workspace=256, workspace_bytes=1 << 40)),
+                                None) == fa.FA_ERR_INVALID_ARG
     assert lib.fa_decode_gather(ctypes.byref(gather_params(row_stride=580)), None) == fa.FA_ERR_INVALID_ARG
     assert lib.fa_decode_gather(ctypes.byref(gather_params(idx=50)), None) == fa.FA_ERR_INVALID_ARG
     assert lib.fa_decode_gather(ctypes.byref(gather_params(T=0)), None) == fa.FA_OK

@@ -108,3 +108,20 @@ def test_row_gather_bitexact():
             for t in range(T):
                 ref = rr[want[t], 64:576].float()
                 assert torch.equal(o[t], ref.expand(128, 512)), (trial, splits, t)
+
+
+
+def test_decode_512_rows():
+    # 512-wide rows that are both key and value (v_offset 0), selected rows, causal by row index
+    T, topk, n_rows = 6, 300, 5000
+    q = W.randn_bf16((T, 128, 512), 1301)
+    rows = W.randn_bf16((n_rows, 512), 2301)
+    g = torch.Generator().manual_seed(4301)
+    idx = torch.stack([torch.randperm(n_rows, generator=g)[:topk] for _ in range(T)]).to(torch.int32)
+    idx[1, 17] = -1
+    qpos = torch.randint(0, n_rows, (T,), generator=g).to(torch.int32)
+    o, lse = fa.decode_gather(q.cuda(), rows.cuda(), idx.cuda(), q_pos=qpos.cuda(), scale=1 / 24, dk=512)
+    torch.cuda.synchronize()
+    assert fa.device_error() == 0
+    o_ref, l_ref = oracle.decode_latent(W.bits(q), W.bits(rows), idx.numpy(), 1 / 24, 512, 512, 0, q_pos=qpos.numpy())
+    check(o, o_ref, lse, l_ref, what="gather decode 512 rows")

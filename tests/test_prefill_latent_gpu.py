@@ -13,19 +13,28 @@ from parity import check
 pytestmark = pytest.mark.gpu
 
 
-def run(Sq, Sk, causal, seed, pitch=576, num_splits=0):
+def run(Sq, Sk, causal, seed, pitch=576, num_splits=0, dk=576):
     scale = 1.0 / 24
-    q = W.randn_bf16((Sq, 128, 576), 1000 + seed)
+    q = W.randn_bf16((Sq, 128, dk), 1000 + seed)
     rows_full = W.randn_bf16((Sk, pitch), 2000 + seed)
-    rows = rows_full[:, :576]
-    o, lse = fa.prefill_latent(q.cuda(), rows_full.cuda()[:, :576], causal=causal, scale=scale,
-                               num_splits=num_splits)
+    rows = rows_full[:, :dk]
+    o, lse = fa.prefill_latent(q.cuda(), rows_full.cuda()[:, :dk], causal=causal, scale=scale,
+                               num_splits=num_splits, dk=dk)
     torch.cuda.synchronize()
     assert fa.device_error() == 0
     qd = np.ascontiguousarray(W.bits(q).transpose(1, 0, 2))[None]
     rb = W.bits(rows.contiguous())
-    od, ld = oracle.attention(qd, rb[None, None], np.ascontiguousarray(rb[:, 64:])[None, None], scale, causal)
-    check(o, od[0].transpose(1, 0, 2), lse, ld[0].T, what="latent prefill Sq%d Sk%d causal%d" % (Sq, Sk, causal))
+    vb = np.ascontiguousarray(rb[:, dk - 512:])  # 576: the latent part; 512: the whole row
+    od, ld = oracle.attention(qd, rb[None, None], vb[None, None], scale, causal)
+    check(o, od[0].transpose(1, 0, 2), lse, ld[0].T,
+          what="latent prefill dk%d Sq%d Sk%d causal%d" % (dk, Sq, Sk, causal))
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_512_rows_are_key_and_value(causal):
+    # the (512, 512) pair: rows of 512 serve as both key and value
+    run(80, 300, causal, seed=4, dk=512)
+    run(33, 300, True, seed=5, dk=512, pitch=520, num_splits=2)
 
 
 @pytest.mark.parametrize("causal", [False, True])
