@@ -6,9 +6,18 @@
 One step = one pass of the path over one batch of synthetic input.  The
 headline workload is causal MHA prefill, B=2, H=16, S=2048, d=128 (bf16
 in, fp32 accumulate, fp32 out), reported in TFLOP/s with the causal-halved
-count 4*B*H*S*S*d/2.  The other workloads of this path (tiny full prefill,
-GQA d=256 prefill, paged GQA decode, latent sparse decode) are timed in the
-same run and reported under "workloads".
+count 4*B*H*S*S*d/2.  The other workloads of this path are timed in the
+same run and reported under "workloads":
+- tiny full prefill and GQA d=256 prefill;
+- prefill with every score modifier;
+- the (192,128), (192,192) and (320,256) head-size pairs;
+- prefill over q8_0 K/V (the pre-pass plus prefill);
+- chunked prefill over the paged cache;
+- paged GQA decode, over bf16 and over q8_0 caches;
+- latent sparse decode;
+- the MLA decode tail.
+More workloads run alone with --only NAME (FP8 K/V, the dequant kernels,
+latent prefill).
 
 Timing: inputs already resident in HBM; several copies of every input are
 rotated so that consecutive steps never find their operands in L2; steps are
