@@ -1,12 +1,16 @@
 // prefill.cu -- fused attention forward (prefill) for sm_100a.
 //
-// One CTA computes one 128-row query tile of one (batch, query head):
+// The kernel for the head-size pairs the two-tile kernel (prefill2.cu)
+// cannot hold in TMEM: dv >= 192 or dk != dv -- (256,256), (192,128),
+// (192,192), (320,256).  One CTA computes one 128-row query tile of one
+// (batch, query head):
 //
 //   warp 0      TMA producer: Q tile once, then a ring of K and V tiles
 //               (128-byte swizzled shared memory, zero fill past Sk).
-//   warp 1      MMA issuer (one thread): S = Q K^T with tcgen05.mma into
-//               TMEM (two S buffers, so QK^T of tile t+1 overlaps the
-//               softmax of tile t), then O += P V with P read from TMEM.
+//   warp 1      MMA issuer (the whole warp runs the loop; one elected lane
+//               issues each tcgen05.mma): S = Q K^T into TMEM (two S
+//               buffers, so QK^T of tile t+1 overlaps the softmax of tile
+//               t), then O += P V with P read from TMEM.
 //   warps 2-5   softmax / correction / epilogue, one thread per query row:
 //               S row from TMEM -> scale + mask -> online softmax in base 2
 //               (scale*log2(e) folded into one FMA) -> P as bf16 written back

@@ -5,7 +5,11 @@
 // head); both tiles stream the SAME K/V tiles, so every K/V byte staged in
 // shared memory feeds twice the tensor-core work of the one-tile kernel.
 //
-//   warp 0       TMA producer: Q (both tiles) per unit, then the K and V ring.
+//   warp 0       TMA producer: Q (both tiles) per unit, then the K and V ring
+//                (dense K/V, or -- chunked prefill -- 64-key blocks looked
+//                up in a paged cache's block table).
+//   warps 2, 3   with a score mask: TMA loaders of 64-key mask chunks into
+//                the two softmax groups' staging tiles.
 //   warp 1       MMA issuer.  Per KV tile t:  PV0(t), QK0(t+1), PV1(t),
 //                QK1(t+1).  While softmax warpgroup A works on S0(t+1), the
 //                tensor core runs PV1(t) and QK1(t+1), and vice versa: the
