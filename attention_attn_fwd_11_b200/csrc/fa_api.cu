@@ -390,8 +390,8 @@ fa_status fa_prefill_paged(const fa_prefill_paged_params *p, void *stream) {
         return fail(FA_ERR_INVALID_ARG, "fa_prefill_paged: NULL tensor pointer");
     if (!aligned16(p->q) || !aligned16(p->o) || !aligned16(p->k_cache) || !aligned16(p->v_cache))
         return fail(FA_ERR_INVALID_ARG, "fa_prefill_paged: q, caches and o must be 16-byte aligned");
-    if (((uintptr_t)p->lse | (uintptr_t)p->block_table | (uintptr_t)p->seq_lens) & 3u)
-        return fail(FA_ERR_INVALID_ARG, "fa_prefill_paged: lse, block_table, seq_lens must be 4-byte aligned");
+    if (((uintptr_t)p->lse | (uintptr_t)p->block_table | (uintptr_t)p->seq_lens | (uintptr_t)p->q_lens) & 3u)
+        return fail(FA_ERR_INVALID_ARG, "fa_prefill_paged: lse, block_table, seq_lens, q_lens must be 4-byte aligned");
     const int ovec = p->o_dtype == FA_F32 ? 4 : 8;
     if (p->o_ss % ovec || p->o_sh % ovec || p->o_sb % ovec || p->o_ss < p->dv)
         return fail(FA_ERR_INVALID_ARG, "fa_prefill_paged: o strides must be multiples of %d elements and o_ss >= dv",
@@ -432,6 +432,7 @@ fa_status fa_prefill_paged(const fa_prefill_paged_params *p, void *stream) {
     L.has_mods = false;
     L.block_table = p->block_table;
     L.seq_lens = p->seq_lens;
+    L.q_lens = p->q_lens;
     L.max_blocks = p->max_blocks_per_seq;
     L.num_blocks = p->num_blocks;
     int sms = 0;

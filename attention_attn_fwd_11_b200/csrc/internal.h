@@ -33,6 +33,7 @@ struct PrefillLaunch {
     // are min(seq_lens[b], max_blocks * 64) (Sk is unused).
     const int32_t *block_table;
     const int32_t *seq_lens;
+    const int32_t *q_lens;  // NULL: every sequence has Sq new rows
     int max_blocks, num_blocks;
 };
 // Returns cudaSuccess or the launch error.

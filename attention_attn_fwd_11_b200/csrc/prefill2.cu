@@ -84,6 +84,7 @@ struct Prefill2Args {
     // Paged K/V: block_table [B, max_blocks] and seq_lens [B] (NULL: dense).
     const int32_t *block_table;
     const int32_t *seq_lens;
+    const int32_t *q_lens;  // paged only: new rows per sequence (NULL: all Sq)
     int max_blocks, num_blocks;
 };
 
@@ -92,6 +93,14 @@ FA_DEV int p2_keys(const Prefill2Args &a, int b) {
     if (!a.seq_lens) return a.Sk;
     const int n = __ldg(a.seq_lens + b);
     return n < 0 ? 0 : min(n, a.max_blocks * 64);
+}
+
+// Live query rows of batch entry b: Sq, or its clamped q_lens entry.  Rows
+// past it see no key (O = 0, LSE = -inf).
+FA_DEV int p2_rows(const Prefill2Args &a, int b) {
+    if (!a.q_lens) return a.Sq;
+    const int n = __ldg(a.q_lens + b);
+    return n < 0 ? 0 : min(n, a.Sq);
 }
 
 template <int D>
@@ -167,7 +176,7 @@ constexpr float kP2RescaleThreshold = 8.0f;
 // Plain scalars, never an indexed array, so that a unit's fields stay in
 // registers.
 struct UnitInfo {
-    int b, hq, q0, n0, n1, N, Sk;
+    int b, hq, q0, n0, n1, N, Sk, Sq;
     FA_DEV int nt(int i) const { return i ? n1 : n0; }
 };
 
@@ -181,15 +190,16 @@ FA_DEV bool p2_unit(const Prefill2Args &a, int round, UnitInfo &u) {
     u.hq = bh % a.Hq;
     u.q0 = qp * 256;
     u.Sk = p2_keys(a, u.b);
+    u.Sq = p2_rows(a, u.b);
     int n[2];
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
         const int r0 = u.q0 + 128 * i;
         n[i] = 0;
-        if (r0 < a.Sq) {
-            const int last = min(r0 + 127, a.Sq - 1);
+        if (r0 < u.Sq) {
+            const int last = min(r0 + 127, u.Sq - 1);
             int kmax = u.Sk - 1;
-            if (a.causal) kmax = min(kmax, last + u.Sk - a.Sq);
+            if (a.causal) kmax = min(kmax, last + u.Sk - u.Sq);
             n[i] = kmax < 0 ? 0 : kmax / 128 + 1;
         }
     }
@@ -591,7 +601,8 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             if (!mbar_wait(bar(P2_USTART + ti), (uint32_t)uc & 1u, abort_flag, &g_prefill2_err)) break;
             const int n = u.nt(ti);
             const int qrow = u.q0 + 128 * ti + row;
-            const int lim_all = a.causal ? min(u.Sk, qrow + u.Sk - a.Sq + 1) : u.Sk;
+            const int lim_all =
+                qrow >= u.Sq ? 0 : (a.causal ? min(u.Sk, qrow + u.Sk - u.Sq + 1) : u.Sk);
             const float slope = MODS ? alibi_slope(a.mods, u.hq) : 1.f;
             const __half *mrow = MODS ? mask_row(a.mods, u.b, u.hq, qrow, a.Sq) : nullptr;
             (void)slope;
@@ -921,6 +932,7 @@ static cudaError_t launch_p2(const PrefillLaunch &L, int num_sms, cudaStream_t s
     a.mask_staged = MODS && L.mask_staged ? 1 : 0;
     a.block_table = L.block_table;
     a.seq_lens = L.seq_lens;
+    a.q_lens = L.q_lens;
     a.max_blocks = L.max_blocks;
     a.num_blocks = L.num_blocks;
 #if defined(FA_P2_SETMAXNREG) && FA_P2_THREADS == 384

@@ -50,7 +50,7 @@ class PrefillPagedParams(ctypes.Structure):
                 ("block_table", _vp), ("seq_lens", _vp), ("max_blocks_per_seq", _i32), ("B", _i32), ("Hq", _i32),
                 ("Hkv", _i32), ("Sq", _i32), ("dk", _i32), ("dv", _i32), ("block_size", _i32), ("num_blocks", _i32),
                 ("scale", ctypes.c_float), ("causal", _i32), ("o", _vp), ("o_sb", _i64), ("o_sh", _i64),
-                ("o_ss", _i64), ("lse", _vp), ("o_dtype", _i32)]
+                ("o_ss", _i64), ("lse", _vp), ("o_dtype", _i32), ("q_lens", _vp)]
 
 
 class GatherParams(ctypes.Structure):
@@ -266,7 +266,7 @@ def decode_paged(q, k_cache, v_cache, block_table, seq_lens, scale=None, num_spl
 
 # ----------------------------------------------------------- paged prefill --
 
-def prefill_paged_params(q, k_cache, v_cache, block_table, seq_lens, o, lse, scale, causal):
+def prefill_paged_params(q, k_cache, v_cache, block_table, seq_lens, o, lse, scale, causal, q_lens=None):
     B, Hq, Sq, dk = q.shape
     nb, Hkv, bs, _ = k_cache.shape
     p = PrefillPagedParams()
@@ -280,17 +280,21 @@ def prefill_paged_params(q, k_cache, v_cache, block_table, seq_lens, o, lse, sca
     p.o, p.o_sb, p.o_sh, p.o_ss = _ptr(o), o.stride(0), o.stride(1), o.stride(2)
     p.lse = _ptr(lse)
     p.o_dtype = _odt(o.dtype)
+    p.q_lens = _ptr(q_lens)
     return p
 
 
 def prefill_paged(q, k_cache, v_cache, block_table, seq_lens, scale=None, causal=True, out=None,
-                  return_lse=True, out_dtype=torch.float32, stream=None):
+                  return_lse=True, out_dtype=torch.float32, stream=None, q_lens=None):
     """Chunked prefill over a paged cache (fa_prefill_paged).  q [B,Hq,Sq,d]
     bf16 (head dim contiguous); caches [num_blocks,Hkv,64,d] bf16
     contiguous; block_table int32 [B,max_blocks]; seq_lens int32 [B] (keys
-    including the Sq new ones).  Returns (O [B,Hq,Sq,d], LSE [B,Hq,Sq] or
-    None)."""
-    _need_cuda(q, k_cache, v_cache, block_table, seq_lens, out)
+    including the new ones); q_lens: None or int32 [B], new rows per
+    sequence (rows past it come back as O = 0, LSE = -inf).
+    Returns (O [B,Hq,Sq,d], LSE [B,Hq,Sq] or None)."""
+    _need_cuda(q, k_cache, v_cache, block_table, seq_lens, out, q_lens)
+    if q_lens is not None and (q_lens.dtype != torch.int32 or not q_lens.is_contiguous()):
+        raise ValueError("q_lens must be contiguous int32")
     for t in (q, k_cache, v_cache):
         if t.dtype != torch.bfloat16 or t.stride(-1) != 1:
             raise ValueError("q and the caches must be bf16 with a contiguous head dimension")
@@ -304,7 +308,7 @@ def prefill_paged(q, k_cache, v_cache, block_table, seq_lens, scale=None, causal
     if out is None:
         out = torch.empty((B, Hq, Sq, v_cache.shape[3]), device=q.device, dtype=out_dtype)
     lse = torch.empty((B, Hq, Sq), device=q.device, dtype=torch.float32) if return_lse else None
-    p = prefill_paged_params(q, k_cache, v_cache, block_table, seq_lens, out, lse, scale, causal)
+    p = prefill_paged_params(q, k_cache, v_cache, block_table, seq_lens, out, lse, scale, causal, q_lens)
     _check(load().fa_prefill_paged(ctypes.byref(p), _stream(stream)))
     return out, lse
 

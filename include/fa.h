@@ -145,9 +145,13 @@ fa_status fa_fwd(const fa_fwd_params *p, void *stream);
  *   seq_lens: [B] int32, the keys of each sequence INCLUDING its Sq new
  *     tokens (the caller writes their K/V into the cache first); values are
  *     clamped to [0, max_blocks_per_seq * block_size].
- *   causal != 0: query i of sequence b sits at position seq_lens[b] - Sq + i
- *     and sees keys j <= that position (bottom-right, as in fa_fwd); a row
- *     with no visible key (seq_lens[b] < Sq) gets O = 0, LSE = -inf.
+ *   q_lens: NULL (every sequence has Sq new rows) or [B] int32: sequence b
+ *     has q_lens[b] new rows (clamped to [0, Sq]), rows 0 .. q_lens[b] - 1
+ *     of its Q and O; its rows past that are written as O = 0, LSE = -inf.
+ *   causal != 0: new row i of sequence b sits at position seq_lens[b] -
+ *     n_b + i (n_b = q_lens[b], or Sq) and sees keys j <= that position
+ *     (bottom-right, as in fa_fwd); a row with no visible key gets O = 0,
+ *     LSE = -inf.
  *   o: [B, Hq, Sq, dv] (o_dtype) with strides o_sb, o_sh, o_ss (multiples of
  *     4 elements for fp32, 8 for bf16; o_ss >= dv); lse: NULL or [B, Hq, Sq]
  *     fp32 contiguous.
@@ -174,6 +178,7 @@ typedef struct {
     int64_t o_sb, o_sh, o_ss;
     float *lse;
     int o_dtype; /* fa_dtype */
+    const int32_t *q_lens;
 } fa_prefill_paged_params;
 
 fa_status fa_prefill_paged(const fa_prefill_paged_params *p, void *stream);

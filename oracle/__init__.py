@@ -196,12 +196,14 @@ def decode_paged(q, k_cache, v_cache, block_table, seq_lens, scale):
     return o, lse
 
 
-def prefill_paged(q, k_cache, v_cache, block_table, seq_lens, scale, causal=True):
+def prefill_paged(q, k_cache, v_cache, block_table, seq_lens, scale, causal=True, q_lens=None):
     """Chunked prefill over a paged cache: per sequence b, its keys are
     gathered from the cache (paged_gather) and the dense oracle runs on
     them.  q [B,Hq,Sq,dk]; caches [num_blocks,Hkv,block_size,d]; seq_lens
-    counts the Sq new keys too.  Returns (O [B,Hq,Sq,dv], LSE [B,Hq,Sq])
-    float64."""
+    counts the new keys too.  q_lens: None, or the new rows per sequence
+    (clamped to [0, Sq]); only rows 0 .. q_lens[b] - 1 of sequence b are
+    queries, the rest come back as O = 0, LSE = -inf.
+    Returns (O [B,Hq,Sq,dv], LSE [B,Hq,Sq]) float64."""
     q = _u16(q)
     bs = k_cache.shape[2]
     sl = np.ascontiguousarray(seq_lens, dtype=np.int32)
@@ -209,10 +211,14 @@ def prefill_paged(q, k_cache, v_cache, block_table, seq_lens, scale, causal=True
     vv = paged_gather(v_cache, block_table, sl, bs)
     B, Hq, Sq, _ = q.shape
     o = np.zeros((B, Hq, Sq, vv.shape[3]), np.float64)
-    lse = np.zeros((B, Hq, Sq), np.float64)
+    lse = np.full((B, Hq, Sq), -np.inf, np.float64)
     for b in range(B):
         n = int(sl[b])
-        o[b:b + 1], lse[b:b + 1] = attention(q[b:b + 1], kk[b:b + 1, :, :n], vv[b:b + 1, :, :n], scale, causal)
+        nq = Sq if q_lens is None else min(max(int(q_lens[b]), 0), Sq)
+        if nq == 0:
+            continue
+        o[b:b + 1, :, :nq], lse[b:b + 1, :, :nq] = attention(q[b:b + 1, :, :nq], kk[b:b + 1, :, :n],
+                                                             vv[b:b + 1, :, :n], scale, causal)
     return o, lse
 
 

@@ -66,3 +66,22 @@ def test_rows_before_the_first_key_are_empty():
     vv = oracle.paged_gather(vc, table, sl, 64)
     v0 = torch.from_numpy(vv[0, 0, 0].view(np.int16)).view(torch.bfloat16).double().numpy()
     assert np.array_equal(o[0, 0, 8], v0)
+
+
+
+def test_per_sequence_new_rows():
+    # q_lens: sequence b's first q_lens[b] rows are its new tokens, the last
+    # at position seq_len - 1 -- so its row q_lens[b] - 1 is the decode of
+    # that sequence (the oracle's separate paged-decode function); rows past
+    # q_lens[b] are empty.
+    c, q, kc, vc, table, sl = case(3, 4, 2, 12, 64, (90, 5, 300), seed=7)
+    ql = np.array([12, 3, 7], np.int32)
+    o, lse = oracle.prefill_paged(q, kc, vc, table, sl, c.scale, causal=True, q_lens=ql)
+    for b in range(3):
+        n = int(ql[b])
+        od, ld = oracle.decode_paged(q[b:b + 1, :, n - 1], kc, vc, table[b:b + 1], sl[b:b + 1], c.scale)
+        assert np.allclose(o[b, :, n - 1], od[0], rtol=0, atol=1e-13)
+        assert np.allclose(lse[b, :, n - 1], ld[0], rtol=0, atol=1e-13)
+        assert np.all(o[b, :, n:] == 0) and np.all(lse[b, :, n:] == -np.inf)
+    full, _ = oracle.prefill_paged(q, kc, vc, table, sl, c.scale, causal=True)
+    assert np.array_equal(o[0], full[0])  # q_lens[0] == Sq: the uniform case

@@ -13,18 +13,19 @@ from parity import check
 pytestmark = pytest.mark.gpu
 
 
-def run(B, Hq, Hkv, Sq, d, lens, causal, seed, out_dtype=torch.float32, seq_major=False):
+def run(B, Hq, Hkv, Sq, d, lens, causal, seed, out_dtype=torch.float32, seq_major=False, q_lens=None):
     c = W.PagedPrefillCase("t", B, Hq, Hkv, Sq, d, 0, 0, causal=causal, seed=seed, lens=tuple(lens))
     q, kc, vc, table, sl = W.paged_prefill_inputs(c)
     qd = q.cuda()
     if seq_major:  # Q stored [B, Sq, Hq, d], viewed as [B, Hq, Sq, d]
         qd = q.permute(0, 2, 1, 3).contiguous().cuda().permute(0, 2, 1, 3)
+    qlt = None if q_lens is None else torch.tensor(q_lens, dtype=torch.int32).cuda()
     o, lse = fa.prefill_paged(qd, kc.cuda(), vc.cuda(), table.cuda(), sl.cuda(), scale=c.scale, causal=causal,
-                              out_dtype=out_dtype)
+                              out_dtype=out_dtype, q_lens=qlt)
     torch.cuda.synchronize()
     assert fa.device_error() == 0
     o_ref, l_ref = oracle.prefill_paged(W.bits(q), W.bits(kc), W.bits(vc), table.numpy(), sl.numpy(), c.scale,
-                                        causal)
+                                        causal, q_lens=q_lens)
     bf = out_dtype == torch.bfloat16
     check(o, o_ref, lse, l_ref, max_abs=2e-2 if bf else 1e-2, min_cos=0.9999 if bf else 0.99999,
           what="paged prefill d%d Sq%d lens %s causal %d" % (d, Sq, list(lens), causal))
@@ -82,3 +83,11 @@ def test_workload_sampled_rows():
                                                 np.array([Lb], np.int32), c.scale, True)
             check(o[b:b + 1, :, r0:r0 + n], o_ref, lse[b:b + 1, :, r0:r0 + n], l_ref,
                   what="paged prefill workload b%d rows %d.." % (b, r0))
+
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+def test_per_sequence_new_rows(d, causal):
+    # ragged chunks: 300 rows padded, 300 / 1 / 129 / 0 / 256 of them live
+    run(5, 8, 2, 300, d, (300, 517, 1088, 333, 700), causal, seed=40 + d, q_lens=(300, 1, 129, 0, 256))
