@@ -429,7 +429,35 @@ fa_status fa_prefill_paged(const fa_prefill_paged_params *p, void *stream) {
     L.o_ss = p->o_ss;
     L.o_bf16 = p->o_dtype == FA_BF16;
     L.lse = p->lse;
-    L.has_mods = false;
+    if (!isfinite(p->max_bias) || p->max_bias < 0.f || !isfinite(p->softcap) || p->softcap < 0.f)
+        return fail(FA_ERR_INVALID_ARG, "fa_prefill_paged: max_bias and softcap must be finite and >= 0");
+    if (p->mask && (!aligned16(p->mask) || p->m_ss % 8 || p->m_sh % 8 || p->m_sb % 8 || p->m_ss <= 0 ||
+                    p->m_sh < 0 || p->m_sb < 0))
+        return fail(FA_ERR_INVALID_ARG,
+                    "fa_prefill_paged: mask must be 16-byte aligned, its strides multiples of 8 elements, m_ss > 0");
+    if ((uintptr_t)p->sinks & 3u) return fail(FA_ERR_INVALID_ARG, "fa_prefill_paged: sinks must be 4-byte aligned");
+    L.mods.mask = static_cast<const __half *>(p->mask);
+    L.mods.m_sb = p->m_sb;
+    L.mods.m_sh = p->m_sh;
+    L.mods.m_ss = p->m_ss;
+    L.mods.softcap = p->softcap;
+    L.mods.sinks = p->sinks;
+    if (p->max_bias > 0.f) {  // ALiBi bases, as read in score_mods.cuh
+        int n2 = 1;
+        while (n2 * 2 <= p->Hq) n2 *= 2;
+        L.mods.n_head_log2 = n2;
+        L.mods.log2_m0 = -p->max_bias / (float)n2;
+        L.mods.log2_m1 = -p->max_bias / 2.f / (float)n2;
+    }
+    L.has_mods = p->mask || p->softcap > 0.f || p->sinks;
+    if (p->mask) {
+        // (keys, new rows, heads, batch) with rows m_ss long; stride-0 dims broadcast
+        st = encode_4d(&L.tmM, p->mask, (int)(p->m_ss < (1 << 30) ? p->m_ss : (1 << 30)), p->Sq,
+                       p->m_sh ? p->Hq : 1, p->m_sb ? p->B : 1, p->m_ss, p->m_sh ? p->m_sh : p->m_ss * p->Sq,
+                       p->m_sb ? p->m_sb : p->m_ss * p->Sq, 128, "fa_prefill_paged mask");
+        if (st != FA_OK) return st;
+        L.mask_staged = true;
+    }
     L.block_table = p->block_table;
     L.seq_lens = p->seq_lens;
     L.q_lens = p->q_lens;

@@ -845,6 +845,7 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 inv_l = l_o > 0.f ? 1.f / l_o : 0.f;
                 if (a.mods.sinks) inv_l = sink_normalise(m_run, l_run, l_o, a.mods.sinks[u.hq], &lse2);
             }
+            if (qrow >= u.Sq) lse2 = -INFINITY;  // past the sequence's new rows: not a query (sinks aside)
             if (qrow < a.Sq && a.lse)
                 a.lse[((int64_t)u.b * a.Hq + u.hq) * a.Sq + qrow] = lse2 * 0.69314718055994530942f;
             // Rows are written through a 16 KB staging tile (128 rows x 128

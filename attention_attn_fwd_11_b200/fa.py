@@ -50,7 +50,9 @@ class PrefillPagedParams(ctypes.Structure):
                 ("block_table", _vp), ("seq_lens", _vp), ("max_blocks_per_seq", _i32), ("B", _i32), ("Hq", _i32),
                 ("Hkv", _i32), ("Sq", _i32), ("dk", _i32), ("dv", _i32), ("block_size", _i32), ("num_blocks", _i32),
                 ("scale", ctypes.c_float), ("causal", _i32), ("o", _vp), ("o_sb", _i64), ("o_sh", _i64),
-                ("o_ss", _i64), ("lse", _vp), ("o_dtype", _i32), ("q_lens", _vp)]
+                ("o_ss", _i64), ("lse", _vp), ("o_dtype", _i32), ("q_lens", _vp), ("mask", _vp),
+                ("m_sb", _i64), ("m_sh", _i64), ("m_ss", _i64), ("max_bias", ctypes.c_float),
+                ("softcap", ctypes.c_float), ("sinks", _vp)]
 
 
 class GatherParams(ctypes.Structure):
@@ -266,7 +268,8 @@ def decode_paged(q, k_cache, v_cache, block_table, seq_lens, scale=None, num_spl
 
 # ----------------------------------------------------------- paged prefill --
 
-def prefill_paged_params(q, k_cache, v_cache, block_table, seq_lens, o, lse, scale, causal, q_lens=None):
+def prefill_paged_params(q, k_cache, v_cache, block_table, seq_lens, o, lse, scale, causal, q_lens=None,
+                         mask=None, max_bias=0.0, softcap=0.0, sinks=None):
     B, Hq, Sq, dk = q.shape
     nb, Hkv, bs, _ = k_cache.shape
     p = PrefillPagedParams()
@@ -281,17 +284,31 @@ def prefill_paged_params(q, k_cache, v_cache, block_table, seq_lens, o, lse, sca
     p.lse = _ptr(lse)
     p.o_dtype = _odt(o.dtype)
     p.q_lens = _ptr(q_lens)
+    if mask is not None:
+        p.mask = _ptr(mask)
+        p.m_sb = mask.stride(0) if mask.shape[0] > 1 else 0
+        p.m_sh = mask.stride(1) if mask.shape[1] > 1 else 0
+        p.m_ss = mask.stride(2)
+    p.max_bias, p.softcap, p.sinks = max_bias, softcap, _ptr(sinks)
     return p
 
 
 def prefill_paged(q, k_cache, v_cache, block_table, seq_lens, scale=None, causal=True, out=None,
-                  return_lse=True, out_dtype=torch.float32, stream=None, q_lens=None):
+                  return_lse=True, out_dtype=torch.float32, stream=None, q_lens=None, mask=None, max_bias=0.0,
+                  softcap=0.0, sinks=None):
     """Chunked prefill over a paged cache (fa_prefill_paged).  q [B,Hq,Sq,d]
     bf16 (head dim contiguous); caches [num_blocks,Hkv,64,d] bf16
     contiguous; block_table int32 [B,max_blocks]; seq_lens int32 [B] (keys
     including the new ones); q_lens: None or int32 [B], new rows per
-    sequence (rows past it come back as O = 0, LSE = -inf).
+    sequence (rows past it come back as O = 0, LSE = -inf); mask [1|B, 1|Hq,
+    Sq, >= max seq_len] float16 (last dim contiguous), max_bias, softcap,
+    sinks [Hq] float32: the score modifiers of fwd().
     Returns (O [B,Hq,Sq,d], LSE [B,Hq,Sq] or None)."""
+    _need_cuda(mask, sinks)
+    if mask is not None and (mask.dtype != torch.float16 or mask.dim() != 4 or mask.stride(3) != 1):
+        raise ValueError("mask must be a 4-D float16 tensor with a contiguous last dim")
+    if sinks is not None and (sinks.dtype != torch.float32 or not sinks.is_contiguous()):
+        raise ValueError("sinks must be contiguous float32 [Hq]")
     _need_cuda(q, k_cache, v_cache, block_table, seq_lens, out, q_lens)
     if q_lens is not None and (q_lens.dtype != torch.int32 or not q_lens.is_contiguous()):
         raise ValueError("q_lens must be contiguous int32")
@@ -308,7 +325,8 @@ def prefill_paged(q, k_cache, v_cache, block_table, seq_lens, scale=None, causal
     if out is None:
         out = torch.empty((B, Hq, Sq, v_cache.shape[3]), device=q.device, dtype=out_dtype)
     lse = torch.empty((B, Hq, Sq), device=q.device, dtype=torch.float32) if return_lse else None
-    p = prefill_paged_params(q, k_cache, v_cache, block_table, seq_lens, out, lse, scale, causal, q_lens)
+    p = prefill_paged_params(q, k_cache, v_cache, block_table, seq_lens, out, lse, scale, causal, q_lens, mask,
+                             max_bias, softcap, sinks)
     _check(load().fa_prefill_paged(ctypes.byref(p), _stream(stream)))
     return out, lse
 

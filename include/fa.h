@@ -155,8 +155,11 @@ fa_status fa_fwd(const fa_fwd_params *p, void *stream);
  *   o: [B, Hq, Sq, dv] (o_dtype) with strides o_sb, o_sh, o_ss (multiples of
  *     4 elements for fp32, 8 for bf16; o_ss >= dv); lse: NULL or [B, Hq, Sq]
  *     fp32 contiguous.
- * Supported: dk == dv in {64, 128}, block_size == 64, Hq % Hkv == 0.  No
- * score modifiers on this path.
+ * Supported: dk == dv in {64, 128}, block_size == 64, Hq % Hkv == 0.
+ * Score modifiers: as in fa_fwd (mask, max_bias, softcap, sinks), with the
+ *   mask element (b, h, i, j) at b*m_sb + h*m_sh + i*m_ss + j for new row i
+ *   and key j of the sequence (j < seq_lens[b]); m_ss must be >= every
+ *   seq_lens[b] (keys at or past m_ss read as 0).
  * Cache slots past seq_lens[b] inside the sequence's last block are read and
  * must hold finite values (their weight is zero, and 0 * NaN is NaN).
  * Entries past a sequence's last block are never read.  A block id outside
@@ -179,6 +182,12 @@ typedef struct {
     float *lse;
     int o_dtype; /* fa_dtype */
     const int32_t *q_lens;
+    /* score modifiers (zero / NULL: off), as in fa_fwd */
+    const void *mask; /* f16 */
+    int64_t m_sb, m_sh, m_ss;
+    float max_bias;
+    float softcap;
+    const float *sinks;
 } fa_prefill_paged_params;
 
 fa_status fa_prefill_paged(const fa_prefill_paged_params *p, void *stream);

@@ -196,13 +196,17 @@ def decode_paged(q, k_cache, v_cache, block_table, seq_lens, scale):
     return o, lse
 
 
-def prefill_paged(q, k_cache, v_cache, block_table, seq_lens, scale, causal=True, q_lens=None):
+def prefill_paged(q, k_cache, v_cache, block_table, seq_lens, scale, causal=True, q_lens=None, mask=None,
+                  max_bias=0.0, softcap=0.0, sinks=None):
     """Chunked prefill over a paged cache: per sequence b, its keys are
     gathered from the cache (paged_gather) and the dense oracle runs on
     them.  q [B,Hq,Sq,dk]; caches [num_blocks,Hkv,block_size,d]; seq_lens
     counts the new keys too.  q_lens: None, or the new rows per sequence
     (clamped to [0, Sq]); only rows 0 .. q_lens[b] - 1 of sequence b are
-    queries, the rest come back as O = 0, LSE = -inf.
+    queries, the rest come back as O = 0, LSE = -inf.  mask [1|B, 1|Hq,
+    Sq, >= max seq_len] (f16), max_bias, softcap, sinks: the score
+    modifiers of attention_ext, applied per sequence with key j of the
+    sequence at mask column j.
     Returns (O [B,Hq,Sq,dv], LSE [B,Hq,Sq]) float64."""
     q = _u16(q)
     bs = k_cache.shape[2]
@@ -217,8 +221,14 @@ def prefill_paged(q, k_cache, v_cache, block_table, seq_lens, scale, causal=True
         nq = Sq if q_lens is None else min(max(int(q_lens[b]), 0), Sq)
         if nq == 0:
             continue
-        o[b:b + 1, :, :nq], lse[b:b + 1, :, :nq] = attention(q[b:b + 1, :, :nq], kk[b:b + 1, :, :n],
-                                                             vv[b:b + 1, :, :n], scale, causal)
+        if mask is None and not max_bias and not softcap and sinks is None:
+            o[b:b + 1, :, :nq], lse[b:b + 1, :, :nq] = attention(q[b:b + 1, :, :nq], kk[b:b + 1, :, :n],
+                                                                 vv[b:b + 1, :, :n], scale, causal)
+        else:
+            mb = None if mask is None else np.ascontiguousarray(mask[b % mask.shape[0]:b % mask.shape[0] + 1, :, :nq, :n])
+            o[b:b + 1, :, :nq], lse[b:b + 1, :, :nq] = attention_ext(
+                q[b:b + 1, :, :nq], kk[b:b + 1, :, :n], vv[b:b + 1, :, :n], scale, causal, mask=mb,
+                max_bias=max_bias, softcap=softcap, sinks=sinks)
     return o, lse
 
 

@@ -85,3 +85,28 @@ def test_per_sequence_new_rows():
         assert np.all(o[b, :, n:] == 0) and np.all(lse[b, :, n:] == -np.inf)
     full, _ = oracle.prefill_paged(q, kc, vc, table, sl, c.scale, causal=True)
     assert np.array_equal(o[0], full[0])  # q_lens[0] == Sq: the uniform case
+
+
+
+def test_modifiers_with_identity_table_equal_dense():
+    # identity block table over a contiguous cache: the paged prefill with
+    # every modifier equals the dense attention_ext on the same keys
+    B, Hkv, Hq, Sq, d, L = 2, 1, 4, 20, 64, 100
+    nb = (L + 63) // 64
+    k = W.bits(W.randn_bf16((B, Hkv, nb * 64, d), 21))
+    v = W.bits(W.randn_bf16((B, Hkv, nb * 64, d), 22))
+    q = W.bits(W.randn_bf16((B, Hq, Sq, d), 23))
+    kc = k.reshape(B, Hkv, nb, 64, d).transpose(0, 2, 1, 3, 4).reshape(B * nb, Hkv, 64, d).copy()
+    vc = v.reshape(B, Hkv, nb, 64, d).transpose(0, 2, 1, 3, 4).reshape(B * nb, Hkv, 64, d).copy()
+    table = np.arange(B * nb, dtype=np.int32).reshape(B, nb)
+    sl = np.array([L, L - 30], np.int32)
+    mask = W.random_mask(B, 1, Sq, nb * 64, seed=24, scale=1.0).numpy()
+    sinks = W.random_sinks(Hq, seed=25).double().numpy()
+    kw = dict(mask=mask, max_bias=4.0, softcap=5.0, sinks=sinks)
+    o, lse = oracle.prefill_paged(q, kc, vc, table, sl, 0.125, True, **kw)
+    for b in range(B):
+        n = int(sl[b])
+        od, ld = oracle.attention_ext(q[b:b + 1], k[b:b + 1, :, :n], v[b:b + 1, :, :n], 0.125, True,
+                                      mask=np.ascontiguousarray(mask[b:b + 1, :, :, :n]), max_bias=4.0, softcap=5.0,
+                                      sinks=sinks)
+        assert np.array_equal(o[b:b + 1], od) and np.array_equal(lse[b:b + 1], ld)

@@ -91,3 +91,22 @@ def test_workload_sampled_rows():
 def test_per_sequence_new_rows(d, causal):
     # ragged chunks: 300 rows padded, 300 / 1 / 129 / 0 / 256 of them live
     run(5, 8, 2, 300, d, (300, 517, 1088, 333, 700), causal, seed=40 + d, q_lens=(300, 1, 129, 0, 256))
+
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_score_modifiers(d):
+    # every modifier (head-shared mask with ALiBi, softcap, sinks) with ragged chunks
+    c = W.PagedPrefillCase("t", 3, 8, 2, 130, d, 0, 0, causal=True, seed=60 + d, lens=(130, 517, 300))
+    q, kc, vc, table, sl = W.paged_prefill_inputs(c)
+    ql = torch.tensor([130, 77, 1], dtype=torch.int32)
+    mask = W.random_mask(3, 1, 130, 520, seed=61, scale=1.0)  # rows 520 >= every seq_len, a multiple of 8
+    sinks = W.random_sinks(8, seed=62)
+    o, lse = fa.prefill_paged(q.cuda(), kc.cuda(), vc.cuda(), table.cuda(), sl.cuda(), scale=c.scale, causal=True,
+                              q_lens=ql.cuda(), mask=mask.cuda(), max_bias=4.0, softcap=6.0, sinks=sinks.cuda())
+    torch.cuda.synchronize()
+    assert fa.device_error() == 0
+    o_ref, l_ref = oracle.prefill_paged(W.bits(q), W.bits(kc), W.bits(vc), table.numpy(), sl.numpy(), c.scale, True,
+                                        q_lens=ql.numpy(), mask=mask.numpy(), max_bias=4.0, softcap=6.0,
+                                        sinks=sinks.double().numpy())
+    check(o, o_ref, lse, l_ref, what="paged prefill with modifiers d%d" % d)
