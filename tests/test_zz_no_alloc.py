@@ -31,7 +31,8 @@ def noalloc_fn():
 
 
 def call_noalloc(fn, q, kc, vc, tb, sl, scale, num_splits=0):
-    o = torch.full((q.shape[0], q.shape[1], vc.shape[3]), float("nan"), device="cuda")
+    dv = vc.shape[3] // 34 * 32 if vc.dtype == torch.uint8 else vc.shape[3]  # q8_0 rows: 34 bytes per 32 values
+    o = torch.full((q.shape[0], q.shape[1], dv), float("nan"), device="cuda")
     lse = torch.full((q.shape[0], q.shape[1]), float("nan"), device="cuda")
     p = fa.paged_params(q, kc, vc, tb, sl, o, lse, scale, num_splits, None)
     st = fn(ctypes.byref(p), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
@@ -49,6 +50,21 @@ def test_noalloc_matches_workspace_entry_point_twice():
         assert st == fa.FA_OK, lib.fa_last_error().decode()
         torch.cuda.synchronize()
         check(o, ref_o, lse, ref_l, what=c.name)
+    assert fa.device_error() == 0
+
+
+def test_noalloc_q8_0_caches():
+    # the in-kernel q8_0 prologue through the allocation-free entry point
+    lib, fn = noalloc_fn()
+    c = W.PagedCase("noalloc_q8", 7, 16, 4, 128, 128, 64, 0, 2000, seed=126, lens=(0, 1, 64, 65, 700, 2000, 129))
+    q, _, _, tb, sl = W.paged_inputs(c)
+    kq, vq = W.paged_q8_caches(c, int(tb.max()) + 1)
+    q, kq, vq, tb, sl = q.cuda(), kq.cuda(), vq.cuda(), tb.cuda(), sl.cuda()
+    ref_o, ref_l = fa.decode_paged(q, kq, vq, tb, sl, scale=c.scale)
+    st, o, lse = call_noalloc(fn, q, kq, vq, tb, sl, c.scale)
+    assert st == fa.FA_OK, lib.fa_last_error().decode()
+    torch.cuda.synchronize()
+    check(o, ref_o, lse, ref_l, what=c.name)
     assert fa.device_error() == 0
 
 
