@@ -27,6 +27,7 @@
 // bandwidth-bound kernel (llama.cpp "ggml-metal: FA tensor path", the vec
 // decode rule); the split merge is the log-sum-exp ("D5") merge of the
 // nvfp4-megamoe-kernel notes.
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <math.h>
 
@@ -56,14 +57,22 @@ constexpr int PD_SMEM = PD_OFF_BAR + 128 + 1024;  // ring + barriers + 1024-byte
 #ifndef FA_PD_Q8_PRMT
 #define FA_PD_Q8_PRMT 1
 #endif
-constexpr int PDQ_ROW = 136;
-constexpr int PDQ_TILE = PD_BS * PDQ_ROW;          // 8704 bytes
-constexpr int PDQ_STAGE = 2 * PDQ_TILE;            // K + V, 17 KB (1024-byte multiple)
-constexpr int PDQ_NST = 4;
-constexpr int PDQ_WBUF = 2 * 16 * PD_D * 2;        // one warp's 16 keys of K and V in bf16: 8 KB
-constexpr int PDQ_OFF_WB = PDQ_NST * PDQ_STAGE;
-constexpr int PDQ_OFF_BAR = PDQ_OFF_WB + 4 * PDQ_WBUF;
-constexpr int PDQ_SMEM = PDQ_OFF_BAR + 128 + 1024;
+// FP8 E4M3 caches take the same prologue with 128-byte rows (one byte per
+// value) and one fp32 scale per tensor (k_scale, v_scale).
+//
+// Raw-tile geometry per cache type KVT (8 = q8_0, 2 = fp8 e4m3):
+template <int KVT>
+struct PdRaw {
+    static constexpr int ROW = KVT == 8 ? 136 : 128;          // bytes per cache row of 128 values
+    static constexpr int TILE = PD_BS * ROW;                  // one (block, head) tile of K or V
+    static constexpr int STAGE = 2 * TILE;                    // K + V (1024-byte multiple)
+    static constexpr int NST = 4;
+    static constexpr int WBUF = 2 * 16 * PD_D * 2;            // one warp's 16 keys of K and V in bf16: 8 KB
+    static constexpr int OFF_WB = NST * STAGE;
+    static constexpr int OFF_BAR = OFF_WB + 4 * WBUF;
+    static constexpr int SMEM = OFF_BAR + 128 + 1024;
+    static_assert(STAGE % 1024 == 0, "stage alignment");
+};
 
 // Two int8 codes (low and high byte of w) times the block scale d -> a bf16
 // pair.  A code's byte xor 0x80 is code + 128; OR-ed into the mantissa of
@@ -92,14 +101,15 @@ FA_DEV uint32_t q8_pair_to_bf16(uint32_t w, uint64_t d2) {
 
 struct PagedArgs {
     const __nv_bfloat16 *q;
-    const uint8_t *kq, *vq;  // q8_0 caches (KVQ instantiation)
+    const uint8_t *kq, *vq;  // quantised caches (KVT != 0)
+    float k_scale, v_scale;  // fp8 caches: the tensors' scales
     const int32_t *block_table, *seq_lens;
     int max_blocks, Hq, Hkv, num_blocks, bps, num_splits;
     float scale_log2;
     float *part_o, *part_lse;
 };
 
-template <int G, bool KVQ>
+template <int G, int KVT>
 __global__ void __launch_bounds__(160) paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                                                            const __grid_constant__ CUtensorMap tmV,
                                                            const PagedArgs a) {
@@ -119,9 +129,11 @@ __global__ void __launch_bounds__(160) paged_decode_kernel(const __grid_constant
     if (blk0 >= nb) return;  // this split holds no key of this sequence (uniform exit)
     const int nblk = min(a.bps, nb - blk0);
 
-    constexpr int NST = KVQ ? PDQ_NST : PD_NST;
-    constexpr int STAGE = KVQ ? PDQ_STAGE : PD_STAGE;
-    constexpr int OFF_BAR = KVQ ? PDQ_OFF_BAR : PD_OFF_BAR;
+    constexpr bool KVQ = KVT != 0;
+    using R = PdRaw<KVQ ? KVT : 8>;
+    constexpr int NST = KVQ ? R::NST : PD_NST;
+    constexpr int STAGE = KVQ ? R::STAGE : PD_STAGE;
+    constexpr int OFF_BAR = KVQ ? R::OFF_BAR : PD_OFF_BAR;
     const uint32_t sbase = smem_u32(smem);
     const uint32_t bar0 = sbase + OFF_BAR;
     auto full = [&](int s) { return bar0 + 8u * s; };
@@ -164,11 +176,11 @@ __global__ void __launch_bounds__(160) paged_decode_kernel(const __grid_constant
             if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
             if (lane == 0) {
                 if constexpr (KVQ) {
-                    const int64_t off = ((int64_t)blk * a.Hkv + hkv) * PDQ_TILE;  // this (block, head) tile
-                    const uint32_t dst = sbase + s * PDQ_STAGE;
-                    mbar_arrive_expect_tx(full(s), PDQ_STAGE);
-                    bulk_load(dst, a.kq + off, PDQ_TILE, full(s));
-                    bulk_load(dst + PDQ_TILE, a.vq + off, PDQ_TILE, full(s));
+                    const int64_t off = ((int64_t)blk * a.Hkv + hkv) * R::TILE;  // this (block, head) tile
+                    const uint32_t dst = sbase + s * R::STAGE;
+                    mbar_arrive_expect_tx(full(s), R::STAGE);
+                    bulk_load(dst, a.kq + off, R::TILE, full(s));
+                    bulk_load(dst + R::TILE, a.vq + off, R::TILE, full(s));
                 } else {
                     const int row0 = (blk * a.Hkv + hkv) * PD_BS;  // first cache row of this (block, head)
                     const uint32_t dst = sbase + s * PD_STAGE;
@@ -227,17 +239,49 @@ __global__ void __launch_bounds__(160) paged_decode_kernel(const __grid_constant
         // between the two 64-column halves.
         uint32_t sK, sV, hstr;
         int kof;
-        if constexpr (KVQ) {
+        if constexpr (KVT == 2) {
+            // lane (lk, h) converts row lk's half h (64 fp8 bytes) of K and of
+            // V: e4m3 pairs -> f16 pairs (exact) -> f32 times the tensor scale
+            // -> a bf16 pair.  (The fp32 product rounds once before the bf16
+            // conversion; the pre-pass forms it in fp64 and rounds once.)
+            const int lk = lane >> 1, h = lane & 1;
+            const uint8_t *raw = smem + s * R::STAGE + (warp * 16 + lk) * R::ROW + 64 * h;
+            uint8_t *wb = smem + R::OFF_WB + warp * R::WBUF + h * (16 * 128) + lk * 128;
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {  // K, then V
+                const uint64_t sc2 = t == 0 ? f2_pack(a.k_scale, a.k_scale) : f2_pack(a.v_scale, a.v_scale);
+                uint4 bytes[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) bytes[i] = *reinterpret_cast<const uint4 *>(raw + t * R::TILE + 16 * i);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {  // 16-byte output chunk j: values 8 j .. 8 j + 7
+                    const uint32_t w0 = (&bytes[j >> 1].x)[(j & 1) * 2], w1 = (&bytes[j >> 1].x)[(j & 1) * 2 + 1];
+                    uint32_t outw[4];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const uint32_t w = k < 2 ? w0 : w1;
+                        const __half2_raw hr =
+                            __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)((w >> (16 * (k & 1))) & 0xffffu), __NV_E4M3);
+                        const float2 f = __half22float2(__half2(hr));
+                        float x0, x1;
+                        f2_unpack(f2_mul(f2_pack(f.x, f.y), sc2), x0, x1);
+                        outw[k] = pack_bf16x2(x0, x1);
+                    }
+                    *reinterpret_cast<uint4 *>(wb + t * (2 * 16 * 128) + ((j ^ (lk & 7)) << 4)) =
+                        make_uint4(outw[0], outw[1], outw[2], outw[3]);
+                }
+            }
+        } else if constexpr (KVT == 8) {
             // lane (lk, h) converts row lk's half h (two q8_0 blocks, 64 values)
             // of K and of V into eight 16-byte chunks of the swizzled buffer
             const int lk = lane >> 1, h = lane & 1;
-            const uint8_t *raw = smem + s * PDQ_STAGE + (warp * 16 + lk) * PDQ_ROW + 68 * h;
-            uint8_t *wb = smem + PDQ_OFF_WB + warp * PDQ_WBUF + h * (16 * 128) + lk * 128;
+            const uint8_t *raw = smem + s * R::STAGE + (warp * 16 + lk) * R::ROW + 68 * h;
+            uint8_t *wb = smem + R::OFF_WB + warp * R::WBUF + h * (16 * 128) + lk * 128;
 #pragma unroll
             for (int t = 0; t < 2; ++t) {  // K, then V
 #pragma unroll
                 for (int qb = 0; qb < 2; ++qb) {
-                    const uint8_t *p = raw + t * PDQ_TILE + 34 * qb;
+                    const uint8_t *p = raw + t * R::TILE + 34 * qb;
                     const float d = __half2float(*reinterpret_cast<const __half *>(p));
                     const uint64_t d2 = f2_pack(d, d);
                     const uint16_t *cw = reinterpret_cast<const uint16_t *>(p + 2);
@@ -251,9 +295,11 @@ __global__ void __launch_bounds__(160) paged_decode_kernel(const __grid_constant
                     }
                 }
             }
+        }
+        if constexpr (KVQ) {
             __syncwarp();
             if (lane == 0) mbar_arrive(empty(s));  // the raw stage may be refilled now
-            sK = sbase + PDQ_OFF_WB + warp * PDQ_WBUF;
+            sK = sbase + R::OFF_WB + warp * R::WBUF;
             sV = sK + 2 * 16 * 128;
             hstr = 16 * 128;
             kof = warp * 16;
@@ -459,10 +505,10 @@ cudaError_t launch_combine(const float *part_o, const float *part_lse, int rows,
     return cudaGetLastError();
 }
 
-template <int G, bool KVQ>
+template <int G, int KVT>
 static cudaError_t launch_g(const PagedLaunch &L, const PagedArgs &a, int B, cudaStream_t stream) {
-    auto kern = paged_decode_kernel<G, KVQ>;
-    constexpr int smem = KVQ ? PDQ_SMEM : PD_SMEM;
+    auto kern = paged_decode_kernel<G, KVT>;
+    constexpr int smem = KVT == 0 ? PD_SMEM : PdRaw<KVT == 0 ? 8 : KVT>::SMEM;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)a.num_splits, (unsigned)a.Hkv, (unsigned)B);
@@ -472,7 +518,9 @@ static cudaError_t launch_g(const PagedLaunch &L, const PagedArgs &a, int B, cud
 
 template <int G>
 static cudaError_t launch_gq(const PagedLaunch &L, const PagedArgs &a, int B, cudaStream_t stream) {
-    return L.kv_q8 ? launch_g<G, true>(L, a, B, stream) : launch_g<G, false>(L, a, B, stream);
+    return L.kv_type == 8   ? launch_g<G, 8>(L, a, B, stream)
+           : L.kv_type == 2 ? launch_g<G, 2>(L, a, B, stream)
+                            : launch_g<G, 0>(L, a, B, stream);
 }
 
 cudaError_t launch_decode_paged(const PagedLaunch &L, cudaStream_t stream) {
@@ -480,6 +528,8 @@ cudaError_t launch_decode_paged(const PagedLaunch &L, cudaStream_t stream) {
     a.q = static_cast<const __nv_bfloat16 *>(L.q);
     a.kq = static_cast<const uint8_t *>(L.k_cache);
     a.vq = static_cast<const uint8_t *>(L.v_cache);
+    a.k_scale = L.k_scale;
+    a.v_scale = L.v_scale;
     a.block_table = L.block_table;
     a.seq_lens = L.seq_lens;
     a.max_blocks = L.max_blocks_per_seq;

@@ -57,7 +57,8 @@ struct PagedLaunch {
     int o_bf16;
     float *part_o;    // [B*Hq, num_splits, 128]
     float *part_lse;  // [B*Hq, num_splits]   (log2 units)
-    bool kv_q8;       // caches hold q8_0 rows of 136 bytes (bulk copies; tmK/tmV unused)
+    int kv_type;      // 0: bf16 (TMA); 8: q8_0 rows of 136 bytes, 2: fp8 rows of 128 (bulk copies)
+    float k_scale, v_scale;  // fp8 caches
 };
 cudaError_t launch_decode_paged(const PagedLaunch &L, cudaStream_t stream);
 // Log-sum-exp merge of split partials (D = 128 or 512).  seq_lens != NULL:

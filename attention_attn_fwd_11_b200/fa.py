@@ -42,7 +42,8 @@ class PagedParams(ctypes.Structure):
                 ("max_blocks_per_seq", _i32), ("B", _i32), ("Hq", _i32), ("Hkv", _i32), ("dk", _i32),
                 ("dv", _i32), ("block_size", _i32), ("num_blocks", _i32), ("scale", ctypes.c_float),
                 ("num_splits", _i32), ("o", _vp), ("lse", _vp), ("o_dtype", _i32), ("workspace", _vp),
-                ("workspace_bytes", ctypes.c_size_t), ("kv_type", _i32)]
+                ("workspace_bytes", ctypes.c_size_t), ("kv_type", _i32), ("k_scale", ctypes.c_float),
+                ("v_scale", ctypes.c_float)]
 
 
 class PrefillPagedParams(ctypes.Structure):
@@ -216,7 +217,8 @@ def fwd(q, k, v, scale=None, causal=False, out=None, return_lse=True, out_dtype=
 
 # ------------------------------------------------------------- paged decode --
 
-def paged_params(q, k_cache, v_cache, block_table, seq_lens, o, lse, scale, num_splits, ws):
+def paged_params(q, k_cache, v_cache, block_table, seq_lens, o, lse, scale, num_splits, ws, kv_type=None,
+                 k_scale=1.0, v_scale=1.0):
     B, Hq, dk = q.shape
     nb, Hkv, bs, _ = k_cache.shape
     p = PagedParams()
@@ -224,9 +226,12 @@ def paged_params(q, k_cache, v_cache, block_table, seq_lens, o, lse, scale, num_
     p.block_table, p.seq_lens = _ptr(block_table), _ptr(seq_lens)
     p.max_blocks_per_seq = block_table.shape[1]
     dv = v_cache.shape[3]
-    if k_cache.dtype == torch.uint8:  # q8_0 rows: 34 bytes per 32 values
-        p.kv_type = FA_KV_Q8_0
-        dv = v_cache.shape[3] // 34 * 32
+    if k_cache.dtype == torch.uint8:  # q8_0 rows (34 bytes per 32 values) or fp8 bytes
+        if kv_type is None:
+            kv_type = "fp8_e4m3" if v_cache.shape[3] % 34 else "q8_0"
+        p.kv_type = KV_QUANT[kv_type][0]
+        dv = v_cache.shape[3] // 34 * 32 if kv_type == "q8_0" else v_cache.shape[3]
+        p.k_scale, p.v_scale = k_scale, v_scale
     p.B, p.Hq, p.Hkv, p.dk, p.dv, p.block_size, p.num_blocks = B, Hq, Hkv, dk, dv, bs, nb
     p.scale = scale
     p.num_splits = num_splits
@@ -245,23 +250,28 @@ def paged_workspace_bytes(q, k_cache, v_cache, block_table, seq_lens, num_splits
 
 
 def decode_paged(q, k_cache, v_cache, block_table, seq_lens, scale=None, num_splits=0, out=None,
-                 return_lse=True, out_dtype=torch.float32, workspace=None, stream=None):
+                 return_lse=True, out_dtype=torch.float32, workspace=None, stream=None, kv_type=None, k_scale=1.0,
+                 v_scale=1.0):
     """Split-KV decode over a paged cache.  q [B,Hq,dk]; caches
-    [num_blocks,Hkv,block_size,d] bf16, or uint8 [...,136] of q8_0 rows
+    [num_blocks,Hkv,block_size,d] bf16, or uint8 [...,136] of q8_0 rows, or
+    uint8 [...,128] of fp8 e4m3 bytes read as e4m3 * k_scale / v_scale
     (dequantised in the kernel); block_table int32 [B,max_blocks];
     seq_lens int32 [B].  Returns (O [B,Hq,dv], LSE [B,Hq] or None)."""
     _need_cuda(q, k_cache, v_cache, block_table, seq_lens)
     B, Hq, dk = q.shape
     if scale is None:
         scale = 1.0 / math.sqrt(dk)
-    dv = v_cache.shape[3] // 34 * 32 if v_cache.dtype == torch.uint8 else v_cache.shape[3]
+    if v_cache.dtype == torch.uint8 and kv_type is None:
+        kv_type = "fp8_e4m3" if v_cache.shape[3] % 34 else "q8_0"
+    dv = v_cache.shape[3] // 34 * 32 if kv_type == "q8_0" else v_cache.shape[3]
     if out is None:
         out = torch.empty((B, Hq, dv), device=q.device, dtype=out_dtype)
     lse = torch.empty((B, Hq), device=q.device, dtype=torch.float32) if return_lse else None
     if workspace is None:
         n = paged_workspace_bytes(q, k_cache, v_cache, block_table, seq_lens, num_splits)
         workspace = torch.empty(max(n, 256), device=q.device, dtype=torch.uint8)
-    p = paged_params(q, k_cache, v_cache, block_table, seq_lens, out, lse, scale, num_splits, workspace)
+    p = paged_params(q, k_cache, v_cache, block_table, seq_lens, out, lse, scale, num_splits, workspace, kv_type,
+                     k_scale, v_scale)
     _check(load().fa_decode_paged(ctypes.byref(p), _stream(stream)))
     return out, lse
 

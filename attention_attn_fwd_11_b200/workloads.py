@@ -220,6 +220,14 @@ def paged_inputs(c: PagedCase):
     return q, kc, vc, table, lens.to(torch.int32)
 
 
+def paged_fp8_caches(c: PagedCase, num_blocks: int):
+    """FP8 E4M3 K and V caches [num_blocks, Hkv, block_size, d] uint8 for
+    the same pool (seeds 7000 + c and 7100 + c; tensor scale FP8_SCALE)."""
+    kf = random_quant_rows((num_blocks, c.Hkv, c.block_size), c.dk, "fp8_e4m3", c.seed)
+    vf = random_quant_rows((num_blocks, c.Hkv, c.block_size), c.dv, "fp8_e4m3", c.seed + 100)
+    return kf, vf
+
+
 def paged_q8_caches(c: PagedCase, num_blocks: int):
     """q8_0 K and V caches [num_blocks, Hkv, block_size, dk / 32 * 34] uint8
     for the same pool (seeds 7000 + c and 7100 + c)."""
@@ -228,18 +236,20 @@ def paged_q8_caches(c: PagedCase, num_blocks: int):
     return kq, vq
 
 
-def paged_bytes(c: PagedCase, seq_lens, max_blocks: int, q8: bool = False) -> int:
+def paged_bytes(c: PagedCase, seq_lens, max_blocks: int, q8: bool = False, fp8: bool = False) -> int:
     """Algorithmic HBM bytes of one paged decode: every visible K/V element
-    once (2 bytes, or 34 / 32 for q8_0 rows), the used block-table entries,
-    lengths, Q, fp32 O and LSE."""
+    once (2 bytes, 34 / 32 for q8_0 rows, 1 for fp8), the used block-table
+    entries, lengths, Q, fp32 O and LSE."""
     sl = [int(x) for x in seq_lens]
-    kv = sum(sl) * c.Hkv * ((c.dk + c.dv) // 32 * 34 if q8 else (c.dk + c.dv) * 2)
+    per = (c.dk + c.dv) // 32 * 34 if q8 else ((c.dk + c.dv) if fp8 else (c.dk + c.dv) * 2)
+    kv = sum(sl) * c.Hkv * per
     tbl = sum((n + c.block_size - 1) // c.block_size for n in sl) * 4
     return kv + tbl + c.B * 4 + c.B * c.Hq * c.dk * 2 + c.B * c.Hq * c.dv * 4 + c.B * c.Hq * 4
 
 
 PAGED_GQA = PagedCase("paged_gqa_b64_hq32_hkv8_d128_bs64", 64, 32, 8, 128, 128, 64, 1024, 8192, seed=4)
 PAGED_Q8_NAME = "paged_gqa_q8_0kv_b64_hq32_hkv8_d128_bs64"  # the same decode over q8_0 caches
+PAGED_FP8_NAME = "paged_gqa_fp8kv_b64_hq32_hkv8_d128_bs64"  # ... and over fp8 e4m3 caches
 
 
 # ----------------------------------------------------------- paged prefill --

@@ -380,13 +380,16 @@ def latent_prefill_workload(torch, fa, W_, c, l2):
     return launch, n, c.flops, 2
 
 
-def paged_workload(torch, fa, W_, c, l2, q8=False):
-    """Paged decode (decode kernel + LSE combine per step); q8: the caches
-    hold q8_0 rows, converted inside the decode kernel."""
+def paged_workload(torch, fa, W_, c, l2, q8=False, fp8=False):
+    """Paged decode (decode kernel + LSE combine per step); q8 / fp8: the
+    caches hold q8_0 rows or fp8 e4m3 bytes, converted inside the decode
+    kernel."""
     q0, kc0, vc0, tb0, sl0 = W_.paged_inputs(c)
     if q8:
         kc0, vc0 = W_.paged_q8_caches(c, kc0.shape[0])
-    byts = W_.paged_bytes(c, sl0, tb0.shape[1], q8=q8)
+    elif fp8:
+        kc0, vc0 = W_.paged_fp8_caches(c, kc0.shape[0])
+    byts = W_.paged_bytes(c, sl0, tb0.shape[1], q8=q8, fp8=fp8)
     foot = (kc0.numel() + vc0.numel()) * kc0.element_size()
     n = rotation_copies(foot, l2)
     import ctypes
@@ -399,7 +402,9 @@ def paged_workload(torch, fa, W_, c, l2, q8=False):
         nws = fa.paged_workspace_bytes(q, kc, vc, tb, sl, 0)
         ws = torch.empty(nws, dtype=torch.uint8, device="cuda")
         bufs.append((q, kc, vc, tb, sl, o, lse, ws))
-        params.append(fa.paged_params(q, kc, vc, tb, sl, o, lse, c.scale, 0, ws))
+        params.append(fa.paged_params(q, kc, vc, tb, sl, o, lse, c.scale, 0, ws,
+                                      kv_type="fp8_e4m3" if fp8 else None, k_scale=W_.FP8_SCALE,
+                                      v_scale=W_.FP8_SCALE))
 
     def launch(i):
         st = lib.fa_decode_paged(ctypes.byref(params[i]), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
@@ -529,6 +534,7 @@ def run_only(args):
                                  W_.CAUSAL_DK192_DV192, W_.CAUSAL_DK320, W_.PAGED_GQA, W_.LATENT_SPARSE,
                                  W_.QUANT_C2, W_.PAGED_PREFILL, W_.MLA_TAIL)}
     table[W_.PAGED_Q8_NAME] = W_.PAGED_GQA
+    table[W_.PAGED_FP8_NAME] = W_.PAGED_GQA
     table[W_.LATENT_PREFILL.name] = W_.LATENT_PREFILL
     table[W_.LATENT_PREFILL_512.name] = W_.LATENT_PREFILL_512
     table["kv_dequant_" + W_.QUANT_C2.name] = W_.QUANT_C2
@@ -555,7 +561,8 @@ def run_only(args):
         launch, n, work, kpl = paged_prefill_workload(torch, fa, W_, c, l2)
         unit, amount = "TFLOP/s", work / 1e12
     elif isinstance(c, W_.PagedCase):
-        launch, n, work, kpl = paged_workload(torch, fa, W_, c, l2, q8=args.only == W_.PAGED_Q8_NAME)
+        launch, n, work, kpl = paged_workload(torch, fa, W_, c, l2, q8=args.only == W_.PAGED_Q8_NAME,
+                                              fp8=args.only == W_.PAGED_FP8_NAME)
         unit, amount = "GB/s", work / 1e9
     else:
         launch, n, work, kpl = latent_workload(torch, fa, W_, c, l2)
@@ -776,19 +783,20 @@ def main():
         result["gpu_launches"] += st2 * kpl
         del launch
         # the same decode over q8_0 caches (dequant prologue in the kernel)
-        launch, ncopy, byts, kpl = paged_workload(torch, fa, W_, pc, l2, q8=True)
-        ms2, st2 = time_graph(torch, launch, ncopy, Ks, Wm, dist)
-        ms2 = max_over_ranks(torch, dist, ms2)
-        per = ms2 / st2
-        ach = byts / (per * 1e-3) / 1e9
-        wl[W_.PAGED_Q8_NAME] = {"value": round(sum_over_ranks(torch, dist, byts * st2) / (ms2 * 1e-3) / 1e9, 1),
-                                "unit": "GB/s", "ms_per_step": round(per, 5), "steps": st2, "l2_copies": ncopy,
-                                "bytes_per_step": byts,
-                                "roofline": roofline("hbm", ach, peaks["hbm_gbs"], "GB/s",
-                                                     NCU_TRAFFIC.get(W_.PAGED_Q8_NAME)),
-                                "kernels": "paged decode with the q8_0 prologue + LSE combine"}
-        result["gpu_launches"] += st2 * kpl
-        del launch
+        for qname, qkw in ((W_.PAGED_Q8_NAME, dict(q8=True)), (W_.PAGED_FP8_NAME, dict(fp8=True))):
+            launch, ncopy, byts, kpl = paged_workload(torch, fa, W_, pc, l2, **qkw)
+            ms2, st2 = time_graph(torch, launch, ncopy, Ks, Wm, dist)
+            ms2 = max_over_ranks(torch, dist, ms2)
+            per = ms2 / st2
+            ach = byts / (per * 1e-3) / 1e9
+            wl[qname] = {"value": round(sum_over_ranks(torch, dist, byts * st2) / (ms2 * 1e-3) / 1e9, 1),
+                         "unit": "GB/s", "ms_per_step": round(per, 5), "steps": st2, "l2_copies": ncopy,
+                         "bytes_per_step": byts,
+                         "roofline": roofline("hbm", ach, peaks["hbm_gbs"], "GB/s", NCU_TRAFFIC.get(qname)),
+                         "kernels": "paged decode with the %s prologue + LSE combine" % ("q8_0" if "q8" in qkw else
+                                                                                         "fp8 e4m3")}
+            result["gpu_launches"] += st2 * kpl
+            del launch
         try:
             lc = W_.LATENT_SPARSE
             launch, ncopy, (byts, flops), kpl = latent_workload(torch, fa, W_, lc, l2)

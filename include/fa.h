@@ -203,6 +203,10 @@ fa_status fa_prefill_paged(const fa_prefill_paged_params *p, void *stream);
  *     [num_blocks, Hkv, block_size, 136] bytes.  The kernel converts each
  *     tile in shared memory (the same single rounding to bf16 as
  *     fa_kv_dequant), so the cache is read once, at 1.06 bytes per value.
+ *     With kv_type FA_KV_FP8_E4M3: OCP E4M3 bytes [num_blocks, Hkv,
+ *     block_size, 128], value = e4m3 * k_scale (K) or * v_scale (V), formed
+ *     in fp32 and converted to bf16 in the kernel (two roundings where
+ *     fa_kv_dequant rounds once).
  *   block_table: [B, max_blocks_per_seq] int32; key j of sequence b is slot
  *     j % block_size of physical block block_table[b][j / block_size].
  *     Entries past a sequence's last block are never read.
@@ -235,7 +239,8 @@ typedef struct {
     int o_dtype; /* fa_dtype */
     void *workspace;
     size_t workspace_bytes;
-    int kv_type; /* FA_KV_BF16 (0) or FA_KV_Q8_0 */
+    int kv_type; /* FA_KV_BF16 (0), FA_KV_Q8_0 or FA_KV_FP8_E4M3 */
+    float k_scale, v_scale; /* FA_KV_FP8_E4M3: the caches' tensor scales (finite) */
 } fa_decode_paged_params;
 
 /* Workspace bytes for these shapes and num_splits; reads no pointer field. */

@@ -1,6 +1,7 @@
-"""Paged decode over q8_0 caches (the dequant prologue inside the decode
-kernel) against the oracle: the oracle dequantises the caches (one rounding
-to bf16, as the kernel does) and runs its paged decode on them."""
+"""Paged decode over q8_0 and FP8 E4M3 caches (the dequant prologue inside
+the decode kernel) against the oracle: the oracle dequantises the caches
+(one rounding to bf16; the q8_0 prologue makes the same rounding, the FP8 one
+forms e4m3 * scale in fp32 first) and runs its paged decode on them."""
 import numpy as np
 import pytest
 import torch
@@ -63,3 +64,22 @@ def test_workload_shape():
         tb1 = np.arange(nbk, dtype=np.int32)[None]
         o_ref, l_ref = oracle.decode_paged(W.bits(q[b:b + 1]), kb, vb, tb1, np.array([n], np.int32), c.scale)
         check(o[b:b + 1], o_ref, lse[b:b + 1], l_ref, what="q8_0 workload seq %d" % b)
+
+
+
+@pytest.mark.parametrize("g", [1, 4, 8])
+def test_fp8_caches(g):
+    c = W.PagedCase("t", 5, 2 * g, 2, 128, 128, 64, 1, 1, seed=30 + g, lens=(1, 63, 64, 65, 1500))
+    q, _, _, table, sl = W.paged_inputs(c)
+    nb = int(sum((n + 63) // 64 for n in c.lens))
+    kf = W.random_quant_rows((nb, 2, 64), 128, "fp8_e4m3", c.seed)
+    vf = W.random_quant_rows((nb, 2, 64), 128, "fp8_e4m3", c.seed + 100)
+    ks, vs = W.FP8_SCALE, 1.5 * W.FP8_SCALE
+    o, lse = fa.decode_paged(q.cuda(), kf.cuda(), vf.cuda(), table.cuda(), sl.cuda(), scale=c.scale,
+                             k_scale=ks, v_scale=vs)
+    torch.cuda.synchronize()
+    assert fa.device_error() == 0
+    kb = oracle.dequant_rows(kf.numpy(), "fp8_e4m3", 128, scale=ks)
+    vb = oracle.dequant_rows(vf.numpy(), "fp8_e4m3", 128, scale=vs)
+    o_ref, l_ref = oracle.decode_paged(W.bits(q), kb, vb, table.numpy(), sl.numpy(), c.scale)
+    check(o, o_ref, lse, l_ref, what="fp8 paged decode g%d" % g)
