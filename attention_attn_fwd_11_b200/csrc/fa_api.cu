@@ -251,10 +251,10 @@ fa_status check_tail(const fa_mla_tail_params *p) {
     if (!p) return fail(FA_ERR_INVALID_ARG, "fa_mla_tail: params is NULL");
     if (p->T < 0 || p->Hq <= 0 || p->R <= 0 || p->V <= 0 || p->Hd <= 0)
         return fail(FA_ERR_INVALID_ARG, "fa_mla_tail: need T >= 0 and Hq, R, V, Hd > 0");
-    if (p->V != 128 || p->R % 64 != 0 || p->Hd % 128 != 0 || ((int64_t)p->Hq * p->V) % 64 != 0 || p->T > 256)
-        return fail(FA_ERR_UNSUPPORTED,
-                    "fa_mla_tail: supported V = 128, R % 64 == 0, Hd % 128 == 0, T <= 256 (got V %d R %d Hd %d T %d)",
-                    p->V, p->R, p->Hd, p->T);
+    if (p->V != 128 || p->R % 64 != 0 || p->Hd % 128 != 0 || ((int64_t)p->Hq * p->V) % 64 != 0)
+        return fail(FA_ERR_UNSUPPORTED, "fa_mla_tail: supported V = 128, R % 64 == 0, Hd % 128 == 0 (got V %d R %d Hd %d)",
+                    p->V, p->R, p->Hd);
+    if ((int64_t)p->T * p->Hq > 0x7fffffffLL) return fail(FA_ERR_INVALID_ARG, "fa_mla_tail: T * Hq out of range");
     if ((int64_t)p->Hq * p->V > (1 << 30) || p->R > (1 << 20) || p->Hd > (1 << 24))
         return fail(FA_ERR_INVALID_ARG, "fa_mla_tail: sizes out of range");
     if (p->y_dtype != FA_F32 && p->y_dtype != FA_BF16) return fail(FA_ERR_INVALID_ARG, "fa_mla_tail: y_dtype");
@@ -638,7 +638,7 @@ fa_status fa_mla_tail(const fa_mla_tail_params *p, void *stream) {
     if (!p->workspace || p->workspace_bytes < need || ((uintptr_t)p->workspace & 255u))
         return fail(FA_ERR_WORKSPACE, "fa_mla_tail: workspace must be 256-byte aligned and >= %zu bytes", need);
     if (!get_encoder()) return fail(FA_ERR_CUDA, "fa_mla_tail: cuTensorMapEncodeTiled is not available");
-    const int NP = (p->T + 15) / 16 * 16;
+    const int NP = p->T < 256 ? (p->T + 15) / 16 * 16 : 256;  // token rows per chunk load
     const int64_t K = (int64_t)p->Hq * p->V;
     // (inner, rows, batch, 1) views; element strides.
     st = encode_4d(&L.tmAbsA, p->w_abs, p->R, p->V, p->Hq, 1, p->R, (int64_t)p->V * p->R,

@@ -40,8 +40,9 @@ constexpr int TG_THREADS = 128;     // warp 0: TMA, warp 1: MMA, all four: epilo
 constexpr int TG_A_BYTES = TG_BM * TG_BK * 2;
 
 struct TailGemmArgs {
-    int NP;        // MMA N: tokens rounded up to 16 (<= 256)
-    int N;         // tokens
+    int NP;        // MMA N: tokens of this chunk rounded up to 16 (<= 256)
+    int N;         // tokens of this chunk
+    int n0;        // the chunk's first token
     int ks;        // stages of 64 K per split (the last split may have fewer)
     int k_total;   // stages of 64 K in the whole contraction
     int stages;    // ring depth
@@ -151,7 +152,7 @@ tail_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                     tma_load_4d(sA(s), &tmA, full(s), (k0 + i) * TG_BK, m0, bz, 0);
                     issued = i + 1;
                 }
-                tma_load_4d(sB(s), &tmB, full(s), (k0 + i) * TG_BK, 0, bz, 0);
+                tma_load_4d(sB(s), &tmB, full(s), (k0 + i) * TG_BK, a.n0, bz, 0);
             }
             if (*abort_flag) {  // let the copies in flight land before the CTA exits
                 for (int i = issued - a.stages > 0 ? issued - a.stages : 0; i < issued; ++i)
@@ -206,7 +207,7 @@ tail_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             if (go) {
 #pragma unroll
                 for (int j = 0; j < 32; ++j)
-                    if (32 * c + j < a.N) store_out(a, bz, 32 * c + j, m0 + row, __uint_as_float(r[j]));
+                    if (32 * c + j < a.N) store_out(a, bz, a.n0 + 32 * c + j, m0 + row, __uint_as_float(r[j]));
             }
             continue;
         }
@@ -233,7 +234,7 @@ tail_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                     acc.z += v[q].z;
                     acc.w += v[q].w;
                 }
-            if (!*abort_flag) store_out4(a, bz, n, m0 + 4 * (g & 31), acc);
+            if (!*abort_flag) store_out4(a, bz, a.n0 + n, m0 + 4 * (g & 31), acc);
         }
         cluster_sync();
     }
@@ -308,45 +309,56 @@ int mla_tail_splits(const TailLaunch &L, int num_sms) {
 size_t mla_tail_ws_bytes(const TailLaunch &L) { return ((size_t)L.T * L.Hq * L.V * 2 + 255) & ~size_t(255); }
 
 cudaError_t launch_mla_tail(const TailLaunch &L, int num_sms, cudaStream_t stream) {
-    if (L.T == 0) return cudaSuccess;
-    const int NP = (L.T + 15) / 16 * 16;
+    // Tokens are the MMA's N (at most 256), so larger batches run in chunks
+    // of 256 tokens: each chunk's out-absorb, then its o-projection.  Every
+    // chunk loads NP token rows -- the box height the B-operand tensor maps
+    // were encoded with (T rounded up to 16, or 256 when T > 256); rows past
+    // T read as zero and are not stored.
+    const int NP = L.T < 256 ? (L.T + 15) / 16 * 16 : 256;
     int ncols = 32;
     while (ncols < NP) ncols *= 2;
     const int stages = tail_stages(NP);
+    for (int n0 = 0; n0 < L.T; n0 += 256) {
+        const int nt = L.T - n0 < 256 ? L.T - n0 : 256;
 
-    // out-absorb: batch = heads, M = V, K = R split over a cluster; u[t][h*V + v] in bf16.
-    TailGemmArgs a{};
-    a.NP = NP;
-    a.N = L.T;
-    a.k_total = L.R / TG_BK;
-    const int sa = fit_splits(FA_TAIL_ABSORB_SPLITS > 0 ? FA_TAIL_ABSORB_SPLITS : (2 * num_sms) / (L.Hq * (L.V / TG_BM)),
-                              a.k_total);
-    a.ks = (a.k_total + sa - 1) / sa;
-    a.stages = stages;
-    a.ncols = ncols;
-    a.out = L.workspace;
-    a.ob = L.V;
-    a.on = (int64_t)L.Hq * L.V;
-    a.out_bf16 = 1;
-    a.pdl_trigger = FA_TAIL_PDL;
-    cudaError_t e = run_gemm(L.tmAbsA, L.tmAbsB, a, L.V / TG_BM, sa, L.Hq, false, stream);
-    if (e != cudaSuccess) return e;
+        // out-absorb: batch = heads, M = V, K = R split over a cluster; u[t][h*V + v] in bf16.
+        TailGemmArgs a{};
+        a.NP = NP;
+        a.N = nt;
+        a.n0 = n0;
+        a.k_total = L.R / TG_BK;
+        const int sa = fit_splits(
+            FA_TAIL_ABSORB_SPLITS > 0 ? FA_TAIL_ABSORB_SPLITS : (2 * num_sms) / (L.Hq * (L.V / TG_BM)), a.k_total);
+        a.ks = (a.k_total + sa - 1) / sa;
+        a.stages = stages;
+        a.ncols = ncols;
+        a.out = L.workspace;
+        a.ob = L.V;
+        a.on = (int64_t)L.Hq * L.V;
+        a.out_bf16 = 1;
+        a.pdl_trigger = FA_TAIL_PDL;
+        cudaError_t e = run_gemm(L.tmAbsA, L.tmAbsB, a, L.V / TG_BM, sa, L.Hq, false, stream);
+        if (e != cudaSuccess) return e;
 
-    // o-projection: M = Hd, K = Hq * V split over a cluster; y[t][j].
-    const int so = mla_tail_splits(L, num_sms);
-    TailGemmArgs b{};
-    b.NP = NP;
-    b.N = L.T;
-    b.k_total = L.Hq * L.V / TG_BK;
-    b.ks = (b.k_total + so - 1) / so;
-    b.stages = stages;
-    b.ncols = ncols;
-    b.out = L.y;
-    b.ob = 0;
-    b.on = L.Hd;
-    b.out_bf16 = L.y_bf16;
-    b.pdl_wait = FA_TAIL_PDL;
-    return run_gemm(L.tmOA, L.tmOB, b, L.Hd / TG_BM, so, 1, FA_TAIL_PDL != 0, stream);
+        // o-projection: M = Hd, K = Hq * V split over a cluster; y[t][j].
+        const int so = mla_tail_splits(L, num_sms);
+        TailGemmArgs b{};
+        b.NP = NP;
+        b.N = nt;
+        b.n0 = n0;
+        b.k_total = L.Hq * L.V / TG_BK;
+        b.ks = (b.k_total + so - 1) / so;
+        b.stages = stages;
+        b.ncols = ncols;
+        b.out = L.y;
+        b.ob = 0;
+        b.on = L.Hd;
+        b.out_bf16 = L.y_bf16;
+        b.pdl_wait = FA_TAIL_PDL;
+        e = run_gemm(L.tmOA, L.tmOB, b, L.Hd / TG_BM, so, 1, FA_TAIL_PDL != 0, stream);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
 }
 
 cudaError_t tail_device_error(int clear, int *code) {

@@ -339,7 +339,8 @@ typedef struct {
  *   workspace: at least fa_mla_tail_workspace_size() bytes (u), 256-byte
  *     aligned, overwritten on every call.
  * Supported: V == 128, R a positive multiple of 64, Hd a positive multiple
- * of 128, Hq * V a multiple of 64, T <= 256.  T == 0 is a no-op.
+ * of 128, Hq * V a multiple of 64.  Tokens run in chunks of up to 256 (the
+ * MMA's N).  T == 0 is a no-op.
  */
 typedef struct {
     const void *o_lat, *w_abs, *w_o;

@@ -202,7 +202,7 @@ def test_mla_tail_workspace_size_and_validation():
         assert lib.fa_mla_tail_workspace_size(ctypes.byref(tail_params(num_splits=ns)), ctypes.byref(n)) == fa.FA_OK
         assert n.value == 32 * 16384 * 2
     assert lib.fa_mla_tail(ctypes.byref(tail_params()), None) == fa.FA_ERR_WORKSPACE
-    for kw in (dict(V=64), dict(R=500), dict(Hd=7000), dict(T=257)):
+    for kw in (dict(V=64), dict(R=500), dict(Hd=7000)):
         assert lib.fa_mla_tail(ctypes.byref(tail_params(**kw)), None) == fa.FA_ERR_UNSUPPORTED, kw
     for kw in (dict(T=-1), dict(Hq=0), dict(y_dtype=5), dict(num_splits=-2), dict(w_o=40)):
         st = lib.fa_mla_tail(ctypes.byref(tail_params(workspace=256, workspace_bytes=1 << 30, **kw)), None)

@@ -32,9 +32,10 @@ def run(c, num_splits=0, out_dtype=torch.float32, rows=None):
     return y
 
 
-@pytest.mark.parametrize("T", [1, 5, 16, 32, 40, 129])
+@pytest.mark.parametrize("T", [1, 5, 16, 32, 40, 129, 256, 300, 530])
 def test_token_counts(T):
-    # T spans N = 16 .. 144 (padded to 16) and one or several 32-column reads.
+    # T spans N = 16 .. 256 (padded to 16), one or several 32-column reads,
+    # and more than 256 tokens (chunks of 256, the last one partly empty).
     run(W.MlaTailCase("t", T, 4, R=128, V=128, Hd=256, seed=T))
 
 
