@@ -381,9 +381,13 @@ fa_status fa_prefill_paged(const fa_prefill_paged_params *p, void *stream) {
                     "fa_prefill_paged: need B >= 0, Hq > 0, Hkv > 0, Sq >= 0, num_blocks > 0, max_blocks_per_seq > 0");
     if (p->Hq % p->Hkv != 0)
         return fail(FA_ERR_INVALID_ARG, "fa_prefill_paged: Hq (%d) %% Hkv (%d) != 0", p->Hq, p->Hkv);
-    if (p->dk != p->dv || (p->dk != 64 && p->dk != 128) || p->block_size != 64)
-        return fail(FA_ERR_UNSUPPORTED, "fa_prefill_paged: supported dk = dv in {64, 128}, block_size = 64 (got %d/%d/%d)",
-                    p->dk, p->dv, p->block_size);
+    const bool pair_ok = (p->dk == p->dv && (p->dk == 64 || p->dk == 128 || p->dk == 256)) ||
+                         (p->dk == 192 && (p->dv == 128 || p->dv == 192)) || (p->dk == 320 && p->dv == 256);
+    if (!pair_ok || p->block_size != 64)
+        return fail(FA_ERR_UNSUPPORTED,
+                    "fa_prefill_paged: supported (dk, dv) as fa_fwd, block_size = 64 (got %d/%d/%d)", p->dk, p->dv,
+                    p->block_size);
+    const bool two_tile = p->dk == p->dv && p->dk <= 128;
     if (!finite_pos(p->scale)) return fail(FA_ERR_INVALID_ARG, "fa_prefill_paged: scale must be finite and > 0");
     if (p->o_dtype != FA_F32 && p->o_dtype != FA_BF16) return fail(FA_ERR_INVALID_ARG, "fa_prefill_paged: o_dtype");
     if ((long long)p->B * p->Hq > 0x7fffffffLL || p->Sq > (1 << 30) ||
@@ -415,9 +419,11 @@ fa_status fa_prefill_paged(const fa_prefill_paged_params *p, void *stream) {
     st = encode_4d(&L.tmV, p->v_cache, p->dv, p->block_size, p->Hkv, p->num_blocks, p->dv, bs * p->dv,
                    bs * p->dv * p->Hkv, 64, "fa_prefill_paged v_cache");
     if (st != FA_OK) return st;
-    st = encode_4d(&L.tmO, p->o, p->dv, p->Sq, p->Hq, p->B, p->o_ss, p->o_sh, p->o_sb, 128, "fa_prefill_paged o",
-                   p->o_dtype == FA_F32 ? 4 : 2);
-    if (st != FA_OK) return st;
+    if (two_tile) {  // the two-tile kernel writes O with TMA stores
+        st = encode_4d(&L.tmO, p->o, p->dv, p->Sq, p->Hq, p->B, p->o_ss, p->o_sh, p->o_sb, 128, "fa_prefill_paged o",
+                       p->o_dtype == FA_F32 ? 4 : 2);
+        if (st != FA_OK) return st;
+    }
     L.B = p->B;
     L.Hq = p->Hq;
     L.Hkv = p->Hkv;
@@ -454,7 +460,7 @@ fa_status fa_prefill_paged(const fa_prefill_paged_params *p, void *stream) {
         L.mods.log2_m1 = -p->max_bias / 2.f / (float)n2;
     }
     L.has_mods = p->mask || p->softcap > 0.f || p->sinks;
-    if (p->mask) {
+    if (p->mask && two_tile) {
         // (keys, new rows, heads, batch) with rows m_ss long; stride-0 dims broadcast
         st = encode_4d(&L.tmM, p->mask, (int)(p->m_ss < (1 << 30) ? p->m_ss : (1 << 30)), p->Sq,
                        p->m_sh ? p->Hq : 1, p->m_sb ? p->B : 1, p->m_ss, p->m_sh ? p->m_sh : p->m_ss * p->Sq,
@@ -467,9 +473,14 @@ fa_status fa_prefill_paged(const fa_prefill_paged_params *p, void *stream) {
     L.q_lens = p->q_lens;
     L.max_blocks = p->max_blocks_per_seq;
     L.num_blocks = p->num_blocks;
-    int sms = 0;
-    cudaError_t e = num_sms(&sms);
-    if (e == cudaSuccess) e = fa::launch_prefill2(L, sms, static_cast<cudaStream_t>(stream));
+    cudaError_t e;
+    if (two_tile) {
+        int sms = 0;
+        e = num_sms(&sms);
+        if (e == cudaSuccess) e = fa::launch_prefill2(L, sms, static_cast<cudaStream_t>(stream));
+    } else {
+        e = fa::launch_prefill(L, static_cast<cudaStream_t>(stream));
+    }
     if (e != cudaSuccess) return cuda_fail(e, "fa_prefill_paged: launch");
     return FA_OK;
 }

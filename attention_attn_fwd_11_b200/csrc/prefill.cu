@@ -53,6 +53,10 @@ struct PrefillArgs {
     int64_t o_sb, o_sh, o_ss;
     int o_bf16;
     float *lse;
+    // Paged K/V (chunked prefill): block_table [B, max_blocks], seq_lens [B]
+    // and optional q_lens [B]; NULL block_table: dense K/V.
+    const int32_t *block_table, *seq_lens, *q_lens;
+    int max_blocks, num_blocks;
 };
 
 // DK: head dim of Q and K; DV: head dim of V and O.
@@ -110,13 +114,20 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const int hkv = hq / a.group;
     const int qt = a.causal ? (int)(gridDim.y - 1 - blockIdx.y) : (int)blockIdx.y;
     const int q0 = qt * C::BM;
+    // Keys and live query rows of this batch entry: Sk and Sq, or (paged) the
+    // sequence's clamped length and new-row count.
+    int Sk = a.Sk, Sq = a.Sq;
+    if (a.block_table) {
+        Sk = max(0, min(__ldg(a.seq_lens + b), a.max_blocks * 64));
+        if (a.q_lens) Sq = max(0, min(__ldg(a.q_lens + b), a.Sq));
+    }
 
     // KV tiles this query tile needs (causal: up to the last row's diagonal).
-    int n_tiles;
-    {
-        const int last_row = min(C::BM - 1, a.Sq - 1 - q0);
-        int kmax = a.Sk - 1;
-        if (a.causal) kmax = min(kmax, q0 + last_row + a.Sk - a.Sq);
+    int n_tiles = 0;
+    if (q0 < Sq) {
+        const int last_row = min(C::BM - 1, Sq - 1 - q0);
+        int kmax = Sk - 1;
+        if (a.causal) kmax = min(kmax, q0 + last_row + Sk - Sq);
         n_tiles = kmax < 0 ? 0 : kmax / BN + 1;
     }
 
@@ -157,20 +168,40 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             for (int c = 0; c < C::NCHK; ++c)
                 tma_load_4d(sQ + c * C::Q_CHUNK, &tmQ, bar(B_QFULL), c * 64, q0, hq, b);
             int issued_k = 0, issued_v = 0;
+            // Key tile t into a ring slot.  Dense: one BN-row box per 64-column
+            // chunk.  Paged: the tile's BN / 64 blocks, each a 64-row box per
+            // chunk, 8 KB apart in the chunk -- the layout one BN-row box
+            // gives under the 128-byte swizzle.  A block past the sequence's
+            // last re-reads the last (its keys are masked); an entry outside
+            // [0, num_blocks) is latched as FA_DEVERR_BAD_BLOCK, block 0 read.
+            auto load_tile = [&](uint32_t dst, const CUtensorMap *tm, uint32_t full, int nch, int t) {
+                if (a.block_table) {
+                    const int nblk = (Sk + 63) / 64;
+#pragma unroll
+                    for (int h = 0; h < BN / 64; ++h) {
+                        const int j = min(t * (BN / 64) + h, nblk - 1);
+                        int blk = __ldg(a.block_table + (int64_t)b * a.max_blocks + j);
+                        if (blk < 0 || blk >= a.num_blocks) {
+                            atomicCAS(&g_prefill_err, 0, 2 /* FA_DEVERR_BAD_BLOCK */);
+                            blk = 0;
+                        }
+                        for (int c = 0; c < nch; ++c)
+                            tma_load_4d(dst + c * C::KV_CHUNK + h * 8192, tm, full, c * 64, 0, hkv, blk);
+                    }
+                } else {
+                    for (int c = 0; c < nch; ++c) tma_load_4d(dst + c * C::KV_CHUNK, tm, full, c * 64, t * BN, hkv, b);
+                }
+            };
             for (int t = 0; t < n_tiles; ++t) {
                 const int s = t % NST;
                 const uint32_t ph = (uint32_t)(t / NST) & 1u;
                 if (!mbar_wait(k_empty(s), ph ^ 1u, abort_flag, &g_prefill_err)) break;
                 mbar_arrive_expect_tx(k_full(s), C::K_BYTES);
-#pragma unroll
-                for (int c = 0; c < C::NCHK; ++c)
-                    tma_load_4d(sK + s * C::K_BYTES + c * C::KV_CHUNK, &tmK, k_full(s), c * 64, t * BN, hkv, b);
+                load_tile(sK + s * C::K_BYTES, &tmK, k_full(s), C::NCHK, t);
                 issued_k = t + 1;
                 if (!mbar_wait(v_empty(s), ph ^ 1u, abort_flag, &g_prefill_err)) break;
                 mbar_arrive_expect_tx(v_full(s), C::V_BYTES);
-#pragma unroll
-                for (int c = 0; c < C::NCHV; ++c)
-                    tma_load_4d(sV + s * C::V_BYTES + c * C::KV_CHUNK, &tmV, v_full(s), c * 64, t * BN, hkv, b);
+                load_tile(sV + s * C::V_BYTES, &tmV, v_full(s), C::NCHV, t);
                 issued_v = t + 1;
             }
             if (*abort_flag) {
@@ -239,9 +270,12 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         const bool transform = MODS && (a.mods.mask != nullptr || a.mods.softcap != 0.f);
         const float c = transform ? 1.f : a.scale_log2;
         // keys j < lim_all are visible to this row
-        const int lim_all = a.causal ? min(a.Sk, qrow + a.Sk - a.Sq + 1) : a.Sk;
+        const int lim_all = qrow >= Sq ? 0 : (a.causal ? min(Sk, qrow + Sk - Sq + 1) : Sk);
         const float slope = MODS ? alibi_slope(a.mods, hq) : 1.f;
         const __half *mrow = MODS ? mask_row(a.mods, b, hq, qrow, a.Sq) : nullptr;
+        // mask values are read for keys below min(Sk, row length); later keys read as 0
+        const int mkeys = MODS && a.mods.mask ? (int)min((int64_t)Sk, (int64_t)a.mods.m_ss) : Sk;
+        (void)mkeys;
         (void)slope;
         (void)mrow;
         // l_run sums the fp32 weights (it gives the LSE); with modifiers l_o
@@ -268,7 +302,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             }
             const int lim = lim_all - t * BN;
             if (transform) {
-                modify_scores<BN>(x, a.mods, a.scale, slope, mrow, t * BN, a.Sk, lim);
+                modify_scores<BN>(x, a.mods, a.scale, slope, mrow, t * BN, mkeys, lim);
             } else if (lim < BN) {
 #pragma unroll
                 for (int i = 0; i < BN; ++i)
@@ -383,6 +417,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 }
             }
         }
+        if (qrow >= Sq) lse2 = -INFINITY;  // past the sequence's new rows: not a query (sinks aside)
         if (store && a.lse) a.lse[((int64_t)b * a.Hq + hq) * a.Sq + qrow] = lse2 * 0.69314718055994530942f;
     }
 
@@ -405,6 +440,11 @@ static cudaError_t launch_cfg(const PrefillLaunch &L, cudaStream_t stream) {
     a.group = L.Hq / L.Hkv;
     a.Sq = L.Sq;
     a.Sk = L.Sk;
+    a.block_table = L.block_table;
+    a.seq_lens = L.seq_lens;
+    a.q_lens = L.q_lens;
+    a.max_blocks = L.max_blocks;
+    a.num_blocks = L.num_blocks;
     a.scale = L.scale;
     a.scale_log2 = L.scale * 1.4426950408889634f;
     a.mods = L.mods;

@@ -306,14 +306,14 @@ def prefill_paged_params(q, k_cache, v_cache, block_table, seq_lens, o, lse, sca
 def prefill_paged(q, k_cache, v_cache, block_table, seq_lens, scale=None, causal=True, out=None,
                   return_lse=True, out_dtype=torch.float32, stream=None, q_lens=None, mask=None, max_bias=0.0,
                   softcap=0.0, sinks=None):
-    """Chunked prefill over a paged cache (fa_prefill_paged).  q [B,Hq,Sq,d]
-    bf16 (head dim contiguous); caches [num_blocks,Hkv,64,d] bf16
-    contiguous; block_table int32 [B,max_blocks]; seq_lens int32 [B] (keys
+    """Chunked prefill over a paged cache (fa_prefill_paged).  q [B,Hq,Sq,dk]
+    bf16 (head dim contiguous); k_cache [num_blocks,Hkv,64,dk], v_cache
+    [num_blocks,Hkv,64,dv] bf16 contiguous, (dk, dv) a pair fwd() takes; block_table int32 [B,max_blocks]; seq_lens int32 [B] (keys
     including the new ones); q_lens: None or int32 [B], new rows per
     sequence (rows past it come back as O = 0, LSE = -inf); mask [1|B, 1|Hq,
     Sq, >= max seq_len] float16 (last dim contiguous), max_bias, softcap,
     sinks [Hq] float32: the score modifiers of fwd().
-    Returns (O [B,Hq,Sq,d], LSE [B,Hq,Sq] or None)."""
+    Returns (O [B,Hq,Sq,dv], LSE [B,Hq,Sq] or None)."""
     _need_cuda(mask, sinks)
     if mask is not None and (mask.dtype != torch.float16 or mask.dim() != 4 or mask.stride(3) != 1):
         raise ValueError("mask must be a 4-D float16 tensor with a contiguous last dim")

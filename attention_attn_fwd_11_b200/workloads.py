@@ -273,8 +273,11 @@ class PagedPrefillCase:
     seed: int = 0
     scale: float = field(default=0.0)
     lens: tuple | None = None  # explicit per-sequence lengths (tests)
+    dv: int = 0  # head dim of V and O; 0: d (d is the head dim of Q and K)
 
     def __post_init__(self):
+        if not self.dv:
+            self.dv = self.d
         if not self.scale:
             self.scale = 1.0 / math.sqrt(self.d)
 
@@ -288,13 +291,14 @@ class PagedPrefillCase:
                 pairs += sum(max(0, lo + i) for i in range(self.Sq))
             else:
                 pairs += self.Sq * L
-        return 2.0 * self.Hq * 2 * self.d * pairs
+        return 2.0 * self.Hq * (self.d + self.dv) * pairs
 
 
 def paged_prefill_inputs(c: PagedPrefillCase):
-    """Returns q [B,Hq,Sq,d], k_cache/v_cache [nb,Hkv,bs,d] bf16, block_table
-    int32 [B, max_blocks] (-1 past the end), seq_lens int32 [B]."""
-    pc = PagedCase(c.name, c.B, c.Hq, c.Hkv, c.d, c.d, c.block_size, max(c.min_len, c.Sq), c.max_len, seed=c.seed,
+    """Returns q [B,Hq,Sq,d], k_cache [nb,Hkv,bs,d] and v_cache [nb,Hkv,bs,dv]
+    bf16, block_table int32 [B, max_blocks] (-1 past the end), seq_lens int32
+    [B]."""
+    pc = PagedCase(c.name, c.B, c.Hq, c.Hkv, c.d, c.dv, c.block_size, max(c.min_len, c.Sq), c.max_len, seed=c.seed,
                    lens=c.lens)
     _, kc, vc, table, lens = paged_inputs(pc)
     q = randn_bf16((c.B, c.Hq, c.Sq, c.d), 1000 + c.seed)

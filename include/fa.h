@@ -155,7 +155,7 @@ fa_status fa_fwd(const fa_fwd_params *p, void *stream);
  *   o: [B, Hq, Sq, dv] (o_dtype) with strides o_sb, o_sh, o_ss (multiples of
  *     4 elements for fp32, 8 for bf16; o_ss >= dv); lse: NULL or [B, Hq, Sq]
  *     fp32 contiguous.
- * Supported: dk == dv in {64, 128}, block_size == 64, Hq % Hkv == 0.
+ * Supported: the (dk, dv) pairs of fa_fwd, block_size == 64, Hq % Hkv == 0.
  * Score modifiers: as in fa_fwd (mask, max_bias, softcap, sinks), with the
  *   mask element (b, h, i, j) at b*m_sb + h*m_sh + i*m_ss + j for new row i
  *   and key j of the sequence (j < seq_lens[b]); m_ss must be >= every

@@ -159,8 +159,9 @@ def prefill_paged_params(**kw):
 
 
 @pytest.mark.parametrize("kw,status", [
-    (dict(dk=256, dv=256), fa.FA_ERR_UNSUPPORTED),
+    (dict(dk=96, dv=96), fa.FA_ERR_UNSUPPORTED),
     (dict(dk=128, dv=64), fa.FA_ERR_UNSUPPORTED),
+    (dict(dk=256, dv=128), fa.FA_ERR_UNSUPPORTED),
     (dict(block_size=16), fa.FA_ERR_UNSUPPORTED),
     (dict(Hq=30), fa.FA_ERR_INVALID_ARG),
     (dict(num_blocks=0), fa.FA_ERR_INVALID_ARG),

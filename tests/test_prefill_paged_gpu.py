@@ -13,8 +13,8 @@ from parity import check
 pytestmark = pytest.mark.gpu
 
 
-def run(B, Hq, Hkv, Sq, d, lens, causal, seed, out_dtype=torch.float32, seq_major=False, q_lens=None):
-    c = W.PagedPrefillCase("t", B, Hq, Hkv, Sq, d, 0, 0, causal=causal, seed=seed, lens=tuple(lens))
+def run(B, Hq, Hkv, Sq, d, lens, causal, seed, out_dtype=torch.float32, seq_major=False, q_lens=None, dv=0):
+    c = W.PagedPrefillCase("t", B, Hq, Hkv, Sq, d, 0, 0, causal=causal, seed=seed, lens=tuple(lens), dv=dv)
     q, kc, vc, table, sl = W.paged_prefill_inputs(c)
     qd = q.cuda()
     if seq_major:  # Q stored [B, Sq, Hq, d], viewed as [B, Hq, Sq, d]
@@ -28,7 +28,7 @@ def run(B, Hq, Hkv, Sq, d, lens, causal, seed, out_dtype=torch.float32, seq_majo
                                         causal, q_lens=q_lens)
     bf = out_dtype == torch.bfloat16
     check(o, o_ref, lse, l_ref, max_abs=2e-2 if bf else 1e-2, min_cos=0.9999 if bf else 0.99999,
-          what="paged prefill d%d Sq%d lens %s causal %d" % (d, Sq, list(lens), causal))
+          what="paged prefill d%d/%d Sq%d lens %s causal %d" % (d, c.dv, Sq, list(lens), causal))
 
 
 @pytest.mark.parametrize("d", [64, 128])
@@ -110,3 +110,54 @@ def test_score_modifiers(d):
                                         q_lens=ql.numpy(), mask=mask.numpy(), max_bias=4.0, softcap=6.0,
                                         sinks=sinks.double().numpy())
     check(o, o_ref, lse, l_ref, what="paged prefill with modifiers d%d" % d)
+
+
+# The one-tile kernel (head sizes above 128 and the asymmetric pairs): its
+# 64- or 128-key tiles are one or two cache blocks.
+PAIRS = [(256, 256), (192, 128), (192, 192), (320, 256)]
+
+
+@pytest.mark.parametrize("dk,dv", PAIRS)
+@pytest.mark.parametrize("causal", [False, True])
+def test_large_heads_ragged(dk, dv, causal):
+    # Sq = 200 spans two 128-row query tiles, the second partial; lengths end
+    # inside blocks, inside the second block of a 128-key tile, on a block
+    # edge, and below Sq; one sequence has no new row.
+    run(5, 8, 2, 200, dk, (200, 517, 1088, 64, 150), causal, seed=dk + dv, dv=dv, q_lens=(200, 1, 129, 64, 0))
+
+
+@pytest.mark.parametrize("dk,dv", [(256, 256), (192, 128)])
+def test_large_heads_short_sequences_bf16(dk, dv):
+    # all rows of a sequence with 0 keys are empty; 1 key: the 128-key
+    # tile's second block lies past the end
+    run(3, 4, 4, 40, dk, (17, 0, 1), True, seed=7, dv=dv, out_dtype=torch.bfloat16)
+
+
+@pytest.mark.parametrize("dk,dv", [(256, 256), (192, 128)])
+def test_large_heads_score_modifiers(dk, dv):
+    # mask with ALiBi, softcap and sinks through the one-tile kernel (the mask
+    # is read per row from global memory there)
+    c = W.PagedPrefillCase("t", 3, 8, 2, 130, dk, 0, 0, causal=True, seed=70 + dk, lens=(130, 517, 300), dv=dv)
+    q, kc, vc, table, sl = W.paged_prefill_inputs(c)
+    ql = torch.tensor([130, 77, 1], dtype=torch.int32)
+    mask = W.random_mask(3, 8, 130, 520, seed=71, scale=1.0)
+    sinks = W.random_sinks(8, seed=72)
+    o, lse = fa.prefill_paged(q.cuda(), kc.cuda(), vc.cuda(), table.cuda(), sl.cuda(), scale=c.scale, causal=True,
+                              q_lens=ql.cuda(), mask=mask.cuda(), max_bias=4.0, softcap=6.0, sinks=sinks.cuda())
+    torch.cuda.synchronize()
+    assert fa.device_error() == 0
+    o_ref, l_ref = oracle.prefill_paged(W.bits(q), W.bits(kc), W.bits(vc), table.numpy(), sl.numpy(), c.scale, True,
+                                        q_lens=ql.numpy(), mask=mask.numpy(), max_bias=4.0, softcap=6.0,
+                                        sinks=sinks.double().numpy())
+    check(o, o_ref, lse, l_ref, what="paged prefill with modifiers d%d/%d" % (dk, dv))
+
+
+def test_large_heads_bad_block_id_is_latched():
+    c = W.PagedPrefillCase("t", 2, 4, 2, 64, 256, 0, 0, seed=8, lens=(200, 100))
+    q, kc, vc, table, sl = W.paged_prefill_inputs(c)
+    bad = table.clone()
+    bad[0, 2] = -3
+    fa.prefill_paged(q.cuda(), kc.cuda(), vc.cuda(), bad.cuda(), sl.cuda(), causal=True)
+    torch.cuda.synchronize()
+    assert fa.device_error(clear=True) == 2  # FA_DEVERR_BAD_BLOCK
+    assert fa.device_error() == 0
