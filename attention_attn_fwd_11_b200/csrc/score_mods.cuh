@@ -57,16 +57,35 @@ FA_DEV float rcp_approx(float x) {
     return y;
 }
 
-// tanh(s) = 1 - 2 / (e^(2s) + 1), with e^(2s) from ex2: exact limits +-1 for
-// |s| large, absolute error of order 1e-7 elsewhere.  Two MUFU operations.
-FA_DEV float tanh_via_exp(float s) {
-    const float e = ex2(2.f * kLog2e * s);
-    return 1.f - 2.f * rcp_approx(e + 1.f);
-}
-
 // One 64-key chunk: raw scores x[0..64) (unscaled q.k) and the chunk's mask
 // values w (64 f16 in key order; all zero without a mask) -> base-2 scores
 // (modified score) * log2(e).
+// softcap * tanh(scale * x) * log2(e) for four raw scores x[0..4), as
+// tanh(u) = 1 - 2 / d with d = e^(2u) + 1.  One reciprocal serves the four:
+// r = 1 / (d0 d1 d2 d3), then 1 / d0 = r d1 d2 d3 and so on.  e^(2u) is
+// clamped to 2^30 (tanh is 1 in fp32 from about 2^26 on), so the product
+// stays below 2^121 and its reciprocal a normal number; each 1 / d carries a
+// few ulp of rounding.  MUFU work: four ex2 and one rcp for four scores.
+FA_DEV void softcap4(float *x, float scale, float softcap) {
+    const float k = 2.f * kLog2e * scale;
+    const uint64_t k2 = f2_pack(k, k), one2 = f2_pack(1.f, 1.f);
+    float a0, a1, a2, a3;
+    f2_unpack(f2_mul(f2_pack(x[0], x[1]), k2), a0, a1);
+    f2_unpack(f2_mul(f2_pack(x[2], x[3]), k2), a2, a3);
+    float d0, d1, d2, d3;
+    f2_unpack(f2_add(f2_pack(ex2(fminf(a0, 30.f)), ex2(fminf(a1, 30.f))), one2), d0, d1);
+    f2_unpack(f2_add(f2_pack(ex2(fminf(a2, 30.f)), ex2(fminf(a3, 30.f))), one2), d2, d3);
+    const float d01 = d0 * d1, d23 = d2 * d3;
+    const float r = rcp_approx(d01 * d23);
+    float r01, r23;  // 1 / (d0 d1), 1 / (d2 d3)
+    f2_unpack(f2_mul(f2_pack(r, r), f2_pack(d23, d01)), r01, r23);
+    const float c = softcap * kLog2e;
+    // softcap * log2(e) * (1 - 2 / d) = c - 2c / d
+    const uint64_t m2c = f2_pack(-2.f * c, -2.f * c), c2 = f2_pack(c, c);
+    f2_unpack(f2_fma(f2_mul(f2_pack(r01, r01), f2_pack(d1, d0)), m2c, c2), x[0], x[1]);
+    f2_unpack(f2_fma(f2_mul(f2_pack(r23, r23), f2_pack(d3, d2)), m2c, c2), x[2], x[3]);
+}
+
 FA_DEV void modify_chunk(float *x, const uint4 (&w)[8], const ScoreMods &m, float scale, float slope) {
     const float cs = scale * kLog2e;   // raw score -> base-2 units, without softcap
     const float cm = slope * kLog2e;   // mask value -> base-2 units
@@ -74,15 +93,17 @@ FA_DEV void modify_chunk(float *x, const uint4 (&w)[8], const ScoreMods &m, floa
 #pragma unroll
     for (int g = 0; g < 8; ++g) {
         const uint32_t mw[4] = {w[g].x, w[g].y, w[g].z, w[g].w};  // four f16 pairs
+        if (m.softcap != 0.f) {
+            softcap4(x + 8 * g, scale, m.softcap);
+            softcap4(x + 8 * g + 4, scale, m.softcap);
+        }
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const int k = 8 * g + 2 * j;
             const float2 mf = __half22float2(*reinterpret_cast<const __half2 *>(&mw[j]));
             uint64_t y;
-            if (m.softcap != 0.f) {
-                const float s0 = m.softcap * tanh_via_exp(x[k] * scale);
-                const float s1 = m.softcap * tanh_via_exp(x[k + 1] * scale);
-                y = f2_fma(f2_pack(mf.x, mf.y), cm2, f2_mul(f2_pack(s0, s1), f2_pack(kLog2e, kLog2e)));
+            if (m.softcap != 0.f) {  // x holds the capped score in base-2 units already
+                y = f2_fma(f2_pack(mf.x, mf.y), cm2, f2_pack(x[k], x[k + 1]));
             } else {
                 y = f2_fma(f2_pack(x[k], x[k + 1]), cs2, f2_mul(f2_pack(mf.x, mf.y), cm2));
             }
