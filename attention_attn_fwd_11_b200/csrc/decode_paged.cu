@@ -66,7 +66,10 @@ struct PdRaw {
     static constexpr int ROW = KVT == 8 ? 136 : 128;          // bytes per cache row of 128 values
     static constexpr int TILE = PD_BS * ROW;                  // one (block, head) tile of K or V
     static constexpr int STAGE = 2 * TILE;                    // K + V (1024-byte multiple)
-    static constexpr int NST = 4;
+    // Two raw stages keep the CTA at about 68 KB of shared memory, so three
+    // CTAs (twelve converting warps) share an SM: the in-warp conversion is
+    // latency-bound, and occupancy, not ring depth, feeds it.
+    static constexpr int NST = 2;
     static constexpr int WBUF = 2 * 16 * PD_D * 2;            // one warp's 16 keys of K and V in bf16: 8 KB
     static constexpr int OFF_WB = NST * STAGE;
     static constexpr int OFF_BAR = OFF_WB + 4 * WBUF;
@@ -109,8 +112,9 @@ struct PagedArgs {
     float *part_o, *part_lse;
 };
 
+// Quantised caches: three CTAs per SM (at most 136 registers a thread).
 template <int G, int KVT>
-__global__ void __launch_bounds__(160) paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
+__global__ void __launch_bounds__(160, KVT ? 3 : 1) paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                                                            const __grid_constant__ CUtensorMap tmV,
                                                            const PagedArgs a) {
     extern __shared__ uint8_t smem_raw[];
