@@ -59,18 +59,19 @@ NCU_TRAFFIC = {
     # dram__bytes_read.sum + dram__bytes_write.sum of one launch; the summary
     # under profiles/ named for the kernel and workload gives the capture.
     "causal_mha_b2_h16_s2048_d128": 54526208,
-    "gqa_full_b1_hq32_hkv8_s4096_d256": 215937536,
-    "causal_mha_mods_b2_h16_s2048_d128": 58235904,
+    "gqa_full_b1_hq32_hkv8_s4096_d256": 215944192,
+    "causal_mha_mods_b2_h16_s2048_d128": 58342656,
     "paged_gqa_b64_hq32_hkv8_d128_bs64": 1236853248,
-    "paged_gqa_q8_0kv_b64_hq32_hkv8_d128_bs64": 660243200,
+    "paged_gqa_q8_0kv_b64_hq32_hkv8_d128_bs64": 674241024,
     "latent_sparse_t32_hq128_dk576_dv512_top2048": 45249792,
-    "causal_mha_b2_h16_s2048_dk192_dv128": 73713408,
-    "causal_gqa_b2_hq16_hkv4_s2048_dk192_dv192": 40004096,
+    "causal_mha_b2_h16_s2048_dk192_dv128": 72717056,
+    "causal_gqa_b2_hq16_hkv4_s2048_dk192_dv192": 39777792,
     "kv_dequant causal_mha_q8_0kv_b2_h16_s2048_d128": 17835776,
     "kv_dequant causal_mha_fp8kv_b2_h16_s2048_d128": 16799744,
     "paged_prefill_gqa_b16_hq32_hkv8_sq512_d128_bs64": 651760896,
     "mla_tail_t32_hq128_r512_v128_hidden7168": 257049088,
-    "causal_gqa_b1_hq16_hkv4_s4096_dk320_dv256": 77931264,
+    "causal_gqa_b1_hq16_hkv4_s4096_dk320_dv256": 78919168,
+    "paged_gqa_fp8kv_b64_hq32_hkv8_d128_bs64": 636363776,
 }
 
 
