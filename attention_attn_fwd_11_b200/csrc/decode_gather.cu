@@ -19,7 +19,9 @@
 //     and latent [0, 256)), CTA 1 owns [320, 576).  Each CTA gathers ONLY
 //     its columns of every selected row -- exactly the columns its PV needs
 //     as well -- so each row is read from memory once per cluster and no
-//     score is computed twice.  Each CTA holds the matching part of Q.
+//     score is computed twice.  Each CTA holds the matching part of Q,
+//     which TMA brings into shared memory and the softmax warps copy into
+//     TMEM, the A operand of QK^T.
 //   - Partial scores (128 heads x 32 keys, fp32) are swapped through
 //     distributed shared memory every tile; both CTAs add own + peer (the
 //     same sum in either order), so both run the identical online softmax.
@@ -76,12 +78,19 @@ constexpr int LG_SMEM = LG_OFF_AUX + 1024 + 1024;
 // partial scores to the exchange before the softmax of tile i.
 constexpr int LG_NSB = FA_LG_NSB;
 constexpr int LG_T_O = LG_NSB * LG_BN;           // TMEM column of O (S buffers at 0, 32, 64)
+// Q of the CTA's columns in TMEM after O: 128 lanes (heads) x up to 320 bf16
+// = 160 columns, as the A operand of QK^T, which then reads only the 32 key
+// rows from shared memory.
+constexpr int LG_T_Q = LG_T_O + LG_HALF;
+static_assert(LG_T_Q + LG_NCH_MAX * 32 <= 512, "TMEM budget");
 static_assert(LG_SMEM <= 232448, "shared memory budget");
 
 enum {
     G_QFULL = 0, G_SFULL = 1, G_PREADY = 4, G_PVDONE = 7, G_DRAIN = 8, G_XFULL = 9, G_XFREE = 11, G_XOREADY = 13,
-    G_XOFREE = 15, G_XREAD = 17, G_FULL = 19, G_EMPTY = 19 + LG_NST, G_NBAR = 19 + 2 * LG_NST
+    G_XOFREE = 15, G_XREAD = 17, G_FULL = 19, G_EMPTY = 19 + LG_NST, G_QTMEM = 19 + 2 * LG_NST,
+    G_NBAR = G_QTMEM + 1
 };
+static_assert(G_NBAR <= 40, "barrier space");
 
 struct GatherArgs {
     const __nv_bfloat16 *rows;
@@ -132,6 +141,7 @@ latent_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const GatherArgs a
 
     if (threadIdx.x == 0) {
         mbar_init(bar(G_QFULL), 1);
+        mbar_init(bar(G_QTMEM), 128);  // softmax threads: Q rows are in TMEM
         mbar_init(bar(G_PVDONE), 1);
         mbar_init(bar(G_DRAIN), 1);
         for (int i = 0; i < LG_NSB; ++i) {
@@ -244,9 +254,8 @@ latent_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const GatherArgs a
                 const uint32_t tS = tmem + (uint32_t)((i % LG_NSB) * LG_BN);
                 for (int kk = 0; kk < nch * 4; ++kk) {
                     const int c = kk >> 2, sub = kk & 3;
-                    const uint64_t ad = sdesc_sw128(sQ + c * LG_QCH + sub * 32, 16, 1024);
                     const uint64_t bd = sdesc_sw128(sK + s * LG_KSTAGE + c * LG_KCH + sub * 32, 16, 1024);
-                    mma_ss(tS, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
+                    mma_ts(tS, tmem + (uint32_t)(LG_T_Q + kk * 8), bd, idesc_qk, kk > 0 ? 1u : 0u);
                 }
                 mma_commit(bar(G_SFULL + i % LG_NSB));
                 LG_TRACE(2, i);
@@ -254,7 +263,7 @@ latent_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const GatherArgs a
             };
             // QK^T runs NSB - 1 tiles ahead of PV: S buffer (i + NSB - 1) % NSB
             // held P of tile i - 1, which PV(i - 1) (issued before) consumed.
-            bool ok = mbar_wait(bar(G_QFULL), 0, abort_flag, &g_gather_err);
+            bool ok = mbar_wait(bar(G_QTMEM), 0, abort_flag, &g_gather_err);
             for (int j = 0; ok && j < LG_NSB - 1 && j < n_tiles; ++j) ok = issue_qk(j);
             for (int i = 0; ok && i < n_tiles; ++i) {
                 if (i + LG_NSB - 1 < n_tiles && !issue_qk(i + LG_NSB - 1)) break;
@@ -345,8 +354,33 @@ latent_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const GatherArgs a
             return true;
         };
         uint32_t r[32], rn[32];
+        bool qok = true;
+        // Q into TMEM: this thread's head row, 64 columns a chunk, read from
+        // the swizzled TMA tile (16-byte piece j of row h sits at slot
+        // j ^ (h & 7)); each 32-bit column holds two consecutive dims, the
+        // lower one in the low half -- the A-operand layout of the MMA.
+        if (n_tiles > 0) {
+            qok = mbar_wait(bar(G_QFULL), 0, abort_flag, &g_gather_err);
+            if (qok) {
+                for (int ch = 0; ch < nch; ++ch) {
+                    const uint4 *qrow = reinterpret_cast<const uint4 *>(smem + ch * LG_QCH + head * 128);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const uint4 w = qrow[j ^ (head & 7)];
+                        r[4 * j] = w.x;
+                        r[4 * j + 1] = w.y;
+                        r[4 * j + 2] = w.z;
+                        r[4 * j + 3] = w.w;
+                    }
+                    tmem_st32(tl + (uint32_t)(LG_T_Q + ch * 32), r);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(bar(G_QTMEM));
+            }
+        }
         constexpr bool kPipe = LG_NSB >= 3;
-        bool ok = !kPipe || n_tiles == 0 || send(0, r);
+        bool ok = qok && (!kPipe || n_tiles == 0 || send(0, r));
         for (int i = 0; ok && i < n_tiles; ++i) {
             const int buf = i & 1, s = i % LG_NST;
             const uint32_t ph = (uint32_t)(i >> 1) & 1u;
