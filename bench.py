@@ -63,7 +63,7 @@ NCU_TRAFFIC = {
     "causal_mha_mods_b2_h16_s2048_d128": 58342656,
     "paged_gqa_b64_hq32_hkv8_d128_bs64": 1236853248,
     "paged_gqa_q8_0kv_b64_hq32_hkv8_d128_bs64": 674241024,
-    "latent_sparse_t32_hq128_dk576_dv512_top2048": None,
+    "latent_sparse_t32_hq128_dk576_dv512_top2048": 45067264,
     "causal_mha_b2_h16_s2048_dk192_dv128": 72717056,
     "causal_gqa_b2_hq16_hkv4_s2048_dk192_dv192": 39777792,
     "kv_dequant causal_mha_q8_0kv_b2_h16_s2048_d128": 17835776,
