@@ -110,3 +110,32 @@ def test_modifiers_with_identity_table_equal_dense():
                                       mask=np.ascontiguousarray(mask[b:b + 1, :, :, :n]), max_bias=4.0, softcap=5.0,
                                       sinks=sinks)
         assert np.array_equal(o[b:b + 1], od) and np.array_equal(lse[b:b + 1], ld)
+
+
+@pytest.mark.parametrize("dk,dv", [(192, 128), (320, 256)])
+def test_identity_table_equals_dense_asymmetric_heads(dk, dv):
+    # K rows of dk and V rows of dv in separate caches: an identity table
+    # gives dense attention over the same keys; a dropped dv (V read with
+    # K's width) or K read with V's width would change the shapes or values.
+    B, Hkv, Hq, Sq, L = 2, 1, 2, 20, 100
+    nb = (L + 63) // 64
+    k = W.bits(W.randn_bf16((B, Hkv, nb * 64, dk), 21))
+    v = W.bits(W.randn_bf16((B, Hkv, nb * 64, dv), 22))
+    q = W.bits(W.randn_bf16((B, Hq, Sq, dk), 23))
+    kc = k.reshape(B, Hkv, nb, 64, dk).transpose(0, 2, 1, 3, 4).reshape(B * nb, Hkv, 64, dk).copy()
+    vc = v.reshape(B, Hkv, nb, 64, dv).transpose(0, 2, 1, 3, 4).reshape(B * nb, Hkv, 64, dv).copy()
+    table = np.arange(B * nb, dtype=np.int32).reshape(B, nb)
+    sl = np.array([L, L - 37], np.int32)
+    scale = 1.0 / np.sqrt(dk)
+    o, lse = oracle.prefill_paged(q, kc, vc, table, sl, scale, causal=True)
+    assert o.shape == (B, Hq, Sq, dv)
+    for b in range(B):
+        n = int(sl[b])
+        od, ld = oracle.attention(q[b:b + 1], k[b:b + 1, :, :n], v[b:b + 1, :, :n], scale, True)
+        assert np.array_equal(o[b:b + 1], od) and np.array_equal(lse[b:b + 1], ld)
+
+
+def test_workload_flops_count_dk_plus_dv():
+    # 2 Hq (dk + dv) per visible pair; full attention: Sq * L pairs per sequence
+    c = W.PagedPrefillCase("t", 2, 4, 2, 8, 192, 0, 0, causal=False, lens=(10, 20), dv=128)
+    assert c.flops(np.array([10, 20])) == 2.0 * 4 * (192 + 128) * 8 * 30
