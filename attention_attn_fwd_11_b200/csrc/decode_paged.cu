@@ -60,10 +60,10 @@ constexpr int PD_SMEM = PD_OFF_BAR + 128 + 1024;  // ring + barriers + 1024-byte
 // FP8 E4M3 caches take the same prologue with 128-byte rows (one byte per
 // value) and one fp32 scale per tensor (k_scale, v_scale).
 //
-// Raw-tile geometry per cache type KVT (8 = q8_0, 2 = fp8 e4m3):
+// Raw-tile geometry per cache type KVT (8 = q8_0, 4 = q4_0, 2 = fp8 e4m3):
 template <int KVT>
 struct PdRaw {
-    static constexpr int ROW = KVT == 8 ? 136 : 128;          // bytes per cache row of 128 values
+    static constexpr int ROW = KVT == 8 ? 136 : (KVT == 4 ? 72 : 128);  // bytes per cache row of 128 values
     static constexpr int TILE = PD_BS * ROW;                  // one (block, head) tile of K or V
     static constexpr int STAGE = 2 * TILE;                    // K + V (1024-byte multiple)
     // Two raw stages keep the CTA at about 68 KB of shared memory, so three
@@ -100,6 +100,18 @@ FA_DEV uint32_t q8_pair_to_bf16(uint32_t w, uint64_t d2) {
     const float f1 = __uint_as_float(0x4B000000u | (((w >> 8) & 0xffu) ^ 0x80u)) - 8388736.f;
     return pack_bf16x2(f0 * d, f1 * d);
 #endif
+}
+
+// Two 4-bit codes n0, n1 (bits 0-3 and 8-11 of x) -> the bf16 pair
+// d (n0 - 8), d (n1 - 8).  OR-ed into the mantissa of 2^23 a code gives
+// 2^23 + n exactly; subtracting 2^23 + 8 leaves n - 8, and the product with
+// d is exact in fp32 (4 + 11 significant bits), so the bf16 conversion is
+// the only rounding, as in the pre-pass.
+FA_DEV uint32_t q4_pair_to_bf16(uint32_t x, uint64_t d2) {
+    const uint64_t f = f2_pack(__uint_as_float(0x4B000000u | (x & 0xfu)), __uint_as_float(0x4B000000u | ((x >> 8) & 0xfu)));
+    float a, b;
+    f2_unpack(f2_mul(f2_add(f, f2_pack(-8388616.f, -8388616.f)), d2), a, b);
+    return pack_bf16x2(a, b);
 }
 
 struct PagedArgs {
@@ -273,6 +285,36 @@ __global__ void __launch_bounds__(160, KVT ? 3 : 1) paged_decode_kernel(const __
                     }
                     *reinterpret_cast<uint4 *>(wb + t * (2 * 16 * 128) + ((j ^ (lk & 7)) << 4)) =
                         make_uint4(outw[0], outw[1], outw[2], outw[3]);
+                }
+            }
+        } else if constexpr (KVT == 4) {
+            // lane (lk, h) converts row lk's half h (two q4_0 blocks of 18
+            // bytes, 64 values) of K and of V.  In a block, byte j holds value
+            // j in its low nibble and value j + 16 in its high nibble.
+            const int lk = lane >> 1, h = lane & 1;
+            const uint8_t *raw = smem + s * R::STAGE + (warp * 16 + lk) * R::ROW + 36 * h;
+            uint8_t *wb = smem + R::OFF_WB + warp * R::WBUF + h * (16 * 128) + lk * 128;
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {  // K, then V
+#pragma unroll
+                for (int qb = 0; qb < 2; ++qb) {
+                    const uint8_t *p = raw + t * R::TILE + 18 * qb;
+                    const float d = __half2float(*reinterpret_cast<const __half *>(p));
+                    const uint64_t d2 = f2_pack(d, d);
+                    const uint16_t *cw = reinterpret_cast<const uint16_t *>(p + 2);  // 8 byte pairs
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj) {
+                        // chunk jj of the block: values 8 jj .. 8 jj + 7 -- the
+                        // low nibbles of bytes 8 (jj & 1) .., high ones for jj >= 2
+                        const int j = 4 * qb + jj;
+                        const int sh = jj >= 2 ? 4 : 0;
+                        const uint16_t *cp = cw + 4 * (jj & 1);
+                        const uint4 v = make_uint4(q4_pair_to_bf16((uint32_t)cp[0] >> sh, d2),
+                                                   q4_pair_to_bf16((uint32_t)cp[1] >> sh, d2),
+                                                   q4_pair_to_bf16((uint32_t)cp[2] >> sh, d2),
+                                                   q4_pair_to_bf16((uint32_t)cp[3] >> sh, d2));
+                        *reinterpret_cast<uint4 *>(wb + t * (2 * 16 * 128) + ((j ^ (lk & 7)) << 4)) = v;
+                    }
                 }
             }
         } else if constexpr (KVT == 8) {
@@ -523,6 +565,7 @@ static cudaError_t launch_g(const PagedLaunch &L, const PagedArgs &a, int B, cud
 template <int G>
 static cudaError_t launch_gq(const PagedLaunch &L, const PagedArgs &a, int B, cudaStream_t stream) {
     return L.kv_type == 8   ? launch_g<G, 8>(L, a, B, stream)
+           : L.kv_type == 4 ? launch_g<G, 4>(L, a, B, stream)
            : L.kv_type == 2 ? launch_g<G, 2>(L, a, B, stream)
                             : launch_g<G, 0>(L, a, B, stream);
 }

@@ -145,9 +145,11 @@ fa_status check_paged(const fa_decode_paged_params *p) {
         return fail(FA_ERR_UNSUPPORTED, "fa_decode_paged: Hq / Hkv must be 1, 2, 4 or 8 (got %d)", g);
     if (!finite_pos(p->scale)) return fail(FA_ERR_INVALID_ARG, "fa_decode_paged: scale must be finite and > 0");
     if (p->o_dtype != FA_F32 && p->o_dtype != FA_BF16) return fail(FA_ERR_INVALID_ARG, "fa_decode_paged: o_dtype");
-    if (p->kv_type != FA_KV_BF16 && p->kv_type != FA_KV_Q8_0 && p->kv_type != FA_KV_FP8_E4M3)
+    if (p->kv_type != FA_KV_BF16 && p->kv_type != FA_KV_Q8_0 && p->kv_type != FA_KV_Q4_0 &&
+        p->kv_type != FA_KV_FP8_E4M3)
         return fail(FA_ERR_UNSUPPORTED,
-                    "fa_decode_paged: kv_type must be FA_KV_BF16, FA_KV_Q8_0 or FA_KV_FP8_E4M3 (got %d)", p->kv_type);
+                    "fa_decode_paged: kv_type must be FA_KV_BF16, FA_KV_Q8_0, FA_KV_Q4_0 or FA_KV_FP8_E4M3 (got %d)",
+                    p->kv_type);
     if (p->kv_type == FA_KV_FP8_E4M3 && (!isfinite(p->k_scale) || !isfinite(p->v_scale)))
         return fail(FA_ERR_INVALID_ARG, "fa_decode_paged: k_scale and v_scale must be finite");
     return FA_OK;
@@ -170,7 +172,7 @@ fa_status check_paged_ptrs(const fa_decode_paged_params *p) {
 // (128-byte swizzle, 64 x 64 boxes).
 fa_status encode_paged_caches(const fa_decode_paged_params *p, fa::PagedLaunch *L) {
     memset(L, 0, sizeof *L);
-    if (p->kv_type == FA_KV_Q8_0 || p->kv_type == FA_KV_FP8_E4M3) {  // bulk-copied raw tiles: no tensor maps
+    if (p->kv_type != FA_KV_BF16) {  // bulk-copied raw tiles: no tensor maps
         L->kv_type = p->kv_type;
         L->k_scale = p->k_scale;
         L->v_scale = p->v_scale;

@@ -217,6 +217,20 @@ def fwd(q, k, v, scale=None, causal=False, out=None, return_lse=True, out_dtype=
 
 # ------------------------------------------------------------- paged decode --
 
+def _paged_kv(q, v_cache, kv_type):
+    """(cache type, dv) of a paged cache: bf16 rows, or uint8 rows of q8_0
+    (34 bytes per 32 values), q4_0 (18) or fp8 e4m3 (32) -- told apart by
+    the row length against dk when kv_type is not given."""
+    if v_cache.dtype != torch.uint8:
+        return None, v_cache.shape[3]
+    if kv_type is None:
+        dk, r = q.shape[-1], v_cache.shape[3]
+        kv_type = {dk // 32 * 34: "q8_0", dk // 32 * 18: "q4_0", dk: "fp8_e4m3"}.get(r)
+        if kv_type is None:
+            raise ValueError("cannot tell the cache type from a row of %d bytes; pass kv_type" % r)
+    return kv_type, v_cache.shape[3] // KV_QUANT[kv_type][1] * 32
+
+
 def paged_params(q, k_cache, v_cache, block_table, seq_lens, o, lse, scale, num_splits, ws, kv_type=None,
                  k_scale=1.0, v_scale=1.0):
     B, Hq, dk = q.shape
@@ -225,12 +239,9 @@ def paged_params(q, k_cache, v_cache, block_table, seq_lens, o, lse, scale, num_
     p.q, p.k_cache, p.v_cache = _ptr(q), _ptr(k_cache), _ptr(v_cache)
     p.block_table, p.seq_lens = _ptr(block_table), _ptr(seq_lens)
     p.max_blocks_per_seq = block_table.shape[1]
-    dv = v_cache.shape[3]
-    if k_cache.dtype == torch.uint8:  # q8_0 rows (34 bytes per 32 values) or fp8 bytes
-        if kv_type is None:
-            kv_type = "fp8_e4m3" if v_cache.shape[3] % 34 else "q8_0"
+    kv_type, dv = _paged_kv(q, v_cache, kv_type)
+    if kv_type is not None:  # quantised rows, converted inside the kernel
         p.kv_type = KV_QUANT[kv_type][0]
-        dv = v_cache.shape[3] // 34 * 32 if kv_type == "q8_0" else v_cache.shape[3]
         p.k_scale, p.v_scale = k_scale, v_scale
     p.B, p.Hq, p.Hkv, p.dk, p.dv, p.block_size, p.num_blocks = B, Hq, Hkv, dk, dv, bs, nb
     p.scale = scale
@@ -253,17 +264,16 @@ def decode_paged(q, k_cache, v_cache, block_table, seq_lens, scale=None, num_spl
                  return_lse=True, out_dtype=torch.float32, workspace=None, stream=None, kv_type=None, k_scale=1.0,
                  v_scale=1.0):
     """Split-KV decode over a paged cache.  q [B,Hq,dk]; caches
-    [num_blocks,Hkv,block_size,d] bf16, or uint8 [...,136] of q8_0 rows, or
-    uint8 [...,128] of fp8 e4m3 bytes read as e4m3 * k_scale / v_scale
-    (dequantised in the kernel); block_table int32 [B,max_blocks];
-    seq_lens int32 [B].  Returns (O [B,Hq,dv], LSE [B,Hq] or None)."""
+    [num_blocks,Hkv,block_size,d] bf16, or uint8 [...,136] of q8_0 rows,
+    [...,72] of q4_0 rows, or [...,128] of fp8 e4m3 bytes read as
+    e4m3 * k_scale / v_scale (dequantised in the kernel); block_table int32
+    [B,max_blocks]; seq_lens int32 [B].  Returns (O [B,Hq,dv], LSE [B,Hq] or
+    None)."""
     _need_cuda(q, k_cache, v_cache, block_table, seq_lens)
     B, Hq, dk = q.shape
     if scale is None:
         scale = 1.0 / math.sqrt(dk)
-    if v_cache.dtype == torch.uint8 and kv_type is None:
-        kv_type = "fp8_e4m3" if v_cache.shape[3] % 34 else "q8_0"
-    dv = v_cache.shape[3] // 34 * 32 if kv_type == "q8_0" else v_cache.shape[3]
+    kv_type, dv = _paged_kv(q, v_cache, kv_type)
     if out is None:
         out = torch.empty((B, Hq, dv), device=q.device, dtype=out_dtype)
     lse = torch.empty((B, Hq), device=q.device, dtype=torch.float32) if return_lse else None

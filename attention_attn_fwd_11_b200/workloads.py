@@ -236,12 +236,26 @@ def paged_q8_caches(c: PagedCase, num_blocks: int):
     return kq, vq
 
 
-def paged_bytes(c: PagedCase, seq_lens, max_blocks: int, q8: bool = False, fp8: bool = False) -> int:
+def paged_q4_caches(c: PagedCase, num_blocks: int):
+    """q4_0 K and V caches [num_blocks, Hkv, block_size, dk / 32 * 18] uint8
+    for the same pool (seeds 7000 + c and 7100 + c)."""
+    kq = random_quant_rows((num_blocks, c.Hkv, c.block_size), c.dk, "q4_0", c.seed)
+    vq = random_quant_rows((num_blocks, c.Hkv, c.block_size), c.dv, "q4_0", c.seed + 100)
+    return kq, vq
+
+
+def paged_bytes(c: PagedCase, seq_lens, max_blocks: int, q8: bool = False, fp8: bool = False,
+                q4: bool = False) -> int:
     """Algorithmic HBM bytes of one paged decode: every visible K/V element
-    once (2 bytes, 34 / 32 for q8_0 rows, 1 for fp8), the used block-table
-    entries, lengths, Q, fp32 O and LSE."""
+    once (2 bytes, 34 / 32 for q8_0 rows, 18 / 32 for q4_0, 1 for fp8), the
+    used block-table entries, lengths, Q, fp32 O and LSE."""
     sl = [int(x) for x in seq_lens]
-    per = (c.dk + c.dv) // 32 * 34 if q8 else ((c.dk + c.dv) if fp8 else (c.dk + c.dv) * 2)
+    if q8:
+        per = (c.dk + c.dv) // 32 * 34
+    elif q4:
+        per = (c.dk + c.dv) // 32 * 18
+    else:
+        per = (c.dk + c.dv) if fp8 else (c.dk + c.dv) * 2
     kv = sum(sl) * c.Hkv * per
     tbl = sum((n + c.block_size - 1) // c.block_size for n in sl) * 4
     return kv + tbl + c.B * 4 + c.B * c.Hq * c.dk * 2 + c.B * c.Hq * c.dv * 4 + c.B * c.Hq * 4
@@ -250,6 +264,7 @@ def paged_bytes(c: PagedCase, seq_lens, max_blocks: int, q8: bool = False, fp8: 
 PAGED_GQA = PagedCase("paged_gqa_b64_hq32_hkv8_d128_bs64", 64, 32, 8, 128, 128, 64, 1024, 8192, seed=4)
 PAGED_Q8_NAME = "paged_gqa_q8_0kv_b64_hq32_hkv8_d128_bs64"  # the same decode over q8_0 caches
 PAGED_FP8_NAME = "paged_gqa_fp8kv_b64_hq32_hkv8_d128_bs64"  # ... and over fp8 e4m3 caches
+PAGED_Q4_NAME = "paged_gqa_q4_0kv_b64_hq32_hkv8_d128_bs64"  # ... and over q4_0 caches
 
 
 # ----------------------------------------------------------- paged prefill --

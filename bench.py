@@ -72,6 +72,7 @@ NCU_TRAFFIC = {
     "mla_tail_t32_hq128_r512_v128_hidden7168": 257049088,
     "causal_gqa_b1_hq16_hkv4_s4096_dk320_dv256": 78919168,
     "paged_gqa_fp8kv_b64_hq32_hkv8_d128_bs64": 636363776,
+    "paged_gqa_q4_0kv_b64_hq32_hkv8_d128_bs64": 356117760,
 }
 
 
@@ -381,16 +382,18 @@ def latent_prefill_workload(torch, fa, W_, c, l2):
     return launch, n, c.flops, 2
 
 
-def paged_workload(torch, fa, W_, c, l2, q8=False, fp8=False):
-    """Paged decode (decode kernel + LSE combine per step); q8 / fp8: the
-    caches hold q8_0 rows or fp8 e4m3 bytes, converted inside the decode
-    kernel."""
+def paged_workload(torch, fa, W_, c, l2, q8=False, fp8=False, q4=False):
+    """Paged decode (decode kernel + LSE combine per step); q8 / q4 / fp8:
+    the caches hold q8_0 rows, q4_0 rows or fp8 e4m3 bytes, converted inside
+    the decode kernel."""
     q0, kc0, vc0, tb0, sl0 = W_.paged_inputs(c)
     if q8:
         kc0, vc0 = W_.paged_q8_caches(c, kc0.shape[0])
+    elif q4:
+        kc0, vc0 = W_.paged_q4_caches(c, kc0.shape[0])
     elif fp8:
         kc0, vc0 = W_.paged_fp8_caches(c, kc0.shape[0])
-    byts = W_.paged_bytes(c, sl0, tb0.shape[1], q8=q8, fp8=fp8)
+    byts = W_.paged_bytes(c, sl0, tb0.shape[1], q8=q8, fp8=fp8, q4=q4)
     foot = (kc0.numel() + vc0.numel()) * kc0.element_size()
     n = rotation_copies(foot, l2)
     import ctypes
@@ -536,6 +539,7 @@ def run_only(args):
                                  W_.QUANT_C2, W_.PAGED_PREFILL, W_.MLA_TAIL)}
     table[W_.PAGED_Q8_NAME] = W_.PAGED_GQA
     table[W_.PAGED_FP8_NAME] = W_.PAGED_GQA
+    table[W_.PAGED_Q4_NAME] = W_.PAGED_GQA
     table[W_.LATENT_PREFILL.name] = W_.LATENT_PREFILL
     table[W_.LATENT_PREFILL_512.name] = W_.LATENT_PREFILL_512
     table["kv_dequant_" + W_.QUANT_C2.name] = W_.QUANT_C2
@@ -563,7 +567,7 @@ def run_only(args):
         unit, amount = "TFLOP/s", work / 1e12
     elif isinstance(c, W_.PagedCase):
         launch, n, work, kpl = paged_workload(torch, fa, W_, c, l2, q8=args.only == W_.PAGED_Q8_NAME,
-                                              fp8=args.only == W_.PAGED_FP8_NAME)
+                                              fp8=args.only == W_.PAGED_FP8_NAME, q4=args.only == W_.PAGED_Q4_NAME)
         unit, amount = "GB/s", work / 1e9
     else:
         launch, n, work, kpl = latent_workload(torch, fa, W_, c, l2)
@@ -784,7 +788,8 @@ def main():
         result["gpu_launches"] += st2 * kpl
         del launch
         # the same decode over q8_0 caches (dequant prologue in the kernel)
-        for qname, qkw in ((W_.PAGED_Q8_NAME, dict(q8=True)), (W_.PAGED_FP8_NAME, dict(fp8=True))):
+        for qname, qkw in ((W_.PAGED_Q8_NAME, dict(q8=True)), (W_.PAGED_Q4_NAME, dict(q4=True)),
+                           (W_.PAGED_FP8_NAME, dict(fp8=True))):
             launch, ncopy, byts, kpl = paged_workload(torch, fa, W_, pc, l2, **qkw)
             ms2, st2 = time_graph(torch, launch, ncopy, Ks, Wm, dist)
             ms2 = max_over_ranks(torch, dist, ms2)
@@ -794,8 +799,8 @@ def main():
                          "unit": "GB/s", "ms_per_step": round(per, 5), "steps": st2, "l2_copies": ncopy,
                          "bytes_per_step": byts,
                          "roofline": roofline("hbm", ach, peaks["hbm_gbs"], "GB/s", NCU_TRAFFIC.get(qname)),
-                         "kernels": "paged decode with the %s prologue + LSE combine" % ("q8_0" if "q8" in qkw else
-                                                                                         "fp8 e4m3")}
+                         "kernels": "paged decode with the %s prologue + LSE combine" % (
+                             "q8_0" if "q8" in qkw else ("q4_0" if "q4" in qkw else "fp8 e4m3"))}
             result["gpu_launches"] += st2 * kpl
             del launch
         try:

@@ -203,6 +203,9 @@ fa_status fa_prefill_paged(const fa_prefill_paged_params *p, void *stream);
  *     [num_blocks, Hkv, block_size, 136] bytes.  The kernel converts each
  *     tile in shared memory (the same single rounding to bf16 as
  *     fa_kv_dequant), so the cache is read once, at 1.06 bytes per value.
+ *     With kv_type FA_KV_Q4_0: dk / 32 ggml q4_0 blocks per row (18 bytes
+ *     each, layout as in fa_kv_dequant: 72 bytes for 128 values),
+ *     [num_blocks, Hkv, block_size, 72] bytes, converted the same way.
  *     With kv_type FA_KV_FP8_E4M3: OCP E4M3 bytes [num_blocks, Hkv,
  *     block_size, 128], value = e4m3 * k_scale (K) or * v_scale (V), formed
  *     in fp32 and converted to bf16 in the kernel (two roundings where
@@ -220,7 +223,7 @@ fa_status fa_prefill_paged(const fa_prefill_paged_params *p, void *stream);
  * Supported: dk == dv == 128, block_size == 64, Hq / Hkv in {1, 2, 4, 8}.
  * Cache slots past seq_lens[b] inside the sequence's last block are read and
  * must hold finite values (their weight is zero, and 0 * NaN is NaN; for
- * q8_0 their scales must be finite).
+ * q8_0 and q4_0 their scales must be finite).
  * A block id outside [0, num_blocks) is latched as FA_DEVERR_BAD_BLOCK and
  * block 0 is read in its place (the output for that sequence is then
  * meaningless).
@@ -239,7 +242,7 @@ typedef struct {
     int o_dtype; /* fa_dtype */
     void *workspace;
     size_t workspace_bytes;
-    int kv_type; /* FA_KV_BF16 (0), FA_KV_Q8_0 or FA_KV_FP8_E4M3 */
+    int kv_type; /* FA_KV_BF16 (0), FA_KV_Q8_0, FA_KV_Q4_0 or FA_KV_FP8_E4M3 */
     float k_scale, v_scale; /* FA_KV_FP8_E4M3: the caches' tensor scales (finite) */
 } fa_decode_paged_params;
 

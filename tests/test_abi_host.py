@@ -113,6 +113,25 @@ def test_paged_workspace_size_and_validation():
     assert lib.fa_decode_paged(ctypes.byref(paged_params(B=0)), None) == fa.FA_OK
 
 
+@pytest.mark.parametrize("kv_type,status", [(0, 0), (8, 0), (4, 0), (2, 0), (5, None), (1, None)])
+def test_paged_cache_types(kv_type, status):
+    # bf16, q8_0, q4_0 and fp8 caches pass the shape check; other codes are unsupported
+    n = ctypes.c_size_t(0)
+    st = fa.load().fa_decode_paged_workspace_size(ctypes.byref(paged_params(kv_type=kv_type)), ctypes.byref(n))
+    assert st == (fa.FA_OK if status == 0 else fa.FA_ERR_UNSUPPORTED)
+
+
+def test_paged_kv_type_from_row_length():
+    import torch
+    q = torch.empty(2, 4, 128, dtype=torch.bfloat16)
+    for width, name in ((136, "q8_0"), (72, "q4_0"), (128, "fp8_e4m3")):
+        v = torch.empty(3, 2, 64, width, dtype=torch.uint8)
+        assert fa._paged_kv(q, v, None) == (name, 128)
+    assert fa._paged_kv(q, torch.empty(3, 2, 64, 128, dtype=torch.bfloat16), None) == (None, 128)
+    with pytest.raises(ValueError):
+        fa._paged_kv(q, torch.empty(3, 2, 64, 100, dtype=torch.uint8), None)
+
+
 def gather_params(**kw):
     p = fa.GatherParams()
     base = dict(q=16, kv_rows=32, n_rows=65536, row_stride=576, dk=576, dv=512, v_offset=64, idx=48, topk=2048,

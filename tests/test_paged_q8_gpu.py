@@ -83,3 +83,43 @@ def test_fp8_caches(g):
     vb = oracle.dequant_rows(vf.numpy(), "fp8_e4m3", 128, scale=vs)
     o_ref, l_ref = oracle.decode_paged(W.bits(q), kb, vb, table.numpy(), sl.numpy(), c.scale)
     check(o, o_ref, lse, l_ref, what="fp8 paged decode g%d" % g)
+
+
+def run_q4(B, Hq, Hkv, lens, seed, num_splits=0, out_dtype=torch.float32):
+    c = W.PagedCase("t", B, Hq, Hkv, 128, 128, 64, 1, 1, seed=seed, lens=tuple(lens))
+    q, _, _, table, sl = W.paged_inputs(c)
+    nb = max(1, int(sum((n + 63) // 64 for n in lens)))
+    kq, vq = W.paged_q4_caches(c, nb)
+    assert kq.shape[-1] == 72
+    o, lse = fa.decode_paged(q.cuda(), kq.cuda(), vq.cuda(), table.cuda(), sl.cuda(), scale=c.scale,
+                             num_splits=num_splits, out_dtype=out_dtype)
+    torch.cuda.synchronize()
+    assert fa.device_error() == 0
+    kb = oracle.dequant_rows(kq.numpy(), "q4_0", 128)
+    vb = oracle.dequant_rows(vq.numpy(), "q4_0", 128)
+    o_ref, l_ref = oracle.decode_paged(W.bits(q), kb, vb, table.numpy(), sl.numpy(), c.scale)
+    bf = out_dtype == torch.bfloat16
+    check(o, o_ref, lse, l_ref, max_abs=2e-2 if bf else 1e-2, min_cos=0.9999 if bf else 0.99999,
+          what="q4_0 paged decode lens %s" % (list(lens),))
+    return c, q, kq, vq, table, sl, o, lse
+
+
+@pytest.mark.parametrize("g", [1, 2, 4, 8])
+def test_q4_caches_group_sizes(g):
+    run_q4(5, 2 * g, 2, (1, 63, 64, 65, 1000), seed=40 + g)
+
+
+def test_q4_caches_splits_bf16_output_zero_length():
+    run_q4(4, 16, 4, (0, 3000, 129, 64 * 9 + 5), seed=50, num_splits=3, out_dtype=torch.bfloat16)
+
+
+def test_q4_prologue_equals_bf16_caches_from_the_pre_pass():
+    # The prologue rounds d * (n - 8) to bf16 once, like the pre-pass, and the
+    # MMA path after it is the bf16 one: decoding the q4_0 caches equals
+    # decoding their pre-pass output, bit for bit.
+    c, q, kq, vq, table, sl, o, lse = run_q4(3, 8, 2, (700, 64, 1), seed=60)
+    kb = fa.kv_dequant(kq.cuda(), "q4_0", 128)
+    vb = fa.kv_dequant(vq.cuda(), "q4_0", 128)
+    o2, l2 = fa.decode_paged(q.cuda(), kb, vb, table.cuda(), sl.cuda(), scale=c.scale)
+    torch.cuda.synchronize()
+    assert torch.equal(o, o2) and torch.equal(lse, l2)
