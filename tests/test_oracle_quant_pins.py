@@ -154,3 +154,17 @@ def test_fp8_rows_scaled_round_once():
     # a scale whose product needs rounding: 1 + 2^-8 rounds to 1 (ties to even)
     one = np.full((1, 32), 0x38, np.uint8)
     assert np.all(oracle.dequant_rows(one, "fp8_e4m3", 32, scale=1.0 + 2.0 ** -8) == 0x3F80)
+
+
+def test_paged_cache_bytes_per_value():
+    # algorithmic K/V bytes of the paged decode lines: 2 per value for bf16,
+    # 34 / 32 for q8_0, 18 / 32 for q4_0, 1 for fp8 (plus the same table, Q,
+    # O and LSE bytes in every case)
+    from attention_attn_fwd_11_b200 import workloads as W
+    c = W.PagedCase("t", 2, 4, 2, 128, 128, 64, 1, 1, lens=(100, 30))
+    lens = [100, 30]
+    base = W.paged_bytes(c, lens, 2) - 130 * 2 * 256 * 2
+    for kw, per_value in ((dict(), 2.0), (dict(q8=True), 34 / 32), (dict(q4=True), 18 / 32), (dict(fp8=True), 1.0)):
+        assert W.paged_bytes(c, lens, 2, **kw) - base == 130 * 2 * 256 * per_value
+    # the q4_0 rows the decode takes are 72 bytes for 128 values
+    assert W.random_quant_rows((1, 1, 2), 128, "q4_0", 0).shape[-1] == 72
