@@ -13,11 +13,11 @@ same run and reported under "workloads":
 - the (192,128), (192,192) and (320,256) head-size pairs;
 - prefill over q8_0 K/V (the pre-pass plus prefill);
 - chunked prefill over the paged cache;
-- paged GQA decode, over bf16 and over q8_0 caches;
+- paged GQA decode, over bf16, q8_0, q4_0 and FP8 E4M3 caches;
 - latent sparse decode;
 - the MLA decode tail.
-More workloads run alone with --only NAME (FP8 K/V, the dequant kernels,
-latent prefill).
+More workloads run alone with --only NAME (prefill over FP8 K/V, the
+dequant kernels, latent prefill).
 
 Timing: inputs already resident in HBM; several copies of every input are
 rotated so that consecutive steps never find their operands in L2; steps are
