@@ -532,7 +532,7 @@ cudaError_t launch_decode_gather(const GatherLaunch &L, cudaStream_t stream) {
     latent_decode_kernel<<<grid, 320, LG_SMEM, stream>>>(L.tmQ, a);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    return launch_combine(L.part_o, L.part_lse, L.T * L.Hq, L.num_splits, L.Hq, nullptr, 0, L.o, L.lse, L.o_bf16,
+    return launch_combine(L.part_o, L.part_lse, L.T * L.Hq, L.num_splits, L.Hq, nullptr, 0, 0, L.o, L.lse, L.o_bf16,
                           LG_DV, stream);
 }
 

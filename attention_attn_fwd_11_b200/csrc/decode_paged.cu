@@ -122,6 +122,11 @@ struct PagedArgs {
     int max_blocks, Hq, Hkv, num_blocks, bps, num_splits;
     float scale_log2;
     float *part_o, *part_lse;
+    unsigned long long wait_ns;  // bound of every pipeline wait (kWaitLimitNs unless a test passes less)
+    // Test of the timeout path: the consumer warps first wait on a barrier
+    // that nothing ever completes, so that wait runs out after wait_ns, the
+    // CTA aborts, drains its copies and returns with FA_DEVERR_TIMEOUT latched.
+    int stall;
 };
 
 // Quantised caches: three CTAs per SM (at most 136 registers a thread).
@@ -155,6 +160,8 @@ __global__ void __launch_bounds__(160, KVT ? 3 : 1) paged_decode_kernel(const __
     auto full = [&](int s) { return bar0 + 8u * s; };
     auto empty = [&](int s) { return bar0 + 8u * (NST + s); };
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_BAR + 8 * 2 * NST);
+    const uint32_t stall_bar = bar0 + 8u * (2 * NST + 1);  // a.stall only: never arrived on
+    const unsigned long long wait_ns = a.wait_ns;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -162,6 +169,7 @@ __global__ void __launch_bounds__(160, KVT ? 3 : 1) paged_decode_kernel(const __
             mbar_init(full(s), 1);
             mbar_init(empty(s), 4);
         }
+        mbar_init(stall_bar, 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -188,7 +196,7 @@ __global__ void __launch_bounds__(160, KVT ? 3 : 1) paged_decode_kernel(const __
             const int s = i % NST;
             const uint32_t ph = (uint32_t)(i / NST) & 1u;
             bool ok = true;
-            if (lane == 0) ok = mbar_wait(empty(s), ph ^ 1u, abort_flag, &g_decode_err);
+            if (lane == 0) ok = mbar_wait(empty(s), ph ^ 1u, abort_flag, &g_decode_err, wait_ns);
             if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
             if (lane == 0) {
                 if constexpr (KVQ) {
@@ -242,10 +250,11 @@ __global__ void __launch_bounds__(160, KVT ? 3 : 1) paged_decode_kernel(const __
     // ldmatrix lane roles: matrix mi = lane / 8, row lr = lane % 8
     const int mi = lane >> 3, lr = lane & 7;
 
-    bool ok = true;
-    for (int i = 0; i < nblk; ++i) {
+    // a.stall: the wait that runs out (nothing arrives on stall_bar)
+    bool ok = !a.stall || mbar_wait(stall_bar, 0, abort_flag, &g_decode_err, wait_ns);
+    for (int i = 0; ok && i < nblk; ++i) {
         const int s = i % NST;
-        if (!mbar_wait(full(s), (uint32_t)(i / NST) & 1u, abort_flag, &g_decode_err)) {
+        if (!mbar_wait(full(s), (uint32_t)(i / NST) & 1u, abort_flag, &g_decode_err, wait_ns)) {
             ok = false;
             break;
         }
@@ -467,6 +476,7 @@ struct CombineArgs {
     // sequence length, gather mode uses every split.
     const int32_t *seq_lens;
     int bps;
+    int max_blocks;  // paged mode: the decode kernel reads at most this many blocks of a sequence
     void *o;
     float *lse;
     int o_bf16;
@@ -481,7 +491,9 @@ __global__ void __launch_bounds__(128) lse_combine_kernel(const CombineArgs a) {
     if (a.seq_lens) {
         int sl = a.seq_lens[row / a.Hq];
         if (sl < 0) sl = 0;
-        const int nb = (sl + PD_BS - 1) / PD_BS;
+        // capped as in paged_decode_kernel (a longer sequence latches
+        // FA_DEVERR_BAD_BLOCK there): splits past the cap write nothing
+        const int nb = min((sl + PD_BS - 1) / PD_BS, a.max_blocks);
         ns = min(ns, (nb + a.bps - 1) / a.bps);
     }
     const float *pl = a.part_lse + (int64_t)row * a.num_splits;
@@ -528,9 +540,10 @@ __global__ void __launch_bounds__(128) lse_combine_kernel(const CombineArgs a) {
 }
 
 cudaError_t launch_combine(const float *part_o, const float *part_lse, int rows, int num_splits, int Hq,
-                           const int32_t *seq_lens, int bps, void *o, float *lse, int o_bf16, int D,
+                           const int32_t *seq_lens, int bps, int max_blocks, void *o, float *lse, int o_bf16, int D,
                            cudaStream_t stream) {
     CombineArgs c;
+    c.max_blocks = max_blocks;
     c.part_o = part_o;
     c.part_lse = part_lse;
     c.rows = rows;
@@ -588,6 +601,8 @@ cudaError_t launch_decode_paged(const PagedLaunch &L, cudaStream_t stream) {
     a.scale_log2 = L.scale * 1.4426950408889634f;
     a.part_o = L.part_o;
     a.part_lse = L.part_lse;
+    a.wait_ns = L.wait_ns ? L.wait_ns : kWaitLimitNs;
+    a.stall = L.stall;
     cudaError_t e;
     switch (L.Hq / L.Hkv) {
         case 1: e = launch_gq<1>(L, a, L.B, stream); break;
@@ -597,8 +612,8 @@ cudaError_t launch_decode_paged(const PagedLaunch &L, cudaStream_t stream) {
         default: return cudaErrorInvalidValue;
     }
     if (e != cudaSuccess) return e;
-    return launch_combine(L.part_o, L.part_lse, L.B * L.Hq, L.num_splits, L.Hq, L.seq_lens, L.blocks_per_split, L.o,
-                          L.lse, L.o_bf16, PD_D, stream);
+    return launch_combine(L.part_o, L.part_lse, L.B * L.Hq, L.num_splits, L.Hq, L.seq_lens, L.blocks_per_split,
+                          L.max_blocks_per_seq, L.o, L.lse, L.o_bf16, PD_D, stream);
 }
 
 // ----------------------------------------------------------------------------
@@ -607,8 +622,11 @@ cudaError_t launch_decode_paged(const PagedLaunch &L, cudaStream_t stream) {
 // caller-supplied workspace.  It is a file-scope device array, so every GPU
 // that loads the library holds these bytes until the process exits.  All
 // calls share it and it keeps whatever the previous call wrote; nothing in it
-// needs to start at zero (each call writes every partial its combine reads),
-// but two such calls running on the GPU at the same time race on it.
+// needs to start at zero (each call writes every partial its combine reads:
+// the combine counts a sequence's splits from the same capped block count as
+// the decode kernel), but two such calls running on the GPU at the same time
+// race on it.  The device address is cached per device; a cudaDeviceReset
+// (which unloads the module) makes the cached address stale.
 constexpr size_t kPagedStaticScratchBytes = size_t(8) << 20;  // 8 MiB
 static __device__ __align__(256) unsigned char g_paged_scratch[kPagedStaticScratchBytes];
 

@@ -119,17 +119,27 @@ cudaError_t num_sms(int *out) {
 
 // ---------------------------------------------------------------- paged --
 
-int paged_splits(const fa_decode_paged_params *p) {
-    if (p->num_splits > 0) return p->num_splits < p->max_blocks_per_seq ? p->num_splits : p->max_blocks_per_seq;
-    // Automatic: enough (sequence, KV head, split) units to fill every SM
-    // several times over, with splits of at least 8 blocks.
+// Split count of a paged decode: the caller's, clamped to the table width,
+// or (num_splits == 0) enough (sequence, KV head, split) units to fill
+// every SM of the current device several times over (two resident CTAs an
+// SM, six waves), with splits of at least 8 blocks.  The automatic count
+// needs the device's SM count: FA_ERR_CUDA if it cannot be read.
+fa_status paged_splits(const fa_decode_paged_params *p, int *out) {
+    if (p->num_splits > 0) {
+        *out = p->num_splits < p->max_blocks_per_seq ? p->num_splits : p->max_blocks_per_seq;
+        return FA_OK;
+    }
+    int sms = 0;
+    cudaError_t e = num_sms(&sms);
+    if (e != cudaSuccess) return cuda_fail(e, "fa_decode_paged: SM count for the automatic split count");
     const long long units = (long long)p->B * p->Hkv;
-    const long long want = 148LL * 2 * 6;
+    const long long want = (long long)sms * 2 * 6;
     long long s = (want + units - 1) / units;
     long long max_by_len = (p->max_blocks_per_seq + 7) / 8;
     if (s > max_by_len) s = max_by_len;
     if (s < 1) s = 1;
-    return (int)s;
+    *out = (int)s;
+    return FA_OK;
 }
 
 fa_status check_paged(const fa_decode_paged_params *p) {
@@ -187,6 +197,39 @@ fa_status encode_paged_caches(const fa_decode_paged_params *p, fa::PagedLaunch *
     return encode_2d(&L->tmV, p->v_cache, p->dv, rows, p->dv, 64, "fa_decode_paged v_cache");
 }
 
+// Everything a paged-decode launch needs except where its split partials
+// go (shared by fa_decode_paged, fa_decode_paged_noalloc and the timeout
+// test hook).
+fa_status paged_launch_setup(const fa_decode_paged_params *p, int splits, fa::PagedLaunch *L) {
+    fa_status st = encode_paged_caches(p, L);
+    if (st != FA_OK) return st;
+    L->q = p->q;
+    L->k_cache = p->k_cache;
+    L->v_cache = p->v_cache;
+    L->block_table = p->block_table;
+    L->seq_lens = p->seq_lens;
+    L->max_blocks_per_seq = p->max_blocks_per_seq;
+    L->B = p->B;
+    L->Hq = p->Hq;
+    L->Hkv = p->Hkv;
+    L->num_blocks = p->num_blocks;
+    L->scale = p->scale;
+    L->num_splits = splits;
+    L->blocks_per_split = (p->max_blocks_per_seq + splits - 1) / splits;
+    L->o = p->o;
+    L->lse = p->lse;
+    L->o_bf16 = p->o_dtype == FA_BF16;
+    L->part_o = nullptr;
+    L->part_lse = nullptr;
+    return FA_OK;
+}
+
+// Byte offset of the partial LSEs in a paged workspace of `splits` splits.
+size_t paged_lse_offset(const fa_decode_paged_params *p, int splits) {
+    const size_t rows = (size_t)p->B * p->Hq * (size_t)splits;
+    return (rows * 128 * sizeof(float) + 255) & ~size_t(255);
+}
+
 size_t paged_ws_bytes(const fa_decode_paged_params *p, int splits) {
     const size_t rows = (size_t)p->B * p->Hq * (size_t)splits;
     size_t o = rows * 128 * sizeof(float);
@@ -196,18 +239,27 @@ size_t paged_ws_bytes(const fa_decode_paged_params *p, int splits) {
 
 // --------------------------------------------------------------- gather --
 
-int gather_splits(const fa_decode_gather_params *p) {
+// Split count of a latent decode: the caller's, clamped to one split per 64
+// keys, or (num_splits == 0) one two-CTA cluster per (token, split) and at
+// most one wave of clusters (half the device's SMs), with at least 128
+// keys per split.
+fa_status gather_splits(const fa_decode_gather_params *p, int *out) {
     const int max_s = (p->topk + 63) / 64 > 0 ? (p->topk + 63) / 64 : 1;
-    if (p->num_splits > 0) return p->num_splits < max_s ? p->num_splits : max_s;
-    // Automatic: one two-CTA cluster per (token, split) and at most one wave
-    // of clusters (74 on 148 SMs), with at least 128 keys per split.
-    const long long want = 74;
+    if (p->num_splits > 0) {
+        *out = p->num_splits < max_s ? p->num_splits : max_s;
+        return FA_OK;
+    }
+    int sms = 0;
+    cudaError_t e = num_sms(&sms);
+    if (e != cudaSuccess) return cuda_fail(e, "fa_decode_gather: SM count for the automatic split count");
+    const long long want = sms / 2 > 0 ? sms / 2 : 1;
     const long long T = p->T > 0 ? p->T : 1;
     long long s = want / T;
     long long max_by_len = (p->topk + 127) / 128;
     if (s > max_by_len) s = max_by_len;
     if (s < 1) s = 1;
-    return (int)s;
+    *out = (int)s;
+    return FA_OK;
 }
 
 fa_status check_gather(const fa_decode_gather_params *p) {
@@ -491,7 +543,10 @@ fa_status fa_decode_paged_workspace_size(const fa_decode_paged_params *p, size_t
     fa_status st = check_paged(p);
     if (st != FA_OK) return st;
     if (!bytes) return fail(FA_ERR_INVALID_ARG, "fa_decode_paged_workspace_size: bytes is NULL");
-    *bytes = paged_ws_bytes(p, paged_splits(p));
+    int splits = 0;
+    st = paged_splits(p, &splits);
+    if (st != FA_OK) return st;
+    *bytes = paged_ws_bytes(p, splits);
     return FA_OK;
 }
 
@@ -499,33 +554,17 @@ fa_status fa_decode_paged(const fa_decode_paged_params *p, void *stream) {
     fa_status st = check_paged_ptrs(p);
     if (st != FA_OK) return st;
     if (p->B == 0) return FA_OK;
-    const int splits = paged_splits(p);
+    int splits = 0;
+    st = paged_splits(p, &splits);
+    if (st != FA_OK) return st;
     const size_t need = paged_ws_bytes(p, splits);
     if (!p->workspace || p->workspace_bytes < need || ((uintptr_t)p->workspace & 255u))
         return fail(FA_ERR_WORKSPACE, "fa_decode_paged: workspace needs %zu bytes, 256-byte aligned", need);
     fa::PagedLaunch L;
-    st = encode_paged_caches(p, &L);
+    st = paged_launch_setup(p, splits, &L);
     if (st != FA_OK) return st;
-    L.q = p->q;
-    L.k_cache = p->k_cache;
-    L.v_cache = p->v_cache;
-    L.block_table = p->block_table;
-    L.seq_lens = p->seq_lens;
-    L.max_blocks_per_seq = p->max_blocks_per_seq;
-    L.B = p->B;
-    L.Hq = p->Hq;
-    L.Hkv = p->Hkv;
-    L.num_blocks = p->num_blocks;
-    L.scale = p->scale;
-    L.num_splits = splits;
-    L.blocks_per_split = (p->max_blocks_per_seq + splits - 1) / splits;
-    L.o = p->o;
-    L.lse = p->lse;
-    L.o_bf16 = p->o_dtype == FA_BF16;
-    const size_t rows = (size_t)p->B * p->Hq * splits;
     L.part_o = static_cast<float *>(p->workspace);
-    L.part_lse = reinterpret_cast<float *>(static_cast<char *>(p->workspace) +
-                                           ((rows * 128 * sizeof(float) + 255) & ~size_t(255)));
+    L.part_lse = reinterpret_cast<float *>(static_cast<char *>(p->workspace) + paged_lse_offset(p, splits));
     cudaError_t e = fa::launch_decode_paged(L, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "fa_decode_paged: launch");
     return FA_OK;
@@ -535,7 +574,9 @@ fa_status fa_decode_paged_noalloc(const fa_decode_paged_params *p, void *stream)
     fa_status st = check_paged_ptrs(p);
     if (st != FA_OK) return st;
     if (p->B == 0) return FA_OK;
-    const int splits = paged_splits(p);
+    int splits = 0;
+    st = paged_splits(p, &splits);
+    if (st != FA_OK) return st;
     const size_t need = paged_ws_bytes(p, splits);
     const size_t have = fa::paged_static_scratch_bytes();
     if (need > have)
@@ -544,30 +585,35 @@ fa_status fa_decode_paged_noalloc(const fa_decode_paged_params *p, void *stream)
                     "holds %zu; pass fewer num_splits or call fa_decode_paged with a workspace",
                     need, have);
     fa::PagedLaunch L;
-    st = encode_paged_caches(p, &L);
+    st = paged_launch_setup(p, splits, &L);
     if (st != FA_OK) return st;
-    L.q = p->q;
-    L.k_cache = p->k_cache;
-    L.v_cache = p->v_cache;
-    L.block_table = p->block_table;
-    L.seq_lens = p->seq_lens;
-    L.max_blocks_per_seq = p->max_blocks_per_seq;
-    L.B = p->B;
-    L.Hq = p->Hq;
-    L.Hkv = p->Hkv;
-    L.num_blocks = p->num_blocks;
-    L.scale = p->scale;
-    L.num_splits = splits;
-    L.blocks_per_split = (p->max_blocks_per_seq + splits - 1) / splits;
-    L.o = p->o;
-    L.lse = p->lse;
-    L.o_bf16 = p->o_dtype == FA_BF16;
-    L.part_o = nullptr;
-    L.part_lse = nullptr;
-    const size_t rows = (size_t)p->B * p->Hq * splits;
-    const size_t lse_offset = (rows * 128 * sizeof(float) + 255) & ~size_t(255);
-    cudaError_t e = fa::launch_decode_paged_static(L, lse_offset, static_cast<cudaStream_t>(stream));
+    cudaError_t e = fa::launch_decode_paged_static(L, paged_lse_offset(p, splits), static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "fa_decode_paged_noalloc: launch");
+    return FA_OK;
+}
+
+fa_status fa_debug_decode_paged_stall(const fa_decode_paged_params *p, uint64_t wait_limit_ns, void *stream) {
+    fa_status st = check_paged_ptrs(p);
+    if (st != FA_OK) return st;
+    if (wait_limit_ns < 1000 || wait_limit_ns > 2000000000ull)
+        return fail(FA_ERR_INVALID_ARG, "fa_debug_decode_paged_stall: wait_limit_ns must be in [1e3, 2e9]");
+    if (p->B == 0) return FA_OK;
+    int splits = 0;
+    st = paged_splits(p, &splits);
+    if (st != FA_OK) return st;
+    const size_t need = paged_ws_bytes(p, splits);
+    if (!p->workspace || p->workspace_bytes < need || ((uintptr_t)p->workspace & 255u))
+        return fail(FA_ERR_WORKSPACE, "fa_debug_decode_paged_stall: workspace needs %zu bytes, 256-byte aligned",
+                    need);
+    fa::PagedLaunch L;
+    st = paged_launch_setup(p, splits, &L);
+    if (st != FA_OK) return st;
+    L.part_o = static_cast<float *>(p->workspace);
+    L.part_lse = reinterpret_cast<float *>(static_cast<char *>(p->workspace) + paged_lse_offset(p, splits));
+    L.wait_ns = wait_limit_ns;
+    L.stall = 1;
+    cudaError_t e = fa::launch_decode_paged(L, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "fa_debug_decode_paged_stall: launch");
     return FA_OK;
 }
 
@@ -575,7 +621,10 @@ fa_status fa_decode_gather_workspace_size(const fa_decode_gather_params *p, size
     fa_status st = check_gather(p);
     if (st != FA_OK) return st;
     if (!bytes) return fail(FA_ERR_INVALID_ARG, "fa_decode_gather_workspace_size: bytes is NULL");
-    *bytes = gather_ws_bytes(p, gather_splits(p));
+    int splits = 0;
+    st = gather_splits(p, &splits);
+    if (st != FA_OK) return st;
+    *bytes = gather_ws_bytes(p, splits);
     return FA_OK;
 }
 
@@ -583,7 +632,9 @@ fa_status fa_decode_gather(const fa_decode_gather_params *p, void *stream) {
     fa_status st = check_gather_ptrs(p);
     if (st != FA_OK) return st;
     if (p->T == 0) return FA_OK;
-    const int splits = gather_splits(p);
+    int splits = 0;
+    st = gather_splits(p, &splits);
+    if (st != FA_OK) return st;
     const size_t need = gather_ws_bytes(p, splits);
     if (!p->workspace || p->workspace_bytes < need || ((uintptr_t)p->workspace & 255u))
         return fail(FA_ERR_WORKSPACE, "fa_decode_gather: workspace needs %zu bytes, 256-byte aligned", need);

@@ -59,13 +59,15 @@ struct PagedLaunch {
     float *part_lse;  // [B*Hq, num_splits]   (log2 units)
     int kv_type;      // 0: bf16 (TMA); 8: q8_0 rows of 136 bytes, 2: fp8 rows of 128 (bulk copies)
     float k_scale, v_scale;  // fp8 caches
+    unsigned long long wait_ns;  // 0: the default bound of a pipeline wait (2 s)
+    int stall;                   // test of the timeout path (fa_debug_decode_paged_stall)
 };
 cudaError_t launch_decode_paged(const PagedLaunch &L, cudaStream_t stream);
 // Log-sum-exp merge of split partials (D = 128 or 512).  seq_lens != NULL:
 // paged mode (row r belongs to sequence r / Hq, which has
-// ceil(ceil(len / 64) / bps) splits); NULL: every split exists.
+// ceil(min(ceil(len / 64), max_blocks) / bps) splits); NULL: every split exists.
 cudaError_t launch_combine(const float *part_o, const float *part_lse, int rows, int num_splits, int Hq,
-                           const int32_t *seq_lens, int bps, void *o, float *lse, int o_bf16, int D,
+                           const int32_t *seq_lens, int bps, int max_blocks, void *o, float *lse, int o_bf16, int D,
                            cudaStream_t stream);
 cudaError_t decode_device_error(int clear, int *code);
 // Allocation-free variant: the partials go to a fixed device array owned by

@@ -82,15 +82,16 @@ FA_DEV bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 
 // Bounded wait for the phase of parity `parity` to complete.  Returns false
 // if the CTA-wide abort flag is (or becomes) set, or if the wait exceeds
-// kWaitLimitNs -- then it sets the abort flag and latches `*err` (first
-// error wins).
-FA_DEV bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag, int *err) {
+// limit_ns (kWaitLimitNs unless a launch passes a shorter one) -- then it
+// sets the abort flag and latches `*err` (first error wins).
+FA_DEV bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag, int *err,
+                      unsigned long long limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
         if (*abort_flag) return false;
-        if (global_timer_ns() - t0 > kWaitLimitNs) {
+        if (global_timer_ns() - t0 > limit_ns) {
             *abort_flag = 1;
             atomicCAS(err, 0, 1 /* FA_DEVERR_TIMEOUT */);
             return false;
@@ -201,6 +202,8 @@ FA_DEV void bulk_copy_to_peer(uint32_t dst_cluster, uint32_t src_cta, uint32_t b
 FA_DEV void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Waits until every committed bulk copy of this thread has finished READING its source.
 FA_DEV void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// Waits until every committed bulk copy of this thread but the newest has finished READING its source.
+FA_DEV void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
 // Waits until every committed bulk copy of this thread has completed.
 FA_DEV void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 

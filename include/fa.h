@@ -107,8 +107,9 @@ enum {
  *   exp(sink_h) in each row's softmax denominator, with no value row.  The
  *   returned LSE includes it; a row with no visible key then gets O = 0 and
  *   LSE = sink_h.
- * These run in the same kernels.  Each row loads its 2-byte mask values per
- * key tile straight from global memory.
+ * These run in the same kernels.  For dk = dv <= 128 the mask is staged
+ * into shared memory by TMA (64-key x 128-row tiles) by loader warps; for
+ * the larger head sizes each row reads its mask values from global memory.
  */
 typedef struct {
     const void *q, *k, *v;
@@ -215,8 +216,9 @@ fa_status fa_prefill_paged(const fa_prefill_paged_params *p, void *stream);
  *     Entries past a sequence's last block are never read.
  *   seq_lens: [B] int32, each in [0, max_blocks_per_seq * block_size].
  *   o: [B, Hq, dv] (o_dtype) contiguous; lse: NULL or [B, Hq] fp32.
- *   num_splits: 0 = choose automatically, else the number of key splits
- *     per sequence (clamped to [1, max_blocks_per_seq]).
+ *   num_splits: 0 = choose automatically (from the current device's SM
+ *     count; FA_ERR_CUDA if it cannot be read), else the number of key
+ *     splits per sequence (clamped to [1, max_blocks_per_seq]).
  *   workspace: device scratch of at least fa_decode_paged_workspace_size()
  *     bytes, 256-byte aligned; it holds the split partials and is
  *     overwritten on every call.
@@ -266,8 +268,10 @@ fa_status fa_decode_paged(const fa_decode_paged_params *p, void *stream);
  *   FA_ERR_WORKSPACE before any launch; pass a smaller num_splits or use
  *   fa_decode_paged.
  *   The first call on each device looks up the scratch array's device
- *   address with that device current; make that first call before any
- *   stream capture.  Every call shares the one array and it keeps the last
+ *   address with that device current and caches it; make that first call
+ *   before any stream capture.  cudaDeviceReset unloads the library's
+ *   device code, so the cached address is stale afterwards: do not call
+ *   this entry point again in a process that reset the device.  Every call shares the one array and it keeps the last
  *   call's contents (nothing in it needs to start at zero): calls whose
  *   work overlaps on the GPU -- concurrent streams, or several host threads
  *   -- race on it and must be serialised by the caller.
@@ -292,7 +296,8 @@ fa_status fa_decode_paged_noalloc(const fa_decode_paged_params *p, void *stream)
  *   q_pos: NULL (no causal mask) or [T] int32; slot j is visible to token t
  *     iff idx[t][j] >= 0 and key_pos <= q_pos[t].
  *   o: [T, Hq, dv] (o_dtype) contiguous; lse: NULL or [T, Hq] fp32.
- *   num_splits: 0 = automatic, else the number of key splits per token.
+ *   num_splits: 0 = automatic (from the current device's SM count), else
+ *     the number of key splits per token.
  *   workspace: at least fa_decode_gather_workspace_size() bytes, 256-byte
  *     aligned, overwritten on every call.
  * Supported: (dk, dv, v_offset) = (576, 512, 64) -- rows [k_pe | latent] --
@@ -425,6 +430,21 @@ fa_status fa_device_error(int clear, int *code);
 
 /* Library version, major * 10000 + minor * 100 + patch. */
 int fa_version(void);
+
+/*
+ * fa_debug_decode_paged_stall -- a test of the bounded-wait path, not part of
+ * the computation.  It launches exactly what fa_decode_paged launches (same
+ * arguments, same workspace rule), except that (1) every pipeline wait of the
+ * decode kernel gives up after wait_limit_ns (in [1e3, 2e9] ns; the normal
+ * bound is 2 s) and (2) the consumer warps first wait on a barrier that
+ * nothing ever completes.  That wait runs out; the CTA latches
+ * FA_DEVERR_TIMEOUT, leaves its loops, waits (again bounded) for its own
+ * copies in flight and returns.  Nothing traps and the context stays usable.
+ * Every row then gets O = 0 and LSE = -inf, and fa_device_error() reports
+ * FA_DEVERR_TIMEOUT.  The pages describe no such hook; it has no
+ * counterpart there.
+ */
+fa_status fa_debug_decode_paged_stall(const fa_decode_paged_params *p, uint64_t wait_limit_ns, void *stream);
 
 #ifdef __cplusplus
 }

@@ -94,17 +94,26 @@ def paged_params(**kw):
 
 
 def test_paged_workspace_size_and_validation():
+    import torch
     lib = fa.load()
     n = ctypes.c_size_t(0)
-    assert lib.fa_decode_paged_workspace_size(ctypes.byref(paged_params()), ctypes.byref(n)) == fa.FA_OK
-    splits = min(128, max(1, -(-148 * 2 * 6 // (64 * 8))), (128 + 7) // 8)
-    rows = 64 * 32 * splits
-    assert n.value == ((rows * 128 * 4 + 255) // 256) * 256 + ((rows * 4 + 255) // 256) * 256
+    st = lib.fa_decode_paged_workspace_size(ctypes.byref(paged_params()), ctypes.byref(n))
+    if torch.cuda.is_available():
+        # automatic splits: two CTAs an SM, six waves, splits of >= 8 blocks
+        assert st == fa.FA_OK
+        sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+        splits = min(128, max(1, -(-sms * 2 * 6 // (64 * 8))), (128 + 7) // 8)
+        rows = 64 * 32 * splits
+        assert n.value == ((rows * 128 * 4 + 255) // 256) * 256 + ((rows * 4 + 255) // 256) * 256
+    else:
+        # the automatic split count is sized from the device's SM count
+        assert st == fa.FA_ERR_CUDA
     assert lib.fa_decode_paged_workspace_size(ctypes.byref(paged_params(num_splits=5)), ctypes.byref(n)) == 0
     assert n.value == ((64 * 32 * 5 * 512 + 255) // 256) * 256 + ((64 * 32 * 5 * 4 + 255) // 256) * 256
     # the workspace check happens before any launch
-    assert lib.fa_decode_paged(ctypes.byref(paged_params()), None) == fa.FA_ERR_WORKSPACE
-    assert lib.fa_decode_paged(ctypes.byref(paged_params(workspace=256, workspace_bytes=10)), None) == fa.FA_ERR_WORKSPACE
+    assert lib.fa_decode_paged(ctypes.byref(paged_params(num_splits=5)), None) == fa.FA_ERR_WORKSPACE
+    assert lib.fa_decode_paged(ctypes.byref(paged_params(num_splits=5, workspace=256, workspace_bytes=10)),
+                               None) == fa.FA_ERR_WORKSPACE
     assert lib.fa_decode_paged(ctypes.byref(paged_params(dk=64, dv=64)), None) == fa.FA_ERR_UNSUPPORTED
     assert lib.fa_decode_paged(ctypes.byref(paged_params(block_size=16)), None) == fa.FA_ERR_UNSUPPORTED
     assert lib.fa_decode_paged(ctypes.byref(paged_params(Hq=24, Hkv=8)), None) == fa.FA_ERR_UNSUPPORTED
@@ -117,7 +126,8 @@ def test_paged_workspace_size_and_validation():
 def test_paged_cache_types(kv_type, status):
     # bf16, q8_0, q4_0 and fp8 caches pass the shape check; other codes are unsupported
     n = ctypes.c_size_t(0)
-    st = fa.load().fa_decode_paged_workspace_size(ctypes.byref(paged_params(kv_type=kv_type)), ctypes.byref(n))
+    st = fa.load().fa_decode_paged_workspace_size(ctypes.byref(paged_params(kv_type=kv_type, num_splits=4)),
+                                                  ctypes.byref(n))
     assert st == (fa.FA_OK if status == 0 else fa.FA_ERR_UNSUPPORTED)
 
 
@@ -135,7 +145,7 @@ def test_paged_kv_type_from_row_length():
 def gather_params(**kw):
     p = fa.GatherParams()
     base = dict(q=16, kv_rows=32, n_rows=65536, row_stride=576, dk=576, dv=512, v_offset=64, idx=48, topk=2048,
-                key_pos=0, q_pos=64, T=32, Hq=128, scale=1 / 24, num_splits=0, o=80, lse=0, o_dtype=0,
+                key_pos=0, q_pos=64, T=32, Hq=128, scale=1 / 24, num_splits=2, o=80, lse=0, o_dtype=0,
                 workspace=0, workspace_bytes=0)
     base.update(kw)
     for k_, v_ in base.items():
@@ -144,10 +154,14 @@ def gather_params(**kw):
 
 
 def test_gather_workspace_size_and_validation():
+    import torch
     lib = fa.load()
     n = ctypes.c_size_t(0)
     assert lib.fa_decode_gather_workspace_size(ctypes.byref(gather_params()), ctypes.byref(n)) == fa.FA_OK
-    assert n.value > 0 and n.value % 256 == 0
+    assert n.value == ((32 * 128 * 2 * 512 * 4 + 255) // 256) * 256 + ((32 * 128 * 2 * 4 + 255) // 256) * 256
+    st = lib.fa_decode_gather_workspace_size(ctypes.byref(gather_params(num_splits=0)), ctypes.byref(n))
+    # automatic splits are sized from the current device's SM count
+    assert st == (fa.FA_OK if torch.cuda.is_available() else fa.FA_ERR_CUDA)
     assert lib.fa_decode_gather(ctypes.byref(gather_params()), None) == fa.FA_ERR_WORKSPACE
     assert lib.fa_decode_gather(ctypes.byref(gather_params(dk=128)), None) == fa.FA_ERR_UNSUPPORTED
     assert lib.fa_decode_gather(ctypes.byref(gather_params(Hq=64)), None) == fa.FA_ERR_UNSUPPORTED

@@ -65,7 +65,7 @@ def test_explicit_key_positions():
 def test_bf16_output():
     c = W.LatentCase("t", 2, 128, 2000, 256, seed=53, select_from_all=True, q_pos0=1999)
     o, lse, o_ref, l_ref = run(c, out_dtype=torch.bfloat16)
-    check(o, o_ref, lse, l_ref, max_abs=2e-2, min_cos=0.9999)
+    check(o, o_ref, lse, l_ref, what="bf16 output")
 
 
 def test_latent_config_sampled_tokens():

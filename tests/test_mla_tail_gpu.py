@@ -5,7 +5,8 @@ Tolerance: u is held in bf16 between the two contractions (the operand type
 of the second), which the fp64 oracle does not do.  With the workload's
 scaling (u, y ~ N(0, 1), weights ~ N(0, 1/fan_in)) that rounding moves y by
 about 2^-9 / sqrt(3) ~ 1.1e-3 rms, so max |dy| stays well inside 1e-2 and the
-cosine above 0.99999; bf16 output adds up to half an ulp of y (2e-2)."""
+cosine above 0.99999.  bf16 output is checked against the stated bar plus
+its own rounding, |dy| <= 1e-2 + 2^-8 (|y_ref| + 1e-2) (tests/parity.py)."""
 import numpy as np
 import pytest
 import torch
@@ -26,8 +27,7 @@ def run(c, num_splits=0, out_dtype=torch.float32, rows=None):
     w_ref = w_o if rows is None else w_o[rows]
     _, y_ref = oracle.mla_tail(W.bits(o_lat), W.bits(w_abs), W.bits(w_ref))
     got = y if rows is None else y[:, rows]
-    bf = out_dtype == torch.bfloat16
-    check(got, y_ref, max_abs=2e-2 if bf else 1e-2, min_cos=0.9999 if bf else 0.99999,
+    check(got, y_ref,
           what="%s splits %d" % (c.name, num_splits))
     return y
 

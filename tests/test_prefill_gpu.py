@@ -46,9 +46,7 @@ def run_and_check(B, Hq, Hkv, Sq, Sk, d, causal, seed, layout="bhsd", out_dtype=
     torch.cuda.synchronize()
     assert fa.device_error() == 0
     o_ref, l_ref = oracle_full(q, k, v, scale, causal)
-    tol = 1e-2 if out_dtype == torch.float32 else 2e-2
-    check(o, o_ref, lse, l_ref, max_abs=tol,
-          min_cos=0.99999 if out_dtype == torch.float32 else 0.9999,
+    check(o, o_ref, lse, l_ref,
           what="B%d Hq%d Hkv%d Sq%d Sk%d d%d causal%d %s" % (B, Hq, Hkv, Sq, Sk, d, causal, layout))
 
 

@@ -6,7 +6,8 @@ reserved up front and may not call cudaMalloc on its hot path): instead of a
 caller-supplied workspace it uses a fixed scratch array inside the library.
 This test calls it through the C ABI twice in a row, on two different
 workloads, and checks each result against the workspace entry point
-(fa_decode_paged) within the parity tolerances used everywhere else.  It
+(fa_decode_paged) and against the fp64 oracle, within the parity
+tolerances used everywhere else.  It
 also checks that shapes needing more scratch than the library holds are
 rejected before any launch.  The file is named to be collected last.
 """
@@ -15,6 +16,7 @@ import ctypes
 import pytest
 import torch
 
+import oracle
 from attention_attn_fwd_11_b200 import fa
 from attention_attn_fwd_11_b200 import workloads as W
 from parity import check
@@ -44,12 +46,16 @@ def test_noalloc_matches_workspace_entry_point_twice():
     cases = [W.PagedCase("noalloc_a", 16, 32, 8, 128, 128, 64, 1, 4000, seed=123),
              W.PagedCase("noalloc_b", 9, 16, 4, 128, 128, 64, 0, 2500, seed=124, lens=(0, 1, 64, 65, 700, 2500, 3, 128, 129))]
     for c in cases:  # two calls in a row; the second finds the first's leftovers in the scratch
-        q, kc, vc, tb, sl = [t.cuda() for t in W.paged_inputs(c)]
+        host = W.paged_inputs(c)
+        q, kc, vc, tb, sl = [t.cuda() for t in host]
         ref_o, ref_l = fa.decode_paged(q, kc, vc, tb, sl, scale=c.scale)
         st, o, lse = call_noalloc(fn, q, kc, vc, tb, sl, c.scale)
         assert st == fa.FA_OK, lib.fa_last_error().decode()
         torch.cuda.synchronize()
         check(o, ref_o, lse, ref_l, what=c.name)
+        qh, kh, vh, th, lh = host
+        o64, l64 = oracle.decode_paged(W.bits(qh), W.bits(kh), W.bits(vh), th.numpy(), lh.numpy(), c.scale)
+        check(o, o64, lse, l64, what=c.name + " vs the oracle")
     assert fa.device_error() == 0
 
 
