@@ -329,13 +329,16 @@ fa_status fa_fwd(const fa_fwd_params *p, void *stream) {
     if (p->B < 0 || p->Hq <= 0 || p->Hkv <= 0 || p->Sq < 0 || p->Sk < 0)
         return fail(FA_ERR_INVALID_ARG, "fa_fwd: need B >= 0, Hq > 0, Hkv > 0, Sq >= 0, Sk >= 0");
     if (p->Hq % p->Hkv != 0) return fail(FA_ERR_INVALID_ARG, "fa_fwd: Hq (%d) %% Hkv (%d) != 0", p->Hq, p->Hkv);
+    const bool d512 = p->dv == 512 && (p->dk == 576 || p->dk == 512);
     const bool pair_ok = (p->dk == p->dv && (p->dk == 64 || p->dk == 128 || p->dk == 256)) ||
-                         (p->dk == 192 && (p->dv == 128 || p->dv == 192)) || (p->dk == 320 && p->dv == 256);
+                         (p->dk == 192 && (p->dv == 128 || p->dv == 192)) || (p->dk == 320 && p->dv == 256) || d512;
     if (!pair_ok)
         return fail(FA_ERR_UNSUPPORTED,
-                    "fa_fwd: supported (dk, dv) = (64, 64), (128, 128), (192, 192), (256, 256), (192, 128), (320, 256); got "
-                    "(%d, %d)",
+                    "fa_fwd: supported (dk, dv) = (64, 64), (128, 128), (192, 192), (256, 256), (192, 128), (320, 256), "
+                    "(576, 512), (512, 512); got (%d, %d)",
                     p->dk, p->dv);
+    if (d512 && (p->mask || p->softcap != 0.f || p->sinks || p->max_bias != 0.f))
+        return fail(FA_ERR_UNSUPPORTED, "fa_fwd: score modifiers are not supported with dv = 512");
     if (!finite_pos(p->scale)) return fail(FA_ERR_INVALID_ARG, "fa_fwd: scale must be finite and > 0");
     if (p->o_dtype != FA_F32 && p->o_dtype != FA_BF16) return fail(FA_ERR_INVALID_ARG, "fa_fwd: o_dtype");
     if ((long long)p->B * p->Hq > 0x7fffffffLL || p->Sq > (1 << 30) || p->Sk > (1 << 30))
@@ -358,6 +361,43 @@ fa_status fa_fwd(const fa_fwd_params *p, void *stream) {
                     "fa_fwd: mask must be 16-byte aligned, its strides multiples of 8 elements, m_ss >= Sk");
     if ((uintptr_t)p->sinks & 3u) return fail(FA_ERR_INVALID_ARG, "fa_fwd: sinks must be 4-byte aligned");
     if (!get_encoder()) return fail(FA_ERR_CUDA, "fa_fwd: cuTensorMapEncodeTiled is not available");
+
+    if (d512) {
+        // The latent kernel's CTA pair: each CTA keeps half of the 512-wide O
+        // in TMEM and the pair splits the dk-wide score contraction by columns.
+        fa::Dense512Launch D;
+        memset(&D, 0, sizeof D);
+        fa_status st = encode_4d(&D.tmQ, p->q, p->dk, p->Sq, p->Hq, p->B, p->q_ss, p->q_sh, p->q_sb, 128, "fa_fwd q");
+        if (st != FA_OK) return st;
+        const void *kb = p->Sk > 0 ? p->k : p->q;
+        const void *vb = p->Sk > 0 ? p->v : p->q;
+        st = encode_4d(&D.tmK, kb, p->dk, p->Sk, p->Hkv, p->B, p->k_ss, p->k_sh, p->k_sb, 32, "fa_fwd k");
+        if (st != FA_OK) return st;
+        st = encode_4d(&D.tmV, vb, p->dv, p->Sk, p->Hkv, p->B, p->v_ss, p->v_sh, p->v_sb, 32, "fa_fwd v");
+        if (st != FA_OK) return st;
+        st = encode_4d(&D.tmO, p->o, p->dv, p->Sq, p->Hq, p->B, p->o_ss, p->o_sh, p->o_sb, 32, "fa_fwd o",
+                       p->o_dtype == FA_F32 ? 4 : 2);
+        if (st != FA_OK) return st;
+        if ((long long)p->B * p->Hq > 65535 || (p->Sq + 127) / 128 > 65535)
+            return fail(FA_ERR_INVALID_ARG, "fa_fwd: B * Hq and ceil(Sq / 128) must be <= 65535 for dv = 512");
+        D.B = p->B;
+        D.Hq = p->Hq;
+        D.Hkv = p->Hkv;
+        D.Sq = p->Sq;
+        D.Sk = p->Sk;
+        D.dk = p->dk;
+        D.scale = p->scale;
+        D.causal = p->causal ? 1 : 0;
+        D.o = p->o;
+        D.o_sb = p->o_sb;
+        D.o_sh = p->o_sh;
+        D.o_ss = p->o_ss;
+        D.o_bf16 = p->o_dtype == FA_BF16;
+        D.lse = p->lse;
+        cudaError_t e = fa::launch_prefill_d512(D, static_cast<cudaStream_t>(stream));
+        if (e != cudaSuccess) return cuda_fail(e, "fa_fwd: launch");
+        return FA_OK;
+    }
 
     fa::PrefillLaunch L;
     memset(&L, 0, sizeof L);
@@ -663,6 +703,11 @@ fa_status fa_decode_gather(const fa_decode_gather_params *p, void *stream) {
     L.part_o = static_cast<float *>(p->workspace);
     L.part_lse = reinterpret_cast<float *>(static_cast<char *>(p->workspace) +
                                            ((rows * 512 * sizeof(float) + 255) & ~size_t(255)));
+    // The kernel writes its partials with TMA stores: (512 values, T * Hq
+    // rows, splits) fp32, 32 x 32 boxes.
+    st = encode_4d(&L.tmPO, L.part_o, 512, p->T * p->Hq, splits, 1, (int64_t)splits * 512, 512,
+                   (int64_t)splits * 512 * p->T * p->Hq, 32, "fa_decode_gather partials", 4);
+    if (st != FA_OK) return st;
     cudaError_t e = fa::launch_decode_gather(L, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "fa_decode_gather: launch");
     return FA_OK;

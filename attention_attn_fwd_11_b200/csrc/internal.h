@@ -79,6 +79,7 @@ cudaError_t launch_decode_paged_static(PagedLaunch L, size_t lse_offset, cudaStr
 // ---- latent gather decode ------------------------------------------------
 struct GatherLaunch {
     CUtensorMap tmQ;  // q viewed as [T * Hq, dk], box 64 x 128, 128-byte swizzle
+    CUtensorMap tmPO;  // part_o as (512, T * Hq, num_splits, 1) fp32, box 32 x 32 rows, 128-byte swizzle
     const void *q, *rows;
     int64_t n_rows, row_stride;
     const int32_t *idx, *key_pos, *q_pos;
@@ -94,6 +95,23 @@ struct GatherLaunch {
 };
 cudaError_t launch_decode_gather(const GatherLaunch &L, cudaStream_t stream);
 cudaError_t gather_device_error(int clear, int *code);
+
+// Prefill with dv = 512 and separate K and V tensors, (dk, dv) = (576, 512)
+// or (512, 512), on the latent kernel's CTA pair (decode_gather.cu).
+struct Dense512Launch {
+    CUtensorMap tmQ;  // q as (dk, Sq, Hq, B), box 64 x 128 rows, 128-byte swizzle
+    CUtensorMap tmK;  // k as (dk, Sk, Hkv, B), box 64 x 32 rows
+    CUtensorMap tmV;  // v as (512, Sk, Hkv, B), box 64 x 32 rows
+    CUtensorMap tmO;  // o as (512, Sq, Hq, B), box 128 bytes x 32 rows (fp32 or bf16)
+    int B, Hq, Hkv, Sq, Sk, dk;
+    float scale;
+    int causal;
+    void *o;
+    int64_t o_sb, o_sh, o_ss;
+    int o_bf16;
+    float *lse;
+};
+cudaError_t launch_prefill_d512(const Dense512Launch &L, cudaStream_t stream);
 
 // MLA decode tail (mla_tail.cu): out-absorb then o-projection.
 struct TailLaunch {

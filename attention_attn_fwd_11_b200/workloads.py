@@ -83,6 +83,10 @@ CAUSAL_DK192 = PrefillCase("causal_mha_b2_h16_s2048_dk192_dv128", 2, 16, 16, 204
 CAUSAL_DK192_DV192 = PrefillCase("causal_gqa_b2_hq16_hkv4_s2048_dk192_dv192", 2, 16, 4, 2048, 2048, 192, 192, True,
                                  seed=9)
 CAUSAL_DK320 = PrefillCase("causal_gqa_b1_hq16_hkv4_s4096_dk320_dv256", 1, 16, 4, 4096, 4096, 320, 256, True, seed=8)
+# The dv = 512 pairs with separate K and V: one KV head shared by 16 query
+# heads (MQA, as latent attention shares its latent rows), causal.
+CAUSAL_DK576 = PrefillCase("causal_mqa_b1_hq16_hkv1_s4096_dk576_dv512", 1, 16, 1, 4096, 4096, 576, 512, True, seed=11)
+CAUSAL_DK512 = PrefillCase("causal_mqa_b1_hq16_hkv1_s4096_dk512_dv512", 1, 16, 1, 4096, 4096, 512, 512, True, seed=14)
 
 
 # ------------------------------------------------ prefill score modifiers --

@@ -701,7 +701,8 @@ def run_only(args):
     torch.cuda.set_device(0)
     l2 = torch.cuda.get_device_properties(0).L2_cache_size
     table = {c.name: c for c in (W_.TINY_FULL, W_.CAUSAL_MHA, W_.GQA_FULL, W_.MODS_C2, W_.CAUSAL_DK192,
-                                 W_.CAUSAL_DK192_DV192, W_.CAUSAL_DK320, W_.PAGED_GQA, W_.LATENT_SPARSE,
+                                 W_.CAUSAL_DK192_DV192, W_.CAUSAL_DK320, W_.CAUSAL_DK576, W_.CAUSAL_DK512,
+                                 W_.PAGED_GQA, W_.LATENT_SPARSE,
                                  W_.QUANT_C2, W_.PAGED_PREFILL, W_.MLA_TAIL)}
     table[W_.PAGED_Q8_NAME] = W_.PAGED_GQA
     table[W_.PAGED_FP8_NAME] = W_.PAGED_GQA
@@ -907,7 +908,7 @@ def main():
         wl = {}
         Ks = 200
         for cc in (W_.TINY_FULL, W_.GQA_FULL, W_.MODS_C2, W_.CAUSAL_DK192, W_.CAUSAL_DK192_DV192,
-                   W_.CAUSAL_DK320):
+                   W_.CAUSAL_DK320, W_.CAUSAL_DK576):
             launch, ncopy, foot, kpl = prefill_workload(torch, fa, W_, cc, l2)
             ms2, st2 = time_graph(torch, launch, ncopy, Ks, Wm, dist)
             ms2 = max_over_ranks(torch, dist, ms2)
