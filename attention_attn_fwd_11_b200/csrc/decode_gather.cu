@@ -379,52 +379,55 @@ latent_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         }
     } else if (warp == LG_W_MMA) {
         // --------------------------------------------------- MMA issuer --
-        if (lane == 0 && n_tiles > 0) {
+        // The whole warp runs the issue loop and its waits; one elected lane
+        // issues each group of MMAs.  Issued from one lane of a diverged warp,
+        // every small MMA cost about 95 cycles of issue, six times its tensor
+        // time at N = 32.
+        if (n_tiles > 0) {
             constexpr uint32_t idesc_qk = idesc_bf16_f32(128, LG_BN, false, false);
             constexpr uint32_t idesc_pv = idesc_bf16_f32(128, LG_HALF, false, true);
             const uint32_t tO = tmem + LG_T_O;
             auto issue_qk = [&](int i) -> bool {
                 const int s = i % NST;
-                if (!mbar_wait(bar(G_FULL + s), (uint32_t)(i / NST) & 1u, abort_flag, &g_gather_err)) return false;
-                LG_TRACE(14, i);
+                if (!mbar_wait_warp(bar(G_FULL + s), (uint32_t)(i / NST) & 1u, abort_flag, &g_gather_err))
+                    return false;
+                if (lane == 0) LG_TRACE(14, i);
                 if (!DENSE) fence_proxy_async_smem();  // the gathered rows were written by cp.async (generic proxy)
                 tc_fence_after();
                 const uint32_t tS = tmem + (uint32_t)((i % LG_NSB) * LG_BN);
-                const uint32_t st = stage_addr(s);
-                for (int kk = 0; kk < nch * 4; ++kk) {
-                    const int c = kk >> 2, sub = kk & 3;
-                    const uint64_t bd = sdesc_sw128(st + c * LG_KCH + sub * 32, 16, 1024);
-                    mma_ts(tS, tmem + (uint32_t)(LG_T_Q + kk * 8), bd, idesc_qk, kk > 0 ? 1u : 0u);
-                }
-                mma_commit(bar(G_SFULL + i % LG_NSB));
-                LG_TRACE(2, i);
+                const uint64_t bd0 = sdesc_sw128(stage_addr(s), 16, 1024);
+                // one 64-column chunk = four 16-wide K steps: A steps 8 TMEM
+                // columns, B 32 bytes (2 descriptor units)
+                for (int c = 0; c < nch; ++c)
+                    mma_ts4_warp<8, 2>(tS, tmem + (uint32_t)(LG_T_Q + c * 32), bd0 + (uint64_t)((c * LG_KCH) >> 4),
+                                       idesc_qk, c > 0 ? 1u : 0u);
+                mma_commit_warp(bar(G_SFULL + i % LG_NSB));
+                if (lane == 0) LG_TRACE(2, i);
                 return true;
             };
             // QK^T runs NSB - 1 tiles ahead of PV.  S buffer (i + NSB - 1) %
             // NSB last held P of tile i - 1, which PV(i - 1), issued before
             // and executed in order, has consumed.
-            bool ok = mbar_wait(bar(G_QTMEM), 0, abort_flag, &g_gather_err);
+            bool ok = mbar_wait_warp(bar(G_QTMEM), 0, abort_flag, &g_gather_err);
             for (int j = 0; ok && j < LG_NSB - 1 && j < n_tiles; ++j) ok = issue_qk(j);
             for (int i = 0; ok && i < n_tiles; ++i) {
                 if (i + LG_NSB - 1 < n_tiles && !issue_qk(i + LG_NSB - 1)) break;
-                if (!mbar_wait(bar(G_PREADY + i % LG_NSB), (uint32_t)(i / LG_NSB) & 1u, abort_flag, &g_gather_err))
+                if (!mbar_wait_warp(bar(G_PREADY + i % LG_NSB), (uint32_t)(i / LG_NSB) & 1u, abort_flag,
+                                    &g_gather_err))
                     break;
-                LG_TRACE(15, i);
+                if (lane == 0) LG_TRACE(15, i);
                 tc_fence_after();
                 const int s = i % NST;
                 const uint32_t tP = tmem + (uint32_t)((i % LG_NSB) * LG_BN);
-                const uint32_t st = stage_addr(s);
-#pragma unroll
-                for (int kk = 0; kk < LG_BN / 16; ++kk) {
-                    const uint64_t bd = sdesc_sw128(st + vch * LG_KCH + kk * 2048, LG_KCH, 1024);
-                    mma_ts(tO, tP + kk * 8, bd, idesc_pv, (i > 0 || kk > 0) ? 1u : 0u);
-                }
-                mma_commit(bar(G_EMPTY + s));
-                mma_commit(bar(G_PVDONE + i % LG_NSB));
-                LG_TRACE(3, i);
+                const uint64_t bd = sdesc_sw128(stage_addr(s) + vch * LG_KCH, LG_KCH, 1024);
+                mma_ts_warp(tO, tP, bd, idesc_pv, i > 0 ? 1u : 0u);
+                mma_ts_warp(tO, tP + 8, bd + (uint64_t)(2048 >> 4), idesc_pv, 1u);
+                mma_commit_warp(bar(G_EMPTY + s));
+                mma_commit_warp(bar(G_PVDONE + i % LG_NSB));
+                if (lane == 0) LG_TRACE(3, i);
             }
-            mma_commit(bar(G_DRAIN));
-            mbar_wait_drain(bar(G_DRAIN), 0);
+            mma_commit_warp(bar(G_DRAIN));
+            if (lane == 0) mbar_wait_drain(bar(G_DRAIN), 0);
         }
         __syncwarp();
     } else if (warp == LG_W_SEND) {
