@@ -184,8 +184,21 @@ FA_DEV bool p2_unit(const Prefill2Args &a, int round, UnitInfo &u) {
     const int G = gridDim.x, c = blockIdx.x;
     const int idx = round * G + ((round & 1) ? (G - 1 - c) : c);
     if (idx >= a.n_units) return false;
-    const int qp = a.causal ? (a.n_qp - 1 - idx / a.BH) : (idx / a.BH);
-    const int bh = idx % a.BH;
+    int qp, bh;
+    if (a.seq_lens) {
+        // Paged: the query tiles of one head are consecutive units, and the
+        // heads of one KV head are consecutive too, so the units sharing a
+        // KV head's blocks run side by side in the same round and its blocks
+        // stream from DRAM once.  (The tiles of one sequence differ by at
+        // most Sq keys, far less than the spread across sequences.)
+        qp = a.n_qp - 1 - idx % a.n_qp;
+        bh = idx / a.n_qp;
+    } else {
+        // Dense: query-tile-major, the longest tiles (causal: the last rows)
+        // of every head first.
+        qp = a.causal ? (a.n_qp - 1 - idx / a.BH) : (idx / a.BH);
+        bh = idx % a.BH;
+    }
     u.b = bh / a.Hq;
     u.hq = bh % a.Hq;
     u.q0 = qp * 256;

@@ -63,16 +63,17 @@ NCU_TRAFFIC = {
     "causal_mha_mods_b2_h16_s2048_d128": 58342656,
     "paged_gqa_b64_hq32_hkv8_d128_bs64": 1236853248,
     "paged_gqa_q8_0kv_b64_hq32_hkv8_d128_bs64": 674241024,
-    "latent_sparse_t32_hq128_dk576_dv512_top2048": 45067264,
+    "latent_sparse_t32_hq128_dk576_dv512_top2048": 45273088,
     "causal_mha_b2_h16_s2048_dk192_dv128": 72717056,
     "causal_gqa_b2_hq16_hkv4_s2048_dk192_dv192": 39777792,
     "kv_dequant causal_mha_q8_0kv_b2_h16_s2048_d128": 17835776,
     "kv_dequant causal_mha_fp8kv_b2_h16_s2048_d128": 16799744,
-    "paged_prefill_gqa_b16_hq32_hkv8_sq512_d128_bs64": 651760896,
+    "paged_prefill_gqa_b16_hq32_hkv8_sq512_d128_bs64": 417585664,
     "mla_tail_t32_hq128_r512_v128_hidden7168": 257049088,
     "causal_gqa_b1_hq16_hkv4_s4096_dk320_dv256": 78919168,
     "paged_gqa_fp8kv_b64_hq32_hkv8_d128_bs64": 636363776,
     "paged_gqa_q4_0kv_b64_hq32_hkv8_d128_bs64": 356117760,
+    "causal_mqa_b1_hq16_hkv1_s4096_dk576_dv512": 167481088,
 }
 
 
@@ -87,6 +88,8 @@ def parse_args():
     ap.add_argument("--only", default=None,
                     help="time one named workload alone (for profiling), e.g. causal_mha_b2_h16_s2048_d128")
     ap.add_argument("--eager", action="store_true", help="with --only: launch every step eagerly (no CUDA graph)")
+    ap.add_argument("--soak-s", type=float, default=0.25,
+                    help="untimed replays before each headline region, in seconds (0 under a profiler)")
     return ap.parse_args()
 
 
@@ -240,7 +243,7 @@ def time_graph_repeats(torch, launch, n_copies, K, W, dist=None, repeats=5, soak
         g.replay()
         e1.record(stream)
     stream.synchronize()
-    n_soak = int(max(1, min(20000, soak_s * 1e3 / max(e0.elapsed_time(e1), 1e-3))))
+    n_soak = int(max(0, min(20000, soak_s * 1e3 / max(e0.elapsed_time(e1), 1e-3))))
     out = []
     t_host0 = time.time()
     for r in range(repeats):
@@ -803,7 +806,7 @@ def main():
     time.sleep(0.3)
     win = []
     R = 5
-    region_ms = time_graph_repeats(torch, launch, ncopy, K, Wm, dist, repeats=R, window=win)
+    region_ms = time_graph_repeats(torch, launch, ncopy, K, Wm, dist, repeats=R, soak_s=args.soak_s, window=win)
     clocks = sampler.stop(win[0], win[1])
     clocks["window_s"] = round(win[1] - win[0], 3)
     clocks["note"] = "samples over the %d timed regions and the untimed replays between them" % R
