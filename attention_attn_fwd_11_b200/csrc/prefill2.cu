@@ -164,12 +164,6 @@ constexpr float kP2RescaleThreshold = 8.0f;
 #define FA_P2_PACKED 1
 #endif
 
-// Every FA_EXP2_POLY_EVERY-th pair of softmax elements takes 2^x on the FMA
-// pipe (ex2_poly) instead of the MUFU unit, which the two softmax
-// warpgroups otherwise saturate (0 = never).
-#ifndef FA_EXP2_POLY_EVERY
-#define FA_EXP2_POLY_EVERY 0
-#endif
 
 // One unit: query rows [q0, q0 + 256) of head hq in batch b, as two
 // 128-row tiles with n0 and n1 key tiles (N = the larger) over Sk keys.
@@ -749,16 +743,7 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                         for (int k = 0; k < 16; ++k) {
                             float a0, a1;
                             f2_unpack(f2_fma(f2_pack(x[g * 32 + 2 * k], x[g * 32 + 2 * k + 1]), c2, nm2), a0, a1);
-                            float p0, p1;
-                            if (FA_EXP2_POLY_EVERY > 0 &&
-                                (k % (FA_EXP2_POLY_EVERY > 0 ? FA_EXP2_POLY_EVERY : 1)) ==
-                                    (FA_EXP2_POLY_EVERY > 0 ? FA_EXP2_POLY_EVERY - 1 : 0)) {
-                                ex2_poly2(a0, a1, p0, p1);
-                                if (empty_row) p0 = p1 = 0.f;
-                            } else {
-                                p0 = ex2(a0);
-                                p1 = ex2(a1);
-                            }
+                            const float p0 = ex2(a0), p1 = ex2(a1);
                             if (k & 1)
                                 acc1 = f2_add(acc1, f2_pack(p0, p1));
                             else
@@ -798,15 +783,7 @@ prefill2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                     for (int k = 0; k < 16; ++k) {
                         const float a0 = fmaf(x[g * 32 + 2 * k], c, -msub);
                         const float a1 = fmaf(x[g * 32 + 2 * k + 1], c, -msub);
-                        float p0, p1;
-                        if (FA_EXP2_POLY_EVERY > 0 && (k % (FA_EXP2_POLY_EVERY > 0 ? FA_EXP2_POLY_EVERY : 1)) ==
-                                                          (FA_EXP2_POLY_EVERY > 0 ? FA_EXP2_POLY_EVERY - 1 : 0)) {
-                            p0 = empty_row ? 0.f : ex2_poly(a0);
-                            p1 = empty_row ? 0.f : ex2_poly(a1);
-                        } else {
-                            p0 = ex2(a0);
-                            p1 = ex2(a1);
-                        }
+                        const float p0 = ex2(a0), p1 = ex2(a1);
                         s0 += p0;
                         s1 += p1;
                         pk[k] = pack_bf16x2(p0, p1);

@@ -518,21 +518,6 @@ FA_DEV float ex2(float x) {
     return y;
 }
 
-// 2^x on the FMA pipe, for the softmax argument x <= 0: x = k + f with
-// k = round(x) (taken from the low mantissa bits of x + 1.5 * 2^23) and
-// f in [-0.5, 0.5]; 2^f from a degree-3 polynomial fitted by a Remez
-// exchange for minimax relative error on [-0.5, 0.5] (7.5e-5, far below
-// bf16's 2^-9); 2^k is applied by adding k to the exponent field.  Inputs
-// are clamped at -126, so -inf yields 2^-126 rather than 0: callers must
-// not use it for a row with no visible key.
-FA_DEV float ex2_poly(float x) {
-    x = fmaxf(x, -126.f);
-    const float t = x + 12582912.f;
-    const float f = x - (t - 12582912.f);
-    const float p = fmaf(fmaf(fmaf(0.0551716685f, f, 0.2426111251f), f, 0.6932609677f), f, 0.9999280572f);
-    return __int_as_float(__float_as_int(p) + __float_as_int(t) * 8388608);
-}
-
 // Packed fp32 pairs (sm_100 f32x2 instructions): one instruction applies the
 // operation to both halves of a 64-bit register pair.
 FA_DEV uint64_t f2_pack(float lo, float hi) {
@@ -563,25 +548,6 @@ FA_DEV float fmax3(float a, float b, float c) {
     float d;
     asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
     return d;
-}
-
-// ex2_poly on a packed pair, with the f32x2 instructions where they exist.
-FA_DEV void ex2_poly2(float a0, float a1, float &p0, float &p1) {
-    a0 = fmaxf(a0, -126.f);
-    a1 = fmaxf(a1, -126.f);
-    const uint64_t magic = f2_pack(12582912.f, 12582912.f);
-    const uint64_t nmagic = f2_pack(-12582912.f, -12582912.f);
-    const uint64_t x = f2_pack(a0, a1);
-    const uint64_t t = f2_add(x, magic);
-    const uint64_t f = f2_add(x, f2_mul(f2_add(t, nmagic), f2_pack(-1.f, -1.f)));
-    uint64_t q = f2_fma(f2_pack(0.0551716685f, 0.0551716685f), f, f2_pack(0.2426111251f, 0.2426111251f));
-    q = f2_fma(q, f, f2_pack(0.6932609677f, 0.6932609677f));
-    q = f2_fma(q, f, f2_pack(0.9999280572f, 0.9999280572f));
-    float q0, q1, t0, t1;
-    f2_unpack(q, q0, q1);
-    f2_unpack(t, t0, t1);
-    p0 = __int_as_float(__float_as_int(q0) + __float_as_int(t0) * 8388608);
-    p1 = __int_as_float(__float_as_int(q1) + __float_as_int(t1) * 8388608);
 }
 
 FA_DEV uint32_t pack_bf16x2(float lo, float hi) {
