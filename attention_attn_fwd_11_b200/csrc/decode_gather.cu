@@ -33,19 +33,19 @@
 //   - Partial scores (128 rows x 32 keys, fp32) are swapped through
 //     distributed shared memory every tile; both CTAs add own + peer (the
 //     same sum in either order), so both run the identical online softmax.
-//   - Warp roles (15 warps):
-//       0-3    decode: gather 32 selected rows per tile with 16-byte cp.async
-//              into 128-byte-swizzled shared memory; prefill: warp 0 loads
-//              the K and V tiles with TMA.  The ring has 6 (decode) or 4
-//              (prefill) stages; stages past the first two reuse the Q
-//              staging area once Q is in TMEM.
-//       4-7    softmax (one row per thread), O correction, epilogue.
-//       8-11   move each tile's partial scores from TMEM to the exchange slot
-//              as soon as QK^T lands, ahead of the softmax.
-//       12     TMEM allocation and MMA issue: QK^T runs two tiles ahead of
-//              PV (three S buffers).
-//       13     one bulk shared-memory copy per tile into the peer's slot.
-//       14     tells the peer when a slot it filled has been read.
+//   - Warp roles, after GW loader warps (decode GW = 8, prefill GW = 4):
+//       loaders  decode: gather 32 selected rows per tile with 16-byte
+//                cp.async into 128-byte-swizzled shared memory; prefill:
+//                the first loader warp loads the K and V tiles with TMA.
+//                The ring has 6 (decode) or 4 (prefill) stages; stages past
+//                the first two reuse the Q staging area once Q is in TMEM.
+//       +0..3    softmax (one row per thread), O correction, epilogue.
+//       +4..7    move each tile's partial scores from TMEM to the exchange
+//                slot as soon as QK^T lands, ahead of the softmax.
+//       +8       TMEM allocation and MMA issue: QK^T runs two tiles ahead of
+//                PV (three S buffers).
+//       +9       one bulk shared-memory copy per tile into the peer's slot.
+//       +10      tells the peer when a slot it filled has been read.
 //   - The epilogue stages O in 128-byte-swizzled shared memory and writes it
 //     with TMA tensor stores: split partials for the log-sum-exp combine in
 //     decode, the normalised O (and LSE) in prefill.
@@ -134,13 +134,23 @@ enum {
 };
 static_assert(G_NBAR * 8 <= 512, "barrier space");
 
-// Warp roles (480 threads).
-constexpr int LG_W_SOFT = 4;    // warps 4-7: softmax, correction, epilogue
-constexpr int LG_W_MOVE = 8;    // warps 8-11: partial scores TMEM -> xout
-constexpr int LG_W_MMA = 12;    // warp 12: TMEM allocation, MMA issue
-constexpr int LG_W_SEND = 13;   // warp 13: bulk copies xout -> the peer's xin
-constexpr int LG_W_REL = 14;    // warp 14: tells the peer its xin slot is free again
-constexpr int LG_THREADS = 15 * 32;
+// Warp roles: GW loader warps (decode: 8 row-gather warps; prefill: warp 0
+// is the TMA producer), then 4 softmax warps, 4 movers, the MMA warp, the
+// send warp and the release warp.  (8 gather warps instead of 4: +2.7 % on
+// the benchmark decode; the gather is capped per SM, not per warp.)
+#ifndef FA_LG_GATHER_WARPS
+#define FA_LG_GATHER_WARPS 8
+#endif
+template <bool DENSE>
+struct LgRoles {
+    static constexpr int GW = DENSE ? 4 : FA_LG_GATHER_WARPS;
+    static constexpr int W_SOFT = GW;        // softmax, correction, epilogue
+    static constexpr int W_MOVE = GW + 4;    // partial scores TMEM -> xout
+    static constexpr int W_MMA = GW + 8;     // TMEM allocation, MMA issue
+    static constexpr int W_SEND = GW + 9;    // bulk copies xout -> the peer's xin
+    static constexpr int W_REL = GW + 10;    // tells the peer its xin slot is free again
+    static constexpr int THREADS = (GW + 11) * 32;
+};
 
 struct GatherArgs {
     // latent decode
@@ -165,12 +175,15 @@ constexpr float kGatherRescaleThreshold = 8.0f;
 // T * 128 heads, splits, 1); prefill: O as (512, Sq, Hq, B); 32-row boxes of
 // 128 bytes, 128-byte swizzle.
 template <bool DENSE>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(LG_THREADS, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(LgRoles<DENSE>::THREADS, 1)
 latent_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmOut,
                      const GatherArgs a) {
     using C = LgCfg<DENSE>;
     constexpr int NST = C::NST, NX = C::NX, NFRESH = C::NFRESH;
+    using Rl = LgRoles<DENSE>;
+    constexpr int LG_W_SOFT = Rl::W_SOFT, LG_W_MOVE = Rl::W_MOVE, LG_W_MMA = Rl::W_MMA, LG_W_SEND = Rl::W_SEND,
+                  LG_W_REL = Rl::W_REL, GW = Rl::GW;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
@@ -240,7 +253,7 @@ latent_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             mbar_init(bar(G_XREAD + i), 128);        // softmax threads: xin has been read
         }
         for (int s = 0; s < NST; ++s) {
-            mbar_init(bar(G_FULL + s), DENSE ? 1 : 128);  // TMA producer, or every gatherer's cp.async arrival
+            mbar_init(bar(G_FULL + s), DENSE ? 1 : 32 * GW);  // TMA producer, or every gatherer's cp.async arrival
             mbar_init(bar(G_EMPTY + s), 1);
         }
         *abort_flag = 0;
@@ -330,7 +343,7 @@ latent_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                 // One thread waits for the stage to be free (PV of tile i - NST
                 // has read it; the first use of a stage in the Q area also
                 // waits until Q has moved to TMEM) and publishes the outcome,
-                // so all 128 gatherers take the same branch below.
+                // so all gatherers take the same branch below.
                 if (tid == 0) {
                     const bool g = i != NFRESH || mbar_wait(bar(G_QTMEM), 0, abort_flag, &g_gather_err);
                     *go = g && mbar_wait(bar(G_EMPTY + s), ((uint32_t)(i / NST) & 1u) ^ 1u, abort_flag,
@@ -353,14 +366,14 @@ latent_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                     if (lane == 0) maskw[s] = m;
                     if (i + 1 < n_tiles) fetch(i + 1);
                 }
-                asm volatile("bar.sync 1, 128;" ::: "memory");
+                named_bar_sync(1, 32 * GW);
                 const bool proceed = *go != 0;
-                asm volatile("bar.sync 1, 128;" ::: "memory");
+                named_bar_sync(1, 32 * GW);
                 if (!proceed) break;
                 if (tid == 0) LG_TRACE(12, i);
                 const uint32_t dst0 = stage_addr(s);
 #pragma unroll
-                for (int row = warp; row < LG_BN; row += 4) {
+                for (int row = warp; row < LG_BN; row += GW) {
                     const __nv_bfloat16 *src = a.rows + (int64_t)rowid[s * LG_BN + row] * a.row_stride + chunk0 * 64;
                     const uint32_t d = dst0 + row * 128;
                     const int x = row & 7;
@@ -761,7 +774,8 @@ cudaError_t launch_decode_gather(const GatherLaunch &L, cudaStream_t stream) {
     a.dk512 = L.dk == 512 ? 1 : 0;
     a.part_lse = L.part_lse;
     dim3 grid(2u, (unsigned)L.num_splits, (unsigned)L.T);
-    latent_decode_kernel<false><<<grid, LG_THREADS, LgCfg<false>::SMEM, stream>>>(L.tmQ, L.tmQ, L.tmQ, L.tmPO, a);
+    latent_decode_kernel<false><<<grid, LgRoles<false>::THREADS, LgCfg<false>::SMEM, stream>>>(L.tmQ, L.tmQ, L.tmQ,
+                                                                                               L.tmPO, a);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     return launch_combine(L.part_o, L.part_lse, L.T * L.Hq, L.num_splits, L.Hq, nullptr, 0, 0, L.o, L.lse, L.o_bf16,
@@ -784,7 +798,8 @@ cudaError_t launch_prefill_d512(const Dense512Launch &L, cudaStream_t stream) {
     a.dk512 = L.dk == 512 ? 1 : 0;
     a.scale_log2 = L.scale * 1.4426950408889634f;
     dim3 grid(2u, (unsigned)a.n_qt, (unsigned)(L.B * L.Hq));
-    latent_decode_kernel<true><<<grid, LG_THREADS, LgCfg<true>::SMEM, stream>>>(L.tmQ, L.tmK, L.tmV, L.tmO, a);
+    latent_decode_kernel<true><<<grid, LgRoles<true>::THREADS, LgCfg<true>::SMEM, stream>>>(L.tmQ, L.tmK, L.tmV,
+                                                                                             L.tmO, a);
     return cudaGetLastError();
 }
 

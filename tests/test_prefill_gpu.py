@@ -152,8 +152,19 @@ def test_causal_mha_config_sampled():
 
 
 def test_gqa_config_sampled():
-    """B=1, Hq=32, Hkv=8, S=4096, d=256, full -- the benchmark launch, sampled rows."""
-    check_sampled(W.GQA_FULL, n_rows=12)
+    """B=1, Hq=32, Hkv=8, S=4096, d=256, full -- the benchmark launch, checked
+    on a seeded sample of 512 query rows of every head (full attention:
+    each row depends only on its own query, so the sampled rows are the
+    oracle's exact rows)."""
+    c = W.GQA_FULL
+    q, k, v = W.prefill_inputs(c)
+    o, lse = fa.fwd(*to_dev(q, k, v), scale=c.scale, causal=False)
+    torch.cuda.synchronize()
+    assert fa.device_error() == 0
+    rows = np.sort(np.random.default_rng(4242).choice(c.Sq, 512, replace=False))
+    qb = np.ascontiguousarray(W.bits(q)[:, :, rows])
+    o_ref, l_ref = oracle.attention(qb, W.bits(k), W.bits(v), c.scale, False)
+    check(o[:, :, rows], o_ref, lse[:, :, rows], l_ref, what=c.name + " 512 sampled rows of every head")
 
 
 @pytest.mark.parametrize("d", [64, 128])
