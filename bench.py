@@ -539,6 +539,12 @@ HBM_SPEC_GBS = 8000.0  # B200 HBM3e, nominal (the ~8 TB/s the decode target is s
 def roofline(bound, achieved, peak, unit, traffic):
     r = {"bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": unit,
          "frac": round(achieved / peak, 4), "traffic": traffic}
+    if bound == "tensor":
+        # the long-loop cuBLAS figure, for kernels timed under sustained load
+        # (the headline's regions follow a quarter second of replays)
+        pk, _ = load_peaks()
+        r["peak_sustained"] = pk["bf16_tflops_sustained"]
+        r["frac_sustained"] = round(achieved / pk["bf16_tflops_sustained"], 4)
     if bound == "hbm":
         # the measured peak is a copy (half reads, half writes); a read-mostly
         # kernel can pass it, so the nominal figure is given beside it
