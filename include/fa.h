@@ -84,8 +84,11 @@ enum {
  * scale must be finite and > 0 (the caller passes 1/sqrt(dk) for standard
  * attention).
  * Supported (dk, dv): (64, 64), (128, 128), (192, 192), (256, 256),
- * (192, 128) and (320, 256) (the pairs up to dv = 256 of the llama.cpp
- * tensor path's head-size table); anything else is FA_ERR_UNSUPPORTED.
+ * (192, 128), (320, 256), (576, 512) and (512, 512) (the llama.cpp tensor
+ * path's head-size table); anything else is FA_ERR_UNSUPPORTED.  For the
+ * two dv = 512 pairs K and V are separate strided tensors (V may be a view
+ * of K's last 512 columns, the MLA latent layout) and the score modifiers
+ * below are FA_ERR_UNSUPPORTED; B * Hq and ceil(Sq / 128) must be <= 65535.
  * Sq == 0 or B == 0 is a no-op; Sk == 0 writes O = 0, LSE = -inf.
  *
  * Score modifiers (all off when zero / NULL), as the llama.cpp tensor
@@ -156,7 +159,8 @@ fa_status fa_fwd(const fa_fwd_params *p, void *stream);
  *   o: [B, Hq, Sq, dv] (o_dtype) with strides o_sb, o_sh, o_ss (multiples of
  *     4 elements for fp32, 8 for bf16; o_ss >= dv); lse: NULL or [B, Hq, Sq]
  *     fp32 contiguous.
- * Supported: the (dk, dv) pairs of fa_fwd, block_size == 64, Hq % Hkv == 0.
+ * Supported: the (dk, dv) pairs of fa_fwd up to dv = 256, block_size == 64,
+ * Hq % Hkv == 0.
  * Score modifiers: as in fa_fwd (mask, max_bias, softcap, sinks), with the
  *   mask element (b, h, i, j) at b*m_sb + h*m_sh + i*m_ss + j for new row i
  *   and key j of the sequence (j < seq_lens[b]); m_ss must be >= every

@@ -67,12 +67,27 @@ def fwd_params(**kw):
     (dict(mask=16, m_ss=120), fa.FA_ERR_INVALID_ARG),         # row stride < Sk
     (dict(mask=16, m_ss=128, m_sh=4), fa.FA_ERR_INVALID_ARG),  # head stride not a multiple of 8
     (dict(sinks=2), fa.FA_ERR_INVALID_ARG),                   # sinks not 4-byte aligned
+    # the dv = 512 pairs: separate K and V, no score modifiers
+    (dict(dk=576, dv=256), fa.FA_ERR_UNSUPPORTED),
+    (dict(dk=256, dv=512), fa.FA_ERR_UNSUPPORTED),
+    (dict(dk=576, dv=512, o_ss=512, softcap=30.0), fa.FA_ERR_UNSUPPORTED),
+    (dict(dk=512, dv=512, o_ss=512, mask=16, m_ss=128), fa.FA_ERR_UNSUPPORTED),
+    (dict(dk=576, dv=512, o_ss=512, sinks=16), fa.FA_ERR_UNSUPPORTED),
+    (dict(dk=576, dv=512, o_ss=512, max_bias=8.0), fa.FA_ERR_UNSUPPORTED),
+    (dict(dk=576, dv=512, o_ss=510), fa.FA_ERR_INVALID_ARG),  # o rows shorter than dv
 ])
 def test_fwd_rejects(kw, status):
     lib = fa.load()
     st = lib.fa_fwd(ctypes.byref(fwd_params(**kw)), None)
     assert st == status, lib.fa_last_error()
     assert lib.fa_last_error().decode().startswith("fa_fwd")
+
+
+def test_fwd_accepts_the_dv512_pairs():
+    # accepted by validation: with Sq == 0 nothing is launched
+    lib = fa.load()
+    for dk in (576, 512):
+        assert lib.fa_fwd(ctypes.byref(fwd_params(dk=dk, dv=512, o_ss=512, Sq=0)), None) == fa.FA_OK
 
 
 def test_fwd_null_params_and_noop():
