@@ -10,9 +10,9 @@
 //   - one producer warp resolves block ids through the block table (32 table
 //     entries per coalesced read) and moves each block's K and V tile with
 //     TMA tensor copies into a 3-stage, 128-byte-swizzled shared-memory ring;
-//   - four consumer warps each own 16 of the block's 64 keys.  The small
-//     contractions run as warp-level bf16 MMAs (m16n8k16, fp32 accumulate):
-//     the query heads are the M rows (padded to 16), so QK^T is 16 MMAs and
+//   - four MMA warps each own 16 of the block's 64 keys.  The small contractions run as
+//     warp-level bf16 MMAs (m16n8k16, fp32 accumulate): the query heads are
+//     the M rows (padded to 16, only rows 0..7 kept), so QK^T is 16 MMAs and
 //     PV 16 MMAs per warp per block, with the score fragments reused directly
 //     as the P operand; swizzled ldmatrix reads are bank-conflict free.
 //     (The 128-row tcgen05 MMA would leave 124 of 128 rows idle here and
@@ -40,6 +40,27 @@ namespace fa {
 
 static __device__ int g_decode_err;
 
+#ifdef FA_PD_TRACE
+// Debug-only timeline: clock64 stamps of one CTA in fixed slots [event][tile
+// < 64], and per CTA its start / end (global timer) and SM.
+#ifndef FA_PD_TRACE_B
+#define FA_PD_TRACE_B 0
+#endif
+constexpr int kPdTraceCap = 16 * 64, kPdCtaCap = 3 * 4096;
+static __device__ unsigned long long g_pd_trace[kPdTraceCap];
+static __device__ unsigned long long g_pd_cta[kPdCtaCap];
+#define PD_TRACE(ev, i) \
+    do { if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == FA_PD_TRACE_B && (i) < 64) g_pd_trace[(ev) * 64 + (i)] = clock64(); } while (0)
+FA_DEV unsigned long long pd_gtimer() { unsigned long long t; asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t)); return t; }
+FA_DEV unsigned pd_smid() { unsigned r; asm volatile("mov.u32 %0, %%smid;" : "=r"(r)); return r; }
+#define PD_CTA(slot, v) \
+    do { const int cid_ = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z); \
+         if (3 * cid_ + 2 < kPdCtaCap) g_pd_cta[3 * cid_ + (slot)] = (v); } while (0)
+#else
+#define PD_TRACE(ev, i) ((void)0)
+#define PD_CTA(slot, v) ((void)0)
+#endif
+
 constexpr int PD_D = 128;
 constexpr int PD_BS = 64;
 constexpr int PD_NST = 3;
@@ -48,17 +69,35 @@ constexpr int PD_STAGE = 2 * PD_TILE;            // K + V
 constexpr int PD_OFF_BAR = PD_NST * PD_STAGE;
 constexpr int PD_SMEM = PD_OFF_BAR + 128 + 1024;  // ring + barriers + 1024-byte alignment slack
 
-// q8_0 caches (the dequant prologue): a cache row is 4 ggml q8_0 blocks
-// (f16 scale + 32 int8 codes, 34 bytes), 136 bytes for 128 values.  A
-// (block, head) tile of K or V is 64 such rows, contiguous, moved with one
-// bulk copy.  Each consumer warp converts its own 16 keys of K and V into a
-// private bf16 buffer laid out like the bf16 ring (two 64-column halves,
-// 128-byte swizzle), then runs the bf16 path on it.
-#ifndef FA_PD_Q8_PRMT
-#define FA_PD_Q8_PRMT 1
+// Quantised caches (the dequant prologue): q8_0 rows are 4 ggml q8_0 blocks
+// (f16 scale + 32 int8 codes, 34 bytes), 136 bytes for 128 values; q4_0 rows
+// 4 blocks of 18 bytes (72 bytes); FP8 E4M3 rows one byte a value (128
+// bytes) with one fp32 scale per tensor (k_scale, v_scale).  A (block, head)
+// tile of K or V is 64 such rows, contiguous, moved with one bulk copy into
+// a raw ring.  Eight converter warps turn each raw tile into the bf16 tile
+// the bf16 path reads (two 64-column halves, 128-byte swizzle, exactly the
+// layout of the TMA-filled bf16 ring) in a second ring, from which the four
+// MMA warps run the unchanged bf16 path.  Conversion and MMAs thus overlap
+// across warps instead of following one another inside each warp.
+#ifndef FA_PDQ_NR
+#define FA_PDQ_NR 4
 #endif
-// FP8 E4M3 caches take the same prologue with 128-byte rows (one byte per
-// value) and one fp32 scale per tensor (k_scale, v_scale).
+#ifndef FA_PDQ_NB
+#define FA_PDQ_NB 4
+#endif
+#ifndef FA_PDQ_NCV
+#define FA_PDQ_NCV 4
+#endif
+constexpr int PDQ_NCV = FA_PDQ_NCV;                // converter warps (4 doing K and V, or 8)
+static_assert(PDQ_NCV == 8 || PDQ_NCV == 4, "converter warps");
+// Groups of four MMA warps taking alternate blocks (each group with its own
+// online softmax, all warps merging at the end).  One group: two groups
+// (eight MMA warps) measured 3-8 % slower on every cache type.
+constexpr int PD_NG = 1;
+constexpr int PD_MMA_WARPS = 4 * PD_NG;
+constexpr int PD_THREADS = (PD_MMA_WARPS + 1) * 32;            // bf16: MMA warps + the producer
+constexpr int PDQ_THREADS = (PD_MMA_WARPS + 1 + PDQ_NCV) * 32;  // quantised: + the converters
+static_assert((PD_MMA_WARPS * 8 * PD_D + 2 * PD_MMA_WARPS * 8) * 4 <= PD_NST * PD_STAGE, "merge area");
 //
 // Raw-tile geometry per cache type KVT (8 = q8_0, 4 = q4_0, 2 = fp8 e4m3):
 template <int KVT>
@@ -66,53 +105,183 @@ struct PdRaw {
     static constexpr int ROW = KVT == 8 ? 136 : (KVT == 4 ? 72 : 128);  // bytes per cache row of 128 values
     static constexpr int TILE = PD_BS * ROW;                  // one (block, head) tile of K or V
     static constexpr int STAGE = 2 * TILE;                    // K + V (1024-byte multiple)
-    // Two raw stages keep the CTA at about 68 KB of shared memory, so three
-    // CTAs (twelve converting warps) share an SM: the in-warp conversion is
-    // latency-bound, and occupancy, not ring depth, feeds it.
-    static constexpr int NST = 2;
-    static constexpr int WBUF = 2 * 16 * PD_D * 2;            // one warp's 16 keys of K and V in bf16: 8 KB
-    static constexpr int OFF_WB = NST * STAGE;
-    static constexpr int OFF_BAR = OFF_WB + 4 * WBUF;
-    static constexpr int SMEM = OFF_BAR + 128 + 1024;
+    static constexpr int NR = FA_PDQ_NR;                      // raw stages
+    static constexpr int NB = FA_PDQ_NB;                      // bf16 stages (PD_STAGE bytes each)
+    static constexpr int OFF_RAW = NB * PD_STAGE;             // the bf16 ring starts at 0
+    static constexpr int OFF_BAR = OFF_RAW + NR * STAGE;
+    static constexpr int SMEM = OFF_BAR + 256 + 1024;
     static_assert(STAGE % 1024 == 0, "stage alignment");
+    static_assert(TILE % 16 == 0, "bulk copy size");
+    static_assert(SMEM <= 232448, "shared memory budget");
+    static_assert((PD_MMA_WARPS * 8 * PD_D + 2 * PD_MMA_WARPS * 8) * 4 <= NB * PD_STAGE, "merge area");
 };
 
-// Two int8 codes (low and high byte of w) times the block scale d -> a bf16
-// pair.  A code's byte xor 0x80 is code + 128; OR-ed into the mantissa of
-// 2^23 it gives 2^23 + code + 128 exactly, and subtracting 2^23 + 128
-// leaves the code (both steps exact).  code * d is exact in fp32 (8 + 11
-// significant bits), so the bf16 conversion is the only rounding -- the
-// same value the pre-pass (fa_kv_dequant) writes.
-FA_DEV uint32_t q8_pair_to_bf16(uint32_t w, uint64_t d2) {
-#if FA_PD_Q8_PRMT
-    // byte permutes build both fp32 patterns; the subtract and the scale run
-    // as packed fp32 pairs
-    const uint32_t x = w ^ 0x8080u;
-    const uint64_t f = f2_pack(__uint_as_float(__byte_perm(x, 0x4B000000u, 0x7440)),
-                               __uint_as_float(__byte_perm(x, 0x4B000000u, 0x7441)));
+// Two int8 codes at byte offset OFF (0 or 2) of a word whose bytes were
+// already xor-ed with 0x80, times the block scale d -> a bf16 pair.  A
+// code's byte xor 0x80 is code + 128; OR-ed into the mantissa of 2^23 it
+// gives 2^23 + code + 128 exactly, and subtracting 2^23 + 128 leaves the
+// code (both steps exact).  code * d is exact in fp32 (8 + 11 significant
+// bits), so the bf16 conversion is the only rounding -- the same value the
+// pre-pass (fa_kv_dequant) writes.
+template <int OFF>
+FA_DEV uint32_t q8_pair_to_bf16(uint32_t x, uint64_t d2) {
+    const uint64_t f = f2_pack(__uint_as_float(__byte_perm(x, 0x4B000000u, 0x7440 + OFF)),
+                               __uint_as_float(__byte_perm(x, 0x4B000000u, 0x7441 + OFF)));
     float a, b;
     f2_unpack(f2_mul(f2_add(f, f2_pack(-8388736.f, -8388736.f)), d2), a, b);
     return pack_bf16x2(a, b);
-#else
-    float d, d_;
-    f2_unpack(d2, d, d_);
-    const float f0 = __uint_as_float(0x4B000000u | ((w & 0xffu) ^ 0x80u)) - 8388736.f;
-    const float f1 = __uint_as_float(0x4B000000u | (((w >> 8) & 0xffu) ^ 0x80u)) - 8388736.f;
-    return pack_bf16x2(f0 * d, f1 * d);
-#endif
 }
 
-// Two 4-bit codes n0, n1 (bits 0-3 and 8-11 of x) -> the bf16 pair
-// d (n0 - 8), d (n1 - 8).  OR-ed into the mantissa of 2^23 a code gives
-// 2^23 + n exactly; subtracting 2^23 + 8 leaves n - 8, and the product with
-// d is exact in fp32 (4 + 11 significant bits), so the bf16 conversion is
-// the only rounding, as in the pre-pass.
+// Two 4-bit codes n0, n1 (bytes OFF and OFF + 1 of x, each byte < 16) ->
+// the bf16 pair d (n0 - 8), d (n1 - 8).  OR-ed into the mantissa of 2^23 a
+// code gives 2^23 + n exactly; subtracting 2^23 + 8 leaves n - 8, and the
+// product with d is exact in fp32 (4 + 11 significant bits), so the bf16
+// conversion is the only rounding, as in the pre-pass.
+template <int OFF>
 FA_DEV uint32_t q4_pair_to_bf16(uint32_t x, uint64_t d2) {
-    const uint64_t f = f2_pack(__uint_as_float(0x4B000000u | (x & 0xfu)), __uint_as_float(0x4B000000u | ((x >> 8) & 0xfu)));
+    const uint64_t f = f2_pack(__uint_as_float(__byte_perm(x, 0x4B000000u, 0x7440 + OFF)),
+                               __uint_as_float(__byte_perm(x, 0x4B000000u, 0x7441 + OFF)));
     float a, b;
     f2_unpack(f2_mul(f2_add(f, f2_pack(-8388616.f, -8388616.f)), d2), a, b);
     return pack_bf16x2(a, b);
 }
+
+// Two e4m3 bytes (the low 16 bits of w) times the tensor scale -> a bf16
+// pair: e4m3 -> f16 is exact, f16 -> f32 is exact, the fp32 product rounds
+// once before the bf16 conversion (the pre-pass forms it in fp64 and rounds
+// once).
+FA_DEV uint32_t e4m3_pair_to_bf16(uint32_t w, uint64_t sc2) {
+    const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w & 0xffffu), __NV_E4M3);
+    const float2 f = __half22float2(__half2(hr));
+    float x0, x1;
+    f2_unpack(f2_mul(f2_pack(f.x, f.y), sc2), x0, x1);
+    return pack_bf16x2(x0, x1);
+}
+
+// The 64 values of one half-row (tensor t, row r, half h) of a q8_0 or q4_0
+// raw tile, as 32 bf16 pairs in order.  A lane's half-row is two whole
+// quant blocks; it is read as aligned 32-bit words (row pitches 136 and 72
+// bytes keep the halves 4-byte aligned).
+//   q8_0 (68 bytes, 17 words): [scale | codes 0, 1] in word 0, codes 2..29
+//   in words 1-7, [codes 30, 31 | block 1's scale] in word 8, block 1's
+//   codes in words 9-16.  Code pair k of block 0 sits at byte 2 of word
+//   (k + 1) / 2 for even k, byte 0 for odd k; of block 1 at byte 0 (even k)
+//   or 2 (odd k) of word 9 + k / 2.
+//   q4_0 (36 bytes, 9 words): [scale | bytes 0, 1] in word 0, bytes 2..13
+//   in words 1-3, [bytes 14, 15 | block 1's scale] in word 4, block 1's 16
+//   bytes in words 5-8.  Byte j of a block holds value j in its low nibble
+//   and value j + 16 in its high nibble, so value pair k < 8 is the low
+//   nibbles of bytes 2k, 2k + 1 and pair k >= 8 the high nibbles of bytes
+//   2 (k - 8), 2 (k - 8) + 1; byte pair m of block 0 sits at byte 2 of word
+//   (m + 1) / 2 for even m, byte 0 for odd m; of block 1 at byte 0 (even m)
+//   or 2 (odd m) of word 5 + m / 2.
+template <int KVT>
+FA_DEV void convert_half_row(const uint8_t *src, uint32_t (&pr)[32]) {
+    if constexpr (KVT == 8) {
+        const uint32_t *wp = reinterpret_cast<const uint32_t *>(src);
+        uint32_t wd[17];
+#pragma unroll
+        for (int i = 0; i < 17; ++i) wd[i] = wp[i];
+        const float d0 = __half2float(__ushort_as_half((unsigned short)(wd[0] & 0xffffu)));
+        const float d1 = __half2float(__ushort_as_half((unsigned short)(wd[8] >> 16)));
+        const uint64_t d02 = f2_pack(d0, d0), d12 = f2_pack(d1, d1);
+#pragma unroll
+        for (int i = 0; i < 17; ++i) wd[i] ^= 0x80808080u;  // code + 128 in every byte
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            pr[k] = (k & 1) ? q8_pair_to_bf16<0>(wd[(k + 1) >> 1], d02) : q8_pair_to_bf16<2>(wd[(k + 1) >> 1], d02);
+            pr[16 + k] = (k & 1) ? q8_pair_to_bf16<2>(wd[9 + (k >> 1)], d12) : q8_pair_to_bf16<0>(wd[9 + (k >> 1)], d12);
+        }
+    } else {
+        const uint32_t *wp = reinterpret_cast<const uint32_t *>(src);
+        uint32_t wd[9];
+#pragma unroll
+        for (int i = 0; i < 9; ++i) wd[i] = wp[i];
+        const float d0 = __half2float(__ushort_as_half((unsigned short)(wd[0] & 0xffffu)));
+        const float d1 = __half2float(__ushort_as_half((unsigned short)(wd[4] >> 16)));
+        const uint64_t d02 = f2_pack(d0, d0), d12 = f2_pack(d1, d1);
+        uint32_t lo[9], hi[9];
+#pragma unroll
+        for (int i = 0; i < 9; ++i) {
+            lo[i] = wd[i] & 0x0F0F0F0Fu;
+            hi[i] = (wd[i] >> 4) & 0x0F0F0F0Fu;
+        }
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            const int m = k & 7;  // byte pair of the block
+            const uint32_t *nb = k < 8 ? lo : hi;
+            pr[k] = (m & 1) ? q4_pair_to_bf16<0>(nb[(m + 1) >> 1], d02) : q4_pair_to_bf16<2>(nb[(m + 1) >> 1], d02);
+            pr[16 + k] = (m & 1) ? q4_pair_to_bf16<2>(nb[5 + (m >> 1)], d12) : q4_pair_to_bf16<0>(nb[5 + (m >> 1)], d12);
+        }
+    }
+}
+
+// Converter warp cw (0..7) turns its share of raw stage `raw` into bf16
+// stage `bf`: warps 0-3 take K, 4-7 take V, each 16 rows of the 64.
+//   q8_0 / q4_0: lane (r = 16 (cw % 4) + lane % 16, h = lane / 16) converts
+//   half h of row r (64 values), 8 bf16 chunks of 16 bytes.  Word reads hit
+//   32 distinct banks (row pitches of 34 or 18 words); in each quarter-warp
+//   of a 16-byte store the 8 lanes write 8 rows at 8 distinct chunk slots.
+//   FP8: in each of 4 steps lane (R = 16 (cw % 4) + 4 step + lane / 8, U =
+//   lane % 8) converts the 16 bytes U of row R (one conflict-free 16-byte
+//   read per lane), values 16 U .. 16 U + 15: bf16 chunks 2 U, 2 U + 1 (mod
+//   8) of half U / 4.  Lanes with U >= 4 store their odd chunk first, so the
+//   8 lanes of a quarter-warp again hit 8 distinct chunk slots.
+// The loads all come first: the caller releases the raw stage between
+// `load` and `store`.
+template <int KVT>
+struct Converter {
+    using R = PdRaw<KVT>;
+    uint32_t pr[32];
+    FA_DEV void load(const uint8_t *raw, int t, int rg, int lane, float k_scale, float v_scale) {
+        if constexpr (KVT == 2) {
+            const uint64_t sc2 = t == 0 ? f2_pack(k_scale, k_scale) : f2_pack(v_scale, v_scale);
+            uint4 u[4];
+#pragma unroll
+            for (int st = 0; st < 4; ++st) {
+                const int row = rg * 16 + 4 * st + (lane >> 3);
+                u[st] = *reinterpret_cast<const uint4 *>(raw + t * R::TILE + row * R::ROW + 16 * (lane & 7));
+            }
+#pragma unroll
+            for (int st = 0; st < 4; ++st) {
+                const uint32_t w[4] = {u[st].x, u[st].y, u[st].z, u[st].w};
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    pr[8 * st + 2 * k] = e4m3_pair_to_bf16(w[k], sc2);
+                    pr[8 * st + 2 * k + 1] = e4m3_pair_to_bf16(w[k] >> 16, sc2);
+                }
+            }
+        } else {
+            const int row = rg * 16 + (lane & 15), h = lane >> 4;
+            convert_half_row<KVT>(raw + t * R::TILE + row * R::ROW + (R::ROW / 2) * h, pr);
+        }
+    }
+    FA_DEV void store(uint8_t *bf, int t, int rg, int lane) const {
+        uint8_t *dst = bf + t * PD_TILE;
+        if constexpr (KVT == 2) {
+            const int U = lane & 7;
+            const bool odd_first = U >= 4;
+#pragma unroll
+            for (int st = 0; st < 4; ++st) {
+                const int row = rg * 16 + 4 * st + (lane >> 3);
+                uint8_t *rp = dst + (U >> 2) * (PD_TILE / 2) + row * 128;
+                const uint4 a = make_uint4(pr[8 * st], pr[8 * st + 1], pr[8 * st + 2], pr[8 * st + 3]);
+                const uint4 b = make_uint4(pr[8 * st + 4], pr[8 * st + 5], pr[8 * st + 6], pr[8 * st + 7]);
+                const int ca = (2 * U) & 7, cb = (2 * U + 1) & 7;
+                const int c0 = odd_first ? cb : ca, c1 = odd_first ? ca : cb;
+                *reinterpret_cast<uint4 *>(rp + ((c0 ^ (row & 7)) << 4)) = odd_first ? b : a;
+                *reinterpret_cast<uint4 *>(rp + ((c1 ^ (row & 7)) << 4)) = odd_first ? a : b;
+            }
+        } else {
+            const int row = rg * 16 + (lane & 15), h = lane >> 4;
+            uint8_t *rp = dst + h * (PD_TILE / 2) + row * 128;
+#pragma unroll
+            for (int j = 0; j < 8; ++j)  // chunk j of the half-row: values 8 j .. 8 j + 7
+                *reinterpret_cast<uint4 *>(rp + ((j ^ (row & 7)) << 4)) =
+                    make_uint4(pr[4 * j], pr[4 * j + 1], pr[4 * j + 2], pr[4 * j + 3]);
+        }
+    }
+};
 
 struct PagedArgs {
     const __nv_bfloat16 *q;
@@ -129,9 +298,12 @@ struct PagedArgs {
     int stall;
 };
 
-// Quantised caches: three CTAs per SM (at most 136 registers a thread).
+// bf16 caches: one CTA of 160 threads per SM (its ring fills shared memory).
+// Quantised caches: one CTA of 288 threads per SM.  A sub-partition of the
+// SM holds 16 K registers and runs at most 3 of the 9 warps, so a thread
+// gets up to 168.
 template <int G, int KVT>
-__global__ void __launch_bounds__(160, KVT ? 3 : 1) paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
+__global__ void __launch_bounds__(KVT ? PDQ_THREADS : PD_THREADS, 1) paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                                                            const __grid_constant__ CUtensorMap tmV,
                                                            const PagedArgs a) {
     extern __shared__ uint8_t smem_raw[];
@@ -149,25 +321,48 @@ __global__ void __launch_bounds__(160, KVT ? 3 : 1) paged_decode_kernel(const __
     const int blk0 = split * a.bps;
     if (blk0 >= nb) return;  // this split holds no key of this sequence (uniform exit)
     const int nblk = min(a.bps, nb - blk0);
+#ifdef FA_PD_TRACE
+    if (threadIdx.x == 0) { PD_CTA(0, pd_gtimer()); PD_CTA(2, pd_smid() | ((unsigned long long)nblk << 16)); }
+    PD_TRACE(15, 0);
+#endif
 
     constexpr bool KVQ = KVT != 0;
     using R = PdRaw<KVQ ? KVT : 8>;
-    constexpr int NST = KVQ ? R::NST : PD_NST;
-    constexpr int STAGE = KVQ ? R::STAGE : PD_STAGE;
+    // The producer's ring (bf16 stages filled by TMA, or raw stages) and the
+    // ring the MMA warps read (the same one for bf16; the converted bf16
+    // stages for quantised caches).
+    constexpr int NP = KVQ ? R::NR : PD_NST;
+    constexpr int NC = KVQ ? R::NB : PD_NST;
     constexpr int OFF_BAR = KVQ ? R::OFF_BAR : PD_OFF_BAR;
     const uint32_t sbase = smem_u32(smem);
     const uint32_t bar0 = sbase + OFF_BAR;
-    auto full = [&](int s) { return bar0 + 8u * s; };
-    auto empty = [&](int s) { return bar0 + 8u * (NST + s); };
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_BAR + 8 * 2 * NST);
-    const uint32_t stall_bar = bar0 + 8u * (2 * NST + 1);  // a.stall only: never arrived on
+    // barriers: pfull[NP], pempty[NP], then (quantised) cfull[NC], cempty[NC]
+    auto pfull = [&](int s) { return bar0 + 8u * s; };
+    auto pempty = [&](int s) { return bar0 + 8u * (NP + s); };
+    auto cfull = [&](int s) { return KVQ ? bar0 + 8u * (2 * NP + s) : pfull(s); };
+    auto cempty = [&](int s) { return KVQ ? bar0 + 8u * (2 * NP + NC + s) : pempty(s); };
+    constexpr int NBARS = KVQ ? 2 * (NP + NC) : 2 * NP;
+    // Tile i sits in stage i % NC and is read by MMA group i % PD_NG.  With
+    // NC a multiple of PD_NG every tile of a stage belongs to the same group,
+    // so when a group waits for phase k of a stage's full barrier it has
+    // itself consumed phase k - 1: the barrier is at most one phase away and
+    // the parity wait cannot pass on an older phase.
+    static_assert(NC % PD_NG == 0, "ring stages per MMA group");
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_BAR + 8 * NBARS);
+    const uint32_t stall_bar = bar0 + 8u * (NBARS + 1);  // a.stall only: never arrived on
     const unsigned long long wait_ns = a.wait_ns;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
-        for (int s = 0; s < NST; ++s) {
-            mbar_init(full(s), 1);
-            mbar_init(empty(s), 4);
+        for (int s = 0; s < NP; ++s) {
+            mbar_init(pfull(s), 1);
+            mbar_init(pempty(s), KVQ ? PDQ_NCV : 4);
+        }
+        if (KVQ) {
+            for (int s = 0; s < NC; ++s) {
+                mbar_init(cfull(s), PDQ_NCV);
+                mbar_init(cempty(s), 4);
+            }
         }
         mbar_init(stall_bar, 1);
         *abort_flag = 0;
@@ -175,7 +370,7 @@ __global__ void __launch_bounds__(160, KVT ? 3 : 1) paged_decode_kernel(const __
     }
     __syncthreads();
 
-    if (warp == 4) {
+    if (warp == PD_MMA_WARPS) {
         // ---------------------------------------------------- producer --
         if (!KVQ && lane == 0) {
             prefetch_tmap(&tmK);
@@ -193,42 +388,75 @@ __global__ void __launch_bounds__(160, KVT ? 3 : 1) paged_decode_kernel(const __
                 }
             }
             const int blk = __shfl_sync(0xffffffffu, ids, i & 31);
-            const int s = i % NST;
-            const uint32_t ph = (uint32_t)(i / NST) & 1u;
+            const int s = i % NP;
+            const uint32_t ph = (uint32_t)(i / NP) & 1u;
             bool ok = true;
-            if (lane == 0) ok = mbar_wait(empty(s), ph ^ 1u, abort_flag, &g_decode_err, wait_ns);
+            if (lane == 0) ok = mbar_wait(pempty(s), ph ^ 1u, abort_flag, &g_decode_err, wait_ns);
             if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
             if (lane == 0) {
                 if constexpr (KVQ) {
                     const int64_t off = ((int64_t)blk * a.Hkv + hkv) * R::TILE;  // this (block, head) tile
-                    const uint32_t dst = sbase + s * R::STAGE;
-                    mbar_arrive_expect_tx(full(s), R::STAGE);
-                    bulk_load(dst, a.kq + off, R::TILE, full(s));
-                    bulk_load(dst + R::TILE, a.vq + off, R::TILE, full(s));
+                    const uint32_t dst = sbase + R::OFF_RAW + s * R::STAGE;
+                    mbar_arrive_expect_tx(pfull(s), R::STAGE);
+                    bulk_load(dst, a.kq + off, R::TILE, pfull(s));
+                    bulk_load(dst + R::TILE, a.vq + off, R::TILE, pfull(s));
                 } else {
                     const int row0 = (blk * a.Hkv + hkv) * PD_BS;  // first cache row of this (block, head)
                     const uint32_t dst = sbase + s * PD_STAGE;
-                    mbar_arrive_expect_tx(full(s), PD_STAGE);
-                    tma_load_2d(dst, &tmK, full(s), 0, row0);
-                    tma_load_2d(dst + PD_TILE / 2, &tmK, full(s), 64, row0);
-                    tma_load_2d(dst + PD_TILE, &tmV, full(s), 0, row0);
-                    tma_load_2d(dst + PD_TILE + PD_TILE / 2, &tmV, full(s), 64, row0);
+                    mbar_arrive_expect_tx(pfull(s), PD_STAGE);
+                    tma_load_2d(dst, &tmK, pfull(s), 0, row0);
+                    tma_load_2d(dst + PD_TILE / 2, &tmK, pfull(s), 64, row0);
+                    tma_load_2d(dst + PD_TILE, &tmV, pfull(s), 0, row0);
+                    tma_load_2d(dst + PD_TILE + PD_TILE / 2, &tmV, pfull(s), 64, row0);
                 }
             }
             issued = i + 1;
+            if (lane == 0) PD_TRACE(0, i);
         }
         if (lane == 0 && *abort_flag) {
-            for (int i = max(0, issued - NST); i < issued; ++i)
-                mbar_wait_drain(full(i % NST), (uint32_t)(i / NST) & 1u);
+            for (int i = max(0, issued - NP); i < issued; ++i)
+                mbar_wait_drain(pfull(i % NP), (uint32_t)(i / NP) & 1u);
         }
         return;
     }
 
-    // --------------------------------------------------------- consumers --
-    // Warp w owns keys [16 w, 16 w + 16) of every block.  MMA fragment roles:
+    if constexpr (KVQ) {
+        if (warp > PD_MMA_WARPS) {
+            // ------------------------------------------------- converters --
+            const int cw = warp - PD_MMA_WARPS - 1;
+            constexpr int NT = 8 / PDQ_NCV;  // tensors (K, V) per converter warp
+            Converter<KVT> cv[NT];
+            for (int i = 0; i < nblk; ++i) {
+                const int s = i % NP, sb = i % NC;
+                if (!mbar_wait(pfull(s), (uint32_t)(i / NP) & 1u, abort_flag, &g_decode_err, wait_ns)) break;
+                if (lane == 0 && cw == 0) PD_TRACE(1, i);
+#pragma unroll
+                for (int j = 0; j < NT; ++j)
+                    cv[j].load(smem + R::OFF_RAW + s * R::STAGE, NT == 1 ? cw >> 2 : j, NT == 1 ? cw & 3 : cw, lane,
+                               a.k_scale, a.v_scale);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(pempty(s));  // the raw stage may be refilled now
+                if (lane == 0 && cw == 0) PD_TRACE(2, i);
+                if (!mbar_wait(cempty(sb), ((uint32_t)(i / NC) & 1u) ^ 1u, abort_flag, &g_decode_err, wait_ns)) break;
+                if (lane == 0 && cw == 0) PD_TRACE(3, i);
+#pragma unroll
+                for (int j = 0; j < NT; ++j) cv[j].store(smem + sb * PD_STAGE, NT == 1 ? cw >> 2 : j, NT == 1 ? cw & 3 : cw, lane);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(cfull(sb));
+                if (lane == 0 && cw == 0) PD_TRACE(4, i);
+                if (lane == 0 && cw == 7) PD_TRACE(5, i);
+            }
+            return;
+        }
+    }
+
+    // ------------------------------------------------------- MMA warps --
+    // Group grp = w / 4 takes blocks grp, grp + PD_NG, ...; warp w owns keys
+    // [16 wq, 16 wq + 16) of each of them, wq = w % 4.  MMA fragment roles:
     // gid = lane / 4 is the M row (query head, valid when gid < G), tig =
     // lane % 4 picks the column pairs.
     const int gid = lane >> 2, tig = lane & 3;
+    const int grp = warp >> 2, wq = warp & 3;
     const bool head_ok = gid < G;
     uint32_t qa[8][2];
     {
@@ -242,132 +470,32 @@ __global__ void __launch_bounds__(160, KVT ? 3 : 1) paged_decode_kernel(const __
     }
     const float c = a.scale_log2;
     float m_run = -INFINITY, l_run = 0.f;
-    float o[16][4];
+    // O rows of the query heads (the MMA's M rows 0..7; rows 8..15 are
+    // padding and never kept)
+    float o[16][2];
 #pragma unroll
-    for (int nt = 0; nt < 16; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) o[nt][e] = 0.f;
+    for (int nt = 0; nt < 16; ++nt) o[nt][0] = o[nt][1] = 0.f;
     // ldmatrix lane roles: matrix mi = lane / 8, row lr = lane % 8
     const int mi = lane >> 3, lr = lane & 7;
 
     // a.stall: the wait that runs out (nothing arrives on stall_bar)
     bool ok = !a.stall || mbar_wait(stall_bar, 0, abort_flag, &g_decode_err, wait_ns);
-    for (int i = 0; ok && i < nblk; ++i) {
-        const int s = i % NST;
-        if (!mbar_wait(full(s), (uint32_t)(i / NST) & 1u, abort_flag, &g_decode_err, wait_ns)) {
+    for (int i = grp; ok && i < nblk; i += PD_NG) {
+        const int s = i % NC;
+        if (lane == 0 && warp == 0) PD_TRACE(6, i);
+        if (!mbar_wait(cfull(s), (uint32_t)(i / NC) & 1u, abort_flag, &g_decode_err, wait_ns)) {
             ok = false;
             break;
         }
-        // K and V tiles of this warp's keys: the ring stage (bf16), or the
-        // warp's private buffer after the q8_0 prologue.  `kof` maps a key of
-        // the block to its row in the tile; `hstr` is the byte distance
-        // between the two 64-column halves.
-        uint32_t sK, sV, hstr;
-        int kof;
-        if constexpr (KVT == 2) {
-            // lane (lk, h) converts row lk's half h (64 fp8 bytes) of K and of
-            // V: e4m3 pairs -> f16 pairs (exact) -> f32 times the tensor scale
-            // -> a bf16 pair.  (The fp32 product rounds once before the bf16
-            // conversion; the pre-pass forms it in fp64 and rounds once.)
-            const int lk = lane >> 1, h = lane & 1;
-            const uint8_t *raw = smem + s * R::STAGE + (warp * 16 + lk) * R::ROW + 64 * h;
-            uint8_t *wb = smem + R::OFF_WB + warp * R::WBUF + h * (16 * 128) + lk * 128;
-#pragma unroll
-            for (int t = 0; t < 2; ++t) {  // K, then V
-                const uint64_t sc2 = t == 0 ? f2_pack(a.k_scale, a.k_scale) : f2_pack(a.v_scale, a.v_scale);
-                uint4 bytes[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) bytes[i] = *reinterpret_cast<const uint4 *>(raw + t * R::TILE + 16 * i);
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {  // 16-byte output chunk j: values 8 j .. 8 j + 7
-                    const uint32_t w0 = (&bytes[j >> 1].x)[(j & 1) * 2], w1 = (&bytes[j >> 1].x)[(j & 1) * 2 + 1];
-                    uint32_t outw[4];
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const uint32_t w = k < 2 ? w0 : w1;
-                        const __half2_raw hr =
-                            __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)((w >> (16 * (k & 1))) & 0xffffu), __NV_E4M3);
-                        const float2 f = __half22float2(__half2(hr));
-                        float x0, x1;
-                        f2_unpack(f2_mul(f2_pack(f.x, f.y), sc2), x0, x1);
-                        outw[k] = pack_bf16x2(x0, x1);
-                    }
-                    *reinterpret_cast<uint4 *>(wb + t * (2 * 16 * 128) + ((j ^ (lk & 7)) << 4)) =
-                        make_uint4(outw[0], outw[1], outw[2], outw[3]);
-                }
-            }
-        } else if constexpr (KVT == 4) {
-            // lane (lk, h) converts row lk's half h (two q4_0 blocks of 18
-            // bytes, 64 values) of K and of V.  In a block, byte j holds value
-            // j in its low nibble and value j + 16 in its high nibble.
-            const int lk = lane >> 1, h = lane & 1;
-            const uint8_t *raw = smem + s * R::STAGE + (warp * 16 + lk) * R::ROW + 36 * h;
-            uint8_t *wb = smem + R::OFF_WB + warp * R::WBUF + h * (16 * 128) + lk * 128;
-#pragma unroll
-            for (int t = 0; t < 2; ++t) {  // K, then V
-#pragma unroll
-                for (int qb = 0; qb < 2; ++qb) {
-                    const uint8_t *p = raw + t * R::TILE + 18 * qb;
-                    const float d = __half2float(*reinterpret_cast<const __half *>(p));
-                    const uint64_t d2 = f2_pack(d, d);
-                    const uint16_t *cw = reinterpret_cast<const uint16_t *>(p + 2);  // 8 byte pairs
-#pragma unroll
-                    for (int jj = 0; jj < 4; ++jj) {
-                        // chunk jj of the block: values 8 jj .. 8 jj + 7 -- the
-                        // low nibbles of bytes 8 (jj & 1) .., high ones for jj >= 2
-                        const int j = 4 * qb + jj;
-                        const int sh = jj >= 2 ? 4 : 0;
-                        const uint16_t *cp = cw + 4 * (jj & 1);
-                        const uint4 v = make_uint4(q4_pair_to_bf16((uint32_t)cp[0] >> sh, d2),
-                                                   q4_pair_to_bf16((uint32_t)cp[1] >> sh, d2),
-                                                   q4_pair_to_bf16((uint32_t)cp[2] >> sh, d2),
-                                                   q4_pair_to_bf16((uint32_t)cp[3] >> sh, d2));
-                        *reinterpret_cast<uint4 *>(wb + t * (2 * 16 * 128) + ((j ^ (lk & 7)) << 4)) = v;
-                    }
-                }
-            }
-        } else if constexpr (KVT == 8) {
-            // lane (lk, h) converts row lk's half h (two q8_0 blocks, 64 values)
-            // of K and of V into eight 16-byte chunks of the swizzled buffer
-            const int lk = lane >> 1, h = lane & 1;
-            const uint8_t *raw = smem + s * R::STAGE + (warp * 16 + lk) * R::ROW + 68 * h;
-            uint8_t *wb = smem + R::OFF_WB + warp * R::WBUF + h * (16 * 128) + lk * 128;
-#pragma unroll
-            for (int t = 0; t < 2; ++t) {  // K, then V
-#pragma unroll
-                for (int qb = 0; qb < 2; ++qb) {
-                    const uint8_t *p = raw + t * R::TILE + 34 * qb;
-                    const float d = __half2float(*reinterpret_cast<const __half *>(p));
-                    const uint64_t d2 = f2_pack(d, d);
-                    const uint16_t *cw = reinterpret_cast<const uint16_t *>(p + 2);
-#pragma unroll
-                    for (int jj = 0; jj < 4; ++jj) {
-                        const int j = 4 * qb + jj;  // 16-byte chunk of the half-row
-                        const uint4 v = make_uint4(q8_pair_to_bf16(cw[4 * jj], d2), q8_pair_to_bf16(cw[4 * jj + 1], d2),
-                                                   q8_pair_to_bf16(cw[4 * jj + 2], d2),
-                                                   q8_pair_to_bf16(cw[4 * jj + 3], d2));
-                        *reinterpret_cast<uint4 *>(wb + t * (2 * 16 * 128) + ((j ^ (lk & 7)) << 4)) = v;
-                    }
-                }
-            }
-        }
-        if constexpr (KVQ) {
-            __syncwarp();
-            if (lane == 0) mbar_arrive(empty(s));  // the raw stage may be refilled now
-            sK = sbase + R::OFF_WB + warp * R::WBUF;
-            sV = sK + 2 * 16 * 128;
-            hstr = 16 * 128;
-            kof = warp * 16;
-        } else {
-            sK = sbase + s * PD_STAGE;
-            sV = sK + PD_TILE;
-            hstr = PD_TILE / 2;
-            kof = 0;
-        }
+        if (lane == 0 && warp == 0) PD_TRACE(7, i);
+        // K and V tiles of the block: bf16, 128-byte swizzled, each as two
+        // 64-column halves of 64 rows x 128 bytes
+        const uint32_t sK = sbase + s * PD_STAGE, sV = sK + PD_TILE;
+        constexpr uint32_t hstr = PD_TILE / 2;  // byte distance between the two halves
         // ---- S = Q K^T for this warp's 16 keys (two n-tiles of 8) ----
-        float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        float sc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
         {
-            const int key = warp * 16 + (mi >> 1) * 8 + lr - kof;
+            const int key = wq * 16 + (mi >> 1) * 8 + lr;
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
                 const int d0 = ks * 16 + (mi & 1) * 8;
@@ -375,12 +503,13 @@ __global__ void __launch_bounds__(160, KVT ? 3 : 1) paged_decode_kernel(const __
                                                       ((((d0 & 63) >> 3) ^ (key & 7)) << 4));
                 uint32_t b00, b01, b10, b11;
                 ldsm_x4(addr, b00, b01, b10, b11);
-                mma_16816(sc[0], qa[ks][0], 0u, qa[ks][1], 0u, b00, b01);
-                mma_16816(sc[1], qa[ks][0], 0u, qa[ks][1], 0u, b10, b11);
+                mma_16816_top(sc[0], qa[ks][0], qa[ks][1], b00, b01);
+                mma_16816_top(sc[1], qa[ks][0], qa[ks][1], b10, b11);
             }
         }
+        if (lane == 0 && warp == 0) PD_TRACE(10, i);
         // ---- online softmax over the 4 scores this thread holds ----
-        const int key0 = (blk0 + i) * PD_BS + warp * 16 + 2 * tig;
+        const int key0 = (blk0 + i) * PD_BS + wq * 16 + 2 * tig;
         float x[4];
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt)
@@ -403,11 +532,12 @@ __global__ void __launch_bounds__(160, KVT ? 3 : 1) paged_decode_kernel(const __
             o[nt][0] *= alpha;
             o[nt][1] *= alpha;
         }
+        if (lane == 0 && warp == 0) PD_TRACE(11, i);
         // ---- O += P V: the score fragments are the A operand ----
         const uint32_t pa0 = pack_bf16x2(p[0], p[1]);
         const uint32_t pa2 = pack_bf16x2(p[2], p[3]);
         {
-            const int key = warp * 16 + (mi & 1) * 8 + lr - kof;
+            const int key = wq * 16 + (mi & 1) * 8 + lr;
 #pragma unroll
             for (int pr = 0; pr < 8; ++pr) {
                 const int nt = 2 * pr + (mi >> 1);  // 8-wide slice of head dims
@@ -415,22 +545,25 @@ __global__ void __launch_bounds__(160, KVT ? 3 : 1) paged_decode_kernel(const __
                                                       (((nt & 7) ^ (key & 7)) << 4));
                 uint32_t v0l, v0h, v1l, v1h;
                 ldsm_x4_t(addr, v0l, v0h, v1l, v1h);
-                mma_16816(o[2 * pr], pa0, 0u, pa2, 0u, v0l, v0h);
-                mma_16816(o[2 * pr + 1], pa0, 0u, pa2, 0u, v1l, v1h);
+                mma_16816_top(o[2 * pr], pa0, pa2, v0l, v0h);
+                mma_16816_top(o[2 * pr + 1], pa0, pa2, v1l, v1h);
             }
         }
         __syncwarp();
-        if (!KVQ && lane == 0) mbar_arrive(empty(s));
+        if (lane == 0) mbar_arrive(cempty(s));
+        if (lane == 0 && warp == 0) PD_TRACE(8, i);
+        if (lane == 0 && warp == 3) PD_TRACE(9, i);
     }
     // the four lanes of a quad hold partial sums of the same head
     l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
     l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
 
-    // ---- merge the four warps (the ring is free: every copy has landed) ----
-    asm volatile("bar.sync 1, 128;" ::: "memory");
-    float *mo = reinterpret_cast<float *>(smem);  // [4][G][128]
-    float *mm = mo + 4 * G * PD_D;                 // [4][G]
-    float *ml = mm + 4 * G;                        // [4][G]
+    // ---- merge the MMA warps (the rings are free: every copy has landed) ----
+    constexpr int NW = PD_MMA_WARPS;
+    asm volatile("bar.sync 1, %0;" ::"n"(NW * 32) : "memory");
+    float *mo = reinterpret_cast<float *>(smem);  // [NW][G][128]
+    float *mm = mo + NW * G * PD_D;                // [NW][G]
+    float *ml = mm + NW * G;                       // [NW][G]
     if (head_ok) {
 #pragma unroll
         for (int nt = 0; nt < 16; ++nt) {
@@ -442,17 +575,18 @@ __global__ void __launch_bounds__(160, KVT ? 3 : 1) paged_decode_kernel(const __
             ml[warp * G + gid] = l_run;
         }
     }
-    asm volatile("bar.sync 1, 128;" ::: "memory");
+    asm volatile("bar.sync 1, %0;" ::"n"(NW * 32) : "memory");
+    if (threadIdx.x >= PD_D) return;
     const int d = threadIdx.x;  // 0..127
 #pragma unroll
     for (int g = 0; g < G; ++g) {
         float M = -INFINITY;
 #pragma unroll
-        for (int k = 0; k < 4; ++k) M = fmaxf(M, mm[k * G + g]);
+        for (int k = 0; k < NW; ++k) M = fmaxf(M, mm[k * G + g]);
         const float msub = (M == -INFINITY) ? 0.f : M;
         float L = 0.f, O = 0.f;
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
+        for (int k = 0; k < NW; ++k) {
             const float w = ex2(mm[k * G + g] - msub);
             L = fmaf(w, ml[k * G + g], L);
             O = fmaf(w, mo[(k * G + g) * PD_D + d], O);
@@ -462,7 +596,24 @@ __global__ void __launch_bounds__(160, KVT ? 3 : 1) paged_decode_kernel(const __
         a.part_o[row * PD_D + d] = good ? O / L : 0.f;
         if (d == 0) a.part_lse[row] = good ? msub + __log2f(L) : -INFINITY;
     }
+#ifdef FA_PD_TRACE
+    if (threadIdx.x == 0) { PD_CTA(1, pd_gtimer()); PD_TRACE(15, 1); }
+#endif
 }
+
+#ifdef FA_PD_TRACE
+extern "C" int fa_debug_pd_trace_read(unsigned long long *host, unsigned long long *cta) {
+    cudaMemcpyFromSymbol(host, fa::g_pd_trace, sizeof(fa::g_pd_trace));
+    cudaMemcpyFromSymbol(cta, fa::g_pd_cta, sizeof(fa::g_pd_cta));
+    return (int)cudaDeviceSynchronize();
+}
+extern "C" int fa_debug_pd_trace_reset() {
+    static unsigned long long z[fa::kPdCtaCap] = {};
+    cudaMemcpyToSymbol(fa::g_pd_trace, z, sizeof(fa::g_pd_trace));
+    cudaMemcpyToSymbol(fa::g_pd_cta, z, sizeof(fa::g_pd_cta));
+    return (int)cudaDeviceSynchronize();
+}
+#endif
 
 // ----------------------------------------------------------------------------
 // Log-sum-exp combine: one warp per (sequence or token, query head) merges
@@ -571,7 +722,7 @@ static cudaError_t launch_g(const PagedLaunch &L, const PagedArgs &a, int B, cud
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)a.num_splits, (unsigned)a.Hkv, (unsigned)B);
-    kern<<<grid, 160, smem, stream>>>(L.tmK, L.tmV, a);
+    kern<<<grid, KVT ? PDQ_THREADS : PD_THREADS, smem, stream>>>(L.tmK, L.tmV, a);
     return cudaGetLastError();
 }
 

@@ -509,6 +509,20 @@ FA_DEV void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// The same with rows 8..15 of A zero (a1 = a3 = 0): rows 8..15 of D stay
+// zero, so only rows 0..7 (d[0], d[1] of each lane) are kept; the other two
+// outputs are dead at once and hold no registers between calls.
+FA_DEV void mma_16816_top(float (&d)[2], uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1) {
+    float z0, z1;
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %10, %10};"
+        : "+f"(d[0]), "+f"(d[1]), "=f"(z0), "=f"(z1)
+        : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1), "f"(0.f));
+    (void)z0;
+    (void)z1;
+}
+
 // ------------------------------------------------------------ arithmetic --
 
 // 2^x with the hardware approximation (MUFU.EX2); 2^-inf = 0.
