@@ -452,29 +452,39 @@ __global__ void __launch_bounds__(KVT ? PDQ_THREADS : PD_THREADS, 1) paged_decod
 
     // ------------------------------------------------------- MMA warps --
     // Group grp = w / 4 takes blocks grp, grp + PD_NG, ...; warp w owns keys
-    // [16 wq, 16 wq + 16) of each of them, wq = w % 4.  MMA fragment roles:
-    // gid = lane / 4 is the M row (query head, valid when gid < G), tig =
-    // lane % 4 picks the column pairs.
+    // [16 wq, 16 wq + 16) of each of them, wq = w % 4.  Both contractions run
+    // transposed, with the (at most 8) query heads as the N = 8 columns of
+    // m16n8k16 MMAs (fp32 accumulate):
+    //   S^T (16 keys x 8 heads)  = K (16 keys x 128 dims) Q^T: 8 MMAs;
+    //   O^T (128 dims x 8 heads) += V^T (128 dims x 16 keys) P^T: 8 MMAs,
+    // K and V^T as A operands from the swizzled tile (ldmatrix, .trans for
+    // V), Q^T as a register B operand.  Fragment roles: gid = lane / 4, tig =
+    // lane % 4; a C fragment holds rows gid and gid + 8, columns (heads) 2 tig
+    // and 2 tig + 1.  P^T is the transpose of the score fragment, formed in
+    // registers with movmatrix.
     const int gid = lane >> 2, tig = lane & 3;
     const int grp = warp >> 2, wq = warp & 3;
-    const bool head_ok = gid < G;
-    uint32_t qa[8][2];
+    // Q^T fragments (B operand, k = dims, n = heads): head gid, dims
+    // 16 ks + 2 tig, +1 and 16 ks + 8 + 2 tig, +1; heads >= G are zero
+    uint32_t qb[8][2];
     {
+        const bool head_ok = gid < G;
         const uint32_t *qp = reinterpret_cast<const uint32_t *>(
             a.q + ((int64_t)b * a.Hq + (int64_t)hkv * G + (head_ok ? gid : 0)) * PD_D);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
-            qa[ks][0] = head_ok ? qp[(ks * 16 + 2 * tig) >> 1] : 0u;
-            qa[ks][1] = head_ok ? qp[(ks * 16 + 8 + 2 * tig) >> 1] : 0u;
+            qb[ks][0] = head_ok ? qp[(ks * 16 + 2 * tig) >> 1] : 0u;
+            qb[ks][1] = head_ok ? qp[(ks * 16 + 8 + 2 * tig) >> 1] : 0u;
         }
     }
     const float c = a.scale_log2;
-    float m_run = -INFINITY, l_run = 0.f;
-    // O rows of the query heads (the MMA's M rows 0..7; rows 8..15 are
-    // padding and never kept)
-    float o[16][2];
+    // running max and (lane-partial) sum of heads 2 tig and 2 tig + 1
+    float m_run0 = -INFINITY, m_run1 = -INFINITY, l_run0 = 0.f, l_run1 = 0.f;
+    // O^T: 8 m-tiles of 16 dims; o[mt][0..1] = dim 16 mt + gid, o[mt][2..3] =
+    // dim 16 mt + gid + 8, each for heads 2 tig, 2 tig + 1
+    float o[8][4];
 #pragma unroll
-    for (int nt = 0; nt < 16; ++nt) o[nt][0] = o[nt][1] = 0.f;
+    for (int mt = 0; mt < 8; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
     // ldmatrix lane roles: matrix mi = lane / 8, row lr = lane % 8
     const int mi = lane >> 3, lr = lane & 7;
 
@@ -492,61 +502,68 @@ __global__ void __launch_bounds__(KVT ? PDQ_THREADS : PD_THREADS, 1) paged_decod
         // 64-column halves of 64 rows x 128 bytes
         const uint32_t sK = sbase + s * PD_STAGE, sV = sK + PD_TILE;
         constexpr uint32_t hstr = PD_TILE / 2;  // byte distance between the two halves
-        // ---- S = Q K^T for this warp's 16 keys (two n-tiles of 8) ----
-        float sc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+        // ---- S^T = K Q^T: even and odd dim steps in two accumulators ----
+        float se[4] = {0.f, 0.f, 0.f, 0.f}, so[4] = {0.f, 0.f, 0.f, 0.f};
         {
-            const int key = wq * 16 + (mi >> 1) * 8 + lr;
+            // matrices (A fragment order): keys 0-7 | 8-15 (mi & 1) x dims lo | hi (mi >> 1)
+            const int key = wq * 16 + (mi & 1) * 8 + lr;
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
-                const int d0 = ks * 16 + (mi & 1) * 8;
+                const int d0 = ks * 16 + (mi >> 1) * 8;
                 const uint32_t addr = sK + (uint32_t)(d0 >> 6) * hstr + (uint32_t)(key * 128 +
                                                       ((((d0 & 63) >> 3) ^ (key & 7)) << 4));
-                uint32_t b00, b01, b10, b11;
-                ldsm_x4(addr, b00, b01, b10, b11);
-                mma_16816_top(sc[0], qa[ks][0], qa[ks][1], b00, b01);
-                mma_16816_top(sc[1], qa[ks][0], qa[ks][1], b10, b11);
+                uint32_t a0, a1, a2, a3;
+                ldsm_x4(addr, a0, a1, a2, a3);
+                mma_16816((ks & 1) ? so : se, a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
             }
         }
         if (lane == 0 && warp == 0) PD_TRACE(10, i);
-        // ---- online softmax over the 4 scores this thread holds ----
-        const int key0 = (blk0 + i) * PD_BS + wq * 16 + 2 * tig;
-        float x[4];
+        // ---- online softmax: this lane holds keys gid, gid + 8 of heads 2 tig, 2 tig + 1 ----
+        const int key0 = (blk0 + i) * PD_BS + wq * 16 + gid;
+        const bool v0 = key0 < seq_len, v1 = key0 + 8 < seq_len;
+        const float x0 = v0 ? (se[0] + so[0]) * c : -INFINITY, x1 = v0 ? (se[1] + so[1]) * c : -INFINITY;
+        const float x2 = v1 ? (se[2] + so[2]) * c : -INFINITY, x3 = v1 ? (se[3] + so[3]) * c : -INFINITY;
+        float mt0 = fmaxf(x0, x2), mt1 = fmaxf(x1, x3);
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
+        for (int off = 4; off < 32; off <<= 1) {  // over the 8 key rows gid
+            mt0 = fmaxf(mt0, __shfl_xor_sync(0xffffffffu, mt0, off));
+            mt1 = fmaxf(mt1, __shfl_xor_sync(0xffffffffu, mt1, off));
+        }
+        const float mn0 = fmaxf(m_run0, mt0), mn1 = fmaxf(m_run1, mt1);
+        const float ms0 = (mn0 == -INFINITY) ? 0.f : mn0, ms1 = (mn1 == -INFINITY) ? 0.f : mn1;
+        const float al0 = ex2(m_run0 - ms0), al1 = ex2(m_run1 - ms1);
+        const float p0 = ex2(x0 - ms0), p1 = ex2(x1 - ms1), p2 = ex2(x2 - ms0), p3 = ex2(x3 - ms1);
+        l_run0 = l_run0 * al0 + (p0 + p2);
+        l_run1 = l_run1 * al1 + (p1 + p3);
+        m_run0 = mn0;
+        m_run1 = mn1;
+        {
+            const uint64_t al = f2_pack(al0, al1);
 #pragma unroll
-            for (int e = 0; e < 2; ++e)
-                x[nt * 2 + e] = (key0 + nt * 8 + e < seq_len) ? sc[nt][e] * c : -INFINITY;
-        float mt = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
-        mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 1));
-        mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 2));
-        const float mn = fmaxf(m_run, mt);
-        const float msub = (mn == -INFINITY) ? 0.f : mn;
-        const float alpha = ex2(m_run - msub);
-        float p[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) p[k] = ex2(x[k] - msub);
-        l_run = l_run * alpha + (p[0] + p[1]) + (p[2] + p[3]);
-        m_run = mn;
-#pragma unroll
-        for (int nt = 0; nt < 16; ++nt) {
-            o[nt][0] *= alpha;
-            o[nt][1] *= alpha;
+            for (int mt = 0; mt < 8; ++mt) {
+                f2_unpack(f2_mul(f2_pack(o[mt][0], o[mt][1]), al), o[mt][0], o[mt][1]);
+                f2_unpack(f2_mul(f2_pack(o[mt][2], o[mt][3]), al), o[mt][2], o[mt][3]);
+            }
         }
         if (lane == 0 && warp == 0) PD_TRACE(11, i);
-        // ---- O += P V: the score fragments are the A operand ----
-        const uint32_t pa0 = pack_bf16x2(p[0], p[1]);
-        const uint32_t pa2 = pack_bf16x2(p[2], p[3]);
+        // ---- O^T += V^T P^T ----
+        // P^T as the B operand (k = keys, n = heads): lane (gid, tig) needs
+        // head gid at keys 2 tig, 2 tig + 1 (and + 8): the transposes of the
+        // 8 x 8 bf16 score blocks this lane holds row gid of.
+        const uint32_t pb0 = movmatrix_trans(pack_bf16x2(p0, p1));
+        const uint32_t pb1 = movmatrix_trans(pack_bf16x2(p2, p3));
         {
-            const int key = wq * 16 + (mi & 1) * 8 + lr;
+            // matrices (A fragment order, transposed on load): dims lo | hi
+            // (mi & 1) x keys 0-7 | 8-15 (mi >> 1); rows of the stored tile are keys
+            const int key = wq * 16 + (mi >> 1) * 8 + lr;
 #pragma unroll
-            for (int pr = 0; pr < 8; ++pr) {
-                const int nt = 2 * pr + (mi >> 1);  // 8-wide slice of head dims
-                const uint32_t addr = sV + (uint32_t)((nt * 8) >> 6) * hstr + (uint32_t)(key * 128 +
-                                                      (((nt & 7) ^ (key & 7)) << 4));
-                uint32_t v0l, v0h, v1l, v1h;
-                ldsm_x4_t(addr, v0l, v0h, v1l, v1h);
-                mma_16816_top(o[2 * pr], pa0, pa2, v0l, v0h);
-                mma_16816_top(o[2 * pr + 1], pa0, pa2, v1l, v1h);
+            for (int mt = 0; mt < 8; ++mt) {
+                const int d0 = mt * 16 + (mi & 1) * 8;
+                const uint32_t addr = sV + (uint32_t)(d0 >> 6) * hstr + (uint32_t)(key * 128 +
+                                                      ((((d0 & 63) >> 3) ^ (key & 7)) << 4));
+                uint32_t a0, a1, a2, a3;
+                ldsm_x4_t(addr, a0, a1, a2, a3);
+                mma_16816(o[mt], a0, a1, a2, a3, pb0, pb1);
             }
         }
         __syncwarp();
@@ -554,9 +571,12 @@ __global__ void __launch_bounds__(KVT ? PDQ_THREADS : PD_THREADS, 1) paged_decod
         if (lane == 0 && warp == 0) PD_TRACE(8, i);
         if (lane == 0 && warp == 3) PD_TRACE(9, i);
     }
-    // the four lanes of a quad hold partial sums of the same head
-    l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
-    l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
+    // the sums over this warp's keys: add the 8 key rows gid
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+        l_run0 += __shfl_xor_sync(0xffffffffu, l_run0, off);
+        l_run1 += __shfl_xor_sync(0xffffffffu, l_run1, off);
+    }
 
     // ---- merge the MMA warps (the rings are free: every copy has landed) ----
     constexpr int NW = PD_MMA_WARPS;
@@ -564,15 +584,19 @@ __global__ void __launch_bounds__(KVT ? PDQ_THREADS : PD_THREADS, 1) paged_decod
     float *mo = reinterpret_cast<float *>(smem);  // [NW][G][128]
     float *mm = mo + NW * G * PD_D;                // [NW][G]
     float *ml = mm + NW * G;                       // [NW][G]
-    if (head_ok) {
 #pragma unroll
-        for (int nt = 0; nt < 16; ++nt) {
-            mo[(warp * G + gid) * PD_D + nt * 8 + 2 * tig] = o[nt][0];
-            mo[(warp * G + gid) * PD_D + nt * 8 + 2 * tig + 1] = o[nt][1];
-        }
-        if (tig == 0) {
-            mm[warp * G + gid] = m_run;
-            ml[warp * G + gid] = l_run;
+    for (int e = 0; e < 2; ++e) {
+        const int h = 2 * tig + e;
+        if (h < G) {
+#pragma unroll
+            for (int mt = 0; mt < 8; ++mt) {
+                mo[(warp * G + h) * PD_D + mt * 16 + gid] = o[mt][e];
+                mo[(warp * G + h) * PD_D + mt * 16 + gid + 8] = o[mt][2 + e];
+            }
+            if (gid == 0) {
+                mm[warp * G + h] = e ? m_run1 : m_run0;
+                ml[warp * G + h] = e ? l_run1 : l_run0;
+            }
         }
     }
     asm volatile("bar.sync 1, %0;" ::"n"(NW * 32) : "memory");

@@ -500,6 +500,15 @@ FA_DEV void ldsm_x4_t(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, u
                  : "r"(addr));
 }
 
+// Transpose of an 8 x 8 matrix of 16-bit elements held as a warp fragment
+// (lane l holds row l / 4, columns 2 (l % 4), +1): afterwards lane l holds
+// row l / 4 of the transpose.
+FA_DEV uint32_t movmatrix_trans(uint32_t x) {
+    uint32_t y;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+    return y;
+}
+
 // D(16x8, fp32) += A(16x16, bf16, row) * B(16x8, bf16, col).
 FA_DEV void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0, uint32_t b1) {
     asm volatile(
@@ -507,20 +516,6 @@ FA_DEV void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint
         "{%0, %1, %2, %3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-// The same with rows 8..15 of A zero (a1 = a3 = 0): rows 8..15 of D stay
-// zero, so only rows 0..7 (d[0], d[1] of each lane) are kept; the other two
-// outputs are dead at once and hold no registers between calls.
-FA_DEV void mma_16816_top(float (&d)[2], uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1) {
-    float z0, z1;
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
-        "{%0, %1, %10, %10};"
-        : "+f"(d[0]), "+f"(d[1]), "=f"(z0), "=f"(z1)
-        : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1), "f"(0.f));
-    (void)z0;
-    (void)z1;
 }
 
 // ------------------------------------------------------------ arithmetic --
