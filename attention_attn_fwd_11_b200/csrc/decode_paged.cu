@@ -74,11 +74,12 @@ constexpr int PD_SMEM = PD_OFF_BAR + 128 + 1024;  // ring + barriers + 1024-byte
 // 4 blocks of 18 bytes (72 bytes); FP8 E4M3 rows one byte a value (128
 // bytes) with one fp32 scale per tensor (k_scale, v_scale).  A (block, head)
 // tile of K or V is 64 such rows, contiguous, moved with one bulk copy into
-// a raw ring.  Eight converter warps turn each raw tile into the bf16 tile
-// the bf16 path reads (two 64-column halves, 128-byte swizzle, exactly the
-// layout of the TMA-filled bf16 ring) in a second ring, from which the four
-// MMA warps run the unchanged bf16 path.  Conversion and MMAs thus overlap
-// across warps instead of following one another inside each warp.
+// a raw ring.  Converter warps (two teams of four taking alternate tiles;
+// a warp converts 16 rows of K and of V) turn each raw tile into the bf16
+// tile the bf16 path reads (two 64-column halves, 128-byte swizzle, exactly
+// the layout of the TMA-filled bf16 ring) in a second ring, from which the
+// four MMA warps run the unchanged bf16 path.  Conversion and MMAs thus
+// overlap across warps instead of following one another inside each warp.
 #ifndef FA_PDQ_NR
 #define FA_PDQ_NR 4
 #endif
@@ -88,15 +89,24 @@ constexpr int PD_SMEM = PD_OFF_BAR + 128 + 1024;  // ring + barriers + 1024-byte
 #ifndef FA_PDQ_NCV
 #define FA_PDQ_NCV 4
 #endif
-constexpr int PDQ_NCV = FA_PDQ_NCV;                // converter warps (4 doing K and V, or 8)
+constexpr int PDQ_NCV = FA_PDQ_NCV;                // converter warps per tile (4 doing K and V, or 8)
 static_assert(PDQ_NCV == 8 || PDQ_NCV == 4, "converter warps");
+// Teams of PDQ_NCV converter warps take alternate tiles.  Two teams (eight
+// converter warps, 13 warps a CTA, at most 128 registers a thread): the
+// conversion is latency-bound, and with one team it alone took about 0.20
+// ms of a 0.24 ms q8_0 decode step (64 sequences of 1 024-8 192 keys, 8 KV
+// heads); three or four teams (96 or 80 registers) measured slower.
+#ifndef FA_PDQ_TEAMS
+#define FA_PDQ_TEAMS 2
+#endif
+constexpr int PDQ_TEAMS = FA_PDQ_TEAMS;
 // Groups of four MMA warps taking alternate blocks (each group with its own
 // online softmax, all warps merging at the end).  One group: two groups
 // (eight MMA warps) measured 3-8 % slower on every cache type.
 constexpr int PD_NG = 1;
 constexpr int PD_MMA_WARPS = 4 * PD_NG;
 constexpr int PD_THREADS = (PD_MMA_WARPS + 1) * 32;            // bf16: MMA warps + the producer
-constexpr int PDQ_THREADS = (PD_MMA_WARPS + 1 + PDQ_NCV) * 32;  // quantised: + the converters
+constexpr int PDQ_THREADS = (PD_MMA_WARPS + 1 + PDQ_NCV * PDQ_TEAMS) * 32;  // quantised: + the converters
 static_assert((PD_MMA_WARPS * 8 * PD_D + 2 * PD_MMA_WARPS * 8) * 4 <= PD_NST * PD_STAGE, "merge area");
 //
 // Raw-tile geometry per cache type KVT (8 = q8_0, 4 = q4_0, 2 = fp8 e4m3):
@@ -299,9 +309,9 @@ struct PagedArgs {
 };
 
 // bf16 caches: one CTA of 160 threads per SM (its ring fills shared memory).
-// Quantised caches: one CTA of 288 threads per SM.  A sub-partition of the
-// SM holds 16 K registers and runs at most 3 of the 9 warps, so a thread
-// gets up to 168.
+// Quantised caches: one CTA of 416 threads per SM.  A sub-partition of the
+// SM holds 16 K registers and runs up to 4 of the 13 warps, so a thread gets
+// at most 128.
 template <int G, int KVT>
 __global__ void __launch_bounds__(KVT ? PDQ_THREADS : PD_THREADS, 1) paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                                                            const __grid_constant__ CUtensorMap tmV,
@@ -348,6 +358,8 @@ __global__ void __launch_bounds__(KVT ? PDQ_THREADS : PD_THREADS, 1) paged_decod
     // itself consumed phase k - 1: the barrier is at most one phase away and
     // the parity wait cannot pass on an older phase.
     static_assert(NC % PD_NG == 0, "ring stages per MMA group");
+    // the same for the converter teams on both rings
+    static_assert(!KVQ || (NP % PDQ_TEAMS == 0 && NC % PDQ_TEAMS == 0), "ring stages per converter team");
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_BAR + 8 * NBARS);
     const uint32_t stall_bar = bar0 + 8u * (NBARS + 1);  // a.stall only: never arrived on
     const unsigned long long wait_ns = a.wait_ns;
@@ -423,10 +435,11 @@ __global__ void __launch_bounds__(KVT ? PDQ_THREADS : PD_THREADS, 1) paged_decod
     if constexpr (KVQ) {
         if (warp > PD_MMA_WARPS) {
             // ------------------------------------------------- converters --
-            const int cw = warp - PD_MMA_WARPS - 1;
+            const int team = (warp - PD_MMA_WARPS - 1) / PDQ_NCV;
+            const int cw = (warp - PD_MMA_WARPS - 1) % PDQ_NCV;
             constexpr int NT = 8 / PDQ_NCV;  // tensors (K, V) per converter warp
             Converter<KVT> cv[NT];
-            for (int i = 0; i < nblk; ++i) {
+            for (int i = team; i < nblk; i += PDQ_TEAMS) {
                 const int s = i % NP, sb = i % NC;
                 if (!mbar_wait(pfull(s), (uint32_t)(i / NP) & 1u, abort_flag, &g_decode_err, wait_ns)) break;
                 if (lane == 0 && cw == 0) PD_TRACE(1, i);
