@@ -28,6 +28,7 @@ def run(B, Hq, Hkv, lens, seed, num_splits=0, out_dtype=torch.float32):
     o_ref, l_ref = oracle.decode_paged(W.bits(q), kb, vb, table.numpy(), sl.numpy(), c.scale)
     check(o, o_ref, lse, l_ref,
           what="q8_0 paged decode lens %s" % (list(lens),))
+    return c, q, kq, vq, table, sl, o, lse
 
 
 @pytest.mark.parametrize("g", [1, 2, 4, 8])
@@ -43,6 +44,18 @@ def test_split_counts(splits):
 
 def test_bf16_output_and_zero_length():
     run(4, 8, 8, (0, 200, 1, 4097), seed=20, out_dtype=torch.bfloat16)
+
+
+def test_q8_prologue_equals_bf16_caches_from_the_pre_pass():
+    # The prologue rounds d * code to bf16 once, like the pre-pass, and the
+    # MMA path after it is the bf16 one: decoding the q8_0 caches equals
+    # decoding their pre-pass output, bit for bit.
+    c, q, kq, vq, table, sl, o, lse = run(3, 8, 2, (700, 64, 1), seed=61)
+    kb = fa.kv_dequant(kq.cuda(), "q8_0", 128)
+    vb = fa.kv_dequant(vq.cuda(), "q8_0", 128)
+    o2, l2 = fa.decode_paged(q.cuda(), kb, vb, table.cuda(), sl.cuda(), scale=c.scale)
+    torch.cuda.synchronize()
+    assert torch.equal(o, o2) and torch.equal(lse, l2)
 
 
 def test_workload_shape():
