@@ -221,8 +221,9 @@ fa_status fa_prefill_paged(const fa_prefill_paged_params *p, void *stream);
  *   seq_lens: [B] int32, each in [0, max_blocks_per_seq * block_size].
  *   o: [B, Hq, dv] (o_dtype) contiguous; lse: NULL or [B, Hq] fp32.
  *   num_splits: 0 = choose automatically (from the current device's SM
- *     count; FA_ERR_CUDA if it cannot be read), else the number of key
- *     splits per sequence (clamped to [1, max_blocks_per_seq]).
+ *     count and the cache type; FA_ERR_CUDA if the SM count cannot be
+ *     read), else the number of key splits per sequence (clamped to
+ *     [1, max_blocks_per_seq]).
  *   workspace: device scratch of at least fa_decode_paged_workspace_size()
  *     bytes, 256-byte aligned; it holds the split partials and is
  *     overwritten on every call.
