@@ -62,7 +62,7 @@ NCU_TRAFFIC = {
     "gqa_full_b1_hq32_hkv8_s4096_d256": 215944192,
     "causal_mha_mods_b2_h16_s2048_d128": 58342656,
     "paged_gqa_b64_hq32_hkv8_d128_bs64": 1236043776,
-    "paged_gqa_q8_0kv_b64_hq32_hkv8_d128_bs64": 659442176,
+    "paged_gqa_q8_0kv_b64_hq32_hkv8_d128_bs64": 658865408,
     "latent_sparse_t32_hq128_dk576_dv512_top2048": 45273088,
     "causal_mha_b2_h16_s2048_dk192_dv128": 72717056,
     "causal_gqa_b2_hq16_hkv4_s2048_dk192_dv192": 39777792,
@@ -71,8 +71,8 @@ NCU_TRAFFIC = {
     "paged_prefill_gqa_b16_hq32_hkv8_sq512_d128_bs64": 417585664,
     "mla_tail_t32_hq128_r512_v128_hidden7168": 257049088,
     "causal_gqa_b1_hq16_hkv4_s4096_dk320_dv256": 78919168,
-    "paged_gqa_fp8kv_b64_hq32_hkv8_d128_bs64": 620966912,
-    "paged_gqa_q4_0kv_b64_hq32_hkv8_d128_bs64": 351834368,
+    "paged_gqa_fp8kv_b64_hq32_hkv8_d128_bs64": 620406528,
+    "paged_gqa_q4_0kv_b64_hq32_hkv8_d128_bs64": 351211008,
     "causal_mqa_b1_hq16_hkv1_s4096_dk576_dv512": 167481088,
 }
 
