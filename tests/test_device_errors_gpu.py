@@ -159,3 +159,35 @@ def test_bounded_wait_runs_out_and_the_context_stays_usable():
     qh, kh, vh, th, lh = W.paged_inputs(c)
     o_ref, l_ref = oracle.decode_paged(W.bits(qh), W.bits(kh), W.bits(vh), th.numpy(), lh.numpy(), c.scale)
     check(o2, o_ref, l2, l_ref, what="after the timeout")
+
+
+def test_bounded_wait_runs_out_with_converter_warps():
+    # q8_0 caches: the CTA also runs converter warps between the raw and the
+    # bf16 rings.  With the MMA warps stuck on the stall barrier, the
+    # converters fill the bf16 ring and then wait for a stage that is never
+    # released; the producer waits for raw stages.  Every one of those waits
+    # is bounded and watches the abort flag, so the CTA leaves.
+    c = W.PagedCase("stall_q8", 6, 8, 2, 128, 128, 64, 0, 0, seed=306, lens=(100, 2000, 64, 4000, 1, 700))
+    q, _, _, table, lens = [t.cuda() for t in W.paged_inputs(c)]
+    nbk = int(table.max()) + 1
+    kq, vq = W.paged_q8_caches(c, nbk)
+    kq, vq = kq.cuda(), vq.cuda()
+    fn = stall_fn()
+    n = fa.paged_workspace_bytes(q, kq, vq, table, lens)
+    ws = torch.empty(max(n, 256), device="cuda", dtype=torch.uint8)
+    o = torch.full((6, 8, 128), float("nan"), device="cuda")
+    lse = torch.full((6, 8), float("nan"), device="cuda")
+    p = fa.paged_params(q, kq, vq, table, lens, o, lse, c.scale, 0, ws)
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    fa.device_error()
+    assert fn(ctypes.byref(p), ctypes.c_uint64(200_000), stream) == fa.FA_OK  # 200 us
+    torch.cuda.synchronize()  # returns: every role gave up and left
+    assert fa.device_error() == FA_DEVERR_TIMEOUT
+    assert torch.all(o == 0) and torch.all(lse == -float("inf"))
+    # the same context, an ordinary call over the same caches
+    o2, l2 = fa.decode_paged(q, kq, vq, table, lens, scale=c.scale)
+    assert fa.device_error() == 0
+    kb = oracle.dequant_rows(kq.cpu().numpy(), "q8_0", 128)
+    vb = oracle.dequant_rows(vq.cpu().numpy(), "q8_0", 128)
+    o_ref, l_ref = oracle.decode_paged(W.bits(q.cpu()), kb, vb, table.cpu().numpy(), lens.cpu().numpy(), c.scale)
+    check(o2, o_ref, l2, l_ref, what="q8_0 after the timeout")
