@@ -108,7 +108,7 @@ constexpr int PD_MMA_WARPS = 4 * PD_NG;
 constexpr int PD_THREADS = (PD_MMA_WARPS + 1) * 32;            // bf16: MMA warps + the producer
 constexpr int PDQ_THREADS = (PD_MMA_WARPS + 1 + PDQ_NCV * PDQ_TEAMS) * 32;  // quantised: + the converters
 static_assert((PD_MMA_WARPS * 8 * PD_D + 2 * PD_MMA_WARPS * 8) * 4 <= PD_NST * PD_STAGE, "merge area");
-//
+
 // Raw-tile geometry per cache type KVT (8 = q8_0, 4 = q4_0, 2 = fp8 e4m3):
 template <int KVT>
 struct PdRaw {
